@@ -1,0 +1,164 @@
+"""Reference model of the refcounted physical block pool -- TEST INFRASTRUCTURE ONLY.
+
+Plain Python, one step per rule on the pages:
+
+* "PagedAttention 机制" §5.3.4, BlockAllocator: a free list and a per-block
+  reference count; allocate fails when the free list is empty, else takes a
+  block and sets its count to 1; free decrements and returns the block to the
+  free list when the count reaches 0; incr_ref adds a reference (sharing).
+* "01. PagedAttention 详解" self-check 3 (get_new_blocks / free_blocks): the
+  free list is a queue -- allocation takes from the head, a block whose count
+  drops to 0 goes to the tail (least recently freed is reused first).  Where
+  this and the first page's list pop() differ, the queue is taken.
+* "PagedAttention 机制" §5.3.2, BlockTable.allocate: a sequence of n tokens
+  holds ceil(n / block_size) blocks; a table maps logical block i to a
+  physical id.
+* intelliparadigm PagedAttention article §3.3, maybe_copy_block: writing into a
+  block whose count is above 1 first allocates a new block, copies, drops one
+  reference from the old block and continues in the new one.
+* "01. PagedAttention 详解" §6 and summary: sequences may share blocks (a common
+  prefix, or a fork for beam search / parallel sampling) by adding references.
+
+Misuse (freeing a free block, adding a reference to a free block, an unknown
+sequence) raises PoolError with the matching status name; running out of free
+blocks raises OutOfBlocks and leaves the state unchanged.
+"""
+from __future__ import annotations
+
+from collections import deque
+
+
+class PoolError(Exception):
+    status = "PA_ERR_REFCOUNT"
+
+
+class OutOfBlocks(PoolError):
+    status = "PA_ERR_OUT_OF_BLOCKS"
+
+
+class InvalidArg(PoolError):
+    status = "PA_ERR_INVALID_ARG"
+
+
+class PoolModel:
+    def __init__(self, num_blocks: int, block_size: int):
+        if num_blocks <= 0 or block_size <= 0:
+            raise InvalidArg("bad sizes")
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+        self.free_queue = deque(range(num_blocks))
+        self.ref = [0] * num_blocks
+        self.seqs = {}            # id -> [blocks list, num tokens]
+        self.next_seq = 0
+        self.cow_count = 0
+
+    # -- blocks -----------------------------------------------------------
+    def _check_block(self, b):
+        if not (0 <= b < self.num_blocks):
+            raise InvalidArg(f"block {b} out of range")
+
+    def alloc(self) -> int:
+        if not self.free_queue:
+            raise OutOfBlocks("no free blocks")
+        b = self.free_queue.popleft()
+        self.ref[b] = 1
+        return b
+
+    def free(self, b: int) -> None:
+        self._check_block(b)
+        if self.ref[b] <= 0:
+            raise PoolError(f"block {b} is already free")
+        self.ref[b] -= 1
+        if self.ref[b] == 0:
+            self.free_queue.append(b)
+
+    def incr_ref(self, b: int) -> None:
+        self._check_block(b)
+        if self.ref[b] <= 0:
+            raise PoolError(f"block {b} is free")
+        self.ref[b] += 1
+
+    # -- sequences --------------------------------------------------------
+    def _seq(self, sid):
+        if sid not in self.seqs:
+            raise InvalidArg(f"unknown sequence {sid}")
+        return self.seqs[sid]
+
+    def seq_new(self) -> int:
+        sid = self.next_seq
+        self.next_seq += 1
+        self.seqs[sid] = [[], 0]
+        return sid
+
+    def seq_fork(self, parent: int) -> int:
+        blocks, n = self._seq(parent)
+        for b in blocks:
+            self.incr_ref(b)
+        sid = self.seq_new()
+        self.seqs[sid] = [list(blocks), n]
+        return sid
+
+    def seq_share_prefix(self, sid: int, blocks, num_tokens: int) -> None:
+        """An empty sequence takes references on existing blocks holding its first
+        num_tokens tokens (ceil(num_tokens / block_size) == len(blocks))."""
+        seq = self._seq(sid)
+        bs = self.block_size
+        if seq[1] != 0 or len(blocks) != (num_tokens + bs - 1) // bs:
+            raise InvalidArg("prefix must go into an empty sequence and fill its blocks")
+        for b in blocks:
+            self._check_block(b)
+            if self.ref[b] <= 0:
+                raise PoolError(f"block {b} is free")
+        for b in blocks:
+            self.ref[b] += 1
+        seq[0] = list(blocks)
+        seq[1] = num_tokens
+
+    def seq_append(self, sid: int):
+        """Room for one more token: returns (slot, cow_src, cow_dst), -1 when no copy."""
+        blocks, n = self._seq(sid)
+        bs = self.block_size
+        src = dst = -1
+        if n % bs == 0:
+            blocks.append(self.alloc())
+        else:
+            last = blocks[-1]
+            if self.ref[last] > 1:
+                new = self.alloc()
+                self.ref[last] -= 1          # stays >= 1: the other holders keep it
+                blocks[-1] = new
+                src, dst = last, new
+                self.cow_count += 1
+        slot = blocks[-1] * bs + n % bs
+        self.seqs[sid][1] = n + 1
+        return slot, src, dst
+
+    def seq_free(self, sid: int) -> None:
+        blocks, _ = self._seq(sid)
+        for b in blocks:
+            self.free(b)
+        del self.seqs[sid]
+
+    def seq_len(self, sid: int) -> int:
+        return self._seq(sid)[1]
+
+    def seq_blocks(self, sid: int):
+        return list(self._seq(sid)[0])
+
+    # -- packing ----------------------------------------------------------
+    def build_block_tables(self, sids, max_blocks: int):
+        """Rows of physical ids padded with -1, plus the context lengths."""
+        tables, lens = [], []
+        for sid in sids:
+            blocks, n = self._seq(sid)
+            if len(blocks) > max_blocks:
+                raise InvalidArg("table wider than max_blocks")
+            tables.append(list(blocks) + [-1] * (max_blocks - len(blocks)))
+            lens.append(n)
+        return tables, lens
+
+    def stats(self):
+        used = sum(1 for r in self.ref if r > 0)
+        shared = sum(1 for r in self.ref if r > 1)
+        return dict(num_blocks=self.num_blocks, free=len(self.free_queue), used=used,
+                    shared=shared, cow_copies=self.cow_count, num_seqs=len(self.seqs))
