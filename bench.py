@@ -1,0 +1,456 @@
+"""Paged decode benchmark on B200: KV-read GB/s, decode seqs/s, roofline fraction.
+
+One step = one decode step of the whole hot path for one batch:
+  cache append (pa_reshape_and_cache) -> [copy-on-write copies] -> pa_decode
+  (split-K partition kernel + merge kernel)
+on the synthetic workload (default: Llama-3-8B-shaped GQA decode, 128 sequences,
+32 q / 8 kv heads, head_dim 128, block 16, bf16, context lens uniform in
+[1024, 8192], shuffled physical blocks).  The KV cache (2.4 GB) is larger than
+L2, so no flush is needed between steps.
+
+Printed (rank 0, one JSON line):
+  value   -- algorithmic bytes per step / device step time (CUDA events), GB/s
+  e2e     -- the same metric through the public API with host buffers: host
+             pool appends + table packing, H2D of q/k/v/slots/tables, the step,
+             D2H of the output, every step
+  roofline -- pa_decode's algorithmic bytes / its measured launch time against
+             the measured HBM copy bandwidth
+  cpu_baseline -- the fp64 oracle on the host cores over a bounded sample
+
+--impl reference runs the oracle (the only reference this method has here) on
+a bounded sample of the same workload on the host cores.
+With torchrun, N ranks each run an independent replica (no data-path
+collective); value = total bytes of all ranks / max time over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "paged decode KV-read GB/s (% of B200 HBM peak) and decode seqs/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def algorithmic_bytes(cfg: wl.DecodeConfig, lens: torch.Tensor) -> dict:
+    """Bytes the step must move at minimum (no tail slots, no split-K partials)."""
+    e_kv, e_q = wl.elem_bytes(cfg.kv_dtype), wl.elem_bytes(cfg.q_dtype)
+    S, Hq, Hkv, D, bs = cfg.num_seqs, cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim, cfg.block_size
+    n = lens.to(torch.int64)
+    kv = int(n.sum()) * Hkv * D * 2 * e_kv
+    qo = S * Hq * D * 2 * e_q
+    tables = int(((n + bs - 1) // bs).sum()) * 4 + S * 4
+    decode = kv + qo + tables
+    append = S * Hkv * D * 2 * (e_q + e_kv) + S * 8
+    return {"decode": decode, "append": append, "kv": kv}
+
+
+def _pci_id(dev: int) -> str | None:
+    p = torch.cuda.get_device_properties(dev)
+    try:
+        return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+    except AttributeError:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev: int):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{dev}.csv")
+        pid = _pci_id(dev)
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            args = ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                    "-lms", "200"]
+            if pid:
+                args += ["-i", pid]
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(args, stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            c = [x.strip() for x in line.split(",")]
+            if len(c) < 9:
+                continue
+            try:
+                sm.append(float(c[1]))
+                smax = float(c[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, c[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ oracle arm
+
+def _sample_cfg(cfg: wl.DecodeConfig, nseq: int) -> wl.DecodeConfig:
+    """nseq sequences drawn like the workload's (same heads, dtypes, lengths)."""
+    import dataclasses
+    nseq = max(1, min(nseq, cfg.num_seqs))
+    if cfg.fixed_lens:
+        return dataclasses.replace(cfg, num_seqs=nseq, fixed_lens=cfg.fixed_lens[:nseq],
+                                   fixed_num_blocks=None, name=cfg.name + f"_sample{nseq}")
+    if cfg.prefix_tokens:
+        return wl.small_variant(cfg, nseq, cfg.suffix_lo, cfg.suffix_hi)
+    return wl.small_variant(cfg, nseq, cfg.ctx_lo, cfg.ctx_hi)
+
+
+def _oracle_pass(inp: wl.DecodeInputs, cores: int) -> float:
+    import oracle  # test infrastructure: only the CPU-baseline / reference legs use it
+    c = inp.cfg
+    t0 = time.perf_counter()
+    oracle.paged_decode(inp.q, c.q_dtype, inp.key_cache, inp.value_cache, c.kv_dtype,
+                        inp.block_tables, inp.context_lens, inp.scale, inp.k_scale, inp.v_scale,
+                        nthreads=cores)
+    return time.perf_counter() - t0
+
+
+def oracle_sample(cfg: wl.DecodeConfig, seed: int, pass_s: float):
+    """A sample sized so one oracle pass takes about pass_s seconds."""
+    cores = os.cpu_count() or 1
+    probe = wl.make_decode_inputs(_sample_cfg(cfg, 1), seed=seed)
+    t1 = max(_oracle_pass(probe, cores), 1e-3)
+    # one sequence occupies at most Hkv threads; more sequences fill the rest
+    per_seq = t1 / max(1.0, min(cores, cfg.num_kv_heads) / cfg.num_kv_heads * 1.0)
+    nseq = int(max(1, min(cfg.num_seqs, pass_s / per_seq * max(1, cores // cfg.num_kv_heads))))
+    return wl.make_decode_inputs(_sample_cfg(cfg, nseq), seed=seed), cores
+
+
+def cpu_oracle_rate(cfg: wl.DecodeConfig, seed: int, budget_s: float = 15.0) -> dict:
+    """The fp64 oracle on the host cores over a bounded sample of the workload."""
+    inp, cores = oracle_sample(cfg, seed, budget_s / 2)
+    t, reps = 0.0, 0
+    while reps < 1 or t < budget_s / 2:
+        t += _oracle_pass(inp, cores)
+        reps += 1
+    kv = algorithmic_bytes(inp.cfg, inp.context_lens)["kv"]
+    S = inp.cfg.num_seqs
+    return {"gbs": kv * reps / t / 1e9, "seqs_per_s": S * reps / t, "cores": cores,
+            "seconds": t / reps,
+            "sample": f"{S} sequences drawn like the workload's ({kv / 1e9:.3f} GB of K/V), "
+                      f"fp64 oracle on {cores} threads, {reps} passes"}
+
+
+def run_reference(args, cfg, rank, world):
+    if rank != 0:
+        return
+    budget = max(1.0, 150.0 / (args.warmup + args.steps))   # whole run within a few minutes
+    inp, cores = oracle_sample(cfg, args.seed, budget)
+    for _ in range(args.warmup):
+        _oracle_pass(inp, cores)
+    ts = [_oracle_pass(inp, cores) for _ in range(args.steps)]
+    kv = algorithmic_bytes(inp.cfg, inp.context_lens)["kv"]
+    sec = sum(ts) / len(ts)
+    gbs = kv / sec / 1e9
+    sample = (f"{inp.cfg.num_seqs} sequences drawn like the workload's ({kv / 1e9:.3f} GB of K/V) "
+              f"per step, fp64 oracle on {cores} threads")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * sec, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": _config_dict(cfg, args),
+        "seqs_per_s": round(inp.cfg.num_seqs / sec, 3),
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def _config_dict(cfg, args, partition=None, l2_note=None):
+    d = {"workload": cfg.name, "num_seqs": cfg.num_seqs, "q_heads": cfg.num_q_heads,
+         "kv_heads": cfg.num_kv_heads, "head_dim": cfg.head_dim, "block_size": cfg.block_size,
+         "kv_dtype": cfg.kv_dtype, "q_dtype": cfg.q_dtype,
+         "context_lens": list(cfg.fixed_lens[:1]) * 1 if cfg.fixed_lens else [cfg.ctx_lo, cfg.ctx_hi],
+         "parallelism": f"replicas{args.gpus}"}
+    if cfg.prefix_tokens:
+        d.update(prefix_tokens=cfg.prefix_tokens, suffix=[cfg.suffix_lo, cfg.suffix_hi])
+    if partition is not None:
+        d["partition"] = partition
+    if l2_note:
+        d["l2"] = l2_note
+    return d
+
+
+# --------------------------------------------------------------------- GPU arm
+
+def run_gpu(args, cfg, rank, world, local_rank):
+    import paged_kv_cache_338_b200 as pa
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    inp = wl.make_decode_inputs(cfg, seed=args.seed + rank, device=dev)
+    S, Hq, D = inp.q.shape
+    part = args.partition if args.partition >= 0 else (
+        cfg.partition or pa.pa_decode_suggest_partition(cfg.num_kv_heads, cfg.block_size,
+                                                        inp.context_lens.cpu()))
+    max_ctx = inp.max_ctx + args.warmup + args.steps + 2     # room for e2e growth
+    ws_bytes = pa.pa_decode_workspace_size(S, Hq, D, max_ctx, part)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(inp.q)
+    kc, vc = inp.key_cache, inp.value_cache
+    pairs = inp.copy_pairs
+    nbytes = algorithmic_bytes(cfg, inp.context_lens.cpu())
+    step_bytes = nbytes["decode"] + nbytes["append"]
+
+    def step(ev=None):
+        if pairs.numel():
+            pa.pa_copy_blocks(kc, vc, pairs)
+        pa.pa_reshape_and_cache(inp.key_new, inp.value_new, kc, vc, inp.slot_mapping,
+                                inp.k_scale, inp.v_scale)
+        if ev is not None:
+            ev[0].record(stream)
+        pa.pa_decode(out, inp.q, kc, vc, inp.block_tables, inp.context_lens, max_ctx, inp.scale,
+                     inp.k_scale, inp.v_scale, part, ws if ws_bytes else None)
+        if ev is not None:
+            ev[1].record(stream)
+
+    launches_per_step = (1 if pairs.numel() else 0) + 1 + 1 + (1 if ws_bytes else 0)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert pa.pa_device_status() == 0
+
+    dist = world > 1
+    if dist:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if dist:
+        torch.distributed.barrier()
+    ms = t0.elapsed_time(t1)
+    dec_ms = [a.elapsed_time(b) for a, b in evs]
+    dec_avg = sum(dec_ms) / len(dec_ms)
+    if dist:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+    value = world * step_bytes / (ms_step * 1e-3) / 1e9
+
+    # ---- end to end through the public API with host buffers -------------
+    e2e = run_e2e(args, cfg, pa, dev, part, max_ctx) if not args.no_e2e else None
+    if dist and e2e is not None:
+        t = torch.tensor([e2e["ms"]], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e["value"] = world * e2e["bytes"] / (float(t.item()) * 1e-3) / 1e9
+
+    if rank != 0:
+        return
+    peak, peak_kind = _peaks()
+    achieved = nbytes["decode"] / (dec_avg * 1e-3) / 1e9
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", f"traffic_{cfg.name}.json")
+    if os.path.exists(prof):
+        try:
+            with open(prof) as f:
+                pj = json.load(f)
+            if pj.get("partition") == part:
+                traffic = pj.get("dram_bytes_per_launch")
+        except Exception:
+            traffic = None
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        r = cpu_oracle_rate(cfg, args.seed, budget_s=args.cpu_budget)
+        cpu = {"value": round(r["gbs"], 4), "unit": "GB/s", "cores": r["cores"],
+               "kind": "oracle", "sample": r["sample"], "seqs_per_s": round(r["seqs_per_s"], 3)}
+    kv_gb = nbytes["kv"] / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.kv_dtype,
+        "data": "synthetic",
+        "config": _config_dict(cfg, args, part,
+                               f"inputs larger than L2 ({kv_gb:.2f} GB of K/V per step), no flush"),
+        "seqs_per_s": round(world * S / (ms_step * 1e-3), 1),
+        "pct_of_hbm_peak": {"measured_copy": round(100 * value / world / peak, 2),
+                            "spec_8000": round(100 * value / world / 8000.0, 2)},
+        "decode_ms": round(dec_avg, 4),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "peak_kind": peak_kind, "kernel": "pa_decode (partition + merge)"},
+        "cpu_baseline": cpu,
+        "e2e": None if e2e is None else {
+            "value": round(e2e["value"], 2), "unit": "GB/s",
+            "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+            "ms_per_step": round(e2e["ms"], 4)},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, cfg, pa, dev, part, max_ctx):
+    """Host pool + pinned host buffers + H2D / step / D2H every step."""
+    g = torch.Generator().manual_seed(args.seed + 77)
+    inp = wl.make_decode_inputs(cfg, seed=args.seed + 5, device=dev)
+    S, Hq, D = inp.q.shape
+    bs = cfg.block_size
+    NB = inp.num_blocks + S * (args.warmup + args.steps + 2) // bs + S
+    kc = torch.empty((NB,) + tuple(inp.key_cache.shape[1:]), dtype=inp.key_cache.dtype, device=dev)
+    vc = torch.empty_like(kc)
+    kc[:inp.num_blocks] = inp.key_cache
+    vc[:inp.num_blocks] = inp.value_cache
+    kc[inp.num_blocks:].zero_()
+    vc[inp.num_blocks:].zero_()
+    pool = pa.BlockPool(NB, bs)
+    # shuffle the free queue: take every block, give them back in a seeded order
+    ids = [pool.alloc() for _ in range(NB)]
+    for i in torch.randperm(NB, generator=g).tolist():
+        pool.free(ids[i])
+    lens = inp.context_lens.cpu().tolist()
+    seqs = []
+    for s in range(S):
+        sid = pool.seq_new()
+        for _ in range(lens[s] - 1):
+            pool.seq_append(sid)
+        seqs.append(sid)
+    MB = (max(lens) + args.warmup + args.steps + 2 + bs - 1) // bs
+    pin = dict(pin_memory=True)
+    q_h = inp.q.cpu().pin_memory()
+    k_h, v_h = inp.key_new.cpu().pin_memory(), inp.value_new.cpu().pin_memory()
+    out_h = torch.empty(inp.q.shape, dtype=inp.q.dtype, **pin)
+    slots_h = torch.empty(S, dtype=torch.int64, **pin)
+    tab_h = torch.empty((S, MB), dtype=torch.int32, **pin)
+    len_h = torch.empty(S, dtype=torch.int32, **pin)
+    q_d, k_d, v_d = torch.empty_like(inp.q), torch.empty_like(inp.key_new), torch.empty_like(inp.value_new)
+    slots_d = torch.empty(S, dtype=torch.int64, device=dev)
+    tab_d = torch.empty((S, MB), dtype=torch.int32, device=dev)
+    len_d = torch.empty(S, dtype=torch.int32, device=dev)
+    out_d = torch.empty_like(inp.q)
+    ws_bytes = pa.pa_decode_workspace_size(S, Hq, D, max_ctx, part)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    total_bytes = 0
+
+    def step():
+        nonlocal total_bytes
+        pairs = []
+        for i, sid in enumerate(seqs):
+            slot, src, dst = pool.seq_append(sid)
+            slots_h[i] = slot
+            if src >= 0:
+                pairs.append((src, dst))
+        pool.build_block_tables(seqs, MB, tab_h, len_h)
+        for h, d in ((q_h, q_d), (k_h, k_d), (v_h, v_d), (slots_h, slots_d), (tab_h, tab_d),
+                     (len_h, len_d)):
+            d.copy_(h, non_blocking=True)
+        if pairs:
+            pa.pa_copy_blocks(kc, vc, pairs)
+        pa.pa_reshape_and_cache(k_d, v_d, kc, vc, slots_d, inp.k_scale, inp.v_scale)
+        pa.pa_decode(out_d, q_d, kc, vc, tab_d, len_d, max_ctx, inp.scale, inp.k_scale,
+                     inp.v_scale, part, ws if ws_bytes else None)
+        out_h.copy_(out_d, non_blocking=True)
+        nb = algorithmic_bytes(cfg, len_h)
+        return nb["decode"] + nb["append"]
+
+    for _ in range(args.warmup):
+        step()
+        torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ms = 0.0
+    for _ in range(args.steps):
+        e0.record(stream)
+        total_bytes += step()
+        e1.record(stream)
+        e1.synchronize()          # the result is on the host: the step is over
+        ms += e0.elapsed_time(e1)
+    assert pa.pa_device_status() == 0
+    h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h, slots_h, tab_h, len_h))
+    d2h = out_h.numel() * out_h.element_size()
+    pool.close()
+    return {"ms": ms / args.steps, "bytes": total_bytes / args.steps,
+            "value": (total_bytes / args.steps) / (ms / args.steps * 1e-3) / 1e9,
+            "h2d": h2d, "d2h": d2h}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=3, choices=sorted(wl.CONFIGS))
+    ap.add_argument("--partition", type=int, default=-1, help="-1: workload default / heuristic")
+    ap.add_argument("--seed", type=int, default=2)
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("at least 3 warm-up steps")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    cfg = wl.CONFIGS[args.config]
+    if args.impl == "reference":
+        run_reference(args, cfg, rank, world)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_gpu(args, cfg, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,268 @@
+/*
+ * pa.h -- C ABI of the paged decode library (libpa_b200.so, sm_100a).
+ *
+ * The library implements single-token decode attention over a KV cache kept
+ * in fixed-size physical blocks ("PagedAttention 机制" §5.3.1-§5.3.4;
+ * "01. PagedAttention 详解" §3-§6), together with the cache append, the
+ * copy-on-write block copy and a host-side refcounted block pool.
+ *
+ * Conventions for every function:
+ *   - Returns a pa_status; PA_OK is 0.  No exception crosses this boundary.
+ *     pa_last_error() gives a message for the last failure on the calling
+ *     thread.
+ *   - Device pointers are plain CUDA device addresses; the CALLER owns and
+ *     allocates all device memory (caches, q, out, tables, workspace).  The
+ *     library allocates no device memory.
+ *   - Device work is enqueued asynchronously on the caller's stream
+ *     (pa_stream_t is cudaStream_t; NULL is the legacy default stream).
+ *     Argument checks are done on the host before anything is enqueued; a
+ *     failed check enqueues nothing.  A launch failure returns PA_ERR_CUDA.
+ *   - Values that live in device memory (block ids, slots) cannot be checked
+ *     on the host without a synchronisation.  The kernels check them, skip the
+ *     offending access (a TMA load outside the cache reads zeros; a store is
+ *     dropped) and set a sticky bit readable with pa_device_status().  No
+ *     kernel here traps, asserts, or waits without a bound.
+ *
+ * Layouts ("01. PagedAttention 详解" §3, the cache shape of its
+ * FlashAttention backend), all row-major:
+ *   key_cache, value_cache : [NB, bs, Hkv, D]     physical blocks
+ *   q, out                 : [S, Hq, D]
+ *   block_tables           : [S, MB] int32         physical block ids
+ *   context_lens           : [S] int32             tokens to attend, >= 0
+ *   slot_mapping           : [T] int64             block * bs + offset, < 0 skips
+ *   key, value (append)    : [T, Hkv, D]
+ * where S = sequences, Hq / Hkv = query / kv heads (Hq % Hkv == 0, query head
+ * h reads kv head h / (Hq / Hkv)), D = head dim, bs = block size, NB = number
+ * of physical blocks, MB = table width.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* pa_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = 1,   /* a size, pointer, dtype or value is not acceptable */
+    PA_ERR_UNSUPPORTED = 2,   /* valid, but no kernel is built for this shape/dtype */
+    PA_ERR_OUT_OF_BLOCKS = 3, /* the pool has no free block (state unchanged) */
+    PA_ERR_REFCOUNT = 4,      /* free of a free block, sharing a free block */
+    PA_ERR_BAD_INDEX = 5,     /* unknown sequence / block id (host side) */
+    PA_ERR_CUDA = 6           /* a CUDA runtime call failed */
+} pa_status;
+
+typedef enum {
+    PA_F32 = 0,
+    PA_F16 = 1,
+    PA_BF16 = 2,
+    PA_FP8_E4M3 = 3 /* OCP E4M3 "FN": bias 7, max 448, no inf, S.1111.111 = NaN */
+} pa_dtype;
+
+/* Device-side error bits (sticky until read with clear != 0). */
+enum {
+    PA_DEV_BAD_SLOT = 1,      /* pa_reshape_and_cache: slot >= NB * bs, token skipped */
+    PA_DEV_BAD_BLOCK = 2,     /* pa_decode: table entry outside [0, NB) (read as zeros) */
+    PA_DEV_WAIT_TIMEOUT = 4,  /* a pipeline wait gave up after its bound; output invalid */
+    PA_DEV_BAD_CONTEXT = 8    /* pa_decode: context_lens[s] < 0, > max_ctx or > MB * bs (clamped) */
+};
+
+/* Message for the last failing call on this thread ("" if none). */
+const char* pa_last_error(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int pa_version(void);
+
+/*
+ * Read (and with clear != 0, reset) the sticky device error bits of the
+ * current device.  Synchronises `stream` first so the bits cover all work
+ * enqueued on it.
+ */
+pa_status pa_device_status(unsigned int* bits, int clear, pa_stream_t stream);
+
+/*
+ * Cache append -- "01. PagedAttention 详解" §4, decode step 2 (write the new
+ * token's k, v into the next slot of the last block) and prefill step 2 (write
+ * N tokens' K, V through the block table).
+ *
+ * For every t < T with slot = slot_mapping[t] >= 0, b = slot / bs,
+ * o = slot % bs:  key_cache[b, o, h, :] = cvt(key[t, h, :]) for all h, and the
+ * same for value.  cvt is a byte copy when in_dt == cache_dt.  With
+ * cache_dt == PA_FP8_E4M3 (intelliparadigm PagedAttention article §4.3,
+ * kv_cache_dtype "fp8"), cvt(x) rounds x / k_scale (binary32 division) to the
+ * nearest E4M3 value, ties to even, saturating at +-448; in_dt is then
+ * PA_F32, PA_F16 or PA_BF16.  Other dtype pairs: PA_ERR_UNSUPPORTED.
+ * k_scale and v_scale must be finite and > 0, and 1.0 unless the cache is fp8.
+ *
+ * key, value: device [T, Hkv, D] in_dt.  slot_mapping: device int64 [T].
+ * A slot >= NB * bs is skipped and sets PA_DEV_BAD_SLOT.  Two tokens with the
+ * same slot: one of them wins (unspecified which).  T == 0 is a no-op.
+ * D * element size must be a multiple of 16 bytes; pointers 16-byte aligned.
+ */
+pa_status pa_reshape_and_cache(const void* key, const void* value, pa_dtype in_dt,
+                               void* key_cache, void* value_cache, pa_dtype cache_dt,
+                               const int64_t* slot_mapping, int T, int Hkv, int D, int bs,
+                               int64_t NB, float k_scale, float v_scale, pa_stream_t stream);
+
+/*
+ * Copy-on-write block copy -- intelliparadigm PagedAttention article §3.3
+ * (maybe_copy_block: allocate, copy_block, drop the old reference) and
+ * "PagedAttention 机制" §5.3.2 (copy only when a shared block is written).
+ *
+ * For each pair i: key_cache block pairs[2i+1] = key_cache block pairs[2i]
+ * (all block_bytes of it), and the same for value_cache.  block_bytes is
+ * bs * Hkv * D * element size and must be a multiple of 16.
+ * pairs: HOST int32 [n, 2] (src, dst) -- the pool decides copies on the host,
+ * and the list travels in the kernel's parameters, so no device buffer is
+ * needed.  Rejected on the host (PA_ERR_INVALID_ARG): an id outside [0, NB), a
+ * destination that repeats, a destination that is also a source.
+ * n == 0 is a no-op.
+ */
+pa_status pa_copy_blocks(void* key_cache, void* value_cache, size_t block_bytes, int64_t NB,
+                         const int32_t* pairs, int n, pa_stream_t stream);
+
+/*
+ * Bytes of split-K workspace pa_decode needs for these sizes (0 when
+ * partition == 0 or max_ctx <= partition).  Layout (fp32): per (s, query
+ * head, partition) a running max m, a sum l, and an unnormalised o[D].
+ */
+pa_status pa_decode_workspace_size(int S, int Hq, int D, int max_ctx, int partition,
+                                   size_t* bytes);
+
+/*
+ * Split size pa_decode would pick for this batch to fill the GPU: a multiple
+ * of bs, or 0 for a single pass.  Host-only heuristic, no device access.
+ */
+pa_status pa_decode_suggest_partition(int S, int Hkv, int bs, const int32_t* context_lens_host,
+                                      int* partition);
+
+/*
+ * Paged decode attention -- "PagedAttention 机制" §5.3.4 (paged_attention:
+ * logical token i is key_cache[block_tables[i // bs], i % bs]);
+ * intelliparadigm PagedAttention article §2.3 (q.K per block, softmax
+ * normalised over all blocks, weighted sum of V); "01. PagedAttention 详解" §4
+ * (per-block partial results accumulated; v2 splits long sequences, split-K).
+ *
+ * For every s < S and query head h, g = h / (Hq / Hkv), n = context_lens[s]:
+ *   k_i = deq(key_cache[block_tables[s, i / bs], i % bs, g, :]),  i < n
+ *   z_i = scale * <q[s, h, :], k_i>
+ *   out[s, h, :] = sum_i softmax(z)_i * deq(value_cache[..same slot.., g, :])
+ * deq(x) = x * k_scale (keys) or x * v_scale (values) for fp8, x otherwise.
+ * Accumulation is fp32; out is rounded to nearest-even in q_dt.  n == 0 gives
+ * a zero row.  Table entries at or past ceil(n / bs) and cache slots at or
+ * past n are never read.
+ *
+ * dtypes: cache_dt == q_dt for F32 / F16 / BF16; cache_dt == PA_FP8_E4M3 with
+ * q_dt F16 or BF16.  bs in {8, 16, 32}; D in {64, 128, 256} with D * element
+ * size of the cache in {128, 256, 512} bytes; Hq / Hkv in {1, 2, 4, 8, 16}.
+ * Base pointers 16-byte aligned (TMA requirement).
+ *
+ * partition: 0 = one pass per (sequence, kv head); otherwise tokens per
+ * split-K partition, a positive multiple of bs.  Sequences longer than one
+ * partition are split; each partition writes (m, l, o) into `workspace`
+ * (device, >= pa_decode_workspace_size() bytes, no initialisation needed)
+ * and a second kernel on the same stream merges them.  max_ctx must be
+ * >= every context_lens[s] (it sizes the grid and the workspace).
+ */
+pa_status pa_decode(void* out, const void* q, pa_dtype q_dt,
+                    const void* key_cache, const void* value_cache, pa_dtype cache_dt,
+                    const int32_t* block_tables, int MB, const int32_t* context_lens,
+                    int S, int Hq, int Hkv, int D, int bs, int64_t NB, int max_ctx,
+                    float scale, float k_scale, float v_scale, int partition,
+                    void* workspace, size_t workspace_bytes, pa_stream_t stream);
+
+/*
+ * Consumer selection for pa_decode (process-wide; for tests and tuning):
+ * 0 = automatic (tensor-core consumer for grouped-query heads with 16-bit
+ * caches and D <= 128, CUDA-core consumer otherwise), 1 = CUDA-core consumer
+ * everywhere.  Both compute the same function.
+ */
+pa_status pa_decode_select(int mode);
+
+/* ------------------------------------------------------------------------
+ * Host block pool -- "PagedAttention 机制" §5.3.4 (BlockAllocator: free list,
+ * per-block reference count, allocate / free / incr_ref, out-of-memory when
+ * empty) with the FIFO free queue of "01. PagedAttention 详解" self-check 3
+ * (get_new_blocks takes from the head, free_blocks returns a block to the
+ * tail when its count reaches 0), per-sequence block tables ("PagedAttention
+ * 机制" §5.3.2), sharing by reference counts (same page §6: prefix sharing,
+ * beam search and parallel sampling) and copy-on-write (intelliparadigm
+ * PagedAttention article §3.3).
+ *
+ * Not thread-safe: one scheduler thread owns a pool.  No device access.
+ * Sequence ids are int64 handles returned by the pool.
+ * ------------------------------------------------------------------------ */
+typedef struct pa_pool pa_pool;
+
+typedef struct {
+    int64_t num_blocks;
+    int64_t free_blocks;
+    int64_t used_blocks;    /* reference count > 0 */
+    int64_t shared_blocks;  /* reference count > 1 */
+    int64_t cow_copies;     /* copies requested by pa_pool_seq_append so far */
+    int64_t num_seqs;
+} pa_pool_stats_t;
+
+pa_status pa_pool_create(int64_t NB, int bs, pa_pool** out);
+void pa_pool_destroy(pa_pool* pool);
+
+/* Take the head of the free queue; its count becomes 1. */
+pa_status pa_pool_alloc(pa_pool* pool, int32_t* block);
+/* Drop one reference; at 0 the block goes to the tail of the free queue. */
+pa_status pa_pool_free(pa_pool* pool, int32_t block);
+/* Add a reference to a block in use (PA_ERR_REFCOUNT if it is free). */
+pa_status pa_pool_incr_ref(pa_pool* pool, int32_t block);
+/* Reference count of a block (-1 if the id is out of range). */
+int pa_pool_ref(const pa_pool* pool, int32_t block);
+
+/* New empty sequence. */
+pa_status pa_pool_seq_new(pa_pool* pool, int64_t* seq);
+/* New sequence sharing all of parent's blocks (one more reference each).
+ * PA_ERR_REFCOUNT (and no change) if one of them was freed behind the pool's back. */
+pa_status pa_pool_seq_fork(pa_pool* pool, int64_t parent, int64_t* child);
+/*
+ * An EMPTY sequence takes a reference on n existing blocks holding its first
+ * num_tokens tokens (a shared prefix); n must equal ceil(num_tokens / bs).
+ */
+pa_status pa_pool_seq_share_prefix(pa_pool* pool, int64_t seq, const int32_t* blocks, int n,
+                                   int64_t num_tokens);
+/*
+ * Make room for one more token of `seq` and return its slot
+ * (block * bs + offset).  A new block is taken when the last one is full.  If
+ * the last block is shared (count > 1) it is copied first: a fresh block is
+ * taken, *cow_src / *cow_dst name the copy the caller must enqueue (with
+ * pa_copy_blocks, before writing the slot), the old block loses one reference
+ * and the table now points at the new one; otherwise both are -1.  On
+ * PA_ERR_OUT_OF_BLOCKS nothing changes.
+ */
+pa_status pa_pool_seq_append(pa_pool* pool, int64_t seq, int64_t* slot, int32_t* cow_src,
+                             int32_t* cow_dst);
+/* Drop the sequence's reference on each of its blocks, in table order.  All
+ * or nothing: PA_ERR_REFCOUNT (and no change) if a block holds fewer
+ * references than the sequence does. */
+pa_status pa_pool_seq_free(pa_pool* pool, int64_t seq);
+/* Tokens held by a sequence (-1 if unknown). */
+int64_t pa_pool_seq_len(const pa_pool* pool, int64_t seq);
+
+/*
+ * Pack the tables of `seqs` into one host buffer for one host-to-device copy
+ * per step ("01. PagedAttention 详解" §10: all active tables go to the GPU as
+ * one tensor, not one small copy per request).  tables_host: [S, MB] int32,
+ * entries past a sequence's blocks are -1; ctx_lens_host: [S] int32.
+ * PA_ERR_INVALID_ARG if a sequence holds more than MB blocks.
+ */
+pa_status pa_pool_build_block_tables(const pa_pool* pool, const int64_t* seqs, int S, int MB,
+                                     int32_t* tables_host, int32_t* ctx_lens_host);
+
+pa_status pa_pool_stats(const pa_pool* pool, pa_pool_stats_t* stats);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

@@ -19,13 +19,15 @@ Plain Python, one step per rule on the pages:
 * "01. PagedAttention 详解" §6 and summary: sequences may share blocks (a common
   prefix, or a fork for beam search / parallel sampling) by adding references.
 
-Misuse (freeing a free block, adding a reference to a free block, an unknown
-sequence) raises PoolError with the matching status name; running out of free
-blocks raises OutOfBlocks and leaves the state unchanged.
+Misuse raises a PoolError subclass whose ``status`` names the library's
+status code: freeing a free block or sharing a free block (PA_ERR_REFCOUNT),
+an unknown sequence or an out-of-range block id (PA_ERR_BAD_INDEX), malformed
+requests (PA_ERR_INVALID_ARG); running out of free blocks raises OutOfBlocks
+(PA_ERR_OUT_OF_BLOCKS) and leaves the state unchanged.
 """
 from __future__ import annotations
 
-from collections import deque
+from collections import Counter, deque
 
 
 class PoolError(Exception):
@@ -38,6 +40,10 @@ class OutOfBlocks(PoolError):
 
 class InvalidArg(PoolError):
     status = "PA_ERR_INVALID_ARG"
+
+
+class BadIndex(PoolError):
+    status = "PA_ERR_BAD_INDEX"
 
 
 class PoolModel:
@@ -55,7 +61,7 @@ class PoolModel:
     # -- blocks -----------------------------------------------------------
     def _check_block(self, b):
         if not (0 <= b < self.num_blocks):
-            raise InvalidArg(f"block {b} out of range")
+            raise BadIndex(f"block {b} out of range")
 
     def alloc(self) -> int:
         if not self.free_queue:
@@ -81,7 +87,7 @@ class PoolModel:
     # -- sequences --------------------------------------------------------
     def _seq(self, sid):
         if sid not in self.seqs:
-            raise InvalidArg(f"unknown sequence {sid}")
+            raise BadIndex(f"unknown sequence {sid}")
         return self.seqs[sid]
 
     def seq_new(self) -> int:
@@ -92,8 +98,11 @@ class PoolModel:
 
     def seq_fork(self, parent: int) -> int:
         blocks, n = self._seq(parent)
+        for b in blocks:                     # all or nothing
+            if self.ref[b] <= 0:
+                raise PoolError(f"block {b} is free")
         for b in blocks:
-            self.incr_ref(b)
+            self.ref[b] += 1
         sid = self.seq_new()
         self.seqs[sid] = [list(blocks), n]
         return sid
@@ -135,6 +144,9 @@ class PoolModel:
 
     def seq_free(self, sid: int) -> None:
         blocks, _ = self._seq(sid)
+        for b, k in Counter(blocks).items():  # all or nothing
+            if self.ref[b] < k:
+                raise PoolError(f"block {b} has fewer references than the sequence holds")
         for b in blocks:
             self.free(b)
         del self.seqs[sid]

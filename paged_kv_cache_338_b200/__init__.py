@@ -1,0 +1,295 @@
+"""Python binding of libpa_b200.so: paged decode attention on B200 (sm_100a).
+
+Thin ctypes marshalling over the C ABI declared in include/pa.h -- every
+function here has the name of the C entry point it calls, takes torch tensors
+(device memory, owned by the caller) and passes their pointers, sizes and
+dtypes through.  All computation happens in the library's CUDA kernels; there
+is no fallback: if the shared library is missing or fails to load, every call
+raises.
+
+Build the library with ``python -m paged_kv_cache_338_b200.build`` (or
+``__graft_entry__.build()``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+__all__ = [
+    "PaError", "lib", "pa_version", "pa_last_error", "pa_device_status",
+    "pa_reshape_and_cache", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_size",
+    "pa_decode_suggest_partition", "pa_decode_select", "BlockPool",
+    "PA_DEV_BAD_SLOT", "PA_DEV_BAD_BLOCK", "PA_DEV_WAIT_TIMEOUT", "PA_DEV_BAD_CONTEXT",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpa_b200.so")
+
+# pa_status / pa_dtype / device error bits (include/pa.h)
+STATUS = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED",
+          3: "PA_ERR_OUT_OF_BLOCKS", 4: "PA_ERR_REFCOUNT", 5: "PA_ERR_BAD_INDEX",
+          6: "PA_ERR_CUDA"}
+PA_F32, PA_F16, PA_BF16, PA_FP8_E4M3 = 0, 1, 2, 3
+PA_DEV_BAD_SLOT, PA_DEV_BAD_BLOCK, PA_DEV_WAIT_TIMEOUT, PA_DEV_BAD_CONTEXT = 1, 2, 4, 8
+
+_TORCH_DT = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16,
+             torch.float8_e4m3fn: PA_FP8_E4M3, torch.uint8: PA_FP8_E4M3}
+
+
+class PaError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        self.status = STATUS.get(status, str(status))
+        super().__init__(f"{self.status}: {msg}")
+
+
+class _Stats(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in
+                ("num_blocks", "free_blocks", "used_blocks", "shared_blocks", "cow_copies",
+                 "num_seqs")]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library; raises if it is not built (no CPU fallback exists)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m paged_kv_cache_338_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, I32, I64, F, SZ = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int32, ctypes.c_int64,
+                             ctypes.c_float, ctypes.c_size_t)
+    sig = {
+        "pa_last_error": ([], ctypes.c_char_p),
+        "pa_version": ([], I),
+        "pa_device_status": ([ctypes.POINTER(ctypes.c_uint), I, P], I),
+        "pa_reshape_and_cache": ([P, P, I, P, P, I, P, I, I, I, I, I64, F, F, P], I),
+        "pa_copy_blocks": ([P, P, SZ, I64, P, I, P], I),
+        "pa_decode_workspace_size": ([I, I, I, I, I, ctypes.POINTER(SZ)], I),
+        "pa_decode_suggest_partition": ([I, I, I, P, ctypes.POINTER(I)], I),
+        "pa_decode_select": ([I], I),
+        "pa_decode": ([P, P, I, P, P, I, P, I, P, I, I, I, I, I, I64, I, F, F, F, I, P, SZ, P], I),
+        "pa_pool_create": ([I64, I, ctypes.POINTER(P)], I),
+        "pa_pool_destroy": ([P], None),
+        "pa_pool_alloc": ([P, ctypes.POINTER(I32)], I),
+        "pa_pool_free": ([P, I32], I),
+        "pa_pool_incr_ref": ([P, I32], I),
+        "pa_pool_ref": ([P, I32], I),
+        "pa_pool_seq_new": ([P, ctypes.POINTER(I64)], I),
+        "pa_pool_seq_fork": ([P, I64, ctypes.POINTER(I64)], I),
+        "pa_pool_seq_share_prefix": ([P, I64, P, I, I64], I),
+        "pa_pool_seq_append": ([P, I64, ctypes.POINTER(I64), ctypes.POINTER(I32),
+                                ctypes.POINTER(I32)], I),
+        "pa_pool_seq_free": ([P, I64], I),
+        "pa_pool_seq_len": ([P, I64], I64),
+        "pa_pool_build_block_tables": ([P, P, I, I, P, P], I),
+        "pa_pool_stats": ([P, ctypes.POINTER(_Stats)], I),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = L
+    return L
+
+
+def pa_last_error() -> str:
+    return lib().pa_last_error().decode()
+
+
+def _check(st: int) -> None:
+    if st != 0:
+        raise PaError(st, pa_last_error())
+
+
+def pa_version() -> int:
+    return lib().pa_version()
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        if not torch.cuda.is_available():       # host-only calls (argument checks)
+            return ctypes.c_void_p(0)
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        stream = stream.cuda_stream
+    return ctypes.c_void_p(int(stream))
+
+
+def _dt(t: torch.Tensor) -> int:
+    try:
+        return _TORCH_DT[t.dtype]
+    except KeyError:
+        raise PaError(1, f"unsupported dtype {t.dtype}") from None
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise PaError(1, "tensors must be contiguous")
+    return t.data_ptr()
+
+
+def pa_device_status(clear: bool = True, stream=None) -> int:
+    """Sticky device error bits (PA_DEV_*); synchronises the stream."""
+    bits = ctypes.c_uint(0)
+    _check(lib().pa_device_status(ctypes.byref(bits), int(clear), _stream(stream)))
+    return bits.value
+
+
+def pa_reshape_and_cache(key: torch.Tensor, value: torch.Tensor, key_cache: torch.Tensor,
+                         value_cache: torch.Tensor, slot_mapping: torch.Tensor,
+                         k_scale: float = 1.0, v_scale: float = 1.0, stream=None) -> None:
+    """key/value [T, Hkv, D]; caches [NB, bs, Hkv, D]; slot_mapping [T] int64."""
+    T, Hkv, D = key.shape
+    NB, bs = key_cache.shape[0], key_cache.shape[1]
+    if slot_mapping.dtype != torch.int64:
+        raise PaError(1, "slot_mapping must be int64")
+    _check(lib().pa_reshape_and_cache(_ptr(key), _ptr(value), _dt(key), _ptr(key_cache),
+                                      _ptr(value_cache), _dt(key_cache), _ptr(slot_mapping),
+                                      T, Hkv, D, bs, NB, float(k_scale), float(v_scale),
+                                      _stream(stream)))
+
+
+def pa_copy_blocks(key_cache: torch.Tensor, value_cache: torch.Tensor, pairs,
+                   stream=None) -> None:
+    """pairs: host [n, 2] int32 (src, dst) -- a CPU tensor, array or list of pairs."""
+    pr = torch.as_tensor(pairs, dtype=torch.int32).reshape(-1, 2).contiguous()
+    if pr.device.type != "cpu":
+        raise PaError(1, "pairs live in host memory")
+    NB = key_cache.shape[0]
+    block_bytes = key_cache[0].numel() * key_cache.element_size() if NB else 0
+    _check(lib().pa_copy_blocks(_ptr(key_cache), _ptr(value_cache), block_bytes, NB,
+                                pr.data_ptr() if pr.numel() else None, pr.shape[0],
+                                _stream(stream)))
+
+
+def pa_decode_workspace_size(S: int, Hq: int, D: int, max_ctx: int, partition: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().pa_decode_workspace_size(S, Hq, D, max_ctx, partition, ctypes.byref(n)))
+    return n.value
+
+
+def pa_decode_suggest_partition(Hkv: int, block_size: int, context_lens_host) -> int:
+    cl = torch.as_tensor(context_lens_host, dtype=torch.int32).contiguous()
+    out = ctypes.c_int(0)
+    _check(lib().pa_decode_suggest_partition(cl.numel(), Hkv, block_size,
+                                             cl.data_ptr() if cl.numel() else None,
+                                             ctypes.byref(out)))
+    return out.value
+
+
+def pa_decode_select(mode: int) -> None:
+    """0: automatic consumer choice; 1: CUDA-core consumer everywhere."""
+    _check(lib().pa_decode_select(int(mode)))
+
+
+def pa_decode(out: torch.Tensor, q: torch.Tensor, key_cache: torch.Tensor,
+              value_cache: torch.Tensor, block_tables: torch.Tensor, context_lens: torch.Tensor,
+              max_ctx: int, scale: float, k_scale: float = 1.0, v_scale: float = 1.0,
+              partition: int = 0, workspace: Optional[torch.Tensor] = None,
+              stream=None) -> None:
+    """out/q [S, Hq, D]; caches [NB, bs, Hkv, D]; block_tables [S, MB] int32;
+    context_lens [S] int32; workspace: device bytes >= pa_decode_workspace_size()."""
+    S, Hq, D = q.shape
+    NB, bs, Hkv, _ = key_cache.shape
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise PaError(1, "block_tables and context_lens must be int32")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().pa_decode(_ptr(out), _ptr(q), _dt(q), _ptr(key_cache), _ptr(value_cache),
+                           _dt(key_cache), _ptr(block_tables), MB, _ptr(context_lens), S, Hq,
+                           Hkv, D, bs, NB, int(max_ctx), float(scale), float(k_scale),
+                           float(v_scale), int(partition), _ptr(workspace), ws_bytes,
+                           _stream(stream)))
+
+
+class BlockPool:
+    """Host refcounted block pool (pa_pool_*): FIFO free queue, per-sequence
+    block tables, sharing and copy-on-write decisions.  Not thread-safe."""
+
+    def __init__(self, num_blocks: int, block_size: int):
+        self._p = ctypes.c_void_p()
+        _check(lib().pa_pool_create(num_blocks, block_size, ctypes.byref(self._p)))
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+
+    def close(self):
+        if self._p:
+            lib().pa_pool_destroy(self._p)
+            self._p = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:  # interpreter shutdown
+            pass
+
+    def alloc(self) -> int:
+        b = ctypes.c_int32()
+        _check(lib().pa_pool_alloc(self._p, ctypes.byref(b)))
+        return b.value
+
+    def free(self, block: int) -> None:
+        _check(lib().pa_pool_free(self._p, block))
+
+    def incr_ref(self, block: int) -> None:
+        _check(lib().pa_pool_incr_ref(self._p, block))
+
+    def ref(self, block: int) -> int:
+        return lib().pa_pool_ref(self._p, block)
+
+    def seq_new(self) -> int:
+        s = ctypes.c_int64()
+        _check(lib().pa_pool_seq_new(self._p, ctypes.byref(s)))
+        return s.value
+
+    def seq_fork(self, parent: int) -> int:
+        s = ctypes.c_int64()
+        _check(lib().pa_pool_seq_fork(self._p, parent, ctypes.byref(s)))
+        return s.value
+
+    def seq_share_prefix(self, seq: int, blocks: Sequence[int], num_tokens: int) -> None:
+        arr = (ctypes.c_int32 * len(blocks))(*blocks)
+        _check(lib().pa_pool_seq_share_prefix(self._p, seq, arr, len(blocks), num_tokens))
+
+    def seq_append(self, seq: int):
+        """-> (slot, cow_src, cow_dst); cow_* are -1 when no copy is needed."""
+        slot, src, dst = ctypes.c_int64(), ctypes.c_int32(), ctypes.c_int32()
+        _check(lib().pa_pool_seq_append(self._p, seq, ctypes.byref(slot), ctypes.byref(src),
+                                        ctypes.byref(dst)))
+        return slot.value, src.value, dst.value
+
+    def seq_free(self, seq: int) -> None:
+        _check(lib().pa_pool_seq_free(self._p, seq))
+
+    def seq_len(self, seq: int) -> int:
+        return lib().pa_pool_seq_len(self._p, seq)
+
+    def build_block_tables(self, seqs: Sequence[int], max_blocks: int,
+                           tables_out: Optional[torch.Tensor] = None,
+                           lens_out: Optional[torch.Tensor] = None):
+        """Pack the tables into host int32 [S, max_blocks] (-1 padded) + lens [S]."""
+        S = len(seqs)
+        ids = (ctypes.c_int64 * S)(*seqs)
+        if tables_out is None:
+            tables_out = torch.empty((S, max_blocks), dtype=torch.int32)
+        if lens_out is None:
+            lens_out = torch.empty((S,), dtype=torch.int32)
+        assert tables_out.device.type == "cpu" and lens_out.device.type == "cpu"
+        _check(lib().pa_pool_build_block_tables(self._p, ids, S, max_blocks,
+                                                 tables_out.data_ptr() if tables_out.numel() else None,
+                                                 lens_out.data_ptr() if S else None))
+        return tables_out, lens_out
+
+    def stats(self) -> dict:
+        st = _Stats()
+        _check(lib().pa_pool_stats(self._p, ctypes.byref(st)))
+        return {n: getattr(st, n) for n, _ in _Stats._fields_}

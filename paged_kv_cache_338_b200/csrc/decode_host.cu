@@ -1,0 +1,242 @@
+// Host side of pa_decode: argument checks, tensor maps over the paged caches,
+// split-K partitioning, kernel selection and launches.
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <mutex>
+
+#include "decode_launch.h"
+#include "pa_internal.h"
+
+namespace pa {
+namespace {
+
+std::atomic<int> g_select{0};   // 0: automatic, 1: CUDA-core consumer only
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
+                                             cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+CUtensorMapDataType tma_type(pa_dtype dt) {
+    switch (dt) {
+    case PA_F32: return CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    case PA_F16: return CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    case PA_BF16: return CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    default: return CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    }
+}
+
+// The cache [NB, bs, Hkv, D] as a 5-D tensor {D/seg, seg_count, Hkv, bs, NB}
+// (innermost first) whose box {seg, seg_count, 1, bs, 1} is the K (or V)
+// tile of one block for one kv head, in 128-byte swizzled rows.
+pa_status make_map(CUtensorMap* m, const void* base, pa_dtype dt, int64_t NB, int bs, int Hkv,
+                   int D) {
+    auto fn = encode_fn();
+    if (!fn) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    const int e = elem_size(dt);
+    const cuuint64_t row = (cuuint64_t)D * e;            // bytes of one (token, head) row
+    const cuuint64_t seg = 128 / e;                      // elements per 128-byte segment
+    cuuint64_t dims[5] = {seg, row / 128, (cuuint64_t)Hkv, (cuuint64_t)bs, (cuuint64_t)NB};
+    cuuint64_t strides[4] = {128, row, row * Hkv, row * Hkv * bs};
+    cuuint32_t box[5] = {(cuuint32_t)seg, (cuuint32_t)(row / 128), 1, (cuuint32_t)bs, 1};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = fn(m, tma_type(dt), 5, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return PA_OK;
+}
+
+template <int QT, int D>
+cudaError_t launch_merge_t(const dec::Params& p, dim3 grid, cudaStream_t st) {
+    dec::decode_merge<QT, D><<<grid, D, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+template <int QT>
+cudaError_t launch_merge_q(const dec::Params& p, int D, dim3 grid, cudaStream_t st) {
+    switch (D) {
+    case 64: return launch_merge_t<QT, 64>(p, grid, st);
+    case 128: return launch_merge_t<QT, 128>(p, grid, st);
+    case 256: return launch_merge_t<QT, 256>(p, grid, st);
+    }
+    return cudaErrorNotSupported;
+}
+
+cudaError_t launch_merge(const dec::Params& p, pa_dtype qt, int D, dim3 grid, cudaStream_t st) {
+    switch (qt) {
+    case PA_F32: return launch_merge_q<PA_F32>(p, D, grid, st);
+    case PA_F16: return launch_merge_q<PA_F16>(p, D, grid, st);
+    case PA_BF16: return launch_merge_q<PA_BF16>(p, D, grid, st);
+    default: return cudaErrorNotSupported;
+    }
+}
+
+int64_t parts_for(int max_ctx, int partition) {
+    if (partition <= 0 || max_ctx <= partition) return 1;
+    return ((int64_t)max_ctx + partition - 1) / partition;
+}
+
+bool is_pow2_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8 || g == 16; }
+
+}  // namespace
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" pa_status pa_decode_workspace_size(int S, int Hq, int D, int max_ctx, int partition,
+                                              size_t* bytes) {
+    clear_error();
+    if (!bytes) return fail(PA_ERR_INVALID_ARG, "bytes is NULL");
+    if (S < 0 || Hq <= 0 || D <= 0 || max_ctx < 0 || partition < 0)
+        return fail(PA_ERR_INVALID_ARG, "negative or zero size");
+    const int64_t mp = parts_for(max_ctx, partition);
+    *bytes = mp <= 1 ? 0 : (size_t)S * Hq * mp * (sizeof(float) * 2 + sizeof(float) * D);
+    return PA_OK;
+}
+
+extern "C" pa_status pa_decode_suggest_partition(int S, int Hkv, int bs,
+                                                 const int32_t* context_lens_host, int* partition) {
+    clear_error();
+    if (!partition || (S > 0 && !context_lens_host) || S < 0 || Hkv <= 0 ||
+        !(bs == 8 || bs == 16 || bs == 32))
+        return fail(PA_ERR_INVALID_ARG, "bad arguments");
+    // Enough CTAs for several waves on 148 SMs (a few resident per SM) so the
+    // last wave is short, with partitions no shorter than 256 tokens.
+    const int64_t want = 148LL * 3 * 8;
+    int64_t maxn = 0;
+    for (int s = 0; s < S; ++s) maxn = context_lens_host[s] > maxn ? context_lens_host[s] : maxn;
+    auto items = [&](int64_t P) {
+        int64_t it = 0;
+        for (int s = 0; s < S; ++s) it += (context_lens_host[s] + P - 1) / P;
+        return it * Hkv;
+    };
+    if (maxn == 0 || items(maxn) >= want) { *partition = 0; return PA_OK; }
+    int64_t best = 256;
+    for (int64_t P = 256; P < maxn; P *= 2)
+        if (items(P) >= want) best = P;
+    best = (best + bs - 1) / bs * bs;
+    *partition = best >= maxn ? 0 : (int)best;
+    return PA_OK;
+}
+
+extern "C" pa_status pa_decode_select(int mode) {
+    clear_error();
+    if (mode < 0 || mode > 1) return fail(PA_ERR_INVALID_ARG, "mode must be 0 or 1");
+    g_select.store(mode);
+    return PA_OK;
+}
+
+extern "C" pa_status pa_decode(void* out, const void* q, pa_dtype q_dt, const void* key_cache,
+                               const void* value_cache, pa_dtype cache_dt,
+                               const int32_t* block_tables, int MB, const int32_t* context_lens,
+                               int S, int Hq, int Hkv, int D, int bs, int64_t NB, int max_ctx,
+                               float scale, float k_scale, float v_scale, int partition,
+                               void* workspace, size_t workspace_bytes, pa_stream_t stream) {
+    clear_error();
+    if (!valid_dtype(q_dt) || !valid_dtype(cache_dt)) return fail(PA_ERR_INVALID_ARG, "bad dtype");
+    if (S < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || MB < 0 || NB <= 0 || max_ctx < 0 || partition < 0)
+        return fail(PA_ERR_INVALID_ARG, "negative or zero size");
+    if (Hq % Hkv) return fail(PA_ERR_INVALID_ARG, "Hq (%d) is not a multiple of Hkv (%d)", Hq, Hkv);
+    if (!(bs == 8 || bs == 16 || bs == 32))
+        return fail(PA_ERR_UNSUPPORTED, "block size %d (supported: 8, 16, 32)", bs);
+    if (partition % bs) return fail(PA_ERR_INVALID_ARG, "partition %d is not a multiple of bs", partition);
+    if (NB > 0x7fffffffLL) return fail(PA_ERR_INVALID_ARG, "NB exceeds int32 block ids");
+    if (!(std::isfinite(scale)) || !(std::isfinite(k_scale) && k_scale > 0) ||
+        !(std::isfinite(v_scale) && v_scale > 0))
+        return fail(PA_ERR_INVALID_ARG, "scales must be finite (k_scale, v_scale > 0)");
+    if (cache_dt != PA_FP8_E4M3 && (k_scale != 1.f || v_scale != 1.f))
+        return fail(PA_ERR_INVALID_ARG, "k_scale / v_scale apply to fp8 caches only");
+    const bool pair_ok = (cache_dt == q_dt && cache_dt != PA_FP8_E4M3) ||
+                         (cache_dt == PA_FP8_E4M3 && (q_dt == PA_F16 || q_dt == PA_BF16));
+    if (!pair_ok) return fail(PA_ERR_UNSUPPORTED, "cache dtype %d with q dtype %d", cache_dt, q_dt);
+    const int row = D * elem_size(cache_dt);
+    if (!((D == 64 || D == 128 || D == 256) && (row == 128 || row == 256 || row == 512)))
+        return fail(PA_ERR_UNSUPPORTED, "head dim %d with this cache dtype", D);
+    const int G = Hq / Hkv;
+    if (!is_pow2_group(G)) return fail(PA_ERR_UNSUPPORTED, "group size %d", G);
+    if (S == 0) return PA_OK;
+    if (S > 65535 || (int64_t)Hkv * G > 65535) return fail(PA_ERR_UNSUPPORTED, "grid too large");
+    if (!out || !q || !key_cache || !value_cache || !block_tables || !context_lens)
+        return fail(PA_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned16(key_cache) || !aligned16(value_cache) || !aligned16(q) || !aligned16(out))
+        return fail(PA_ERR_INVALID_ARG, "caches, q and out must be 16-byte aligned");
+    if (MB == 0 && max_ctx > 0) return fail(PA_ERR_INVALID_ARG, "MB == 0 with max_ctx > 0");
+
+    const int64_t max_parts = parts_for(max_ctx, partition);
+    if (max_parts > 65535) return fail(PA_ERR_UNSUPPORTED, "too many partitions");
+    size_t need = 0;
+    pa_decode_workspace_size(S, Hq, D, max_ctx, partition, &need);
+    if (need && (!workspace || workspace_bytes < need || !aligned16(workspace)))
+        return fail(PA_ERR_INVALID_ARG, "workspace needs %zu bytes, 16-byte aligned (got %zu)",
+                    need, workspace_bytes);
+
+    dec::Launch L{};
+    pa_status st = make_map(&L.tmk, key_cache, cache_dt, NB, bs, Hkv, D);
+    if (st) return st;
+    st = make_map(&L.tmv, value_cache, cache_dt, NB, bs, Hkv, D);
+    if (st) return st;
+    unsigned int* err = device_error_word();
+    if (!err) return PA_ERR_CUDA;
+
+    dec::Params& p = L.p;
+    p.out = out;
+    p.q = q;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.err = err;
+    p.S = S;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.MB = MB;
+    p.max_parts = (int)max_parts;
+    p.part_blocks = max_parts > 1 ? partition / bs : 0;
+    p.part_tokens = max_parts > 1 ? partition : 0;
+    p.max_ctx = max_ctx;
+    p.evict_first = 0;
+    p.NB = NB;
+    p.qk_scale = (float)((double)scale * (double)k_scale * 1.4426950408889634);
+    p.v_scale = v_scale;
+    if (max_parts > 1) {
+        p.ws_ml = static_cast<float2*>(workspace);
+        p.ws_o = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                          sizeof(float2) * (size_t)S * Hq * max_parts);
+    }
+
+    L.bs = bs;
+    L.D = D;
+    L.mma = g_select.load() == 0 && G >= 2 && (cache_dt == PA_F16 || cache_dt == PA_BF16) &&
+            D <= 128;
+    L.mrows = G <= 8 ? 8 : 16;
+    L.gc = G < (D == 256 ? 2 : 4) ? G : (D == 256 ? 2 : 4);
+    const int chunks = L.mma ? 1 : G / L.gc;
+    L.grid = dim3((unsigned)max_parts, (unsigned)(Hkv * chunks), (unsigned)S);
+    L.stream = reinterpret_cast<cudaStream_t>(stream);
+
+    cudaError_t e;
+    switch (cache_dt) {
+    case PA_F32: e = dec::launch_f32(L); break;
+    case PA_F16: e = dec::launch_f16(L); break;
+    case PA_BF16: e = dec::launch_bf16(L); break;
+    default: e = q_dt == PA_F16 ? dec::launch_fp8_q_f16(L) : dec::launch_fp8_q_bf16(L); break;
+    }
+    if (e == cudaErrorNotSupported) return fail(PA_ERR_UNSUPPORTED, "no kernel for this shape");
+    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    if (max_parts > 1) {
+        e = launch_merge(p, q_dt, D, dim3((unsigned)Hq, (unsigned)S), L.stream);
+        if (e != cudaSuccess) return cuda_fail(e, "split-K merge launch");
+    }
+    return PA_OK;
+}

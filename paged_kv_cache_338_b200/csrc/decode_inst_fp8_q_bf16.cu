@@ -1,0 +1,9 @@
+// Decode kernel instantiations: cache PA_FP8_E4M3, q/out PA_BF16 (one unit per dtype pair
+// so the build compiles them in parallel).
+#include "decode_launch.h"
+
+namespace pa {
+namespace dec {
+cudaError_t launch_fp8_q_bf16(const Launch& L) { return launch_dtype<PA_FP8_E4M3, PA_BF16>(L); }
+}  // namespace dec
+}  // namespace pa

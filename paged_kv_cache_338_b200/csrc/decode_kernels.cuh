@@ -1,0 +1,713 @@
+// Paged decode attention kernels for sm_100a.
+//
+// What is computed ("PagedAttention 机制" §5.3.4; intelliparadigm PagedAttention
+// article §2.3; "01. PagedAttention 详解" §4): for sequence s, query head h and
+// kv head g = h / G, over the n_s tokens whose keys sit at
+// key_cache[block_tables[s][i / bs], i % bs, g, :],
+//     out = softmax(scale * K q) V.
+//
+// How (B200 design, not the pages' sketch):
+//  * One CTA per (split-K partition, kv head [, head chunk], sequence).  It
+//    streams the partition's physical blocks of ONE kv head through a ring of
+//    STAGES shared-memory stages.  A stage holds the K tile and the V tile of
+//    one block: bs rows of D elements each (bs * D * elt bytes, rows strided by
+//    Hkv * D * elt in HBM).  Each tile arrives by one 5-D tensor-map (TMA)
+//    load whose coordinates come from the block table, so the gather needs no
+//    address arithmetic in the consumers; out-of-range ids read zeros.
+//  * A producer warp (one elected lane) issues the loads; per-stage "full"
+//    mbarriers carry the byte count, per-stage "empty" mbarriers return the
+//    stage.  Every wait is bounded in time; on timeout the CTA records
+//    PA_DEV_WAIT_TIMEOUT, drains its in-flight copies (again bounded) and
+//    returns without writing.
+//  * Consumer warp w takes blocks w, w + NW, ... and keeps its own online
+//    softmax state (running max m, sum l, accumulator o) in the base-2
+//    domain (scores pre-multiplied by log2(e)); the warps are merged once at
+//    the end through shared memory.  All G query heads of the kv head share
+//    each K/V tile, so K/V is read from HBM once per kv head.
+//  * Two consumers:
+//      - SIMT: 8 lanes per token row, each lane holding D/8 dims; dot
+//        products on FP32 FMA units with a 3-step butterfly; any dtype.
+//      - MMA (GQA, 16-bit K/V): the G query rows padded to 8 (or 16) form the
+//        A operand of mma.sync m16n8k16 (bf16/f16 in, fp32 accumulate):
+//        S = Q K^T with K^T fed by ldmatrix from the swizzled tile, then
+//        O += P V with V fed by ldmatrix.trans; P stays in registers (its
+//        accumulator layout is the A-operand layout of the second product).
+//  * With more than one partition, (m, l, o) go to the fp32 workspace and
+//    decode_merge combines them; otherwise the CTA writes out directly.
+#pragma once
+
+#include <type_traits>
+
+#include "pa_device.cuh"
+
+namespace pa {
+namespace dec {
+
+struct Params {
+    void* out;                   // [S, Hq, D] q dtype
+    const void* q;               // [S, Hq, D]
+    const int32_t* block_tables; // [S, MB]
+    const int32_t* context_lens; // [S]
+    float2* ws_ml;               // [S, Hq, max_parts] (m, l)   (split-K only)
+    float* ws_o;                 // [S, Hq, max_parts, D]       (split-K only)
+    unsigned int* err;           // sticky device error word
+    int S, Hq, Hkv, MB;
+    int max_parts;               // partitions per sequence in the grid
+    int part_blocks;             // blocks per partition (0: the whole sequence)
+    int part_tokens;             // part_blocks * bs
+    int max_ctx;                 // upper bound the grid / workspace were sized for
+    int evict_first;             // 1: stream K/V with an L2 evict-first hint
+    int64_t NB;
+    float qk_scale;              // scale * k_scale * log2(e)
+    float v_scale;
+};
+
+// Context length of sequence s, clamped to what the grid, the workspace and
+// the table row can hold; anything out of range is reported, never followed.
+__device__ __forceinline__ int checked_len(const Params& p, int s, int bs) {
+    int n = p.context_lens[s];
+    const int lim = min(p.max_ctx, p.MB * bs);
+    if (n < 0 || n > lim) {
+        dev::raise_error(p.err, PA_DEV_BAD_CONTEXT);
+        n = n < 0 ? 0 : lim;
+    }
+    return n;
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int DT_, int QT_, int BS_, int D_, int GC_, bool MMA_, int MROWS_ = 8>
+struct Cfg {
+    static constexpr int DT = DT_, QT = QT_, BS = BS_, D = D_, GC = GC_, MROWS = MROWS_;
+    static constexpr bool MMA = MMA_;
+    static constexpr int E = dev::Storage<DT>::bytes;
+    static constexpr int R = D * E;          // bytes of one token row of one kv head
+    static constexpr int CH = R / 128;       // 128-byte segments per row
+    static constexpr int EPS = 128 / E;      // elements per segment
+    static constexpr int EPC = 16 / E;       // elements per 16-byte chunk
+    static constexpr int DPL = D / 8;        // dims per lane (SIMT consumer)
+    static constexpr int TILE = BS * R;      // bytes of a K (or V) tile
+    static constexpr int STAGE = 2 * TILE;
+    static constexpr int NW = 4;             // consumer warps
+    static constexpr int THREADS = (NW + 1) * 32;
+    static constexpr int STAGES_RAW = (64 * 1024) / STAGE;   // 3 CTAs per SM fit
+    static constexpr int STAGES = STAGES_RAW < NW ? NW : (STAGES_RAW > 16 ? 16 : STAGES_RAW);
+    static constexpr int COMBINE_FLOATS = NW * GC * (D + 2);
+    static constexpr size_t SMEM = 1024 /*align slack*/ + size_t(STAGES) * STAGE + 2 * 8 * STAGES;
+    static_assert(R == 128 || R == 256 || R == 512, "row bytes must be 128, 256 or 512");
+    static_assert(BS == 8 || BS == 16 || BS == 32, "block size");
+    static_assert(COMBINE_FLOATS * 4 <= STAGES * STAGE, "combine area must fit in the stages");
+    static_assert(SMEM <= 227 * 1024, "shared memory");
+};
+
+// ------------------------------------------------------------------ producer
+// One warp; lane 0 issues.  Block ids are fetched 32 at a time (one per lane)
+// and handed to lane 0 with a shuffle, so the issue loop never waits on a
+// dependent global load.
+template <class C>
+__device__ __forceinline__ void produce(const CUtensorMap* tmk, const CUtensorMap* tmv,
+                                        const Params& p, const int32_t* bt_row, int blk0, int nblk,
+                                        int kvh, uint8_t* stages, uint32_t full0, uint32_t empty0,
+                                        volatile int* s_abort, int* issued_out) {
+    const int lane = threadIdx.x & 31;
+    const uint64_t pol = p.evict_first ? dev::policy_evict_first() : dev::policy_evict_normal();
+    int issued = 0;
+    for (int jb = 0; jb < nblk; jb += 32) {
+        const int mine = (jb + lane < nblk) ? __ldg(bt_row + blk0 + jb + lane) : 0;
+        const int cnt = min(32, nblk - jb);
+        for (int jj = 0; jj < cnt; ++jj) {
+            const int id = __shfl_sync(0xffffffffu, mine, jj);
+            int stop = 0;
+            if (lane == 0) {
+                const int j = jb + jj;
+                const int st = j % C::STAGES;
+                if (j >= C::STAGES) {
+                    const uint32_t par = ((j / C::STAGES) & 1) ^ 1;
+                    if (!dev::mbar_wait_bounded(empty0 + 8 * st, par)) {
+                        dev::raise_error(p.err, PA_DEV_WAIT_TIMEOUT);
+                        *s_abort = 1;
+                        stop = 1;
+                    }
+                }
+                if (!stop) {
+                    if (id < 0 || (int64_t)id >= p.NB) dev::raise_error(p.err, PA_DEV_BAD_BLOCK);
+                    const uint32_t bar = full0 + 8 * st;
+                    const uint32_t dk = dev::smem_addr(stages + (size_t)st * C::STAGE);
+                    dev::mbar_arrive_expect_tx(bar, C::STAGE);
+                    dev::tma_load_5d(dk, tmk, bar, 0, 0, kvh, 0, id, pol);
+                    dev::tma_load_5d(dk + C::TILE, tmv, bar, 0, 0, kvh, 0, id, pol);
+                    ++issued;
+                }
+            }
+            stop = __shfl_sync(0xffffffffu, stop, 0);
+            if (stop) {
+                if (lane == 0) *issued_out = issued;
+                return;
+            }
+        }
+    }
+    if (lane == 0) *issued_out = issued;
+}
+
+// --------------------------------------------------------- SIMT consumer
+template <class C>
+struct SimtState {
+    float q[C::GC][C::DPL];
+    float acc[C::GC][C::DPL];
+    float m[C::GC];
+    float l[C::GC];
+};
+
+template <class C>
+__device__ __forceinline__ void simt_load_q(SimtState<C>& st, const Params& p, int s, int h0) {
+    const int lane = threadIdx.x & 31;
+    const int l8 = lane & 7;
+    #pragma unroll
+    for (int g = 0; g < C::GC; ++g) {
+        const size_t base = ((size_t)s * p.Hq + h0 + g) * C::D;
+        #pragma unroll
+        for (int k = 0; k < C::CH; ++k)
+            #pragma unroll
+            for (int e = 0; e < C::EPC; ++e)
+                st.q[g][k * C::EPC + e] =
+                    dev::load_q<C::QT>(p.q, base + k * C::EPS + l8 * C::EPC + e) * p.qk_scale;
+        #pragma unroll
+        for (int j = 0; j < C::DPL; ++j) st.acc[g][j] = 0.f;
+        st.m[g] = -INFINITY;
+        st.l[g] = 0.f;
+    }
+}
+
+// Dims of token row t of a tile held by this lane, as floats.
+template <class C>
+__device__ __forceinline__ void simt_row(const uint8_t* tile, int t, int l8, float* f) {
+    #pragma unroll
+    for (int k = 0; k < C::CH; ++k) {
+        const uint4 r = *reinterpret_cast<const uint4*>(tile + dev::swz128(t * C::CH + k, l8));
+        dev::Chunk<C::DT>::to_float(r, f + k * C::EPC);
+    }
+}
+
+template <class C>
+__device__ __forceinline__ void simt_block(SimtState<C>& st, const uint8_t* ktile,
+                                           const uint8_t* vtile, int nvalid) {
+    const int lane = threadIdx.x & 31;
+    const int l8 = lane & 7, grp = lane >> 3;
+    constexpr int SUB = C::BS < 16 ? C::BS : 16;   // tokens per online-softmax update
+    constexpr int IT = SUB / 4;                     // 4 tokens per warp pass
+    float f[C::DPL];
+    #pragma unroll
+    for (int sb = 0; sb < C::BS / SUB; ++sb) {
+        float sc[IT][C::GC];
+        #pragma unroll
+        for (int it = 0; it < IT; ++it) {
+            const int t = sb * SUB + it * 4 + grp;
+            simt_row<C>(ktile, t, l8, f);
+            #pragma unroll
+            for (int g = 0; g < C::GC; ++g) {
+                float a = 0.f;
+                #pragma unroll
+                for (int j = 0; j < C::DPL; ++j) a = fmaf(st.q[g][j], f[j], a);
+                a += __shfl_xor_sync(0xffffffffu, a, 1);
+                a += __shfl_xor_sync(0xffffffffu, a, 2);
+                a += __shfl_xor_sync(0xffffffffu, a, 4);
+                sc[it][g] = (t < nvalid) ? a : -INFINITY;
+            }
+        }
+        #pragma unroll
+        for (int g = 0; g < C::GC; ++g) {
+            float bm = sc[0][g];
+            #pragma unroll
+            for (int it = 1; it < IT; ++it) bm = fmaxf(bm, sc[it][g]);
+            bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
+            bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16));
+            if (bm > st.m[g]) {                       // warp-uniform
+                const float alpha = exp2f(st.m[g] - bm);
+                st.l[g] *= alpha;
+                #pragma unroll
+                for (int j = 0; j < C::DPL; ++j) st.acc[g][j] *= alpha;
+                st.m[g] = bm;
+            }
+        }
+        #pragma unroll
+        for (int it = 0; it < IT; ++it) {
+            const int t = sb * SUB + it * 4 + grp;
+            if (t < nvalid) {
+                simt_row<C>(vtile, t, l8, f);
+                #pragma unroll
+                for (int g = 0; g < C::GC; ++g) {
+                    const float pr = exp2f(sc[it][g] - st.m[g]);
+                    st.l[g] += pr;
+                    #pragma unroll
+                    for (int j = 0; j < C::DPL; ++j) st.acc[g][j] = fmaf(pr, f[j], st.acc[g][j]);
+                }
+            }
+        }
+    }
+}
+
+// Reduce the four token groups of the warp and publish (m, l, acc) to smem.
+template <class C>
+__device__ __forceinline__ void simt_publish(SimtState<C>& st, float* cm, float* cl, float* co,
+                                             int w) {
+    const int lane = threadIdx.x & 31;
+    const int l8 = lane & 7, grp = lane >> 3;
+    #pragma unroll
+    for (int g = 0; g < C::GC; ++g) {
+        float l = st.l[g];
+        l += __shfl_xor_sync(0xffffffffu, l, 8);
+        l += __shfl_xor_sync(0xffffffffu, l, 16);
+        #pragma unroll
+        for (int j = 0; j < C::DPL; ++j) {
+            float a = st.acc[g][j];
+            a += __shfl_xor_sync(0xffffffffu, a, 8);
+            a += __shfl_xor_sync(0xffffffffu, a, 16);
+            st.acc[g][j] = a;
+        }
+        if (lane == 0) {
+            cm[w * C::GC + g] = st.m[g];
+            cl[w * C::GC + g] = l;
+        }
+        if (grp == 0) {
+            #pragma unroll
+            for (int k = 0; k < C::CH; ++k)
+                #pragma unroll
+                for (int e = 0; e < C::EPC; ++e)
+                    co[(w * C::GC + g) * C::D + k * C::EPS + l8 * C::EPC + e] =
+                        st.acc[g][k * C::EPC + e];
+        }
+    }
+}
+
+// ---------------------------------------------------------- MMA consumer
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+
+template <int DT>
+__device__ __forceinline__ void mma16816(float* c, uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+    if constexpr (DT == PA_BF16) {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+            "{%8,%9}, {%0,%1,%2,%3};"
+            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    } else {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+            "{%8,%9}, {%0,%1,%2,%3};"
+            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    }
+}
+
+template <int DT>
+__device__ __forceinline__ void mma1688(float* c, uint32_t a0, uint32_t a1, uint32_t b0) {
+    if constexpr (DT == PA_BF16) {
+        asm volatile(
+            "mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, "
+            "{%0,%1,%2,%3};"
+            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+            : "r"(a0), "r"(a1), "r"(b0));
+    } else {
+        asm volatile(
+            "mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, "
+            "{%0,%1,%2,%3};"
+            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+            : "r"(a0), "r"(a1), "r"(b0));
+    }
+}
+
+// Round two floats into a packed 16-bit pair (lower index in the low half),
+// and return the rounded values.
+template <int DT>
+__device__ __forceinline__ uint32_t pack2(float x, float y, float& rx, float& ry) {
+    if constexpr (DT == PA_BF16) {
+        __nv_bfloat162 v = __floats2bfloat162_rn(x, y);
+        float2 r = __bfloat1622float2(v);
+        rx = r.x; ry = r.y;
+        return *reinterpret_cast<uint32_t*>(&v);
+    } else {
+        __half2 v = __floats2half2_rn(x, y);
+        float2 r = __half22float2(v);
+        rx = r.x; ry = r.y;
+        return *reinterpret_cast<uint32_t*>(&v);
+    }
+}
+
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
+// Tensor-core consumer.  Per KV block of bs tokens and the query heads of one
+// kv head (NH tiles of 8 heads):
+//   S^T [tokens x heads] = K [tokens x D] . Q^T [D x heads]    (m16n8k16, tokens on M)
+//   P^T = 2^(S^T - m), rounded to 16 bits; movmatrix turns its accumulator
+//         fragments into the B fragments of the second product
+//   O^T [D x heads]     += V^T [D x tokens] . P^T [tokens x heads]
+// A thread owns heads 2*tig, 2*tig+1 of each head tile for softmax state.
+template <class C>
+struct MmaState {
+    static constexpr int NH = C::MROWS / 8;  // head tiles of 8
+    static constexpr int KS = C::D / 16;     // k-steps over D
+    static constexpr int MD = C::D / 16;     // m-tiles of O^T
+    uint32_t qb[NH][KS][2];                  // B fragments of Q^T
+    float o[NH][MD][4];                      // O^T accumulators
+    float m[NH][2], l[NH][2];                // heads 2*tig, 2*tig+1 of each tile
+};
+
+template <class C>
+__device__ __forceinline__ void mma_load_q(MmaState<C>& st, const Params& p, int s, int h0,
+                                           int G) {
+    using S = MmaState<C>;
+    const int lane = threadIdx.x & 31;
+    const int gid = lane >> 2, tig = lane & 3;
+    const uint32_t* q32 = static_cast<const uint32_t*>(p.q);
+    #pragma unroll
+    for (int nh = 0; nh < S::NH; ++nh) {
+        const int head = nh * 8 + gid;
+        const size_t base = (((size_t)s * p.Hq + h0 + head) * C::D) / 2;
+        #pragma unroll
+        for (int ks = 0; ks < S::KS; ++ks) {
+            // b0: dims ks*16 + 2tig, +1;  b1: dims ks*16 + 8 + 2tig, +1
+            st.qb[nh][ks][0] = head < G ? __ldg(q32 + base + ks * 8 + tig) : 0u;
+            st.qb[nh][ks][1] = head < G ? __ldg(q32 + base + ks * 8 + 4 + tig) : 0u;
+        }
+        #pragma unroll
+        for (int md = 0; md < S::MD; ++md)
+            #pragma unroll
+            for (int i = 0; i < 4; ++i) st.o[nh][md][i] = 0.f;
+        st.m[nh][0] = st.m[nh][1] = -INFINITY;
+        st.l[nh][0] = st.l[nh][1] = 0.f;
+    }
+}
+
+// smem address of 16-byte chunk c (over the whole row) of token row t
+template <class C>
+__device__ __forceinline__ uint32_t chunk_addr(uint32_t tile, int t, int c) {
+    return tile + dev::swz128(t * C::CH + (c >> 3), c & 7);
+}
+
+template <class C>
+__device__ __forceinline__ void mma_block(MmaState<C>& st, uint8_t* ktile_p, uint8_t* vtile_p,
+                                          int nvalid, float qk_scale) {
+    using S = MmaState<C>;
+    constexpr int BS = C::BS;
+    constexpr int MT = BS >= 16 ? BS / 16 : 1;   // token m-tiles of S^T
+    const int lane = threadIdx.x & 31;
+    const int gid = lane >> 2, tig = lane & 3;
+    const uint32_t ktile = dev::smem_addr(ktile_p), vtile = dev::smem_addr(vtile_p);
+
+    // ---- S^T = K Q^T --------------------------------------------------------
+    float sc[MT][S::NH][4];
+    #pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+        #pragma unroll
+        for (int nh = 0; nh < S::NH; ++nh)
+            #pragma unroll
+            for (int i = 0; i < 4; ++i) sc[mt][nh][i] = 0.f;
+        if constexpr (BS >= 16) {
+            #pragma unroll
+            for (int ks = 0; ks < S::KS; ++ks) {
+                // matrices: (tok 0-7, chunk 2ks) (tok 8-15, 2ks) (tok 0-7, 2ks+1) (tok 8-15, 2ks+1)
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4(chunk_addr<C>(ktile, mt * 16 + ((lane >> 3) & 1) * 8 + (lane & 7),
+                                      2 * ks + (lane >> 4)),
+                        a0, a1, a2, a3);
+                #pragma unroll
+                for (int nh = 0; nh < S::NH; ++nh)
+                    mma16816<C::DT>(sc[mt][nh], a0, a1, a2, a3, st.qb[nh][ks][0], st.qb[nh][ks][1]);
+            }
+        } else {
+            // 8 tokens: rows 8-15 of the A operand are zero
+            #pragma unroll
+            for (int ks = 0; ks < S::KS; ks += 2) {
+                uint32_t a0, a2, b0, b2;   // chunks 2ks, 2ks+1, 2ks+2, 2ks+3 of tokens 0-7
+                ldsm_x4(chunk_addr<C>(ktile, lane & 7, 2 * ks + (lane >> 3)), a0, a2, b0, b2);
+                #pragma unroll
+                for (int nh = 0; nh < S::NH; ++nh) {
+                    mma16816<C::DT>(sc[mt][nh], a0, 0u, a2, 0u, st.qb[nh][ks][0], st.qb[nh][ks][1]);
+                    mma16816<C::DT>(sc[mt][nh], b0, 0u, b2, 0u, st.qb[nh][ks + 1][0],
+                                    st.qb[nh][ks + 1][1]);
+                }
+            }
+        }
+    }
+    // ---- online softmax over the block's tokens, per head ------------------
+    #pragma unroll
+    for (int nh = 0; nh < S::NH; ++nh) {
+        float bm0 = -INFINITY, bm1 = -INFINITY;
+        #pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            const int t0 = mt * 16 + gid, t1 = t0 + 8;
+            const bool v0 = t0 < nvalid, v1 = (BS >= 16) && t1 < nvalid;
+            sc[mt][nh][0] = v0 ? sc[mt][nh][0] * qk_scale : -INFINITY;
+            sc[mt][nh][1] = v0 ? sc[mt][nh][1] * qk_scale : -INFINITY;
+            sc[mt][nh][2] = v1 ? sc[mt][nh][2] * qk_scale : -INFINITY;
+            sc[mt][nh][3] = v1 ? sc[mt][nh][3] * qk_scale : -INFINITY;
+            bm0 = fmaxf(bm0, fmaxf(sc[mt][nh][0], sc[mt][nh][2]));
+            bm1 = fmaxf(bm1, fmaxf(sc[mt][nh][1], sc[mt][nh][3]));
+        }
+        #pragma unroll
+        for (int x = 4; x <= 16; x <<= 1) {
+            bm0 = fmaxf(bm0, __shfl_xor_sync(0xffffffffu, bm0, x));
+            bm1 = fmaxf(bm1, __shfl_xor_sync(0xffffffffu, bm1, x));
+        }
+        const bool grow = bm0 > st.m[nh][0] || bm1 > st.m[nh][1];
+        if (__any_sync(0xffffffffu, grow)) {
+            const float m0 = fmaxf(st.m[nh][0], bm0), m1 = fmaxf(st.m[nh][1], bm1);
+            const float al0 = exp2f(st.m[nh][0] - m0), al1 = exp2f(st.m[nh][1] - m1);  // 0 from -inf
+            st.m[nh][0] = m0;
+            st.m[nh][1] = m1;
+            st.l[nh][0] *= al0;
+            st.l[nh][1] *= al1;
+            #pragma unroll
+            for (int md = 0; md < S::MD; ++md) {
+                st.o[nh][md][0] *= al0; st.o[nh][md][2] *= al0;
+                st.o[nh][md][1] *= al1; st.o[nh][md][3] *= al1;
+            }
+        }
+    }
+    // P^T fragments -> B fragments of O^T += V^T P^T (via an in-register transpose)
+    uint32_t pb[MT][S::NH][2];
+    #pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+        #pragma unroll
+        for (int nh = 0; nh < S::NH; ++nh) {
+            float r0, r1, r2, r3;
+            const uint32_t x = pack2<C::DT>(exp2f(sc[mt][nh][0] - st.m[nh][0]),
+                                            exp2f(sc[mt][nh][1] - st.m[nh][1]), r0, r1);
+            st.l[nh][0] += r0;
+            st.l[nh][1] += r1;
+            pb[mt][nh][0] = movmatrix_t(x);                 // tokens mt*16 + 0..7
+            if constexpr (BS >= 16) {
+                const uint32_t y = pack2<C::DT>(exp2f(sc[mt][nh][2] - st.m[nh][0]),
+                                                exp2f(sc[mt][nh][3] - st.m[nh][1]), r2, r3);
+                st.l[nh][0] += r2;
+                st.l[nh][1] += r3;
+                pb[mt][nh][1] = movmatrix_t(y);             // tokens mt*16 + 8..15
+            }
+        }
+    }
+    // ---- the tail rows of V past nvalid may hold anything: zero them -------
+    if (nvalid < BS) {
+        uint4* v4 = reinterpret_cast<uint4*>(vtile_p + (size_t)nvalid * C::R);
+        const int n16 = (BS - nvalid) * C::R / 16;
+        for (int i = lane; i < n16; i += 32) v4[i] = make_uint4(0, 0, 0, 0);
+        __syncwarp();
+    }
+    // ---- O^T += V^T P^T -------------------------------------------------------
+    if constexpr (BS >= 16) {
+        #pragma unroll
+        for (int kt = 0; kt < MT; ++kt) {
+            #pragma unroll
+            for (int md = 0; md < S::MD; ++md) {
+                // matrices: (tok 0-7, chunk 2md) (tok 0-7, 2md+1) (tok 8-15, 2md) (tok 8-15, 2md+1)
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4_t(chunk_addr<C>(vtile, kt * 16 + (lane >> 4) * 8 + (lane & 7),
+                                        2 * md + ((lane >> 3) & 1)),
+                          a0, a1, a2, a3);
+                #pragma unroll
+                for (int nh = 0; nh < S::NH; ++nh)
+                    mma16816<C::DT>(st.o[nh][md], a0, a1, a2, a3, pb[kt][nh][0], pb[kt][nh][1]);
+            }
+        }
+    } else {
+        #pragma unroll
+        for (int md = 0; md < S::MD; md += 2) {
+            // matrices: tokens 0-7 of chunks 2md, 2md+1, 2md+2, 2md+3
+            uint32_t a0, a1, b0, b1;
+            ldsm_x4_t(chunk_addr<C>(vtile, lane & 7, 2 * md + (lane >> 3)), a0, a1, b0, b1);
+            #pragma unroll
+            for (int nh = 0; nh < S::NH; ++nh) {
+                mma1688<C::DT>(st.o[nh][md], a0, a1, pb[0][nh][0]);
+                mma1688<C::DT>(st.o[nh][md + 1], b0, b1, pb[0][nh][0]);
+            }
+        }
+    }
+    if (nvalid < BS) dev::fence_proxy_async_smem();   // generic writes before the next TMA fill
+}
+
+template <class C>
+__device__ __forceinline__ void mma_publish(MmaState<C>& st, float* cm, float* cl, float* co,
+                                            int w, int G) {
+    using S = MmaState<C>;
+    const int lane = threadIdx.x & 31;
+    const int gid = lane >> 2, tig = lane & 3;
+    #pragma unroll
+    for (int nh = 0; nh < S::NH; ++nh) {
+        #pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            float l = st.l[nh][j];
+            l += __shfl_xor_sync(0xffffffffu, l, 4);
+            l += __shfl_xor_sync(0xffffffffu, l, 8);
+            l += __shfl_xor_sync(0xffffffffu, l, 16);
+            const int head = nh * 8 + 2 * tig + j;
+            if (head < G) {
+                if (gid == 0) {
+                    cm[w * C::GC + head] = st.m[nh][j];
+                    cl[w * C::GC + head] = l;
+                }
+                #pragma unroll
+                for (int md = 0; md < S::MD; ++md) {
+                    co[(w * C::GC + head) * C::D + md * 16 + gid] = st.o[nh][md][j];
+                    co[(w * C::GC + head) * C::D + md * 16 + gid + 8] = st.o[nh][md][2 + j];
+                }
+            }
+        }
+    }
+}
+
+// ----------------------------------------------------------------- kernel
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, C::MMA ? 3 : 2)
+decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                 const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ int s_abort;
+    __shared__ int s_issued;
+    uint8_t* stages = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t full0 = dev::smem_addr(stages + (size_t)C::STAGES * C::STAGE);
+    const uint32_t empty0 = full0 + 8 * C::STAGES;
+
+    const int G = p.Hq / p.Hkv;
+    const int gc = C::MMA ? G : C::GC;          // query heads this CTA serves
+    const int chunks = G / gc;                  // head chunks per kv head
+    const int part = blockIdx.x;
+    const int kvh = blockIdx.y / chunks;
+    const int h0 = kvh * G + (blockIdx.y % chunks) * gc;
+    const int s = blockIdx.z;
+    const int n = checked_len(p, s, C::BS);
+    const int nblk_all = (n + C::BS - 1) / C::BS;
+    int blk0 = 0, nblk = nblk_all, nparts = 1;
+    if (p.part_blocks > 0) {
+        blk0 = part * p.part_blocks;
+        nblk = min(p.part_blocks, nblk_all - blk0);
+        nparts = max(1, (nblk_all + p.part_blocks - 1) / p.part_blocks);
+    }
+    if (part > 0 && nblk <= 0) return;          // this sequence has fewer partitions
+    nblk = max(nblk, 0);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < C::STAGES; ++i) {
+            dev::mbar_init(full0 + 8 * i, 1);
+            dev::mbar_init(empty0 + 8 * i, 1);
+        }
+        dev::fence_mbar_init();
+        s_abort = 0;
+        s_issued = 0;
+    }
+    if (warp == C::NW && lane == 0) {
+        dev::prefetch_tensormap(&tmk);
+        dev::prefetch_tensormap(&tmv);
+    }
+    __syncthreads();
+
+    float* comb = reinterpret_cast<float*>(stages);
+    float* cm = comb;
+    float* cl = cm + C::NW * C::GC;
+    float* co = cl + C::NW * C::GC;
+
+    using State = typename std::conditional<C::MMA, MmaState<C>, SimtState<C>>::type;
+    State st;
+    if (warp == C::NW) {
+        produce<C>(&tmk, &tmv, p, p.block_tables + (size_t)s * p.MB, blk0, nblk, kvh, stages,
+                   full0, empty0, &s_abort, &s_issued);
+    } else {
+        if constexpr (C::MMA) mma_load_q<C>(st, p, s, h0, G);
+        else simt_load_q<C>(st, p, s, h0);
+        for (int j = warp; j < nblk; j += C::NW) {
+            const int stg = j % C::STAGES;
+            if (!dev::mbar_wait_bounded(full0 + 8 * stg, (j / C::STAGES) & 1)) {
+                if (lane == 0) { dev::raise_error(p.err, PA_DEV_WAIT_TIMEOUT); s_abort = 1; }
+                break;
+            }
+            uint8_t* kt = stages + (size_t)stg * C::STAGE;
+            const int nvalid = min(C::BS, n - (blk0 + j) * C::BS);
+            if constexpr (C::MMA) mma_block<C>(st, kt, kt + C::TILE, nvalid, p.qk_scale);
+            else simt_block<C>(st, kt, kt + C::TILE, nvalid);
+            __syncwarp();
+            if (lane == 0) dev::mbar_arrive(empty0 + 8 * stg);
+            if (*(volatile int*)&s_abort) break;
+        }
+    }
+    __syncthreads();                             // every stage consumed (or abort)
+
+    if (s_abort) {
+        // Drain: wait (bounded) until every issued copy has landed, then leave.
+        if (warp == C::NW && lane == 0) {
+            const int issued = s_issued;
+            for (int j = max(0, issued - C::STAGES); j < issued; ++j)
+                dev::mbar_wait_bounded(full0 + 8 * (j % C::STAGES), (j / C::STAGES) & 1);
+        }
+        return;
+    }
+    if (warp < C::NW) {
+        if constexpr (C::MMA) mma_publish<C>(st, cm, cl, co, warp, G);
+        else simt_publish<C>(st, cm, cl, co, warp);
+    }
+    __syncthreads();
+
+    // ---- merge the warps' states and write -----------------------------
+    for (int idx = threadIdx.x; idx < gc * C::D; idx += C::THREADS) {
+        const int g = idx / C::D, d = idx % C::D;
+        float M = -INFINITY;
+        #pragma unroll
+        for (int w = 0; w < C::NW; ++w) M = fmaxf(M, cm[w * C::GC + g]);
+        float L = 0.f, O = 0.f;
+        if (M != -INFINITY) {
+            #pragma unroll
+            for (int w = 0; w < C::NW; ++w) {
+                const float f = exp2f(cm[w * C::GC + g] - M);
+                L = fmaf(f, cl[w * C::GC + g], L);
+                O = fmaf(f, co[(w * C::GC + g) * C::D + d], O);
+            }
+        }
+        const int h = h0 + g;
+        if (nparts == 1) {
+            dev::store_out<C::QT>(p.out, ((size_t)s * p.Hq + h) * C::D + d,
+                                  L > 0.f ? (O / L) * p.v_scale : 0.f);
+        } else {
+            const size_t row = ((size_t)s * p.Hq + h) * p.max_parts + part;
+            p.ws_o[row * C::D + d] = O * p.v_scale;
+            if (d == 0) p.ws_ml[row] = make_float2(M, L);
+        }
+    }
+}
+
+// Merge split-K partials: out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p.
+template <int QT, int D>
+__global__ void __launch_bounds__(D) decode_merge(const Params p) {
+    const int h = blockIdx.x, s = blockIdx.y, d = threadIdx.x;
+    int n = p.context_lens[s];
+    n = max(0, min(n, min(p.max_ctx, p.MB * (p.part_tokens / p.part_blocks))));
+    const int nparts = min(p.max_parts, (n + p.part_tokens - 1) / p.part_tokens);
+    if (nparts <= 1) return;
+    const size_t row0 = ((size_t)s * p.Hq + h) * p.max_parts;
+    float M = -INFINITY;
+    for (int i = 0; i < nparts; ++i) M = fmaxf(M, p.ws_ml[row0 + i].x);
+    float L = 0.f, O = 0.f;
+    for (int i = 0; i < nparts; ++i) {
+        const float2 ml = p.ws_ml[row0 + i];
+        const float f = exp2f(ml.x - M);
+        L = fmaf(f, ml.y, L);
+        O = fmaf(f, p.ws_o[(row0 + i) * D + d], O);
+    }
+    dev::store_out<QT>(p.out, ((size_t)s * p.Hq + h) * D + d, L > 0.f ? O / L : 0.f);
+}
+
+}  // namespace dec
+}  // namespace pa

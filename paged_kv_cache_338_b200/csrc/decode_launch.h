@@ -1,0 +1,93 @@
+// Launch descriptors shared by the host code of pa_decode and the per-dtype
+// instantiation units of the decode kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "decode_kernels.cuh"
+
+namespace pa {
+namespace dec {
+
+struct Launch {
+    CUtensorMap tmk, tmv;
+    Params p;
+    int bs, D;
+    int gc;        // SIMT: query heads per CTA
+    bool mma;      // tensor-core consumer
+    int mrows;     // MMA: 8 or 16 query rows
+    dim3 grid;
+    cudaStream_t stream;
+};
+
+// cudaErrorNotSupported when no kernel is built for the combination.
+cudaError_t launch_f32(const Launch& L);
+cudaError_t launch_f16(const Launch& L);
+cudaError_t launch_bf16(const Launch& L);
+cudaError_t launch_fp8_q_f16(const Launch& L);
+cudaError_t launch_fp8_q_bf16(const Launch& L);
+
+template <class C>
+cudaError_t launch_one(const Launch& L) {
+    auto kern = decode_partition<C>;
+    // opt in to > 48 KB of dynamic shared memory (idempotent, cheap)
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(C::SMEM));
+    if (e != cudaSuccess) return e;
+    kern<<<L.grid, C::THREADS, C::SMEM, L.stream>>>(L.tmk, L.tmv, L.p);
+    return cudaGetLastError();
+}
+
+template <int DT, int D>
+constexpr bool row_ok() {
+    return D * dev::Storage<DT>::bytes == 128 || D * dev::Storage<DT>::bytes == 256 ||
+           D * dev::Storage<DT>::bytes == 512;
+}
+
+template <int DT, int QT, int BS, int D>
+cudaError_t launch_by_heads(const Launch& L) {
+    if constexpr (!row_ok<DT, D>()) {
+        return cudaErrorNotSupported;
+    } else {
+        if (L.mma) {
+            if constexpr (DT == QT && (DT == PA_F16 || DT == PA_BF16) && D <= 128) {
+                if (L.mrows == 8) return launch_one<Cfg<DT, QT, BS, D, 8, true, 8>>(L);
+                return launch_one<Cfg<DT, QT, BS, D, 16, true, 16>>(L);
+            } else {
+                return cudaErrorNotSupported;
+            }
+        }
+        switch (L.gc) {
+        case 1: return launch_one<Cfg<DT, QT, BS, D, 1, false>>(L);
+        case 2: return launch_one<Cfg<DT, QT, BS, D, 2, false>>(L);
+        case 4:
+            if constexpr (D <= 128) return launch_one<Cfg<DT, QT, BS, D, 4, false>>(L);
+            else return cudaErrorNotSupported;
+        }
+        return cudaErrorNotSupported;
+    }
+}
+
+template <int DT, int QT, int BS>
+cudaError_t launch_by_dim(const Launch& L) {
+    switch (L.D) {
+    case 64: return launch_by_heads<DT, QT, BS, 64>(L);
+    case 128: return launch_by_heads<DT, QT, BS, 128>(L);
+    case 256: return launch_by_heads<DT, QT, BS, 256>(L);
+    }
+    return cudaErrorNotSupported;
+}
+
+template <int DT, int QT>
+cudaError_t launch_dtype(const Launch& L) {
+    switch (L.bs) {
+    case 8: return launch_by_dim<DT, QT, 8>(L);
+    case 16: return launch_by_dim<DT, QT, 16>(L);
+    case 32: return launch_by_dim<DT, QT, 32>(L);
+    }
+    return cudaErrorNotSupported;
+}
+
+}  // namespace dec
+}  // namespace pa

@@ -1,0 +1,242 @@
+// Host-side refcounted physical block pool and per-sequence block tables.
+//
+// "PagedAttention 机制" §5.3.4 (BlockAllocator: free list, reference counts,
+// allocate / free / incr_ref, out-of-memory error when the list is empty);
+// "01. PagedAttention 详解" self-check 3 (the free list is a FIFO queue:
+// allocation takes the head, a block whose count reaches 0 goes to the tail);
+// "PagedAttention 机制" §5.3.2 (a sequence of n tokens holds ceil(n / bs)
+// blocks, mapped logical -> physical by its table); "01. PagedAttention 详解"
+// §6 and summary (sharing by reference counts: common prefixes, beam search,
+// parallel sampling); intelliparadigm PagedAttention article §3.3 (writing
+// into a block with count > 1 first copies it: maybe_copy_block).
+#include <cstdint>
+#include <deque>
+#include <new>
+#include <unordered_map>
+#include <vector>
+
+#include "pa_internal.h"
+
+struct pa_pool {
+    int64_t nb = 0;
+    int bs = 0;
+    std::deque<int32_t> free_q;
+    std::vector<int32_t> ref;
+    struct Seq {
+        std::vector<int32_t> blocks;
+        int64_t n = 0;
+    };
+    std::unordered_map<int64_t, Seq> seqs;
+    int64_t next_seq = 0;
+    int64_t cow = 0;
+
+    bool in_range(int64_t b) const { return b >= 0 && b < nb; }
+    Seq* find(int64_t s) {
+        auto it = seqs.find(s);
+        return it == seqs.end() ? nullptr : &it->second;
+    }
+    const Seq* find(int64_t s) const {
+        auto it = seqs.find(s);
+        return it == seqs.end() ? nullptr : &it->second;
+    }
+    int32_t take() {             // caller checked that the queue is not empty
+        const int32_t b = free_q.front();
+        free_q.pop_front();
+        ref[b] = 1;
+        return b;
+    }
+    void drop(int32_t b) {       // caller checked ref[b] > 0
+        if (--ref[b] == 0) free_q.push_back(b);
+    }
+};
+
+using pa::fail;
+
+extern "C" pa_status pa_pool_create(int64_t NB, int bs, pa_pool** out) {
+    pa::clear_error();
+    if (!out) return fail(PA_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    if (NB <= 0 || NB > 0x7fffffffLL || bs <= 0)
+        return fail(PA_ERR_INVALID_ARG, "NB must be in [1, 2^31), bs > 0");
+    pa_pool* p = new (std::nothrow) pa_pool();
+    if (!p) return fail(PA_ERR_INVALID_ARG, "out of host memory");
+    p->nb = NB;
+    p->bs = bs;
+    p->ref.assign((size_t)NB, 0);
+    for (int64_t b = 0; b < NB; ++b) p->free_q.push_back((int32_t)b);
+    *out = p;
+    return PA_OK;
+}
+
+extern "C" void pa_pool_destroy(pa_pool* pool) { delete pool; }
+
+extern "C" pa_status pa_pool_alloc(pa_pool* pool, int32_t* block) {
+    pa::clear_error();
+    if (!pool || !block) return fail(PA_ERR_INVALID_ARG, "NULL argument");
+    if (pool->free_q.empty()) return fail(PA_ERR_OUT_OF_BLOCKS, "no free blocks");
+    *block = pool->take();
+    return PA_OK;
+}
+
+extern "C" pa_status pa_pool_free(pa_pool* pool, int32_t block) {
+    pa::clear_error();
+    if (!pool) return fail(PA_ERR_INVALID_ARG, "pool is NULL");
+    if (!pool->in_range(block)) return fail(PA_ERR_BAD_INDEX, "block %d out of range", block);
+    if (pool->ref[block] <= 0) return fail(PA_ERR_REFCOUNT, "block %d is already free", block);
+    pool->drop(block);
+    return PA_OK;
+}
+
+extern "C" pa_status pa_pool_incr_ref(pa_pool* pool, int32_t block) {
+    pa::clear_error();
+    if (!pool) return fail(PA_ERR_INVALID_ARG, "pool is NULL");
+    if (!pool->in_range(block)) return fail(PA_ERR_BAD_INDEX, "block %d out of range", block);
+    if (pool->ref[block] <= 0) return fail(PA_ERR_REFCOUNT, "block %d is free", block);
+    ++pool->ref[block];
+    return PA_OK;
+}
+
+extern "C" int pa_pool_ref(const pa_pool* pool, int32_t block) {
+    if (!pool || !pool->in_range(block)) return -1;
+    return pool->ref[block];
+}
+
+extern "C" pa_status pa_pool_seq_new(pa_pool* pool, int64_t* seq) {
+    pa::clear_error();
+    if (!pool || !seq) return fail(PA_ERR_INVALID_ARG, "NULL argument");
+    const int64_t id = pool->next_seq++;
+    pool->seqs.emplace(id, pa_pool::Seq{});
+    *seq = id;
+    return PA_OK;
+}
+
+extern "C" pa_status pa_pool_seq_fork(pa_pool* pool, int64_t parent, int64_t* child) {
+    pa::clear_error();
+    if (!pool || !child) return fail(PA_ERR_INVALID_ARG, "NULL argument");
+    const pa_pool::Seq* par = pool->find(parent);
+    if (!par) return fail(PA_ERR_BAD_INDEX, "unknown sequence %lld", (long long)parent);
+    for (int32_t b : par->blocks)            // all or nothing
+        if (pool->ref[b] <= 0) return fail(PA_ERR_REFCOUNT, "block %d is free", b);
+    pa_pool::Seq copy = *par;
+    for (int32_t b : copy.blocks) ++pool->ref[b];
+    const int64_t id = pool->next_seq++;
+    pool->seqs.emplace(id, std::move(copy));
+    *child = id;
+    return PA_OK;
+}
+
+extern "C" pa_status pa_pool_seq_share_prefix(pa_pool* pool, int64_t seq, const int32_t* blocks,
+                                              int n, int64_t num_tokens) {
+    pa::clear_error();
+    if (!pool || (n > 0 && !blocks) || n < 0 || num_tokens < 0)
+        return fail(PA_ERR_INVALID_ARG, "bad arguments");
+    pa_pool::Seq* s = pool->find(seq);
+    if (!s) return fail(PA_ERR_BAD_INDEX, "unknown sequence %lld", (long long)seq);
+    if (s->n != 0 || !s->blocks.empty())
+        return fail(PA_ERR_INVALID_ARG, "a prefix can only be shared into an empty sequence");
+    if ((int64_t)n != (num_tokens + pool->bs - 1) / pool->bs)
+        return fail(PA_ERR_INVALID_ARG, "%d blocks cannot hold exactly %lld tokens", n,
+                    (long long)num_tokens);
+    for (int i = 0; i < n; ++i) {
+        if (!pool->in_range(blocks[i])) return fail(PA_ERR_BAD_INDEX, "block %d out of range", blocks[i]);
+        if (pool->ref[blocks[i]] <= 0) return fail(PA_ERR_REFCOUNT, "block %d is free", blocks[i]);
+    }
+    for (int i = 0; i < n; ++i) ++pool->ref[blocks[i]];
+    s->blocks.assign(blocks, blocks + n);
+    s->n = num_tokens;
+    return PA_OK;
+}
+
+extern "C" pa_status pa_pool_seq_append(pa_pool* pool, int64_t seq, int64_t* slot,
+                                        int32_t* cow_src, int32_t* cow_dst) {
+    pa::clear_error();
+    if (!pool || !slot || !cow_src || !cow_dst) return fail(PA_ERR_INVALID_ARG, "NULL argument");
+    pa_pool::Seq* s = pool->find(seq);
+    if (!s) return fail(PA_ERR_BAD_INDEX, "unknown sequence %lld", (long long)seq);
+    int32_t src = -1, dst = -1;
+    const int64_t off = s->n % pool->bs;
+    if (off == 0) {
+        if (pool->free_q.empty()) return fail(PA_ERR_OUT_OF_BLOCKS, "no free blocks");
+        s->blocks.push_back(pool->take());
+    } else {
+        const int32_t last = s->blocks.back();
+        if (pool->ref[last] > 1) {
+            if (pool->free_q.empty()) return fail(PA_ERR_OUT_OF_BLOCKS, "no free blocks");
+            const int32_t fresh = pool->take();
+            --pool->ref[last];               // other holders keep it (count stays >= 1)
+            s->blocks.back() = fresh;
+            src = last;
+            dst = fresh;
+            ++pool->cow;
+        }
+    }
+    *slot = (int64_t)s->blocks.back() * pool->bs + off;
+    *cow_src = src;
+    *cow_dst = dst;
+    ++s->n;
+    return PA_OK;
+}
+
+extern "C" pa_status pa_pool_seq_free(pa_pool* pool, int64_t seq) {
+    pa::clear_error();
+    if (!pool) return fail(PA_ERR_INVALID_ARG, "pool is NULL");
+    auto it = pool->seqs.find(seq);
+    if (it == pool->seqs.end()) return fail(PA_ERR_BAD_INDEX, "unknown sequence %lld", (long long)seq);
+    std::unordered_map<int32_t, int> held;   // all or nothing: check every reference first
+    for (int32_t b : it->second.blocks) ++held[b];
+    for (const auto& kv : held)
+        if (pool->ref[kv.first] < kv.second)
+            return fail(PA_ERR_REFCOUNT, "block %d has fewer references than the sequence holds",
+                        kv.first);
+    for (int32_t b : it->second.blocks) pool->drop(b);
+    pool->seqs.erase(it);
+    return PA_OK;
+}
+
+extern "C" int64_t pa_pool_seq_len(const pa_pool* pool, int64_t seq) {
+    if (!pool) return -1;
+    const pa_pool::Seq* s = pool->find(seq);
+    return s ? s->n : -1;
+}
+
+extern "C" pa_status pa_pool_build_block_tables(const pa_pool* pool, const int64_t* seqs, int S,
+                                                int MB, int32_t* tables_host,
+                                                int32_t* ctx_lens_host) {
+    pa::clear_error();
+    if (!pool || S < 0 || MB < 0 || (S > 0 && (!seqs || !ctx_lens_host || (MB > 0 && !tables_host))))
+        return fail(PA_ERR_INVALID_ARG, "bad arguments");
+    for (int i = 0; i < S; ++i) {
+        const pa_pool::Seq* s = pool->find(seqs[i]);
+        if (!s) return fail(PA_ERR_BAD_INDEX, "unknown sequence %lld", (long long)seqs[i]);
+        if ((int64_t)s->blocks.size() > MB)
+            return fail(PA_ERR_INVALID_ARG, "sequence %lld holds %zu blocks > MB %d",
+                        (long long)seqs[i], s->blocks.size(), MB);
+        if (s->n > 0x7fffffffLL) return fail(PA_ERR_INVALID_ARG, "context length overflows int32");
+    }
+    for (int i = 0; i < S; ++i) {
+        const pa_pool::Seq* s = pool->find(seqs[i]);
+        int32_t* row = tables_host + (size_t)i * MB;
+        const size_t nb = s->blocks.size();
+        for (size_t j = 0; j < nb; ++j) row[j] = s->blocks[j];
+        for (size_t j = nb; j < (size_t)MB; ++j) row[j] = -1;
+        ctx_lens_host[i] = (int32_t)s->n;
+    }
+    return PA_OK;
+}
+
+extern "C" pa_status pa_pool_stats(const pa_pool* pool, pa_pool_stats_t* st) {
+    pa::clear_error();
+    if (!pool || !st) return fail(PA_ERR_INVALID_ARG, "NULL argument");
+    st->num_blocks = pool->nb;
+    st->free_blocks = (int64_t)pool->free_q.size();
+    int64_t used = 0, shared = 0;
+    for (int32_t r : pool->ref) {
+        used += r > 0;
+        shared += r > 1;
+    }
+    st->used_blocks = used;
+    st->shared_blocks = shared;
+    st->cow_copies = pool->cow;
+    st->num_seqs = (int64_t)pool->seqs.size();
+    return PA_OK;
+}

@@ -1,0 +1,205 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+* The shared library loads and exports every function include/pa.h declares.
+* Argument checks reject bad calls before anything reaches a device.
+* The C++ block pool replays the pages' examples and long random call
+  sequences exactly like the oracle's pool model (same slots, copy-on-write
+  pairs, tables, reference counts, free order and errors).
+"""
+import os
+import random
+import re
+
+import pytest
+import torch
+
+import paged_kv_cache_338_b200 as pa
+from oracle.pool_model import PoolError, PoolModel
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "pa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared_functions()
+    assert len(names) >= 20
+    L = pa.lib()
+    missing = [n for n in names if not hasattr(L, n)]
+    assert not missing, missing
+    assert pa.pa_version() == 10000
+
+
+def test_no_symbol_leaks_beyond_the_abi():
+    # the static CUDA runtime stays private to the library
+    out = os.popen(f"nm -D --defined-only {pa.LIB_PATH}").read().split("\n")
+    exported = {l.split()[-1] for l in out if l.strip() and l.split()[1] in "TtWw"}
+    extra = {n for n in exported if not n.startswith("pa_")}
+    assert not {n for n in extra if n.startswith("cuda")}, sorted(extra)[:10]
+
+
+def _bad(fn, *a, status="PA_ERR_INVALID_ARG"):
+    with pytest.raises(pa.PaError) as e:
+        fn(*a)
+    assert e.value.status == status, str(e.value)
+
+
+def test_host_argument_checks():
+    L = pa.lib()
+    nb = torch.zeros(1, dtype=torch.int64)
+    # decode: bad dtype, group not a divisor, block size, partition not a multiple of bs
+    assert L.pa_decode(None, None, 7, None, None, 2, None, 1, None, 1, 8, 2, 128, 16, 10, 16,
+                       1.0, 1.0, 1.0, 0, None, 0, None) == 1
+    assert L.pa_decode(None, None, 2, None, None, 2, None, 1, None, 1, 6, 4, 128, 16, 10, 16,
+                       1.0, 1.0, 1.0, 0, None, 0, None) == 1
+    assert L.pa_decode(None, None, 2, None, None, 2, None, 1, None, 1, 8, 2, 128, 12, 10, 16,
+                       1.0, 1.0, 1.0, 0, None, 0, None) == 2
+    assert L.pa_decode(None, None, 2, None, None, 2, None, 1, None, 1, 8, 2, 128, 16, 10, 16,
+                       1.0, 1.0, 1.0, 24, None, 0, None) == 1
+    # non-fp8 caches take unit scales only; fp8 needs f16/bf16 q
+    assert L.pa_decode(None, None, 2, None, None, 2, None, 1, None, 1, 8, 2, 128, 16, 10, 16,
+                       1.0, 2.0, 1.0, 0, None, 0, None) == 1
+    assert L.pa_decode(None, None, 0, None, None, 3, None, 1, None, 1, 8, 2, 128, 16, 10, 16,
+                       1.0, 1.0, 1.0, 0, None, 0, None) == 2
+    # S == 0 is a no-op even without pointers
+    assert L.pa_decode(None, None, 2, None, None, 2, None, 1, None, 0, 8, 2, 128, 16, 10, 16,
+                       1.0, 1.0, 1.0, 0, None, 0, None) == 0
+    # split-K without enough workspace
+    assert L.pa_decode(16, 16, 2, 16, 16, 2, 16, 8, 16, 1, 8, 2, 128, 16, 10, 1000,
+                       1.0, 1.0, 1.0, 256, None, 0, None) == 1
+    assert "workspace" in pa.pa_last_error()
+    # append: unsupported dtype pair, scales, zero tokens is a no-op
+    assert L.pa_reshape_and_cache(None, None, 2, None, None, 1, None, 4, 8, 128, 16, 10,
+                                  1.0, 1.0, None) == 2
+    assert L.pa_reshape_and_cache(None, None, 2, None, None, 3, None, 4, 8, 128, 16, 10,
+                                  0.0, 1.0, None) == 1
+    assert L.pa_reshape_and_cache(None, None, 2, None, None, 2, None, 0, 8, 128, 16, 10,
+                                  1.0, 1.0, None) == 0
+
+
+def test_copy_blocks_host_rejections():
+    kc = torch.zeros((8, 16, 2, 64), dtype=torch.bfloat16)   # host memory: never launched
+    for bad in ([[1, 2], [3, 2]], [[1, 2], [2, 4]], [[1, 8]], [[-1, 3]]):
+        _bad(pa.pa_copy_blocks, kc, kc, bad)
+    pa.pa_copy_blocks(kc, kc, [])   # no pairs: nothing to do
+
+
+def test_workspace_size_and_suggested_partition():
+    assert pa.pa_decode_workspace_size(4, 32, 128, 100000, 512) == 4 * 32 * 196 * (8 + 4 * 128)
+    assert pa.pa_decode_workspace_size(4, 32, 128, 512, 512) == 0
+    assert pa.pa_decode_workspace_size(4, 32, 128, 100000, 0) == 0
+    p = pa.pa_decode_suggest_partition(8, 16, [100000] * 4)
+    assert p > 0 and p % 16 == 0 and p < 100000
+    assert pa.pa_decode_suggest_partition(32, 16, [64] * 4096) == 0
+
+
+# ------------------------------------------------------------------ pool
+
+def _run_both(model, pool, op, *args):
+    err_m = err_p = None
+    try:
+        rm = getattr(model, op)(*args)
+    except PoolError as e:
+        err_m, rm = e.status, None
+    try:
+        rp = getattr(pool, op)(*args)
+    except pa.PaError as e:
+        err_p, rp = e.status, None
+    assert err_m == err_p, (op, args, err_m, err_p)
+    return rm, rp
+
+
+def test_pool_replays_page_examples(golden):
+    g = golden("shared_blocks_example.json")
+    pool = pa.BlockPool(100, 16)
+    held = [pool.alloc() for _ in range(100)]
+    assert held == list(range(100))
+    for b in (42, 17, 99, 88):
+        pool.free(b)
+    a = pool.seq_new()
+    for _ in range(48):
+        pool.seq_append(a)
+    b = pool.seq_new()
+    pool.seq_share_prefix(b, [42, 17], 32)
+    for _ in range(16):
+        assert pool.seq_append(b)[1:] == (-1, -1)
+    t, lens = pool.build_block_tables([a, b], 3)
+    assert t.tolist() == [g["table_a"], g["table_b"]] and lens.tolist() == [48, 48]
+    for blk, r in g["ref_cnt"].items():
+        assert pool.ref(int(blk)) == r
+    # 100000 tokens -> 6250 int32 entries (25000 bytes)
+    f = golden("table_size_facts.json")
+    big = pa.BlockPool(7000, 16)
+    s = big.seq_new()
+    for _ in range(f["num_tokens"]):
+        big.seq_append(s)
+    t, lens = big.build_block_tables([s], f["entries"])
+    assert t.numel() * 4 == f["table_bytes"] and int(lens[0]) == f["num_tokens"]
+    assert (t >= 0).all()
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_pool_matches_model_on_random_call_sequences(seed):
+    rnd = random.Random(seed)
+    nb, bs = rnd.choice([(12, 4), (40, 8), (64, 16), (7, 32)])
+    model, pool = PoolModel(nb, bs), pa.BlockPool(nb, bs)
+    live = []
+    for step in range(1500):
+        r = rnd.random()
+        if r < 0.08 or not live:
+            m, p = _run_both(model, pool, "seq_new")
+            assert m == p
+            live.append(m)
+        elif r < 0.55:
+            s = rnd.choice(live)
+            m, p = _run_both(model, pool, "seq_append", s)
+            assert m == p
+        elif r < 0.62:
+            m, p = _run_both(model, pool, "seq_fork", rnd.choice(live))
+            assert m == p
+            if m is not None:
+                live.append(m)
+        elif r < 0.70 and len(live) > 1:
+            s = live.pop(rnd.randrange(len(live)))
+            _run_both(model, pool, "seq_free", s)
+        elif r < 0.75:
+            s = rnd.choice(live)
+            if model.seq_len(s) > 0:
+                src = model.seq_blocks(s)
+                n = rnd.randint(1, len(src))
+                t = model.seq_new()
+                assert pool.seq_new() == t
+                live.append(t)
+                ntok = min(model.seq_len(s), n * bs)
+                _run_both(model, pool, "seq_share_prefix", t, src[:n], ntok)
+        elif r < 0.80:
+            _run_both(model, pool, "free", rnd.randrange(-1, nb + 1))
+        elif r < 0.85:
+            _run_both(model, pool, "incr_ref", rnd.randrange(nb))
+        elif r < 0.88:
+            m, p = _run_both(model, pool, "alloc")
+            assert m == p
+        else:
+            _run_both(model, pool, "seq_append", 10_000 + step)     # unknown sequence
+        assert [pool.ref(b) for b in range(nb)] == model.ref
+        st = pool.stats()
+        ms = model.stats()
+        for k in ("free", "used", "shared"):
+            assert st[k if k != "free" else "free_blocks"] == ms[k] if k == "free" else \
+                st[k + "_blocks"] == ms[k]
+        assert st["cow_copies"] == ms["cow_copies"] and st["num_seqs"] == ms["num_seqs"]
+    mb = max([len(model.seq_blocks(s)) for s in live] + [1])
+    tm, lm = model.build_block_tables(live, mb)
+    tp, lp = pool.build_block_tables(live, mb)
+    assert tp.tolist() == tm and lp.tolist() == lm
+    # drain: free order must match (observed through the next allocations)
+    for s in live:
+        _run_both(model, pool, "seq_free", s)
+    while model.free_queue:
+        m, p = _run_both(model, pool, "alloc")
+        assert m == p
+    _run_both(model, pool, "alloc")

@@ -13,7 +13,7 @@
 import numpy as np
 import pytest
 
-from oracle.pool_model import InvalidArg, OutOfBlocks, PoolError, PoolModel
+from oracle.pool_model import BadIndex, InvalidArg, OutOfBlocks, PoolError, PoolModel
 
 
 def _pool_with_queue(nb, bs, order):
@@ -99,7 +99,7 @@ def test_allocator_rules():
         p.free(1)                                 # already free
     with pytest.raises(PoolError):
         p.incr_ref(0)                             # a free block cannot be shared
-    with pytest.raises(InvalidArg):
+    with pytest.raises(BadIndex):
         p.free(3)
 
 
