@@ -177,6 +177,38 @@ pa_status pa_decode(void* out, const void* q, pa_dtype q_dt,
                     void* workspace, size_t workspace_bytes, pa_stream_t stream);
 
 /*
+ * pa_decode without a caller-provided workspace.  (The pages have no
+ * counterpart of this entry point: it exists for callers of this library.)
+ *
+ * For callers that cannot allocate device memory for the split-K partials:
+ * a serving runtime that hands all device memory to its KV cache at start-up
+ * and owns the only allocator, a plugin inside a framework that exposes no
+ * allocation hook, or a step loop that must not call cudaMalloc / cudaFree
+ * (cudaFree waits for the whole device) while it runs.  Same arguments and
+ * result as pa_decode, minus the workspace: the partials live in a fixed
+ * device array of PA_DECODE_NOALLOC_SCRATCH_BYTES inside the library, which
+ * every GPU that loads the library holds until the process exits.  This
+ * function allocates nothing.
+ *
+ * Limits: if pa_decode_workspace_size() for these sizes exceeds the array,
+ * the call fails with PA_ERR_INVALID_ARG before enqueuing anything (choose a
+ * larger partition, or use pa_decode).  All calls share the one array, so
+ * calls whose device work may overlap (different streams or host threads)
+ * race on it: the caller must order them.  Nothing in the array needs to
+ * start at zero; a call reads only partials it wrote itself.
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and caches it; make that
+ * first call before any stream capture.
+ */
+#define PA_DECODE_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20) /* 32 MiB */
+pa_status pa_decode_noalloc(void* out, const void* q, pa_dtype q_dt,
+                            const void* key_cache, const void* value_cache, pa_dtype cache_dt,
+                            const int32_t* block_tables, int MB, const int32_t* context_lens,
+                            int S, int Hq, int Hkv, int D, int bs, int64_t NB, int max_ctx,
+                            float scale, float k_scale, float v_scale, int partition,
+                            pa_stream_t stream);
+
+/*
  * Consumer selection for pa_decode (process-wide; for tests and tuning):
  * 0 = automatic (tensor-core consumer for grouped-query heads with 16-bit
  * caches and D <= 128, CUDA-core consumer otherwise), 1 = CUDA-core consumer

@@ -21,7 +21,7 @@ import torch
 __all__ = [
     "PaError", "lib", "pa_version", "pa_last_error", "pa_device_status",
     "pa_reshape_and_cache", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_size",
-    "pa_decode_suggest_partition", "pa_decode_select", "BlockPool",
+    "pa_decode_suggest_partition", "pa_decode_select", "pa_decode_noalloc", "BlockPool",
     "PA_DEV_BAD_SLOT", "PA_DEV_BAD_BLOCK", "PA_DEV_WAIT_TIMEOUT", "PA_DEV_BAD_CONTEXT",
 ]
 
@@ -75,6 +75,7 @@ def lib() -> ctypes.CDLL:
         "pa_decode_suggest_partition": ([I, I, I, P, ctypes.POINTER(I)], I),
         "pa_decode_select": ([I], I),
         "pa_decode": ([P, P, I, P, P, I, P, I, P, I, I, I, I, I, I64, I, F, F, F, I, P, SZ, P], I),
+        "pa_decode_noalloc": ([P, P, I, P, P, I, P, I, P, I, I, I, I, I, I64, I, F, F, F, I, P], I),
         "pa_pool_create": ([I64, I, ctypes.POINTER(P)], I),
         "pa_pool_destroy": ([P], None),
         "pa_pool_alloc": ([P, ctypes.POINTER(I32)], I),
@@ -209,6 +210,26 @@ def pa_decode(out: torch.Tensor, q: torch.Tensor, key_cache: torch.Tensor,
                            Hkv, D, bs, NB, int(max_ctx), float(scale), float(k_scale),
                            float(v_scale), int(partition), _ptr(workspace), ws_bytes,
                            _stream(stream)))
+
+
+def pa_decode_noalloc(out: torch.Tensor, q: torch.Tensor, key_cache: torch.Tensor,
+                      value_cache: torch.Tensor, block_tables: torch.Tensor,
+                      context_lens: torch.Tensor, max_ctx: int, scale: float,
+                      k_scale: float = 1.0, v_scale: float = 1.0, partition: int = 0,
+                      stream=None) -> None:
+    """pa_decode for callers that cannot allocate device memory: the split-K
+    partials go to the library's built-in scratch array (see include/pa.h for
+    its size and for the rule that calls overlapping on the GPU race on it)."""
+    S, Hq, D = q.shape
+    NB, bs, Hkv, _ = key_cache.shape
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise PaError(1, "block_tables and context_lens must be int32")
+    _check(lib().pa_decode_noalloc(_ptr(out), _ptr(q), _dt(q), _ptr(key_cache),
+                                   _ptr(value_cache), _dt(key_cache), _ptr(block_tables), MB,
+                                   _ptr(context_lens), S, Hq, Hkv, D, bs, NB, int(max_ctx),
+                                   float(scale), float(k_scale), float(v_scale), int(partition),
+                                   _stream(stream)))
 
 
 class BlockPool:
