@@ -74,55 +74,77 @@ def _pci_id(dev: int) -> str | None:
 
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+    """SM clock, power and clock-event reasons sampled DURING a timed region.
+
+    A background thread polls NVML about every millisecond (a decode step is
+    well under a millisecond, so nvidia-smi's 200 ms period would miss most
+    regions); nvidia-smi's own sampling runs beside it and is kept in
+    gpurun_out/ as the raw record.  Nothing is changed on the GPU: read-only
+    queries.
+    """
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, dev: int):
+        import threading
+        self.samples, self.max_mhz, self.reason_bits = [], None, 0
+        self.stop_flag = threading.Event()
+        self.thread = None
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{dev}.csv")
         pid = _pci_id(dev)
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            import pynvml as nv
+            nv.nvmlInit()
+            h = nv.nvmlDeviceGetHandleByPciBusId(pid) if pid else nv.nvmlDeviceGetHandleByIndex(dev)
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            self.nv, self.h = nv, h
+
+            def poll():
+                while not self.stop_flag.is_set():
+                    try:
+                        self.samples.append(float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)))
+                        self.reason_bits |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))
+                    except Exception:
+                        pass
+                    time.sleep(0.001)
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.thread = None
+        try:
+            path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{dev}.csv")
+            os.makedirs(os.path.dirname(path), exist_ok=True)
             args = ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                    "-lms", "200"]
-            if pid:
-                args += ["-i", pid]
-            self.f = open(self.path, "w")
+                    "-lms", "200"] + (["-i", pid] if pid else [])
+            self.f = open(path, "w")
             self.proc = subprocess.Popen(args, stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
     def stop(self) -> dict:
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        time.sleep(0.25)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.f.close()
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            c = [x.strip() for x in line.split(",")]
-            if len(c) < 9:
-                continue
+        if self.thread is not None:
+            self.stop_flag.set()
+            self.thread.join(timeout=2)
+        if self.proc is not None:
+            self.proc.terminate()
             try:
-                sm.append(float(c[1]))
-                smax = float(c[2])
-            except ValueError:
-                continue
-            for nm, v in zip(names, c[5:9]):
-                if v.lower() == "active":
-                    reasons.add(nm)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        sm.sort()
-        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": smax, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"]}
+        nv = self.nv
+        names = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                 "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                 "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                 "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap,
+                 "hw_power_brake_slowdown": nv.nvmlClocksEventReasonHwPowerBrakeSlowdown}
+        sm = sorted(self.samples)
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(n for n, b in names.items() if self.reason_bits & b),
+                "samples": len(sm), "sm_mhz_min": sm[0], "source": "nvml, 1 ms"}
 
 
 # ------------------------------------------------------------------ oracle arm
@@ -230,7 +252,7 @@ def run_gpu(args, cfg, rank, world, local_rank):
     part = args.partition if args.partition >= 0 else (
         cfg.partition or pa.pa_decode_suggest_partition(cfg.num_kv_heads, cfg.block_size,
                                                         inp.context_lens.cpu()))
-    max_ctx = inp.max_ctx + args.warmup + args.steps + 2     # room for e2e growth
+    max_ctx = inp.max_ctx
     ws_bytes = pa.pa_decode_workspace_size(S, Hq, D, max_ctx, part)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
     out = torch.empty_like(inp.q)
@@ -284,7 +306,7 @@ def run_gpu(args, cfg, rank, world, local_rank):
     value = world * step_bytes / (ms_step * 1e-3) / 1e9
 
     # ---- end to end through the public API with host buffers -------------
-    e2e = run_e2e(args, cfg, pa, dev, part, max_ctx) if not args.no_e2e else None
+    e2e = run_e2e(args, cfg, pa, dev, part) if not args.no_e2e else None
     if dist and e2e is not None:
         t = torch.tensor([e2e["ms"]], dtype=torch.float64, device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
@@ -335,30 +357,41 @@ def run_gpu(args, cfg, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
-def run_e2e(args, cfg, pa, dev, part, max_ctx):
+def run_e2e(args, cfg, pa, dev, part):
     """Host pool + pinned host buffers + H2D / step / D2H every step."""
     g = torch.Generator().manual_seed(args.seed + 77)
     inp = wl.make_decode_inputs(cfg, seed=args.seed + 5, device=dev)
+    max_ctx = inp.max_ctx + args.warmup + args.steps + 2     # sequences grow one token a step
     S, Hq, D = inp.q.shape
     bs = cfg.block_size
     NB = inp.num_blocks + S * (args.warmup + args.steps + 2) // bs + S
     kc = torch.empty((NB,) + tuple(inp.key_cache.shape[1:]), dtype=inp.key_cache.dtype, device=dev)
     vc = torch.empty_like(kc)
-    kc[:inp.num_blocks] = inp.key_cache
-    vc[:inp.num_blocks] = inp.value_cache
-    kc[inp.num_blocks:].zero_()
-    vc[inp.num_blocks:].zero_()
+    for t in (kc, vc):                         # finite random contents (timing only)
+        t.copy_(torch.randn(t.shape, device=dev, dtype=torch.float32).to(t.dtype))
     pool = pa.BlockPool(NB, bs)
     # shuffle the free queue: take every block, give them back in a seeded order
     ids = [pool.alloc() for _ in range(NB)]
     for i in torch.randperm(NB, generator=g).tolist():
         pool.free(ids[i])
     lens = inp.context_lens.cpu().tolist()
-    seqs = []
+    seqs, parents = [], []
+    prefix_blocks = []
+    if cfg.prefix_tokens:                      # one owner writes the shared prefix once
+        owner = pool.seq_new()
+        for _ in range(cfg.prefix_tokens):
+            pool.seq_append(owner)
+        prefix_blocks = pool.build_block_tables([owner], cfg.prefix_tokens // bs)[0][0].tolist()
     for s in range(S):
         sid = pool.seq_new()
-        for _ in range(lens[s] - 1):
+        have = 0
+        if prefix_blocks:
+            pool.seq_share_prefix(sid, prefix_blocks, cfg.prefix_tokens)
+            have = cfg.prefix_tokens
+        for _ in range(lens[s] - 1 - have):
             pool.seq_append(sid)
+        if cfg.cow_last_block:                 # a sampling parent keeps the last block shared
+            parents.append(pool.seq_fork(sid))
         seqs.append(sid)
     MB = (max(lens) + args.warmup + args.steps + 2 + bs - 1) // bs
     pin = dict(pin_memory=True)
@@ -422,8 +455,8 @@ def run_e2e(args, cfg, pa, dev, part, max_ctx):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=3, choices=sorted(wl.CONFIGS))
     ap.add_argument("--partition", type=int, default=-1, help="-1: workload default / heuristic")
@@ -431,6 +464,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--seqs", type=int, default=0,
+                    help="profiling only: a sub-batch of this many sequences of the workload")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")
@@ -438,6 +473,8 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     cfg = wl.CONFIGS[args.config]
+    if args.seqs:
+        cfg = _sample_cfg(cfg, args.seqs)
     if args.impl == "reference":
         run_reference(args, cfg, rank, world)
         return

@@ -61,7 +61,7 @@ pa_status make_map(CUtensorMap* m, const void* base, pa_dtype dt, int64_t NB, in
 
 template <int QT, int D>
 cudaError_t launch_merge_t(const dec::Params& p, dim3 grid, cudaStream_t st) {
-    dec::decode_merge<QT, D><<<grid, D, 0, st>>>(p);
+    dec::decode_merge<QT, D><<<grid, dec::kMergeWarps * 32, 0, st>>>(p);
     return cudaGetLastError();
 }
 

@@ -689,24 +689,65 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
 }
 
 // Merge split-K partials: out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p.
+// One CTA per (query head, sequence); its 8 warps split the partitions and
+// each lane holds D/32 dims, so every partial row is one coalesced load.
+constexpr int kMergeWarps = 8;
+
 template <int QT, int D>
-__global__ void __launch_bounds__(D) decode_merge(const Params p) {
-    const int h = blockIdx.x, s = blockIdx.y, d = threadIdx.x;
+__global__ void __launch_bounds__(kMergeWarps * 32) decode_merge(const Params p) {
+    constexpr int DL = D / 32;                        // dims per lane
+    __shared__ float s_max[kMergeWarps];
+    __shared__ float s_l[kMergeWarps];
+    __shared__ float s_o[kMergeWarps][D];
+    const int h = blockIdx.x, s = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int n = p.context_lens[s];
     n = max(0, min(n, min(p.max_ctx, p.MB * (p.part_tokens / p.part_blocks))));
     const int nparts = min(p.max_parts, (n + p.part_tokens - 1) / p.part_tokens);
     if (nparts <= 1) return;
     const size_t row0 = ((size_t)s * p.Hq + h) * p.max_parts;
-    float M = -INFINITY;
-    for (int i = 0; i < nparts; ++i) M = fmaxf(M, p.ws_ml[row0 + i].x);
-    float L = 0.f, O = 0.f;
-    for (int i = 0; i < nparts; ++i) {
+
+    float mx = -INFINITY;
+    for (int i = threadIdx.x; i < nparts; i += blockDim.x) mx = fmaxf(mx, p.ws_ml[row0 + i].x);
+    #pragma unroll
+    for (int x = 16; x > 0; x >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, x));
+    if (lane == 0) s_max[warp] = mx;
+    __syncthreads();
+    float M = s_max[0];
+    #pragma unroll
+    for (int w = 1; w < kMergeWarps; ++w) M = fmaxf(M, s_max[w]);
+
+    float L = 0.f, o[DL];
+    #pragma unroll
+    for (int k = 0; k < DL; ++k) o[k] = 0.f;
+    #pragma unroll 4
+    for (int i = warp; i < nparts; i += kMergeWarps) {
         const float2 ml = p.ws_ml[row0 + i];
         const float f = exp2f(ml.x - M);
         L = fmaf(f, ml.y, L);
-        O = fmaf(f, p.ws_o[(row0 + i) * D + d], O);
+        const float* src = p.ws_o + (row0 + i) * D + lane * DL;
+        if constexpr (DL == 4) {
+            const float4 v = *reinterpret_cast<const float4*>(src);
+            o[0] = fmaf(f, v.x, o[0]); o[1] = fmaf(f, v.y, o[1]);
+            o[2] = fmaf(f, v.z, o[2]); o[3] = fmaf(f, v.w, o[3]);
+        } else {
+            #pragma unroll
+            for (int k = 0; k < DL; ++k) o[k] = fmaf(f, src[k], o[k]);
+        }
     }
-    dev::store_out<QT>(p.out, ((size_t)s * p.Hq + h) * D + d, L > 0.f ? O / L : 0.f);
+    if (lane == 0) s_l[warp] = L;
+    #pragma unroll
+    for (int k = 0; k < DL; ++k) s_o[warp][lane * DL + k] = o[k];
+    __syncthreads();
+    for (int d = threadIdx.x; d < D; d += blockDim.x) {
+        float Lt = 0.f, Ot = 0.f;
+        #pragma unroll
+        for (int w = 0; w < kMergeWarps; ++w) {
+            Lt += s_l[w];
+            Ot += s_o[w][d];
+        }
+        dev::store_out<QT>(p.out, ((size_t)s * p.Hq + h) * D + d, Lt > 0.f ? Ot / Lt : 0.f);
+    }
 }
 
 }  // namespace dec
