@@ -209,10 +209,15 @@ pa_status pa_decode_noalloc(void* out, const void* q, pa_dtype q_dt,
                             pa_stream_t stream);
 
 /*
- * Consumer selection for pa_decode (process-wide; for tests and tuning):
- * 0 = automatic (tensor-core consumer for grouped-query heads with 16-bit
- * caches and D <= 128, CUDA-core consumer otherwise), 1 = CUDA-core consumer
- * everywhere.  Both compute the same function.
+ * Kernel selection and tuning for pa_decode (process-wide; for tests and
+ * tuning), a bit mask:
+ *   1: CUDA-core consumer everywhere (otherwise grouped-query heads with
+ *      f16 / bf16 / fp8 caches and D <= 128 use the tensor-core consumer);
+ *   2: stream K/V with an L2 evict-first hint;
+ *   4: partition-major grid (the kv heads of one partition are neighbouring
+ *      CTAs, so the interleaved heads of a block are read at about the same
+ *      time); otherwise kv-head-major.
+ * Default 4.  Every setting computes the same function.
  */
 pa_status pa_decode_select(int mode);
 

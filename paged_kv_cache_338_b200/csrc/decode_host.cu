@@ -13,7 +13,10 @@
 namespace pa {
 namespace {
 
-std::atomic<int> g_select{0};   // 0: automatic, 1: CUDA-core consumer only
+// pa_decode_select bits: 1 = CUDA-core consumer only, 2 = L2 evict-first
+// hint on K/V loads, 4 = partition-major grid (kv heads of a partition side
+// by side); the default is 4.
+std::atomic<int> g_select{4};
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -38,48 +41,64 @@ CUtensorMapDataType tma_type(pa_dtype dt) {
     }
 }
 
-// The cache [NB, bs, Hkv, D] as a 5-D tensor {D/seg, seg_count, Hkv, bs, NB}
-// (innermost first) whose box {seg, seg_count, 1, bs, 1} is the K (or V)
-// tile of one block for one kv head, in 128-byte swizzled rows.
+// The cache [NB, bs, Hkv, D] as a 4-D tensor {D, Hkv, bs, NB} (innermost
+// first).  A box {128 bytes of D, 1, bs, 1} is one 128-byte segment of the
+// K (or V) tile of one block for one kv head, swizzled per 128-byte row; a
+// tile takes D * elt / 128 boxes, at x = 0, 128 / elt, ...
 pa_status make_map(CUtensorMap* m, const void* base, pa_dtype dt, int64_t NB, int bs, int Hkv,
                    int D) {
     auto fn = encode_fn();
     if (!fn) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
     const int e = elem_size(dt);
     const cuuint64_t row = (cuuint64_t)D * e;            // bytes of one (token, head) row
-    const cuuint64_t seg = 128 / e;                      // elements per 128-byte segment
-    cuuint64_t dims[5] = {seg, row / 128, (cuuint64_t)Hkv, (cuuint64_t)bs, (cuuint64_t)NB};
-    cuuint64_t strides[4] = {128, row, row * Hkv, row * Hkv * bs};
-    cuuint32_t box[5] = {(cuuint32_t)seg, (cuuint32_t)(row / 128), 1, (cuuint32_t)bs, 1};
-    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-    CUresult r = fn(m, tma_type(dt), 5, const_cast<void*>(base), dims, strides, box, estr,
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)bs, (cuuint64_t)NB};
+    cuuint64_t strides[3] = {row, row * Hkv, row * Hkv * bs};
+    cuuint32_t box[4] = {(cuuint32_t)(128 / e), 1, (cuuint32_t)bs, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, tma_type(dt), 4, const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
     return PA_OK;
 }
 
+// Launched as a programmatic dependent of the partition kernel so its launch
+// overlaps that grid's last wave (it waits for the grid's memory itself).
 template <int QT, int D>
-cudaError_t launch_merge_t(const dec::Params& p, dim3 grid, cudaStream_t st) {
-    dec::decode_merge<QT, D><<<grid, dec::kMergeWarps * 32, 0, st>>>(p);
-    return cudaGetLastError();
+cudaError_t launch_merge_t(const dec::Params& p, int wph, dim3 grid, cudaStream_t st) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(dec::kMergeWarps * 32);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, dec::decode_merge<QT, D>, p, wph);
 }
 
 template <int QT>
-cudaError_t launch_merge_q(const dec::Params& p, int D, dim3 grid, cudaStream_t st) {
+cudaError_t launch_merge_q(const dec::Params& p, int D, int wph, dim3 grid, cudaStream_t st) {
     switch (D) {
-    case 64: return launch_merge_t<QT, 64>(p, grid, st);
-    case 128: return launch_merge_t<QT, 128>(p, grid, st);
-    case 256: return launch_merge_t<QT, 256>(p, grid, st);
+    case 64: return launch_merge_t<QT, 64>(p, wph, grid, st);
+    case 128: return launch_merge_t<QT, 128>(p, wph, grid, st);
+    case 256: return launch_merge_t<QT, 256>(p, wph, grid, st);
     }
     return cudaErrorNotSupported;
 }
 
-cudaError_t launch_merge(const dec::Params& p, pa_dtype qt, int D, dim3 grid, cudaStream_t st) {
+// Warps per head: enough to split a sequence's partitions, at most 8.
+cudaError_t launch_merge(const dec::Params& p, pa_dtype qt, int D, int Hq, int S,
+                         cudaStream_t st) {
+    int wph = 1;
+    while (wph < dec::kMergeWarps && p.max_parts > 8 * wph) wph *= 2;
+    const int hpc = dec::kMergeWarps / wph;
+    const dim3 grid((unsigned)((Hq + hpc - 1) / hpc), (unsigned)S);
     switch (qt) {
-    case PA_F32: return launch_merge_q<PA_F32>(p, D, grid, st);
-    case PA_F16: return launch_merge_q<PA_F16>(p, D, grid, st);
-    case PA_BF16: return launch_merge_q<PA_BF16>(p, D, grid, st);
+    case PA_F32: return launch_merge_q<PA_F32>(p, D, wph, grid, st);
+    case PA_F16: return launch_merge_q<PA_F16>(p, D, wph, grid, st);
+    case PA_BF16: return launch_merge_q<PA_BF16>(p, D, wph, grid, st);
     default: return cudaErrorNotSupported;
     }
 }
@@ -134,7 +153,7 @@ extern "C" pa_status pa_decode_suggest_partition(int S, int Hkv, int bs,
 
 extern "C" pa_status pa_decode_select(int mode) {
     clear_error();
-    if (mode < 0 || mode > 1) return fail(PA_ERR_INVALID_ARG, "mode must be 0 or 1");
+    if (mode < 0 || mode > 7) return fail(PA_ERR_INVALID_ARG, "mode must be in [0, 7]");
     g_select.store(mode);
     return PA_OK;
 }
@@ -176,7 +195,8 @@ extern "C" pa_status pa_decode(void* out, const void* q, pa_dtype q_dt, const vo
     if (MB == 0 && max_ctx > 0) return fail(PA_ERR_INVALID_ARG, "MB == 0 with max_ctx > 0");
 
     const int64_t max_parts = parts_for(max_ctx, partition);
-    if (max_parts > 65535) return fail(PA_ERR_UNSUPPORTED, "too many partitions");
+    if (max_parts > 65535 || (int64_t)Hkv * G > 65535)
+        return fail(PA_ERR_UNSUPPORTED, "too many partitions or heads for the grid");
     size_t need = 0;
     pa_decode_workspace_size(S, Hq, D, max_ctx, partition, &need);
     if (need && (!workspace || workspace_bytes < need || !aligned16(workspace)))
@@ -205,7 +225,9 @@ extern "C" pa_status pa_decode(void* out, const void* q, pa_dtype q_dt, const vo
     p.part_blocks = max_parts > 1 ? partition / bs : 0;
     p.part_tokens = max_parts > 1 ? partition : 0;
     p.max_ctx = max_ctx;
-    p.evict_first = 0;
+    const int sel = g_select.load();
+    p.evict_first = (sel & 2) ? 1 : 0;
+    p.heads_fastest = (sel & 4) ? 1 : 0;
     p.NB = NB;
     p.qk_scale = (float)((double)scale * (double)k_scale * 1.4426950408889634);
     p.v_scale = v_scale;
@@ -217,12 +239,12 @@ extern "C" pa_status pa_decode(void* out, const void* q, pa_dtype q_dt, const vo
 
     L.bs = bs;
     L.D = D;
-    L.mma = g_select.load() == 0 && G >= 2 && (cache_dt == PA_F16 || cache_dt == PA_BF16) &&
-            D <= 128;
+    L.mma = !(sel & 1) && G >= 2 && D <= 128 && cache_dt != PA_F32;
     L.mrows = G <= 8 ? 8 : 16;
     L.gc = G < (D == 256 ? 2 : 4) ? G : (D == 256 ? 2 : 4);
     const int chunks = L.mma ? 1 : G / L.gc;
-    L.grid = dim3((unsigned)max_parts, (unsigned)(Hkv * chunks), (unsigned)S);
+    L.grid = p.heads_fastest ? dim3((unsigned)(Hkv * chunks), (unsigned)max_parts, (unsigned)S)
+                             : dim3((unsigned)max_parts, (unsigned)(Hkv * chunks), (unsigned)S);
     L.stream = reinterpret_cast<cudaStream_t>(stream);
 
     cudaError_t e;
@@ -235,7 +257,7 @@ extern "C" pa_status pa_decode(void* out, const void* q, pa_dtype q_dt, const vo
     if (e == cudaErrorNotSupported) return fail(PA_ERR_UNSUPPORTED, "no kernel for this shape");
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
     if (max_parts > 1) {
-        e = launch_merge(p, q_dt, D, dim3((unsigned)Hq, (unsigned)S), L.stream);
+        e = launch_merge(p, q_dt, D, Hq, S, L.stream);
         if (e != cudaSuccess) return cuda_fail(e, "split-K merge launch");
     }
     return PA_OK;

@@ -57,6 +57,7 @@ struct Params {
     int part_tokens;             // part_blocks * bs
     int max_ctx;                 // upper bound the grid / workspace were sized for
     int evict_first;             // 1: stream K/V with an L2 evict-first hint
+    int heads_fastest;           // grid order: 1 = (kv head, partition, seq), 0 = (partition, kv head, seq)
     int64_t NB;
     float qk_scale;              // scale * k_scale * log2(e)
     float v_scale;
@@ -90,15 +91,33 @@ struct Cfg {
     static constexpr int STAGE = 2 * TILE;
     static constexpr int NW = 4;             // consumer warps
     static constexpr int THREADS = (NW + 1) * 32;
-    static constexpr int STAGES_RAW = (64 * 1024) / STAGE;   // 3 CTAs per SM fit
-    static constexpr int STAGES = STAGES_RAW < NW ? NW : (STAGES_RAW > 16 ? 16 : STAGES_RAW);
-    static constexpr int COMBINE_FLOATS = NW * GC * (D + 2);
-    static constexpr size_t SMEM = 1024 /*align slack*/ + size_t(STAGES) * STAGE + 2 * 8 * STAGES;
+    // fp8 + tensor cores: each consumer warp dequantises V into an f16 tile
+    static constexpr bool FP8MMA = MMA && DT == PA_FP8_E4M3;
+    static constexpr int VSTG = FP8MMA ? BS * D * 2 : 0;     // per-warp staging bytes
+    static constexpr int BUDGET = (FP8MMA ? 72 : 64) * 1024;  // 3 CTAs per SM fit
+    static constexpr int COMBINE_FLOATS = NW * GC * (D + 2);   // warp merge reuses the stages
+    static constexpr int STAGES_RAW = (BUDGET - NW * VSTG) / STAGE;
+    static constexpr int STAGES_MIN_C = (COMBINE_FLOATS * 4 + STAGE - 1) / STAGE;
+    static constexpr int STAGES_MIN = STAGES_MIN_C > NW ? STAGES_MIN_C : NW;
+    static constexpr int STAGES_MAX = STAGES_MIN > 16 ? STAGES_MIN : 16;
+    static constexpr int STAGES = STAGES_RAW < STAGES_MIN ? STAGES_MIN
+                                  : (STAGES_RAW > STAGES_MAX ? STAGES_MAX : STAGES_RAW);
+    static constexpr size_t SMEM = 1024 /*align slack*/ + size_t(STAGES) * STAGE +
+                                   size_t(NW) * VSTG + 2 * 8 * STAGES;
     static_assert(R == 128 || R == 256 || R == 512, "row bytes must be 128, 256 or 512");
     static_assert(BS == 8 || BS == 16 || BS == 32, "block size");
     static_assert(COMBINE_FLOATS * 4 <= STAGES * STAGE, "combine area must fit in the stages");
     static_assert(SMEM <= 227 * 1024, "shared memory");
 };
+
+// Tiles are stored segment-major: [128-byte segment][token][128 bytes], each
+// 128-byte row swizzled by its token index (TMA SWIZZLE_128B, one box per
+// segment).  Eight consecutive tokens of one 16-byte chunk column therefore
+// sit in eight different bank groups, which keeps ldmatrix conflict-free.
+template <class C>
+__device__ __forceinline__ uint32_t tile_off(int t, int seg, int chunk) {
+    return (uint32_t)seg * (C::BS * 128) + dev::swz128(t, chunk);
+}
 
 // ------------------------------------------------------------------ producer
 // One warp; lane 0 issues.  Block ids are fetched 32 at a time (one per lane)
@@ -134,8 +153,12 @@ __device__ __forceinline__ void produce(const CUtensorMap* tmk, const CUtensorMa
                     const uint32_t bar = full0 + 8 * st;
                     const uint32_t dk = dev::smem_addr(stages + (size_t)st * C::STAGE);
                     dev::mbar_arrive_expect_tx(bar, C::STAGE);
-                    dev::tma_load_5d(dk, tmk, bar, 0, 0, kvh, 0, id, pol);
-                    dev::tma_load_5d(dk + C::TILE, tmv, bar, 0, 0, kvh, 0, id, pol);
+                    #pragma unroll
+                    for (int k = 0; k < C::CH; ++k) {
+                        dev::tma_load_4d(dk + k * C::BS * 128, tmk, bar, k * C::EPS, kvh, 0, id, pol);
+                        dev::tma_load_4d(dk + C::TILE + k * C::BS * 128, tmv, bar, k * C::EPS, kvh,
+                                         0, id, pol);
+                    }
                     ++issued;
                 }
             }
@@ -183,7 +206,7 @@ template <class C>
 __device__ __forceinline__ void simt_row(const uint8_t* tile, int t, int l8, float* f) {
     #pragma unroll
     for (int k = 0; k < C::CH; ++k) {
-        const uint4 r = *reinterpret_cast<const uint4*>(tile + dev::swz128(t * C::CH + k, l8));
+        const uint4 r = *reinterpret_cast<const uint4*>(tile + tile_off<C>(t, k, l8));
         dev::Chunk<C::DT>::to_float(r, f + k * C::EPC);
     }
 }
@@ -356,8 +379,17 @@ __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
 //         fragments into the B fragments of the second product
 //   O^T [D x heads]     += V^T [D x tokens] . P^T [tokens x heads]
 // A thread owns heads 2*tig, 2*tig+1 of each head tile for softmax state.
+// 16-bit caches feed both products straight from the stage with ldmatrix.
+// An fp8 cache computes in f16: K fragments come from ldmatrix on the bytes
+// (a b16 lane holds 2 codes, so a thread receives 4 consecutive dims) and are
+// widened with cvt.f16x2.e4m3x2; the contraction index is permuted the same
+// way on Q, so logical k (2t, 2t+1 | 2t+8, 2t+9) of a 16-dim step is physical
+// dim (4t, 4t+1 | 4t+2, 4t+3).  V is widened into a per-warp f16 tile first
+// (ldmatrix.trans has no byte form), with rows past the valid tokens zeroed.
 template <class C>
 struct MmaState {
+    static constexpr bool FP8 = C::DT == PA_FP8_E4M3;
+    static constexpr int CT = FP8 ? PA_F16 : C::DT;   // tensor-core input type
     static constexpr int NH = C::MROWS / 8;  // head tiles of 8
     static constexpr int KS = C::D / 16;     // k-steps over D
     static constexpr int MD = C::D / 16;     // m-tiles of O^T
@@ -365,6 +397,23 @@ struct MmaState {
     float o[NH][MD][4];                      // O^T accumulators
     float m[NH][2], l[NH][2];                // heads 2*tig, 2*tig+1 of each tile
 };
+
+template <int QT>
+__device__ __forceinline__ uint32_t to_f16x2(uint32_t w) {
+    if constexpr (QT == PA_F16) {
+        return w;
+    } else {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
+        __half2 h = __floats2half2_rn(f.x, f.y);
+        return *reinterpret_cast<uint32_t*>(&h);
+    }
+}
+
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
+    __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_codes & 0xffffu),
+                                               __NV_E4M3);
+    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
 
 template <class C>
 __device__ __forceinline__ void mma_load_q(MmaState<C>& st, const Params& p, int s, int h0,
@@ -379,9 +428,20 @@ __device__ __forceinline__ void mma_load_q(MmaState<C>& st, const Params& p, int
         const size_t base = (((size_t)s * p.Hq + h0 + head) * C::D) / 2;
         #pragma unroll
         for (int ks = 0; ks < S::KS; ++ks) {
-            // b0: dims ks*16 + 2tig, +1;  b1: dims ks*16 + 8 + 2tig, +1
-            st.qb[nh][ks][0] = head < G ? __ldg(q32 + base + ks * 8 + tig) : 0u;
-            st.qb[nh][ks][1] = head < G ? __ldg(q32 + base + ks * 8 + 4 + tig) : 0u;
+            uint32_t b0 = 0u, b1 = 0u;
+            if (head < G) {
+                if constexpr (S::FP8) {
+                    // physical dims ks*16 + 4tig, +1  and  ks*16 + 4tig + 2, +3
+                    b0 = to_f16x2<C::QT>(__ldg(q32 + base + ks * 8 + 2 * tig));
+                    b1 = to_f16x2<C::QT>(__ldg(q32 + base + ks * 8 + 2 * tig + 1));
+                } else {
+                    // dims ks*16 + 2tig, +1  and  ks*16 + 8 + 2tig, +1
+                    b0 = __ldg(q32 + base + ks * 8 + tig);
+                    b1 = __ldg(q32 + base + ks * 8 + 4 + tig);
+                }
+            }
+            st.qb[nh][ks][0] = b0;
+            st.qb[nh][ks][1] = b1;
         }
         #pragma unroll
         for (int md = 0; md < S::MD; ++md)
@@ -395,18 +455,49 @@ __device__ __forceinline__ void mma_load_q(MmaState<C>& st, const Params& p, int
 // smem address of 16-byte chunk c (over the whole row) of token row t
 template <class C>
 __device__ __forceinline__ uint32_t chunk_addr(uint32_t tile, int t, int c) {
-    return tile + dev::swz128(t * C::CH + (c >> 3), c & 7);
+    return tile + tile_off<C>(t, c >> 3, c & 7);
+}
+
+// fp8 V tile -> f16 tile (same segment-major swizzled layout, 64 dims per
+// segment); rows at or past nvalid become zeros.
+template <class C>
+__device__ __forceinline__ void stage_v_f16(const uint8_t* vt, uint8_t* dst, int nvalid) {
+    const int lane = threadIdx.x & 31;
+    __syncwarp();                                  // previous block's reads of dst are done
+    #pragma unroll
+    for (int i = 0; i < C::BS / 4; ++i) {
+        const int idx = lane + 32 * i;
+        const int t = idx >> 3, j = idx & 7;       // token, 16-dim chunk of the fp8 row
+        uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
+        if (t < nvalid) {
+            const uint4 r = *reinterpret_cast<const uint4*>(vt + tile_off<C>(t, 0, j));
+            lo = make_uint4(e4m3x2_to_f16x2(r.x), e4m3x2_to_f16x2(r.x >> 16),
+                            e4m3x2_to_f16x2(r.y), e4m3x2_to_f16x2(r.y >> 16));
+            hi = make_uint4(e4m3x2_to_f16x2(r.z), e4m3x2_to_f16x2(r.z >> 16),
+                            e4m3x2_to_f16x2(r.w), e4m3x2_to_f16x2(r.w >> 16));
+        }
+        // f16 dims 16j..16j+7 -> segment j/4, chunk 2(j%4); +8.. -> chunk 2(j%4)+1.
+        // Lanes j >= 4 store their second chunk first, so each store instruction
+        // covers 8 distinct bank groups.
+        const int seg = j >> 2, c0 = 2 * (j & 3);
+        const bool swap = j >= 4;
+        uint8_t* base = dst + seg * (C::BS * 128);
+        *reinterpret_cast<uint4*>(base + dev::swz128(t, c0 + (swap ? 1 : 0))) = swap ? hi : lo;
+        *reinterpret_cast<uint4*>(base + dev::swz128(t, c0 + (swap ? 0 : 1))) = swap ? lo : hi;
+    }
+    __syncwarp();
 }
 
 template <class C>
 __device__ __forceinline__ void mma_block(MmaState<C>& st, uint8_t* ktile_p, uint8_t* vtile_p,
-                                          int nvalid, float qk_scale) {
+                                          uint8_t* vstage_p, int nvalid, float qk_scale) {
     using S = MmaState<C>;
     constexpr int BS = C::BS;
+    constexpr int CT = S::CT;
     constexpr int MT = BS >= 16 ? BS / 16 : 1;   // token m-tiles of S^T
     const int lane = threadIdx.x & 31;
     const int gid = lane >> 2, tig = lane & 3;
-    const uint32_t ktile = dev::smem_addr(ktile_p), vtile = dev::smem_addr(vtile_p);
+    const uint32_t ktile = dev::smem_addr(ktile_p);
 
     // ---- S^T = K Q^T --------------------------------------------------------
     float sc[MT][S::NH][4];
@@ -416,7 +507,36 @@ __device__ __forceinline__ void mma_block(MmaState<C>& st, uint8_t* ktile_p, uin
         for (int nh = 0; nh < S::NH; ++nh)
             #pragma unroll
             for (int i = 0; i < 4; ++i) sc[mt][nh][i] = 0.f;
-        if constexpr (BS >= 16) {
+        if constexpr (S::FP8) {
+            // a 16-byte chunk is one 16-dim k-step; ldmatrix rows are 8 tokens
+            #pragma unroll
+            for (int ks = 0; ks < S::KS; ks += 2) {
+                uint32_t r0, r1, r2, r3;
+                if constexpr (BS >= 16) {
+                    // (tok 0-7, chunk ks) (tok 8-15, ks) (tok 0-7, ks+1) (tok 8-15, ks+1)
+                    ldsm_x4(chunk_addr<C>(ktile, mt * 16 + ((lane >> 3) & 1) * 8 + (lane & 7),
+                                          ks + (lane >> 4)),
+                            r0, r1, r2, r3);
+                } else {
+                    // (tok 0-7, chunk ks) (tok 0-7, ks+1); rows 8-15 of A are zero
+                    uint32_t u0, u1;
+                    ldsm_x4(chunk_addr<C>(ktile, lane & 7, ks + ((lane >> 3) & 1)), r0, r2, u0, u1);
+                    r1 = r3 = 0u;
+                }
+                const uint32_t a00 = e4m3x2_to_f16x2(r0), a02 = e4m3x2_to_f16x2(r0 >> 16);
+                const uint32_t a01 = BS >= 16 ? e4m3x2_to_f16x2(r1) : 0u;
+                const uint32_t a03 = BS >= 16 ? e4m3x2_to_f16x2(r1 >> 16) : 0u;
+                const uint32_t a10 = e4m3x2_to_f16x2(r2), a12 = e4m3x2_to_f16x2(r2 >> 16);
+                const uint32_t a11 = BS >= 16 ? e4m3x2_to_f16x2(r3) : 0u;
+                const uint32_t a13 = BS >= 16 ? e4m3x2_to_f16x2(r3 >> 16) : 0u;
+                #pragma unroll
+                for (int nh = 0; nh < S::NH; ++nh) {
+                    mma16816<CT>(sc[mt][nh], a00, a01, a02, a03, st.qb[nh][ks][0], st.qb[nh][ks][1]);
+                    mma16816<CT>(sc[mt][nh], a10, a11, a12, a13, st.qb[nh][ks + 1][0],
+                                 st.qb[nh][ks + 1][1]);
+                }
+            }
+        } else if constexpr (BS >= 16) {
             #pragma unroll
             for (int ks = 0; ks < S::KS; ++ks) {
                 // matrices: (tok 0-7, chunk 2ks) (tok 8-15, 2ks) (tok 0-7, 2ks+1) (tok 8-15, 2ks+1)
@@ -426,7 +546,7 @@ __device__ __forceinline__ void mma_block(MmaState<C>& st, uint8_t* ktile_p, uin
                         a0, a1, a2, a3);
                 #pragma unroll
                 for (int nh = 0; nh < S::NH; ++nh)
-                    mma16816<C::DT>(sc[mt][nh], a0, a1, a2, a3, st.qb[nh][ks][0], st.qb[nh][ks][1]);
+                    mma16816<CT>(sc[mt][nh], a0, a1, a2, a3, st.qb[nh][ks][0], st.qb[nh][ks][1]);
             }
         } else {
             // 8 tokens: rows 8-15 of the A operand are zero
@@ -436,9 +556,9 @@ __device__ __forceinline__ void mma_block(MmaState<C>& st, uint8_t* ktile_p, uin
                 ldsm_x4(chunk_addr<C>(ktile, lane & 7, 2 * ks + (lane >> 3)), a0, a2, b0, b2);
                 #pragma unroll
                 for (int nh = 0; nh < S::NH; ++nh) {
-                    mma16816<C::DT>(sc[mt][nh], a0, 0u, a2, 0u, st.qb[nh][ks][0], st.qb[nh][ks][1]);
-                    mma16816<C::DT>(sc[mt][nh], b0, 0u, b2, 0u, st.qb[nh][ks + 1][0],
-                                    st.qb[nh][ks + 1][1]);
+                    mma16816<CT>(sc[mt][nh], a0, 0u, a2, 0u, st.qb[nh][ks][0], st.qb[nh][ks][1]);
+                    mma16816<CT>(sc[mt][nh], b0, 0u, b2, 0u, st.qb[nh][ks + 1][0],
+                                 st.qb[nh][ks + 1][1]);
                 }
             }
         }
@@ -485,26 +605,35 @@ __device__ __forceinline__ void mma_block(MmaState<C>& st, uint8_t* ktile_p, uin
         #pragma unroll
         for (int nh = 0; nh < S::NH; ++nh) {
             float r0, r1, r2, r3;
-            const uint32_t x = pack2<C::DT>(exp2f(sc[mt][nh][0] - st.m[nh][0]),
-                                            exp2f(sc[mt][nh][1] - st.m[nh][1]), r0, r1);
+            const uint32_t x = pack2<CT>(exp2f(sc[mt][nh][0] - st.m[nh][0]),
+                                         exp2f(sc[mt][nh][1] - st.m[nh][1]), r0, r1);
             st.l[nh][0] += r0;
             st.l[nh][1] += r1;
             pb[mt][nh][0] = movmatrix_t(x);                 // tokens mt*16 + 0..7
             if constexpr (BS >= 16) {
-                const uint32_t y = pack2<C::DT>(exp2f(sc[mt][nh][2] - st.m[nh][0]),
-                                                exp2f(sc[mt][nh][3] - st.m[nh][1]), r2, r3);
+                const uint32_t y = pack2<CT>(exp2f(sc[mt][nh][2] - st.m[nh][0]),
+                                             exp2f(sc[mt][nh][3] - st.m[nh][1]), r2, r3);
                 st.l[nh][0] += r2;
                 st.l[nh][1] += r3;
                 pb[mt][nh][1] = movmatrix_t(y);             // tokens mt*16 + 8..15
             }
         }
     }
-    // ---- the tail rows of V past nvalid may hold anything: zero them -------
-    if (nvalid < BS) {
-        uint4* v4 = reinterpret_cast<uint4*>(vtile_p + (size_t)nvalid * C::R);
-        const int n16 = (BS - nvalid) * C::R / 16;
-        for (int i = lane; i < n16; i += 32) v4[i] = make_uint4(0, 0, 0, 0);
-        __syncwarp();
+    // ---- V operand: the 16-bit tile itself (tail rows zeroed), or fp8 widened
+    uint32_t vtile;
+    if constexpr (S::FP8) {
+        stage_v_f16<C>(vtile_p, vstage_p, nvalid);
+        vtile = dev::smem_addr(vstage_p);
+    } else {
+        if (nvalid < BS) {
+            #pragma unroll
+            for (int k = 0; k < C::CH; ++k) {
+                uint4* v4 = reinterpret_cast<uint4*>(vtile_p + k * BS * 128 + nvalid * 128);
+                for (int i = lane; i < (BS - nvalid) * 8; i += 32) v4[i] = make_uint4(0, 0, 0, 0);
+            }
+            __syncwarp();
+        }
+        vtile = dev::smem_addr(vtile_p);
     }
     // ---- O^T += V^T P^T -------------------------------------------------------
     if constexpr (BS >= 16) {
@@ -519,7 +648,7 @@ __device__ __forceinline__ void mma_block(MmaState<C>& st, uint8_t* ktile_p, uin
                           a0, a1, a2, a3);
                 #pragma unroll
                 for (int nh = 0; nh < S::NH; ++nh)
-                    mma16816<C::DT>(st.o[nh][md], a0, a1, a2, a3, pb[kt][nh][0], pb[kt][nh][1]);
+                    mma16816<CT>(st.o[nh][md], a0, a1, a2, a3, pb[kt][nh][0], pb[kt][nh][1]);
             }
         }
     } else {
@@ -530,12 +659,14 @@ __device__ __forceinline__ void mma_block(MmaState<C>& st, uint8_t* ktile_p, uin
             ldsm_x4_t(chunk_addr<C>(vtile, lane & 7, 2 * md + (lane >> 3)), a0, a1, b0, b1);
             #pragma unroll
             for (int nh = 0; nh < S::NH; ++nh) {
-                mma1688<C::DT>(st.o[nh][md], a0, a1, pb[0][nh][0]);
-                mma1688<C::DT>(st.o[nh][md + 1], b0, b1, pb[0][nh][0]);
+                mma1688<CT>(st.o[nh][md], a0, a1, pb[0][nh][0]);
+                mma1688<CT>(st.o[nh][md + 1], b0, b1, pb[0][nh][0]);
             }
         }
     }
-    if (nvalid < BS) dev::fence_proxy_async_smem();   // generic writes before the next TMA fill
+    if constexpr (!S::FP8) {
+        if (nvalid < BS) dev::fence_proxy_async_smem();   // generic writes before the next TMA fill
+    }
 }
 
 template <class C>
@@ -578,15 +709,17 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     __shared__ int s_issued;
     uint8_t* stages = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const uint32_t full0 = dev::smem_addr(stages + (size_t)C::STAGES * C::STAGE);
+    uint8_t* vstage = stages + (size_t)C::STAGES * C::STAGE;         // C::NW * C::VSTG bytes
+    const uint32_t full0 = dev::smem_addr(vstage + (size_t)C::NW * C::VSTG);
     const uint32_t empty0 = full0 + 8 * C::STAGES;
 
     const int G = p.Hq / p.Hkv;
     const int gc = C::MMA ? G : C::GC;          // query heads this CTA serves
     const int chunks = G / gc;                  // head chunks per kv head
-    const int part = blockIdx.x;
-    const int kvh = blockIdx.y / chunks;
-    const int h0 = kvh * G + (blockIdx.y % chunks) * gc;
+    const int part = p.heads_fastest ? blockIdx.y : blockIdx.x;
+    const int hc = p.heads_fastest ? blockIdx.x : blockIdx.y;
+    const int kvh = hc / chunks;
+    const int h0 = kvh * G + (hc % chunks) * gc;
     const int s = blockIdx.z;
     const int n = checked_len(p, s, C::BS);
     const int nblk_all = (n + C::BS - 1) / C::BS;
@@ -637,7 +770,8 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
             }
             uint8_t* kt = stages + (size_t)stg * C::STAGE;
             const int nvalid = min(C::BS, n - (blk0 + j) * C::BS);
-            if constexpr (C::MMA) mma_block<C>(st, kt, kt + C::TILE, nvalid, p.qk_scale);
+            if constexpr (C::MMA)
+                mma_block<C>(st, kt, kt + C::TILE, vstage + warp * C::VSTG, nvalid, p.qk_scale);
             else simt_block<C>(st, kt, kt + C::TILE, nvalid);
             __syncwarp();
             if (lane == 0) dev::mbar_arrive(empty0 + 8 * stg);
@@ -645,6 +779,7 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
         }
     }
     __syncthreads();                             // every stage consumed (or abort)
+    dev::launch_dependents();                    // the merge kernel may start launching
 
     if (s_abort) {
         // Drain: wait (bounded) until every issued copy has landed, then leave.
@@ -689,64 +824,77 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
 }
 
 // Merge split-K partials: out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p.
-// One CTA per (query head, sequence); its 8 warps split the partitions and
-// each lane holds D/32 dims, so every partial row is one coalesced load.
+// A CTA of 8 warps serves 8 / wph query heads of one sequence; the wph warps
+// of a head split its partitions, and each lane holds D/32 dims, so every
+// partial row is one coalesced load.  Launched as a programmatic dependent of
+// the partition kernel: it waits for that grid's memory before reading.
 constexpr int kMergeWarps = 8;
 
 template <int QT, int D>
-__global__ void __launch_bounds__(kMergeWarps * 32) decode_merge(const Params p) {
+__global__ void __launch_bounds__(kMergeWarps * 32) decode_merge(const Params p, int wph) {
     constexpr int DL = D / 32;                        // dims per lane
     __shared__ float s_max[kMergeWarps];
     __shared__ float s_l[kMergeWarps];
-    __shared__ float s_o[kMergeWarps][D];
-    const int h = blockIdx.x, s = blockIdx.y;
+    __shared__ __align__(16) float s_o[kMergeWarps][D];
+    dev::grid_dependency_wait();
+    const int hpc = kMergeWarps / wph;                // heads per CTA
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int hl = warp / wph, sub = warp % wph;
+    const int h = blockIdx.x * hpc + hl, s = blockIdx.y;
     int n = p.context_lens[s];
     n = max(0, min(n, min(p.max_ctx, p.MB * (p.part_tokens / p.part_blocks))));
     const int nparts = min(p.max_parts, (n + p.part_tokens - 1) / p.part_tokens);
-    if (nparts <= 1) return;
-    const size_t row0 = ((size_t)s * p.Hq + h) * p.max_parts;
+    if (nparts <= 1) return;                          // written by the partition kernel
+    const bool live = h < p.Hq;
+    const size_t row0 = ((size_t)s * p.Hq + (live ? h : 0)) * p.max_parts;
 
     float mx = -INFINITY;
-    for (int i = threadIdx.x; i < nparts; i += blockDim.x) mx = fmaxf(mx, p.ws_ml[row0 + i].x);
+    if (live)
+        for (int i = sub * 32 + lane; i < nparts; i += wph * 32) mx = fmaxf(mx, p.ws_ml[row0 + i].x);
     #pragma unroll
     for (int x = 16; x > 0; x >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, x));
     if (lane == 0) s_max[warp] = mx;
     __syncthreads();
-    float M = s_max[0];
-    #pragma unroll
-    for (int w = 1; w < kMergeWarps; ++w) M = fmaxf(M, s_max[w]);
+    float M = -INFINITY;
+    for (int w = hl * wph; w < (hl + 1) * wph; ++w) M = fmaxf(M, s_max[w]);
 
     float L = 0.f, o[DL];
     #pragma unroll
     for (int k = 0; k < DL; ++k) o[k] = 0.f;
-    #pragma unroll 4
-    for (int i = warp; i < nparts; i += kMergeWarps) {
-        const float2 ml = p.ws_ml[row0 + i];
-        const float f = exp2f(ml.x - M);
-        L = fmaf(f, ml.y, L);
-        const float* src = p.ws_o + (row0 + i) * D + lane * DL;
-        if constexpr (DL == 4) {
-            const float4 v = *reinterpret_cast<const float4*>(src);
-            o[0] = fmaf(f, v.x, o[0]); o[1] = fmaf(f, v.y, o[1]);
-            o[2] = fmaf(f, v.z, o[2]); o[3] = fmaf(f, v.w, o[3]);
-        } else {
-            #pragma unroll
-            for (int k = 0; k < DL; ++k) o[k] = fmaf(f, src[k], o[k]);
+    if (live) {
+        #pragma unroll 4
+        for (int i = sub; i < nparts; i += wph) {
+            const float2 ml = p.ws_ml[row0 + i];
+            const float f = exp2f(ml.x - M);
+            L = fmaf(f, ml.y, L);
+            const float* src = p.ws_o + (row0 + i) * D + lane * DL;
+            if constexpr (DL % 4 == 0) {
+                #pragma unroll
+                for (int k = 0; k < DL; k += 4) {
+                    const float4 v = *reinterpret_cast<const float4*>(src + k);
+                    o[k] = fmaf(f, v.x, o[k]); o[k + 1] = fmaf(f, v.y, o[k + 1]);
+                    o[k + 2] = fmaf(f, v.z, o[k + 2]); o[k + 3] = fmaf(f, v.w, o[k + 3]);
+                }
+            } else {
+                #pragma unroll
+                for (int k = 0; k < DL; ++k) o[k] = fmaf(f, src[k], o[k]);
+            }
         }
     }
     if (lane == 0) s_l[warp] = L;
     #pragma unroll
     for (int k = 0; k < DL; ++k) s_o[warp][lane * DL + k] = o[k];
     __syncthreads();
-    for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    for (int idx = threadIdx.x; idx < hpc * D; idx += blockDim.x) {
+        const int hh = idx / D, d = idx % D;
+        const int head = blockIdx.x * hpc + hh;
+        if (head >= p.Hq) continue;
         float Lt = 0.f, Ot = 0.f;
-        #pragma unroll
-        for (int w = 0; w < kMergeWarps; ++w) {
+        for (int w = hh * wph; w < (hh + 1) * wph; ++w) {
             Lt += s_l[w];
             Ot += s_o[w][d];
         }
-        dev::store_out<QT>(p.out, ((size_t)s * p.Hq + h) * D + d, Lt > 0.f ? Ot / Lt : 0.f);
+        dev::store_out<QT>(p.out, ((size_t)s * p.Hq + head) * D + d, Lt > 0.f ? Ot / Lt : 0.f);
     }
 }
 

@@ -51,7 +51,8 @@ cudaError_t launch_by_heads(const Launch& L) {
         return cudaErrorNotSupported;
     } else {
         if (L.mma) {
-            if constexpr (DT == QT && (DT == PA_F16 || DT == PA_BF16) && D <= 128) {
+            if constexpr (((DT == QT && (DT == PA_F16 || DT == PA_BF16)) || DT == PA_FP8_E4M3) &&
+                          D <= 128) {
                 if (L.mrows == 8) return launch_one<Cfg<DT, QT, BS, D, 8, true, 8>>(L);
                 return launch_one<Cfg<DT, QT, BS, D, 16, true, 16>>(L);
             } else {

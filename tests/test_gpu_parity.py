@@ -26,7 +26,7 @@ def _cuda():
         pytest.skip("needs a GPU")
     pa.pa_device_status(clear=True)
     yield
-    pa.pa_decode_select(0)
+    pa.pa_decode_select(pa.DECODE_DEFAULT)
 
 
 def _to(inp: wl.DecodeInputs, device):
@@ -37,7 +37,7 @@ def _to(inp: wl.DecodeInputs, device):
     return f
 
 
-def gpu_step(inp: wl.DecodeInputs, partition: int, mode: int = 0, max_ctx=None):
+def gpu_step(inp: wl.DecodeInputs, partition: int, mode: int = pa.DECODE_DEFAULT, max_ctx=None):
     d = _to(inp, "cuda")
     kc, vc = d["key_cache"].clone(), d["value_cache"].clone()
     if inp.copy_pairs.numel():
@@ -86,6 +86,11 @@ def _check_out(got: torch.Tensor, want: np.ndarray, dt: str, what: str):
     return err
 
 
+MODES = [pa.DECODE_DEFAULT, pa.DECODE_DEFAULT | pa.DECODE_SIMT_ONLY,
+         pa.DECODE_DEFAULT | pa.DECODE_EVICT_FIRST, 0]
+BOTH = [pa.DECODE_DEFAULT, pa.DECODE_DEFAULT | pa.DECODE_SIMT_ONLY]
+
+
 SMALL = [
     ("cfg1", wl.CONFIGS[1]),
     ("cfg2", wl.small_variant(wl.CONFIGS[2], 5, 1, 200)),
@@ -97,7 +102,7 @@ SMALL = [
 
 @pytest.mark.parametrize("name,cfg", SMALL, ids=[n for n, _ in SMALL])
 @pytest.mark.parametrize("partition_blocks", [0, 2, 7])
-@pytest.mark.parametrize("mode", [0, 1], ids=["auto", "simt"])
+@pytest.mark.parametrize("mode", MODES, ids=["auto", "simt", "evict_first", "head_major"])
 def test_step_parity_small(name, cfg, partition_blocks, mode):
     inp = wl.make_decode_inputs(cfg, seed=101)
     want, kc_o, vc_o = oracle_step(inp)
@@ -122,7 +127,7 @@ def test_decode_shapes(bs, G, D, dt):
     inp = wl.make_decode_inputs(cfg, seed=bs * 1000 + G * 10 + D)
     want, _, _ = oracle_step(inp)
     for part in (0, bs):
-        for mode in (0, 1):
+        for mode in BOTH:
             out, _, _ = gpu_step(inp, part, mode)
             _check_out(out, want, dt, f"P={part} mode={mode}")
     assert pa.pa_device_status() == 0
@@ -136,7 +141,7 @@ def test_lengths_at_partition_edges(dt):
                           fixed_lens=lens, fp8_scaled=dt == "fp8_e4m3")
     inp = wl.make_decode_inputs(cfg, seed=7)
     want, _, _ = oracle_step(inp)
-    for mode in (0, 1):
+    for mode in BOTH:
         out, _, _ = gpu_step(inp, P, mode)
         _check_out(out, want, dt, f"mode={mode}")
 
