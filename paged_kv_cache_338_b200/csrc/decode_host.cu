@@ -132,9 +132,10 @@ extern "C" pa_status pa_decode_suggest_partition(int S, int Hkv, int bs,
     if (!partition || (S > 0 && !context_lens_host) || S < 0 || Hkv <= 0 ||
         !(bs == 8 || bs == 16 || bs == 32))
         return fail(PA_ERR_INVALID_ARG, "bad arguments");
-    // Enough CTAs for several waves on 148 SMs (a few resident per SM) so the
-    // last wave is short, with partitions no shorter than 256 tokens.
-    const int64_t want = 148LL * 3 * 8;
+    // Enough CTAs for several waves on 148 SMs (3 resident per SM) so the last
+    // wave is short, with partitions as long as that allows (each CTA pays a
+    // start-up and drain of a few microseconds) and no shorter than 256 tokens.
+    const int64_t want = 148LL * 3 * 4;
     int64_t maxn = 0;
     for (int s = 0; s < S; ++s) maxn = context_lens_host[s] > maxn ? context_lens_host[s] : maxn;
     auto items = [&](int64_t P) {
