@@ -32,7 +32,28 @@ import subprocess
 import sys
 import time
 
-import torch
+
+def _nvml_sampler(pci_id: str, path: str) -> None:
+    """Child process: append "wall_time sm_mhz max_mhz reason_bits" every ~1 ms."""
+    import pynvml as nv
+    nv.nvmlInit()
+    h = nv.nvmlDeviceGetHandleByPciBusId(pci_id) if pci_id else nv.nvmlDeviceGetHandleByIndex(0)
+    mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+    with open(path, "w", buffering=1) as f:
+        while True:
+            try:
+                f.write(f"{time.time():.6f} {nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)} {mx} "
+                        f"{int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))}\n")
+            except Exception:
+                pass
+            time.sleep(0.001)
+
+
+if __name__ == "__main__" and len(sys.argv) == 4 and sys.argv[1] == "--nvml-sampler":
+    _nvml_sampler(sys.argv[2], sys.argv[3])        # clock-sampling child (no torch import)
+    sys.exit(0)
+
+import torch  # noqa: E402
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
@@ -74,77 +95,83 @@ def _pci_id(dev: int) -> str | None:
 
 
 class ClockSampler:
-    """SM clock, power and clock-event reasons sampled DURING a timed region.
+    """SM clock and clock-event reasons sampled DURING the timed region.
 
-    A background thread polls NVML about every millisecond (a decode step is
-    well under a millisecond, so nvidia-smi's 200 ms period would miss most
-    regions); nvidia-smi's own sampling runs beside it and is kept in
-    gpurun_out/ as the raw record.  Nothing is changed on the GPU: read-only
-    queries.
+    A child process polls NVML about every millisecond and timestamps each
+    sample (a decode step is well under a millisecond, and a thread in this
+    process would be starved by the launch loop); samples inside
+    [mark_start, mark_end] are kept.  nvidia-smi's own log runs beside it as
+    the raw record.  Read-only queries: nothing on the GPU is changed.
     """
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, dev: int):
-        import threading
-        self.samples, self.max_mhz, self.reason_bits = [], None, 0
-        self.stop_flag = threading.Event()
-        self.thread = None
-        self.proc = None
+        self.t0 = self.t1 = None
         pid = _pci_id(dev)
+        os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
+        self.path = os.path.join(ROOT, "gpurun_out", f"nvml_rank{dev}.log")
+        self.child = subprocess.Popen([sys.executable, os.path.abspath(__file__),
+                                       "--nvml-sampler", pid or "", self.path],
+                                      stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        self.proc = None
         try:
-            import pynvml as nv
-            nv.nvmlInit()
-            h = nv.nvmlDeviceGetHandleByPciBusId(pid) if pid else nv.nvmlDeviceGetHandleByIndex(dev)
-            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
-            self.nv, self.h = nv, h
-
-            def poll():
-                while not self.stop_flag.is_set():
-                    try:
-                        self.samples.append(float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)))
-                        self.reason_bits |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))
-                    except Exception:
-                        pass
-                    time.sleep(0.001)
-            self.thread = threading.Thread(target=poll, daemon=True)
-            self.thread.start()
-        except Exception:
-            self.thread = None
-        try:
-            path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{dev}.csv")
-            os.makedirs(os.path.dirname(path), exist_ok=True)
             args = ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
                     "-lms", "200"] + (["-i", pid] if pid else [])
-            self.f = open(path, "w")
+            self.f = open(os.path.join(ROOT, "gpurun_out", f"clocks_rank{dev}.csv"), "w")
             self.proc = subprocess.Popen(args, stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+        # wait until the child has produced its first sample
+        for _ in range(400):
+            if os.path.exists(self.path) and os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.01)
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
 
     def stop(self) -> dict:
-        if self.thread is not None:
-            self.stop_flag.set()
-            self.thread.join(timeout=2)
-        if self.proc is not None:
-            self.proc.terminate()
+        time.sleep(0.01)
+        for p in (self.child, self.proc):
+            if p is None:
+                continue
+            p.terminate()
             try:
-                self.proc.wait(timeout=5)
+                p.wait(timeout=5)
             except Exception:
-                self.proc.kill()
+                p.kill()
+        if self.proc is not None:
             self.f.close()
-        if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"]}
-        nv = self.nv
+        import pynvml as nv
         names = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
                  "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
                  "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
                  "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap,
                  "hw_power_brake_slowdown": nv.nvmlClocksEventReasonHwPowerBrakeSlowdown}
-        sm = sorted(self.samples)
-        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(n for n, b in names.items() if self.reason_bits & b),
-                "samples": len(sm), "sm_mhz_min": sm[0], "source": "nvml, 1 ms"}
+        sm, mx, bits = [], None, 0
+        try:
+            for line in open(self.path):
+                c = line.split()
+                if len(c) != 4:
+                    continue
+                t = float(c[0])
+                if self.t0 is not None and self.t0 <= t <= self.t1:
+                    sm.append(float(c[1]))
+                    mx = float(c[2])
+                    bits |= int(c[3])
+        except OSError:
+            pass
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": ["unsampled"]}
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx,
+                "reasons": sorted(n for n, b in names.items() if bits & b),
+                "samples": len(sm), "sm_mhz_min": sm[0], "source": "nvml child process, 1 ms"}
 
 
 # ------------------------------------------------------------------ oracle arm
@@ -287,11 +314,13 @@ def run_gpu(args, cfg, rank, world, local_rank):
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks.mark_start()
     t0.record(stream)
     for i in range(args.steps):
         step(evs[i])
     t1.record(stream)
     torch.cuda.synchronize()
+    clocks.mark_end()
     clk = clocks.stop()
     if dist:
         torch.distributed.barrier()
@@ -394,42 +423,49 @@ def run_e2e(args, cfg, pa, dev, part):
             parents.append(pool.seq_fork(sid))
         seqs.append(sid)
     MB = (max(lens) + args.warmup + args.steps + 2 + bs - 1) // bs
-    pin = dict(pin_memory=True)
-    q_h = inp.q.cpu().pin_memory()
-    k_h, v_h = inp.key_new.cpu().pin_memory(), inp.value_new.cpu().pin_memory()
-    out_h = torch.empty(inp.q.shape, dtype=inp.q.dtype, **pin)
-    slots_h = torch.empty(S, dtype=torch.int64, **pin)
-    tab_h = torch.empty((S, MB), dtype=torch.int32, **pin)
-    len_h = torch.empty(S, dtype=torch.int32, **pin)
-    q_d, k_d, v_d = torch.empty_like(inp.q), torch.empty_like(inp.key_new), torch.empty_like(inp.value_new)
-    slots_d = torch.empty(S, dtype=torch.int64, device=dev)
-    tab_d = torch.empty((S, MB), dtype=torch.int32, device=dev)
-    len_d = torch.empty(S, dtype=torch.int32, device=dev)
+    seq_ids = torch.tensor(seqs, dtype=torch.int64)
+    # every per-step input lives in one pinned staging buffer (the model would
+    # write q, k, v there; the pool writes slots, tables and lengths there), so
+    # one H2D copy moves a step's inputs; one D2H copy returns its output
+    parts = [("q", inp.q), ("k", inp.key_new), ("v", inp.value_new),
+             ("slots", torch.empty(S, dtype=torch.int64)),
+             ("tables", torch.empty((S, MB), dtype=torch.int32)),
+             ("lens", torch.empty(S, dtype=torch.int32))]
+    offs, total = {}, 0
+    for name, t in parts:
+        offs[name] = total
+        total += (t.numel() * t.element_size() + 255) // 256 * 256
+    stage_h = torch.empty(total, dtype=torch.uint8, pin_memory=True)
+    stage_d = torch.empty(total, dtype=torch.uint8, device=dev)
+
+    def view(buf, name, like):
+        nbytes = like.numel() * like.element_size()
+        return buf[offs[name]:offs[name] + nbytes].view(like.dtype).view(like.shape)
+
+    hv = {name: view(stage_h, name, t) for name, t in parts}
+    dv = {name: view(stage_d, name, t) for name, t in parts}
+    hv["q"].copy_(inp.q.cpu())
+    hv["k"].copy_(inp.key_new.cpu())
+    hv["v"].copy_(inp.value_new.cpu())
+    out_h = torch.empty(inp.q.shape, dtype=inp.q.dtype, pin_memory=True)
     out_d = torch.empty_like(inp.q)
+    cow_buf = torch.empty((S, 2), dtype=torch.int32)
     ws_bytes = pa.pa_decode_workspace_size(S, Hq, D, max_ctx, part)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     total_bytes = 0
 
     def step():
-        nonlocal total_bytes
-        pairs = []
-        for i, sid in enumerate(seqs):
-            slot, src, dst = pool.seq_append(sid)
-            slots_h[i] = slot
-            if src >= 0:
-                pairs.append((src, dst))
-        pool.build_block_tables(seqs, MB, tab_h, len_h)
-        for h, d in ((q_h, q_d), (k_h, k_d), (v_h, v_d), (slots_h, slots_d), (tab_h, tab_d),
-                     (len_h, len_d)):
-            d.copy_(h, non_blocking=True)
-        if pairs:
+        _, pairs = pool.seq_append_batch(seq_ids, hv["slots"], cow_buf)
+        pool.build_block_tables(seq_ids, MB, hv["tables"], hv["lens"])
+        stage_d.copy_(stage_h, non_blocking=True)
+        if pairs.numel():
             pa.pa_copy_blocks(kc, vc, pairs)
-        pa.pa_reshape_and_cache(k_d, v_d, kc, vc, slots_d, inp.k_scale, inp.v_scale)
-        pa.pa_decode(out_d, q_d, kc, vc, tab_d, len_d, max_ctx, inp.scale, inp.k_scale,
-                     inp.v_scale, part, ws if ws_bytes else None)
+        pa.pa_reshape_and_cache(dv["k"], dv["v"], kc, vc, dv["slots"], inp.k_scale, inp.v_scale)
+        pa.pa_decode(out_d, dv["q"], kc, vc, dv["tables"], dv["lens"], max_ctx, inp.scale,
+                     inp.k_scale, inp.v_scale, part, ws if ws_bytes else None)
         out_h.copy_(out_d, non_blocking=True)
-        nb = algorithmic_bytes(cfg, len_h)
+        nb = algorithmic_bytes(cfg, hv["lens"])
         return nb["decode"] + nb["append"]
 
     for _ in range(args.warmup):
@@ -444,7 +480,7 @@ def run_e2e(args, cfg, pa, dev, part):
         e1.synchronize()          # the result is on the host: the step is over
         ms += e0.elapsed_time(e1)
     assert pa.pa_device_status() == 0
-    h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h, slots_h, tab_h, len_h))
+    h2d = total
     d2h = out_h.numel() * out_h.element_size()
     pool.close()
     return {"ms": ms / args.steps, "bytes": total_bytes / args.steps,

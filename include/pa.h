@@ -279,6 +279,16 @@ pa_status pa_pool_seq_share_prefix(pa_pool* pool, int64_t seq, const int32_t* bl
  */
 pa_status pa_pool_seq_append(pa_pool* pool, int64_t seq, int64_t* slot, int32_t* cow_src,
                              int32_t* cow_dst);
+/*
+ * pa_pool_seq_append for each of n distinct sequences, in order, in one call
+ * (one decode step of a batch).  slots[i] receives sequence i's slot;
+ * cow_pairs receives the *n_cow (src, dst) copies to enqueue with
+ * pa_copy_blocks before the append kernel (room for n pairs).  All or
+ * nothing: an unknown or repeated sequence, or fewer free blocks than the
+ * batch needs, returns an error and changes nothing.
+ */
+pa_status pa_pool_seq_append_batch(pa_pool* pool, const int64_t* seqs, int n, int64_t* slots,
+                                   int32_t* cow_pairs, int* n_cow);
 /* Drop the sequence's reference on each of its blocks, in table order.  All
  * or nothing: PA_ERR_REFCOUNT (and no change) if a block holds fewer
  * references than the sequence does. */

@@ -142,6 +142,25 @@ class PoolModel:
         self.seqs[sid][1] = n + 1
         return slot, src, dst
 
+    def seq_append_batch(self, sids):
+        """seq_append on each of distinct sequences in order; all or nothing."""
+        if len(set(sids)) != len(sids):
+            raise InvalidArg("a sequence appears twice")
+        need = 0
+        for sid in sids:
+            blocks, n = self._seq(sid)
+            if n % self.block_size == 0 or self.ref[blocks[-1]] > 1:
+                need += 1
+        if need > len(self.free_queue):
+            raise OutOfBlocks("not enough free blocks for the batch")
+        slots, pairs = [], []
+        for sid in sids:
+            slot, src, dst = self.seq_append(sid)
+            slots.append(slot)
+            if src >= 0:
+                pairs.append((src, dst))
+        return slots, pairs
+
     def seq_free(self, sid: int) -> None:
         blocks, _ = self._seq(sid)
         for b, k in Counter(blocks).items():  # all or nothing

@@ -88,6 +88,7 @@ def lib() -> ctypes.CDLL:
         "pa_pool_seq_append": ([P, I64, ctypes.POINTER(I64), ctypes.POINTER(I32),
                                 ctypes.POINTER(I32)], I),
         "pa_pool_seq_free": ([P, I64], I),
+        "pa_pool_seq_append_batch": ([P, P, I, P, P, ctypes.POINTER(I)], I),
         "pa_pool_seq_len": ([P, I64], I64),
         "pa_pool_build_block_tables": ([P, P, I, I, P, P], I),
         "pa_pool_stats": ([P, ctypes.POINTER(_Stats)], I),
@@ -293,6 +294,22 @@ class BlockPool:
                                         ctypes.byref(dst)))
         return slot.value, src.value, dst.value
 
+    def seq_append_batch(self, seqs, slots_out: Optional[torch.Tensor] = None,
+                         cow_out: Optional[torch.Tensor] = None):
+        """Append one token to each sequence: -> (slots int64 [n], cow pairs int32 [k, 2]).
+        seqs: host int64 tensor or sequence; outputs may be preallocated host tensors."""
+        ids = torch.as_tensor(seqs, dtype=torch.int64).contiguous()
+        n = ids.numel()
+        if slots_out is None:
+            slots_out = torch.empty(n, dtype=torch.int64)
+        if cow_out is None:
+            cow_out = torch.empty((max(n, 1), 2), dtype=torch.int32)
+        nc = ctypes.c_int(0)
+        _check(lib().pa_pool_seq_append_batch(self._p, ids.data_ptr() if n else None, n,
+                                              slots_out.data_ptr() if n else None,
+                                              cow_out.data_ptr(), ctypes.byref(nc)))
+        return slots_out, cow_out[:nc.value]
+
     def seq_free(self, seq: int) -> None:
         _check(lib().pa_pool_seq_free(self._p, seq))
 
@@ -303,8 +320,13 @@ class BlockPool:
                            tables_out: Optional[torch.Tensor] = None,
                            lens_out: Optional[torch.Tensor] = None):
         """Pack the tables into host int32 [S, max_blocks] (-1 padded) + lens [S]."""
-        S = len(seqs)
-        ids = (ctypes.c_int64 * S)(*seqs)
+        if isinstance(seqs, torch.Tensor):
+            assert seqs.dtype == torch.int64 and seqs.device.type == "cpu" and seqs.is_contiguous()
+            S = seqs.numel()
+            ids = ctypes.c_void_p(seqs.data_ptr()) if S else None
+        else:
+            S = len(seqs)
+            ids = (ctypes.c_int64 * S)(*seqs)
         if tables_out is None:
             tables_out = torch.empty((S, max_blocks), dtype=torch.int32)
         if lens_out is None:

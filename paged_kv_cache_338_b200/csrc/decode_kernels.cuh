@@ -100,12 +100,22 @@ struct Cfg {
     static constexpr int STAGES_MIN_C = (COMBINE_FLOATS * 4 + STAGE - 1) / STAGE;
     static constexpr int STAGES_MIN = STAGES_MIN_C > NW ? STAGES_MIN_C : NW;
     static constexpr int STAGES_MAX = STAGES_MIN > 16 ? STAGES_MIN : 16;
-    static constexpr int STAGES = STAGES_RAW < STAGES_MIN ? STAGES_MIN
-                                  : (STAGES_RAW > STAGES_MAX ? STAGES_MAX : STAGES_RAW);
+    static constexpr int STAGES_CLAMPED = STAGES_RAW < STAGES_MIN ? STAGES_MIN
+                                          : (STAGES_RAW > STAGES_MAX ? STAGES_MAX : STAGES_RAW);
+    // Block j goes to consumer warp j % NW and to stage j % STAGES.  With
+    // STAGES a multiple of NW every stage has exactly one consumer warp, so a
+    // warp waiting on a stage's "full" barrier is never more than one phase
+    // behind it and the parity wait cannot mistake an older, still pending
+    // phase for the one it wants.  Round down, or up when the warp merge needs
+    // the room.
+    static constexpr int STAGES_DOWN = STAGES_CLAMPED / NW * NW;
+    static constexpr int STAGES = STAGES_DOWN >= STAGES_MIN ? STAGES_DOWN
+                                  : (STAGES_MIN + NW - 1) / NW * NW;
     static constexpr size_t SMEM = 1024 /*align slack*/ + size_t(STAGES) * STAGE +
                                    size_t(NW) * VSTG + 2 * 8 * STAGES;
     static_assert(R == 128 || R == 256 || R == 512, "row bytes must be 128, 256 or 512");
     static_assert(BS == 8 || BS == 16 || BS == 32, "block size");
+    static_assert(STAGES % NW == 0, "each stage must have a single consumer warp");
     static_assert(COMBINE_FLOATS * 4 <= STAGES * STAGE, "combine area must fit in the stages");
     static_assert(SMEM <= 227 * 1024, "shared memory");
 };

@@ -177,6 +177,40 @@ extern "C" pa_status pa_pool_seq_append(pa_pool* pool, int64_t seq, int64_t* slo
     return PA_OK;
 }
 
+extern "C" pa_status pa_pool_seq_append_batch(pa_pool* pool, const int64_t* seqs, int n,
+                                              int64_t* slots, int32_t* cow_pairs, int* n_cow) {
+    pa::clear_error();
+    if (!pool || n < 0 || (n > 0 && (!seqs || !slots || !cow_pairs)) || !n_cow)
+        return fail(PA_ERR_INVALID_ARG, "bad arguments");
+    *n_cow = 0;
+    // all or nothing: validate every sequence and count the blocks needed first
+    std::unordered_map<int64_t, int> seen;
+    seen.reserve(2 * (size_t)n);
+    int64_t need = 0;
+    for (int i = 0; i < n; ++i) {
+        const pa_pool::Seq* s = pool->find(seqs[i]);
+        if (!s) return fail(PA_ERR_BAD_INDEX, "unknown sequence %lld", (long long)seqs[i]);
+        if (!seen.emplace(seqs[i], i).second)
+            return fail(PA_ERR_INVALID_ARG, "sequence %lld appears twice", (long long)seqs[i]);
+        if (s->n % pool->bs == 0 || pool->ref[s->blocks.back()] > 1) ++need;
+    }
+    if (need > (int64_t)pool->free_q.size())
+        return fail(PA_ERR_OUT_OF_BLOCKS, "%lld blocks needed, %zu free", (long long)need,
+                    pool->free_q.size());
+    int nc = 0;
+    for (int i = 0; i < n; ++i) {
+        int32_t src = -1, dst = -1;
+        pa_pool_seq_append(pool, seqs[i], &slots[i], &src, &dst);   // cannot fail now
+        if (src >= 0) {
+            cow_pairs[2 * nc] = src;
+            cow_pairs[2 * nc + 1] = dst;
+            ++nc;
+        }
+    }
+    *n_cow = nc;
+    return PA_OK;
+}
+
 extern "C" pa_status pa_pool_seq_free(pa_pool* pool, int64_t seq) {
     pa::clear_error();
     if (!pool) return fail(PA_ERR_INVALID_ARG, "pool is NULL");

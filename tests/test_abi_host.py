@@ -203,3 +203,38 @@ def test_pool_matches_model_on_random_call_sequences(seed):
         m, p = _run_both(model, pool, "alloc")
         assert m == p
     _run_both(model, pool, "alloc")
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_pool_batch_append_matches_model(seed):
+    rnd = random.Random(100 + seed)
+    nb, bs = 64, 8
+    model, pool = PoolModel(nb, bs), pa.BlockPool(nb, bs)
+    seqs = []
+    for _ in range(6):
+        s = model.seq_new()
+        assert pool.seq_new() == s
+        seqs.append(s)
+    for step in range(80):
+        if rnd.random() < 0.15:            # a sampling fork shares the last block
+            parent = rnd.choice(seqs)
+            c = model.seq_fork(parent)
+            assert pool.seq_fork(parent) == c
+            seqs.append(c)
+        batch = rnd.sample(seqs, rnd.randint(1, len(seqs)))
+        try:
+            ms, mp = model.seq_append_batch(batch)
+            merr = None
+        except PoolError as e:
+            merr = e.status
+        try:
+            ps, pp = pool.seq_append_batch(batch)
+            perr = None
+        except pa.PaError as e:
+            perr = e.status
+        assert merr == perr
+        if merr is None:
+            assert ps.tolist() == ms and pp.tolist() == [list(x) for x in mp]
+        assert [pool.ref(b) for b in range(nb)] == model.ref
+    with pytest.raises(pa.PaError):
+        pool.seq_append_batch([seqs[0], seqs[0]])      # repeated sequence
