@@ -69,8 +69,12 @@ enum {
     PA_DEV_BAD_SLOT = 1,      /* pa_reshape_and_cache: slot >= NB * bs, token skipped */
     PA_DEV_BAD_BLOCK = 2,     /* pa_decode: table entry outside [0, NB) (read as zeros) */
     PA_DEV_WAIT_TIMEOUT = 4,  /* a pipeline wait gave up after its bound; output invalid */
-    PA_DEV_BAD_CONTEXT = 8    /* pa_decode: context_lens[s] < 0, > max_ctx or > MB * bs (clamped) */
+    PA_DEV_BAD_CONTEXT = 8,   /* pa_decode: context_lens[s] < 0, > max_ctx or > MB * bs (clamped) */
+    PA_DEV_BAD_PIECES = 16    /* pa_decode merge: inconsistent split records (rows left unwritten) */
 };
+/* Bits 16-23 of the device word, when PA_DEV_WAIT_TIMEOUT is set: which wait
+ * gave up last (diagnostics; 1 stage-free, 2 stage-full, 3 descriptor-free,
+ * 4 descriptor-ready, 5 states-published, 6 merge-done). */
 
 /* Message for the last failing call on this thread ("" if none). */
 const char* pa_last_error(void);
@@ -126,10 +130,15 @@ pa_status pa_reshape_and_cache(const void* key, const void* value, pa_dtype in_d
 pa_status pa_copy_blocks(void* key_cache, void* value_cache, size_t block_bytes, int64_t NB,
                          const int32_t* pairs, int n, pa_stream_t stream);
 
+/* partition value selecting the persistent work-balanced decode (see pa_decode) */
+#define PA_PARTITION_BALANCED (-1)
+
 /*
- * Bytes of split-K workspace pa_decode needs for these sizes (0 when
- * partition == 0 or max_ctx <= partition).  Layout (fp32): per (s, query
- * head, partition) a running max m, a sum l, and an unnormalised o[D].
+ * Bytes of split-K workspace pa_decode needs for these sizes: 0 when
+ * partition == 0 or max_ctx <= partition; for fixed partitions, per
+ * (s, query head, partition) a running max m, a sum l and an unnormalised
+ * o[D] in fp32; for PA_PARTITION_BALANCED, an upper bound covering every
+ * kernel choice (per-item piece bounds plus one partial per piece).
  */
 pa_status pa_decode_workspace_size(int S, int Hq, int D, int max_ctx, int partition,
                                    size_t* bytes);
@@ -162,12 +171,15 @@ pa_status pa_decode_suggest_partition(int S, int Hkv, int bs, const int32_t* con
  * size of the cache in {128, 256, 512} bytes; Hq / Hkv in {1, 2, 4, 8, 16}.
  * Base pointers 16-byte aligned (TMA requirement).
  *
- * partition: 0 = one pass per (sequence, kv head); otherwise tokens per
- * split-K partition, a positive multiple of bs.  Sequences longer than one
- * partition are split; each partition writes (m, l, o) into `workspace`
- * (device, >= pa_decode_workspace_size() bytes, no initialisation needed)
- * and a second kernel on the same stream merges them.  max_ctx must be
- * >= every context_lens[s] (it sizes the grid and the workspace).
+ * partition: 0 = one pass per (sequence, kv head); a positive multiple of bs
+ * = tokens per split-K partition: sequences longer than one partition are
+ * split, each partition writes (m, l, o) into `workspace` and a second kernel
+ * on the same stream merges them; PA_PARTITION_BALANCED = a persistent grid
+ * sized to the GPU whose CTAs take equal contiguous shares of all blocks of
+ * all (sequence, kv head) items (items cut at share boundaries are merged
+ * the same way).  `workspace`: device, >= pa_decode_workspace_size() bytes,
+ * 16-byte aligned, no initialisation needed.  max_ctx must be >= every
+ * context_lens[s] (it sizes the grid and the workspace).
  */
 pa_status pa_decode(void* out, const void* q, pa_dtype q_dt,
                     const void* key_cache, const void* value_cache, pa_dtype cache_dt,

@@ -34,6 +34,7 @@ STATUS = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED",
           6: "PA_ERR_CUDA"}
 PA_F32, PA_F16, PA_BF16, PA_FP8_E4M3 = 0, 1, 2, 3
 PA_DEV_BAD_SLOT, PA_DEV_BAD_BLOCK, PA_DEV_WAIT_TIMEOUT, PA_DEV_BAD_CONTEXT = 1, 2, 4, 8
+PA_DEV_BAD_PIECES = 16
 
 _TORCH_DT = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16,
              torch.float8_e4m3fn: PA_FP8_E4M3, torch.uint8: PA_FP8_E4M3}

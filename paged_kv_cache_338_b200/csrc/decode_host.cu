@@ -92,7 +92,8 @@ cudaError_t launch_merge_q(const dec::Params& p, int D, int wph, dim3 grid, cuda
 cudaError_t launch_merge(const dec::Params& p, pa_dtype qt, int D, int Hq, int S,
                          cudaStream_t st) {
     int wph = 1;
-    while (wph < dec::kMergeWarps && p.max_parts > 8 * wph) wph *= 2;
+    if (p.balanced) wph = 2;     // pieces per item: about (item blocks / CTA range) + 1
+    else while (wph < dec::kMergeWarps && p.max_parts > 8 * wph) wph *= 2;
     const int hpc = dec::kMergeWarps / wph;
     const dim3 grid((unsigned)((Hq + hpc - 1) / hpc), (unsigned)S);
     switch (qt) {
@@ -115,12 +116,34 @@ bool is_pow2_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8 || g == 
 
 using namespace pa;
 
+// Balanced mode layout: [items] int2 (first, last CTA), 16-byte aligned, then
+// [pieces * gc] float2 (m, l), then [pieces * gc * D] float (o), with
+// items = S * HC, pieces = items + kMaxBalancedCtas, items * gc = S * Hq.
+static size_t align16(size_t x) { return (x + 15) & ~size_t(15); }
+
+static size_t balanced_bytes(int S, int Hq, int D, int gc) {
+    const size_t items = (size_t)S * (Hq / gc);
+    const size_t rows = (items + dec::kMaxBalancedCtas) * gc;
+    return align16(items * sizeof(int2)) + align16(rows * sizeof(float2)) + rows * sizeof(float) * D;
+}
+
 extern "C" pa_status pa_decode_workspace_size(int S, int Hq, int D, int max_ctx, int partition,
                                               size_t* bytes) {
     clear_error();
     if (!bytes) return fail(PA_ERR_INVALID_ARG, "bytes is NULL");
-    if (S < 0 || Hq <= 0 || D <= 0 || max_ctx < 0 || partition < 0)
+    if (S < 0 || Hq <= 0 || D <= 0 || max_ctx < 0 || partition < PA_PARTITION_BALANCED)
         return fail(PA_ERR_INVALID_ARG, "negative or zero size");
+    if (partition == PA_PARTITION_BALANCED) {
+        *bytes = balanced_bytes(S, Hq, D, 1 > Hq ? Hq : 1) > balanced_bytes(S, Hq, D, Hq)
+                     ? balanced_bytes(S, Hq, D, 1)
+                     : balanced_bytes(S, Hq, D, Hq);
+        // the bound over every heads-per-item value (gc divides Hq, gc <= 16)
+        size_t mx = 0;
+        for (int gc = 1; gc <= 16 && gc <= Hq; gc *= 2)
+            if (Hq % gc == 0 && balanced_bytes(S, Hq, D, gc) > mx) mx = balanced_bytes(S, Hq, D, gc);
+        *bytes = mx;
+        return PA_OK;
+    }
     const int64_t mp = parts_for(max_ctx, partition);
     *bytes = mp <= 1 ? 0 : (size_t)S * Hq * mp * (sizeof(float) * 2 + sizeof(float) * D);
     return PA_OK;
@@ -167,12 +190,15 @@ extern "C" pa_status pa_decode(void* out, const void* q, pa_dtype q_dt, const vo
                                void* workspace, size_t workspace_bytes, pa_stream_t stream) {
     clear_error();
     if (!valid_dtype(q_dt) || !valid_dtype(cache_dt)) return fail(PA_ERR_INVALID_ARG, "bad dtype");
-    if (S < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || MB < 0 || NB <= 0 || max_ctx < 0 || partition < 0)
+    if (S < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || MB < 0 || NB <= 0 || max_ctx < 0 ||
+        partition < PA_PARTITION_BALANCED)
         return fail(PA_ERR_INVALID_ARG, "negative or zero size");
     if (Hq % Hkv) return fail(PA_ERR_INVALID_ARG, "Hq (%d) is not a multiple of Hkv (%d)", Hq, Hkv);
     if (!(bs == 8 || bs == 16 || bs == 32))
         return fail(PA_ERR_UNSUPPORTED, "block size %d (supported: 8, 16, 32)", bs);
-    if (partition % bs) return fail(PA_ERR_INVALID_ARG, "partition %d is not a multiple of bs", partition);
+    const bool balanced = partition == PA_PARTITION_BALANCED;
+    if (!balanced && partition % bs)
+        return fail(PA_ERR_INVALID_ARG, "partition %d is not a multiple of bs", partition);
     if (NB > 0x7fffffffLL) return fail(PA_ERR_INVALID_ARG, "NB exceeds int32 block ids");
     if (!(std::isfinite(scale)) || !(std::isfinite(k_scale) && k_scale > 0) ||
         !(std::isfinite(v_scale) && v_scale > 0))
@@ -195,11 +221,16 @@ extern "C" pa_status pa_decode(void* out, const void* q, pa_dtype q_dt, const vo
         return fail(PA_ERR_INVALID_ARG, "caches, q and out must be 16-byte aligned");
     if (MB == 0 && max_ctx > 0) return fail(PA_ERR_INVALID_ARG, "MB == 0 with max_ctx > 0");
 
-    const int64_t max_parts = parts_for(max_ctx, partition);
+    const int64_t max_parts = balanced ? 1 : parts_for(max_ctx, partition);
     if (max_parts > 65535 || (int64_t)Hkv * G > 65535)
         return fail(PA_ERR_UNSUPPORTED, "too many partitions or heads for the grid");
+    const int sel = g_select.load();
+    const bool use_mma = !(sel & 1) && G >= 2 && D <= 128 && cache_dt != PA_F32;
+    const int gc_simt = G < (D == 256 ? 2 : 4) ? G : (D == 256 ? 2 : 4);
+    const int gc = use_mma ? G : gc_simt;
     size_t need = 0;
-    pa_decode_workspace_size(S, Hq, D, max_ctx, partition, &need);
+    if (balanced) need = balanced_bytes(S, Hq, D, gc);
+    else pa_decode_workspace_size(S, Hq, D, max_ctx, partition, &need);
     if (need && (!workspace || workspace_bytes < need || !aligned16(workspace)))
         return fail(PA_ERR_INVALID_ARG, "workspace needs %zu bytes, 16-byte aligned (got %zu)",
                     need, workspace_bytes);
@@ -226,13 +257,24 @@ extern "C" pa_status pa_decode(void* out, const void* q, pa_dtype q_dt, const vo
     p.part_blocks = max_parts > 1 ? partition / bs : 0;
     p.part_tokens = max_parts > 1 ? partition : 0;
     p.max_ctx = max_ctx;
-    const int sel = g_select.load();
     p.evict_first = (sel & 2) ? 1 : 0;
     p.heads_fastest = (sel & 4) ? 1 : 0;
     p.NB = NB;
     p.qk_scale = (float)((double)scale * (double)k_scale * 1.4426950408889634);
     p.v_scale = v_scale;
-    if (max_parts > 1) {
+    p.bs = bs;
+    p.gc = gc;
+    p.balanced = balanced ? 1 : 0;
+    if (balanced) {
+        const size_t items = (size_t)S * (Hq / gc);
+        const size_t rows = (items + dec::kMaxBalancedCtas) * gc;
+        char* w = static_cast<char*>(workspace);
+        p.ws_item = reinterpret_cast<int2*>(w);
+        p.ws_rows = (int64_t)rows;
+        p.ws_ml = reinterpret_cast<float2*>(w + align16(items * sizeof(int2)));
+        p.ws_o = reinterpret_cast<float*>(w + align16(items * sizeof(int2)) +
+                                          align16(rows * sizeof(float2)));
+    } else if (max_parts > 1) {
         p.ws_ml = static_cast<float2*>(workspace);
         p.ws_o = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                           sizeof(float2) * (size_t)S * Hq * max_parts);
@@ -240,9 +282,18 @@ extern "C" pa_status pa_decode(void* out, const void* q, pa_dtype q_dt, const vo
 
     L.bs = bs;
     L.D = D;
-    L.mma = !(sel & 1) && G >= 2 && D <= 128 && cache_dt != PA_F32;
+    L.mma = use_mma;
     L.mrows = G <= 8 ? 8 : 16;
-    L.gc = G < (D == 256 ? 2 : 4) ? G : (D == 256 ? 2 : 4);
+    L.gc = gc_simt;
+    L.balanced = balanced;
+    if (balanced) {
+        static int sms[256] = {};
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (dev >= 0 && dev < 256 && !sms[dev])
+            cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+        L.num_sms = (dev >= 0 && dev < 256 && sms[dev] > 0) ? sms[dev] : 148;
+    }
     const int chunks = L.mma ? 1 : G / L.gc;
     L.grid = p.heads_fastest ? dim3((unsigned)(Hkv * chunks), (unsigned)max_parts, (unsigned)S)
                              : dim3((unsigned)max_parts, (unsigned)(Hkv * chunks), (unsigned)S);
@@ -257,7 +308,7 @@ extern "C" pa_status pa_decode(void* out, const void* q, pa_dtype q_dt, const vo
     }
     if (e == cudaErrorNotSupported) return fail(PA_ERR_UNSUPPORTED, "no kernel for this shape");
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
-    if (max_parts > 1) {
+    if (max_parts > 1 || balanced) {
         e = launch_merge(p, q_dt, D, Hq, S, L.stream);
         if (e != cudaSuccess) return cuda_fail(e, "split-K merge launch");
     }

@@ -58,10 +58,20 @@ struct Params {
     int max_ctx;                 // upper bound the grid / workspace were sized for
     int evict_first;             // 1: stream K/V with an L2 evict-first hint
     int heads_fastest;           // grid order: 1 = (kv head, partition, seq), 0 = (partition, kv head, seq)
+    int bs;                      // block size (tokens)
+    int balanced;                // 1: persistent work-balanced grid (decode_balanced)
+    int2* ws_item;               // balanced: per item (first CTA, last CTA) holding its pieces
+    int gc;                      // query heads per CTA item (G for the tensor-core consumer)
+    int64_t ws_rows;             // balanced: partial rows the workspace holds
     int64_t NB;
     float qk_scale;              // scale * k_scale * log2(e)
     float v_scale;
 };
+
+// Record a wait that gave up, with the site that gave up (bits 16-23).
+__device__ __forceinline__ void wait_timeout(const Params& p, unsigned site) {
+    dev::raise_error(p.err, PA_DEV_WAIT_TIMEOUT | (site << 16));
+}
 
 // Context length of sequence s, clamped to what the grid, the workspace and
 // the table row can hold; anything out of range is reported, never followed.
@@ -137,10 +147,12 @@ template <class C>
 __device__ __forceinline__ void produce(const CUtensorMap* tmk, const CUtensorMap* tmv,
                                         const Params& p, const int32_t* bt_row, int blk0, int nblk,
                                         int kvh, uint8_t* stages, uint32_t full0, uint32_t empty0,
-                                        volatile int* s_abort, int* issued_out) {
+                                        volatile int* s_abort, int* k_io) {
+    // Streams blocks [blk0, blk0 + nblk) of one (sequence, kv head) through the
+    // stage ring; *k_io is the CTA's running block counter (stage = k % STAGES).
     const int lane = threadIdx.x & 31;
     const uint64_t pol = p.evict_first ? dev::policy_evict_first() : dev::policy_evict_normal();
-    int issued = 0;
+    int k = *k_io;
     for (int jb = 0; jb < nblk; jb += 32) {
         const int mine = (jb + lane < nblk) ? __ldg(bt_row + blk0 + jb + lane) : 0;
         const int cnt = min(32, nblk - jb);
@@ -148,12 +160,11 @@ __device__ __forceinline__ void produce(const CUtensorMap* tmk, const CUtensorMa
             const int id = __shfl_sync(0xffffffffu, mine, jj);
             int stop = 0;
             if (lane == 0) {
-                const int j = jb + jj;
-                const int st = j % C::STAGES;
-                if (j >= C::STAGES) {
-                    const uint32_t par = ((j / C::STAGES) & 1) ^ 1;
+                const int st = k % C::STAGES;
+                if (k >= C::STAGES) {
+                    const uint32_t par = ((k / C::STAGES) & 1) ^ 1;
                     if (!dev::mbar_wait_bounded(empty0 + 8 * st, par)) {
-                        dev::raise_error(p.err, PA_DEV_WAIT_TIMEOUT);
+                        wait_timeout(p, 1);
                         *s_abort = 1;
                         stop = 1;
                     }
@@ -164,22 +175,22 @@ __device__ __forceinline__ void produce(const CUtensorMap* tmk, const CUtensorMa
                     const uint32_t dk = dev::smem_addr(stages + (size_t)st * C::STAGE);
                     dev::mbar_arrive_expect_tx(bar, C::STAGE);
                     #pragma unroll
-                    for (int k = 0; k < C::CH; ++k) {
-                        dev::tma_load_4d(dk + k * C::BS * 128, tmk, bar, k * C::EPS, kvh, 0, id, pol);
-                        dev::tma_load_4d(dk + C::TILE + k * C::BS * 128, tmv, bar, k * C::EPS, kvh,
+                    for (int c = 0; c < C::CH; ++c) {
+                        dev::tma_load_4d(dk + c * C::BS * 128, tmk, bar, c * C::EPS, kvh, 0, id, pol);
+                        dev::tma_load_4d(dk + C::TILE + c * C::BS * 128, tmv, bar, c * C::EPS, kvh,
                                          0, id, pol);
                     }
-                    ++issued;
                 }
             }
             stop = __shfl_sync(0xffffffffu, stop, 0);
             if (stop) {
-                if (lane == 0) *issued_out = issued;
+                *k_io = k;
                 return;
             }
+            ++k;
         }
     }
-    if (lane == 0) *issued_out = issued;
+    *k_io = k;
 }
 
 // --------------------------------------------------------- SIMT consumer
@@ -767,15 +778,17 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     using State = typename std::conditional<C::MMA, MmaState<C>, SimtState<C>>::type;
     State st;
     if (warp == C::NW) {
+        int k = 0;
         produce<C>(&tmk, &tmv, p, p.block_tables + (size_t)s * p.MB, blk0, nblk, kvh, stages,
-                   full0, empty0, &s_abort, &s_issued);
+                   full0, empty0, &s_abort, &k);
+        if (lane == 0) s_issued = k;
     } else {
         if constexpr (C::MMA) mma_load_q<C>(st, p, s, h0, G);
         else simt_load_q<C>(st, p, s, h0);
         for (int j = warp; j < nblk; j += C::NW) {
             const int stg = j % C::STAGES;
             if (!dev::mbar_wait_bounded(full0 + 8 * stg, (j / C::STAGES) & 1)) {
-                if (lane == 0) { dev::raise_error(p.err, PA_DEV_WAIT_TIMEOUT); s_abort = 1; }
+                if (lane == 0) { wait_timeout(p, 2); s_abort = 1; }
                 break;
             }
             uint8_t* kt = stages + (size_t)stg * C::STAGE;
@@ -833,6 +846,289 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     }
 }
 
+// ------------------------------------------------------ balanced kernel
+// Persistent, work-balanced variant ("stream-K").  Items are (sequence, kv
+// head [, head chunk]) pairs, laid end to end in one global block space of W
+// blocks (item i = s * HC + hc holds ceil(n_s / bs) blocks).  CTA c of a
+// grid sized to the GPU's resident capacity takes blocks [c*W/grid,
+// (c+1)*W/grid): equal work to one block, no atomics, no per-call state.
+// Its producer walks that range item by item without draining the stage ring
+// between items, and publishes each piece (the part of one item inside the
+// range) through a small ring of descriptors.  Consumers finish a piece with
+// a two-phase rendezvous on mbarriers (bounded waits): a piece that is a whole
+// item is written out directly; a piece of a split item is written as a
+// partial at row (item + c) * gc + g, and the item's first / last piece record
+// which CTAs hold it, for decode_merge.
+constexpr int kItemQ = 4;
+
+struct PieceDesc {
+    int s, hc, off, take, nblk, n, k0, end;
+};
+
+template <class C>
+struct BalancedSmem {
+    static constexpr int COMB_FLOATS = C::NW * C::GC * (C::D + 2);
+    static constexpr int STAGES_RAW =
+        (100 * 1024 - C::NW * C::VSTG - COMB_FLOATS * 4) / C::STAGE;   // 2 CTAs per SM fit
+    // a multiple of NW: each stage has a single consumer warp (see Cfg)
+    static constexpr int STAGES_CLAMPED = STAGES_RAW < C::NW ? C::NW : (STAGES_RAW > 32 ? 32 : STAGES_RAW);
+    static constexpr int STAGES = STAGES_CLAMPED / C::NW * C::NW;
+    static_assert(STAGES % C::NW == 0, "each stage must have a single consumer warp");
+    static constexpr size_t BYTES = 1024 + size_t(STAGES) * C::STAGE + size_t(C::NW) * C::VSTG +
+                                    size_t(COMB_FLOATS) * 4 + 8 * (2 * STAGES + 2 * kItemQ + 2);
+    static_assert(BYTES <= 227 * 1024, "shared memory");
+};
+
+template <class C>
+__device__ __forceinline__ int blocks_of(const Params& p, int s) {
+    return (checked_len(p, s, C::BS) + C::BS - 1) / C::BS;
+}
+
+// The configuration of the balanced kernel: the same tile shapes, a deeper ring.
+template <class C>
+struct Balanced : C {
+    static constexpr int STAGES = BalancedSmem<C>::STAGES;
+};
+
+template <class C0>
+__global__ void __launch_bounds__(C0::THREADS, 2)
+decode_balanced(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                const Params p) {
+    using B = BalancedSmem<C0>;
+    using C = Balanced<C0>;
+    constexpr int STAGES = B::STAGES;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ int s_abort, s_issued, s_found, s_s0, s_hc0, s_off0;
+    __shared__ long long s_red[C::NW + 1];
+    __shared__ PieceDesc s_ring[kItemQ];
+    uint8_t* stages = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* vstage = stages + (size_t)STAGES * C::STAGE;
+    float* comb = reinterpret_cast<float*>(vstage + (size_t)C::NW * C::VSTG);
+    const uint32_t full0 = dev::smem_addr(comb + B::COMB_FLOATS);
+    const uint32_t empty0 = full0 + 8 * STAGES;
+    const uint32_t ifull0 = empty0 + 8 * STAGES;
+    const uint32_t iempty0 = ifull0 + 8 * kItemQ;
+    const uint32_t rdv_pub = iempty0 + 8 * kItemQ;     // consumers published their states
+    const uint32_t rdv_done = rdv_pub + 8;              // consumers finished the combine
+
+    const int G = p.Hq / p.Hkv;
+    const int gc = C::MMA ? G : C::GC;
+    const int chunks = G / gc;
+    const int HC = p.Hkv * chunks;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // ---- W and this CTA's block range --------------------------------------
+    long long acc = 0;
+    for (int s = threadIdx.x; s < p.S; s += C::THREADS) acc += (long long)blocks_of<C>(p, s) * HC;
+    #pragma unroll
+    for (int x = 16; x > 0; x >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, x);
+    if (lane == 0) s_red[warp] = acc;
+    if (threadIdx.x == 0) s_found = 0;
+    __syncthreads();
+    long long W = 0;
+    #pragma unroll
+    for (int w = 0; w <= C::NW; ++w) W += s_red[w];
+    // With fewer blocks than CTAs only the first W CTAs work, so every working
+    // CTA's share is non-empty and an item's pieces sit on consecutive CTAs.
+    const long long nctas = W < (long long)gridDim.x ? W : (long long)gridDim.x;
+    if ((long long)blockIdx.x >= nctas) return;         // CTA-uniform: no work
+    const long long b0 = (long long)blockIdx.x * W / nctas;
+    const long long b1 = ((long long)blockIdx.x + 1) * W / nctas;
+    __syncthreads();                                    // s_red is reused below
+    long long R = 0;
+    for (int base = 0; base < p.S; base += C::THREADS) {
+        const int s = base + threadIdx.x;
+        const int nb = s < p.S ? blocks_of<C>(p, s) : 0;
+        const long long v = (long long)nb * HC;
+        long long inc = v;
+        #pragma unroll
+        for (int x = 1; x < 32; x <<= 1) {
+            const long long y = __shfl_up_sync(0xffffffffu, inc, x);
+            if (lane >= x) inc += y;
+        }
+        if (lane == 31) s_red[warp] = inc;
+        __syncthreads();
+        long long woff = 0, tile = 0;
+        #pragma unroll
+        for (int w = 0; w <= C::NW; ++w) {
+            if (w < warp) woff += s_red[w];
+            tile += s_red[w];
+        }
+        const long long ex = R + woff + inc - v;
+        if (v > 0 && ex <= b0 && b0 < ex + v) {
+            const long long rel = b0 - ex;
+            s_s0 = s;
+            s_hc0 = (int)(rel / nb);
+            s_off0 = (int)(rel % nb);
+            s_found = 1;
+        }
+        R += tile;
+        __syncthreads();
+        if (s_found || R > b0) break;                  // CTA-uniform
+    }
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES; ++i) {
+            dev::mbar_init(full0 + 8 * i, 1);
+            dev::mbar_init(empty0 + 8 * i, 1);
+        }
+        for (int i = 0; i < kItemQ; ++i) {
+            dev::mbar_init(ifull0 + 8 * i, 1);
+            dev::mbar_init(iempty0 + 8 * i, C::NW);
+        }
+        dev::mbar_init(rdv_pub, C::NW);
+        dev::mbar_init(rdv_done, C::NW);
+        dev::fence_mbar_init();
+        s_abort = 0;
+        s_issued = 0;
+    }
+    if (warp == C::NW && lane == 0) {
+        dev::prefetch_tensormap(&tmk);
+        dev::prefetch_tensormap(&tmv);
+    }
+    __syncthreads();
+
+    using State = typename std::conditional<C::MMA, MmaState<C>, SimtState<C>>::type;
+    State st;
+    if (warp == C::NW) {
+        // ---------------------------------------------------------- producer
+        int s = s_s0, hc = s_hc0, off = s_off0, k = 0, ci = 0;
+        long long b = b0;
+        bool stop = !s_found;
+        auto publish = [&](const PieceDesc& d) {
+            int bad = 0;
+            if (lane == 0) {
+                const int slot = ci % kItemQ;
+                if (ci >= kItemQ &&
+                    !dev::mbar_wait_bounded(iempty0 + 8 * slot, ((ci / kItemQ) & 1) ^ 1)) {
+                    wait_timeout(p, 3);
+                    s_abort = 1;
+                    bad = 1;
+                } else {
+                    s_ring[slot] = d;
+                    dev::mbar_arrive(ifull0 + 8 * slot);
+                }
+            }
+            return __shfl_sync(0xffffffffu, bad, 0) != 0;
+        };
+        while (!stop && b < b1 && s < p.S) {
+            const int n = checked_len(p, s, C::BS);
+            const int nb = (n + C::BS - 1) / C::BS;
+            if (nb > off) {
+                const int take = (int)min((long long)(nb - off), b1 - b);
+                PieceDesc d{s, hc, off, take, nb, n, k, 0};
+                if (publish(d)) break;
+                produce<C>(&tmk, &tmv, p, p.block_tables + (size_t)s * p.MB, off, take,
+                            hc / chunks, stages, full0, empty0, &s_abort, &k);
+                if (*(volatile int*)&s_abort) break;
+                b += take;
+                ++ci;
+            }
+            off = 0;
+            if (++hc == HC) { hc = 0; ++s; }
+        }
+        if (!*(volatile int*)&s_abort) {
+            PieceDesc d{0, 0, 0, 0, 0, 0, k, 1};
+            publish(d);
+        }
+        if (lane == 0) s_issued = k;
+    } else {
+        // --------------------------------------------------------- consumers
+        float* cm = comb;
+        float* cl = cm + C::NW * C::GC;
+        float* co = cl + C::NW * C::GC;
+        for (int ci = 0;; ++ci) {
+            const int slot = ci % kItemQ;
+            if (!dev::mbar_wait_bounded(ifull0 + 8 * slot, (ci / kItemQ) & 1)) {
+                if (lane == 0) { wait_timeout(p, 4); s_abort = 1; }
+                break;
+            }
+            const PieceDesc d = s_ring[slot];
+            if (d.end) break;
+            const int h0 = (d.hc / chunks) * G + (d.hc % chunks) * gc;
+            if constexpr (C::MMA) mma_load_q<C>(st, p, d.s, h0, G);
+            else simt_load_q<C>(st, p, d.s, h0);
+            unsigned bad = 0;
+            // block k goes to warp k % NW (not by its place in the piece), so a
+            // stage, used by blocks k = stage (mod STAGES), keeps a single consumer
+            const int jj0 = ((warp - d.k0) % C::NW + C::NW) % C::NW;
+            for (int jj = jj0; jj < d.take; jj += C::NW) {
+                const int k = d.k0 + jj;
+                const int stg = k % STAGES;
+                if (!dev::mbar_wait_bounded(full0 + 8 * stg, (k / STAGES) & 1)) { bad = 2; break; }
+                uint8_t* kt = stages + (size_t)stg * C::STAGE;
+                const int nvalid = min(C::BS, d.n - (d.off + jj) * C::BS);
+                if constexpr (C::MMA)
+                    mma_block<C>(st, kt, kt + C::TILE, vstage + warp * C::VSTG, nvalid, p.qk_scale);
+                else simt_block<C>(st, kt, kt + C::TILE, nvalid);
+                __syncwarp();
+                if (lane == 0) dev::mbar_arrive(empty0 + 8 * stg);
+            }
+            if (!bad) {
+                if constexpr (C::MMA) mma_publish<C>(st, cm, cl, co, warp, G);
+                else simt_publish<C>(st, cm, cl, co, warp);
+                __syncwarp();
+                if (lane == 0) dev::mbar_arrive(rdv_pub);
+                if (!dev::mbar_wait_bounded(rdv_pub, ci & 1)) bad = 5;
+            }
+            if (bad) {
+                if (lane == 0) { wait_timeout(p, bad); s_abort = 1; }
+                break;
+            }
+            // ---- combine the four warps' states for this piece -----------
+            const int item = d.s * HC + d.hc;
+            const bool first = d.off == 0, last = d.off + d.take == d.nblk;
+            const int piece = item + blockIdx.x;
+            for (int idx = threadIdx.x; idx < gc * C::D; idx += C::NW * 32) {
+                const int g = idx / C::D, dd = idx % C::D;
+                float M = -INFINITY;
+                #pragma unroll
+                for (int w = 0; w < C::NW; ++w) M = fmaxf(M, cm[w * C::GC + g]);
+                float L = 0.f, O = 0.f;
+                if (M != -INFINITY) {
+                    #pragma unroll
+                    for (int w = 0; w < C::NW; ++w) {
+                        const float f = exp2f(cm[w * C::GC + g] - M);
+                        L = fmaf(f, cl[w * C::GC + g], L);
+                        O = fmaf(f, co[(w * C::GC + g) * C::D + dd], O);
+                    }
+                }
+                if (first && last) {
+                    dev::store_out<C::QT>(p.out, ((size_t)d.s * p.Hq + h0 + g) * C::D + dd,
+                                          L > 0.f ? (O / L) * p.v_scale : 0.f);
+                } else {
+                    const size_t row = (size_t)piece * gc + g;
+                    if ((int64_t)row < p.ws_rows) {
+                        p.ws_o[row * C::D + dd] = O * p.v_scale;
+                        if (dd == 0) p.ws_ml[row] = make_float2(M, L);
+                    } else if (dd == 0) {
+                        dev::raise_error(p.err, PA_DEV_BAD_PIECES);
+                    }
+                }
+            }
+            if (threadIdx.x == 0) {
+                if (first) p.ws_item[item].x = blockIdx.x;
+                if (last) p.ws_item[item].y = blockIdx.x;
+            }
+            __syncwarp();
+            if (lane == 0) dev::mbar_arrive(rdv_done);
+            if (!dev::mbar_wait_bounded(rdv_done, ci & 1)) {
+                if (lane == 0) { wait_timeout(p, 6); s_abort = 1; }
+                break;
+            }
+            if (lane == 0) dev::mbar_arrive(iempty0 + 8 * slot);
+        }
+    }
+    __syncthreads();
+    dev::launch_dependents();
+    if (s_abort && warp == C::NW && lane == 0) {
+        const int issued = s_issued;
+        for (int j = max(0, issued - STAGES); j < issued; ++j)
+            dev::mbar_wait_bounded(full0 + 8 * (j % STAGES), (j / STAGES) & 1);
+    }
+}
+
 // Merge split-K partials: out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p.
 // A CTA of 8 warps serves 8 / wph query heads of one sequence; the wph warps
 // of a head split its partitions, and each lane holds D/32 dims, so every
@@ -846,21 +1142,53 @@ __global__ void __launch_bounds__(kMergeWarps * 32) decode_merge(const Params p,
     __shared__ float s_max[kMergeWarps];
     __shared__ float s_l[kMergeWarps];
     __shared__ __align__(16) float s_o[kMergeWarps][D];
+    __shared__ int s_live[kMergeWarps];
     dev::grid_dependency_wait();
     const int hpc = kMergeWarps / wph;                // heads per CTA
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int hl = warp / wph, sub = warp % wph;
     const int h = blockIdx.x * hpc + hl, s = blockIdx.y;
+    const bool head_ok = h < p.Hq;
     int n = p.context_lens[s];
-    n = max(0, min(n, min(p.max_ctx, p.MB * (p.part_tokens / p.part_blocks))));
-    const int nparts = min(p.max_parts, (n + p.part_tokens - 1) / p.part_tokens);
-    if (nparts <= 1) return;                          // written by the partition kernel
-    const bool live = h < p.Hq;
-    const size_t row0 = ((size_t)s * p.Hq + (live ? h : 0)) * p.max_parts;
+    n = max(0, min(n, min(p.max_ctx, p.MB * p.bs)));
+    // pieces of this head: count and first row (rows of consecutive pieces
+    // are `stride` apart)
+    int count = 0;
+    size_t row0 = 0, stride = 1;
+    if (p.balanced) {
+        if (n == 0) {                                 // no CTA saw this sequence
+            for (int idx = threadIdx.x; idx < hpc * D; idx += blockDim.x) {
+                const int head = blockIdx.x * hpc + idx / D;
+                if (head < p.Hq) dev::store_out<QT>(p.out, ((size_t)s * p.Hq + head) * D + idx % D, 0.f);
+            }
+            return;                                   // CTA-uniform
+        }
+        // piece c of item i sits at row (i + c) * gc + g, for c in [first CTA, last CTA]
+        const int gc = p.gc;
+        const int HC = p.Hq / gc;
+        const int item = s * HC + (head_ok ? h : 0) / gc;
+        const int2 fl = p.ws_item[item];
+        count = fl.y - fl.x + 1;
+        const bool sane = fl.x >= 0 && count >= 1 &&
+                          (int64_t)(item + fl.y + 1) * gc <= p.ws_rows;
+        if (!sane) {                                  // never follow a bad record
+            if (head_ok && sub == 0 && lane == 0) dev::raise_error(p.err, PA_DEV_BAD_PIECES);
+            count = 0;
+        }
+        row0 = sane ? (size_t)(item + fl.x) * gc + (head_ok ? h : 0) % gc : 0;
+        stride = (size_t)gc;
+    } else {
+        count = min(p.max_parts, (n + p.part_tokens - 1) / p.part_tokens);
+        if (count <= 1) return;                       // CTA-uniform: written by the partition kernel
+        row0 = ((size_t)s * p.Hq + (head_ok ? h : 0)) * p.max_parts;
+        stride = 1;
+    }
+    const bool live = head_ok && count > 1;           // count <= 1: written by the partition kernel
+    if (sub == 0) s_live[hl] = live ? 1 : 0;
 
     float mx = -INFINITY;
     if (live)
-        for (int i = sub * 32 + lane; i < nparts; i += wph * 32) mx = fmaxf(mx, p.ws_ml[row0 + i].x);
+        for (int i = sub * 32 + lane; i < count; i += wph * 32) mx = fmaxf(mx, p.ws_ml[row0 + i * stride].x);
     #pragma unroll
     for (int x = 16; x > 0; x >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, x));
     if (lane == 0) s_max[warp] = mx;
@@ -873,11 +1201,12 @@ __global__ void __launch_bounds__(kMergeWarps * 32) decode_merge(const Params p,
     for (int k = 0; k < DL; ++k) o[k] = 0.f;
     if (live) {
         #pragma unroll 4
-        for (int i = sub; i < nparts; i += wph) {
-            const float2 ml = p.ws_ml[row0 + i];
+        for (int i = sub; i < count; i += wph) {
+            const size_t row = row0 + i * stride;
+            const float2 ml = p.ws_ml[row];
             const float f = exp2f(ml.x - M);
             L = fmaf(f, ml.y, L);
-            const float* src = p.ws_o + (row0 + i) * D + lane * DL;
+            const float* src = p.ws_o + row * D + lane * DL;
             if constexpr (DL % 4 == 0) {
                 #pragma unroll
                 for (int k = 0; k < DL; k += 4) {
@@ -898,7 +1227,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32) decode_merge(const Params p,
     for (int idx = threadIdx.x; idx < hpc * D; idx += blockDim.x) {
         const int hh = idx / D, d = idx % D;
         const int head = blockIdx.x * hpc + hh;
-        if (head >= p.Hq) continue;
+        if (head >= p.Hq || !s_live[hh]) continue;   // not split: already written
         float Lt = 0.f, Ot = 0.f;
         for (int w = hh * wph; w < (hh + 1) * wph; ++w) {
             Lt += s_l[w];

@@ -19,7 +19,11 @@ struct Launch {
     int mrows;     // MMA: 8 or 16 query rows
     dim3 grid;
     cudaStream_t stream;
+    bool balanced; // persistent work-balanced kernel (grid computed at launch)
+    int num_sms;
 };
+
+constexpr int kMaxBalancedCtas = 1024;   // the workspace layout assumes at most this many
 
 // cudaErrorNotSupported when no kernel is built for the combination.
 cudaError_t launch_f32(const Launch& L);
@@ -30,6 +34,20 @@ cudaError_t launch_fp8_q_bf16(const Launch& L);
 
 template <class C>
 cudaError_t launch_one(const Launch& L) {
+    if (L.balanced) {
+        auto kern = decode_balanced<C>;
+        const int smem = static_cast<int>(BalancedSmem<C>::BYTES);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        int per_sm = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, C::THREADS, smem);
+        if (e != cudaSuccess) return e;
+        if (per_sm < 1) per_sm = 1;
+        int ctas = per_sm * L.num_sms;
+        if (ctas > kMaxBalancedCtas) ctas = kMaxBalancedCtas;
+        kern<<<dim3((unsigned)ctas), C::THREADS, smem, L.stream>>>(L.tmk, L.tmv, L.p);
+        return cudaGetLastError();
+    }
     auto kern = decode_partition<C>;
     // opt in to > 48 KB of dynamic shared memory (idempotent, cheap)
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,

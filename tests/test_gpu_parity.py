@@ -101,12 +101,13 @@ SMALL = [
 
 
 @pytest.mark.parametrize("name,cfg", SMALL, ids=[n for n, _ in SMALL])
-@pytest.mark.parametrize("partition_blocks", [0, 2, 7])
+@pytest.mark.parametrize("partition_blocks", [0, 2, 7, -1], ids=["single", "p2", "p7", "balanced"])
 @pytest.mark.parametrize("mode", MODES, ids=["auto", "simt", "evict_first", "head_major"])
 def test_step_parity_small(name, cfg, partition_blocks, mode):
     inp = wl.make_decode_inputs(cfg, seed=101)
     want, kc_o, vc_o = oracle_step(inp)
-    out, kc, vc = gpu_step(inp, partition_blocks * cfg.block_size, mode)
+    part = -1 if partition_blocks < 0 else partition_blocks * cfg.block_size
+    out, kc, vc = gpu_step(inp, part, mode)
     assert _bits_equal(kc, kc_o, cfg.kv_dtype) and _bits_equal(vc, vc_o, cfg.kv_dtype)
     _check_out(out, want, cfg.kv_dtype, f"{name} P={partition_blocks} mode={mode}")
     assert pa.pa_device_status() == 0
@@ -126,7 +127,7 @@ def test_decode_shapes(bs, G, D, dt):
                           3 * bs + 1, fp8_scaled=dt == "fp8_e4m3")
     inp = wl.make_decode_inputs(cfg, seed=bs * 1000 + G * 10 + D)
     want, _, _ = oracle_step(inp)
-    for part in (0, bs):
+    for part in (0, bs, -1):
         for mode in BOTH:
             out, _, _ = gpu_step(inp, part, mode)
             _check_out(out, want, dt, f"P={part} mode={mode}")
@@ -142,15 +143,16 @@ def test_lengths_at_partition_edges(dt):
     inp = wl.make_decode_inputs(cfg, seed=7)
     want, _, _ = oracle_step(inp)
     for mode in BOTH:
-        out, _, _ = gpu_step(inp, P, mode)
-        _check_out(out, want, dt, f"mode={mode}")
+        for part in (P, -1):
+            out, _, _ = gpu_step(inp, part, mode)
+            _check_out(out, want, dt, f"mode={mode} P={part}")
 
 
 def test_zero_length_sequences_give_zero_rows():
     cfg = wl.DecodeConfig("empty", 3, 8, 2, 128, 16, "bf16", "bf16", 0, 0, fixed_lens=(0, 40, 0))
     inp = wl.make_decode_inputs(cfg, seed=3)
     want, _, _ = oracle_step(inp)
-    for part in (0, 16):
+    for part in (0, 16, -1):
         out, _, _ = gpu_step(inp, part)
         assert (out[0] == 0).all() and (out[2] == 0).all()
         _check_out(out, want, "bf16", f"P={part}")
@@ -185,3 +187,30 @@ def test_device_errors_are_reported_not_followed():
                  partition=16, workspace=ws)
     assert pa.pa_device_status() & pa.PA_DEV_BAD_CONTEXT
     assert pa.pa_device_status() == 0
+
+
+@pytest.mark.parametrize("nseq,lo,hi", [(1, 1, 3), (3, 1, 40), (40, 1, 400), (7, 900, 3000)])
+def test_balanced_grid_cuts(nseq, lo, hi):
+    """Persistent balanced decode: fewer blocks than CTAs, items cut across many
+    CTAs, and many small items per CTA all match the oracle."""
+    cfg = wl.DecodeConfig("bal", nseq, 16, 4, 128, 16, "bf16", "bf16", lo, hi)
+    inp = wl.make_decode_inputs(cfg, seed=nseq * 31 + hi)
+    want, _, _ = oracle_step(inp)
+    for mode in BOTH:
+        out, _, _ = gpu_step(inp, -1, mode)
+        _check_out(out, want, "bf16", f"mode={mode}")
+    assert pa.pa_device_status() == 0
+
+
+def test_balanced_many_pieces_per_cta():
+    """Hundreds of short sequences: each persistent CTA walks tens of pieces,
+    wrapping its descriptor ring several times."""
+    cfg = wl.DecodeConfig("ringwrap", 512, 32, 8, 128, 16, "bf16", "bf16", 1, 48)
+    inp = wl.make_decode_inputs(cfg, seed=5)
+    want, _, _ = oracle_step(inp)
+    pa.pa_device_status(clear=True)
+    for mode in BOTH:
+        out, _, _ = gpu_step(inp, -1, mode)
+        bits = pa.pa_device_status()
+        assert bits == 0, f"device status {bits:#x} (mode {mode})"
+        _check_out(out, want, "bf16", f"mode={mode}")
