@@ -286,6 +286,7 @@ extern "C" pa_status pa_decode(void* out, const void* q, pa_dtype q_dt, const vo
     L.mrows = G <= 8 ? 8 : 16;
     L.gc = gc_simt;
     L.balanced = balanced;
+    L.G = G;
     if (balanced) {
         static int sms[256] = {};
         int dev = 0;

@@ -293,7 +293,7 @@ __device__ __forceinline__ void simt_block(SimtState<C>& st, const uint8_t* ktil
 // Reduce the four token groups of the warp and publish (m, l, acc) to smem.
 template <class C>
 __device__ __forceinline__ void simt_publish(SimtState<C>& st, float* cm, float* cl, float* co,
-                                             int w) {
+                                             int w, int gs = C::GC) {
     const int lane = threadIdx.x & 31;
     const int l8 = lane & 7, grp = lane >> 3;
     #pragma unroll
@@ -309,15 +309,15 @@ __device__ __forceinline__ void simt_publish(SimtState<C>& st, float* cm, float*
             st.acc[g][j] = a;
         }
         if (lane == 0) {
-            cm[w * C::GC + g] = st.m[g];
-            cl[w * C::GC + g] = l;
+            cm[w * gs + g] = st.m[g];
+            cl[w * gs + g] = l;
         }
         if (grp == 0) {
             #pragma unroll
             for (int k = 0; k < C::CH; ++k)
                 #pragma unroll
                 for (int e = 0; e < C::EPC; ++e)
-                    co[(w * C::GC + g) * C::D + k * C::EPS + l8 * C::EPC + e] =
+                    co[(w * gs + g) * C::D + k * C::EPS + l8 * C::EPC + e] =
                         st.acc[g][k * C::EPC + e];
         }
     }
@@ -339,13 +339,13 @@ template <int DT>
 __device__ __forceinline__ void mma16816(float* c, uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
     if constexpr (DT == PA_BF16) {
-        asm volatile(
+        asm(
             "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
             "{%8,%9}, {%0,%1,%2,%3};"
             : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
             : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
     } else {
-        asm volatile(
+        asm(
             "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
             "{%8,%9}, {%0,%1,%2,%3};"
             : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
@@ -356,13 +356,13 @@ __device__ __forceinline__ void mma16816(float* c, uint32_t a0, uint32_t a1, uin
 template <int DT>
 __device__ __forceinline__ void mma1688(float* c, uint32_t a0, uint32_t a1, uint32_t b0) {
     if constexpr (DT == PA_BF16) {
-        asm volatile(
+        asm(
             "mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, "
             "{%0,%1,%2,%3};"
             : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
             : "r"(a0), "r"(a1), "r"(b0));
     } else {
-        asm volatile(
+        asm(
             "mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, "
             "{%0,%1,%2,%3};"
             : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
@@ -389,7 +389,7 @@ __device__ __forceinline__ uint32_t pack2(float x, float y, float& rx, float& ry
 
 __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
     uint32_t y;
-    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
     return y;
 }
 
@@ -530,6 +530,11 @@ __device__ __forceinline__ void mma_block(MmaState<C>& st, uint8_t* ktile_p, uin
             for (int i = 0; i < 4; ++i) sc[mt][nh][i] = 0.f;
         if constexpr (S::FP8) {
             // a 16-byte chunk is one 16-dim k-step; ldmatrix rows are 8 tokens
+            float sc8_odd[S::NH][4];
+            #pragma unroll
+            for (int nh = 0; nh < S::NH; ++nh)
+                #pragma unroll
+                for (int i = 0; i < 4; ++i) sc8_odd[nh][i] = 0.f;
             #pragma unroll
             for (int ks = 0; ks < S::KS; ks += 2) {
                 uint32_t r0, r1, r2, r3;
@@ -553,11 +558,22 @@ __device__ __forceinline__ void mma_block(MmaState<C>& st, uint8_t* ktile_p, uin
                 #pragma unroll
                 for (int nh = 0; nh < S::NH; ++nh) {
                     mma16816<CT>(sc[mt][nh], a00, a01, a02, a03, st.qb[nh][ks][0], st.qb[nh][ks][1]);
-                    mma16816<CT>(sc[mt][nh], a10, a11, a12, a13, st.qb[nh][ks + 1][0],
+                    mma16816<CT>(sc8_odd[nh], a10, a11, a12, a13, st.qb[nh][ks + 1][0],
                                  st.qb[nh][ks + 1][1]);
                 }
             }
+            #pragma unroll
+            for (int nh = 0; nh < S::NH; ++nh)
+                #pragma unroll
+                for (int i = 0; i < 4; ++i) sc[mt][nh][i] += sc8_odd[nh][i];
         } else if constexpr (BS >= 16) {
+            // two independent accumulation chains (even / odd k-steps) halve
+            // the dependent mma latency of the product
+            float sc_odd[S::NH][4];
+            #pragma unroll
+            for (int nh = 0; nh < S::NH; ++nh)
+                #pragma unroll
+                for (int i = 0; i < 4; ++i) sc_odd[nh][i] = 0.f;
             #pragma unroll
             for (int ks = 0; ks < S::KS; ++ks) {
                 // matrices: (tok 0-7, chunk 2ks) (tok 8-15, 2ks) (tok 0-7, 2ks+1) (tok 8-15, 2ks+1)
@@ -567,8 +583,13 @@ __device__ __forceinline__ void mma_block(MmaState<C>& st, uint8_t* ktile_p, uin
                         a0, a1, a2, a3);
                 #pragma unroll
                 for (int nh = 0; nh < S::NH; ++nh)
-                    mma16816<CT>(sc[mt][nh], a0, a1, a2, a3, st.qb[nh][ks][0], st.qb[nh][ks][1]);
+                    mma16816<CT>((ks & 1) ? sc_odd[nh] : sc[mt][nh], a0, a1, a2, a3,
+                                 st.qb[nh][ks][0], st.qb[nh][ks][1]);
             }
+            #pragma unroll
+            for (int nh = 0; nh < S::NH; ++nh)
+                #pragma unroll
+                for (int i = 0; i < 4; ++i) sc[mt][nh][i] += sc_odd[nh][i];
         } else {
             // 8 tokens: rows 8-15 of the A operand are zero
             #pragma unroll
@@ -692,7 +713,7 @@ __device__ __forceinline__ void mma_block(MmaState<C>& st, uint8_t* ktile_p, uin
 
 template <class C>
 __device__ __forceinline__ void mma_publish(MmaState<C>& st, float* cm, float* cl, float* co,
-                                            int w, int G) {
+                                            int w, int G, int gs = C::GC) {
     using S = MmaState<C>;
     const int lane = threadIdx.x & 31;
     const int gid = lane >> 2, tig = lane & 3;
@@ -707,13 +728,13 @@ __device__ __forceinline__ void mma_publish(MmaState<C>& st, float* cm, float* c
             const int head = nh * 8 + 2 * tig + j;
             if (head < G) {
                 if (gid == 0) {
-                    cm[w * C::GC + head] = st.m[nh][j];
-                    cl[w * C::GC + head] = l;
+                    cm[w * gs + head] = st.m[nh][j];
+                    cl[w * gs + head] = l;
                 }
                 #pragma unroll
                 for (int md = 0; md < S::MD; ++md) {
-                    co[(w * C::GC + head) * C::D + md * 16 + gid] = st.o[nh][md][j];
-                    co[(w * C::GC + head) * C::D + md * 16 + gid + 8] = st.o[nh][md][2 + j];
+                    co[(w * gs + head) * C::D + md * 16 + gid] = st.o[nh][md][j];
+                    co[(w * gs + head) * C::D + md * 16 + gid + 8] = st.o[nh][md][2 + j];
                 }
             }
         }
@@ -867,16 +888,16 @@ struct PieceDesc {
 
 template <class C>
 struct BalancedSmem {
-    static constexpr int COMB_FLOATS = C::NW * C::GC * (C::D + 2);
-    static constexpr int STAGES_RAW =
-        (100 * 1024 - C::NW * C::VSTG - COMB_FLOATS * 4) / C::STAGE;   // 2 CTAs per SM fit
+    static constexpr int STAGES_RAW = (64 * 1024 - C::NW * C::VSTG) / C::STAGE;  // 3 CTAs per SM fit
     // a multiple of NW: each stage has a single consumer warp (see Cfg)
     static constexpr int STAGES_CLAMPED = STAGES_RAW < C::NW ? C::NW : (STAGES_RAW > 32 ? 32 : STAGES_RAW);
     static constexpr int STAGES = STAGES_CLAMPED / C::NW * C::NW;
     static_assert(STAGES % C::NW == 0, "each stage must have a single consumer warp");
-    static constexpr size_t BYTES = 1024 + size_t(STAGES) * C::STAGE + size_t(C::NW) * C::VSTG +
-                                    size_t(COMB_FLOATS) * 4 + 8 * (2 * STAGES + 2 * kItemQ + 2);
-    static_assert(BYTES <= 227 * 1024, "shared memory");
+    // the warp-merge area holds NW * gc * (D + 2) floats, gc = query heads per
+    // item (known at launch); it follows the barriers
+    static constexpr size_t FIXED = 1024 + size_t(STAGES) * C::STAGE + size_t(C::NW) * C::VSTG +
+                                    8 * (2 * STAGES + 2 * kItemQ + 2);
+    static size_t bytes(int gc) { return FIXED + size_t(C::NW) * gc * (C::D + 2) * 4; }
 };
 
 template <class C>
@@ -891,7 +912,7 @@ struct Balanced : C {
 };
 
 template <class C0>
-__global__ void __launch_bounds__(C0::THREADS, 2)
+__global__ void __launch_bounds__(C0::THREADS, 3)
 decode_balanced(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                 const Params p) {
     using B = BalancedSmem<C0>;
@@ -904,13 +925,14 @@ decode_balanced(const __grid_constant__ CUtensorMap tmk, const __grid_constant__
     uint8_t* stages = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* vstage = stages + (size_t)STAGES * C::STAGE;
-    float* comb = reinterpret_cast<float*>(vstage + (size_t)C::NW * C::VSTG);
-    const uint32_t full0 = dev::smem_addr(comb + B::COMB_FLOATS);
+    const uint32_t full0 = dev::smem_addr(vstage + (size_t)C::NW * C::VSTG);
     const uint32_t empty0 = full0 + 8 * STAGES;
     const uint32_t ifull0 = empty0 + 8 * STAGES;
     const uint32_t iempty0 = ifull0 + 8 * kItemQ;
     const uint32_t rdv_pub = iempty0 + 8 * kItemQ;     // consumers published their states
     const uint32_t rdv_done = rdv_pub + 8;              // consumers finished the combine
+    float* comb = reinterpret_cast<float*>(vstage + (size_t)C::NW * C::VSTG +
+                                           8 * (2 * STAGES + 2 * kItemQ + 2));
 
     const int G = p.Hq / p.Hkv;
     const int gc = C::MMA ? G : C::GC;
@@ -1035,9 +1057,9 @@ decode_balanced(const __grid_constant__ CUtensorMap tmk, const __grid_constant__
         if (lane == 0) s_issued = k;
     } else {
         // --------------------------------------------------------- consumers
-        float* cm = comb;
-        float* cl = cm + C::NW * C::GC;
-        float* co = cl + C::NW * C::GC;
+        float* cm = comb;                              // stride gc (heads per item)
+        float* cl = cm + C::NW * gc;
+        float* co = cl + C::NW * gc;
         for (int ci = 0;; ++ci) {
             const int slot = ci % kItemQ;
             if (!dev::mbar_wait_bounded(ifull0 + 8 * slot, (ci / kItemQ) & 1)) {
@@ -1066,8 +1088,8 @@ decode_balanced(const __grid_constant__ CUtensorMap tmk, const __grid_constant__
                 if (lane == 0) dev::mbar_arrive(empty0 + 8 * stg);
             }
             if (!bad) {
-                if constexpr (C::MMA) mma_publish<C>(st, cm, cl, co, warp, G);
-                else simt_publish<C>(st, cm, cl, co, warp);
+                if constexpr (C::MMA) mma_publish<C>(st, cm, cl, co, warp, G, gc);
+                else simt_publish<C>(st, cm, cl, co, warp, gc);
                 __syncwarp();
                 if (lane == 0) dev::mbar_arrive(rdv_pub);
                 if (!dev::mbar_wait_bounded(rdv_pub, ci & 1)) bad = 5;
@@ -1084,14 +1106,14 @@ decode_balanced(const __grid_constant__ CUtensorMap tmk, const __grid_constant__
                 const int g = idx / C::D, dd = idx % C::D;
                 float M = -INFINITY;
                 #pragma unroll
-                for (int w = 0; w < C::NW; ++w) M = fmaxf(M, cm[w * C::GC + g]);
+                for (int w = 0; w < C::NW; ++w) M = fmaxf(M, cm[w * gc + g]);
                 float L = 0.f, O = 0.f;
                 if (M != -INFINITY) {
                     #pragma unroll
                     for (int w = 0; w < C::NW; ++w) {
-                        const float f = exp2f(cm[w * C::GC + g] - M);
-                        L = fmaf(f, cl[w * C::GC + g], L);
-                        O = fmaf(f, co[(w * C::GC + g) * C::D + dd], O);
+                        const float f = exp2f(cm[w * gc + g] - M);
+                        L = fmaf(f, cl[w * gc + g], L);
+                        O = fmaf(f, co[(w * gc + g) * C::D + dd], O);
                     }
                 }
                 if (first && last) {

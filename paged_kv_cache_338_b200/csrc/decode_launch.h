@@ -20,6 +20,7 @@ struct Launch {
     dim3 grid;
     cudaStream_t stream;
     bool balanced; // persistent work-balanced kernel (grid computed at launch)
+    int G;         // query heads per kv head
     int num_sms;
 };
 
@@ -36,7 +37,7 @@ template <class C>
 cudaError_t launch_one(const Launch& L) {
     if (L.balanced) {
         auto kern = decode_balanced<C>;
-        const int smem = static_cast<int>(BalancedSmem<C>::BYTES);
+        const int smem = static_cast<int>(BalancedSmem<C>::bytes(L.mma ? L.G : L.gc));
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         int per_sm = 0;
