@@ -255,6 +255,8 @@ typedef struct {
     int64_t shared_blocks;  /* reference count > 1 */
     int64_t cow_copies;     /* copies requested by pa_pool_seq_append so far */
     int64_t num_seqs;
+    int64_t cached_blocks;  /* blocks holding a registered content hash */
+    int64_t cache_hits;     /* prefix-cache hits so far */
 } pa_pool_stats_t;
 
 pa_status pa_pool_create(int64_t NB, int bs, pa_pool** out);
@@ -319,6 +321,35 @@ pa_status pa_pool_build_block_tables(const pa_pool* pool, const int64_t* seqs, i
                                      int32_t* tables_host, int32_t* ctx_lens_host);
 
 pa_status pa_pool_stats(const pa_pool* pool, pa_pool_stats_t* stats);
+
+/* The physical blocks of a sequence, in table order (*n is set even when cap
+ * is too small, which returns PA_ERR_INVALID_ARG). */
+pa_status pa_pool_seq_blocks(const pa_pool* pool, int64_t seq, int32_t* blocks, int cap, int* n);
+
+/*
+ * Prefix cache -- "01. PagedAttention 详解" self-check 3 and summary: a
+ * prefix-cache hit hands an already filled block to a new request by adding
+ * a reference (_get_cached_block: ref_cnt++), and freed blocks are reused in
+ * LRU order.  The caller names the content of a FULL block by a 64-bit hash
+ * of its own choosing (e.g. of the token ids it holds and of the previous
+ * block's hash).
+ *
+ * pa_pool_cache_block: remember that `block` (in use) holds content `hash`.
+ *   *cached = 1 if it is now the block for that hash; 0 if another block
+ *   already holds it.  A block whose count drops to 0 keeps its content and
+ *   hash while it waits in the free queue; taking it from the queue head for
+ *   a new allocation forgets the hash (eviction of the least recently freed).
+ *   Appending into a block the sequence holds alone forgets its hash.
+ * pa_pool_cache_lookup: *block = the block holding `hash` with one more
+ *   reference taken (a freed one leaves the free queue with count 1), or -1.
+ * pa_pool_seq_match_prefix: an EMPTY sequence takes the blocks of the longest
+ *   run of leading hashes that hit, one reference each; *matched = that count
+ *   and the sequence then holds matched * bs tokens.
+ */
+pa_status pa_pool_cache_block(pa_pool* pool, int32_t block, uint64_t hash, int* cached);
+pa_status pa_pool_cache_lookup(pa_pool* pool, uint64_t hash, int32_t* block);
+pa_status pa_pool_seq_match_prefix(pa_pool* pool, int64_t seq, const uint64_t* hashes, int n,
+                                   int* matched);
 
 #ifdef __cplusplus
 }

@@ -18,6 +18,17 @@ Plain Python, one step per rule on the pages:
   reference from the old block and continues in the new one.
 * "01. PagedAttention 详解" §6 and summary: sequences may share blocks (a common
   prefix, or a fork for beam search / parallel sampling) by adding references.
+* Prefix cache, "01. PagedAttention 详解" self-check 3 and summary, with the
+  content hash of "PagedAttention 机制" §6.3 and §5.1 (prefix_hashing): a
+  full block may be registered under a hash of its content; a hit takes a
+  reference on the cached block (_get_cached_block: ref_cnt++), which also
+  revives a block whose count had dropped to 0 but which still sits, content
+  intact, in the free queue; allocation from the head of the queue evicts the
+  oldest freed block's content (LRU reuse).  Which hash names which content is
+  the caller's choice.  Readings where the pages are silent: a hash names at
+  most one block (registering a second block under a held hash leaves the
+  first one in place); writing into a block the writer holds alone drops its
+  hash, since the content changes.
 
 Misuse raises a PoolError subclass whose ``status`` names the library's
 status code: freeing a free block or sharing a free block (PA_ERR_REFCOUNT),
@@ -27,7 +38,7 @@ requests (PA_ERR_INVALID_ARG); running out of free blocks raises OutOfBlocks
 """
 from __future__ import annotations
 
-from collections import Counter, deque
+from collections import Counter, OrderedDict
 
 
 class PoolError(Exception):
@@ -46,17 +57,47 @@ class BadIndex(PoolError):
     status = "PA_ERR_BAD_INDEX"
 
 
+class _FreeQueue:
+    """FIFO of free block ids that a prefix-cache hit can also take from the
+    middle (an insertion-ordered dict used as a set)."""
+
+    def __init__(self, items):
+        self._d = OrderedDict((b, None) for b in items)
+
+    def __len__(self):
+        return len(self._d)
+
+    def __iter__(self):
+        return iter(self._d)
+
+    def __contains__(self, b):
+        return b in self._d
+
+    def popleft(self):
+        b, _ = self._d.popitem(last=False)
+        return b
+
+    def append(self, b):
+        self._d[b] = None
+
+    def remove(self, b):
+        del self._d[b]
+
+
 class PoolModel:
     def __init__(self, num_blocks: int, block_size: int):
         if num_blocks <= 0 or block_size <= 0:
             raise InvalidArg("bad sizes")
         self.num_blocks = num_blocks
         self.block_size = block_size
-        self.free_queue = deque(range(num_blocks))
+        self.free_queue = _FreeQueue(range(num_blocks))
         self.ref = [0] * num_blocks
         self.seqs = {}            # id -> [blocks list, num tokens]
         self.next_seq = 0
         self.cow_count = 0
+        self.cached = {}          # content hash -> block holding it
+        self.block_hash = {}      # block -> its registered hash
+        self.cache_hits = 0
 
     # -- blocks -----------------------------------------------------------
     def _check_block(self, b):
@@ -67,8 +108,14 @@ class PoolModel:
         if not self.free_queue:
             raise OutOfBlocks("no free blocks")
         b = self.free_queue.popleft()
+        self._forget(b)           # reuse evicts whatever the block held
         self.ref[b] = 1
         return b
+
+    def _forget(self, b):
+        h = self.block_hash.pop(b, None)
+        if h is not None and self.cached.get(h) == b:
+            del self.cached[h]
 
     def free(self, b: int) -> None:
         self._check_block(b)
@@ -132,6 +179,8 @@ class PoolModel:
             blocks.append(self.alloc())
         else:
             last = blocks[-1]
+            if self.ref[last] <= 1:
+                self._forget(last)           # sole writer: the content changes
             if self.ref[last] > 1:
                 new = self.alloc()
                 self.ref[last] -= 1          # stays >= 1: the other holders keep it
@@ -188,8 +237,52 @@ class PoolModel:
             lens.append(n)
         return tables, lens
 
+    # -- prefix cache -----------------------------------------------------
+    def cache_block(self, b: int, h: int) -> bool:
+        """Register full block ``b`` (in use) as holding content ``h``.  True
+        when ``b`` is now the block for ``h``; False when another block holds it."""
+        self._check_block(b)
+        if self.ref[b] <= 0:
+            raise PoolError(f"block {b} is free")
+        if b in self.block_hash:
+            if self.block_hash[b] != h:
+                raise InvalidArg(f"block {b} already holds another hash")
+            return True
+        if h in self.cached:
+            return False
+        self.cached[h] = b
+        self.block_hash[b] = h
+        return True
+
+    def cache_lookup(self, h: int) -> int:
+        """The block holding ``h`` with one more reference taken, or -1."""
+        b = self.cached.get(h, -1)
+        if b < 0:
+            return -1
+        if self.ref[b] == 0:
+            self.free_queue.remove(b)        # a freed block comes back to life
+        self.ref[b] += 1
+        self.cache_hits += 1
+        return b
+
+    def seq_match_prefix(self, sid: int, hashes) -> int:
+        """An empty sequence takes the blocks of the leading hashes that hit."""
+        blocks, n = self._seq(sid)
+        if n != 0 or blocks:
+            raise InvalidArg("a prefix can only be matched into an empty sequence")
+        m = 0
+        for h in hashes:
+            b = self.cache_lookup(h)
+            if b < 0:
+                break
+            blocks.append(b)
+            m += 1
+        self.seqs[sid][1] = m * self.block_size
+        return m
+
     def stats(self):
         used = sum(1 for r in self.ref if r > 0)
         shared = sum(1 for r in self.ref if r > 1)
         return dict(num_blocks=self.num_blocks, free=len(self.free_queue), used=used,
-                    shared=shared, cow_copies=self.cow_count, num_seqs=len(self.seqs))
+                    shared=shared, cow_copies=self.cow_count, num_seqs=len(self.seqs),
+                    cached=len(self.cached), cache_hits=self.cache_hits)

@@ -49,7 +49,7 @@ class PaError(RuntimeError):
 class _Stats(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int64) for n in
                 ("num_blocks", "free_blocks", "used_blocks", "shared_blocks", "cow_copies",
-                 "num_seqs")]
+                 "num_seqs", "cached_blocks", "cache_hits")]
 
 
 _lib = None
@@ -93,6 +93,10 @@ def lib() -> ctypes.CDLL:
         "pa_pool_seq_len": ([P, I64], I64),
         "pa_pool_build_block_tables": ([P, P, I, I, P, P], I),
         "pa_pool_stats": ([P, ctypes.POINTER(_Stats)], I),
+        "pa_pool_seq_blocks": ([P, I64, P, I, ctypes.POINTER(I)], I),
+        "pa_pool_cache_block": ([P, I32, ctypes.c_uint64, ctypes.POINTER(I)], I),
+        "pa_pool_cache_lookup": ([P, ctypes.c_uint64, ctypes.POINTER(I32)], I),
+        "pa_pool_seq_match_prefix": ([P, I64, P, I, ctypes.POINTER(I)], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -342,3 +346,34 @@ class BlockPool:
         st = _Stats()
         _check(lib().pa_pool_stats(self._p, ctypes.byref(st)))
         return {n: getattr(st, n) for n, _ in _Stats._fields_}
+
+    def seq_blocks(self, seq: int) -> list:
+        n = ctypes.c_int(0)
+        lib().pa_pool_seq_blocks(self._p, seq, None, 0, ctypes.byref(n))   # size query
+        arr = (ctypes.c_int32 * max(n.value, 1))()
+        _check(lib().pa_pool_seq_blocks(self._p, seq, arr, n.value, ctypes.byref(n)))
+        return list(arr[:n.value])
+
+    # -- prefix cache (content hashes of full blocks) ---------------------------
+    def cache_block(self, block: int, content_hash: int) -> bool:
+        """Register a full, in-use block as holding ``content_hash`` (uint64).
+        True if it is now the block for that hash, False if another block is."""
+        c = ctypes.c_int(0)
+        _check(lib().pa_pool_cache_block(self._p, block, content_hash & 0xFFFFFFFFFFFFFFFF,
+                                         ctypes.byref(c)))
+        return bool(c.value)
+
+    def cache_lookup(self, content_hash: int) -> int:
+        """The cached block for the hash with one more reference taken, or -1."""
+        b = ctypes.c_int32()
+        _check(lib().pa_pool_cache_lookup(self._p, content_hash & 0xFFFFFFFFFFFFFFFF,
+                                          ctypes.byref(b)))
+        return b.value
+
+    def seq_match_prefix(self, seq: int, hashes: Sequence[int]) -> int:
+        """An empty sequence takes the cached blocks of the leading hashes that
+        hit; returns how many matched (it then holds that many full blocks)."""
+        arr = (ctypes.c_uint64 * max(len(hashes), 1))(*[h & 0xFFFFFFFFFFFFFFFF for h in hashes])
+        m = ctypes.c_int(0)
+        _check(lib().pa_pool_seq_match_prefix(self._p, seq, arr, len(hashes), ctypes.byref(m)))
+        return m.value

@@ -10,17 +10,53 @@
 // parallel sampling); intelliparadigm PagedAttention article §3.3 (writing
 // into a block with count > 1 first copies it: maybe_copy_block).
 #include <cstdint>
-#include <deque>
 #include <new>
 #include <unordered_map>
 #include <vector>
 
 #include "pa_internal.h"
 
+// FIFO of free blocks as an intrusive doubly linked list, so a cached block
+// can leave the middle of the queue when a prefix-cache hit revives it.
+struct FreeQueue {
+    std::vector<int32_t> prev, next;
+    std::vector<uint8_t> in;
+    int32_t head = -1, tail = -1;
+    int64_t count = 0;
+
+    void init(int64_t nb) {
+        prev.assign((size_t)nb, -1);
+        next.assign((size_t)nb, -1);
+        in.assign((size_t)nb, 0);
+        head = tail = -1;
+        count = 0;
+        for (int64_t b = 0; b < nb; ++b) push_back((int32_t)b);
+    }
+    bool empty() const { return count == 0; }
+    size_t size() const { return (size_t)count; }
+    int32_t front() const { return head; }
+    void push_back(int32_t b) {
+        prev[b] = tail;
+        next[b] = -1;
+        if (tail >= 0) next[tail] = b; else head = b;
+        tail = b;
+        in[b] = 1;
+        ++count;
+    }
+    void remove(int32_t b) {
+        if (prev[b] >= 0) next[prev[b]] = next[b]; else head = next[b];
+        if (next[b] >= 0) prev[next[b]] = prev[b]; else tail = prev[b];
+        prev[b] = next[b] = -1;
+        in[b] = 0;
+        --count;
+    }
+    void pop_front() { remove(head); }
+};
+
 struct pa_pool {
     int64_t nb = 0;
     int bs = 0;
-    std::deque<int32_t> free_q;
+    FreeQueue free_q;
     std::vector<int32_t> ref;
     struct Seq {
         std::vector<int32_t> blocks;
@@ -29,6 +65,11 @@ struct pa_pool {
     std::unordered_map<int64_t, Seq> seqs;
     int64_t next_seq = 0;
     int64_t cow = 0;
+    // prefix cache: content hash of a full block -> the block holding it
+    std::unordered_map<uint64_t, int32_t> by_hash;
+    std::vector<uint64_t> hash_of;
+    std::vector<uint8_t> hashed;
+    int64_t hits = 0;
 
     bool in_range(int64_t b) const { return b >= 0 && b < nb; }
     Seq* find(int64_t s) {
@@ -39,9 +80,16 @@ struct pa_pool {
         auto it = seqs.find(s);
         return it == seqs.end() ? nullptr : &it->second;
     }
+    void forget_hash(int32_t b) {
+        if (!hashed[b]) return;
+        auto it = by_hash.find(hash_of[b]);
+        if (it != by_hash.end() && it->second == b) by_hash.erase(it);
+        hashed[b] = 0;
+    }
     int32_t take() {             // caller checked that the queue is not empty
         const int32_t b = free_q.front();
         free_q.pop_front();
+        forget_hash(b);          // reusing the block evicts its cached content
         ref[b] = 1;
         return b;
     }
@@ -63,7 +111,9 @@ extern "C" pa_status pa_pool_create(int64_t NB, int bs, pa_pool** out) {
     p->nb = NB;
     p->bs = bs;
     p->ref.assign((size_t)NB, 0);
-    for (int64_t b = 0; b < NB; ++b) p->free_q.push_back((int32_t)b);
+    p->hash_of.assign((size_t)NB, 0);
+    p->hashed.assign((size_t)NB, 0);
+    p->free_q.init(NB);
     *out = p;
     return PA_OK;
 }
@@ -160,6 +210,7 @@ extern "C" pa_status pa_pool_seq_append(pa_pool* pool, int64_t seq, int64_t* slo
         s->blocks.push_back(pool->take());
     } else {
         const int32_t last = s->blocks.back();
+        if (pool->ref[last] <= 1) pool->forget_hash(last);   // its content is about to change
         if (pool->ref[last] > 1) {
             if (pool->free_q.empty()) return fail(PA_ERR_OUT_OF_BLOCKS, "no free blocks");
             const int32_t fresh = pool->take();
@@ -272,5 +323,84 @@ extern "C" pa_status pa_pool_stats(const pa_pool* pool, pa_pool_stats_t* st) {
     st->shared_blocks = shared;
     st->cow_copies = pool->cow;
     st->num_seqs = (int64_t)pool->seqs.size();
+    st->cached_blocks = (int64_t)pool->by_hash.size();
+    st->cache_hits = pool->hits;
+    return PA_OK;
+}
+
+extern "C" pa_status pa_pool_seq_blocks(const pa_pool* pool, int64_t seq, int32_t* blocks, int cap,
+                                        int* n) {
+    pa::clear_error();
+    if (!pool || !n || cap < 0 || (cap > 0 && !blocks)) return fail(PA_ERR_INVALID_ARG, "bad arguments");
+    const pa_pool::Seq* s = pool->find(seq);
+    if (!s) return fail(PA_ERR_BAD_INDEX, "unknown sequence %lld", (long long)seq);
+    *n = (int)s->blocks.size();
+    if ((int64_t)s->blocks.size() > cap) return fail(PA_ERR_INVALID_ARG, "cap %d < %zu blocks", cap,
+                                                      s->blocks.size());
+    for (size_t i = 0; i < s->blocks.size(); ++i) blocks[i] = s->blocks[i];
+    return PA_OK;
+}
+
+extern "C" pa_status pa_pool_cache_block(pa_pool* pool, int32_t block, uint64_t hash, int* cached) {
+    pa::clear_error();
+    if (!pool || !cached) return fail(PA_ERR_INVALID_ARG, "NULL argument");
+    if (!pool->in_range(block)) return fail(PA_ERR_BAD_INDEX, "block %d out of range", block);
+    if (pool->ref[block] <= 0) return fail(PA_ERR_REFCOUNT, "block %d is free", block);
+    *cached = 0;
+    if (pool->hashed[block]) {
+        if (pool->hash_of[block] != hash)
+            return fail(PA_ERR_INVALID_ARG, "block %d already holds another hash", block);
+        *cached = 1;
+        return PA_OK;
+    }
+    auto it = pool->by_hash.find(hash);
+    if (it != pool->by_hash.end()) return PA_OK;    // the content is cached in another block
+    pool->by_hash.emplace(hash, block);
+    pool->hash_of[block] = hash;
+    pool->hashed[block] = 1;
+    *cached = 1;
+    return PA_OK;
+}
+
+// A hit takes a reference: a block still in use gains one more holder; a
+// freed block that still holds the content leaves the free queue with
+// count 1.
+static int32_t cache_take(pa_pool* pool, uint64_t hash) {
+    auto it = pool->by_hash.find(hash);
+    if (it == pool->by_hash.end()) return -1;
+    const int32_t b = it->second;
+    if (pool->ref[b] == 0) {
+        pool->free_q.remove(b);
+        pool->ref[b] = 1;
+    } else {
+        ++pool->ref[b];
+    }
+    ++pool->hits;
+    return b;
+}
+
+extern "C" pa_status pa_pool_cache_lookup(pa_pool* pool, uint64_t hash, int32_t* block) {
+    pa::clear_error();
+    if (!pool || !block) return fail(PA_ERR_INVALID_ARG, "NULL argument");
+    *block = cache_take(pool, hash);
+    return PA_OK;
+}
+
+extern "C" pa_status pa_pool_seq_match_prefix(pa_pool* pool, int64_t seq, const uint64_t* hashes,
+                                              int n, int* matched) {
+    pa::clear_error();
+    if (!pool || !matched || n < 0 || (n > 0 && !hashes)) return fail(PA_ERR_INVALID_ARG, "bad arguments");
+    pa_pool::Seq* s = pool->find(seq);
+    if (!s) return fail(PA_ERR_BAD_INDEX, "unknown sequence %lld", (long long)seq);
+    if (s->n != 0 || !s->blocks.empty())
+        return fail(PA_ERR_INVALID_ARG, "a prefix can only be matched into an empty sequence");
+    int m = 0;
+    for (; m < n; ++m) {
+        const int32_t b = cache_take(pool, hashes[m]);
+        if (b < 0) break;
+        s->blocks.push_back(b);
+    }
+    s->n = (int64_t)m * pool->bs;
+    *matched = m;
     return PA_OK;
 }

@@ -238,3 +238,89 @@ def test_pool_batch_append_matches_model(seed):
         assert [pool.ref(b) for b in range(nb)] == model.ref
     with pytest.raises(pa.PaError):
         pool.seq_append_batch([seqs[0], seqs[0]])      # repeated sequence
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_prefix_cache_matches_model_on_random_call_sequences(seed):
+    """Hash registration, hits on live and freed blocks, LRU eviction through
+    allocation, and prefix matching, replayed against the oracle's model."""
+    rnd = random.Random(1000 + seed)
+    nb, bs = rnd.choice([(16, 4), (48, 8), (9, 16)])
+    model, pool = PoolModel(nb, bs), pa.BlockPool(nb, bs)
+    hashes = [rnd.getrandbits(64) for _ in range(24)]
+    live = []
+    for step in range(1500):
+        r = rnd.random()
+        if r < 0.08 or not live:
+            m, p = _run_both(model, pool, "seq_new")
+            assert m == p
+            live.append(m)
+        elif r < 0.45:
+            m, p = _run_both(model, pool, "seq_append", rnd.choice(live))
+            assert m == p
+        elif r < 0.50:
+            m, p = _run_both(model, pool, "seq_fork", rnd.choice(live))
+            assert m == p
+            if m is not None:
+                live.append(m)
+        elif r < 0.60 and len(live) > 1:
+            _run_both(model, pool, "seq_free", live.pop(rnd.randrange(len(live))))
+        elif r < 0.72:
+            s = rnd.choice(live)
+            blocks = model.seq_blocks(s)
+            full = model.seq_len(s) // bs
+            if full:
+                i = rnd.randrange(full)
+                m, p = _run_both(model, pool, "cache_block", blocks[i], rnd.choice(hashes))
+                assert m == p
+        elif r < 0.80:
+            m, p = _run_both(model, pool, "cache_lookup", rnd.choice(hashes))
+            assert m == p
+            if m is not None and m >= 0:
+                _run_both(model, pool, "free", m)
+        elif r < 0.88:
+            t, tp = _run_both(model, pool, "seq_new")
+            assert t == tp
+            live.append(t)
+            hs = [rnd.choice(hashes) for _ in range(rnd.randint(0, 4))]
+            m, p = _run_both(model, pool, "seq_match_prefix", t, hs)
+            assert m == p
+        elif r < 0.92:
+            m, p = _run_both(model, pool, "alloc")
+            assert m == p
+            if m is not None:
+                _run_both(model, pool, "free", m)
+        else:
+            _run_both(model, pool, "cache_block", rnd.randrange(-1, nb + 1), hashes[0])
+        assert [pool.ref(b) for b in range(nb)] == model.ref
+        st, ms = pool.stats(), model.stats()
+        assert (st["free_blocks"], st["cached_blocks"], st["cache_hits"]) == \
+            (ms["free"], ms["cached"], ms["cache_hits"])
+    for s in live:
+        assert pool.seq_blocks(s) == model.seq_blocks(s)
+        _run_both(model, pool, "seq_free", s)
+    while len(model.free_queue):      # same LRU order, same surviving hashes
+        for h in hashes:
+            m, p = _run_both(model, pool, "cache_lookup", h)
+            assert m == p
+            if m >= 0:
+                _run_both(model, pool, "free", m)
+        m, p = _run_both(model, pool, "alloc")
+        assert m == p
+
+
+def test_prefix_cache_argument_checks():
+    pool = pa.BlockPool(4, 4)
+    s = pool.seq_new()
+    for _ in range(4):
+        pool.seq_append(s)
+    _bad(pool.cache_block, 9, 1, status="PA_ERR_BAD_INDEX")
+    _bad(pool.cache_block, 3, 1, status="PA_ERR_REFCOUNT")
+    assert pool.cache_block(0, 1) and pool.cache_block(0, 1)
+    _bad(pool.cache_block, 0, 2)
+    _bad(pool.seq_match_prefix, s, [1])
+    _bad(pool.seq_match_prefix, 99, [1], status="PA_ERR_BAD_INDEX")
+    _bad(pool.seq_blocks, 99, status="PA_ERR_BAD_INDEX")
+    assert pool.cache_lookup(1) == 0 and pool.ref(0) == 2
+    assert pool.cache_lookup(2 ** 64 - 1) == -1
+    assert pool.stats()["cache_hits"] == 1

@@ -131,3 +131,98 @@ def test_copy_on_write_on_shared_last_block():
     assert p.ref[0] == 1 and p.ref[1] == 0 and list(p.free_queue)[-1] == 1
     p.seq_free(b)
     assert sum(p.ref) == 0 and sorted(p.free_queue) == list(range(8))
+
+
+# -- prefix cache: "01. PagedAttention 详解" self-check 3 and summary (hash hit
+#    -> ref_cnt++, LRU reuse of freed blocks); content hash as in "PagedAttention
+#    机制" §6.3 --------------------------------------------------------------
+
+def _filled_seq(p, ntok):
+    s = p.seq_new()
+    for _ in range(ntok):
+        p.seq_append(s)
+    return s
+
+
+def test_cache_hit_on_a_live_block_adds_a_reference():
+    p = PoolModel(8, 4)
+    a = _filled_seq(p, 8)                        # blocks 0, 1 full
+    assert p.cache_block(0, 111) and p.cache_block(1, 222)
+    assert p.cache_lookup(111) == 0              # _get_cached_block: ref_cnt++
+    assert p.ref[0] == 2 and p.ref[1] == 1
+    assert p.cache_lookup(999) == -1 and p.ref == [2, 1] + [0] * 6
+    assert p.stats()["cache_hits"] == 1 and p.stats()["shared"] == 1
+    p.free(0)
+    p.seq_free(a)
+    assert p.ref[0] == 0 and list(p.free_queue)[-2:] == [0, 1]
+
+
+def test_freed_cached_block_is_revived_from_the_queue():
+    p = PoolModel(4, 4)
+    a = _filled_seq(p, 8)                        # blocks 0, 1
+    p.cache_block(0, 7)
+    p.seq_free(a)                                # both counts reach 0, content kept
+    assert list(p.free_queue) == [2, 3, 0, 1]
+    assert p.cache_lookup(7) == 0                # leaves the middle of the queue
+    assert p.ref[0] == 1 and list(p.free_queue) == [2, 3, 1]
+    assert p.cached == {7: 0}
+
+
+def test_reuse_from_the_queue_head_evicts_the_least_recently_freed():
+    p = PoolModel(3, 2)
+    x, y = _filled_seq(p, 2), _filled_seq(p, 2)  # blocks 0 and 1
+    p.cache_block(0, 10)
+    p.cache_block(1, 11)
+    p.seq_free(x)                                # 0 freed first ...
+    p.seq_free(y)                                # ... then 1
+    assert list(p.free_queue) == [2, 0, 1]
+    assert p.alloc() == 2                        # never cached: no eviction
+    assert p.alloc() == 0                        # reuse evicts hash 10
+    assert p.cache_lookup(10) == -1
+    assert p.cache_lookup(11) == 1               # the more recently freed survives
+    assert p.stats()["cached"] == 1
+
+
+def test_a_hash_names_one_block_and_writes_drop_it():
+    p = PoolModel(6, 4)
+    a = _filled_seq(p, 4)
+    b = _filled_seq(p, 4)
+    assert p.cache_block(0, 5)
+    assert not p.cache_block(1, 5)               # same content elsewhere: first stays
+    assert p.cache_block(0, 5)                   # idempotent
+    with pytest.raises(InvalidArg):
+        p.cache_block(0, 6)
+    with pytest.raises(PoolError):
+        p.cache_block(4, 6)                      # a free block cannot be registered
+    # a partial block registered by the caller loses its hash once written alone
+    c = _filled_seq(p, 2)
+    blk = p.seq_blocks(c)[0]
+    p.cache_block(blk, 77)
+    p.seq_append(c)
+    assert p.cache_lookup(77) == -1
+    # ... but a shared one is copied first and keeps it
+    p.cache_block(blk, 78)
+    d = p.seq_fork(c)
+    slot, src, dst = p.seq_append(d)
+    assert src == blk and p.cache_lookup(78) == blk
+    del a, b
+
+
+def test_match_prefix_takes_the_leading_hits_only():
+    bs = 4
+    p = PoolModel(10, bs)
+    a = _filled_seq(p, 3 * bs + 1)               # blocks 0, 1, 2 full, 3 partial
+    for i, h in enumerate((100, 101, 102)):
+        p.cache_block(i, h)
+    p.seq_free(a)
+    b = p.seq_new()
+    assert p.seq_match_prefix(b, [100, 101, 555, 102]) == 2
+    assert p.seq_blocks(b) == [0, 1] and p.seq_len(b) == 2 * bs
+    assert p.ref[:4] == [1, 1, 0, 0]
+    slot, src, dst = p.seq_append(b)             # next token opens a fresh block
+    assert (src, dst) == (-1, -1) and slot // bs not in (0, 1, 2)
+    with pytest.raises(InvalidArg):
+        p.seq_match_prefix(b, [102])             # only into an empty sequence
+    c = p.seq_new()
+    assert p.seq_match_prefix(c, [100, 101, 102]) == 3
+    assert p.ref[:3] == [2, 2, 1]
