@@ -112,6 +112,8 @@ class ClockSampler:
         pid = _pci_id(dev)
         os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
         self.path = os.path.join(ROOT, "gpurun_out", f"nvml_rank{dev}.log")
+        if os.path.exists(self.path):      # a previous run's log would end the wait below early
+            os.remove(self.path)
         self.child = subprocess.Popen([sys.executable, os.path.abspath(__file__),
                                        "--nvml-sampler", pid or "", self.path],
                                       stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
@@ -124,7 +126,7 @@ class ClockSampler:
         except Exception:
             self.proc = None
         # wait until the child has produced its first sample
-        for _ in range(400):
+        for _ in range(1500):
             if os.path.exists(self.path) and os.path.getsize(self.path) > 0:
                 break
             time.sleep(0.01)
