@@ -9,6 +9,11 @@ Every function takes host arrays (numpy, or CPU torch tensors, which are viewed
 as their raw bytes) and dtype names "f32", "f16", "bf16", "fp8_e4m3".
 
 Parity status of each part (what pins it, see tests/test_oracle_*.py):
+  prefill attention  -- pinned: torch SDPA in float64 with an explicit causal
+                        mask on the unpaged gather, L=1 rows = decode rows,
+                        chunk invariance (one chunk = two chunks), causality
+                        (keys past a row's position do not change it), the
+                        first token of a prefill returns v_0.
   decode attention   -- pinned: torch SDPA in float64 on the unpaged gather,
                         brute force on tiny cases, invariants (block-id
                         permutation, shared prefix, weights sum to 1) and the
@@ -88,6 +93,9 @@ def lib():
         L.orc_paged_decode.restype = I
         L.orc_decode_weights.argtypes = [P, P, I, P, I, P, I, P, I, I, I, I, I64, D, D, I, I]
         L.orc_decode_weights.restype = I
+        L.orc_paged_prefill.argtypes = [P, P, I, P, P, I, P, I, P, P, I, I, I, I, I, I, I64,
+                                        D, D, D, P, I, I]
+        L.orc_paged_prefill.restype = I
     return _lib
 
 
@@ -196,3 +204,28 @@ def decode_weights(q, q_dtype, key_cache, kv_dtype, block_tables, context_lens, 
                                   float(scale), float(k_scale), int(s), int(h))
     _check(rc, "decode_weights")
     return w[:int(cl[s])]
+
+
+def paged_prefill(q, q_dtype, key_cache, value_cache, kv_dtype, block_tables, context_lens,
+                  query_start, scale, k_scale=1.0, v_scale=1.0, rows=None,
+                  nthreads=0) -> np.ndarray:
+    """fp64 causal attention of the new tokens [len(rows) or T, Hq, D]."""
+    qa = raw(q)
+    kc, vc = raw(key_cache), raw(value_cache)
+    bt = np.ascontiguousarray(np.asarray(raw(block_tables), dtype=np.int32))
+    cl = np.ascontiguousarray(np.asarray(raw(context_lens), dtype=np.int32))
+    qs = np.ascontiguousarray(np.asarray(raw(query_start), dtype=np.int32))
+    T, Hq, D = qa.shape
+    NB, bs, Hkv, D2 = kc.shape
+    assert D2 == D
+    S = cl.size
+    MB = bt.shape[1] if bt.ndim == 2 else 0
+    sel = None if rows is None else np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
+    nrow = T if sel is None else sel.size
+    out = np.zeros((nrow, Hq, D), dtype=np.float64)
+    rc = lib().orc_paged_prefill(_ptr(out), _ptr(qa), DT[q_dtype], _ptr(kc), _ptr(vc),
+                                 DT[kv_dtype], _ptr(bt), MB, _ptr(cl), _ptr(qs), S, T, Hq, Hkv,
+                                 D, bs, NB, float(scale), float(k_scale), float(v_scale),
+                                 None if sel is None else _ptr(sel), nrow, int(nthreads))
+    _check(rc, "paged_prefill")
+    return out

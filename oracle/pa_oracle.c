@@ -43,6 +43,17 @@
  *   deq multiplies the stored value by k_scale / v_scale (1 for non-fp8).
  *   The per-block, online or split form the kernels use is a reordering of
  *   this sum and is deliberately not reproduced here.
+ *
+ *   Prefill / chunked prefill ("01. PagedAttention 详解" §4, prefill: the N new
+ *   tokens' K and V are first written into the blocks their table names, then
+ *   ordinary attention runs over the cache).  Sequence s holds n_s tokens in
+ *   the cache, the last L_s of which are this call's new tokens (rows
+ *   query_start[s] .. query_start[s+1]-1 of q).  New token i sits at position
+ *   p = n_s - L_s + i and, reading the attention as the usual causal one of a
+ *   decoder, sees the keys at positions 0..p:
+ *       out[row, h] = softmax(scale * K_s[0..p] q[row, h]) V_s[0..p]
+ *   L_s = 1 is the decode step above; L_s = n_s is a prefill from an empty
+ *   cache; anything between is a chunk of a chunked prefill.
  */
 #include <math.h>
 #include <pthread.h>
@@ -355,4 +366,105 @@ int orc_decode_weights(double* w, const void* q, int q_dt, const void* key_cache
     }
     free(K); free(V); free(qv); free(o);
     return rc;
+}
+
+/* ----------------------------------------------------------------- prefill */
+
+typedef struct {
+    decode_job base;          /* caches, tables, shapes, scales */
+    double* out;              /* [nrow or T, Hq, D] */
+    const int32_t* qstart;    /* [S+1] */
+    const int32_t* rows;      /* NULL: every row; else nrow row ids */
+    int nrow, S, T;
+    int status;
+} prefill_job;
+
+/* Sequence owning q row t (query_start is non-decreasing). */
+static int row_seq(const int32_t* qs, int S, int t) {
+    int lo = 0, hi = S - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) / 2;
+        if (qs[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+static void* prefill_worker(void* arg) {
+    prefill_job* pj = (prefill_job*)arg;
+    const decode_job* j = &pj->base;
+    int G = j->Hq / j->Hkv;
+    double* K = NULL;
+    double* V = NULL;
+    double* w = NULL;
+    double* qv = (double*)malloc(sizeof(double) * j->D);
+    size_t cap = 0;
+    int nr = pj->rows ? pj->nrow : pj->T;
+    /* one unit = (selected row, kv head): gather, then the G heads of the group */
+    for (int u = j->tid; u < nr * j->Hkv; u += j->nthreads) {
+        int ri = u / j->Hkv, g = u % j->Hkv;
+        int t = pj->rows ? pj->rows[ri] : ri;
+        int s = row_seq(pj->qstart, pj->S, t);
+        int n = j->ctx[s];
+        int L = pj->qstart[s + 1] - pj->qstart[s];
+        int p = n - L + (t - pj->qstart[s]);      /* position of this token */
+        int nk = p + 1;                           /* keys 0..p */
+        if ((size_t)nk > cap) {
+            cap = (size_t)nk;
+            free(K); free(V); free(w);
+            K = (double*)malloc(sizeof(double) * cap * j->D);
+            V = (double*)malloc(sizeof(double) * cap * j->D);
+            w = (double*)malloc(sizeof(double) * cap);
+            if (!K || !V || !w) { pj->status = ORC_ENOMEM; break; }
+        }
+        int rc = gather(j, s, g, nk, K, V);
+        if (rc) { pj->status = rc; break; }
+        for (int hh = 0; hh < G; ++hh) {
+            int h = g * G + hh;
+            size_t qoff = ((size_t)t * j->Hq + h) * j->D;
+            for (int d = 0; d < j->D; ++d) qv[d] = value_at(j->q, j->q_dt, qoff + d);
+            attend(qv, K, V, nk, j->D, j->scale, w, pj->out + ((size_t)ri * j->Hq + h) * j->D);
+        }
+    }
+    free(K); free(V); free(w); free(qv);
+    return NULL;
+}
+
+/* out: [nrow or T, Hq, D] double.  q: [T, Hq, D].  query_start: [S+1] with
+ * query_start[0] = 0, query_start[S] = T, and 0 <= L_s <= n_s.  rows: NULL for
+ * every q row, else nrow row ids. */
+int orc_paged_prefill(double* out, const void* q, int q_dt, const void* key_cache,
+                      const void* value_cache, int kv_dt, const int32_t* block_tables, int MB,
+                      const int32_t* context_lens, const int32_t* query_start, int S, int T,
+                      int Hq, int Hkv, int D, int bs, int64_t NB, double scale, double k_scale,
+                      double v_scale, const int32_t* rows, int nrow, int nthreads) {
+    if (S < 0 || T < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || D <= 0 || bs <= 0 || MB < 0)
+        return ORC_EARG;
+    if (query_start[0] != 0 || query_start[S] != T) return ORC_EARG;
+    for (int s = 0; s < S; ++s) {
+        int L = query_start[s + 1] - query_start[s];
+        if (L < 0 || L > context_lens[s]) return ORC_EARG;
+        if ((int64_t)context_lens[s] > (int64_t)MB * bs) return ORC_EARG;
+    }
+    if (rows)
+        for (int i = 0; i < nrow; ++i)
+            if (rows[i] < 0 || rows[i] >= T) return ORC_EARG;
+    int nt = hw_threads(nthreads);
+    prefill_job* jobs = (prefill_job*)calloc((size_t)nt, sizeof(prefill_job));
+    pthread_t* th = (pthread_t*)calloc((size_t)nt, sizeof(pthread_t));
+    for (int t = 0; t < nt; ++t) {
+        decode_job b = {NULL, q, q_dt, key_cache, value_cache, kv_dt, block_tables, MB,
+                        context_lens, NULL, 0, Hq, Hkv, D, bs, NB, scale, k_scale, v_scale,
+                        nt, t, ORC_OK};
+        prefill_job pj = {b, out, query_start, rows, nrow, S, T, ORC_OK};
+        jobs[t] = pj;
+        pthread_create(&th[t], NULL, prefill_worker, &jobs[t]);
+    }
+    int status = ORC_OK;
+    for (int t = 0; t < nt; ++t) {
+        pthread_join(th[t], NULL);
+        if (jobs[t].status && !status) status = jobs[t].status;
+    }
+    free(jobs);
+    free(th);
+    return status;
 }

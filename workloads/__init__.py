@@ -297,3 +297,157 @@ def make_decode_inputs(cfg: DecodeConfig, seed: int, device="cpu") -> DecodeInpu
 def kv_bytes_per_token(cfg: DecodeConfig) -> int:
     """K plus V bytes one token of one sequence occupies (all kv heads)."""
     return 2 * cfg.num_kv_heads * cfg.head_dim * elem_bytes(cfg.kv_dtype)
+
+
+# --------------------------------------------------------------------- prefill
+
+@dataclasses.dataclass(frozen=True)
+class PrefillConfig:
+    """A batch of prefill chunks: sequence s already holds c_s cached tokens and
+    this step appends L_s new ones (their K, V through slot_mapping), then the
+    new tokens attend causally over all c_s + L_s."""
+    name: str
+    num_seqs: int
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int
+    dtype: str               # q / out / cache dtype (f16 or bf16)
+    q_lo: int                # L_s uniform in [q_lo, q_hi]
+    q_hi: int
+    ctx_lo: int              # c_s uniform in [ctx_lo, ctx_hi]
+    ctx_hi: int
+    fixed_q: Optional[tuple] = None
+    fixed_ctx: Optional[tuple] = None
+    slack: float = 0.1
+
+    @property
+    def group(self) -> int:
+        return self.num_q_heads // self.num_kv_heads
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.head_dim)
+
+
+PREFILL_CONFIGS = {
+    # Llama-3-8B attention shapes, chunked prefill: 16 chunks of 2048 new tokens
+    # on top of 0..6144 cached tokens each.
+    "llama3_8b_gqa_bf16_chunked_prefill": PrefillConfig(
+        "llama3_8b_gqa_bf16_chunked_prefill", 16, 32, 8, 128, 16, "bf16", 2048, 2048, 0, 6144),
+    # the same shapes, prefill from an empty cache: 8 prompts of 1024..4096 tokens
+    "llama3_8b_gqa_bf16_prefill": PrefillConfig(
+        "llama3_8b_gqa_bf16_prefill", 8, 32, 8, 128, 16, "bf16", 1024, 4096, 0, 0),
+}
+
+
+@dataclasses.dataclass
+class PrefillInputs:
+    cfg: PrefillConfig
+    q: torch.Tensor                 # [T, Hq, D]
+    key_cache: torch.Tensor         # [NB, bs, Hkv, D], state before this step's append
+    value_cache: torch.Tensor
+    key_new: torch.Tensor           # [T, Hkv, D]: the new tokens' k, v
+    value_new: torch.Tensor
+    slot_mapping: torch.Tensor      # [T] int64
+    block_tables: torch.Tensor      # [S, MB] int32
+    context_lens: torch.Tensor      # [S] int32: c_s + L_s
+    query_start: torch.Tensor       # [S + 1] int32
+    cached_lens: torch.Tensor       # [S] int64: c_s
+    scale: float
+    num_blocks: int
+    max_blocks: int
+
+    @property
+    def max_query_len(self) -> int:
+        qs = self.query_start.cpu()
+        return int((qs[1:] - qs[:-1]).max().item()) if qs.numel() > 1 else 0
+
+    @property
+    def num_tokens(self) -> int:
+        return int(self.query_start[-1].item())
+
+
+def make_prefill_inputs(cfg: PrefillConfig, seed: int, device="cpu") -> PrefillInputs:
+    """Seeded inputs for one prefill step of ``cfg`` on ``device``.
+
+    Every sequence owns ceil((c + L) / bs) shuffled physical blocks.  Cached
+    positions hold N(0,1) draws; positions c..end of the last block, blocks no
+    table references and this step's slots before the append hold NaN codes;
+    table entries past the sequence's blocks are -1.
+    """
+    S, Hkv, D, bs = cfg.num_seqs, cfg.num_kv_heads, cfg.head_dim, cfg.block_size
+    gh = torch.Generator(device="cpu").manual_seed(seed)
+    if cfg.fixed_q is not None:
+        L = torch.tensor(cfg.fixed_q, dtype=torch.int64)
+    else:
+        L = torch.randint(cfg.q_lo, cfg.q_hi + 1, (S,), generator=gh)
+    if cfg.fixed_ctx is not None:
+        c = torch.tensor(cfg.fixed_ctx, dtype=torch.int64)
+    else:
+        c = torch.randint(cfg.ctx_lo, cfg.ctx_hi + 1, (S,), generator=gh)
+    n = c + L
+    nblk = (n + bs - 1) // bs
+    MB = max(int(nblk.max().item()) if S else 1, 1)
+    used = int(nblk.sum().item())
+    NB = max(int(math.ceil(used * (1.0 + cfg.slack))), used, 1)
+    perm = torch.randperm(NB, generator=gh).to(torch.int32)
+    tables = torch.full((S, MB), -1, dtype=torch.int32)
+    cur = 0
+    for s in range(S):
+        k = int(nblk[s])
+        tables[s, :k] = perm[cur:cur + k]
+        cur += k
+    free_ids = perm[cur:]
+
+    dev = torch.device(device)
+    gd = torch.Generator(device=dev).manual_seed(seed + 7919)
+    t = torch_dtype(cfg.dtype)
+    kc = torch.empty((NB, bs, Hkv, D), dtype=t, device=dev)
+    vc = torch.empty_like(kc)
+    _fill_normal(kc, cfg.dtype, gd)
+    _fill_normal(vc, cfg.dtype, gd)
+    T = int(L.sum().item())
+    q = torch.empty((T, cfg.num_q_heads, D), dtype=t, device=dev)
+    kn = torch.empty((T, Hkv, D), dtype=t, device=dev)
+    vn = torch.empty_like(kn)
+    _fill_normal(q, cfg.dtype, gd)
+    _fill_normal(kn, cfg.dtype, gd)
+    _fill_normal(vn, cfg.dtype, gd)
+
+    nan_t = torch.tensor(_NAN_BITS[cfg.dtype], dtype=_RAW[_DT[cfg.dtype][1]], device=dev)
+    rk, rv = raw_view(kc, cfg.dtype), raw_view(vc, cfg.dtype)
+    if free_ids.numel():
+        fi = free_ids.to(dev, torch.int64)
+        rk[fi] = nan_t
+        rv[fi] = nan_t
+    pb, po, slots = [], [], []
+    for s in range(S):
+        for pos in range(int(c[s]), int(nblk[s]) * bs):
+            pb.append(int(tables[s, pos // bs]))
+            po.append(pos % bs)
+        for pos in range(int(c[s]), int(n[s])):
+            slots.append(int(tables[s, pos // bs]) * bs + pos % bs)
+    if pb:
+        bi = torch.tensor(pb, dtype=torch.int64, device=dev)
+        oi = torch.tensor(po, dtype=torch.int64, device=dev)
+        rk[bi, oi] = nan_t
+        rv[bi, oi] = nan_t
+    qs = torch.zeros(S + 1, dtype=torch.int32)
+    qs[1:] = torch.cumsum(L, 0).to(torch.int32)
+    return PrefillInputs(
+        cfg=cfg, q=q, key_cache=kc, value_cache=vc, key_new=kn, value_new=vn,
+        slot_mapping=torch.tensor(slots, dtype=torch.int64).to(dev),
+        block_tables=tables.to(dev), context_lens=n.to(torch.int32).to(dev),
+        query_start=qs.to(dev), cached_lens=c, scale=cfg.scale, num_blocks=NB, max_blocks=MB)
+
+
+def prefill_flops(cfg: PrefillConfig, query_start: torch.Tensor, context_lens: torch.Tensor) -> int:
+    """Multiply-adds x 2 of the causal attention the step must do: each new token
+    at position p scores p + 1 keys (Q.K) and sums p + 1 values (P.V)."""
+    qs = query_start.cpu().to(torch.int64)
+    n = context_lens.cpu().to(torch.int64)
+    L = qs[1:] - qs[:-1]
+    c = n - L
+    keys = int((L * c + L * (L + 1) // 2).sum().item())    # sum over new tokens of p + 1
+    return 4 * keys * cfg.num_q_heads * cfg.head_dim
