@@ -73,8 +73,11 @@ enum {
     PA_DEV_BAD_PIECES = 16    /* pa_decode merge: inconsistent split records (rows left unwritten) */
 };
 /* Bits 16-23 of the device word, when PA_DEV_WAIT_TIMEOUT is set: which wait
- * gave up last (diagnostics; 1 stage-free, 2 stage-full, 3 descriptor-free,
- * 4 descriptor-ready, 5 states-published, 6 merge-done). */
+ * gave up last (diagnostics; decode: 1 stage-free, 2 stage-full,
+ * 3 descriptor-free, 4 descriptor-ready, 5 states-published, 6 merge-done;
+ * prefill: 7 q-tile, 8 k-tile-full, 9 v-tile-full, 10 k-tile-free,
+ * 11 v-tile-free, 12 scores-ready, 13 probabilities-ready, 14 p.v-done,
+ * 15 output-ready, 16 tensor-core drain, 17 load drain). */
 
 /* Message for the last failing call on this thread ("" if none). */
 const char* pa_last_error(void);
@@ -232,6 +235,44 @@ pa_status pa_decode_noalloc(void* out, const void* q, pa_dtype q_dt,
  * Default 4.  Every setting computes the same function.
  */
 pa_status pa_decode_select(int mode);
+
+/*
+ * Prefill / chunked-prefill attention over the paged cache -- "01. PagedAttention
+ * 详解" §4, prefill: the N new tokens' K and V are first written through the
+ * block table (pa_reshape_and_cache with their slots), then attention runs
+ * over the cache.  Sequence s holds n_s = context_lens[s] tokens in the cache,
+ * of which the last L_s = query_start[s+1] - query_start[s] are this call's new
+ * tokens, rows query_start[s] .. query_start[s+1]-1 of q.  New token i sits at
+ * position p = n_s - L_s + i and attends causally to the keys at 0..p:
+ *
+ *   out[row, h, :] = softmax(scale * K_s[0..p] q[row, h, :]) V_s[0..p]
+ *
+ * with K_s, V_s gathered through block_tables exactly as in pa_decode (kv head
+ * h / (Hq / Hkv)).  L_s = n_s is a prefill from an empty cache, L_s < n_s a
+ * chunk of a chunked prefill (or a prefix-cache hit), L_s = 1 a decode step.
+ *
+ * Arguments (device pointers unless stated):
+ *   out, q       [T, Hq, D] of q_dt, T = query_start[S]; rows of one sequence
+ *                are contiguous.  16-byte aligned.
+ *   key_cache, value_cache  [NB, bs, Hkv, D] of cache_dt; cache_dt must equal
+ *                q_dt (PA_F16 or PA_BF16: the tensor cores take both operands
+ *                in one type); other dtypes return PA_ERR_UNSUPPORTED.
+ *   block_tables [S, MB] int32; context_lens [S] int32;
+ *   query_start  [S+1] int32, non-decreasing, query_start[0] = 0.
+ *   max_query_len  host int >= every L_s (sizes the grid).
+ *   D in {64, 128}; Hq / Hkv in {1, 2, 4, 8, 16}; bs in {8, 16, 32}.
+ * Work runs asynchronously on `stream` with no allocation and no workspace.
+ * Host checks return PA_ERR_INVALID_ARG / PA_ERR_UNSUPPORTED before anything is
+ * enqueued.  Device-side, a table entry outside [0, NB) sets PA_DEV_BAD_BLOCK
+ * (its keys are read as whatever the tile held: the rows that need them are
+ * invalid); L_s > n_s, L_s > max_query_len or n_s > MB * bs sets
+ * PA_DEV_BAD_CONTEXT and the sequence's rows are left unwritten.
+ */
+pa_status pa_prefill(void* out, const void* q, pa_dtype q_dt, const void* key_cache,
+                     const void* value_cache, pa_dtype cache_dt, const int32_t* block_tables,
+                     int MB, const int32_t* context_lens, const int32_t* query_start, int S,
+                     int T, int Hq, int Hkv, int D, int bs, int64_t NB, int max_query_len,
+                     float scale, pa_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * Host block pool -- "PagedAttention 机制" §5.3.4 (BlockAllocator: free list,

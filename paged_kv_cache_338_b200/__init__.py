@@ -21,7 +21,8 @@ import torch
 __all__ = [
     "PaError", "lib", "pa_version", "pa_last_error", "pa_device_status",
     "pa_reshape_and_cache", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_size",
-    "pa_decode_suggest_partition", "pa_decode_select", "pa_decode_noalloc", "BlockPool",
+    "pa_decode_suggest_partition", "pa_decode_select", "pa_decode_noalloc", "pa_prefill",
+    "BlockPool",
     "PA_DEV_BAD_SLOT", "PA_DEV_BAD_BLOCK", "PA_DEV_WAIT_TIMEOUT", "PA_DEV_BAD_CONTEXT",
 ]
 
@@ -77,6 +78,7 @@ def lib() -> ctypes.CDLL:
         "pa_decode_select": ([I], I),
         "pa_decode": ([P, P, I, P, P, I, P, I, P, I, I, I, I, I, I64, I, F, F, F, I, P, SZ, P], I),
         "pa_decode_noalloc": ([P, P, I, P, P, I, P, I, P, I, I, I, I, I, I64, I, F, F, F, I, P], I),
+        "pa_prefill": ([P, P, I, P, P, I, P, I, P, P, I, I, I, I, I, I, I64, I, F, P], I),
         "pa_pool_create": ([I64, I, ctypes.POINTER(P)], I),
         "pa_pool_destroy": ([P], None),
         "pa_pool_alloc": ([P, ctypes.POINTER(I32)], I),
@@ -241,6 +243,29 @@ def pa_decode_noalloc(out: torch.Tensor, q: torch.Tensor, key_cache: torch.Tenso
                                    _ptr(context_lens), S, Hq, Hkv, D, bs, NB, int(max_ctx),
                                    float(scale), float(k_scale), float(v_scale), int(partition),
                                    _stream(stream)))
+
+
+def pa_prefill(out: torch.Tensor, q: torch.Tensor, key_cache: torch.Tensor,
+               value_cache: torch.Tensor, block_tables: torch.Tensor, context_lens: torch.Tensor,
+               query_start: torch.Tensor, max_query_len: int, scale: float,
+               stream=None) -> None:
+    """Causal attention of a batch of new-token chunks over the paged cache.
+    out/q [T, Hq, D]; caches [NB, bs, Hkv, D] (same dtype as q); block_tables
+    [S, MB] int32; context_lens [S] int32 (cached + new tokens); query_start
+    [S + 1] int32 (row offsets of each sequence's new tokens in q)."""
+    T, Hq, D = q.shape
+    NB, bs, Hkv, _ = key_cache.shape
+    S = context_lens.numel()
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    for t in (block_tables, context_lens, query_start):
+        if t.dtype != torch.int32:
+            raise PaError(1, "block_tables, context_lens and query_start must be int32")
+    if query_start.numel() != S + 1:
+        raise PaError(1, "query_start must hold S + 1 offsets")
+    _check(lib().pa_prefill(_ptr(out), _ptr(q), _dt(q), _ptr(key_cache), _ptr(value_cache),
+                            _dt(key_cache), _ptr(block_tables), MB, _ptr(context_lens),
+                            _ptr(query_start), S, T, Hq, Hkv, D, bs, NB, int(max_query_len),
+                            float(scale), _stream(stream)))
 
 
 class BlockPool:

@@ -9,6 +9,7 @@
 
 #include "decode_launch.h"
 #include "pa_internal.h"
+#include "tma_host.h"
 
 namespace pa {
 namespace {
@@ -17,50 +18,6 @@ namespace {
 // hint on K/V loads, 4 = partition-major grid (kv heads of a partition side
 // by side); the default is 4.
 std::atomic<int> g_select{4};
-
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
-                                             cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
-CUtensorMapDataType tma_type(pa_dtype dt) {
-    switch (dt) {
-    case PA_F32: return CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-    case PA_F16: return CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-    case PA_BF16: return CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    default: return CU_TENSOR_MAP_DATA_TYPE_UINT8;
-    }
-}
-
-// The cache [NB, bs, Hkv, D] as a 4-D tensor {D, Hkv, bs, NB} (innermost
-// first).  A box {128 bytes of D, 1, bs, 1} is one 128-byte segment of the
-// K (or V) tile of one block for one kv head, swizzled per 128-byte row; a
-// tile takes D * elt / 128 boxes, at x = 0, 128 / elt, ...
-pa_status make_map(CUtensorMap* m, const void* base, pa_dtype dt, int64_t NB, int bs, int Hkv,
-                   int D) {
-    auto fn = encode_fn();
-    if (!fn) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
-    const int e = elem_size(dt);
-    const cuuint64_t row = (cuuint64_t)D * e;            // bytes of one (token, head) row
-    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)bs, (cuuint64_t)NB};
-    cuuint64_t strides[3] = {row, row * Hkv, row * Hkv * bs};
-    cuuint32_t box[4] = {(cuuint32_t)(128 / e), 1, (cuuint32_t)bs, 1};
-    cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = fn(m, tma_type(dt), 4, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
-    return PA_OK;
-}
 
 // Launched as a programmatic dependent of the partition kernel so its launch
 // overlaps that grid's last wave (it waits for the grid's memory itself).
@@ -236,9 +193,9 @@ extern "C" pa_status pa_decode(void* out, const void* q, pa_dtype q_dt, const vo
                     need, workspace_bytes);
 
     dec::Launch L{};
-    pa_status st = make_map(&L.tmk, key_cache, cache_dt, NB, bs, Hkv, D);
+    pa_status st = make_cache_map(&L.tmk, key_cache, cache_dt, NB, bs, Hkv, D);
     if (st) return st;
-    st = make_map(&L.tmv, value_cache, cache_dt, NB, bs, Hkv, D);
+    st = make_cache_map(&L.tmv, value_cache, cache_dt, NB, bs, Hkv, D);
     if (st) return st;
     unsigned int* err = device_error_word();
     if (!err) return PA_ERR_CUDA;

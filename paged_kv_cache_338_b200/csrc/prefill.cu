@@ -1,0 +1,625 @@
+// Prefill / chunked-prefill attention over the paged cache on the 5th-generation
+// tensor cores ("01. PagedAttention 详解" §4, prefill: the new tokens' K, V
+// are written through the block table first, then attention runs over the
+// cache; the keys are gathered block by block through the table as in the
+// decode loop of the same section).
+//
+// One CTA computes a 128-row query tile of one (sequence, kv head): the rows
+// are TQ = 128 / G consecutive new tokens x the G query heads that share the kv
+// head, so K and V tiles are loaded once for the whole group.  Keys run in
+// tiles of 128 (128 / bs blocks, each fetched by its own tensor-map load from
+// the block the table names).  Per key tile j:
+//
+//   S_j = Q K_j^T         tcgen05.mma, M 128, N 128, K = D; S in tensor memory
+//   P_j = exp2(S_j * scale * log2 e - m)   softmax warps, one row per thread,
+//                                           causal + length mask, rounded to
+//                                           the operand type into shared memory
+//   O  += P_j V_j         tcgen05.mma, M 128, N = D, K 128; O in tensor memory
+//
+// The running maximum m is raised only when a tile's maximum exceeds it by
+// more than 8 (in log2 units); O and the running sum are then rescaled in
+// place.  Between raises the probabilities stay below 2^8, so the result is
+// the same softmax (the final division uses the same m for both sums).
+//
+// Warp roles (192 threads): warps 0-3 softmax and epilogue (warp w owns TMEM
+// lanes 32w..32w+31, i.e. query rows), warp 4 loads (tensor-map copies of Q
+// once, then K and V tiles into two-deep rings), warp 5 allocates tensor memory
+// and one of its lanes issues every MMA.  S is double-buffered in tensor
+// memory so S_{j+1} is computed while the softmax warps work on S_j; P is
+// double-buffered in shared memory.  Every wait is bounded (2 s): on timeout
+// the CTA records PA_DEV_WAIT_TIMEOUT with the wait's site, drains its own
+// copies and MMAs, frees its tensor memory and exits.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+
+#include "pa_device.cuh"
+#include "pa_internal.h"
+#include "tma_host.h"
+
+namespace pf {
+
+using namespace pa::dev;
+
+constexpr int kBM = 128;          // query rows per tile
+constexpr int kBN = 128;          // keys per tile
+constexpr int kSeg = 16384;       // 128 rows x 128 bytes: one operand segment
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleLog2 = 8.0f;
+
+struct Params {
+    void* out;
+    const int32_t* block_tables;
+    const int32_t* context_lens;
+    const int32_t* query_start;
+    unsigned int* err;
+    long long NB;
+    int S, Hq, G, log2G, TQ, MB, bs, log2bs, max_qlen, n_qtiles;
+    float sl;                     // scale * log2(e)
+};
+
+template <int D>
+struct Smem {
+    static constexpr int NSEG = D / 64;             // 128-byte segments of a row
+    static constexpr int ST = D == 64 ? 3 : 2;      // K and V ring depth
+    static constexpr int TILE = NSEG * kSeg;        // 128 rows of D elements
+    static constexpr int Q = 0;
+    static constexpr int K = Q + TILE;
+    static constexpr int V = K + ST * TILE;
+    static constexpr int P = V + ST * TILE;         // two 128 x 128 probability tiles
+    static constexpr int BAR = P + 2 * (kBN / 64) * kSeg;
+    // barriers: q, k_full[ST], k_free[ST], v_full[ST], v_free[ST], s_full[2],
+    // p_full[2], pv_done[2], o_full, drain
+    static constexpr int NBAR = 1 + 4 * ST + 2 + 2 + 2 + 1 + 1;
+    static constexpr int TMEM_SLOT = BAR + NBAR * 8;
+    static constexpr int ABORT = TMEM_SLOT + 4;
+    static constexpr int BYTES = ABORT + 4 + 1024;  // + slack to align the base to 1024
+};
+
+// ------------------------------------------------------------- PTX wrappers
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1, int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_4d_plain(uint32_t dst, const CUtensorMap* map,
+                                                  uint32_t bar, int c0, int c1, int c2, int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2),
+          "r"(c3)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t slot, uint32_t cols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(slot), "r"(cols) : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t cols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(bar) : "memory");
+}
+
+// D (tensor memory, fp32) (+)= A (shared) x B (shared), kind::f16.
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// 32 consecutive 32-bit columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32"
+        " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15,"
+        " %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31},"
+        " [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
+    uint32_t r[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(v[i]);
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0],"
+        " {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16,"
+        " %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+          "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]),
+          "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]),
+          "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]),
+          "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle: start address, leading
+// byte offset (between 64-element groups along M/N of an MN-major operand;
+// unused for K-major), stride byte offset 1024 (between groups of 8 rows),
+// the fixed descriptor version bit, and the swizzle mode.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)(1024u >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor of kind::f16: fp32 accumulator, A and B of one type
+// (f16 = 0, bf16 = 1), A K-major, B K-major or MN-major, M 128, N.
+__device__ __forceinline__ uint32_t idesc_f16(int ab_bf16, int b_mn_major, int N) {
+    return (1u << 4) | ((uint32_t)ab_bf16 << 7) | ((uint32_t)ab_bf16 << 10) |
+           ((uint32_t)b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+}
+
+template <int DT> __device__ __forceinline__ uint32_t pack2(float a, float b);
+template <> __device__ __forceinline__ uint32_t pack2<PA_BF16>(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+template <> __device__ __forceinline__ uint32_t pack2<PA_F16>(float a, float b) {
+    __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+template <int DT> __device__ __forceinline__ float2 unpack2(uint32_t u);
+template <> __device__ __forceinline__ float2 unpack2<PA_BF16>(uint32_t u) {
+    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
+template <> __device__ __forceinline__ float2 unpack2<PA_F16>(uint32_t u) {
+    return __half22float2(*reinterpret_cast<__half2*>(&u));
+}
+
+// Bounded wait by every lane of a warp; the verdict is warp-uniform.  A
+// pipeline wait gives up early once another role has aborted the CTA; a drain
+// wait (honor_abort false) does not, since it guards memory still in flight.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned int* err, unsigned site,
+                                          bool honor_abort = true) {
+    bool ok = mbar_try_wait(bar, parity);
+    if (!__all_sync(~0u, ok)) {
+        const uint64_t t0 = global_ns();
+        while (!ok) {
+#pragma unroll 1
+            for (int i = 0; i < 64 && !ok; ++i) ok = mbar_try_wait(bar, parity);
+            if (ok || (honor_abort && *abort_flag)) break;
+            if (global_ns() - t0 > 2000000000ull) {
+                atomicOr(err, PA_DEV_WAIT_TIMEOUT | (site << 16));
+                break;
+            }
+        }
+    }
+    ok = __all_sync(~0u, ok);
+    if (!ok) *abort_flag = 1;
+    return ok;
+}
+
+// ------------------------------------------------------------------- kernel
+
+template <int DT, int D>
+__global__ void __launch_bounds__(kThreads, 1)
+prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+               const __grid_constant__ CUtensorMap tmv, const Params p) {
+    using L = Smem<D>;
+    constexpr int NSEG = L::NSEG, ST = L::ST;
+    const int g = blockIdx.x, s = blockIdx.y;
+    const int qt = p.n_qtiles - 1 - (int)blockIdx.z;      // longest tiles first
+
+    const int q0 = p.query_start[s];
+    const int Ls = p.query_start[s + 1] - q0;
+    const int n = p.context_lens[s];
+    if (Ls < 0 || Ls > n || Ls > p.max_qlen || (long long)n > (long long)p.MB * p.bs) {
+        if (qt == 0 && g == 0 && threadIdx.x == 0) atomicOr(p.err, PA_DEV_BAD_CONTEXT);
+        return;
+    }
+    const int i0 = qt * p.TQ;                 // first new token of this tile
+    if (i0 >= Ls) return;                     // whole CTA: nothing to compute
+    const int c = n - Ls;                     // tokens cached before this chunk
+    const int i1 = min(Ls, i0 + p.TQ);
+    const int kv_len = c + i1;                // the tile's last row sees keys 0..kv_len-1
+    const int nt = (kv_len + kBN - 1) / kBN;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+    const uint32_t sb = smem_addr(sm);
+    const uint32_t sQ = sb + L::Q, sK = sb + L::K, sV = sb + L::V, sP = sb + L::P;
+    const uint32_t bar0 = sb + L::BAR;
+    auto q_full = [&]() { return bar0; };
+    auto k_full = [&](int i) { return bar0 + 8u * (1 + i); };
+    auto k_free = [&](int i) { return bar0 + 8u * (1 + ST + i); };
+    auto v_full = [&](int i) { return bar0 + 8u * (1 + 2 * ST + i); };
+    auto v_free = [&](int i) { return bar0 + 8u * (1 + 3 * ST + i); };
+    auto s_full = [&](int i) { return bar0 + 8u * (1 + 4 * ST + i); };
+    auto p_full = [&](int i) { return bar0 + 8u * (3 + 4 * ST + i); };
+    auto pv_done = [&](int i) { return bar0 + 8u * (5 + 4 * ST + i); };
+    const uint32_t o_full = bar0 + 8u * (7 + 4 * ST);
+    const uint32_t drain = bar0 + 8u * (8 + 4 * ST);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::ABORT);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(q_full(), 1);
+        for (int i = 0; i < ST; ++i) {
+            mbar_init(k_full(i), 1);
+            mbar_init(k_free(i), 1);
+            mbar_init(v_full(i), 1);
+            mbar_init(v_free(i), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(s_full(i), 1);
+            mbar_init(p_full(i), 128);
+            mbar_init(pv_done(i), 1);
+        }
+        mbar_init(o_full, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 5) {
+        tmem_alloc(sb + L::TMEM_SLOT, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + L::TMEM_SLOT);
+    const uint32_t tS = tmem, tO = tmem + 2 * kBN;     // S buffers at columns 0, 128; O at 256
+
+    if (warp == 4) {
+        // ------------------------------------------------------------ loads
+        const int bpt = kBN >> p.log2bs;                       // blocks per key tile
+        const int need = (kv_len + p.bs - 1) >> p.log2bs;      // blocks the tile reads
+        const uint32_t box = (uint32_t)p.bs * 128u;
+        if (lane == 0) {
+            mbar_arrive_expect_tx(q_full(), NSEG * kSeg);
+            for (int sg = 0; sg < NSEG; ++sg)
+                tma_load_3d(sQ + sg * kSeg, &tmq, q_full(), sg * 64, g * p.G, q0 + i0);
+        }
+        int nk = 0, nvl = 0;                                  // K, V tiles started
+        for (int j = 0; j < nt; ++j) {
+            const int st = j % ST;
+            const uint32_t par = ((j / ST) & 1) ^ 1;
+            const int lb = j * bpt + lane;
+            const bool want = lane < bpt && lb < need;
+            int id = -1;
+            if (want) id = p.block_tables[(size_t)s * p.MB + lb];
+            const bool valid = want && id >= 0 && (long long)id < p.NB;
+            if (want && !valid) atomicOr(p.err, PA_DEV_BAD_BLOCK);
+            const uint32_t bytes = (uint32_t)__popc(__ballot_sync(~0u, valid)) * NSEG * box;
+            if (!warp_wait(k_free(st), par, abort_flag, p.err, 10)) break;
+            if (lane == 0) mbar_arrive_expect_tx(k_full(st), bytes);
+            __syncwarp();
+            if (valid)
+                for (int sg = 0; sg < NSEG; ++sg)
+                    tma_load_4d_plain(sK + st * L::TILE + sg * kSeg + lane * box, &tmk, k_full(st),
+                                      sg * 64, g, 0, id);
+            nk = j + 1;
+            if (!warp_wait(v_free(st), par, abort_flag, p.err, 11)) break;
+            if (lane == 0) mbar_arrive_expect_tx(v_full(st), bytes);
+            __syncwarp();
+            if (valid)
+                for (int sg = 0; sg < NSEG; ++sg)
+                    tma_load_4d_plain(sV + st * L::TILE + sg * kSeg + lane * box, &tmv, v_full(st),
+                                      sg * 64, g, 0, id);
+            nvl = j + 1;
+        }
+        // every copy this warp started has landed before the CTA may exit
+        // (immediate on the normal path, where the MMA warp consumed them all)
+        for (int i = 0; i < ST; ++i) {
+            // the last tile started in slot i is the largest j < count with j % ST == i
+            if (nk > i) {
+                const int jl = i + (nk - 1 - i) / ST * ST;
+                warp_wait(k_full(i), (jl / ST) & 1, abort_flag, p.err, 17, false);
+            }
+            if (nvl > i) {
+                const int jl = i + (nvl - 1 - i) / ST * ST;
+                warp_wait(v_full(i), (jl / ST) & 1, abort_flag, p.err, 17, false);
+            }
+        }
+        warp_wait(q_full(), 0, abort_flag, p.err, 17, false);
+    } else if (warp == 5) {
+        // ------------------------------------------------------------- MMAs
+        constexpr int ABF = DT == PA_BF16 ? 1 : 0;
+        const uint32_t id_s = idesc_f16(ABF, 0, kBN);
+        const uint32_t id_o = idesc_f16(ABF, 1, D);
+        bool ok = warp_wait(q_full(), 0, abort_flag, p.err, 7);
+        auto issue_s = [&](int j) -> bool {
+            const int st = j % ST;
+            if (!warp_wait(k_full(st), (j / ST) & 1, abort_flag, p.err, 8)) return false;
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t kb = sK + st * L::TILE;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kSeg + (kk & 3) * 32;
+                    tc_mma(tS + (j & 1) * kBN, sdesc(sQ + off, 16), sdesc(kb + off, 16), id_s,
+                           kk > 0);
+                }
+                tc_commit(s_full(j & 1));
+                tc_commit(k_free(st));
+            }
+            __syncwarp();
+            return true;
+        };
+        if (ok) ok = issue_s(0);
+        for (int j = 0; j < nt && ok; ++j) {
+            if (j + 1 < nt && !(ok = issue_s(j + 1))) break;
+            const int st = j % ST;
+            if (!(ok = warp_wait(p_full(j & 1), (j >> 1) & 1, abort_flag, p.err, 13))) break;
+            if (!(ok = warp_wait(v_full(st), (j / ST) & 1, abort_flag, p.err, 9))) break;
+            const uint32_t vb = sV + st * L::TILE;
+            if (j == nt - 1) {
+                // Rows at or past kv_len hold another token's values, the cache's
+                // unused tail slots or stale tiles: zero them, since a zero
+                // probability times a NaN would still poison the product.
+                const int z0 = kv_len - j * kBN;
+                const int chunks = (kBN - z0) * 8;              // 16-byte chunks per segment
+                for (int sg = 0; sg < NSEG; ++sg)
+                    for (int x = lane; x < chunks; x += 32)
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};"
+                                     ::"r"(vb + sg * kSeg + z0 * 128 + x * 16), "r"(0) : "memory");
+                fence_proxy_async_smem();
+                __syncwarp();
+            }
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t pb = sP + (j & 1) * (kBN / 64) * kSeg;
+#pragma unroll
+                for (int kk = 0; kk < kBN / 16; ++kk) {
+                    const uint32_t aoff = (kk >> 2) * kSeg + (kk & 3) * 32;
+                    tc_mma(tO, sdesc(pb + aoff, 16), sdesc(vb + kk * 16 * 128, kSeg), id_o,
+                           (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                tc_commit(pv_done(j & 1));
+                tc_commit(v_free(st));
+                if (j == nt - 1) tc_commit(o_full);
+            }
+            __syncwarp();
+        }
+        // every MMA this warp issued completes before tensor memory is freed
+        if (lane == 0) tc_commit(drain);
+        __syncwarp();
+        warp_wait(drain, 0, abort_flag, p.err, 16, false);
+    } else {
+        // ------------------------------------------------- softmax (rows)
+        const int r = threadIdx.x;                           // row = TMEM lane
+        const int it = i0 + (r >> p.log2G);                  // new-token index of the row
+        const bool row_ok = it < Ls;
+        const int limit = row_ok ? c + it + 1 : kv_len;      // keys 0..limit-1 are visible
+        const uint32_t lrow = (uint32_t)(warp * 32) << 16;
+        const float sl = p.sl;
+        float m_use = -INFINITY, lsum = 0.f;
+        bool ok = true;
+        for (int j = 0; j < nt; ++j) {
+            if (!(ok = warp_wait(s_full(j & 1), (j >> 1) & 1, abort_flag, p.err, 12))) break;
+            tc_fence_after();
+            float sv[kBN];
+#pragma unroll
+            for (int c4 = 0; c4 < kBN / 32; ++c4) tmem_ld32(tS + lrow + (j & 1) * kBN + c4 * 32,
+                                                           sv + c4 * 32);
+            tmem_wait_ld();
+            const int nv = min(max(limit - j * kBN, 0), kBN);
+            float tmax = -INFINITY;
+#pragma unroll
+            for (int k = 0; k < kBN; ++k) {
+                sv[k] *= sl;
+                if (k < nv) tmax = fmaxf(tmax, sv[k]);
+            }
+            const float m_new = fmaxf(m_use, tmax);
+            const bool raise = m_new > m_use + kRescaleLog2;
+            const float alpha = raise ? exp2f(m_use - m_new) : 1.f;
+            if (raise) m_use = m_new;
+            lsum *= alpha;
+            if (j > 0 && __any_sync(~0u, raise)) {
+                if (!(ok = warp_wait(pv_done((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag, p.err,
+                                     14)))
+                    break;
+                tc_fence_after();
+#pragma unroll 1
+                for (int c4 = 0; c4 < D / 32; ++c4) {
+                    float o[32];
+                    tmem_ld32(tO + lrow + c4 * 32, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] *= alpha;
+                    tmem_st32(tO + lrow + c4 * 32, o);
+                }
+                tmem_wait_st();
+            }
+            if (j >= 2 && !(ok = warp_wait(pv_done(j & 1), ((j - 2) >> 1) & 1, abort_flag, p.err,
+                                           14)))
+                break;
+            // probabilities, rounded to the operand type, into the 128-byte
+            // swizzled K-major tile the P.V MMA reads
+            const uint32_t prow = sP + (j & 1) * (kBN / 64) * kSeg + r * 128;
+#pragma unroll
+            for (int sg = 0; sg < kBN / 64; ++sg) {
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int k = sg * 64 + ch * 8 + 2 * e;
+                        const float a = k < nv ? exp2f(sv[k] - m_use) : 0.f;
+                        const float b = k + 1 < nv ? exp2f(sv[k + 1] - m_use) : 0.f;
+                        w[e] = pack2<DT>(a, b);
+                        const float2 rb = unpack2<DT>(w[e]);
+                        lsum += rb.x + rb.y;
+                    }
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                                 ::"r"(prow + sg * kSeg + ((ch ^ (r & 7)) << 4)), "r"(w[0]),
+                                   "r"(w[1]), "r"(w[2]), "r"(w[3])
+                                 : "memory");
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(p_full(j & 1));
+        }
+        if (ok) ok = warp_wait(o_full, 0, abort_flag, p.err, 15);
+        if (ok) {
+            tc_fence_after();
+            const float inv = 1.f / lsum;
+            const int h = g * p.G + (r & (p.G - 1));
+            uint8_t* orow = static_cast<uint8_t*>(p.out) +
+                            ((size_t)(q0 + it) * p.Hq + h) * (size_t)D * 2;
+#pragma unroll 1
+            for (int c4 = 0; c4 < D / 32; ++c4) {
+                float o[32];
+                tmem_ld32(tO + lrow + c4 * 32, o);
+                tmem_wait_ld();
+                if (row_ok) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + c4 * 64);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        uint4 w;
+                        w.x = pack2<DT>(o[8 * v + 0] * inv, o[8 * v + 1] * inv);
+                        w.y = pack2<DT>(o[8 * v + 2] * inv, o[8 * v + 3] * inv);
+                        w.z = pack2<DT>(o[8 * v + 4] * inv, o[8 * v + 5] * inv);
+                        w.w = pack2<DT>(o[8 * v + 6] * inv, o[8 * v + 7] * inv);
+                        dst[v] = w;
+                    }
+                }
+            }
+        }
+        tc_fence_before();
+    }
+
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+template <int DT, int D>
+cudaError_t launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                   const Params& p, dim3 grid, cudaStream_t st) {
+    static bool attr_set = false;       // per instantiation; idempotent if raced
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(prefill_kernel<DT, D>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             Smem<D>::BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    prefill_kernel<DT, D><<<grid, kThreads, Smem<D>::BYTES, st>>>(mq, mk, mv, p);
+    return cudaGetLastError();
+}
+
+}  // namespace pf
+
+using pa::fail;
+
+extern "C" pa_status pa_prefill(void* out, const void* q, pa_dtype q_dt, const void* key_cache,
+                                const void* value_cache, pa_dtype cache_dt,
+                                const int32_t* block_tables, int MB, const int32_t* context_lens,
+                                const int32_t* query_start, int S, int T, int Hq, int Hkv, int D,
+                                int bs, int64_t NB, int max_query_len, float scale,
+                                pa_stream_t stream) {
+    pa::clear_error();
+    if (!pa::valid_dtype(q_dt) || !pa::valid_dtype(cache_dt))
+        return fail(PA_ERR_INVALID_ARG, "unknown dtype");
+    if (q_dt != cache_dt || (q_dt != PA_F16 && q_dt != PA_BF16))
+        return fail(PA_ERR_UNSUPPORTED, "prefill takes q and cache both f16 or both bf16");
+    if (D != 64 && D != 128) return fail(PA_ERR_UNSUPPORTED, "head size %d (64 or 128)", D);
+    if (bs != 8 && bs != 16 && bs != 32) return fail(PA_ERR_UNSUPPORTED, "block size %d", bs);
+    if (S < 0 || T < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || MB <= 0 || NB <= 0 ||
+        max_query_len < 0)
+        return fail(PA_ERR_INVALID_ARG, "bad sizes");
+    const int G = Hq / Hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16)
+        return fail(PA_ERR_UNSUPPORTED, "group size %d (1, 2, 4, 8 or 16)", G);
+    if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "scale is not finite");
+    if (S == 0 || T == 0 || max_query_len == 0) return PA_OK;
+    if (!out || !q || !key_cache || !value_cache || !block_tables || !context_lens ||
+        !query_start)
+        return fail(PA_ERR_INVALID_ARG, "NULL pointer");
+    if (!pa::aligned16(out) || !pa::aligned16(q) || !pa::aligned16(key_cache) ||
+        !pa::aligned16(value_cache))
+        return fail(PA_ERR_INVALID_ARG, "out, q and the caches must be 16-byte aligned");
+    const int TQ = pf::kBM / G;
+    const long long n_qt = ((long long)max_query_len + TQ - 1) / TQ;
+    if (S > 65535 || n_qt > 65535 || Hkv > 65535)
+        return fail(PA_ERR_UNSUPPORTED, "grid too large (S %d, query tiles %lld)", S, n_qt);
+    if (NB > 0x7fffffffLL) return fail(PA_ERR_INVALID_ARG, "NB must fit int32 block ids");
+
+    CUtensorMap mq, mk, mv;
+    pa_status st = pa::make_rows_map(&mq, q, q_dt, T, Hq, D, G, TQ);
+    if (st) return st;
+    st = pa::make_cache_map(&mk, key_cache, cache_dt, NB, bs, Hkv, D);
+    if (st) return st;
+    st = pa::make_cache_map(&mv, value_cache, cache_dt, NB, bs, Hkv, D);
+    if (st) return st;
+    unsigned int* err = pa::device_error_word();
+    if (!err) return PA_ERR_CUDA;
+
+    pf::Params p;
+    p.out = out;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.query_start = query_start;
+    p.err = err;
+    p.NB = NB;
+    p.S = S;
+    p.Hq = Hq;
+    p.G = G;
+    p.log2G = __builtin_ctz((unsigned)G);
+    p.TQ = TQ;
+    p.MB = MB;
+    p.bs = bs;
+    p.log2bs = __builtin_ctz((unsigned)bs);
+    p.max_qlen = max_query_len;
+    p.n_qtiles = (int)n_qt;
+    p.sl = scale * 1.4426950408889634f;
+
+    const dim3 grid((unsigned)Hkv, (unsigned)S, (unsigned)n_qt);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (q_dt == PA_BF16)
+        e = D == 64 ? pf::launch<PA_BF16, 64>(mq, mk, mv, p, grid, cs)
+                    : pf::launch<PA_BF16, 128>(mq, mk, mv, p, grid, cs);
+    else
+        e = D == 64 ? pf::launch<PA_F16, 64>(mq, mk, mv, p, grid, cs)
+                    : pf::launch<PA_F16, 128>(mq, mk, mv, p, grid, cs);
+    if (e != cudaSuccess) return pa::cuda_fail(e, "prefill launch");
+    return PA_OK;
+}

@@ -324,3 +324,34 @@ def test_prefix_cache_argument_checks():
     assert pool.cache_lookup(1) == 0 and pool.ref(0) == 2
     assert pool.cache_lookup(2 ** 64 - 1) == -1
     assert pool.stats()["cache_hits"] == 1
+
+
+def test_prefill_host_argument_checks():
+    L = pa.lib()
+    # (out, q, q_dt, kc, vc, cache_dt, bt, MB, lens, qs, S, T, Hq, Hkv, D, bs, NB, maxq, scale, st)
+    base = [16, 16, 2, 16, 16, 2, 16, 4, 16, 16, 2, 10, 8, 2, 128, 16, 10, 8, 0.1, None]
+
+    def call(**kw):
+        a = list(base)
+        names = ["out", "q", "q_dt", "kc", "vc", "cache_dt", "bt", "MB", "lens", "qs", "S", "T",
+                 "Hq", "Hkv", "D", "bs", "NB", "maxq", "scale", "st"]
+        for k, v in kw.items():
+            a[names.index(k)] = v
+        return L.pa_prefill(*a)
+
+    assert call(q_dt=2, cache_dt=3) == 2          # fp8 cache: the tensor cores take one type
+    assert call(q_dt=0, cache_dt=0) == 2          # fp32
+    assert call(q_dt=1, cache_dt=2) == 2          # mixed
+    assert call(q_dt=9) == 1                      # unknown dtype
+    assert call(D=256) == 2 and call(D=96) == 2
+    assert call(bs=64) == 2
+    assert call(Hq=6, Hkv=2) == 2                 # group 3
+    assert call(Hq=7, Hkv=2) == 1                 # not a divisor
+    assert call(scale=float("inf")) == 1
+    assert call(out=None) == 1
+    assert call(q=24) == 1                        # misaligned
+    assert call(S=70000) == 2                     # grid limit
+    # nothing to do: no sequences, no tokens or empty chunks
+    assert call(S=0, out=None, q=None) == 0
+    assert call(T=0, out=None, q=None) == 0
+    assert call(maxq=0, out=None) == 0
