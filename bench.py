@@ -490,6 +490,223 @@ def run_e2e(args, cfg, pa, dev, part):
             "h2d": h2d, "d2h": d2h}
 
 
+# ------------------------------------------------------------- prefill (next row)
+
+PREFILL_METRIC = "paged chunked-prefill attention TFLOP/s (causal, of the bf16 tensor peak)"
+
+
+def _prefill_peak(timed_ms: float):
+    """Measured dense bf16 peak: the sustained figure for a loop of a second or
+    more (the power cap has settled), else the burst one."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        if timed_ms >= 1000.0 and "bf16_tflops_sustained" in p:
+            return float(p["bf16_tflops_sustained"]), "measured sustained"
+        return float(p["bf16_tflops"]), "measured burst"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+def _prefill_config_dict(cfg: wl.PrefillConfig, args, note=None):
+    d = {"workload": cfg.name, "num_seqs": cfg.num_seqs, "q_heads": cfg.num_q_heads,
+         "kv_heads": cfg.num_kv_heads, "head_dim": cfg.head_dim, "block_size": cfg.block_size,
+         "dtype": cfg.dtype, "new_tokens": [cfg.q_lo, cfg.q_hi], "cached_tokens":
+         [cfg.ctx_lo, cfg.ctx_hi], "parallelism": f"replicas{args.gpus}"}
+    if note:
+        d["l2"] = note
+    return d
+
+
+def prefill_oracle_rate(cfg: wl.PrefillConfig, seed: int, budget_s: float) -> dict:
+    """The fp64 oracle on the host cores over sampled rows of the workload."""
+    import oracle  # test infrastructure: only the CPU-baseline / reference legs use it
+    cores = os.cpu_count() or 1
+    inp = wl.make_prefill_inputs(cfg, seed=seed)
+    qs = inp.query_start.cpu().tolist()
+    n = inp.context_lens.cpu().tolist()
+    g = torch.Generator().manual_seed(seed)
+    rows, keys, nrow = [], 0, max(cores, 8)
+
+    def run(rs):
+        t0 = time.perf_counter()
+        oracle.paged_prefill(inp.q, cfg.dtype, inp.key_cache, inp.value_cache, cfg.dtype,
+                             inp.block_tables, inp.context_lens, inp.query_start, inp.scale,
+                             rows=rs, nthreads=cores)
+        return time.perf_counter() - t0
+
+    def keys_of(rs):
+        k = 0
+        for t in rs:
+            s = max(i for i in range(cfg.num_seqs) if qs[i] <= t)
+            k += n[s] - (qs[s + 1] - qs[s]) + (t - qs[s]) + 1
+        return k
+
+    # size the sample so that one pass takes about budget_s / 2
+    probe = torch.randint(0, qs[-1], (nrow,), generator=g).tolist()
+    tp = max(run(probe), 1e-3)
+    nrow = int(max(1, min(qs[-1], nrow * (budget_s / 2) / tp)))
+    rows = torch.randint(0, qs[-1], (nrow,), generator=g).tolist()
+    keys = keys_of(rows)
+    t, reps = 0.0, 0
+    while reps < 1 or t < budget_s / 2:
+        t += run(rows)
+        reps += 1
+    flops = 4 * keys * cfg.num_q_heads * cfg.head_dim
+    return {"tflops": flops * reps / t / 1e12, "cores": cores, "seconds": t / reps,
+            "sample": f"{nrow} random query rows of the workload (all {cfg.num_q_heads} heads, "
+                      f"{keys} causal keys), fp64 oracle on {cores} threads, {reps} passes"}
+
+
+def run_gpu_prefill(args, cfg: wl.PrefillConfig, rank, world, local_rank):
+    import paged_kv_cache_338_b200 as pa
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    inp = wl.make_prefill_inputs(cfg, seed=args.seed + rank, device=dev)
+    out = torch.empty_like(inp.q)
+    kc, vc = inp.key_cache, inp.value_cache
+    maxq = inp.max_query_len
+    flops = wl.prefill_flops(cfg, inp.query_start, inp.context_lens)
+    kv_gb = 2 * kc.numel() * kc.element_size() / 1e9
+
+    def step(ev=None):
+        pa.pa_reshape_and_cache(inp.key_new, inp.value_new, kc, vc, inp.slot_mapping)
+        if ev is not None:
+            ev[0].record(stream)
+        pa.pa_prefill(out, inp.q, kc, vc, inp.block_tables, inp.context_lens, inp.query_start,
+                      maxq, inp.scale)
+        if ev is not None:
+            ev[1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert pa.pa_device_status() == 0
+    dist = world > 1
+    if dist:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks.mark_start()
+    t0.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clocks.mark_end()
+    clk = clocks.stop()
+    assert pa.pa_device_status() == 0
+    if dist:
+        torch.distributed.barrier()
+    ms = t0.elapsed_time(t1)
+    k_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    if dist:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+    value = world * flops / (ms_step * 1e-3) / 1e12
+    e2e = None if args.no_e2e else prefill_e2e(args, cfg, pa, dev)
+    if dist and e2e is not None:
+        t = torch.tensor([e2e["ms"]], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e["value"] = world * flops / (float(t.item()) * 1e-3) / 1e12
+    if rank != 0:
+        return
+    peak, peak_kind = _prefill_peak(ms)
+    achieved = flops / (k_ms * 1e-3) / 1e12
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        r = prefill_oracle_rate(cfg, args.seed, args.cpu_budget)
+        cpu = {"value": round(r["tflops"], 6), "unit": "TFLOP/s", "cores": r["cores"],
+               "kind": "oracle", "sample": r["sample"]}
+    line = {
+        "metric": PREFILL_METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
+        "data": "synthetic",
+        "config": _prefill_config_dict(cfg, args, f"K/V cache {kv_gb:.2f} GB; re-read across "
+                                                  f"query tiles, no flush"),
+        "tokens_per_s": round(world * inp.num_tokens / (ms_step * 1e-3), 1),
+        "prefill_ms": round(k_ms, 4),
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak_kind": peak_kind, "kernel": "pa_prefill"},
+        "cpu_baseline": cpu,
+        "e2e": None if e2e is None else {
+            "value": round(e2e["value"], 2), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+            "ms_per_step": round(e2e["ms"], 4)},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def prefill_e2e(args, cfg, pa, dev):
+    """Public API with host buffers: each step copies the new tokens' q, k, v,
+    their slots and the tables from pinned memory, runs append + prefill and
+    reads the output back."""
+    inp = wl.make_prefill_inputs(cfg, seed=args.seed + 11, device=dev)
+    host = {k: getattr(inp, k).cpu().pin_memory() for k in
+            ("q", "key_new", "value_new", "slot_mapping", "block_tables", "context_lens",
+             "query_start")}
+    devb = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+    out = torch.empty_like(inp.q)
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    maxq = inp.max_query_len
+    flops = wl.prefill_flops(cfg, inp.query_start, inp.context_lens)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for k in host:
+            devb[k].copy_(host[k], non_blocking=True)
+        pa.pa_reshape_and_cache(devb["key_new"], devb["value_new"], inp.key_cache,
+                                inp.value_cache, devb["slot_mapping"])
+        pa.pa_prefill(out, devb["q"], inp.key_cache, inp.value_cache, devb["block_tables"],
+                      devb["context_lens"], devb["query_start"], maxq, inp.scale)
+        out_h.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    steps = max(3, min(args.steps, 50))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    e1.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    assert pa.pa_device_status() == 0
+    return {"ms": ms, "value": flops / (ms * 1e-3) / 1e12,
+            "h2d": sum(v.numel() * v.element_size() for v in host.values()),
+            "d2h": out_h.numel() * out_h.element_size()}
+
+
+def run_reference_prefill(args, cfg, rank, world):
+    if rank != 0:
+        return
+    budget = max(1.0, 150.0 / (args.warmup + args.steps))
+    r = prefill_oracle_rate(cfg, args.seed, budget)
+    line = {
+        "impl": "reference", "metric": PREFILL_METRIC, "value": round(r["tflops"], 6),
+        "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * r["seconds"], 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": _prefill_config_dict(cfg, args),
+        "cpu_baseline": {"value": round(r["tflops"], 6), "unit": "TFLOP/s", "cores": r["cores"],
+                         "kind": "oracle", "sample": r["sample"]},
+        "e2e": {"value": round(r["tflops"], 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -504,24 +721,36 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--seqs", type=int, default=0,
                     help="profiling only: a sub-batch of this many sequences of the workload")
+    ap.add_argument("--op", choices=["decode", "prefill"], default="decode",
+                    help="decode: the paged decode step (default); prefill: the chunked-prefill "
+                         "attention step")
+    ap.add_argument("--prefill-workload", default="llama3_8b_gqa_bf16_chunked_prefill",
+                    choices=sorted(wl.PREFILL_CONFIGS))
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    cfg = wl.CONFIGS[args.config]
-    if args.seqs:
-        cfg = _sample_cfg(cfg, args.seqs)
+    if args.op == "prefill":
+        import dataclasses
+        cfg = wl.PREFILL_CONFIGS[args.prefill_workload]
+        if args.seqs:
+            cfg = dataclasses.replace(cfg, num_seqs=min(args.seqs, cfg.num_seqs),
+                                      name=cfg.name + f"_small{args.seqs}")
+    else:
+        cfg = wl.CONFIGS[args.config]
+        if args.seqs:
+            cfg = _sample_cfg(cfg, args.seqs)
     if args.impl == "reference":
-        run_reference(args, cfg, rank, world)
+        (run_reference_prefill if args.op == "prefill" else run_reference)(args, cfg, rank, world)
         return
     if world > 1:
         import datetime
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        run_gpu(args, cfg, rank, world, local_rank)
+        (run_gpu_prefill if args.op == "prefill" else run_gpu)(args, cfg, rank, world, local_rank)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()
