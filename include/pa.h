@@ -260,6 +260,7 @@ pa_status pa_decode_select(int mode);
  *   block_tables [S, MB] int32; context_lens [S] int32;
  *   query_start  [S+1] int32, non-decreasing, query_start[0] = 0.
  *   max_query_len  host int >= every L_s (sizes the grid).
+ *   scale        host float, finite and > 0.
  *   D in {64, 128}; Hq / Hkv in {1, 2, 4, 8, 16}; bs in {8, 16, 32}.
  * Work runs asynchronously on `stream` with no allocation and no workspace.
  * Host checks return PA_ERR_INVALID_ARG / PA_ERR_UNSUPPORTED before anything is

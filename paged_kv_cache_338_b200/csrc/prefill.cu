@@ -190,6 +190,14 @@ __device__ __forceinline__ uint32_t idesc_f16(int ab_bf16, int b_mn_major, int N
            ((uint32_t)b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
 }
 
+// 2^x on the special-function unit (ex2.approx.ftz: relative error about
+// 2^-22, 2^-inf = +0).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 template <int DT> __device__ __forceinline__ uint32_t pack2(float a, float b);
 template <> __device__ __forceinline__ uint32_t pack2<PA_BF16>(float a, float b) {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -199,14 +207,6 @@ template <> __device__ __forceinline__ uint32_t pack2<PA_F16>(float a, float b) 
     __half2 h = __floats2half2_rn(a, b);
     return *reinterpret_cast<uint32_t*>(&h);
 }
-template <int DT> __device__ __forceinline__ float2 unpack2(uint32_t u);
-template <> __device__ __forceinline__ float2 unpack2<PA_BF16>(uint32_t u) {
-    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
-}
-template <> __device__ __forceinline__ float2 unpack2<PA_F16>(uint32_t u) {
-    return __half22float2(*reinterpret_cast<__half2*>(&u));
-}
-
 // Bounded wait by every lane of a warp; the verdict is warp-uniform.  A
 // pipeline wait gives up early once another role has aborted the CTA; a drain
 // wait (honor_abort false) does not, since it guards memory still in flight.
@@ -436,16 +436,20 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             for (int c4 = 0; c4 < kBN / 32; ++c4) tmem_ld32(tS + lrow + (j & 1) * kBN + c4 * 32,
                                                            sv + c4 * 32);
             tmem_wait_ld();
-            const int nv = min(max(limit - j * kBN, 0), kBN);
+            // keys past a row's position (causal bound, or past the tile's last
+            // needed key) become -inf; a tile no row masks skips the compares
+            if ((j + 1) * kBN > c + i0 + 1) {
+                const int nv = limit - j * kBN;
+#pragma unroll
+                for (int k = 0; k < kBN; ++k)
+                    if (k >= nv) sv[k] = -INFINITY;
+            }
             float tmax = -INFINITY;
 #pragma unroll
-            for (int k = 0; k < kBN; ++k) {
-                sv[k] *= sl;
-                if (k < nv) tmax = fmaxf(tmax, sv[k]);
-            }
-            const float m_new = fmaxf(m_use, tmax);
+            for (int k = 0; k < kBN; ++k) tmax = fmaxf(tmax, sv[k]);
+            const float m_new = fmaxf(m_use, tmax * sl);       // scale > 0
             const bool raise = m_new > m_use + kRescaleLog2;
-            const float alpha = raise ? exp2f(m_use - m_new) : 1.f;
+            const float alpha = raise ? ex2(m_use - m_new) : 1.f;
             if (raise) m_use = m_new;
             lsum *= alpha;
             if (j > 0 && __any_sync(~0u, raise)) {
@@ -478,11 +482,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int k = sg * 64 + ch * 8 + 2 * e;
-                        const float a = k < nv ? exp2f(sv[k] - m_use) : 0.f;
-                        const float b = k + 1 < nv ? exp2f(sv[k + 1] - m_use) : 0.f;
+                        const float a = ex2(fmaf(sv[k], sl, -m_use));
+                        const float b = ex2(fmaf(sv[k + 1], sl, -m_use));
+                        lsum += a + b;
                         w[e] = pack2<DT>(a, b);
-                        const float2 rb = unpack2<DT>(w[e]);
-                        lsum += rb.x + rb.y;
                     }
                     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
                                  ::"r"(prow + sg * kSeg + ((ch ^ (r & 7)) << 4)), "r"(w[0]),
@@ -568,7 +571,8 @@ extern "C" pa_status pa_prefill(void* out, const void* q, pa_dtype q_dt, const v
     const int G = Hq / Hkv;
     if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16)
         return fail(PA_ERR_UNSUPPORTED, "group size %d (1, 2, 4, 8 or 16)", G);
-    if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "scale is not finite");
+    if (!std::isfinite(scale) || !(scale > 0.f))
+        return fail(PA_ERR_INVALID_ARG, "scale must be finite and positive");
     if (S == 0 || T == 0 || max_query_len == 0) return PA_OK;
     if (!out || !q || !key_cache || !value_cache || !block_tables || !context_lens ||
         !query_start)

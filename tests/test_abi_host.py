@@ -347,7 +347,7 @@ def test_prefill_host_argument_checks():
     assert call(bs=64) == 2
     assert call(Hq=6, Hkv=2) == 2                 # group 3
     assert call(Hq=7, Hkv=2) == 1                 # not a divisor
-    assert call(scale=float("inf")) == 1
+    assert call(scale=float("inf")) == 1 and call(scale=0.0) == 1 and call(scale=-0.1) == 1
     assert call(out=None) == 1
     assert call(q=24) == 1                        # misaligned
     assert call(S=70000) == 2                     # grid limit
