@@ -4,31 +4,36 @@
 // cache; the keys are gathered block by block through the table as in the
 // decode loop of the same section).
 //
-// One CTA computes a 128-row query tile of one (sequence, kv head): the rows
-// are TQ = 128 / G consecutive new tokens x the G query heads that share the kv
-// head, so K and V tiles are loaded once for the whole group.  Keys run in
-// tiles of 128 (128 / bs blocks, each fetched by its own tensor-map load from
-// the block the table names).  Per key tile j:
+// A query tile is 128 rows: TQ = 128 / G consecutive new tokens x the G query
+// heads that share one kv head, so every K and V tile is loaded once for the
+// whole group.  One CTA computes two adjacent query tiles (A and B) of one
+// (sequence, kv head), so each K/V tile serves 256 rows and the two softmax
+// warpgroups take turns with the tensor core.  Keys run in tiles of 128
+// (128 / bs blocks, each fetched by its own tensor-map load from the block the
+// table names).  Per key tile j and query tile X:
 //
-//   S_j = Q K_j^T         tcgen05.mma, M 128, N 128, K = D; S in tensor memory
-//   P_j = exp2(S_j * scale * log2 e - m)   softmax warps, one row per thread,
-//                                           causal + length mask, rounded to
-//                                           the operand type into shared memory
-//   O  += P_j V_j         tcgen05.mma, M 128, N = D, K 128; O in tensor memory
+//   S_X = Q_X K_j^T       tcgen05.mma, M 128, N 128, K = D, A and B from shared
+//                         memory, S in tensor memory
+//   P_X = exp2(S_X * scale * log2 e - m)   softmax warpgroup X, one row per
+//                         thread, causal + length mask; P is rounded to the
+//                         operand type and written back over S_X in tensor memory
+//   O_X += P_X V_j        tcgen05.mma, M 128, N = D, K 128, A (P) from tensor
+//                         memory, B (V) from shared memory, O in tensor memory
 //
 // The running maximum m is raised only when a tile's maximum exceeds it by
 // more than 8 (in log2 units); O and the running sum are then rescaled in
 // place.  Between raises the probabilities stay below 2^8, so the result is
 // the same softmax (the final division uses the same m for both sums).
 //
-// Warp roles (192 threads): warps 0-3 softmax and epilogue (warp w owns TMEM
-// lanes 32w..32w+31, i.e. query rows), warp 4 loads (tensor-map copies of Q
-// once, then K and V tiles into two-deep rings), warp 5 allocates tensor memory
-// and one of its lanes issues every MMA.  S is double-buffered in tensor
-// memory so S_{j+1} is computed while the softmax warps work on S_j; P is
-// double-buffered in shared memory.  Every wait is bounded (2 s): on timeout
-// the CTA records PA_DEV_WAIT_TIMEOUT with the wait's site, drains its own
-// copies and MMAs, frees its tensor memory and exits.
+// Warp roles (320 threads): warps 0-3 and 4-7 are the softmax and epilogue
+// warpgroups of tiles A and B (warp w reads TMEM lanes 32(w%4)..32(w%4)+31,
+// i.e. its 32 query rows); warp 8 loads (tensor-map copies of the two Q tiles
+// once, then K and V tiles into rings); warp 9 allocates tensor memory and one
+// of its lanes issues every MMA.  Tensor memory: S_A 0..127, O_A 128..255,
+// S_B 256..383, O_B 384..511.  The MMA lane waits for P_X.V to complete before
+// it computes the next S_X into the same columns.  Every wait is bounded (2 s):
+// on timeout the CTA records PA_DEV_WAIT_TIMEOUT with the wait's site, drains
+// its own copies and MMAs, frees its tensor memory and exits.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -45,7 +50,7 @@ using namespace pa::dev;
 constexpr int kBM = 128;          // query rows per tile
 constexpr int kBN = 128;          // keys per tile
 constexpr int kSeg = 16384;       // 128 rows x 128 bytes: one operand segment
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;     // 2 softmax warpgroups, a load warp, an MMA warp
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
 
@@ -56,7 +61,7 @@ struct Params {
     const int32_t* query_start;
     unsigned int* err;
     long long NB;
-    int S, Hq, G, log2G, TQ, MB, bs, log2bs, max_qlen, n_qtiles;
+    int S, Hq, G, log2G, TQ, MB, bs, log2bs, max_qlen, n_pairs;
     float sl;                     // scale * log2(e)
 };
 
@@ -65,14 +70,13 @@ struct Smem {
     static constexpr int NSEG = D / 64;             // 128-byte segments of a row
     static constexpr int ST = D == 64 ? 3 : 2;      // K and V ring depth
     static constexpr int TILE = NSEG * kSeg;        // 128 rows of D elements
-    static constexpr int Q = 0;
-    static constexpr int K = Q + TILE;
+    static constexpr int Q = 0;                     // query tiles A and B
+    static constexpr int K = Q + 2 * TILE;
     static constexpr int V = K + ST * TILE;
-    static constexpr int P = V + ST * TILE;         // two 128 x 128 probability tiles
-    static constexpr int BAR = P + 2 * (kBN / 64) * kSeg;
-    // barriers: q, k_full[ST], k_free[ST], v_full[ST], v_free[ST], s_full[2],
-    // p_full[2], pv_done[2], o_full, drain
-    static constexpr int NBAR = 1 + 4 * ST + 2 + 2 + 2 + 1 + 1;
+    static constexpr int BAR = V + ST * TILE;
+    // barriers: q, k_full[ST], k_free[ST], v_full[ST], v_free[ST], then per
+    // query tile s_full, p_full, pv_done, o_full; drain
+    static constexpr int NBAR = 1 + 4 * ST + 8 + 1;
     static constexpr int TMEM_SLOT = BAR + NBAR * 8;
     static constexpr int ABORT = TMEM_SLOT + 4;
     static constexpr int BYTES = ABORT + 4 + 1024;  // + slack to align the base to 1024
@@ -129,6 +133,28 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
         ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// D (tensor memory, fp32) (+)= A (tensor memory) x B (shared), kind::f16.
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// 16 consecutive 32-bit columns of this thread's lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0],"
+        " {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+          "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]),
+          "r"(r[13]), "r"(r[14]), "r"(r[15])
         : "memory");
 }
 
@@ -240,60 +266,65 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
     using L = Smem<D>;
     constexpr int NSEG = L::NSEG, ST = L::ST;
     const int g = blockIdx.x, s = blockIdx.y;
-    const int qt = p.n_qtiles - 1 - (int)blockIdx.z;      // longest tiles first
+    const int pair = p.n_pairs - 1 - (int)blockIdx.z;     // longest tiles first
 
     const int q0 = p.query_start[s];
     const int Ls = p.query_start[s + 1] - q0;
     const int n = p.context_lens[s];
     if (Ls < 0 || Ls > n || Ls > p.max_qlen || (long long)n > (long long)p.MB * p.bs) {
-        if (qt == 0 && g == 0 && threadIdx.x == 0) atomicOr(p.err, PA_DEV_BAD_CONTEXT);
+        if (pair == 0 && g == 0 && threadIdx.x == 0) atomicOr(p.err, PA_DEV_BAD_CONTEXT);
         return;
     }
-    const int i0 = qt * p.TQ;                 // first new token of this tile
-    if (i0 >= Ls) return;                     // whole CTA: nothing to compute
-    const int c = n - Ls;                     // tokens cached before this chunk
-    const int i1 = min(Ls, i0 + p.TQ);
-    const int kv_len = c + i1;                // the tile's last row sees keys 0..kv_len-1
-    const int nt = (kv_len + kBN - 1) / kBN;
+    const int TQ = p.TQ;
+    const int iA = 2 * pair * TQ, iB = iA + TQ;   // first new token of tiles A and B
+    if (iA >= Ls) return;                         // whole CTA: nothing to compute
+    const bool hasB = iB < Ls;
+    const int c = n - Ls;                         // tokens cached before this chunk
+    const int kvA = c + min(Ls, iB);              // tile A's last row sees keys 0..kvA-1
+    const int kvB = hasB ? c + min(Ls, iB + TQ) : 0;
+    const int ntA = (kvA + kBN - 1) / kBN;
+    const int ntB = (kvB + kBN - 1) / kBN;
+    const int kv_len = hasB ? kvB : kvA;
+    const int nt = hasB ? ntB : ntA;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
     const uint32_t sb = smem_addr(sm);
-    const uint32_t sQ = sb + L::Q, sK = sb + L::K, sV = sb + L::V, sP = sb + L::P;
+    const uint32_t sQ = sb + L::Q, sK = sb + L::K, sV = sb + L::V;
     const uint32_t bar0 = sb + L::BAR;
-    auto q_full = [&]() { return bar0; };
+    const uint32_t q_full = bar0;
     auto k_full = [&](int i) { return bar0 + 8u * (1 + i); };
     auto k_free = [&](int i) { return bar0 + 8u * (1 + ST + i); };
     auto v_full = [&](int i) { return bar0 + 8u * (1 + 2 * ST + i); };
     auto v_free = [&](int i) { return bar0 + 8u * (1 + 3 * ST + i); };
-    auto s_full = [&](int i) { return bar0 + 8u * (1 + 4 * ST + i); };
-    auto p_full = [&](int i) { return bar0 + 8u * (3 + 4 * ST + i); };
-    auto pv_done = [&](int i) { return bar0 + 8u * (5 + 4 * ST + i); };
-    const uint32_t o_full = bar0 + 8u * (7 + 4 * ST);
-    const uint32_t drain = bar0 + 8u * (8 + 4 * ST);
+    auto s_full = [&](int x) { return bar0 + 8u * (1 + 4 * ST + x); };
+    auto p_full = [&](int x) { return bar0 + 8u * (3 + 4 * ST + x); };
+    auto pv_done = [&](int x) { return bar0 + 8u * (5 + 4 * ST + x); };
+    auto o_full = [&](int x) { return bar0 + 8u * (7 + 4 * ST + x); };
+    const uint32_t drain = bar0 + 8u * (9 + 4 * ST);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::ABORT);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        mbar_init(q_full(), 1);
+        mbar_init(q_full, 1);
         for (int i = 0; i < ST; ++i) {
             mbar_init(k_full(i), 1);
             mbar_init(k_free(i), 1);
             mbar_init(v_full(i), 1);
             mbar_init(v_free(i), 1);
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(s_full(i), 1);
-            mbar_init(p_full(i), 128);
-            mbar_init(pv_done(i), 1);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(s_full(x), 1);
+            mbar_init(p_full(x), 128);
+            mbar_init(pv_done(x), 1);
+            mbar_init(o_full(x), 1);
         }
-        mbar_init(o_full, 1);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == 9) {
         tmem_alloc(sb + L::TMEM_SLOT, kTmemCols);
         tmem_relinquish();
     }
@@ -301,19 +332,22 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + L::TMEM_SLOT);
-    const uint32_t tS = tmem, tO = tmem + 2 * kBN;     // S buffers at columns 0, 128; O at 256
+    auto tS = [&](int x) { return tmem + 256u * x; };          // scores, then P over them
+    auto tO = [&](int x) { return tmem + 256u * x + 128u; };   // output accumulator
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ------------------------------------------------------------ loads
         const int bpt = kBN >> p.log2bs;                       // blocks per key tile
-        const int need = (kv_len + p.bs - 1) >> p.log2bs;      // blocks the tile reads
+        const int need = (kv_len + p.bs - 1) >> p.log2bs;      // blocks the CTA reads
         const uint32_t box = (uint32_t)p.bs * 128u;
         if (lane == 0) {
-            mbar_arrive_expect_tx(q_full(), NSEG * kSeg);
-            for (int sg = 0; sg < NSEG; ++sg)
-                tma_load_3d(sQ + sg * kSeg, &tmq, q_full(), sg * 64, g * p.G, q0 + i0);
+            mbar_arrive_expect_tx(q_full, (hasB ? 2 : 1) * NSEG * kSeg);
+            for (int x = 0; x < (hasB ? 2 : 1); ++x)
+                for (int sg = 0; sg < NSEG; ++sg)
+                    tma_load_3d(sQ + x * L::TILE + sg * kSeg, &tmq, q_full, sg * 64, g * p.G,
+                                q0 + (x ? iB : iA));
         }
-        int nk = 0, nvl = 0;                                  // K, V tiles started
+        int nk = 0, nvl = 0;                                   // K, V tiles started
         for (int j = 0; j < nt; ++j) {
             const int st = j % ST;
             const uint32_t par = ((j / ST) & 1) ^ 1;
@@ -354,36 +388,36 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                 warp_wait(v_full(i), (jl / ST) & 1, abort_flag, p.err, 17, false);
             }
         }
-        warp_wait(q_full(), 0, abort_flag, p.err, 17, false);
-    } else if (warp == 5) {
+        warp_wait(q_full, 0, abort_flag, p.err, 17, false);
+    } else if (warp == 9) {
         // ------------------------------------------------------------- MMAs
         constexpr int ABF = DT == PA_BF16 ? 1 : 0;
         const uint32_t id_s = idesc_f16(ABF, 0, kBN);
         const uint32_t id_o = idesc_f16(ABF, 1, D);
-        bool ok = warp_wait(q_full(), 0, abort_flag, p.err, 7);
-        auto issue_s = [&](int j) -> bool {
-            const int st = j % ST;
-            if (!warp_wait(k_full(st), (j / ST) & 1, abort_flag, p.err, 8)) return false;
+        // S_X = Q_X K^T for key tile j (K in ring slot st)
+        auto issue_s = [&](int x, int st) {
             tc_fence_after();
             if (lane == 0) {
-                const uint32_t kb = sK + st * L::TILE;
+                const uint32_t kb = sK + st * L::TILE, qb = sQ + x * L::TILE;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kSeg + (kk & 3) * 32;
-                    tc_mma(tS + (j & 1) * kBN, sdesc(sQ + off, 16), sdesc(kb + off, 16), id_s,
-                           kk > 0);
+                    tc_mma(tS(x), sdesc(qb + off, 16), sdesc(kb + off, 16), id_s, kk > 0);
                 }
-                tc_commit(s_full(j & 1));
-                tc_commit(k_free(st));
+                tc_commit(s_full(x));
             }
             __syncwarp();
-            return true;
         };
-        if (ok) ok = issue_s(0);
+        bool ok = warp_wait(q_full, 0, abort_flag, p.err, 7) &&
+                  warp_wait(k_full(0), 0, abort_flag, p.err, 8);
+        if (ok) {
+            issue_s(0, 0);
+            if (ntB > 0) issue_s(1, 0);
+            if (lane == 0) tc_commit(k_free(0));
+            __syncwarp();
+        }
         for (int j = 0; j < nt && ok; ++j) {
-            if (j + 1 < nt && !(ok = issue_s(j + 1))) break;
-            const int st = j % ST;
-            if (!(ok = warp_wait(p_full(j & 1), (j >> 1) & 1, abort_flag, p.err, 13))) break;
+            const int st = j % ST, st1 = (j + 1) % ST;
             if (!(ok = warp_wait(v_full(st), (j / ST) & 1, abort_flag, p.err, 9))) break;
             const uint32_t vb = sV + st * L::TILE;
             if (j == nt - 1) {
@@ -393,24 +427,42 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                 const int z0 = kv_len - j * kBN;
                 const int chunks = (kBN - z0) * 8;              // 16-byte chunks per segment
                 for (int sg = 0; sg < NSEG; ++sg)
-                    for (int x = lane; x < chunks; x += 32)
+                    for (int xx = lane; xx < chunks; xx += 32)
                         asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};"
-                                     ::"r"(vb + sg * kSeg + z0 * 128 + x * 16), "r"(0) : "memory");
+                                     ::"r"(vb + sg * kSeg + z0 * 128 + xx * 16), "r"(0) : "memory");
                 fence_proxy_async_smem();
                 __syncwarp();
             }
-            tc_fence_after();
-            if (lane == 0) {
-                const uint32_t pb = sP + (j & 1) * (kBN / 64) * kSeg;
+            bool k_next = false;
+            for (int x = 0; x < 2 && ok; ++x) {
+                const int ntx = x ? ntB : ntA;
+                if (j >= ntx) continue;
+                if (!(ok = warp_wait(p_full(x), j & 1, abort_flag, p.err, 13))) break;
+                tc_fence_after();
+                if (lane == 0) {
 #pragma unroll
-                for (int kk = 0; kk < kBN / 16; ++kk) {
-                    const uint32_t aoff = (kk >> 2) * kSeg + (kk & 3) * 32;
-                    tc_mma(tO, sdesc(pb + aoff, 16), sdesc(vb + kk * 16 * 128, kSeg), id_o,
-                           (j > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < kBN / 16; ++kk)
+                        tc_mma_ts(tO(x), tS(x) + kk * 8, sdesc(vb + kk * 16 * 128, kSeg), id_o,
+                                  (j > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit(pv_done(x));
+                    if (j == ntx - 1) tc_commit(o_full(x));
                 }
-                tc_commit(pv_done(j & 1));
+                __syncwarp();
+                if (j + 1 < ntx) {
+                    // the next scores overwrite P_X: wait until P_X.V has read it
+                    if (!k_next) {
+                        if (!(ok = warp_wait(k_full(st1), ((j + 1) / ST) & 1, abort_flag, p.err,
+                                             8)))
+                            break;
+                        k_next = true;
+                    }
+                    if (!(ok = warp_wait(pv_done(x), j & 1, abort_flag, p.err, 14))) break;
+                    issue_s(x, st1);
+                }
+            }
+            if (lane == 0) {
                 tc_commit(v_free(st));
-                if (j == nt - 1) tc_commit(o_full);
+                if (k_next) tc_commit(k_free(st1));
             }
             __syncwarp();
         }
@@ -418,27 +470,30 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
         if (lane == 0) tc_commit(drain);
         __syncwarp();
         warp_wait(drain, 0, abort_flag, p.err, 16, false);
-    } else {
-        // ------------------------------------------------- softmax (rows)
-        const int r = threadIdx.x;                           // row = TMEM lane
-        const int it = i0 + (r >> p.log2G);                  // new-token index of the row
+    } else if (warp < 4 || hasB) {
+        // ---------------------------------------- softmax (rows of tile X)
+        const int x = warp >> 2;
+        const int r = threadIdx.x & 127;                     // row = TMEM lane
+        const int iX = x ? iB : iA;
+        const int kvX = x ? kvB : kvA;
+        const int ntx = x ? ntB : ntA;
+        const int it = iX + (r >> p.log2G);                  // new-token index of the row
         const bool row_ok = it < Ls;
-        const int limit = row_ok ? c + it + 1 : kv_len;      // keys 0..limit-1 are visible
-        const uint32_t lrow = (uint32_t)(warp * 32) << 16;
+        const int limit = row_ok ? c + it + 1 : kvX;         // keys 0..limit-1 are visible
+        const uint32_t lrow = (uint32_t)((warp & 3) * 32) << 16;
         const float sl = p.sl;
         float m_use = -INFINITY, lsum = 0.f;
         bool ok = true;
-        for (int j = 0; j < nt; ++j) {
-            if (!(ok = warp_wait(s_full(j & 1), (j >> 1) & 1, abort_flag, p.err, 12))) break;
+        for (int j = 0; j < ntx; ++j) {
+            if (!(ok = warp_wait(s_full(x), j & 1, abort_flag, p.err, 12))) break;
             tc_fence_after();
             float sv[kBN];
 #pragma unroll
-            for (int c4 = 0; c4 < kBN / 32; ++c4) tmem_ld32(tS + lrow + (j & 1) * kBN + c4 * 32,
-                                                           sv + c4 * 32);
+            for (int c4 = 0; c4 < kBN / 32; ++c4) tmem_ld32(tS(x) + lrow + c4 * 32, sv + c4 * 32);
             tmem_wait_ld();
             // keys past a row's position (causal bound, or past the tile's last
             // needed key) become -inf; a tile no row masks skips the compares
-            if ((j + 1) * kBN > c + i0 + 1) {
+            if ((j + 1) * kBN > c + iX + 1) {
                 const int nv = limit - j * kBN;
 #pragma unroll
                 for (int k = 0; k < kBN; ++k)
@@ -453,51 +508,40 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             if (raise) m_use = m_new;
             lsum *= alpha;
             if (j > 0 && __any_sync(~0u, raise)) {
-                if (!(ok = warp_wait(pv_done((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag, p.err,
-                                     14)))
-                    break;
+                // O_X holds P.V of tiles 0..j-1 once the last of them completes
+                if (!(ok = warp_wait(pv_done(x), (j - 1) & 1, abort_flag, p.err, 14))) break;
                 tc_fence_after();
 #pragma unroll 1
                 for (int c4 = 0; c4 < D / 32; ++c4) {
                     float o[32];
-                    tmem_ld32(tO + lrow + c4 * 32, o);
+                    tmem_ld32(tO(x) + lrow + c4 * 32, o);
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 32; ++i) o[i] *= alpha;
-                    tmem_st32(tO + lrow + c4 * 32, o);
+                    tmem_st32(tO(x) + lrow + c4 * 32, o);
                 }
                 tmem_wait_st();
             }
-            if (j >= 2 && !(ok = warp_wait(pv_done(j & 1), ((j - 2) >> 1) & 1, abort_flag, p.err,
-                                           14)))
-                break;
-            // probabilities, rounded to the operand type, into the 128-byte
-            // swizzled K-major tile the P.V MMA reads
-            const uint32_t prow = sP + (j & 1) * (kBN / 64) * kSeg + r * 128;
+            // probabilities, rounded to the operand type, two per 32-bit
+            // column over the scores they came from (the A operand of P.V)
 #pragma unroll
-            for (int sg = 0; sg < kBN / 64; ++sg) {
+            for (int c16 = 0; c16 < kBN / 32; ++c16) {
+                uint32_t w[16];
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int k = sg * 64 + ch * 8 + 2 * e;
-                        const float a = ex2(fmaf(sv[k], sl, -m_use));
-                        const float b = ex2(fmaf(sv[k + 1], sl, -m_use));
-                        lsum += a + b;
-                        w[e] = pack2<DT>(a, b);
-                    }
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
-                                 ::"r"(prow + sg * kSeg + ((ch ^ (r & 7)) << 4)), "r"(w[0]),
-                                   "r"(w[1]), "r"(w[2]), "r"(w[3])
-                                 : "memory");
+                for (int e = 0; e < 16; ++e) {
+                    const int k = c16 * 32 + 2 * e;
+                    const float a = ex2(fmaf(sv[k], sl, -m_use));
+                    const float b = ex2(fmaf(sv[k + 1], sl, -m_use));
+                    lsum += a + b;
+                    w[e] = pack2<DT>(a, b);
                 }
+                tmem_st16(tS(x) + lrow + c16 * 16, w);
             }
-            fence_proxy_async_smem();
+            tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(p_full(j & 1));
+            mbar_arrive(p_full(x));
         }
-        if (ok) ok = warp_wait(o_full, 0, abort_flag, p.err, 15);
+        if (ok) ok = warp_wait(o_full(x), 0, abort_flag, p.err, 15);
         if (ok) {
             tc_fence_after();
             const float inv = 1.f / lsum;
@@ -507,7 +551,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
 #pragma unroll 1
             for (int c4 = 0; c4 < D / 32; ++c4) {
                 float o[32];
-                tmem_ld32(tO + lrow + c4 * 32, o);
+                tmem_ld32(tO(x) + lrow + c4 * 32, o);
                 tmem_wait_ld();
                 if (row_ok) {
                     uint4* dst = reinterpret_cast<uint4*>(orow + c4 * 64);
@@ -527,7 +571,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
     }
 
     __syncthreads();
-    if (warp == 5) {
+    if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
@@ -582,7 +626,8 @@ extern "C" pa_status pa_prefill(void* out, const void* q, pa_dtype q_dt, const v
         return fail(PA_ERR_INVALID_ARG, "out, q and the caches must be 16-byte aligned");
     const int TQ = pf::kBM / G;
     const long long n_qt = ((long long)max_query_len + TQ - 1) / TQ;
-    if (S > 65535 || n_qt > 65535 || Hkv > 65535)
+    const long long n_pairs = (n_qt + 1) / 2;             // two query tiles per CTA
+    if (S > 65535 || n_pairs > 65535 || Hkv > 65535)
         return fail(PA_ERR_UNSUPPORTED, "grid too large (S %d, query tiles %lld)", S, n_qt);
     if (NB > 0x7fffffffLL) return fail(PA_ERR_INVALID_ARG, "NB must fit int32 block ids");
 
@@ -612,10 +657,10 @@ extern "C" pa_status pa_prefill(void* out, const void* q, pa_dtype q_dt, const v
     p.bs = bs;
     p.log2bs = __builtin_ctz((unsigned)bs);
     p.max_qlen = max_query_len;
-    p.n_qtiles = (int)n_qt;
+    p.n_pairs = (int)n_pairs;
     p.sl = scale * 1.4426950408889634f;
 
-    const dim3 grid((unsigned)Hkv, (unsigned)S, (unsigned)n_qt);
+    const dim3 grid((unsigned)Hkv, (unsigned)S, (unsigned)n_pairs);
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     cudaError_t e;
     if (q_dt == PA_BF16)
