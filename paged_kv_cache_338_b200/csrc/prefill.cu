@@ -25,11 +25,12 @@
 // place.  Between raises the probabilities stay below 2^8, so the result is
 // the same softmax (the final division uses the same m for both sums).
 //
-// Warp roles (320 threads): warps 0-3 and 4-7 are the softmax and epilogue
+// Warp roles (384 threads): warps 0-3 and 4-7 are the softmax and epilogue
 // warpgroups of tiles A and B (warp w reads TMEM lanes 32(w%4)..32(w%4)+31,
 // i.e. its 32 query rows); warp 8 loads (tensor-map copies of the two Q tiles
 // once, then K and V tiles into rings); warp 9 allocates tensor memory and one
-// of its lanes issues every MMA.  Tensor memory: S_A 0..127, O_A 128..255,
+// of its lanes issues every MMA; warps 10-11 only complete the third
+// warpgroup, whose registers go to the softmax warps.  Tensor memory: S_A 0..127, O_A 128..255,
 // S_B 256..383, O_B 384..511.  The MMA lane waits for P_X.V to complete before
 // it computes the next S_X into the same columns.  Every wait is bounded (2 s):
 // on timeout the CTA records PA_DEV_WAIT_TIMEOUT with the wait's site, drains
@@ -50,7 +51,14 @@ using namespace pa::dev;
 constexpr int kBM = 128;          // query rows per tile
 constexpr int kBN = 128;          // keys per tile
 constexpr int kSeg = 16384;       // 128 rows x 128 bytes: one operand segment
-constexpr int kThreads = 320;     // 2 softmax warpgroups, a load warp, an MMA warp
+constexpr int kThreads = 384;     // 2 softmax warpgroups; a load warp, an MMA warp, 2 idle
+// Register split (setmaxnreg): the kernel launches with 384 x 168 registers at
+// most (three warps share each scheduler's 16K).  The softmax warpgroups take
+// 208 each and the third warpgroup gives up to 64: 256 * 208 + 128 * 64 =
+// 61440, which fits any launch allocation of 160 or more per thread.
+constexpr int kRegsSoftmax = 208;
+constexpr int kRegsOther = 64;
+static_assert(256 * kRegsSoftmax + 128 * kRegsOther <= kThreads * 160, "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
 
@@ -101,6 +109,13 @@ __device__ __forceinline__ void tma_load_4d_plain(uint32_t dst, const CUtensorMa
         ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2),
           "r"(c3)
         : "memory");
+}
+
+template <int N> __device__ __forceinline__ void regs_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N> __device__ __forceinline__ void regs_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 __device__ __forceinline__ void tmem_alloc(uint32_t slot, uint32_t cols) {
@@ -337,6 +352,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
 
     if (warp == 8) {
         // ------------------------------------------------------------ loads
+        regs_dec<kRegsOther>();
         const int bpt = kBN >> p.log2bs;                       // blocks per key tile
         const int need = (kv_len + p.bs - 1) >> p.log2bs;      // blocks the CTA reads
         const uint32_t box = (uint32_t)p.bs * 128u;
@@ -391,6 +407,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
         warp_wait(q_full, 0, abort_flag, p.err, 17, false);
     } else if (warp == 9) {
         // ------------------------------------------------------------- MMAs
+        regs_dec<kRegsOther>();
         constexpr int ABF = DT == PA_BF16 ? 1 : 0;
         const uint32_t id_s = idesc_f16(ABF, 0, kBN);
         const uint32_t id_o = idesc_f16(ABF, 1, D);
@@ -470,8 +487,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
         if (lane == 0) tc_commit(drain);
         __syncwarp();
         warp_wait(drain, 0, abort_flag, p.err, 16, false);
+    } else if (warp >= 10) {
+        regs_dec<kRegsOther>();
     } else if (warp < 4 || hasB) {
         // ---------------------------------------- softmax (rows of tile X)
+        regs_inc<kRegsSoftmax>();
         const int x = warp >> 2;
         const int r = threadIdx.x & 127;                     // row = TMEM lane
         const int iX = x ? iB : iA;
@@ -568,6 +588,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             }
         }
         tc_fence_before();
+    } else {
+        regs_inc<kRegsSoftmax>();      // tile B is empty: the warpgroup still takes its share
     }
 
     __syncthreads();
