@@ -519,9 +519,15 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                 for (int k = 0; k < kBN; ++k)
                     if (k >= nv) sv[k] = -INFINITY;
             }
-            float tmax = -INFINITY;
+            // row maximum as 8 independent chains (a single chain of 128
+            // dependent maxima would sit on the critical path)
+            float pm[8];
 #pragma unroll
-            for (int k = 0; k < kBN; ++k) tmax = fmaxf(tmax, sv[k]);
+            for (int i = 0; i < 8; ++i) pm[i] = sv[i];
+#pragma unroll
+            for (int k = 8; k < kBN; ++k) pm[k & 7] = fmaxf(pm[k & 7], sv[k]);
+            const float tmax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                                     fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
             const float m_new = fmaxf(m_use, tmax * sl);       // scale > 0
             const bool raise = m_new > m_use + kRescaleLog2;
             const float alpha = raise ? ex2(m_use - m_new) : 1.f;
@@ -544,6 +550,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             }
             // probabilities, rounded to the operand type, two per 32-bit
             // column over the scores they came from (the A operand of P.V)
+            float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // 8 partial sums
 #pragma unroll
             for (int c16 = 0; c16 < kBN / 32; ++c16) {
                 uint32_t w[16];
@@ -552,11 +559,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                     const int k = c16 * 32 + 2 * e;
                     const float a = ex2(fmaf(sv[k], sl, -m_use));
                     const float b = ex2(fmaf(sv[k + 1], sl, -m_use));
-                    lsum += a + b;
+                    ps[e & 7] += a + b;
                     w[e] = pack2<DT>(a, b);
                 }
                 tmem_st16(tS(x) + lrow + c16 * 16, w);
             }
+            lsum += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(p_full(x));
