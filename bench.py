@@ -389,7 +389,10 @@ def run_gpu(args, cfg, rank, world, local_rank):
 
 
 def run_e2e(args, cfg, pa, dev, part):
-    """Host pool + pinned host buffers + H2D / step / D2H every step."""
+    """Host pool + pinned host buffers + H2D / step / D2H every step, pipelined
+    the way a serving loop runs: the host builds step i + 1's slots and tables
+    while the GPU runs step i; every step's inputs still cross H2D and its
+    output D2H inside the timed region."""
     g = torch.Generator().manual_seed(args.seed + 77)
     inp = wl.make_decode_inputs(cfg, seed=args.seed + 5, device=dev)
     max_ctx = inp.max_ctx + args.warmup + args.steps + 2     # sequences grow one token a step
@@ -437,53 +440,79 @@ def run_e2e(args, cfg, pa, dev, part):
     for name, t in parts:
         offs[name] = total
         total += (t.numel() * t.element_size() + 255) // 256 * 256
-    stage_h = torch.empty(total, dtype=torch.uint8, pin_memory=True)
-    stage_d = torch.empty(total, dtype=torch.uint8, device=dev)
+    # two staging slots: the host fills step i + 1's slot (pool appends, tables)
+    # while the GPU still runs step i; copy streams move inputs in and outputs
+    # out beside the compute stream
+    NSLOT = 2
+    stage_h = [torch.empty(total, dtype=torch.uint8, pin_memory=True) for _ in range(NSLOT)]
+    stage_d = [torch.empty(total, dtype=torch.uint8, device=dev) for _ in range(NSLOT)]
 
     def view(buf, name, like):
         nbytes = like.numel() * like.element_size()
         return buf[offs[name]:offs[name] + nbytes].view(like.dtype).view(like.shape)
 
-    hv = {name: view(stage_h, name, t) for name, t in parts}
-    dv = {name: view(stage_d, name, t) for name, t in parts}
-    hv["q"].copy_(inp.q.cpu())
-    hv["k"].copy_(inp.key_new.cpu())
-    hv["v"].copy_(inp.value_new.cpu())
-    out_h = torch.empty(inp.q.shape, dtype=inp.q.dtype, pin_memory=True)
-    out_d = torch.empty_like(inp.q)
+    hv = [{name: view(stage_h[k], name, t) for name, t in parts} for k in range(NSLOT)]
+    dv = [{name: view(stage_d[k], name, t) for name, t in parts} for k in range(NSLOT)]
+    for k in range(NSLOT):
+        hv[k]["q"].copy_(inp.q.cpu())
+        hv[k]["k"].copy_(inp.key_new.cpu())
+        hv[k]["v"].copy_(inp.value_new.cpu())
+    out_h = [torch.empty(inp.q.shape, dtype=inp.q.dtype, pin_memory=True) for _ in range(NSLOT)]
+    out_d = [torch.empty_like(inp.q) for _ in range(NSLOT)]
     cow_buf = torch.empty((S, 2), dtype=torch.int32)
     ws_bytes = pa.pa_decode_workspace_size(S, Hq, D, max_ctx, part)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
+    h2d_stream = torch.cuda.Stream(device=dev)    # inputs in: never queued behind an output
+    d2h_stream = torch.cuda.Stream(device=dev)    # outputs out
+    inputs_in = [torch.cuda.Event() for _ in range(NSLOT)]   # slot's inputs are on the device
+    kern_done = [torch.cuda.Event() for _ in range(NSLOT)]   # slot's kernels have finished
+    output_out = [torch.cuda.Event() for _ in range(NSLOT)]  # slot's output is on the host
+    used = [False] * NSLOT
     total_bytes = 0
 
-    def step():
-        _, pairs = pool.seq_append_batch(seq_ids, hv["slots"], cow_buf)
-        pool.build_block_tables(seq_ids, MB, hv["tables"], hv["lens"])
-        stage_d.copy_(stage_h, non_blocking=True)
+    def step(i):
+        k = i % NSLOT
+        if used[k]:
+            inputs_in[k].synchronize()         # the copy that read this host slot has finished
+        _, pairs = pool.seq_append_batch(seq_ids, hv[k]["slots"], cow_buf)
+        pool.build_block_tables(seq_ids, MB, hv[k]["tables"], hv[k]["lens"])
+        with torch.cuda.stream(h2d_stream):
+            if used[k]:
+                h2d_stream.wait_event(kern_done[k])    # the device slot's last reader is done
+            stage_d[k].copy_(stage_h[k], non_blocking=True)
+            inputs_in[k].record(h2d_stream)
+        stream.wait_event(inputs_in[k])
+        if used[k]:
+            stream.wait_event(output_out[k])   # the slot's previous output has been read out
         if pairs.numel():
             pa.pa_copy_blocks(kc, vc, pairs)
-        pa.pa_reshape_and_cache(dv["k"], dv["v"], kc, vc, dv["slots"], inp.k_scale, inp.v_scale)
-        pa.pa_decode(out_d, dv["q"], kc, vc, dv["tables"], dv["lens"], max_ctx, inp.scale,
-                     inp.k_scale, inp.v_scale, part, ws if ws_bytes else None)
-        out_h.copy_(out_d, non_blocking=True)
-        nb = algorithmic_bytes(cfg, hv["lens"])
+        pa.pa_reshape_and_cache(dv[k]["k"], dv[k]["v"], kc, vc, dv[k]["slots"], inp.k_scale,
+                                inp.v_scale)
+        pa.pa_decode(out_d[k], dv[k]["q"], kc, vc, dv[k]["tables"], dv[k]["lens"], max_ctx,
+                     inp.scale, inp.k_scale, inp.v_scale, part, ws if ws_bytes else None)
+        kern_done[k].record(stream)
+        with torch.cuda.stream(d2h_stream):
+            d2h_stream.wait_event(kern_done[k])
+            out_h[k].copy_(out_d[k], non_blocking=True)
+            output_out[k].record(d2h_stream)
+        used[k] = True
+        nb = algorithmic_bytes(cfg, hv[k]["lens"])
         return nb["decode"] + nb["append"]
 
-    for _ in range(args.warmup):
-        step()
-        torch.cuda.synchronize()
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ms = 0.0
-    for _ in range(args.steps):
-        e0.record(stream)
-        total_bytes += step()
-        e1.record(stream)
-        e1.synchronize()          # the result is on the host: the step is over
-        ms += e0.elapsed_time(e1)
+    e0.record(stream)
+    for i in range(args.steps):
+        total_bytes += step(args.warmup + i)
+    e1.record(d2h_stream)                     # after the last step's output reached the host
+    e1.synchronize()
+    ms = e0.elapsed_time(e1)
     assert pa.pa_device_status() == 0
     h2d = total
-    d2h = out_h.numel() * out_h.element_size()
+    d2h = out_h[0].numel() * out_h[0].element_size()
     pool.close()
     return {"ms": ms / args.steps, "bytes": total_bytes / args.steps,
             "value": (total_bytes / args.steps) / (ms / args.steps * 1e-3) / 1e9,

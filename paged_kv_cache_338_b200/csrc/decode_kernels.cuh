@@ -517,7 +517,7 @@ __device__ __forceinline__ void mma_block(MmaState<C>& st, uint8_t* ktile_p, uin
     constexpr int CT = S::CT;
     constexpr int MT = BS >= 16 ? BS / 16 : 1;   // token m-tiles of S^T
     const int lane = threadIdx.x & 31;
-    const int gid = lane >> 2, tig = lane & 3;
+    const int gid = lane >> 2;
     const uint32_t ktile = dev::smem_addr(ktile_p);
 
     // ---- S^T = K Q^T --------------------------------------------------------
