@@ -73,6 +73,31 @@ def _peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def _reduce(x: float, dev, op) -> float:
+    """x combined over the ranks of the default process group (x itself when
+    there is none); dev is where the backend takes tensors (cuda for NCCL,
+    cpu for gloo)."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=op)
+    return float(t.item())
+
+
+def max_over_ranks(x: float, dev) -> float:
+    return _reduce(x, dev, torch.distributed.ReduceOp.MAX)
+
+
+def sum_over_ranks(x: float, dev) -> float:
+    return _reduce(x, dev, torch.distributed.ReduceOp.SUM)
+
+
+def whole_job_rate(units: float, ms: float, dev) -> float:
+    """Units all ranks processed per second, over the slowest rank's time: each
+    replica draws its own inputs, so the units differ from rank to rank."""
+    return sum_over_ranks(units, dev) / (max_over_ranks(ms, dev) * 1e-3)
+
+
 def algorithmic_bytes(cfg: wl.DecodeConfig, lens: torch.Tensor) -> dict:
     """Bytes the step must move at minimum (no tail slots, no split-K partials)."""
     e_kv, e_q = wl.elem_bytes(cfg.kv_dtype), wl.elem_bytes(cfg.q_dtype)
@@ -329,19 +354,15 @@ def run_gpu(args, cfg, rank, world, local_rank):
     ms = t0.elapsed_time(t1)
     dec_ms = [a.elapsed_time(b) for a, b in evs]
     dec_avg = sum(dec_ms) / len(dec_ms)
-    if dist:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    value = whole_job_rate(step_bytes * args.steps, ms, dev) / 1e9
+    ms = max_over_ranks(ms, dev)
     ms_step = ms / args.steps
-    value = world * step_bytes / (ms_step * 1e-3) / 1e9
+    seqs_all = sum_over_ranks(S, dev)
 
     # ---- end to end through the public API with host buffers -------------
     e2e = run_e2e(args, cfg, pa, dev, part) if not args.no_e2e else None
-    if dist and e2e is not None:
-        t = torch.tensor([e2e["ms"]], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e["value"] = world * e2e["bytes"] / (float(t.item()) * 1e-3) / 1e9
+    if e2e is not None:
+        e2e["value"] = whole_job_rate(e2e["bytes"], e2e["ms"], dev) / 1e9
 
     if rank != 0:
         return
@@ -370,7 +391,7 @@ def run_gpu(args, cfg, rank, world, local_rank):
         "data": "synthetic",
         "config": _config_dict(cfg, args, part,
                                f"inputs larger than L2 ({kv_gb:.2f} GB of K/V per step), no flush"),
-        "seqs_per_s": round(world * S / (ms_step * 1e-3), 1),
+        "seqs_per_s": round(seqs_all / (ms_step * 1e-3), 1),
         "pct_of_hbm_peak": {"measured_copy": round(100 * value / world / peak, 2),
                             "spec_8000": round(100 * value / world / 8000.0, 2)},
         "decode_ms": round(dec_avg, 4),
@@ -633,17 +654,13 @@ def run_gpu_prefill(args, cfg: wl.PrefillConfig, rank, world, local_rank):
         torch.distributed.barrier()
     ms = t0.elapsed_time(t1)
     k_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
-    if dist:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    value = whole_job_rate(flops * args.steps, ms, dev) / 1e12
+    ms = max_over_ranks(ms, dev)
     ms_step = ms / args.steps
-    value = world * flops / (ms_step * 1e-3) / 1e12
+    tokens_all = sum_over_ranks(inp.num_tokens, dev)
     e2e = None if args.no_e2e else prefill_e2e(args, cfg, pa, dev)
-    if dist and e2e is not None:
-        t = torch.tensor([e2e["ms"]], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e["value"] = world * flops / (float(t.item()) * 1e-3) / 1e12
+    if e2e is not None:
+        e2e["value"] = whole_job_rate(e2e["flops"], e2e["ms"], dev) / 1e12
     if rank != 0:
         return
     peak, peak_kind = _prefill_peak(ms)
@@ -660,7 +677,7 @@ def run_gpu_prefill(args, cfg: wl.PrefillConfig, rank, world, local_rank):
         "data": "synthetic",
         "config": _prefill_config_dict(cfg, args, f"K/V cache {kv_gb:.2f} GB; re-read across "
                                                   f"query tiles, no flush"),
-        "tokens_per_s": round(world * inp.num_tokens / (ms_step * 1e-3), 1),
+        "tokens_per_s": round(tokens_all / (ms_step * 1e-3), 1),
         "prefill_ms": round(k_ms, 4),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
@@ -712,7 +729,7 @@ def prefill_e2e(args, cfg, pa, dev):
     e1.synchronize()
     ms = e0.elapsed_time(e1) / steps
     assert pa.pa_device_status() == 0
-    return {"ms": ms, "value": flops / (ms * 1e-3) / 1e12,
+    return {"ms": ms, "value": flops / (ms * 1e-3) / 1e12, "flops": flops,
             "h2d": sum(v.numel() * v.element_size() for v in host.values()),
             "d2h": out_h.numel() * out_h.element_size()}
 

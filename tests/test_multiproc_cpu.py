@@ -1,0 +1,90 @@
+"""The N > 1 bench path on CPU: two gloo ranks (127.0.0.1) exercise the
+whole-job aggregation bench.py uses under torchrun -- units summed over the
+replicas, time the slowest rank's -- and the reference arm's rank gating (only
+rank 0 runs the oracle and prints)."""
+import json
+import os
+import socket
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank: int, world: int, port: int, out_dir: str):
+    sys.path.insert(0, ROOT)
+    import bench
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    try:
+        res = {
+            "max": bench.max_over_ranks(1.5 + rank, "cpu"),
+            "sum": bench.sum_over_ranks(10.0 * (rank + 1), "cpu"),
+            # rank 0 moved 100 units in 2 ms, rank 1 300 units in 4 ms
+            "rate": bench.whole_job_rate([100.0, 300.0][rank], [2.0, 4.0][rank], "cpu"),
+        }
+        dist.barrier()
+        with open(os.path.join(out_dir, f"rank{rank}.json"), "w") as f:
+            json.dump(res, f)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_whole_job_aggregation_over_two_gloo_ranks(tmp_path):
+    port = _free_port()
+    mp.start_processes(_rank_main, args=(2, port, str(tmp_path)), nprocs=2, join=True,
+                       start_method="spawn")
+    for r in range(2):
+        with open(tmp_path / f"rank{r}.json") as f:
+            res = json.load(f)
+        assert res["max"] == 2.5
+        assert res["sum"] == 30.0
+        assert res["rate"] == pytest.approx(400.0 / 4e-3)
+
+
+def test_single_process_aggregation_is_the_identity():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert not dist.is_initialized()
+    assert bench.max_over_ranks(3.0, "cpu") == 3.0
+    assert bench.whole_job_rate(50.0, 5.0, "cpu") == pytest.approx(10000.0)
+
+
+def _reference_rank(rank: int, world: int, port: int, out_dir: str):
+    sys.path.insert(0, ROOT)
+    import argparse
+    import contextlib
+    import io
+    import bench
+    import workloads as wl
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    try:
+        args = argparse.Namespace(steps=1, warmup=1, seed=2, gpus=world)
+        buf = io.StringIO()
+        cfg = wl.small_variant(wl.CONFIGS[3], 2, 20, 40)
+        with contextlib.redirect_stdout(buf):
+            if rank != 0:
+                bench.run_reference(args, cfg, rank, world)
+        with open(os.path.join(out_dir, f"ref{rank}.txt"), "w") as f:
+            f.write(buf.getvalue())
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_reference_arm_runs_on_rank_zero_only(tmp_path):
+    port = _free_port()
+    mp.start_processes(_reference_rank, args=(2, port, str(tmp_path)), nprocs=2, join=True,
+                       start_method="spawn")
+    assert (tmp_path / "ref1.txt").read_text() == ""      # rank 1 did no work, printed nothing
