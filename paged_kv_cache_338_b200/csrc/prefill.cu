@@ -239,6 +239,35 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// (a * b + c) on a pair of lanes in one instruction (fma.rn.f32x2).
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
+// a + b on a pair of lanes in one instruction (add.rn.f32x2).
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
 template <int DT> __device__ __forceinline__ uint32_t pack2(float a, float b);
 template <> __device__ __forceinline__ uint32_t pack2<PA_BF16>(float a, float b) {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -519,15 +548,15 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                 for (int k = 0; k < kBN; ++k)
                     if (k >= nv) sv[k] = -INFINITY;
             }
-            // row maximum as 8 independent chains (a single chain of 128
-            // dependent maxima would sit on the critical path)
+            // row maximum as 8 independent chains of three-input maxima (a
+            // single chain of dependent maxima would sit on the critical path)
             float pm[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) pm[i] = sv[i];
 #pragma unroll
-            for (int k = 8; k < kBN; ++k) pm[k & 7] = fmaxf(pm[k & 7], sv[k]);
-            const float tmax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                                     fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+            for (int k = 8; k < kBN; k += 2) pm[(k >> 1) & 7] = max3(pm[(k >> 1) & 7], sv[k], sv[k + 1]);
+            const float tmax = fmaxf(max3(pm[0], pm[1], pm[2]),
+                                     fmaxf(max3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7])));
             const float m_new = fmaxf(m_use, tmax * sl);       // scale > 0
             const bool raise = m_new > m_use + kRescaleLog2;
             const float alpha = raise ? ex2(m_use - m_new) : 1.f;
@@ -550,21 +579,24 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             }
             // probabilities, rounded to the operand type, two per 32-bit
             // column over the scores they came from (the A operand of P.V)
-            float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // 8 partial sums
+            // pairs of scores share one packed FMA and one packed add
+            float2 ps[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};   // partial sums
+            const float2 sl2 = make_float2(sl, sl), nm2 = make_float2(-m_use, -m_use);
 #pragma unroll
             for (int c16 = 0; c16 < kBN / 32; ++c16) {
                 uint32_t w[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const int k = c16 * 32 + 2 * e;
-                    const float a = ex2(fmaf(sv[k], sl, -m_use));
-                    const float b = ex2(fmaf(sv[k + 1], sl, -m_use));
-                    ps[e & 7] += a + b;
-                    w[e] = pack2<DT>(a, b);
+                    const float2 xy = fma2(make_float2(sv[k], sv[k + 1]), sl2, nm2);
+                    const float2 pr = make_float2(ex2(xy.x), ex2(xy.y));
+                    ps[e & 3] = add2(ps[e & 3], pr);
+                    w[e] = pack2<DT>(pr.x, pr.y);
                 }
                 tmem_st16(tS(x) + lrow + c16 * 16, w);
             }
-            lsum += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+            lsum += ((ps[0].x + ps[0].y) + (ps[1].x + ps[1].y)) +
+                    ((ps[2].x + ps[2].y) + (ps[3].x + ps[3].y));
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(p_full(x));
