@@ -108,7 +108,9 @@ def algorithmic_bytes(cfg: wl.DecodeConfig, lens: torch.Tensor) -> dict:
     tables = int(((n + bs - 1) // bs).sum()) * 4 + S * 4
     decode = kv + qo + tables
     append = S * Hkv * D * 2 * (e_q + e_kv) + S * 8
-    return {"decode": decode, "append": append, "kv": kv}
+    # with a shared prefix every sequence reads the same prefix blocks: count them once
+    unique_kv = kv - max(S - 1, 0) * cfg.prefix_tokens * Hkv * D * 2 * e_kv
+    return {"decode": decode, "append": append, "kv": kv, "unique_kv": unique_kv}
 
 
 def _pci_id(dev: int) -> str | None:
@@ -316,6 +318,8 @@ def run_gpu(args, cfg, rank, world, local_rank):
     step_bytes = nbytes["decode"] + nbytes["append"]
 
     def step(ev=None):
+        if ev is not None:
+            ev[2].record(stream)
         if pairs.numel():
             pa.pa_copy_blocks(kc, vc, pairs)
         pa.pa_reshape_and_cache(inp.key_new, inp.value_new, kc, vc, inp.slot_mapping,
@@ -338,7 +342,7 @@ def run_gpu(args, cfg, rank, world, local_rank):
         torch.distributed.barrier()
     torch.cuda.synchronize()
     clocks = ClockSampler(local_rank)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3))
            for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks.mark_start()
@@ -352,8 +356,9 @@ def run_gpu(args, cfg, rank, world, local_rank):
     if dist:
         torch.distributed.barrier()
     ms = t0.elapsed_time(t1)
-    dec_ms = [a.elapsed_time(b) for a, b in evs]
+    dec_ms = [a.elapsed_time(b) for a, b, _ in evs]
     dec_avg = sum(dec_ms) / len(dec_ms)
+    app_avg = sum(c.elapsed_time(a) for a, _, c in evs) / len(evs)
     value = whole_job_rate(step_bytes * args.steps, ms, dev) / 1e9
     ms = max_over_ranks(ms, dev)
     ms_step = ms / args.steps
@@ -395,6 +400,8 @@ def run_gpu(args, cfg, rank, world, local_rank):
         "pct_of_hbm_peak": {"measured_copy": round(100 * value / world / peak, 2),
                             "spec_8000": round(100 * value / world / 8000.0, 2)},
         "decode_ms": round(dec_avg, 4),
+        "append_cow_ms": round(app_avg, 4),
+        "unique_kv_gbs": round(nbytes["unique_kv"] / (dec_avg * 1e-3) / 1e9, 1),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
                      "peak_kind": peak_kind, "kernel": "pa_decode (partition + merge)"},
@@ -638,7 +645,7 @@ def run_gpu_prefill(args, cfg: wl.PrefillConfig, rank, world, local_rank):
         torch.distributed.barrier()
     torch.cuda.synchronize()
     clocks = ClockSampler(local_rank)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3))
            for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks.mark_start()
