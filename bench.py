@@ -309,13 +309,29 @@ def run_gpu(args, cfg, rank, world, local_rank):
         cfg.partition or pa.pa_decode_suggest_partition(cfg.num_kv_heads, cfg.block_size,
                                                         inp.context_lens.cpu()))
     max_ctx = inp.max_ctx
-    ws_bytes = pa.pa_decode_workspace_size(S, Hq, D, max_ctx, part)
+    shared = bool(cfg.prefix_tokens) and not args.no_shared_prefix
+    if shared:      # the batch's tables start with the same prefix blocks
+        ws_bytes = pa.pa_decode_shared_prefix_workspace_size(
+            S, Hq, cfg.num_kv_heads, D, cfg.block_size, max_ctx, cfg.prefix_tokens,
+            inp.key_cache.dtype)
+        part = 0
+    else:
+        ws_bytes = pa.pa_decode_workspace_size(S, Hq, D, max_ctx, part)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
     out = torch.empty_like(inp.q)
     kc, vc = inp.key_cache, inp.value_cache
     pairs = inp.copy_pairs
     nbytes = algorithmic_bytes(cfg, inp.context_lens.cpu())
     step_bytes = nbytes["decode"] + nbytes["append"]
+
+    def decode(out_t, q_t, tables, lens):
+        if shared:
+            pa.pa_decode_shared_prefix(out_t, q_t, kc, vc, tables, lens, max_ctx, inp.scale,
+                                       cfg.prefix_tokens, ws if ws_bytes else None,
+                                       inp.k_scale, inp.v_scale)
+        else:
+            pa.pa_decode(out_t, q_t, kc, vc, tables, lens, max_ctx, inp.scale, inp.k_scale,
+                         inp.v_scale, part, ws if ws_bytes else None)
 
     def step(ev=None):
         if ev is not None:
@@ -326,12 +342,14 @@ def run_gpu(args, cfg, rank, world, local_rank):
                                 inp.k_scale, inp.v_scale)
         if ev is not None:
             ev[0].record(stream)
-        pa.pa_decode(out, inp.q, kc, vc, inp.block_tables, inp.context_lens, max_ctx, inp.scale,
-                     inp.k_scale, inp.v_scale, part, ws if ws_bytes else None)
+        decode(out, inp.q, inp.block_tables, inp.context_lens)
         if ev is not None:
             ev[1].record(stream)
 
-    launches_per_step = (1 if pairs.numel() else 0) + 1 + 1 + (1 if ws_bytes else 0)
+    # copy-on-write, append, then the decode's kernels: [prefix conversion (fp8),
+    # prefix records,] partitions [, merge]
+    launches_per_step = (1 if pairs.numel() else 0) + 1 + 1 + (1 if ws_bytes else 0) + (
+        (2 if cfg.kv_dtype == "fp8_e4m3" else 1) if shared else 0)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -375,7 +393,7 @@ def run_gpu(args, cfg, rank, world, local_rank):
     achieved = nbytes["decode"] / (dec_avg * 1e-3) / 1e9
     traffic = None
     prof = os.path.join(ROOT, "profiles", f"traffic_{cfg.name}.json")
-    if os.path.exists(prof):
+    if os.path.exists(prof) and not shared:       # the capture is of the plain decode
         try:
             with open(prof) as f:
                 pj = json.load(f)
@@ -404,7 +422,9 @@ def run_gpu(args, cfg, rank, world, local_rank):
         "unique_kv_gbs": round(nbytes["unique_kv"] / (dec_avg * 1e-3) / 1e9, 1),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "peak_kind": peak_kind, "kernel": "pa_decode (partition + merge)"},
+                     "peak_kind": peak_kind,
+                     "kernel": "pa_decode_shared_prefix (prefix records + partitions + merge)"
+                     if shared else "pa_decode (partition + merge)"},
         "cpu_baseline": cpu,
         "e2e": None if e2e is None else {
             "value": round(e2e["value"], 2), "unit": "GB/s",
@@ -488,7 +508,12 @@ def run_e2e(args, cfg, pa, dev, part):
     out_h = [torch.empty(inp.q.shape, dtype=inp.q.dtype, pin_memory=True) for _ in range(NSLOT)]
     out_d = [torch.empty_like(inp.q) for _ in range(NSLOT)]
     cow_buf = torch.empty((S, 2), dtype=torch.int32)
-    ws_bytes = pa.pa_decode_workspace_size(S, Hq, D, max_ctx, part)
+    shared = bool(cfg.prefix_tokens) and not args.no_shared_prefix
+    if shared:      # every table starts with the owner's prefix blocks
+        ws_bytes = pa.pa_decode_shared_prefix_workspace_size(
+            S, Hq, cfg.num_kv_heads, D, bs, max_ctx, cfg.prefix_tokens, kc.dtype)
+    else:
+        ws_bytes = pa.pa_decode_workspace_size(S, Hq, D, max_ctx, part)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     h2d_stream = torch.cuda.Stream(device=dev)    # inputs in: never queued behind an output
@@ -517,8 +542,13 @@ def run_e2e(args, cfg, pa, dev, part):
             pa.pa_copy_blocks(kc, vc, pairs)
         pa.pa_reshape_and_cache(dv[k]["k"], dv[k]["v"], kc, vc, dv[k]["slots"], inp.k_scale,
                                 inp.v_scale)
-        pa.pa_decode(out_d[k], dv[k]["q"], kc, vc, dv[k]["tables"], dv[k]["lens"], max_ctx,
-                     inp.scale, inp.k_scale, inp.v_scale, part, ws if ws_bytes else None)
+        if shared:
+            pa.pa_decode_shared_prefix(out_d[k], dv[k]["q"], kc, vc, dv[k]["tables"],
+                                       dv[k]["lens"], max_ctx, inp.scale, cfg.prefix_tokens,
+                                       ws if ws_bytes else None, inp.k_scale, inp.v_scale)
+        else:
+            pa.pa_decode(out_d[k], dv[k]["q"], kc, vc, dv[k]["tables"], dv[k]["lens"], max_ctx,
+                         inp.scale, inp.k_scale, inp.v_scale, part, ws if ws_bytes else None)
         kern_done[k].record(stream)
         with torch.cuda.stream(d2h_stream):
             d2h_stream.wait_event(kern_done[k])
@@ -774,6 +804,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--seqs", type=int, default=0,
                     help="profiling only: a sub-batch of this many sequences of the workload")
+    ap.add_argument("--no-shared-prefix", action="store_true",
+                    help="shared-prefix workload: time pa_decode instead of pa_decode_shared_prefix")
     ap.add_argument("--op", choices=["decode", "prefill"], default="decode",
                     help="decode: the paged decode step (default); prefill: the chunked-prefill "
                          "attention step")

@@ -237,6 +237,39 @@ pa_status pa_decode_noalloc(void* out, const void* q, pa_dtype q_dt,
 pa_status pa_decode_select(int mode);
 
 /*
+ * Shared-prefix ("cascade") decode -- "01. PagedAttention 详解" §6 and summary
+ * (requests share the blocks of a common prefix by reference) and
+ * "PagedAttention 机制" §5.3.2.  Computes exactly what pa_decode computes (up
+ * to rounding order), for a batch whose block tables all start with the same
+ * prefix_tokens / bs physical blocks (those of row 0): the prefix is attended
+ * once, by a tensor-core pass with every sequence's queries as rows, and each
+ * sequence's private suffix by the decode kernel; the split-K merge combines
+ * them.  A sequence whose table does not start with row 0's prefix blocks, or
+ * that holds fewer than prefix_tokens tokens, is still computed correctly
+ * (it reads its own prefix blocks).
+ *
+ * Arguments are pa_decode's (same layouts, ownership, errors) except:
+ *   prefix_tokens  host int, a positive multiple of bs, <= MB * bs;
+ *   workspace      device scratch of pa_decode_shared_prefix_workspace_size()
+ *                  bytes, 16-byte aligned (no initialisation needed).
+ * Supported: q f16 or bf16 with a cache of the same type or fp8-e4m3 (the
+ * prefix is converted exactly to the q type inside the workspace), D in
+ * {64, 128} (128 for fp8: a row is at least 128 bytes), Hq / Hkv in
+ * {1, 2, 4, 8, 16}, bs in {8, 16, 32}; scale > 0.
+ * With max_ctx < prefix_tokens it is a plain pa_decode.
+ */
+pa_status pa_decode_shared_prefix_workspace_size(int S, int Hq, int Hkv, int D, int bs,
+                                                 int max_ctx, int prefix_tokens,
+                                                 pa_dtype cache_dt, size_t* bytes);
+pa_status pa_decode_shared_prefix(void* out, const void* q, pa_dtype q_dt, const void* key_cache,
+                                  const void* value_cache, pa_dtype cache_dt,
+                                  const int32_t* block_tables, int MB,
+                                  const int32_t* context_lens, int S, int Hq, int Hkv, int D,
+                                  int bs, int64_t NB, int max_ctx, float scale, float k_scale,
+                                  float v_scale, int prefix_tokens, void* workspace,
+                                  size_t workspace_bytes, pa_stream_t stream);
+
+/*
  * Prefill / chunked-prefill attention over the paged cache -- "01. PagedAttention
  * 详解" §4, prefill: the N new tokens' K and V are first written through the
  * block table (pa_reshape_and_cache with their slots), then attention runs

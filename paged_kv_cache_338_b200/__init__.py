@@ -22,6 +22,7 @@ __all__ = [
     "PaError", "lib", "pa_version", "pa_last_error", "pa_device_status",
     "pa_reshape_and_cache", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_size",
     "pa_decode_suggest_partition", "pa_decode_select", "pa_decode_noalloc", "pa_prefill",
+    "pa_decode_shared_prefix", "pa_decode_shared_prefix_workspace_size",
     "BlockPool",
     "PA_DEV_BAD_SLOT", "PA_DEV_BAD_BLOCK", "PA_DEV_WAIT_TIMEOUT", "PA_DEV_BAD_CONTEXT",
 ]
@@ -79,6 +80,9 @@ def lib() -> ctypes.CDLL:
         "pa_decode": ([P, P, I, P, P, I, P, I, P, I, I, I, I, I, I64, I, F, F, F, I, P, SZ, P], I),
         "pa_decode_noalloc": ([P, P, I, P, P, I, P, I, P, I, I, I, I, I, I64, I, F, F, F, I, P], I),
         "pa_prefill": ([P, P, I, P, P, I, P, I, P, P, I, I, I, I, I, I, I64, I, F, P], I),
+        "pa_decode_shared_prefix_workspace_size": ([I, I, I, I, I, I, I, I, ctypes.POINTER(SZ)], I),
+        "pa_decode_shared_prefix": ([P, P, I, P, P, I, P, I, P, I, I, I, I, I, I64, I, F, F, F, I,
+                                     P, SZ, P], I),
         "pa_pool_create": ([I64, I, ctypes.POINTER(P)], I),
         "pa_pool_destroy": ([P], None),
         "pa_pool_alloc": ([P, ctypes.POINTER(I32)], I),
@@ -243,6 +247,36 @@ def pa_decode_noalloc(out: torch.Tensor, q: torch.Tensor, key_cache: torch.Tenso
                                    _ptr(context_lens), S, Hq, Hkv, D, bs, NB, int(max_ctx),
                                    float(scale), float(k_scale), float(v_scale), int(partition),
                                    _stream(stream)))
+
+
+def pa_decode_shared_prefix_workspace_size(S: int, Hq: int, Hkv: int, D: int, bs: int,
+                                           max_ctx: int, prefix_tokens: int, cache_dtype) -> int:
+    n = ctypes.c_size_t()
+    dt = _TORCH_DT[cache_dtype] if isinstance(cache_dtype, torch.dtype) else int(cache_dtype)
+    _check(lib().pa_decode_shared_prefix_workspace_size(S, Hq, Hkv, D, bs, int(max_ctx),
+                                                         int(prefix_tokens), dt, ctypes.byref(n)))
+    return n.value
+
+
+def pa_decode_shared_prefix(out: torch.Tensor, q: torch.Tensor, key_cache: torch.Tensor,
+                            value_cache: torch.Tensor, block_tables: torch.Tensor,
+                            context_lens: torch.Tensor, max_ctx: int, scale: float,
+                            prefix_tokens: int, workspace: Optional[torch.Tensor],
+                            k_scale: float = 1.0, v_scale: float = 1.0, stream=None) -> None:
+    """pa_decode for a batch whose tables start with the same prefix blocks (row
+    0's first prefix_tokens / bs): the prefix is attended once for all queries."""
+    S, Hq, D = q.shape
+    NB, bs, Hkv, _ = key_cache.shape
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise PaError(1, "block_tables and context_lens must be int32")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().pa_decode_shared_prefix(_ptr(out), _ptr(q), _dt(q), _ptr(key_cache),
+                                         _ptr(value_cache), _dt(key_cache), _ptr(block_tables),
+                                         MB, _ptr(context_lens), S, Hq, Hkv, D, bs, NB,
+                                         int(max_ctx), float(scale), float(k_scale),
+                                         float(v_scale), int(prefix_tokens), _ptr(workspace),
+                                         ws_bytes, _stream(stream)))
 
 
 def pa_prefill(out: torch.Tensor, q: torch.Tensor, key_cache: torch.Tensor,

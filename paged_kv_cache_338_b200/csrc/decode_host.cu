@@ -3,6 +3,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <mutex>
@@ -91,9 +92,6 @@ extern "C" pa_status pa_decode_workspace_size(int S, int Hq, int D, int max_ctx,
     if (S < 0 || Hq <= 0 || D <= 0 || max_ctx < 0 || partition < PA_PARTITION_BALANCED)
         return fail(PA_ERR_INVALID_ARG, "negative or zero size");
     if (partition == PA_PARTITION_BALANCED) {
-        *bytes = balanced_bytes(S, Hq, D, 1 > Hq ? Hq : 1) > balanced_bytes(S, Hq, D, Hq)
-                     ? balanced_bytes(S, Hq, D, 1)
-                     : balanced_bytes(S, Hq, D, Hq);
         // the bound over every heads-per-item value (gc divides Hq, gc <= 16)
         size_t mx = 0;
         for (int gc = 1; gc <= 16 && gc <= Hq; gc *= 2)
@@ -139,13 +137,16 @@ extern "C" pa_status pa_decode_select(int mode) {
     return PA_OK;
 }
 
-extern "C" pa_status pa_decode(void* out, const void* q, pa_dtype q_dt, const void* key_cache,
-                               const void* value_cache, pa_dtype cache_dt,
-                               const int32_t* block_tables, int MB, const int32_t* context_lens,
-                               int S, int Hq, int Hkv, int D, int bs, int64_t NB, int max_ctx,
-                               float scale, float k_scale, float v_scale, int partition,
-                               void* workspace, size_t workspace_bytes, pa_stream_t stream) {
-    clear_error();
+// pa_decode, plus the shared-prefix decode's two switches: the first
+// `prefix_parts` partitions of sequences whose table starts with row 0's
+// blocks were written by the prefix kernel, and every record goes through the
+// workspace (force_ws) so the merge sees them all.
+pa_status pa::decode_impl(void* out, const void* q, pa_dtype q_dt, const void* key_cache,
+                          const void* value_cache, pa_dtype cache_dt, const int32_t* block_tables,
+                          int MB, const int32_t* context_lens, int S, int Hq, int Hkv, int D,
+                          int bs, int64_t NB, int max_ctx, float scale, float k_scale,
+                          float v_scale, int partition, void* workspace, size_t workspace_bytes,
+                          pa_stream_t stream, int prefix_parts, int force_ws) {
     if (!valid_dtype(q_dt) || !valid_dtype(cache_dt)) return fail(PA_ERR_INVALID_ARG, "bad dtype");
     if (S < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || MB < 0 || NB <= 0 || max_ctx < 0 ||
         partition < PA_PARTITION_BALANCED)
@@ -178,7 +179,13 @@ extern "C" pa_status pa_decode(void* out, const void* q, pa_dtype q_dt, const vo
         return fail(PA_ERR_INVALID_ARG, "caches, q and out must be 16-byte aligned");
     if (MB == 0 && max_ctx > 0) return fail(PA_ERR_INVALID_ARG, "MB == 0 with max_ctx > 0");
 
-    const int64_t max_parts = balanced ? 1 : parts_for(max_ctx, partition);
+    // shared-prefix decode: records up to partition prefix_parts exist even
+    // when max_ctx ends inside the prefix (irregular sequences write them)
+    const int64_t max_parts = balanced ? 1
+                              : prefix_parts > 0
+                                  ? std::max<int64_t>(parts_for(max_ctx, partition), prefix_parts + 1)
+                                  : parts_for(max_ctx, partition);
+    const int64_t grid_parts = prefix_parts > 0 ? max_parts - prefix_parts : max_parts;
     if (max_parts > 65535 || (int64_t)Hkv * G > 65535)
         return fail(PA_ERR_UNSUPPORTED, "too many partitions or heads for the grid");
     const int sel = g_select.load();
@@ -187,7 +194,9 @@ extern "C" pa_status pa_decode(void* out, const void* q, pa_dtype q_dt, const vo
     const int gc = use_mma ? G : gc_simt;
     size_t need = 0;
     if (balanced) need = balanced_bytes(S, Hq, D, gc);
+    else if (force_ws) need = (size_t)S * Hq * max_parts * (sizeof(float) * 2 + sizeof(float) * D);
     else pa_decode_workspace_size(S, Hq, D, max_ctx, partition, &need);
+    if (force_ws && balanced) return fail(PA_ERR_INVALID_ARG, "the balanced grid has no prefix mode");
     if (need && (!workspace || workspace_bytes < need || !aligned16(workspace)))
         return fail(PA_ERR_INVALID_ARG, "workspace needs %zu bytes, 16-byte aligned (got %zu)",
                     need, workspace_bytes);
@@ -211,8 +220,10 @@ extern "C" pa_status pa_decode(void* out, const void* q, pa_dtype q_dt, const vo
     p.Hkv = Hkv;
     p.MB = MB;
     p.max_parts = (int)max_parts;
-    p.part_blocks = max_parts > 1 ? partition / bs : 0;
-    p.part_tokens = max_parts > 1 ? partition : 0;
+    p.part_blocks = max_parts > 1 || force_ws ? partition / bs : 0;
+    p.part_tokens = max_parts > 1 || force_ws ? partition : 0;
+    p.prefix_parts = prefix_parts;
+    p.force_ws = force_ws ? 1 : 0;
     p.max_ctx = max_ctx;
     p.evict_first = (sel & 2) ? 1 : 0;
     p.heads_fastest = (sel & 4) ? 1 : 0;
@@ -231,7 +242,7 @@ extern "C" pa_status pa_decode(void* out, const void* q, pa_dtype q_dt, const vo
         p.ws_ml = reinterpret_cast<float2*>(w + align16(items * sizeof(int2)));
         p.ws_o = reinterpret_cast<float*>(w + align16(items * sizeof(int2)) +
                                           align16(rows * sizeof(float2)));
-    } else if (max_parts > 1) {
+    } else if (max_parts > 1 || force_ws) {
         p.ws_ml = static_cast<float2*>(workspace);
         p.ws_o = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                           sizeof(float2) * (size_t)S * Hq * max_parts);
@@ -253,8 +264,8 @@ extern "C" pa_status pa_decode(void* out, const void* q, pa_dtype q_dt, const vo
         L.num_sms = (dev >= 0 && dev < 256 && sms[dev] > 0) ? sms[dev] : 148;
     }
     const int chunks = L.mma ? 1 : G / L.gc;
-    L.grid = p.heads_fastest ? dim3((unsigned)(Hkv * chunks), (unsigned)max_parts, (unsigned)S)
-                             : dim3((unsigned)max_parts, (unsigned)(Hkv * chunks), (unsigned)S);
+    L.grid = p.heads_fastest ? dim3((unsigned)(Hkv * chunks), (unsigned)grid_parts, (unsigned)S)
+                             : dim3((unsigned)grid_parts, (unsigned)(Hkv * chunks), (unsigned)S);
     L.stream = reinterpret_cast<cudaStream_t>(stream);
 
     cudaError_t e;
@@ -266,9 +277,21 @@ extern "C" pa_status pa_decode(void* out, const void* q, pa_dtype q_dt, const vo
     }
     if (e == cudaErrorNotSupported) return fail(PA_ERR_UNSUPPORTED, "no kernel for this shape");
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
-    if (max_parts > 1 || balanced) {
+    if (max_parts > 1 || balanced || force_ws) {
         e = launch_merge(p, q_dt, D, Hq, S, L.stream);
         if (e != cudaSuccess) return cuda_fail(e, "split-K merge launch");
     }
     return PA_OK;
+}
+
+extern "C" pa_status pa_decode(void* out, const void* q, pa_dtype q_dt, const void* key_cache,
+                               const void* value_cache, pa_dtype cache_dt,
+                               const int32_t* block_tables, int MB, const int32_t* context_lens,
+                               int S, int Hq, int Hkv, int D, int bs, int64_t NB, int max_ctx,
+                               float scale, float k_scale, float v_scale, int partition,
+                               void* workspace, size_t workspace_bytes, pa_stream_t stream) {
+    clear_error();
+    return decode_impl(out, q, q_dt, key_cache, value_cache, cache_dt, block_tables, MB,
+                       context_lens, S, Hq, Hkv, D, bs, NB, max_ctx, scale, k_scale, v_scale,
+                       partition, workspace, workspace_bytes, stream, 0, 0);
 }

@@ -66,6 +66,9 @@ struct Params {
     int64_t NB;
     float qk_scale;              // scale * k_scale * log2(e)
     float v_scale;
+    int prefix_parts;            // shared-prefix decode: leading partitions another kernel
+                                 // wrote for sequences whose table starts with row 0's blocks
+    int force_ws;                // 1: every sequence's partials go through the workspace
 };
 
 // Record a wait that gave up, with the site that gave up (bits 16-23).
@@ -758,7 +761,7 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     const int G = p.Hq / p.Hkv;
     const int gc = C::MMA ? G : C::GC;          // query heads this CTA serves
     const int chunks = G / gc;                  // head chunks per kv head
-    const int part = p.heads_fastest ? blockIdx.y : blockIdx.x;
+    int part = p.heads_fastest ? blockIdx.y : blockIdx.x;
     const int hc = p.heads_fastest ? blockIdx.x : blockIdx.y;
     const int kvh = hc / chunks;
     const int h0 = kvh * G + (hc % chunks) * gc;
@@ -766,7 +769,40 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     const int n = checked_len(p, s, C::BS);
     const int nblk_all = (n + C::BS - 1) / C::BS;
     int blk0 = 0, nblk = nblk_all, nparts = 1;
-    if (p.part_blocks > 0) {
+    if (p.prefix_parts > 0) {
+        // Shared-prefix decode: the grid covers the partitions past the
+        // prefix (grid index i is partition prefix_parts + i); the prefix
+        // kernel wrote partitions 0 .. prefix_parts-1 of every sequence.  A
+        // sequence whose table does not start with row 0's prefix blocks, or
+        // that is shorter than the prefix, is irregular: its first CTA covers
+        // the prefix and partition prefix_parts in one record (partition 0)
+        // and empties records 1 .. prefix_parts.
+        const int k = p.prefix_parts;
+        const int pb = k * p.part_blocks;
+        int irregular = 0;
+        if (part == 0) {
+            irregular = n < pb * C::BS;
+            for (int i = threadIdx.x; i < pb && !irregular; i += blockDim.x)
+                irregular = p.block_tables[(size_t)s * p.MB + i] != p.block_tables[i];
+            irregular = __syncthreads_or(irregular);
+        }
+        if (irregular) {
+            for (int idx = threadIdx.x; idx < gc * k * (C::D + 1); idx += blockDim.x) {
+                const int g = idx / (k * (C::D + 1)), rest = idx % (k * (C::D + 1));
+                const int pp = 1 + rest / (C::D + 1), d = rest % (C::D + 1);
+                const size_t row = ((size_t)s * p.Hq + h0 + g) * p.max_parts + pp;
+                if (d == C::D) p.ws_ml[row] = make_float2(-INFINITY, 0.f);
+                else p.ws_o[row * C::D + d] = 0.f;
+            }
+            nblk = min((k + 1) * p.part_blocks, nblk_all);   // blk0 = 0, record 0
+        } else {
+            part += k;
+            blk0 = part * p.part_blocks;
+            nblk = min(p.part_blocks, nblk_all - blk0);
+            if (nblk <= 0) return;              // this sequence has fewer partitions
+        }
+        nparts = 2;                             // records always go through the workspace
+    } else if (p.part_blocks > 0) {
         blk0 = part * p.part_blocks;
         nblk = min(p.part_blocks, nblk_all - blk0);
         nparts = max(1, (nblk_all + p.part_blocks - 1) / p.part_blocks);
@@ -856,7 +892,7 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
             }
         }
         const int h = h0 + g;
-        if (nparts == 1) {
+        if (nparts == 1 && !p.force_ws) {
             dev::store_out<C::QT>(p.out, ((size_t)s * p.Hq + h) * C::D + d,
                                   L > 0.f ? (O / L) * p.v_scale : 0.f);
         } else {
@@ -1201,11 +1237,13 @@ __global__ void __launch_bounds__(kMergeWarps * 32) decode_merge(const Params p,
         stride = (size_t)gc;
     } else {
         count = min(p.max_parts, (n + p.part_tokens - 1) / p.part_tokens);
-        if (count <= 1) return;                       // CTA-uniform: written by the partition kernel
+        if (count <= 1 && !p.force_ws) return;        // CTA-uniform: written by the partition kernel
         row0 = ((size_t)s * p.Hq + (head_ok ? h : 0)) * p.max_parts;
         stride = 1;
     }
-    const bool live = head_ok && count > 1;           // count <= 1: written by the partition kernel
+    // count <= 1: written by the partition kernel, unless every record goes
+    // through the workspace (then count 0, an empty sequence, writes zeros)
+    const bool live = head_ok && (count > 1 || (p.force_ws && !p.balanced));
     if (sub == 0) s_live[hl] = live ? 1 : 0;
 
     float mx = -INFINITY;

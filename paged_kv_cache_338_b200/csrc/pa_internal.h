@@ -6,6 +6,8 @@
 #include <cstdio>
 #include <string>
 
+#include <vector_types.h>
+
 #include "pa.h"
 
 namespace pa {
@@ -33,5 +35,26 @@ unsigned int* device_error_word();
 
 // Translate a CUDA runtime error into PA_ERR_CUDA with context.
 pa_status cuda_fail(int err, const char* what);
+
+// pa_decode with the shared-prefix switches (decode_host.cu): partitions
+// below prefix_parts of sequences whose table starts with row 0's blocks are
+// left to the caller's prefix records; force_ws sends every record through
+// the workspace and always runs the merge.
+pa_status decode_impl(void* out, const void* q, pa_dtype q_dt, const void* key_cache,
+                      const void* value_cache, pa_dtype cache_dt, const int32_t* block_tables,
+                      int MB, const int32_t* context_lens, int S, int Hq, int Hkv, int D, int bs,
+                      int64_t NB, int max_ctx, float scale, float k_scale, float v_scale,
+                      int partition, void* workspace, size_t workspace_bytes, pa_stream_t stream,
+                      int prefix_parts, int force_ws);
+
+// Shared-prefix decode, step 1 (prefill.cu): split-K records (m, l, o * v_scale)
+// of partitions 0 .. prefix_tokens / chunk_tokens - 1 of every (sequence, head),
+// from K/V in 16-bit `dt` at k_src / v_src (blocks named by table_row0, or
+// blocks 0.. when it is NULL).  sl = scale * k_scale * log2(e).
+pa_status prefix_records(const void* q, pa_dtype dt, const void* k_src, const void* v_src,
+                         int64_t src_blocks, const int32_t* table_row0, int S, int Hq, int Hkv,
+                         int D, int bs, int prefix_tokens, int chunk_tokens, float sl,
+                         float v_scale, float2* ws_ml, float* ws_o, int max_parts,
+                         pa_stream_t stream);
 
 }  // namespace pa

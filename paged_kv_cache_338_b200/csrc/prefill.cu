@@ -70,7 +70,16 @@ struct Params {
     unsigned int* err;
     long long NB;
     int S, Hq, G, log2G, TQ, MB, bs, log2bs, max_qlen, n_pairs;
-    float sl;                     // scale * log2(e)
+    float sl;                     // scale * log2(e) (* k_scale in prefix mode)
+    // prefix mode (shared-prefix decode): the query rows are the S decode
+    // queries, grid y is the prefix chunk, keys are chunk_tokens of the
+    // prefix (row 0 of block_tables, or blocks 0.. of a converted copy when
+    // identity_blocks), no causal mask, and the result is the split-K record
+    // (m, l, o * v_scale) of partition `chunk` of every (sequence, head)
+    int prefix, chunk_tokens, identity_blocks, max_parts;
+    float2* ws_ml;
+    float* ws_o;
+    float v_scale;
 };
 
 template <int D>
@@ -309,23 +318,31 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                const __grid_constant__ CUtensorMap tmv, const Params p) {
     using L = Smem<D>;
     constexpr int NSEG = L::NSEG, ST = L::ST;
-    const int g = blockIdx.x, s = blockIdx.y;
+    const int g = blockIdx.x;
     const int pair = p.n_pairs - 1 - (int)blockIdx.z;     // longest tiles first
+    const bool pfx = p.prefix != 0;
+    const int s = pfx ? 0 : (int)blockIdx.y;              // the sequence (table row)
+    const int chunk = pfx ? (int)blockIdx.y : 0;          // prefix mode: the key chunk
 
-    const int q0 = p.query_start[s];
-    const int Ls = p.query_start[s + 1] - q0;
-    const int n = p.context_lens[s];
-    if (Ls < 0 || Ls > n || Ls > p.max_qlen || (long long)n > (long long)p.MB * p.bs) {
-        if (pair == 0 && g == 0 && threadIdx.x == 0) atomicOr(p.err, PA_DEV_BAD_CONTEXT);
-        return;
+    int q0 = 0, Ls = p.S, c = 0;
+    if (!pfx) {
+        q0 = p.query_start[s];
+        Ls = p.query_start[s + 1] - q0;
+        const int n = p.context_lens[s];
+        if (Ls < 0 || Ls > n || Ls > p.max_qlen || (long long)n > (long long)p.MB * p.bs) {
+            if (pair == 0 && g == 0 && threadIdx.x == 0) atomicOr(p.err, PA_DEV_BAD_CONTEXT);
+            return;
+        }
+        c = n - Ls;                               // tokens cached before this chunk
     }
     const int TQ = p.TQ;
-    const int iA = 2 * pair * TQ, iB = iA + TQ;   // first new token of tiles A and B
+    const int iA = 2 * pair * TQ, iB = iA + TQ;   // first new token (row group) of tiles A and B
     if (iA >= Ls) return;                         // whole CTA: nothing to compute
     const bool hasB = iB < Ls;
-    const int c = n - Ls;                         // tokens cached before this chunk
-    const int kvA = c + min(Ls, iB);              // tile A's last row sees keys 0..kvA-1
-    const int kvB = hasB ? c + min(Ls, iB + TQ) : 0;
+    // keys each tile needs (causal: its last row's position + 1; prefix: the chunk)
+    const int kvA = pfx ? p.chunk_tokens : c + min(Ls, iB);
+    const int kvB = !hasB ? 0 : pfx ? p.chunk_tokens : c + min(Ls, iB + TQ);
+    const int blk_base = pfx ? chunk * (p.chunk_tokens >> p.log2bs) : 0;
     const int ntA = (kvA + kBN - 1) / kBN;
     const int ntB = (kvB + kBN - 1) / kBN;
     const int kv_len = hasB ? kvB : kvA;
@@ -399,7 +416,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             const int lb = j * bpt + lane;
             const bool want = lane < bpt && lb < need;
             int id = -1;
-            if (want) id = p.block_tables[(size_t)s * p.MB + lb];
+            if (want)
+                id = p.identity_blocks ? blk_base + lb
+                                       : p.block_tables[(size_t)s * p.MB + blk_base + lb];
             const bool valid = want && id >= 0 && (long long)id < p.NB;
             if (want && !valid) atomicOr(p.err, PA_DEV_BAD_BLOCK);
             const uint32_t bytes = (uint32_t)__popc(__ballot_sync(~0u, valid)) * NSEG * box;
@@ -528,7 +547,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
         const int ntx = x ? ntB : ntA;
         const int it = iX + (r >> p.log2G);                  // new-token index of the row
         const bool row_ok = it < Ls;
-        const int limit = row_ok ? c + it + 1 : kvX;         // keys 0..limit-1 are visible
+        const int limit = row_ok && !pfx ? c + it + 1 : kvX;  // keys 0..limit-1 are visible
         const uint32_t lrow = (uint32_t)((warp & 3) * 32) << 16;
         const float sl = p.sl;
         float m_use = -INFINITY, lsum = 0.f;
@@ -542,7 +561,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             tmem_wait_ld();
             // keys past a row's position (causal bound, or past the tile's last
             // needed key) become -inf; a tile no row masks skips the compares
-            if ((j + 1) * kBN > c + iX + 1) {
+            if ((j + 1) * kBN > (pfx ? kvX : c + iX + 1)) {
                 const int nv = limit - j * kBN;
 #pragma unroll
                 for (int k = 0; k < kBN; ++k)
@@ -602,7 +621,28 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             mbar_arrive(p_full(x));
         }
         if (ok) ok = warp_wait(o_full(x), 0, abort_flag, p.err, 15);
-        if (ok) {
+        if (ok && pfx) {
+            // the split-K record of partition `chunk`: running maximum (log2
+            // units), sum, and the unnormalised sum of weighted values
+            tc_fence_after();
+            const int h = g * p.G + (r & (p.G - 1));
+            const size_t row = ((size_t)it * p.Hq + h) * p.max_parts + chunk;
+            float* dst = p.ws_o + row * D;
+#pragma unroll 1
+            for (int c4 = 0; c4 < D / 32; ++c4) {
+                float o[32];
+                tmem_ld32(tO(x) + lrow + c4 * 32, o);
+                tmem_wait_ld();
+                if (row_ok) {
+#pragma unroll
+                    for (int v = 0; v < 8; ++v)
+                        reinterpret_cast<float4*>(dst + c4 * 32)[v] =
+                            make_float4(o[4 * v] * p.v_scale, o[4 * v + 1] * p.v_scale,
+                                        o[4 * v + 2] * p.v_scale, o[4 * v + 3] * p.v_scale);
+                }
+            }
+            if (row_ok) p.ws_ml[row] = make_float2(m_use, lsum);
+        } else if (ok) {
             tc_fence_after();
             const float inv = 1.f / lsum;
             const int h = g * p.G + (r & (p.G - 1));
@@ -658,6 +698,65 @@ cudaError_t launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorM
 
 using pa::fail;
 
+// Shared-prefix decode, step 1 (declared in pa_internal.h): the split-K
+// records of the prefix partitions of every (sequence, head), from one pass
+// of the tensor-core kernel in prefix mode.
+pa_status pa::prefix_records(const void* q, pa_dtype dt, const void* k_src, const void* v_src,
+                             int64_t src_blocks, const int32_t* table_row0, int S, int Hq,
+                             int Hkv, int D, int bs, int prefix_tokens, int chunk_tokens,
+                             float sl, float v_scale, float2* ws_ml, float* ws_o, int max_parts,
+                             pa_stream_t stream) {
+    const int G = Hq / Hkv;
+    const int TQ = pf::kBM / G;
+    const long long n_qt = ((long long)S + TQ - 1) / TQ;
+    const long long n_pairs = (n_qt + 1) / 2;
+    const int chunks = prefix_tokens / chunk_tokens;
+    if (n_pairs > 65535 || chunks > 65535 || Hkv > 65535)
+        return fail(PA_ERR_UNSUPPORTED, "prefix grid too large");
+    CUtensorMap mq, mk, mv;
+    pa_status st = pa::make_rows_map(&mq, q, dt, S, Hq, D, G, TQ);
+    if (st) return st;
+    st = pa::make_cache_map(&mk, k_src, dt, src_blocks, bs, Hkv, D);
+    if (st) return st;
+    st = pa::make_cache_map(&mv, v_src, dt, src_blocks, bs, Hkv, D);
+    if (st) return st;
+    unsigned int* err = pa::device_error_word();
+    if (!err) return PA_ERR_CUDA;
+    pf::Params p = {};
+    p.block_tables = table_row0;
+    p.err = err;
+    p.NB = src_blocks;
+    p.S = S;
+    p.Hq = Hq;
+    p.G = G;
+    p.log2G = __builtin_ctz((unsigned)G);
+    p.TQ = TQ;
+    p.MB = 0;
+    p.bs = bs;
+    p.log2bs = __builtin_ctz((unsigned)bs);
+    p.max_qlen = S;
+    p.n_pairs = (int)n_pairs;
+    p.sl = sl;
+    p.prefix = 1;
+    p.chunk_tokens = chunk_tokens;
+    p.identity_blocks = table_row0 ? 0 : 1;
+    p.max_parts = max_parts;
+    p.ws_ml = ws_ml;
+    p.ws_o = ws_o;
+    p.v_scale = v_scale;
+    const dim3 grid((unsigned)Hkv, (unsigned)chunks, (unsigned)n_pairs);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (dt == PA_BF16)
+        e = D == 64 ? pf::launch<PA_BF16, 64>(mq, mk, mv, p, grid, cs)
+                    : pf::launch<PA_BF16, 128>(mq, mk, mv, p, grid, cs);
+    else
+        e = D == 64 ? pf::launch<PA_F16, 64>(mq, mk, mv, p, grid, cs)
+                    : pf::launch<PA_F16, 128>(mq, mk, mv, p, grid, cs);
+    if (e != cudaSuccess) return pa::cuda_fail(e, "prefix kernel launch");
+    return PA_OK;
+}
+
 extern "C" pa_status pa_prefill(void* out, const void* q, pa_dtype q_dt, const void* key_cache,
                                 const void* value_cache, pa_dtype cache_dt,
                                 const int32_t* block_tables, int MB, const int32_t* context_lens,
@@ -703,7 +802,7 @@ extern "C" pa_status pa_prefill(void* out, const void* q, pa_dtype q_dt, const v
     unsigned int* err = pa::device_error_word();
     if (!err) return PA_ERR_CUDA;
 
-    pf::Params p;
+    pf::Params p = {};
     p.out = out;
     p.block_tables = block_tables;
     p.context_lens = context_lens;

@@ -355,3 +355,36 @@ def test_prefill_host_argument_checks():
     assert call(S=0, out=None, q=None) == 0
     assert call(T=0, out=None, q=None) == 0
     assert call(maxq=0, out=None) == 0
+
+
+def test_shared_prefix_host_argument_checks():
+    L = pa.lib()
+    # (out, q, q_dt, kc, vc, cache_dt, bt, MB, lens, S, Hq, Hkv, D, bs, NB, max_ctx, scale,
+    #  k_scale, v_scale, prefix, ws, ws_bytes, stream)
+    base = [16, 16, 2, 16, 16, 2, 16, 64, 16, 4, 32, 8, 128, 16, 100, 2000, 0.1, 1.0, 1.0, 512,
+            16, 1 << 30, None]
+    names = ["out", "q", "q_dt", "kc", "vc", "cache_dt", "bt", "MB", "lens", "S", "Hq", "Hkv",
+             "D", "bs", "NB", "max_ctx", "scale", "ks", "vs", "prefix", "ws", "wsb", "st"]
+
+    def call(**kw):
+        a = list(base)
+        for k, v in kw.items():
+            a[names.index(k)] = v
+        return L.pa_decode_shared_prefix(*a)
+
+    assert call(q_dt=0, cache_dt=0) == 2            # fp32
+    assert call(cache_dt=3, D=64) == 2              # fp8 rows of 64 bytes
+    assert call(D=256) == 2
+    assert call(prefix=100) == 1                    # not a multiple of bs
+    assert call(prefix=64 * 16 + 16) == 1           # beyond MB * bs
+    assert call(Hq=24, Hkv=8) == 2                  # group 3
+    assert call(scale=0.0) == 1
+    assert call(S=0, out=None) == 0
+    assert call(ws=None) == 1 and "workspace" in pa.pa_last_error()
+    n = pa.pa_decode_shared_prefix_workspace_size(4, 32, 8, 128, 16, 2000, 512, torch.bfloat16)
+    assert n == -(-(4 * 32 * 8 * (8 + 4 * 128)) // 256) * 256      # 8 partitions of 256 tokens
+    n8 = pa.pa_decode_shared_prefix_workspace_size(4, 32, 8, 128, 16, 2000, 512,
+                                                   torch.float8_e4m3fn)
+    assert n8 == n + 2 * 512 * 8 * 128 * 2                          # + 16-bit K, V prefix copies
+    assert pa.pa_decode_shared_prefix_workspace_size(4, 32, 8, 128, 16, 300, 512,
+                                                     torch.bfloat16) == 0   # plain decode
