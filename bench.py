@@ -346,10 +346,15 @@ def run_gpu(args, cfg, rank, world, local_rank):
         if ev is not None:
             ev[1].record(stream)
 
-    # copy-on-write, append, then the decode's kernels: [prefix conversion (fp8),
-    # prefix records,] partitions [, merge]
-    launches_per_step = (1 if pairs.numel() else 0) + 1 + 1 + (1 if ws_bytes else 0) + (
-        (2 if cfg.kv_dtype == "fp8_e4m3" else 1) if shared else 0)
+    # copy-on-write, append, then the decode's kernels: partitions [+ merge];
+    # shared prefix: [fp8 conversion +] prefix records + partitions [+ merge
+    # when a suffix can exceed 4096 tokens]
+    if shared:
+        dec_launches = (1 if cfg.kv_dtype == "fp8_e4m3" else 0) + 1 + 1 + (
+            1 if max_ctx - cfg.prefix_tokens > 4096 else 0)
+    else:
+        dec_launches = 1 + (1 if ws_bytes else 0)
+    launches_per_step = (1 if pairs.numel() else 0) + 1 + dec_launches
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()

@@ -146,7 +146,8 @@ pa_status pa::decode_impl(void* out, const void* q, pa_dtype q_dt, const void* k
                           int MB, const int32_t* context_lens, int S, int Hq, int Hkv, int D,
                           int bs, int64_t NB, int max_ctx, float scale, float k_scale,
                           float v_scale, int partition, void* workspace, size_t workspace_bytes,
-                          pa_stream_t stream, int prefix_parts, int force_ws) {
+                          pa_stream_t stream, int prefix_parts, int force_ws,
+                          int fuse_prefix_blocks) {
     if (!valid_dtype(q_dt) || !valid_dtype(cache_dt)) return fail(PA_ERR_INVALID_ARG, "bad dtype");
     if (S < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || MB < 0 || NB <= 0 || max_ctx < 0 ||
         partition < PA_PARTITION_BALANCED)
@@ -181,11 +182,13 @@ pa_status pa::decode_impl(void* out, const void* q, pa_dtype q_dt, const void* k
 
     // shared-prefix decode: records up to partition prefix_parts exist even
     // when max_ctx ends inside the prefix (irregular sequences write them)
+    const bool fuse = fuse_prefix_blocks > 0;
     const int64_t max_parts = balanced ? 1
+                              : fuse ? prefix_parts            // the prefix records only
                               : prefix_parts > 0
                                   ? std::max<int64_t>(parts_for(max_ctx, partition), prefix_parts + 1)
                                   : parts_for(max_ctx, partition);
-    const int64_t grid_parts = prefix_parts > 0 ? max_parts - prefix_parts : max_parts;
+    const int64_t grid_parts = fuse ? 1 : prefix_parts > 0 ? max_parts - prefix_parts : max_parts;
     if (max_parts > 65535 || (int64_t)Hkv * G > 65535)
         return fail(PA_ERR_UNSUPPORTED, "too many partitions or heads for the grid");
     const int sel = g_select.load();
@@ -194,7 +197,7 @@ pa_status pa::decode_impl(void* out, const void* q, pa_dtype q_dt, const void* k
     const int gc = use_mma ? G : gc_simt;
     size_t need = 0;
     if (balanced) need = balanced_bytes(S, Hq, D, gc);
-    else if (force_ws) need = (size_t)S * Hq * max_parts * (sizeof(float) * 2 + sizeof(float) * D);
+    else if (force_ws || fuse) need = (size_t)S * Hq * max_parts * (sizeof(float) * 2 + sizeof(float) * D);
     else pa_decode_workspace_size(S, Hq, D, max_ctx, partition, &need);
     if (force_ws && balanced) return fail(PA_ERR_INVALID_ARG, "the balanced grid has no prefix mode");
     if (need && (!workspace || workspace_bytes < need || !aligned16(workspace)))
@@ -220,10 +223,11 @@ pa_status pa::decode_impl(void* out, const void* q, pa_dtype q_dt, const void* k
     p.Hkv = Hkv;
     p.MB = MB;
     p.max_parts = (int)max_parts;
-    p.part_blocks = max_parts > 1 || force_ws ? partition / bs : 0;
-    p.part_tokens = max_parts > 1 || force_ws ? partition : 0;
+    p.part_blocks = !fuse && (max_parts > 1 || force_ws) ? partition / bs : 0;
+    p.part_tokens = !fuse && (max_parts > 1 || force_ws) ? partition : 0;
     p.prefix_parts = prefix_parts;
     p.force_ws = force_ws ? 1 : 0;
+    p.fuse_prefix_blocks = fuse_prefix_blocks;
     p.max_ctx = max_ctx;
     p.evict_first = (sel & 2) ? 1 : 0;
     p.heads_fastest = (sel & 4) ? 1 : 0;
@@ -242,7 +246,7 @@ pa_status pa::decode_impl(void* out, const void* q, pa_dtype q_dt, const void* k
         p.ws_ml = reinterpret_cast<float2*>(w + align16(items * sizeof(int2)));
         p.ws_o = reinterpret_cast<float*>(w + align16(items * sizeof(int2)) +
                                           align16(rows * sizeof(float2)));
-    } else if (max_parts > 1 || force_ws) {
+    } else if (max_parts > 1 || force_ws || fuse) {
         p.ws_ml = static_cast<float2*>(workspace);
         p.ws_o = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                           sizeof(float2) * (size_t)S * Hq * max_parts);
@@ -277,7 +281,7 @@ pa_status pa::decode_impl(void* out, const void* q, pa_dtype q_dt, const void* k
     }
     if (e == cudaErrorNotSupported) return fail(PA_ERR_UNSUPPORTED, "no kernel for this shape");
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
-    if (max_parts > 1 || balanced || force_ws) {
+    if (!fuse && (max_parts > 1 || balanced || force_ws)) {
         e = launch_merge(p, q_dt, D, Hq, S, L.stream);
         if (e != cudaSuccess) return cuda_fail(e, "split-K merge launch");
     }
@@ -293,5 +297,5 @@ extern "C" pa_status pa_decode(void* out, const void* q, pa_dtype q_dt, const vo
     clear_error();
     return decode_impl(out, q, q_dt, key_cache, value_cache, cache_dt, block_tables, MB,
                        context_lens, S, Hq, Hkv, D, bs, NB, max_ctx, scale, k_scale, v_scale,
-                       partition, workspace, workspace_bytes, stream, 0, 0);
+                       partition, workspace, workspace_bytes, stream, 0, 0, 0);
 }

@@ -69,6 +69,9 @@ struct Params {
     int prefix_parts;            // shared-prefix decode: leading partitions another kernel
                                  // wrote for sequences whose table starts with row 0's blocks
     int force_ws;                // 1: every sequence's partials go through the workspace
+    int fuse_prefix_blocks;      // > 0: shared-prefix decode with one CTA per (sequence, kv
+                                 // head) over the suffix past this many blocks; its epilogue
+                                 // merges the prefix_parts prefix records and writes the output
 };
 
 // Record a wait that gave up, with the site that gave up (bits 16-23).
@@ -769,7 +772,22 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     const int n = checked_len(p, s, C::BS);
     const int nblk_all = (n + C::BS - 1) / C::BS;
     int blk0 = 0, nblk = nblk_all, nparts = 1;
-    if (p.prefix_parts > 0) {
+    bool fuse_records = false;
+    if (p.fuse_prefix_blocks > 0) {
+        // A sequence whose table starts with row 0's prefix blocks (and that
+        // holds the whole prefix) reads only its suffix here and merges the
+        // prefix kernel's records in the epilogue; any other reads everything.
+        const int pb = p.fuse_prefix_blocks;
+        int irregular = n < pb * C::BS;
+        for (int i = threadIdx.x; i < pb && !irregular; i += blockDim.x)
+            irregular = p.block_tables[(size_t)s * p.MB + i] != p.block_tables[i];
+        irregular = __syncthreads_or(irregular);
+        if (!irregular) {
+            blk0 = pb;
+            nblk = nblk_all - pb;               // may be 0: the prefix alone
+            fuse_records = true;
+        }
+    } else if (p.prefix_parts > 0) {
         // Shared-prefix decode: the grid covers the partitions past the
         // prefix (grid index i is partition prefix_parts + i); the prefix
         // kernel wrote partitions 0 .. prefix_parts-1 of every sequence.  A
@@ -892,7 +910,22 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
             }
         }
         const int h = h0 + g;
-        if (nparts == 1 && !p.force_ws) {
+        if (fuse_records) {
+            // combine with the prefix records (o already times v_scale there)
+            O *= p.v_scale;
+            for (int pp = 0; pp < p.prefix_parts; ++pp) {
+                const size_t row = ((size_t)s * p.Hq + h) * p.max_parts + pp;
+                const float2 ml = p.ws_ml[row];
+                const float Mn = fmaxf(M, ml.x);
+                if (Mn == -INFINITY) continue;
+                const float a = exp2f(M - Mn), b = exp2f(ml.x - Mn);
+                L = L * a + ml.y * b;
+                O = O * a + p.ws_o[row * C::D + d] * b;
+                M = Mn;
+            }
+            dev::store_out<C::QT>(p.out, ((size_t)s * p.Hq + h) * C::D + d,
+                                  L > 0.f ? O / L : 0.f);
+        } else if (nparts == 1 && !p.force_ws) {
             dev::store_out<C::QT>(p.out, ((size_t)s * p.Hq + h) * C::D + d,
                                   L > 0.f ? (O / L) * p.v_scale : 0.f);
         } else {

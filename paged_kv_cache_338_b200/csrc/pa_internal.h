@@ -39,13 +39,15 @@ pa_status cuda_fail(int err, const char* what);
 // pa_decode with the shared-prefix switches (decode_host.cu): partitions
 // below prefix_parts of sequences whose table starts with row 0's blocks are
 // left to the caller's prefix records; force_ws sends every record through
-// the workspace and always runs the merge.
+// the workspace and always runs the merge.  With fuse_prefix_blocks > 0 one
+// CTA per (sequence, kv head) reads the suffix past that many blocks and
+// merges the prefix_parts records itself (no merge kernel).
 pa_status decode_impl(void* out, const void* q, pa_dtype q_dt, const void* key_cache,
                       const void* value_cache, pa_dtype cache_dt, const int32_t* block_tables,
                       int MB, const int32_t* context_lens, int S, int Hq, int Hkv, int D, int bs,
                       int64_t NB, int max_ctx, float scale, float k_scale, float v_scale,
                       int partition, void* workspace, size_t workspace_bytes, pa_stream_t stream,
-                      int prefix_parts, int force_ws);
+                      int prefix_parts, int force_ws, int fuse_prefix_blocks);
 
 // Shared-prefix decode, step 1 (prefill.cu): split-K records (m, l, o * v_scale)
 // of partitions 0 .. prefix_tokens / chunk_tokens - 1 of every (sequence, head),

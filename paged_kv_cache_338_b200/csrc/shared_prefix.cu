@@ -12,11 +12,14 @@
 //   2. the prefix kernel: for every (sequence, query head), the record
 //      (m, l, o) of each prefix chunk, with all sequences' queries as the
 //      rows of 128-row tensor-core tiles (prefill kernel, prefix mode);
-//   3. the decode partition kernel over the private suffixes (partitions of
-//      the chunk size past the prefix); a sequence whose table does not start
-//      with row 0's prefix blocks, or that is shorter than the prefix, also
-//      computes its prefix partitions itself, over the prefix kernel's records;
+//   3. the decode kernel over the private suffixes.  Suffixes of up to 4096
+//      tokens: one CTA per (sequence, kv head) reads the whole suffix and
+//      merges the prefix records in its epilogue.  Longer: partitions of the
+//      chunk size past the prefix, then
 //   4. the split-K merge of all records.
+//   Either way a sequence whose table does not start with row 0's prefix
+//   blocks, or that is shorter than the prefix, reads its own prefix blocks
+//   (and, split, blanks the prefix kernel's records for it).
 // The result is pa_decode's, up to rounding order.
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
@@ -75,12 +78,21 @@ int chunk_for(int prefix_tokens) {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Partition records per (sequence, head): those max_ctx needs, and at least
-// one past the prefix (an irregular sequence's first suffix CTA writes it).
+// Suffixes of at most this many tokens are read by one CTA per (sequence, kv
+// head), which also merges the prefix records (no merge kernel); longer ones
+// are split into chunk-sized partitions and merged by the split-K merge.
+constexpr int kFusedSuffixMax = 4096;
+
+bool fused(int max_ctx, int prefix_tokens) { return max_ctx - prefix_tokens <= kFusedSuffixMax; }
+
+// Records per (sequence, head): fused, the prefix chunks; split, those max_ctx
+// needs and at least one past the prefix (an irregular sequence's first
+// suffix CTA writes it).
 int64_t parts(int max_ctx, int chunk, int prefix_tokens) {
+    const int64_t k = prefix_tokens / chunk;
+    if (fused(max_ctx, prefix_tokens)) return k;
     const int64_t need = max_ctx <= chunk ? 1 : ((int64_t)max_ctx + chunk - 1) / chunk;
-    const int64_t k1 = prefix_tokens / chunk + 1;
-    return need > k1 ? need : k1;
+    return need > k + 1 ? need : k + 1;
 }
 
 }  // namespace
@@ -140,7 +152,7 @@ extern "C" pa_status pa_decode_shared_prefix(void* out, const void* q, pa_dtype 
     if (max_ctx < prefix_tokens)        // no sequence can hold the prefix: a plain decode
         return pa::decode_impl(out, q, q_dt, key_cache, value_cache, cache_dt, block_tables, MB,
                                context_lens, S, Hq, Hkv, D, bs, NB, max_ctx, scale, k_scale,
-                               v_scale, 0, nullptr, 0, stream, 0, 0);
+                               v_scale, 0, nullptr, 0, stream, 0, 0, 0);
     if (!out || !q || !key_cache || !value_cache || !block_tables || !context_lens)
         return fail(PA_ERR_INVALID_ARG, "NULL pointer");
     size_t need = 0;
@@ -192,7 +204,12 @@ extern "C" pa_status pa_decode_shared_prefix(void* out, const void* q, pa_dtype 
                             prefix_tokens, chunk, sl, cache_dt == PA_FP8_E4M3 ? v_scale : 1.f,
                             ws_ml, ws_o, (int)mp, stream);
     if (st) return st;
+    if (fused(max_ctx, prefix_tokens))
+        return pa::decode_impl(out, q, q_dt, key_cache, value_cache, cache_dt, block_tables, MB,
+                               context_lens, S, Hq, Hkv, D, bs, NB, max_ctx, scale, k_scale,
+                               v_scale, chunk, workspace, rec_bytes, stream, prefix_tokens / chunk,
+                               0, prefix_tokens / bs);
     return pa::decode_impl(out, q, q_dt, key_cache, value_cache, cache_dt, block_tables, MB,
                            context_lens, S, Hq, Hkv, D, bs, NB, max_ctx, scale, k_scale, v_scale,
-                           chunk, workspace, rec_bytes, stream, prefix_tokens / chunk, 1);
+                           chunk, workspace, rec_bytes, stream, prefix_tokens / chunk, 1, 0);
 }

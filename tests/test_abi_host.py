@@ -381,10 +381,15 @@ def test_shared_prefix_host_argument_checks():
     assert call(scale=0.0) == 1
     assert call(S=0, out=None) == 0
     assert call(ws=None) == 1 and "workspace" in pa.pa_last_error()
+    rec = lambda parts: -(-(4 * 32 * parts * (8 + 4 * 128)) // 256) * 256
+    # suffixes of at most 4096 tokens: the 2 prefix records only (256-token chunks)
     n = pa.pa_decode_shared_prefix_workspace_size(4, 32, 8, 128, 16, 2000, 512, torch.bfloat16)
-    assert n == -(-(4 * 32 * 8 * (8 + 4 * 128)) // 256) * 256      # 8 partitions of 256 tokens
+    assert n == rec(2)
     n8 = pa.pa_decode_shared_prefix_workspace_size(4, 32, 8, 128, 16, 2000, 512,
                                                    torch.float8_e4m3fn)
     assert n8 == n + 2 * 512 * 8 * 128 * 2                          # + 16-bit K, V prefix copies
+    # longer suffixes: every 256-token partition of max_ctx has a record
+    assert pa.pa_decode_shared_prefix_workspace_size(4, 32, 8, 128, 16, 10000, 512,
+                                                     torch.bfloat16) == rec(40)
     assert pa.pa_decode_shared_prefix_workspace_size(4, 32, 8, 128, 16, 300, 512,
                                                      torch.bfloat16) == 0   # plain decode

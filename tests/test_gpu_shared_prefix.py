@@ -129,3 +129,18 @@ def test_prefix_longer_than_every_context_is_a_plain_decode():
     out = _run(inp, kc, vc, wide, inp.context_lens, 64 + 32 * 4, inp.max_ctx)
     assert pa.pa_device_status() == 0
     _check(out, inp, kc, vc, wide, inp.context_lens, "longer prefix")
+
+
+def test_long_suffixes_take_the_split_path():
+    """Suffixes past 4096 tokens are cut into 256-token partitions and merged by
+    the split-K merge; an irregular sequence is exact there too."""
+    cfg = wl.small_variant(dataclasses.replace(wl.CONFIGS[5], kv_dtype="bf16", block_size=16,
+                                               fp8_scaled=False, cow_last_block=False),
+                           3, 4000, 5200, prefix_tokens=256)
+    inp = wl.make_decode_inputs(cfg, seed=12)
+    kc, vc = _appended(inp)
+    tables, lens = inp.block_tables.clone(), inp.context_lens.clone()
+    lens[1] = 200                                            # shorter than the prefix
+    out = _run(inp, kc, vc, tables, lens, 256, inp.max_ctx)
+    assert pa.pa_device_status() == 0
+    _check(out, inp, kc, vc, tables, lens, "split")
