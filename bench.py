@@ -680,7 +680,7 @@ def run_gpu_prefill(args, cfg: wl.PrefillConfig, rank, world, local_rank):
         torch.distributed.barrier()
     torch.cuda.synchronize()
     clocks = ClockSampler(local_rank)
-    evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks.mark_start()
@@ -707,6 +707,14 @@ def run_gpu_prefill(args, cfg: wl.PrefillConfig, rank, world, local_rank):
         return
     peak, peak_kind = _prefill_peak(ms)
     achieved = flops / (k_ms * 1e-3) / 1e12
+    traffic = None                  # DRAM bytes of one pa_prefill, from the committed capture
+    prof = os.path.join(ROOT, "profiles", f"traffic_{cfg.name}.json")
+    if os.path.exists(prof) and not args.seqs:
+        try:
+            with open(prof) as f:
+                traffic = json.load(f).get("dram_bytes_per_launch")
+        except Exception:
+            traffic = None
     cpu = None
     if not args.no_cpu_baseline and world == 1:
         r = prefill_oracle_rate(cfg, args.seed, args.cpu_budget)
@@ -722,7 +730,7 @@ def run_gpu_prefill(args, cfg: wl.PrefillConfig, rank, world, local_rank):
         "tokens_per_s": round(tokens_all / (ms_step * 1e-3), 1),
         "prefill_ms": round(k_ms, 4),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
-                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic,
                      "peak_kind": peak_kind, "kernel": "pa_prefill"},
         "cpu_baseline": cpu,
         "e2e": None if e2e is None else {
