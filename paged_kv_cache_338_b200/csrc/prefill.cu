@@ -30,11 +30,17 @@
 // i.e. its 32 query rows); warp 8 loads (tensor-map copies of the two Q tiles
 // once, then K and V tiles into rings); warp 9 allocates tensor memory and one
 // of its lanes issues every MMA; warps 10-11 only complete the third
-// warpgroup, whose registers go to the softmax warps.  Tensor memory: S_A 0..127, O_A 128..255,
-// S_B 256..383, O_B 384..511.  The MMA lane waits for P_X.V to complete before
-// it computes the next S_X into the same columns.  Every wait is bounded (2 s):
-// on timeout the CTA records PA_DEV_WAIT_TIMEOUT with the wait's site, drains
-// its own copies and MMAs, frees its tensor memory and exits.
+// warpgroup, whose registers go to the softmax warps.  Tensor memory: S_A
+// 0..127, O_A 128..255, S_B 256..383, O_B 384..511.  The MMA lane waits for
+// P_X.V to complete before it computes the next S_X into the same columns.
+// Every wait is bounded (2 s): on timeout the CTA records PA_DEV_WAIT_TIMEOUT
+// with the wait's site, drains its own copies and MMAs, frees its tensor
+// memory and exits.
+//
+// Prefix mode (shared-prefix decode, shared_prefix.cu): the query rows are the
+// decode queries of all sequences, grid y is a chunk of the prefix every table
+// shares, there is no causal mask, and the epilogue writes split-K records
+// (m, l, o * v_scale) instead of normalised rows.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -50,6 +56,7 @@ using namespace pa::dev;
 
 constexpr int kBM = 128;          // query rows per tile
 constexpr int kBN = 128;          // keys per tile
+constexpr int kPairGroup = 16;    // adjacent tile pairs scheduled side by side
 constexpr int kSeg = 16384;       // 128 rows x 128 bytes: one operand segment
 constexpr int kThreads = 384;     // 2 softmax warpgroups; a load warp, an MMA warp, 2 idle
 // Register split (setmaxnreg): the kernel launches with 384 x 168 registers at
@@ -318,8 +325,14 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                const __grid_constant__ CUtensorMap tmv, const Params p) {
     using L = Smem<D>;
     constexpr int NSEG = L::NSEG, ST = L::ST;
-    const int g = blockIdx.x;
-    const int pair = p.n_pairs - 1 - (int)blockIdx.z;     // longest tiles first
+    // grid (kPairGroup tile pairs x kv heads, sequences | prefix chunks, pair
+    // groups): a group of adjacent tile pairs of one (sequence, kv head) runs
+    // side by side and shares its K/V through L2, while groups run longest
+    // first across all sequences (the causal tail stays short)
+    const int g = (int)blockIdx.x / kPairGroup;
+    const int pair = ((int)gridDim.z - 1 - (int)blockIdx.z) * kPairGroup +
+                     (kPairGroup - 1 - (int)blockIdx.x % kPairGroup);
+    if (pair >= p.n_pairs) return;                        // past the last pair
     const bool pfx = p.prefix != 0;
     const int s = pfx ? 0 : (int)blockIdx.y;              // the sequence (table row)
     const int chunk = pfx ? (int)blockIdx.y : 0;          // prefix mode: the key chunk
@@ -682,14 +695,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
 template <int DT, int D>
 cudaError_t launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                    const Params& p, dim3 grid, cudaStream_t st) {
-    static bool attr_set = false;       // per instantiation; idempotent if raced
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(prefill_kernel<DT, D>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             Smem<D>::BYTES);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    // once per instantiation (a function-local static initialises thread-safely)
+    static const cudaError_t attr = cudaFuncSetAttribute(
+        prefill_kernel<DT, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Smem<D>::BYTES);
+    if (attr != cudaSuccess) return attr;
     prefill_kernel<DT, D><<<grid, kThreads, Smem<D>::BYTES, st>>>(mq, mk, mv, p);
     return cudaGetLastError();
 }
@@ -744,7 +753,8 @@ pa_status pa::prefix_records(const void* q, pa_dtype dt, const void* k_src, cons
     p.ws_ml = ws_ml;
     p.ws_o = ws_o;
     p.v_scale = v_scale;
-    const dim3 grid((unsigned)Hkv, (unsigned)chunks, (unsigned)n_pairs);
+    const dim3 grid((unsigned)(Hkv * pf::kPairGroup), (unsigned)chunks,
+                    (unsigned)((n_pairs + pf::kPairGroup - 1) / pf::kPairGroup));
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     cudaError_t e;
     if (dt == PA_BF16)
@@ -821,7 +831,8 @@ extern "C" pa_status pa_prefill(void* out, const void* q, pa_dtype q_dt, const v
     p.n_pairs = (int)n_pairs;
     p.sl = scale * 1.4426950408889634f;
 
-    const dim3 grid((unsigned)Hkv, (unsigned)S, (unsigned)n_pairs);
+    const dim3 grid((unsigned)(Hkv * pf::kPairGroup), (unsigned)S,
+                    (unsigned)((n_pairs + pf::kPairGroup - 1) / pf::kPairGroup));
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     cudaError_t e;
     if (q_dt == PA_BF16)
