@@ -568,6 +568,7 @@ def run_e2e(args, cfg, pa, dev, part):
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
+    h2d_stream.wait_event(e0)                 # the first timed copy starts after e0
     for i in range(args.steps):
         total_bytes += step(args.warmup + i)
     e1.record(d2h_stream)                     # after the last step's output reached the host
@@ -746,42 +747,65 @@ def run_gpu_prefill(args, cfg: wl.PrefillConfig, rank, world, local_rank):
 def prefill_e2e(args, cfg, pa, dev):
     """Public API with host buffers: each step copies the new tokens' q, k, v,
     their slots and the tables from pinned memory, runs append + prefill and
-    reads the output back."""
+    reads the output back.  Pipelined like the decode leg: two slots, inputs in
+    on one copy stream while the previous step computes, outputs out on
+    another."""
     inp = wl.make_prefill_inputs(cfg, seed=args.seed + 11, device=dev)
-    host = {k: getattr(inp, k).cpu().pin_memory() for k in
-            ("q", "key_new", "value_new", "slot_mapping", "block_tables", "context_lens",
-             "query_start")}
-    devb = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
-    out = torch.empty_like(inp.q)
-    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    names = ("q", "key_new", "value_new", "slot_mapping", "block_tables", "context_lens",
+             "query_start")
+    host = {k: getattr(inp, k).cpu().pin_memory() for k in names}   # one copy of the inputs
+    NSLOT = 2
+    devb = [{k: torch.empty_like(v, device=dev) for k, v in host.items()} for _ in range(NSLOT)]
+    out_d = [torch.empty_like(inp.q) for _ in range(NSLOT)]
+    out_h = [torch.empty(inp.q.shape, dtype=inp.q.dtype).pin_memory() for _ in range(NSLOT)]
     maxq = inp.max_query_len
     flops = wl.prefill_flops(cfg, inp.query_start, inp.context_lens)
     stream = torch.cuda.current_stream()
+    h2d_stream, d2h_stream = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    inputs_in = [torch.cuda.Event() for _ in range(NSLOT)]
+    kern_done = [torch.cuda.Event() for _ in range(NSLOT)]
+    output_out = [torch.cuda.Event() for _ in range(NSLOT)]
+    used = [False] * NSLOT
 
-    def step():
-        for k in host:
-            devb[k].copy_(host[k], non_blocking=True)
-        pa.pa_reshape_and_cache(devb["key_new"], devb["value_new"], inp.key_cache,
-                                inp.value_cache, devb["slot_mapping"])
-        pa.pa_prefill(out, devb["q"], inp.key_cache, inp.value_cache, devb["block_tables"],
-                      devb["context_lens"], devb["query_start"], maxq, inp.scale)
-        out_h.copy_(out, non_blocking=True)
+    def step(i):
+        k = i % NSLOT
+        with torch.cuda.stream(h2d_stream):
+            if used[k]:
+                h2d_stream.wait_event(kern_done[k])     # the slot's last reader is done
+            for name in names:
+                devb[k][name].copy_(host[name], non_blocking=True)
+            inputs_in[k].record(h2d_stream)
+        stream.wait_event(inputs_in[k])
+        if used[k]:
+            stream.wait_event(output_out[k])            # the slot's output has been read out
+        d = devb[k]
+        pa.pa_reshape_and_cache(d["key_new"], d["value_new"], inp.key_cache, inp.value_cache,
+                                d["slot_mapping"])
+        pa.pa_prefill(out_d[k], d["q"], inp.key_cache, inp.value_cache, d["block_tables"],
+                      d["context_lens"], d["query_start"], maxq, inp.scale)
+        kern_done[k].record(stream)
+        with torch.cuda.stream(d2h_stream):
+            d2h_stream.wait_event(kern_done[k])
+            out_h[k].copy_(out_d[k], non_blocking=True)
+            output_out[k].record(d2h_stream)
+        used[k] = True
 
-    for _ in range(args.warmup):
-        step()
+    for i in range(args.warmup):
+        step(i)
     torch.cuda.synchronize()
     steps = max(3, min(args.steps, 50))
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(steps):
-        step()
-    e1.record(stream)
+    h2d_stream.wait_event(e0)                 # the first timed copy starts after e0
+    for i in range(steps):
+        step(args.warmup + i)
+    e1.record(d2h_stream)
     e1.synchronize()
     ms = e0.elapsed_time(e1) / steps
     assert pa.pa_device_status() == 0
     return {"ms": ms, "value": flops / (ms * 1e-3) / 1e12, "flops": flops,
             "h2d": sum(v.numel() * v.element_size() for v in host.values()),
-            "d2h": out_h.numel() * out_h.element_size()}
+            "d2h": out_h[0].numel() * out_h[0].element_size()}
 
 
 def run_reference_prefill(args, cfg, rank, world):
