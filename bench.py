@@ -533,8 +533,7 @@ def run_e2e(args, cfg, pa, dev, part):
         k = i % NSLOT
         if used[k]:
             inputs_in[k].synchronize()         # the copy that read this host slot has finished
-        _, pairs = pool.seq_append_batch(seq_ids, hv[k]["slots"], cow_buf)
-        pool.build_block_tables(seq_ids, MB, hv[k]["tables"], hv[k]["lens"])
+        pairs = pool.step(seq_ids, MB, hv[k]["slots"], cow_buf, hv[k]["tables"], hv[k]["lens"])
         with torch.cuda.stream(h2d_stream):
             if used[k]:
                 h2d_stream.wait_event(kern_done[k])    # the device slot's last reader is done

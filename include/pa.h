@@ -397,6 +397,18 @@ pa_status pa_pool_build_block_tables(const pa_pool* pool, const int64_t* seqs, i
 
 pa_status pa_pool_stats(const pa_pool* pool, pa_pool_stats_t* stats);
 
+/*
+ * One decode step's host work in one call: pa_pool_seq_append_batch on
+ * `seqs`, then pa_pool_build_block_tables of the same sequences into
+ * tables_host [n, MB] / ctx_lens_host [n] (the lengths include the token just
+ * appended).  All or nothing: an unknown or repeated sequence, a table that
+ * would need more than MB entries, or too few free blocks returns an error
+ * and changes nothing.
+ */
+pa_status pa_pool_step(pa_pool* pool, const int64_t* seqs, int n, int MB, int64_t* slots,
+                       int32_t* cow_pairs, int* n_cow, int32_t* tables_host,
+                       int32_t* ctx_lens_host);
+
 /* The physical blocks of a sequence, in table order (*n is set even when cap
  * is too small, which returns PA_ERR_INVALID_ARG). */
 pa_status pa_pool_seq_blocks(const pa_pool* pool, int64_t seq, int32_t* blocks, int cap, int* n);

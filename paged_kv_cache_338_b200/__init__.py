@@ -100,6 +100,7 @@ def lib() -> ctypes.CDLL:
         "pa_pool_build_block_tables": ([P, P, I, I, P, P], I),
         "pa_pool_stats": ([P, ctypes.POINTER(_Stats)], I),
         "pa_pool_seq_blocks": ([P, I64, P, I, ctypes.POINTER(I)], I),
+        "pa_pool_step": ([P, P, I, I, P, P, ctypes.POINTER(I), P, P], I),
         "pa_pool_cache_block": ([P, I32, ctypes.c_uint64, ctypes.POINTER(I)], I),
         "pa_pool_cache_lookup": ([P, ctypes.c_uint64, ctypes.POINTER(I32)], I),
         "pa_pool_seq_match_prefix": ([P, I64, P, I, ctypes.POINTER(I)], I),
@@ -405,6 +406,20 @@ class BlockPool:
         st = _Stats()
         _check(lib().pa_pool_stats(self._p, ctypes.byref(st)))
         return {n: getattr(st, n) for n, _ in _Stats._fields_}
+
+    def step(self, seqs: torch.Tensor, max_blocks: int, slots_out: torch.Tensor,
+             cow_out: torch.Tensor, tables_out: torch.Tensor, lens_out: torch.Tensor):
+        """One decode step's host work: append a token to every sequence of the
+        contiguous host int64 tensor `seqs` and pack their tables and lengths
+        into the given host tensors.  -> copy-on-write pairs int32 [k, 2]."""
+        n = seqs.numel()
+        nc = ctypes.c_int(0)
+        _check(lib().pa_pool_step(self._p, seqs.data_ptr() if n else None, n, max_blocks,
+                                  slots_out.data_ptr() if n else None, cow_out.data_ptr(),
+                                  ctypes.byref(nc),
+                                  tables_out.data_ptr() if tables_out.numel() else None,
+                                  lens_out.data_ptr() if n else None))
+        return cow_out[:nc.value]
 
     def seq_blocks(self, seq: int) -> list:
         n = ctypes.c_int(0)

@@ -404,3 +404,26 @@ extern "C" pa_status pa_pool_seq_match_prefix(pa_pool* pool, int64_t seq, const 
     *matched = m;
     return PA_OK;
 }
+
+extern "C" pa_status pa_pool_step(pa_pool* pool, const int64_t* seqs, int n, int MB, int64_t* slots,
+                                  int32_t* cow_pairs, int* n_cow, int32_t* tables_host,
+                                  int32_t* ctx_lens_host) {
+    pa::clear_error();
+    if (!pool || n < 0 || MB < 0 || !n_cow ||
+        (n > 0 && (!seqs || !slots || !cow_pairs || !ctx_lens_host || (MB > 0 && !tables_host))))
+        return fail(PA_ERR_INVALID_ARG, "bad arguments");
+    *n_cow = 0;
+    // all or nothing: every table must still fit MB entries after the append
+    for (int i = 0; i < n; ++i) {
+        const pa_pool::Seq* s = pool->find(seqs[i]);
+        if (!s) return fail(PA_ERR_BAD_INDEX, "unknown sequence %lld", (long long)seqs[i]);
+        const int64_t after = (int64_t)s->blocks.size() + (s->n % pool->bs == 0 ? 1 : 0);
+        if (after > MB)
+            return fail(PA_ERR_INVALID_ARG, "sequence %lld needs %lld blocks > MB %d",
+                        (long long)seqs[i], (long long)after, MB);
+        if (s->n + 1 > 0x7fffffffLL) return fail(PA_ERR_INVALID_ARG, "context length overflows int32");
+    }
+    pa_status st = pa_pool_seq_append_batch(pool, seqs, n, slots, cow_pairs, n_cow);
+    if (st) return st;
+    return pa_pool_build_block_tables(pool, seqs, n, MB, tables_host, ctx_lens_host);
+}

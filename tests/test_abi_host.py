@@ -393,3 +393,47 @@ def test_shared_prefix_host_argument_checks():
                                                      torch.bfloat16) == rec(40)
     assert pa.pa_decode_shared_prefix_workspace_size(4, 32, 8, 128, 16, 300, 512,
                                                      torch.bfloat16) == 0   # plain decode
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_pool_step_equals_append_then_pack(seed):
+    """pa_pool_step = seq_append_batch + build_block_tables, all or nothing."""
+    rnd = random.Random(500 + seed)
+    nb, bs, MB = 80, 8, (3, 12, 5)[seed]          # small MB: the table-width rule fires
+    a, b = pa.BlockPool(nb, bs), pa.BlockPool(nb, bs)
+    seqs = []
+    for _ in range(6):
+        s1, s2 = a.seq_new(), b.seq_new()
+        assert s1 == s2
+        seqs.append(s1)
+    for step in range(60):
+        if rnd.random() < 0.1:
+            parent = rnd.choice(seqs)
+            c1, c2 = a.seq_fork(parent), b.seq_fork(parent)
+            assert c1 == c2
+            seqs.append(c1)
+        batch = torch.tensor(rnd.sample(seqs, rnd.randint(1, len(seqs))), dtype=torch.int64)
+        n = batch.numel()
+        slots_a, cow_a = torch.empty(n, dtype=torch.int64), torch.empty((n, 2), dtype=torch.int32)
+        tab_a, len_a = torch.empty((n, MB), dtype=torch.int32), torch.empty(n, dtype=torch.int32)
+        try:
+            pairs_a = a.step(batch, MB, slots_a, cow_a, tab_a, len_a)
+            err_a = None
+        except pa.PaError as e:
+            err_a = e.status
+        # the same through the two separate calls, guarded by the same MB rule
+        fits = all(len(b.seq_blocks(int(s))) + (b.seq_len(int(s)) % bs == 0) <= MB for s in batch)
+        err_b = None
+        if not fits:
+            err_b = "PA_ERR_INVALID_ARG"
+        else:
+            try:
+                slots_b, pairs_b = b.seq_append_batch(batch)
+                tab_b, len_b = b.build_block_tables(batch, MB)
+            except pa.PaError as e:
+                err_b = e.status
+        assert err_a == err_b
+        if err_a is None:
+            assert torch.equal(slots_a, slots_b) and torch.equal(pairs_a, pairs_b)
+            assert torch.equal(tab_a, tab_b) and torch.equal(len_a, len_b)
+        assert [a.ref(i) for i in range(nb)] == [b.ref(i) for i in range(nb)]
