@@ -1,4 +1,4 @@
-"""Seeded synthetic inputs for paged decode: the one module that both the oracle
+"""Seeded synthetic inputs for paged decode and prefill: the one module that both the oracle
 side and the CUDA side of the tests (and bench.py) draw their inputs from.
 
 It holds none of the method's arithmetic.  It only draws random numbers, casts
@@ -22,7 +22,9 @@ or a wrong value instead of passing by luck):
 
 The five workloads are the decode configurations this library is measured on;
 ``small_variant`` shrinks any of them for parity tests the oracle finishes in
-seconds.  Every draw comes from a seeded torch.Generator.
+seconds.  ``PREFILL_CONFIGS`` / ``make_prefill_inputs`` do the same for batches
+of prefill chunks (new tokens appended through slot_mapping, then attended
+causally over the cache).  Every draw comes from a seeded torch.Generator.
 """
 from __future__ import annotations
 
