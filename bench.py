@@ -57,6 +57,8 @@ import torch  # noqa: E402
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
+# raw clock logs (the JSON line carries their summary); PA_BENCH_LOG_DIR overrides
+LOG_DIR = os.environ.get("PA_BENCH_LOG_DIR", os.path.join(ROOT, "bench_logs"))
 
 import workloads as wl  # noqa: E402
 
@@ -137,8 +139,8 @@ class ClockSampler:
     def __init__(self, dev: int):
         self.t0 = self.t1 = None
         pid = _pci_id(dev)
-        os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
-        self.path = os.path.join(ROOT, "gpurun_out", f"nvml_rank{dev}.log")
+        os.makedirs(LOG_DIR, exist_ok=True)
+        self.path = os.path.join(LOG_DIR, f"nvml_rank{dev}.log")
         if os.path.exists(self.path):      # a previous run's log would end the wait below early
             os.remove(self.path)
         self.child = subprocess.Popen([sys.executable, os.path.abspath(__file__),
@@ -148,7 +150,7 @@ class ClockSampler:
         try:
             args = ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
                     "-lms", "200"] + (["-i", pid] if pid else [])
-            self.f = open(os.path.join(ROOT, "gpurun_out", f"clocks_rank{dev}.csv"), "w")
+            self.f = open(os.path.join(LOG_DIR, f"clocks_rank{dev}.csv"), "w")
             self.proc = subprocess.Popen(args, stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None

@@ -293,7 +293,7 @@ template <> __device__ __forceinline__ uint32_t pack2<PA_F16>(float a, float b) 
     __half2 h = __floats2half2_rn(a, b);
     return *reinterpret_cast<uint32_t*>(&h);
 }
-// Bounded wait by every lane of a warp; the verdict is warp-uniform.  A
+// Bounded wait by every lane of a warp; the outcome is warp-uniform.  A
 // pipeline wait gives up early once another role has aborted the CTA; a drain
 // wait (honor_abort false) does not, since it guards memory still in flight.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
