@@ -834,7 +834,11 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", type=int, default=3, choices=sorted(wl.CONFIGS))
+    ap.add_argument("--config", type=int, default=3, choices=sorted(wl.CONFIGS),
+                    help="decode workload by number: " + ", ".join(
+                        f"{k} = {c.name}" for k, c in sorted(wl.CONFIGS.items())))
+    ap.add_argument("--workload", choices=sorted(wl.DECODE_WORKLOADS),
+                    help="decode workload by name (overrides --config)")
     ap.add_argument("--partition", type=int, default=-1, help="-1: workload default / heuristic")
     ap.add_argument("--seed", type=int, default=2)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
@@ -862,7 +866,7 @@ def main():
             cfg = dataclasses.replace(cfg, num_seqs=min(args.seqs, cfg.num_seqs),
                                       name=cfg.name + f"_small{args.seqs}")
     else:
-        cfg = wl.CONFIGS[args.config]
+        cfg = wl.DECODE_WORKLOADS[args.workload] if args.workload else wl.CONFIGS[args.config]
         if args.seqs:
             cfg = _sample_cfg(cfg, args.seqs)
     if args.impl == "reference":

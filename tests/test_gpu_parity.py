@@ -92,11 +92,11 @@ BOTH = [pa.DECODE_DEFAULT, pa.DECODE_DEFAULT | pa.DECODE_SIMT_ONLY]
 
 
 SMALL = [
-    ("cfg1", wl.CONFIGS[1]),
-    ("cfg2", wl.small_variant(wl.CONFIGS[2], 5, 1, 200)),
-    ("cfg3", wl.small_variant(wl.CONFIGS[3], 6, 1, 300)),
-    ("cfg4", wl.small_variant(wl.CONFIGS[4], 2, 1500, 2100)),
-    ("cfg5", wl.small_variant(wl.CONFIGS[5], 6, 1, 120, prefix_tokens=64)),
+    ("tiny_fp32", wl.DECODE_WORKLOADS["tiny_paged_decode_fp32"]),
+    ("mha_fp16", wl.small_variant(wl.DECODE_WORKLOADS["llama2_7b_mha_fp16_b64"], 5, 1, 200)),
+    ("gqa_bf16", wl.small_variant(wl.DECODE_WORKLOADS["llama3_8b_gqa_bf16_b128"], 6, 1, 300)),
+    ("long_splitk", wl.small_variant(wl.DECODE_WORKLOADS["long_context_splitk_bf16_4x100k"], 2, 1500, 2100)),
+    ("prefix_fp8", wl.small_variant(wl.DECODE_WORKLOADS["prefix_shared_fp8_b256"], 6, 1, 120, prefix_tokens=64)),
 ]
 
 
@@ -159,7 +159,7 @@ def test_zero_length_sequences_give_zero_rows():
 
 
 def test_device_errors_are_reported_not_followed():
-    cfg = wl.small_variant(wl.CONFIGS[3], 3, 20, 60)
+    cfg = wl.small_variant(wl.DECODE_WORKLOADS["llama3_8b_gqa_bf16_b128"], 3, 20, 60)
     inp = wl.make_decode_inputs(cfg, seed=9)
     d = _to(inp, "cuda")
     kc, vc = d["key_cache"].clone(), d["value_cache"].clone()

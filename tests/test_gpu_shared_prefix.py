@@ -74,17 +74,17 @@ def _check(got, inp, kc, vc, tables, lens, what):
 
 CASES = [
     # name, base config, seqs, suffix lo/hi, prefix tokens
-    ("fp8_bs32_p256", wl.CONFIGS[5], 12, 1, 200, 256),
-    ("fp8_bs32_p1024", wl.CONFIGS[5], 10, 30, 300, 1024),
-    ("fp8_bs32_p96", wl.CONFIGS[5], 9, 1, 90, 96),
-    ("bf16_bs16_p512", dataclasses.replace(wl.CONFIGS[5], kv_dtype="bf16", block_size=16,
+    ("fp8_bs32_p256", wl.DECODE_WORKLOADS["prefix_shared_fp8_b256"], 12, 1, 200, 256),
+    ("fp8_bs32_p1024", wl.DECODE_WORKLOADS["prefix_shared_fp8_b256"], 10, 30, 300, 1024),
+    ("fp8_bs32_p96", wl.DECODE_WORKLOADS["prefix_shared_fp8_b256"], 9, 1, 90, 96),
+    ("bf16_bs16_p512", dataclasses.replace(wl.DECODE_WORKLOADS["prefix_shared_fp8_b256"], kv_dtype="bf16", block_size=16,
                                            fp8_scaled=False), 11, 1, 300, 512),
-    ("f16_mha_bs8_p128", dataclasses.replace(wl.CONFIGS[5], kv_dtype="f16", q_dtype="f16",
+    ("f16_mha_bs8_p128", dataclasses.replace(wl.DECODE_WORKLOADS["prefix_shared_fp8_b256"], kv_dtype="f16", q_dtype="f16",
                                              num_kv_heads=32, block_size=8, fp8_scaled=False),
      5, 1, 60, 128),
-    ("fp8_q_f16_g8", dataclasses.replace(wl.CONFIGS[5], q_dtype="f16", num_q_heads=16,
+    ("fp8_q_f16_g8", dataclasses.replace(wl.DECODE_WORKLOADS["prefix_shared_fp8_b256"], q_dtype="f16", num_q_heads=16,
                                          num_kv_heads=2), 7, 1, 100, 256),
-    ("bf16_d64_g2", dataclasses.replace(wl.CONFIGS[5], kv_dtype="bf16", head_dim=64,
+    ("bf16_d64_g2", dataclasses.replace(wl.DECODE_WORKLOADS["prefix_shared_fp8_b256"], kv_dtype="bf16", head_dim=64,
                                         num_q_heads=8, num_kv_heads=4, block_size=16,
                                         fp8_scaled=False), 6, 1, 150, 256),
 ]
@@ -102,7 +102,7 @@ def test_shared_prefix_matches_decode(name, base, nseq, lo, hi, prefix):
 
 
 def test_sequences_outside_the_shared_prefix_fall_back():
-    cfg = wl.small_variant(wl.CONFIGS[5], 8, 20, 200, prefix_tokens=512)
+    cfg = wl.small_variant(wl.DECODE_WORKLOADS["prefix_shared_fp8_b256"], 8, 20, 200, prefix_tokens=512)
     inp = wl.make_decode_inputs(cfg, seed=3)
     kc, vc = _appended(inp)
     tables, lens = inp.block_tables.clone(), inp.context_lens.clone()
@@ -121,7 +121,7 @@ def test_sequences_outside_the_shared_prefix_fall_back():
 
 
 def test_prefix_longer_than_every_context_is_a_plain_decode():
-    cfg = wl.small_variant(wl.CONFIGS[5], 4, 1, 30, prefix_tokens=64)
+    cfg = wl.small_variant(wl.DECODE_WORKLOADS["prefix_shared_fp8_b256"], 4, 1, 30, prefix_tokens=64)
     inp = wl.make_decode_inputs(cfg, seed=8)
     kc, vc = _appended(inp)
     wide = torch.full((4, 8), -1, dtype=torch.int32)        # room for the declared prefix
@@ -134,7 +134,7 @@ def test_prefix_longer_than_every_context_is_a_plain_decode():
 def test_long_suffixes_take_the_split_path():
     """Suffixes past 4096 tokens are cut into 256-token partitions and merged by
     the split-K merge; an irregular sequence is exact there too."""
-    cfg = wl.small_variant(dataclasses.replace(wl.CONFIGS[5], kv_dtype="bf16", block_size=16,
+    cfg = wl.small_variant(dataclasses.replace(wl.DECODE_WORKLOADS["prefix_shared_fp8_b256"], kv_dtype="bf16", block_size=16,
                                                fp8_scaled=False, cow_last_block=False),
                            3, 4000, 5200, prefix_tokens=256)
     inp = wl.make_decode_inputs(cfg, seed=12)

@@ -72,7 +72,7 @@ def _reference_rank(rank: int, world: int, port: int, out_dir: str):
     try:
         args = argparse.Namespace(steps=1, warmup=1, seed=2, gpus=world)
         buf = io.StringIO()
-        cfg = wl.small_variant(wl.CONFIGS[3], 2, 20, 40)
+        cfg = wl.small_variant(wl.DECODE_WORKLOADS["llama3_8b_gqa_bf16_b128"], 2, 20, 40)
         with contextlib.redirect_stdout(buf):
             if rank != 0:
                 bench.run_reference(args, cfg, rank, world)

@@ -75,10 +75,10 @@ def _step_caches(inp: wl.DecodeInputs):
 
 
 SMALL = [
-    wl.CONFIGS[1],
-    wl.small_variant(wl.CONFIGS[2], 3, 1, 70),
-    wl.small_variant(wl.CONFIGS[3], 3, 1, 90),
-    wl.small_variant(wl.CONFIGS[5], 3, 1, 70, prefix_tokens=64),
+    wl.DECODE_WORKLOADS["tiny_paged_decode_fp32"],
+    wl.small_variant(wl.DECODE_WORKLOADS["llama2_7b_mha_fp16_b64"], 3, 1, 70),
+    wl.small_variant(wl.DECODE_WORKLOADS["llama3_8b_gqa_bf16_b128"], 3, 1, 90),
+    wl.small_variant(wl.DECODE_WORKLOADS["prefix_shared_fp8_b256"], 3, 1, 70, prefix_tokens=64),
 ]
 
 
@@ -101,7 +101,7 @@ def test_oracle_matches_sdpa_shapes(bs, G, D):
 
 
 def test_block_id_relabelling_invariance():
-    inp = wl.make_decode_inputs(wl.small_variant(wl.CONFIGS[3], 4, 20, 80), seed=5)
+    inp = wl.make_decode_inputs(wl.small_variant(wl.DECODE_WORKLOADS["llama3_8b_gqa_bf16_b128"], 4, 20, 80), seed=5)
     kc, vc = _step_caches(inp)
     base = _oracle(inp, kc, vc)
     g = torch.Generator().manual_seed(99)
@@ -117,7 +117,7 @@ def test_block_id_relabelling_invariance():
 
 
 def test_shared_prefix_equals_private_copies():
-    cfg = wl.small_variant(wl.CONFIGS[5], 4, 5, 60, prefix_tokens=96)
+    cfg = wl.small_variant(wl.DECODE_WORKLOADS["prefix_shared_fp8_b256"], 4, 5, 60, prefix_tokens=96)
     inp = wl.make_decode_inputs(cfg, seed=8)
     kc, vc = _step_caches(inp)
     shared = _oracle(inp, kc, vc)
@@ -139,7 +139,7 @@ def test_shared_prefix_equals_private_copies():
 
 
 def test_weights_sum_to_one():
-    inp = wl.make_decode_inputs(wl.small_variant(wl.CONFIGS[3], 3, 1, 200), seed=2)
+    inp = wl.make_decode_inputs(wl.small_variant(wl.DECODE_WORKLOADS["llama3_8b_gqa_bf16_b128"], 3, 1, 200), seed=2)
     kc, vc = _step_caches(inp)
     for s in range(3):
         for h in (0, 5, 31):
@@ -202,7 +202,7 @@ def test_gqa_equals_replicated_mha():
 
 def test_poison_is_never_read():
     # the generator fills unused blocks / tails with NaN and pads tables with -1
-    inp = wl.make_decode_inputs(wl.CONFIGS[1], seed=0)
+    inp = wl.make_decode_inputs(wl.DECODE_WORKLOADS["tiny_paged_decode_fp32"], seed=0)
     assert torch.isnan(inp.key_cache[inp.free_blocks.long()]).all()
     assert (inp.block_tables == -1).any()
     kc, vc = _step_caches(inp)
@@ -219,7 +219,7 @@ def test_zero_length_sequence_gives_zero_row():
 
 
 def test_bad_block_id_is_an_error():
-    inp = wl.make_decode_inputs(wl.CONFIGS[1], seed=0)
+    inp = wl.make_decode_inputs(wl.DECODE_WORKLOADS["tiny_paged_decode_fp32"], seed=0)
     t = inp.block_tables.clone()
     t[0, 0] = inp.num_blocks
     with pytest.raises(oracle.OracleError):
@@ -228,9 +228,11 @@ def test_bad_block_id_is_an_error():
 
 # ---------------------------------------------------------------- append / copy
 
-@pytest.mark.parametrize("cfg_id", [1, 2, 3])
-def test_append_places_rows_by_slot(cfg_id):
-    cfg = wl.CONFIGS[cfg_id] if cfg_id == 1 else wl.small_variant(wl.CONFIGS[cfg_id], 5, 1, 70)
+@pytest.mark.parametrize("name", ["tiny_paged_decode_fp32", "llama2_7b_mha_fp16_b64",
+                                  "llama3_8b_gqa_bf16_b128"])
+def test_append_places_rows_by_slot(name):
+    base = wl.DECODE_WORKLOADS[name]
+    cfg = base if base.fixed_lens else wl.small_variant(base, 5, 1, 70)
     inp = wl.make_decode_inputs(cfg, seed=3)
     kc, vc = oracle.reshape_and_cache(inp.key_new, inp.value_new, cfg.q_dtype, inp.key_cache,
                                       inp.value_cache, cfg.kv_dtype, inp.slot_mapping,
@@ -244,7 +246,7 @@ def test_append_places_rows_by_slot(cfg_id):
 
 
 def test_append_fp8_matches_torch_quantisation_and_skips_negative_slots():
-    cfg = wl.small_variant(wl.CONFIGS[5], 6, 1, 40, prefix_tokens=32)
+    cfg = wl.small_variant(wl.DECODE_WORKLOADS["prefix_shared_fp8_b256"], 6, 1, 40, prefix_tokens=32)
     inp = wl.make_decode_inputs(cfg, seed=6)
     sm = inp.slot_mapping.clone()
     sm[2] = -1
@@ -262,7 +264,7 @@ def test_append_fp8_matches_torch_quantisation_and_skips_negative_slots():
 
 
 def test_append_out_of_range_slot_is_an_error():
-    inp = wl.make_decode_inputs(wl.CONFIGS[1], seed=0)
+    inp = wl.make_decode_inputs(wl.DECODE_WORKLOADS["tiny_paged_decode_fp32"], seed=0)
     sm = inp.slot_mapping.clone()
     sm[1] = inp.num_blocks * 16
     with pytest.raises(oracle.OracleError):
@@ -271,7 +273,7 @@ def test_append_out_of_range_slot_is_an_error():
 
 
 def test_copy_blocks_and_rejections():
-    inp = wl.make_decode_inputs(wl.CONFIGS[1], seed=0)
+    inp = wl.make_decode_inputs(wl.DECODE_WORKLOADS["tiny_paged_decode_fp32"], seed=0)
     pairs = torch.tensor([[3, 10], [5, 11], [3, 12]], dtype=torch.int32)
     kc, vc = oracle.copy_blocks(inp.key_cache, inp.value_cache, pairs)
     ek, ev = oracle.raw(inp.key_cache).copy(), oracle.raw(inp.value_cache).copy()

@@ -20,7 +20,7 @@ TOL = 1e-2   # bf16 cache, the same bar as the oracle parity tests
 
 
 def _inputs(seed):
-    cfg = wl.small_variant(wl.CONFIGS[3], 8, 200, 1500)
+    cfg = wl.small_variant(wl.DECODE_WORKLOADS["llama3_8b_gqa_bf16_b128"], 8, 200, 1500)
     inp = wl.make_decode_inputs(cfg, seed=seed)
     d = {k: getattr(inp, k).cuda() for k in
          ("q", "key_cache", "value_cache", "key_new", "value_new", "slot_mapping",

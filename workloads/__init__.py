@@ -106,6 +106,10 @@ CONFIGS = {
 }
 
 
+# the same workloads by name
+DECODE_WORKLOADS = {cfg.name: cfg for cfg in CONFIGS.values()}
+
+
 def small_variant(cfg: DecodeConfig, num_seqs: int, ctx_lo: int, ctx_hi: int,
                   prefix_tokens: Optional[int] = None) -> DecodeConfig:
     """Same heads / dims / dtypes / structure, fewer and shorter sequences."""
