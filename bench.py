@@ -1,26 +1,32 @@
-"""Paged decode benchmark on B200: KV-read GB/s, decode seqs/s, roofline fraction.
+"""Paged attention benchmark on B200: KV-read GB/s, decode seqs/s, roofline fraction.
 
-One step = one decode step of the whole hot path for one batch:
+Decode (default).  One step = one decode step of the whole hot path for one batch:
   cache append (pa_reshape_and_cache) -> [copy-on-write copies] -> pa_decode
-  (split-K partition kernel + merge kernel)
-on the synthetic workload (default: Llama-3-8B-shaped GQA decode, 128 sequences,
+  (split-K partition kernel + merge kernel), or pa_decode_shared_prefix for the
+  shared-prefix workload
+on a synthetic workload (default: Llama-3-8B-shaped GQA decode, 128 sequences,
 32 q / 8 kv heads, head_dim 128, block 16, bf16, context lens uniform in
-[1024, 8192], shuffled physical blocks).  The KV cache (2.4 GB) is larger than
-L2, so no flush is needed between steps.
+[1024, 8192], shuffled physical blocks; --config / --workload pick another).
+The KV cache (2.5 GB) is larger than L2, so no flush is needed between steps.
+
+Prefill (--op prefill).  One step = append the chunks' K, V, then pa_prefill;
+metric TFLOP/s of causal attention against the measured bf16 tensor peak.
 
 Printed (rank 0, one JSON line):
-  value   -- algorithmic bytes per step / device step time (CUDA events), GB/s
+  value   -- algorithmic bytes (or FLOPs) per step / device step time (CUDA events)
   e2e     -- the same metric through the public API with host buffers: host
-             pool appends + table packing, H2D of q/k/v/slots/tables, the step,
-             D2H of the output, every step
-  roofline -- pa_decode's algorithmic bytes / its measured launch time against
-             the measured HBM copy bandwidth
+             pool appends + table packing, H2D of the step's inputs, the step,
+             D2H of the output, every step (pipelined over two staging slots)
+  roofline -- the attention call's algorithmic bytes (FLOPs) / its measured
+             launch time against the measured HBM copy bandwidth (bf16 peak),
+             with the DRAM traffic of the committed ncu capture
   cpu_baseline -- the fp64 oracle on the host cores over a bounded sample
+  clocks  -- SM clock and throttle reasons sampled inside the timed region
 
 --impl reference runs the oracle (the only reference this method has here) on
 a bounded sample of the same workload on the host cores.
 With torchrun, N ranks each run an independent replica (no data-path
-collective); value = total bytes of all ranks / max time over ranks.
+collective); value = the units all ranks processed / max time over ranks.
 """
 from __future__ import annotations
 
