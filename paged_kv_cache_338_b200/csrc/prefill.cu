@@ -31,8 +31,9 @@
 // once, then K and V tiles into rings); warp 9 allocates tensor memory and one
 // of its lanes issues every MMA; warps 10-11 only complete the third
 // warpgroup, whose registers go to the softmax warps.  Tensor memory: S_A
-// 0..127, O_A 128..255, S_B 256..383, O_B 384..511.  The MMA lane waits for
-// P_X.V to complete before it computes the next S_X into the same columns.
+// 0..127, O_A 128..255, S_B 256..383, O_B 384..511.  The MMA lane issues the
+// next S_X into the same columns right behind P_X.V (one thread's MMAs run in
+// issue order), so the tensor core never idles waiting for P_X.V to finish.
 // Every wait is bounded (2 s): on timeout the CTA records PA_DEV_WAIT_TIMEOUT
 // with the wait's site, drains its own copies and MMAs, frees its tensor
 // memory and exits.
@@ -527,14 +528,15 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                 }
                 __syncwarp();
                 if (j + 1 < ntx) {
-                    // the next scores overwrite P_X: wait until P_X.V has read it
+                    // The next scores overwrite P_X in the same columns.  They are
+                    // issued right behind P_X.V: the MMAs one thread issues run in
+                    // issue order, so P_X.V has read P_X before S_X(j+1) is written.
                     if (!k_next) {
                         if (!(ok = warp_wait(k_full(st1), ((j + 1) / ST) & 1, abort_flag, p.err,
                                              8)))
                             break;
                         k_next = true;
                     }
-                    if (!(ok = warp_wait(pv_done(x), j & 1, abort_flag, p.err, 14))) break;
                     issue_s(x, st1);
                 }
             }
