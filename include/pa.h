@@ -77,7 +77,7 @@ enum {
  * 3 descriptor-free, 4 descriptor-ready, 5 states-published, 6 merge-done;
  * prefill: 7 q-tile, 8 k-tile-full, 9 v-tile-full, 10 k-tile-free,
  * 11 v-tile-free, 12 scores-ready, 13 probabilities-ready, 14 p.v-done,
- * 15 output-ready, 16 tensor-core drain, 17 load drain). */
+ * 15 output-ready, 16 tensor-core drain, 17 load drain, 18 exponential turn). */
 
 /* Message for the last failing call on this thread ("" if none). */
 const char* pa_last_error(void);

@@ -30,7 +30,10 @@
 // i.e. its 32 query rows); warp 8 loads (tensor-map copies of the two Q tiles
 // once, then K and V tiles into rings); warp 9 allocates tensor memory and one
 // of its lanes issues every MMA; warps 10-11 only complete the third
-// warpgroup, whose registers go to the softmax warps.  Tensor memory: S_A
+// warpgroup, whose registers go to the softmax warps.  The two softmax warps
+// that share a scheduler (w and w + 4) take turns with their exponentials, so
+// each has the special-function unit to itself, and a row's sum is taken
+// after its P is handed to the MMA warp.  Tensor memory: S_A
 // 0..127, O_A 128..255, S_B 256..383, O_B 384..511.  The MMA lane issues the
 // next S_X into the same columns right behind P_X.V (one thread's MMAs run in
 // issue order), so the tensor core never idles waiting for P_X.V to finish.
@@ -100,8 +103,9 @@ struct Smem {
     static constexpr int V = K + ST * TILE;
     static constexpr int BAR = V + ST * TILE;
     // barriers: q, k_full[ST], k_free[ST], v_full[ST], v_free[ST], then per
-    // query tile s_full, p_full, pv_done, o_full; drain
-    static constexpr int NBAR = 1 + 4 * ST + 8 + 1;
+    // query tile s_full, p_full, pv_done, o_full; drain; then per query tile
+    // and softmax warp the turn of its exponentials
+    static constexpr int NBAR = 1 + 4 * ST + 8 + 1 + 8;
     static constexpr int TMEM_SLOT = BAR + NBAR * 8;
     static constexpr int ABORT = TMEM_SLOT + 4;
     static constexpr int BYTES = ABORT + 4 + 1024;  // + slack to align the base to 1024
@@ -378,6 +382,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
     auto pv_done = [&](int x) { return bar0 + 8u * (5 + 4 * ST + x); };
     auto o_full = [&](int x) { return bar0 + 8u * (7 + 4 * ST + x); };
     const uint32_t drain = bar0 + 8u * (9 + 4 * ST);
+    auto turn = [&](int x, int w) { return bar0 + 8u * (10 + 4 * ST + 4 * x + w); };
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::ABORT);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -396,6 +401,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             mbar_init(o_full(x), 1);
         }
         mbar_init(drain, 1);
+        for (int i = 0; i < 8; ++i) mbar_init(turn(i >> 2, i & 3), 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -565,6 +571,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
         const int limit = row_ok && !pfx ? c + it + 1 : kvX;  // keys 0..limit-1 are visible
         const uint32_t lrow = (uint32_t)((warp & 3) * 32) << 16;
         const float sl = p.sl;
+        const uint32_t my_turn = turn(x, warp & 3), next_turn = turn(x ^ 1, warp & 3);
         float m_use = -INFINITY, lsum = 0.f;
         bool ok = true;
         for (int j = 0; j < ntx; ++j) {
@@ -611,10 +618,17 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                 }
                 tmem_wait_st();
             }
+            // The two softmax warps of one scheduler (warp w of tile A, warp
+            // w + 4 of tile B) take turns with their exponentials, A(j), B(j),
+            // A(j + 1) ..., so each runs with the special-function unit to
+            // itself instead of both at half speed; B's tiles past A's last
+            // one need no turn.
+            if (hasB && (x ? j < ntA : j > 0) &&
+                !(ok = warp_wait(my_turn, (j - 1 + x) & 1, abort_flag, p.err, 18)))
+                break;
             // probabilities, rounded to the operand type, two per 32-bit
-            // column over the scores they came from (the A operand of P.V)
-            // pairs of scores share one packed FMA and one packed add
-            float2 ps[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};   // partial sums
+            // column over the scores they came from (the A operand of P.V);
+            // pairs of scores share one packed FMA
             const float2 sl2 = make_float2(sl, sl), nm2 = make_float2(-m_use, -m_use);
 #pragma unroll
             for (int c16 = 0; c16 < kBN / 32; ++c16) {
@@ -623,17 +637,26 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                 for (int e = 0; e < 16; ++e) {
                     const int k = c16 * 32 + 2 * e;
                     const float2 xy = fma2(make_float2(sv[k], sv[k + 1]), sl2, nm2);
-                    const float2 pr = make_float2(ex2(xy.x), ex2(xy.y));
-                    ps[e & 3] = add2(ps[e & 3], pr);
-                    w[e] = pack2<DT>(pr.x, pr.y);
+                    sv[k] = ex2(xy.x);
+                    sv[k + 1] = ex2(xy.y);
+                    w[e] = pack2<DT>(sv[k], sv[k + 1]);
                 }
                 tmem_st16(tS(x) + lrow + c16 * 16, w);
             }
-            lsum += ((ps[0].x + ps[0].y) + (ps[1].x + ps[1].y)) +
-                    ((ps[2].x + ps[2].y) + (ps[3].x + ps[3].y));
+            if (hasB && (x == 0 || j + 1 < ntA)) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(next_turn);
+            }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(p_full(x));
+            // the row sum is not on the way to P.V: it is taken after the hand-off
+            float2 ps[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+            for (int k = 0; k < kBN; k += 2)
+                ps[(k >> 1) & 3] = add2(ps[(k >> 1) & 3], make_float2(sv[k], sv[k + 1]));
+            lsum += ((ps[0].x + ps[0].y) + (ps[1].x + ps[1].y)) +
+                    ((ps[2].x + ps[2].y) + (ps[3].x + ps[3].y));
         }
         if (ok) ok = warp_wait(o_full(x), 0, abort_flag, p.err, 15);
         if (ok && pfx) {
