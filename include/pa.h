@@ -231,7 +231,14 @@ pa_status pa_decode_noalloc(void* out, const void* q, pa_dtype q_dt,
  *   2: stream K/V with an L2 evict-first hint;
  *   4: partition-major grid (the kv heads of one partition are neighbouring
  *      CTAs, so the interleaved heads of a block are read at about the same
- *      time); otherwise kv-head-major.
+ *      time); otherwise kv-head-major;
+ *   8: with split-K partitions, one CTA streams three consecutive partitions
+ *      whenever there are several (the grouped path at any size; without
+ *      this bit it is taken for partitions under 512 KB of K/V per kv head,
+ *      about 2 MB per CTA, while the grid keeps 1.5 waves of 3 CTAs per SM).
+ *      Each partition still gets its own record, so the result is the same.
+ *      Tensor-core consumer only, and only where the CTA's extra merge area
+ *      costs no resident CTA per SM.
  * Default 4.  Every setting computes the same function.
  */
 pa_status pa_decode_select(int mode);

@@ -201,12 +201,14 @@ def pa_decode_suggest_partition(Hkv: int, block_size: int, context_lens_host) ->
 
 
 DECODE_SIMT_ONLY, DECODE_EVICT_FIRST, DECODE_PARTITION_MAJOR = 1, 2, 4
+DECODE_GROUP_PARTITIONS = 8
 DECODE_DEFAULT = DECODE_PARTITION_MAJOR
 
 
 def pa_decode_select(mode: int) -> None:
     """Bit mask: 1 CUDA-core consumer everywhere, 2 L2 evict-first K/V loads,
-    4 partition-major grid (default 4)."""
+    4 partition-major grid, 8 split-K partitions grouped three to a CTA whenever
+    there are several (default 4)."""
     _check(lib().pa_decode_select(int(mode)))
 
 

@@ -17,47 +17,67 @@ namespace {
 
 // pa_decode_select bits: 1 = CUDA-core consumer only, 2 = L2 evict-first
 // hint on K/V loads, 4 = partition-major grid (kv heads of a partition side
-// by side); the default is 4.
+// by side), 8 = group split-K partitions three to a CTA whenever there are
+// several (a test hook for the grouped path at small sizes); the default is 4.
 std::atomic<int> g_select{4};
+
+// SMs of the current device (cached per device; 148 if the query fails).
+int sm_count() {
+    static int sms[256] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 256 && !sms[dev])
+        cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+    return (dev >= 0 && dev < 256 && sms[dev] > 0) ? sms[dev] : 148;
+}
 
 // Launched as a programmatic dependent of the partition kernel so its launch
 // overlaps that grid's last wave (it waits for the grid's memory itself).
-template <int QT, int D>
+template <int QT, int D, int NW>
 cudaError_t launch_merge_t(const dec::Params& p, int wph, dim3 grid, cudaStream_t st) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
-    cfg.blockDim = dim3(dec::kMergeWarps * 32);
+    cfg.blockDim = dim3(NW * 32);
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, dec::decode_merge<QT, D>, p, wph);
+    return cudaLaunchKernelEx(&cfg, dec::decode_merge<QT, D, NW>, p, wph);
+}
+
+template <int QT, int D>
+cudaError_t launch_merge_w(const dec::Params& p, int nw, int wph, dim3 grid, cudaStream_t st) {
+    if (nw == dec::kMergeWarpsLong) return launch_merge_t<QT, D, dec::kMergeWarpsLong>(p, wph, grid, st);
+    return launch_merge_t<QT, D, dec::kMergeWarps>(p, wph, grid, st);
 }
 
 template <int QT>
-cudaError_t launch_merge_q(const dec::Params& p, int D, int wph, dim3 grid, cudaStream_t st) {
+cudaError_t launch_merge_q(const dec::Params& p, int D, int nw, int wph, dim3 grid,
+                           cudaStream_t st) {
     switch (D) {
-    case 64: return launch_merge_t<QT, 64>(p, wph, grid, st);
-    case 128: return launch_merge_t<QT, 128>(p, wph, grid, st);
-    case 256: return launch_merge_t<QT, 256>(p, wph, grid, st);
+    case 64: return launch_merge_w<QT, 64>(p, nw, wph, grid, st);
+    case 128: return launch_merge_w<QT, 128>(p, nw, wph, grid, st);
+    case 256: return launch_merge_w<QT, 256>(p, nw, wph, grid, st);
     }
     return cudaErrorNotSupported;
 }
 
-// Warps per head: enough to split a sequence's partitions, at most 8.
+// Warps per head: enough to split a sequence's partitions (8 partitions a
+// warp or fewer), at most the CTA's warps: 8, or 32 past 64 partitions.
 cudaError_t launch_merge(const dec::Params& p, pa_dtype qt, int D, int Hq, int S,
                          cudaStream_t st) {
+    const int nw = !p.balanced && p.max_parts > 64 ? dec::kMergeWarpsLong : dec::kMergeWarps;
     int wph = 1;
     if (p.balanced) wph = 2;     // pieces per item: about (item blocks / CTA range) + 1
-    else while (wph < dec::kMergeWarps && p.max_parts > 8 * wph) wph *= 2;
-    const int hpc = dec::kMergeWarps / wph;
+    else while (wph < nw && p.max_parts > 8 * wph) wph *= 2;
+    const int hpc = nw / wph;
     const dim3 grid((unsigned)((Hq + hpc - 1) / hpc), (unsigned)S);
     switch (qt) {
-    case PA_F32: return launch_merge_q<PA_F32>(p, D, wph, grid, st);
-    case PA_F16: return launch_merge_q<PA_F16>(p, D, wph, grid, st);
-    case PA_BF16: return launch_merge_q<PA_BF16>(p, D, wph, grid, st);
+    case PA_F32: return launch_merge_q<PA_F32>(p, D, nw, wph, grid, st);
+    case PA_F16: return launch_merge_q<PA_F16>(p, D, nw, wph, grid, st);
+    case PA_BF16: return launch_merge_q<PA_BF16>(p, D, nw, wph, grid, st);
     default: return cudaErrorNotSupported;
     }
 }
@@ -132,7 +152,7 @@ extern "C" pa_status pa_decode_suggest_partition(int S, int Hkv, int bs,
 
 extern "C" pa_status pa_decode_select(int mode) {
     clear_error();
-    if (mode < 0 || mode > 7) return fail(PA_ERR_INVALID_ARG, "mode must be in [0, 7]");
+    if (mode < 0 || mode > 15) return fail(PA_ERR_INVALID_ARG, "mode must be in [0, 15]");
     g_select.store(mode);
     return PA_OK;
 }
@@ -188,13 +208,35 @@ pa_status pa::decode_impl(void* out, const void* q, pa_dtype q_dt, const void* k
                               : prefix_parts > 0
                                   ? std::max<int64_t>(parts_for(max_ctx, partition), prefix_parts + 1)
                                   : parts_for(max_ctx, partition);
-    const int64_t grid_parts = fuse ? 1 : prefix_parts > 0 ? max_parts - prefix_parts : max_parts;
     if (max_parts > 65535 || (int64_t)Hkv * G > 65535)
         return fail(PA_ERR_UNSUPPORTED, "too many partitions or heads for the grid");
     const int sel = g_select.load();
     const bool use_mma = !(sel & 1) && G >= 2 && D <= 128 && cache_dt != PA_F32;
     const int gc_simt = G < (D == 256 ? 2 : 4) ? G : (D == 256 ? 2 : 4);
     const int gc = use_mma ? G : gc_simt;
+    const int chunks = use_mma ? 1 : G / gc_simt;
+    const int num_sms = sm_count();
+    // Plain split-K with short partitions: one CTA streams several consecutive
+    // partitions (each still its own record), about 2 MB of K/V per CTA, while
+    // the grid keeps at least 1.5 waves of 3 CTAs per SM.  Each CTA pays a
+    // start-up and drain of a few microseconds, which a 512-token partition
+    // (256 KB at D 128, 16-bit) does not amortise.
+    int part_group = 1;
+    if (!balanced && !fuse && prefix_parts == 0 && !force_ws && max_parts > 1) {
+        const int64_t part_bytes = (int64_t)partition * D * elem_size(cache_dt) * 2;
+        if (sel & 8) {
+            part_group = 3;
+        } else if (part_bytes < (512 << 10)) {
+            int64_t g = std::min<int64_t>(max_parts, ((2 << 20) + part_bytes - 1) / part_bytes);
+            const int64_t units = (int64_t)S * Hkv * chunks;
+            const int64_t min_ctas = (int64_t)num_sms * 3 * 3 / 2;
+            while (g > 1 && units * ((max_parts + g - 1) / g) < min_ctas) --g;
+            part_group = (int)g;
+        }
+    }
+    const int64_t grid_parts = fuse ? 1
+                               : prefix_parts > 0 ? max_parts - prefix_parts
+                                                  : (max_parts + part_group - 1) / part_group;
     size_t need = 0;
     if (balanced) need = balanced_bytes(S, Hq, D, gc);
     else if (force_ws || fuse) need = (size_t)S * Hq * max_parts * (sizeof(float) * 2 + sizeof(float) * D);
@@ -228,6 +270,7 @@ pa_status pa::decode_impl(void* out, const void* q, pa_dtype q_dt, const void* k
     p.prefix_parts = prefix_parts;
     p.force_ws = force_ws ? 1 : 0;
     p.fuse_prefix_blocks = fuse_prefix_blocks;
+    p.part_group = part_group;
     p.max_ctx = max_ctx;
     p.evict_first = (sel & 2) ? 1 : 0;
     p.heads_fastest = (sel & 4) ? 1 : 0;
@@ -259,15 +302,7 @@ pa_status pa::decode_impl(void* out, const void* q, pa_dtype q_dt, const void* k
     L.gc = gc_simt;
     L.balanced = balanced;
     L.G = G;
-    if (balanced) {
-        static int sms[256] = {};
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (dev >= 0 && dev < 256 && !sms[dev])
-            cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
-        L.num_sms = (dev >= 0 && dev < 256 && sms[dev] > 0) ? sms[dev] : 148;
-    }
-    const int chunks = L.mma ? 1 : G / L.gc;
+    L.num_sms = num_sms;
     L.grid = p.heads_fastest ? dim3((unsigned)(Hkv * chunks), (unsigned)grid_parts, (unsigned)S)
                              : dim3((unsigned)grid_parts, (unsigned)(Hkv * chunks), (unsigned)S);
     L.stream = reinterpret_cast<cudaStream_t>(stream);

@@ -72,6 +72,8 @@ struct Params {
     int fuse_prefix_blocks;      // > 0: shared-prefix decode with one CTA per (sequence, kv
                                  // head) over the suffix past this many blocks; its epilogue
                                  // merges the prefix_parts prefix records and writes the output
+    int part_group;              // plain split-K: consecutive partitions one CTA streams (>= 1),
+                                 // still one record per partition
 };
 
 // Record a wait that gave up, with the site that gave up (bits 16-23).
@@ -221,6 +223,17 @@ __device__ __forceinline__ void simt_load_q(SimtState<C>& st, const Params& p, i
             for (int e = 0; e < C::EPC; ++e)
                 st.q[g][k * C::EPC + e] =
                     dev::load_q<C::QT>(p.q, base + k * C::EPS + l8 * C::EPC + e) * p.qk_scale;
+        #pragma unroll
+        for (int j = 0; j < C::DPL; ++j) st.acc[g][j] = 0.f;
+        st.m[g] = -INFINITY;
+        st.l[g] = 0.f;
+    }
+}
+
+template <class C>
+__device__ __forceinline__ void simt_reset(SimtState<C>& st) {
+    #pragma unroll
+    for (int g = 0; g < C::GC; ++g) {
         #pragma unroll
         for (int j = 0; j < C::DPL; ++j) st.acc[g][j] = 0.f;
         st.m[g] = -INFINITY;
@@ -747,8 +760,46 @@ __device__ __forceinline__ void mma_publish(MmaState<C>& st, float* cm, float* c
     }
 }
 
-// ----------------------------------------------------------------- kernel
 template <class C>
+__device__ __forceinline__ void mma_reset(MmaState<C>& st) {
+    using S = MmaState<C>;
+    #pragma unroll
+    for (int nh = 0; nh < S::NH; ++nh) {
+        #pragma unroll
+        for (int md = 0; md < S::MD; ++md)
+            #pragma unroll
+            for (int i = 0; i < 4; ++i) st.o[nh][md][i] = 0.f;
+        st.m[nh][0] = st.m[nh][1] = -INFINITY;
+        st.l[nh][0] = st.l[nh][1] = 0.f;
+    }
+}
+
+// Barrier 1 over the consumer warps only (the producer keeps streaming).
+template <class C>
+__device__ __forceinline__ void consumers_sync() {
+    asm volatile("bar.sync 1, %0;" ::"n"(C::NW * 32) : "memory");
+}
+// The same barrier, returning whether any consumer thread passed `pred`.
+template <class C>
+__device__ __forceinline__ bool consumers_sync_or(bool pred) {
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+                 "bar.red.or.pred q, 1, %2, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+                 : "=r"(r) : "r"((uint32_t)pred), "n"(C::NW * 32) : "memory");
+    return r != 0;
+}
+
+// Smem bytes of the per-partition warp merge area of the grouped-partition
+// mode (it cannot reuse the stages, which keep streaming).
+template <class C>
+constexpr size_t group_merge_bytes(int heads) {
+    return size_t(C::NW) * heads * (C::D + 2) * sizeof(float);
+}
+
+// ----------------------------------------------------------------- kernel
+// GROUPED: the grouped-partition instantiation (p.part_group > 1, plain
+// split-K only); the other one is launched with p.part_group == 1.
+template <class C, bool GROUPED>
 __global__ void __launch_bounds__(C::THREADS, C::MMA ? 3 : 2)
 decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                  const Params p) {
@@ -772,6 +823,7 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     const int n = checked_len(p, s, C::BS);
     const int nblk_all = (n + C::BS - 1) / C::BS;
     int blk0 = 0, nblk = nblk_all, nparts = 1;
+    int q0 = part, nq = 1;                      // partitions (records) this CTA writes
     bool fuse_records = false;
     if (p.fuse_prefix_blocks > 0) {
         // A sequence whose table starts with row 0's prefix blocks (and that
@@ -821,9 +873,12 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
         }
         nparts = 2;                             // records always go through the workspace
     } else if (p.part_blocks > 0) {
-        blk0 = part * p.part_blocks;
-        nblk = min(p.part_blocks, nblk_all - blk0);
+        // grid index `part` covers partitions q0 .. q0 + part_group - 1
+        q0 = part * p.part_group;
+        blk0 = q0 * p.part_blocks;
+        nblk = min(p.part_group * p.part_blocks, nblk_all - blk0);
         nparts = max(1, (nblk_all + p.part_blocks - 1) / p.part_blocks);
+        nq = min(p.part_group, nparts - q0);
     }
     if (part > 0 && nblk <= 0) return;          // this sequence has fewer partitions
     nblk = max(nblk, 0);
@@ -852,6 +907,90 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
 
     using State = typename std::conditional<C::MMA, MmaState<C>, SimtState<C>>::type;
     State st;
+    if constexpr (GROUPED) {
+        // Grouped partitions: the producer streams the blocks of all nq
+        // partitions without a break; the consumers close each partition with
+        // a warp merge through a dedicated area (the stages keep streaming)
+        // and write its record, exactly as nq one-partition CTAs would.
+        const int gh = gc;
+        float* gm = reinterpret_cast<float*>(vstage + (size_t)C::NW * C::VSTG + 16 * C::STAGES);
+        float* gl = gm + C::NW * gh;
+        float* go = gl + C::NW * gh;
+        if (warp == C::NW) {
+            int k = 0;
+            produce<C>(&tmk, &tmv, p, p.block_tables + (size_t)s * p.MB, blk0, nblk, kvh, stages,
+                       full0, empty0, &s_abort, &k);
+            if (lane == 0) s_issued = k;
+        } else {
+            if constexpr (C::MMA) mma_load_q<C>(st, p, s, h0, G);
+            else simt_load_q<C>(st, p, s, h0);
+            bool stop = false;
+            for (int qq = 0; qq < nq; ++qq) {
+                const int jb = qq * p.part_blocks, je = min(jb + p.part_blocks, nblk);
+                // this warp's blocks: j % NW == warp (the stage ring's owner rule)
+                for (int j = jb + (warp - jb % C::NW + C::NW) % C::NW; j < je && !stop;
+                     j += C::NW) {
+                    const int stg = j % C::STAGES;
+                    if (!dev::mbar_wait_bounded(full0 + 8 * stg, (j / C::STAGES) & 1)) {
+                        if (lane == 0) { wait_timeout(p, 2); s_abort = 1; }
+                        stop = true;
+                        break;
+                    }
+                    uint8_t* kt = stages + (size_t)stg * C::STAGE;
+                    const int nvalid = min(C::BS, n - (blk0 + j) * C::BS);
+                    if constexpr (C::MMA)
+                        mma_block<C>(st, kt, kt + C::TILE, vstage + warp * C::VSTG, nvalid,
+                                     p.qk_scale);
+                    else simt_block<C>(st, kt, kt + C::TILE, nvalid);
+                    __syncwarp();
+                    if (lane == 0) dev::mbar_arrive(empty0 + 8 * stg);
+                    if (*(volatile int*)&s_abort) stop = true;
+                }
+                if constexpr (C::MMA) mma_publish<C>(st, gm, gl, go, warp, G, gh);
+                else simt_publish<C>(st, gm, gl, go, warp);
+                consumers_sync<C>();
+                if (!*(volatile int*)&s_abort) {
+                    for (int idx = threadIdx.x; idx < gh * C::D; idx += C::NW * 32) {
+                        const int g = idx / C::D, d = idx % C::D;
+                        float M = -INFINITY;
+                        #pragma unroll
+                        for (int w = 0; w < C::NW; ++w) M = fmaxf(M, gm[w * gh + g]);
+                        float L = 0.f, O = 0.f;
+                        if (M != -INFINITY) {
+                            #pragma unroll
+                            for (int w = 0; w < C::NW; ++w) {
+                                const float f = exp2f(gm[w * gh + g] - M);
+                                L = fmaf(f, gl[w * gh + g], L);
+                                O = fmaf(f, go[(w * gh + g) * C::D + d], O);
+                            }
+                        }
+                        const int h = h0 + g;
+                        if (nparts == 1) {
+                            dev::store_out<C::QT>(p.out, ((size_t)s * p.Hq + h) * C::D + d,
+                                                  L > 0.f ? (O / L) * p.v_scale : 0.f);
+                        } else {
+                            const size_t row = ((size_t)s * p.Hq + h) * p.max_parts + q0 + qq;
+                            p.ws_o[row * C::D + d] = O * p.v_scale;
+                            if (d == 0) p.ws_ml[row] = make_float2(M, L);
+                        }
+                    }
+                }
+                // the merge area is free again; leave together on an abort
+                if (consumers_sync_or<C>(stop || *(volatile int*)&s_abort)) break;
+                if constexpr (C::MMA) mma_reset<C>(st);
+                else simt_reset<C>(st);
+            }
+        }
+        __syncthreads();
+        dev::launch_dependents();
+        if (s_abort && warp == C::NW && lane == 0) {
+            // drain: every issued copy lands before the CTA leaves (bounded)
+            const int issued = s_issued;
+            for (int j = max(0, issued - C::STAGES); j < issued; ++j)
+                dev::mbar_wait_bounded(full0 + 8 * (j % C::STAGES), (j / C::STAGES) & 1);
+        }
+        return;
+    }
     if (warp == C::NW) {
         int k = 0;
         produce<C>(&tmk, &tmv, p, p.block_tables + (size_t)s * p.MB, blk0, nblk, kvh, stages,
@@ -1221,21 +1360,24 @@ decode_balanced(const __grid_constant__ CUtensorMap tmk, const __grid_constant__
 }
 
 // Merge split-K partials: out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p.
-// A CTA of 8 warps serves 8 / wph query heads of one sequence; the wph warps
-// of a head split its partitions, and each lane holds D/32 dims, so every
-// partial row is one coalesced load.  Launched as a programmatic dependent of
-// the partition kernel: it waits for that grid's memory before reading.
+// A CTA of NWARPS warps serves NWARPS / wph query heads of one sequence; the
+// wph warps of a head split its partitions, and each lane holds D/32 dims, so
+// every partial row is one coalesced load.  8 warps by default; 32 for long
+// contexts, whose hundreds of partials per head would otherwise be a chain of
+// dependent loads per warp.  Launched as a programmatic dependent of the
+// partition kernel: it waits for that grid's memory before reading.
 constexpr int kMergeWarps = 8;
+constexpr int kMergeWarpsLong = 32;
 
-template <int QT, int D>
-__global__ void __launch_bounds__(kMergeWarps * 32) decode_merge(const Params p, int wph) {
+template <int QT, int D, int NWARPS>
+__global__ void __launch_bounds__(NWARPS * 32) decode_merge(const Params p, int wph) {
     constexpr int DL = D / 32;                        // dims per lane
-    __shared__ float s_max[kMergeWarps];
-    __shared__ float s_l[kMergeWarps];
-    __shared__ __align__(16) float s_o[kMergeWarps][D];
-    __shared__ int s_live[kMergeWarps];
+    __shared__ float s_max[NWARPS];
+    __shared__ float s_l[NWARPS];
+    __shared__ __align__(16) float s_o[NWARPS][D];
+    __shared__ int s_live[NWARPS];
     dev::grid_dependency_wait();
-    const int hpc = kMergeWarps / wph;                // heads per CTA
+    const int hpc = NWARPS / wph;                // heads per CTA
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int hl = warp / wph, sub = warp % wph;
     const int h = blockIdx.x * hpc + hl, s = blockIdx.y;

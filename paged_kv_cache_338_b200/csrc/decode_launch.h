@@ -49,12 +49,38 @@ cudaError_t launch_one(const Launch& L) {
         kern<<<dim3((unsigned)ctas), C::THREADS, smem, L.stream>>>(L.tmk, L.tmv, L.p);
         return cudaGetLastError();
     }
-    auto kern = decode_partition<C>;
+    Params p = L.p;
+    if constexpr (C::MMA) if (p.part_group > 1) {
+        // Grouped partitions need a warp-merge area of their own; use them
+        // only if it costs no resident CTA per SM.
+        auto kern = decode_partition<C, true>;
+        const size_t big = C::SMEM + group_merge_bytes<C>(L.G);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(big));
+        if (e != cudaSuccess) return e;
+        int occ1 = 0, occ2 = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ1, decode_partition<C, false>,
+                                                          C::THREADS, C::SMEM);
+        if (e != cudaSuccess) return e;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ2, kern, C::THREADS, big);
+        if (e != cudaSuccess) return e;
+        if (occ2 >= occ1 && occ2 > 0) {
+            kern<<<L.grid, C::THREADS, big, L.stream>>>(L.tmk, L.tmv, p);
+            return cudaGetLastError();
+        }
+    }
+    // one partition per CTA
+    dim3 grid = L.grid;
+    if (p.part_group > 1) {
+        p.part_group = 1;
+        (p.heads_fastest ? grid.y : grid.x) = (unsigned)p.max_parts;
+    }
+    auto kern = decode_partition<C, false>;
     // opt in to > 48 KB of dynamic shared memory (idempotent, cheap)
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(C::SMEM));
     if (e != cudaSuccess) return e;
-    kern<<<L.grid, C::THREADS, C::SMEM, L.stream>>>(L.tmk, L.tmv, L.p);
+    kern<<<grid, C::THREADS, C::SMEM, L.stream>>>(L.tmk, L.tmv, p);
     return cudaGetLastError();
 }
 

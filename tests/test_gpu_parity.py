@@ -87,7 +87,8 @@ def _check_out(got: torch.Tensor, want: np.ndarray, dt: str, what: str):
 
 
 MODES = [pa.DECODE_DEFAULT, pa.DECODE_DEFAULT | pa.DECODE_SIMT_ONLY,
-         pa.DECODE_DEFAULT | pa.DECODE_EVICT_FIRST, 0]
+         pa.DECODE_DEFAULT | pa.DECODE_EVICT_FIRST, 0,
+         pa.DECODE_DEFAULT | pa.DECODE_GROUP_PARTITIONS, pa.DECODE_GROUP_PARTITIONS]
 BOTH = [pa.DECODE_DEFAULT, pa.DECODE_DEFAULT | pa.DECODE_SIMT_ONLY]
 
 
@@ -102,7 +103,8 @@ SMALL = [
 
 @pytest.mark.parametrize("name,cfg", SMALL, ids=[n for n, _ in SMALL])
 @pytest.mark.parametrize("partition_blocks", [0, 2, 7, -1], ids=["single", "p2", "p7", "balanced"])
-@pytest.mark.parametrize("mode", MODES, ids=["auto", "simt", "evict_first", "head_major"])
+@pytest.mark.parametrize("mode", MODES, ids=["auto", "simt", "evict_first", "head_major",
+                                            "grouped", "grouped_head_major"])
 def test_step_parity_small(name, cfg, partition_blocks, mode):
     inp = wl.make_decode_inputs(cfg, seed=101)
     want, kc_o, vc_o = oracle_step(inp)
@@ -142,7 +144,7 @@ def test_lengths_at_partition_edges(dt):
                           fixed_lens=lens, fp8_scaled=dt == "fp8_e4m3")
     inp = wl.make_decode_inputs(cfg, seed=7)
     want, _, _ = oracle_step(inp)
-    for mode in BOTH:
+    for mode in BOTH + [pa.DECODE_DEFAULT | pa.DECODE_GROUP_PARTITIONS]:
         for part in (P, -1):
             out, _, _ = gpu_step(inp, part, mode)
             _check_out(out, want, dt, f"mode={mode} P={part}")
@@ -152,10 +154,11 @@ def test_zero_length_sequences_give_zero_rows():
     cfg = wl.DecodeConfig("empty", 3, 8, 2, 128, 16, "bf16", "bf16", 0, 0, fixed_lens=(0, 40, 0))
     inp = wl.make_decode_inputs(cfg, seed=3)
     want, _, _ = oracle_step(inp)
-    for part in (0, 16, -1):
-        out, _, _ = gpu_step(inp, part)
+    for part, mode in ((0, pa.DECODE_DEFAULT), (16, pa.DECODE_DEFAULT), (-1, pa.DECODE_DEFAULT),
+                       (16, pa.DECODE_DEFAULT | pa.DECODE_GROUP_PARTITIONS)):
+        out, _, _ = gpu_step(inp, part, mode)
         assert (out[0] == 0).all() and (out[2] == 0).all()
-        _check_out(out, want, "bf16", f"P={part}")
+        _check_out(out, want, "bf16", f"P={part} mode={mode}")
 
 
 def test_device_errors_are_reported_not_followed():
