@@ -235,7 +235,8 @@ pa_status pa_decode_noalloc(void* out, const void* q, pa_dtype q_dt,
  *   8: with split-K partitions, one CTA streams three consecutive partitions
  *      whenever there are several (the grouped path at any size; without
  *      this bit it is taken for partitions under 512 KB of K/V per kv head,
- *      about 2 MB per CTA, while the grid keeps 1.5 waves of 3 CTAs per SM).
+ *      with the count per CTA that minimises full waves of resident CTAs
+ *      times each CTA's bytes plus its start-up).
  *      Each partition still gets its own record, so the result is the same.
  *      Tensor-core consumer only, and only where the CTA's extra merge area
  *      costs no resident CTA per SM.

@@ -216,22 +216,31 @@ pa_status pa::decode_impl(void* out, const void* q, pa_dtype q_dt, const void* k
     const int gc = use_mma ? G : gc_simt;
     const int chunks = use_mma ? 1 : G / gc_simt;
     const int num_sms = sm_count();
-    // Plain split-K with short partitions: one CTA streams several consecutive
-    // partitions (each still its own record), about 2 MB of K/V per CTA, while
-    // the grid keeps at least 1.5 waves of 3 CTAs per SM.  Each CTA pays a
-    // start-up and drain of a few microseconds, which a 512-token partition
-    // (256 KB at D 128, 16-bit) does not amortise.
+    // Plain split-K with short partitions: one CTA streams g consecutive
+    // partitions (each still its own record).  g minimises a simple model of
+    // the grid's time for equal-length sequences: the number of full waves of
+    // resident CTAs (3 per SM; a part-filled last wave costs nearly a whole
+    // one, since a lone CTA cannot pull its SM's share of HBM) times what a
+    // CTA streams plus its start-up and drain (about 6 us on the 4 x 100k
+    // workload, some 160 KB of a CTA's streaming).  Ties go to the larger g,
+    // the fewer CTAs.
     int part_group = 1;
     if (!balanced && !fuse && prefix_parts == 0 && !force_ws && max_parts > 1) {
         const int64_t part_bytes = (int64_t)partition * D * elem_size(cache_dt) * 2;
         if (sel & 8) {
             part_group = 3;
         } else if (part_bytes < (512 << 10)) {
-            int64_t g = std::min<int64_t>(max_parts, ((2 << 20) + part_bytes - 1) / part_bytes);
             const int64_t units = (int64_t)S * Hkv * chunks;
-            const int64_t min_ctas = (int64_t)num_sms * 3 * 3 / 2;
-            while (g > 1 && units * ((max_parts + g - 1) / g) < min_ctas) --g;
-            part_group = (int)g;
+            const int64_t slots = 3LL * num_sms;
+            double best = 0.0;
+            for (int64_t g = 1; g <= std::min<int64_t>(max_parts, 4096); ++g) {
+                const int64_t waves = (units * ((max_parts + g - 1) / g) + slots - 1) / slots;
+                const double t = (double)waves * (double)(g * part_bytes + (160 << 10));
+                if (g == 1 || t <= best) {
+                    best = t;
+                    part_group = (int)g;
+                }
+            }
         }
     }
     const int64_t grid_parts = fuse ? 1
