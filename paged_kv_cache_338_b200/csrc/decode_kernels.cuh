@@ -34,6 +34,12 @@
 //        accumulator layout is the A-operand layout of the second product).
 //  * With more than one partition, (m, l, o) go to the fp32 workspace and
 //    decode_merge combines them; otherwise the CTA writes out directly.
+//  * Short partitions (decode_partition<C, true>): one CTA streams several
+//    consecutive partitions of one (sequence, kv head) without draining its
+//    ring, closes each with the warp merge through an smem area of its own
+//    and writes that partition's record, so the split and its reduce are
+//    those of one CTA per partition while the start-up and drain of a CTA
+//    are paid once per group.
 #pragma once
 
 #include <type_traits>
