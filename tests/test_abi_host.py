@@ -81,6 +81,18 @@ def test_host_argument_checks():
                                   1.0, 1.0, None) == 0
 
 
+def test_decode_select_modes():
+    """Every documented bit combination is accepted (0..15, bit 8 included)
+    and anything else refused; the default is restored afterwards."""
+    try:
+        for mode in range(16):
+            pa.pa_decode_select(mode)
+        for bad in (-1, 16, 64):
+            _bad(pa.pa_decode_select, bad)
+    finally:
+        pa.pa_decode_select(pa.DECODE_DEFAULT)
+
+
 def test_copy_blocks_host_rejections():
     kc = torch.zeros((8, 16, 2, 64), dtype=torch.bfloat16)   # host memory: never launched
     for bad in ([[1, 2], [3, 2]], [[1, 2], [2, 4]], [[1, 8]], [[-1, 3]]):
