@@ -65,6 +65,8 @@ __global__ void reshape_and_cache_kernel(const uint8_t* __restrict__ key,
                                          const int64_t* __restrict__ slots, int T, int HkvD,
                                          int64_t nslots, float k_scale, float v_scale,
                                          unsigned int* err) {
+    dev::grid_dependency_wait();       // launched as a dependent of the kernel before it
+    dev::launch_dependents();
     constexpr int ein = dev::Storage<IN>::bytes;
     constexpr int per = TO_FP8 ? 8 : 16 / ein;                 // elements per thread
     const int per_row = HkvD / per;
@@ -127,10 +129,10 @@ cudaError_t launch_append(const void* key, const void* value, void* kc, void* vc
     const int threads = 256;
     int64_t blocks = (total + threads - 1) / threads;
     if (blocks > 148 * 16) blocks = 148 * 16;
-    reshape_and_cache_kernel<IN, TO_FP8><<<(unsigned)blocks, threads, 0, st>>>(
-        static_cast<const uint8_t*>(key), static_cast<const uint8_t*>(value),
-        static_cast<uint8_t*>(kc), static_cast<uint8_t*>(vc), slots, T, HkvD, nslots, ks, vs, err);
-    return cudaGetLastError();
+    return dev::launch_pdl(reshape_and_cache_kernel<IN, TO_FP8>, dim3((unsigned)blocks),
+                           dim3(threads), 0, st, static_cast<const uint8_t*>(key),
+                           static_cast<const uint8_t*>(value), static_cast<uint8_t*>(kc),
+                           static_cast<uint8_t*>(vc), slots, T, HkvD, nslots, ks, vs, err);
 }
 
 // ------------------------------------------------------------- block copy
@@ -145,6 +147,8 @@ struct CopyList {
 __global__ void __launch_bounds__(256) copy_blocks_kernel(uint8_t* __restrict__ kc,
                                                           uint8_t* __restrict__ vc, size_t block_bytes,
                                                           const __grid_constant__ CopyList list) {
+    dev::grid_dependency_wait();       // launched as a dependent of the kernel before it
+    dev::launch_dependents();
     const int2 pr = list.pair[blockIdx.x];
     uint8_t* base = blockIdx.y ? vc : kc;
     const uint4* src = reinterpret_cast<const uint4*>(base + (size_t)pr.x * block_bytes);
@@ -268,9 +272,9 @@ extern "C" pa_status pa_copy_blocks(void* key_cache, void* value_cache, size_t b
         list.n = n - off < kMaxPairsPerLaunch ? n - off : kMaxPairsPerLaunch;
         for (int i = 0; i < list.n; ++i)
             list.pair[i] = make_int2(pairs[2 * (off + i)], pairs[2 * (off + i) + 1]);
-        copy_blocks_kernel<<<dim3((unsigned)list.n, 2), 256, 0, st>>>(
-            static_cast<uint8_t*>(key_cache), static_cast<uint8_t*>(value_cache), block_bytes, list);
-        cudaError_t e = cudaGetLastError();
+        cudaError_t e = dev::launch_pdl(copy_blocks_kernel, dim3((unsigned)list.n, 2), dim3(256), 0,
+                                        st, static_cast<uint8_t*>(key_cache),
+                                        static_cast<uint8_t*>(value_cache), block_bytes, list);
         if (e != cudaSuccess) return cuda_fail(e, "copy_blocks launch");
     }
     return PA_OK;

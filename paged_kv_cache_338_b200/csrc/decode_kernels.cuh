@@ -809,6 +809,7 @@ template <class C, bool GROUPED>
 __global__ void __launch_bounds__(C::THREADS, C::MMA ? 3 : 2)
 decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                  const Params p) {
+    dev::grid_dependency_wait();       // launched as a dependent of the kernel before it
     extern __shared__ uint8_t smem_raw[];
     __shared__ int s_abort;
     __shared__ int s_issued;
@@ -1129,6 +1130,7 @@ template <class C0>
 __global__ void __launch_bounds__(C0::THREADS, 3)
 decode_balanced(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                 const Params p) {
+    dev::grid_dependency_wait();       // launched as a dependent of the kernel before it
     using B = BalancedSmem<C0>;
     using C = Balanced<C0>;
     constexpr int STAGES = B::STAGES;

@@ -46,8 +46,8 @@ cudaError_t launch_one(const Launch& L) {
         if (per_sm < 1) per_sm = 1;
         int ctas = per_sm * L.num_sms;
         if (ctas > kMaxBalancedCtas) ctas = kMaxBalancedCtas;
-        kern<<<dim3((unsigned)ctas), C::THREADS, smem, L.stream>>>(L.tmk, L.tmv, L.p);
-        return cudaGetLastError();
+        return dev::launch_pdl(kern, dim3((unsigned)ctas), dim3(C::THREADS), (size_t)smem,
+                               L.stream, L.tmk, L.tmv, L.p);
     }
     Params p = L.p;
     if constexpr (C::MMA) if (p.part_group > 1) {
@@ -65,8 +65,8 @@ cudaError_t launch_one(const Launch& L) {
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ2, kern, C::THREADS, big);
         if (e != cudaSuccess) return e;
         if (occ2 >= occ1 && occ2 > 0) {
-            kern<<<L.grid, C::THREADS, big, L.stream>>>(L.tmk, L.tmv, p);
-            return cudaGetLastError();
+            return dev::launch_pdl(kern, L.grid, dim3(C::THREADS), big, L.stream, L.tmk, L.tmv,
+                                   p);
         }
     }
     // one partition per CTA
@@ -80,8 +80,7 @@ cudaError_t launch_one(const Launch& L) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(C::SMEM));
     if (e != cudaSuccess) return e;
-    kern<<<grid, C::THREADS, C::SMEM, L.stream>>>(L.tmk, L.tmv, p);
-    return cudaGetLastError();
+    return dev::launch_pdl(kern, grid, dim3(C::THREADS), C::SMEM, L.stream, L.tmk, L.tmv, p);
 }
 
 template <int DT, int D>
