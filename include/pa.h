@@ -224,6 +224,18 @@ pa_status pa_decode_noalloc(void* out, const void* q, pa_dtype q_dt,
                             pa_stream_t stream);
 
 /*
+ * How many consecutive split-K partitions one pa_decode CTA streams for this
+ * shape (the grouped path of bit 8 below; each partition still writes its own
+ * record, so the result does not depend on it).  Plain split-K (partition >
+ * 0) with the tensor-core consumer only; num_sms <= 0 means the current
+ * device's SM count (148 without a device).  It is the planned value: the
+ * launch falls back to 1 where the group's merge area would cost a resident
+ * CTA per SM (fp8 tiles, 16-head groups).  *group >= 1 on success.
+ */
+pa_status pa_decode_partition_group(int S, int Hq, int Hkv, int D, pa_dtype cache_dt, int max_ctx,
+                                    int partition, int num_sms, int* group);
+
+/*
  * Kernel selection and tuning for pa_decode (process-wide; for tests and
  * tuning), a bit mask:
  *   1: CUDA-core consumer everywhere (otherwise grouped-query heads with

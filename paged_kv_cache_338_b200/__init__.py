@@ -21,7 +21,7 @@ import torch
 __all__ = [
     "PaError", "lib", "pa_version", "pa_last_error", "pa_device_status",
     "pa_reshape_and_cache", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_size",
-    "pa_decode_suggest_partition", "pa_decode_select", "pa_decode_noalloc", "pa_prefill",
+    "pa_decode_suggest_partition", "pa_decode_partition_group", "pa_decode_select", "pa_decode_noalloc", "pa_prefill",
     "pa_decode_shared_prefix", "pa_decode_shared_prefix_workspace_size",
     "BlockPool",
     "PA_DEV_BAD_SLOT", "PA_DEV_BAD_BLOCK", "PA_DEV_WAIT_TIMEOUT", "PA_DEV_BAD_CONTEXT",
@@ -76,6 +76,7 @@ def lib() -> ctypes.CDLL:
         "pa_copy_blocks": ([P, P, SZ, I64, P, I, P], I),
         "pa_decode_workspace_size": ([I, I, I, I, I, ctypes.POINTER(SZ)], I),
         "pa_decode_suggest_partition": ([I, I, I, P, ctypes.POINTER(I)], I),
+        "pa_decode_partition_group": ([I, I, I, I, I, I, I, I, ctypes.POINTER(I)], I),
         "pa_decode_select": ([I], I),
         "pa_decode": ([P, P, I, P, P, I, P, I, P, I, I, I, I, I, I64, I, F, F, F, I, P, SZ, P], I),
         "pa_decode_noalloc": ([P, P, I, P, P, I, P, I, P, I, I, I, I, I, I64, I, F, F, F, I, P], I),
@@ -197,6 +198,17 @@ def pa_decode_suggest_partition(Hkv: int, block_size: int, context_lens_host) ->
     _check(lib().pa_decode_suggest_partition(cl.numel(), Hkv, block_size,
                                              cl.data_ptr() if cl.numel() else None,
                                              ctypes.byref(out)))
+    return out.value
+
+
+def pa_decode_partition_group(S: int, Hq: int, Hkv: int, D: int, cache_dtype, max_ctx: int,
+                              partition: int, num_sms: int = 0) -> int:
+    """Consecutive split-K partitions one pa_decode CTA streams for this shape
+    (planned; each partition keeps its own record)."""
+    dt = _TORCH_DT[cache_dtype] if isinstance(cache_dtype, torch.dtype) else int(cache_dtype)
+    out = ctypes.c_int(0)
+    _check(lib().pa_decode_partition_group(S, Hq, Hkv, D, dt, max_ctx, partition, num_sms,
+                                           ctypes.byref(out)))
     return out.value
 
 

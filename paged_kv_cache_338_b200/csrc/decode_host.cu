@@ -21,6 +21,33 @@ namespace {
 // several (a test hook for the grouped path at small sizes); the default is 4.
 std::atomic<int> g_select{4};
 
+// Plain split-K with short partitions: one CTA streams g consecutive
+// partitions (each still its own record).  g minimises a simple model of
+// the grid's time for equal-length sequences: the number of full waves of
+// resident CTAs (3 per SM; a part-filled last wave costs nearly a whole
+// one, since a lone CTA cannot pull its SM's share of HBM) times what a
+// CTA streams plus its start-up and drain (about 6 us on the 4 x 100k
+// workload, some 160 KB of a CTA's streaming).  Ties go to the larger g,
+// the fewer CTAs.
+// units: CTAs one partition per CTA would need per partition index (sequences
+// x kv heads x head chunks); part_bytes: K/V bytes of one partition of one kv
+// head.  Partitions of 512 KB or more are long enough on their own: g = 1.
+int plan_part_group(int64_t units, int64_t max_parts, int64_t part_bytes, int num_sms) {
+    if (max_parts <= 1 || part_bytes >= (512 << 10)) return 1;
+    const int64_t slots = 3LL * (num_sms > 0 ? num_sms : 148);
+    double best = 0.0;
+    int group = 1;
+    for (int64_t g = 1; g <= std::min<int64_t>(max_parts, 4096); ++g) {
+        const int64_t waves = (units * ((max_parts + g - 1) / g) + slots - 1) / slots;
+        const double t = (double)waves * (double)(g * part_bytes + (160 << 10));
+        if (g == 1 || t <= best) {
+            best = t;
+            group = (int)g;
+        }
+    }
+    return group;
+}
+
 // SMs of the current device (cached per device; 148 if the query fails).
 int sm_count() {
     static int sms[256] = {};
@@ -150,6 +177,26 @@ extern "C" pa_status pa_decode_suggest_partition(int S, int Hkv, int bs,
     return PA_OK;
 }
 
+extern "C" pa_status pa_decode_partition_group(int S, int Hq, int Hkv, int D, pa_dtype cache_dt,
+                                               int max_ctx, int partition, int num_sms,
+                                               int* group) {
+    clear_error();
+    if (!group || S < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || max_ctx < 0 || partition < 0 ||
+        !valid_dtype(cache_dt) || !(D == 64 || D == 128 || D == 256))
+        return fail(PA_ERR_INVALID_ARG, "bad arguments");
+    const int G = Hq / Hkv;
+    const int sel = g_select.load();
+    const bool use_mma = !(sel & 1) && G >= 2 && D <= 128 && cache_dt != PA_F32;
+    const int64_t max_parts = partition > 0 ? parts_for(max_ctx, partition) : 1;
+    *group = 1;
+    if (use_mma && max_parts > 1)
+        *group = (sel & 8) ? 3
+                           : plan_part_group((int64_t)S * Hkv, max_parts,
+                                             (int64_t)partition * D * elem_size(cache_dt) * 2,
+                                             num_sms > 0 ? num_sms : sm_count());
+    return PA_OK;
+}
+
 extern "C" pa_status pa_decode_select(int mode) {
     clear_error();
     if (mode < 0 || mode > 15) return fail(PA_ERR_INVALID_ARG, "mode must be in [0, 15]");
@@ -216,33 +263,12 @@ pa_status pa::decode_impl(void* out, const void* q, pa_dtype q_dt, const void* k
     const int gc = use_mma ? G : gc_simt;
     const int chunks = use_mma ? 1 : G / gc_simt;
     const int num_sms = sm_count();
-    // Plain split-K with short partitions: one CTA streams g consecutive
-    // partitions (each still its own record).  g minimises a simple model of
-    // the grid's time for equal-length sequences: the number of full waves of
-    // resident CTAs (3 per SM; a part-filled last wave costs nearly a whole
-    // one, since a lone CTA cannot pull its SM's share of HBM) times what a
-    // CTA streams plus its start-up and drain (about 6 us on the 4 x 100k
-    // workload, some 160 KB of a CTA's streaming).  Ties go to the larger g,
-    // the fewer CTAs.
     int part_group = 1;
-    if (!balanced && !fuse && prefix_parts == 0 && !force_ws && max_parts > 1) {
-        const int64_t part_bytes = (int64_t)partition * D * elem_size(cache_dt) * 2;
-        if (sel & 8) {
-            part_group = 3;
-        } else if (part_bytes < (512 << 10)) {
-            const int64_t units = (int64_t)S * Hkv * chunks;
-            const int64_t slots = 3LL * num_sms;
-            double best = 0.0;
-            for (int64_t g = 1; g <= std::min<int64_t>(max_parts, 4096); ++g) {
-                const int64_t waves = (units * ((max_parts + g - 1) / g) + slots - 1) / slots;
-                const double t = (double)waves * (double)(g * part_bytes + (160 << 10));
-                if (g == 1 || t <= best) {
-                    best = t;
-                    part_group = (int)g;
-                }
-            }
-        }
-    }
+    if (use_mma && !balanced && !fuse && prefix_parts == 0 && !force_ws && max_parts > 1)
+        part_group = (sel & 8) ? 3
+                               : plan_part_group((int64_t)S * Hkv * chunks, max_parts,
+                                                 (int64_t)partition * D * elem_size(cache_dt) * 2,
+                                                 num_sms);
     const int64_t grid_parts = fuse ? 1
                                : prefix_parts > 0 ? max_parts - prefix_parts
                                                   : (max_parts + part_group - 1) / part_group;

@@ -93,6 +93,39 @@ def test_decode_select_modes():
         pa.pa_decode_select(pa.DECODE_DEFAULT)
 
 
+def test_partition_group_plan():
+    """The grouped split-K plan (host logic, 148 SMs): the 4 x 100k bf16
+    workload with 512-token partitions streams 16 partitions per CTA (416 CTAs,
+    one wave of 3 per SM); long partitions, a single pass, the CUDA-core
+    consumer and fp32 caches stay at one; the test bit forces three."""
+    grp = pa.pa_decode_partition_group
+    try:
+        pa.pa_decode_select(pa.DECODE_DEFAULT)
+        assert grp(4, 32, 8, 128, torch.bfloat16, 100000, 512, 148) == 16
+        assert grp(4, 32, 8, 128, torch.float8_e4m3fn, 100000, 512, 148) == 16
+        assert grp(128, 32, 8, 128, torch.bfloat16, 8192, 2048, 148) == 1   # 1 MB partitions
+        assert grp(4, 32, 8, 128, torch.bfloat16, 100000, 0, 148) == 1      # single pass
+        assert grp(4, 32, 32, 128, torch.float16, 100000, 512, 148) == 1    # MHA: CUDA-core
+        assert grp(4, 32, 8, 128, torch.float32, 100000, 512, 148) == 1
+        assert grp(4, 32, 8, 128, torch.bfloat16, 400, 512, 148) == 1       # one partition
+        # never more partitions per CTA than a sequence has; no part-filled
+        # second wave when the groups would fit one
+        for S, ctx in ((1, 20000), (2, 50000), (16, 30000), (64, 9000)):
+            g = grp(S, 32, 8, 128, torch.bfloat16, ctx, 256, 148)
+            parts = -(-ctx // 256)
+            ctas = S * 8 * (-(-parts // g))
+            assert 1 <= g <= parts
+            assert not (444 < ctas < 2 * 444 and S * 8 * (-(-parts // (g + 1))) <= 444)
+        pa.pa_decode_select(pa.DECODE_DEFAULT | pa.DECODE_GROUP_PARTITIONS)
+        assert grp(4, 32, 8, 128, torch.bfloat16, 100000, 512, 148) == 3
+        pa.pa_decode_select(pa.DECODE_DEFAULT | pa.DECODE_SIMT_ONLY)
+        assert grp(4, 32, 8, 128, torch.bfloat16, 100000, 512, 148) == 1
+    finally:
+        pa.pa_decode_select(pa.DECODE_DEFAULT)
+    _bad(grp, 4, 32, 6, 128, torch.bfloat16, 1000, 512, 148)           # 32 % 6
+    _bad(grp, 4, 32, 8, 96, torch.bfloat16, 1000, 512, 148)            # head dim
+
+
 def test_copy_blocks_host_rejections():
     kc = torch.zeros((8, 16, 2, 64), dtype=torch.bfloat16)   # host memory: never launched
     for bad in ([[1, 2], [3, 2]], [[1, 2], [2, 4]], [[1, 8]], [[-1, 3]]):
