@@ -18,8 +18,10 @@ Plain Python, one step per rule on the pages:
   reference from the old block and continues in the new one.
 * "01. PagedAttention 详解" §6 and summary: sequences may share blocks (a common
   prefix, or a fork for beam search / parallel sampling) by adding references.
-* Prefix cache, "01. PagedAttention 详解" self-check 3 and summary, with the
-  content hash of "PagedAttention 机制" §6.3 and §5.1 (prefix_hashing): a
+* Prefix cache, "01. PagedAttention 详解" self-check 3 (a hash hit on a
+  block: _get_cached_block raises its ref_cnt) and summary; the
+  intelliparadigm PagedAttention article §5.1 names the same switch
+  (prefix_hashing) in its OOM table: a
   full block may be registered under a hash of its content; a hit takes a
   reference on the cached block (_get_cached_block: ref_cnt++), which also
   revives a block whose count had dropped to 0 but which still sits, content

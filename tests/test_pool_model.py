@@ -134,8 +134,8 @@ def test_copy_on_write_on_shared_last_block():
 
 
 # -- prefix cache: "01. PagedAttention 详解" self-check 3 and summary (hash hit
-#    -> ref_cnt++, LRU reuse of freed blocks); content hash as in "PagedAttention
-#    机制" §6.3 --------------------------------------------------------------
+#    -> ref_cnt++, LRU reuse of freed blocks); prefix_hashing as named in the
+#    intelliparadigm PagedAttention article §5.1 ---------------------------------
 
 def _filled_seq(p, ntok):
     s = p.seq_new()
