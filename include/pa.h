@@ -86,6 +86,14 @@ const char* pa_last_error(void);
 int pa_version(void);
 
 /*
+ * Kernels this library has enqueued since the process loaded it, over every
+ * device and stream (a launch that failed is not counted).  The difference
+ * between two reads is the number of the library's kernels a stretch of host
+ * code launched.  No citation: bookkeeping of this library, not of the method.
+ */
+uint64_t pa_launch_count(void);
+
+/*
  * Read (and with clear != 0, reset) the sticky device error bits of the
  * current device.  Synchronises `stream` first so the bits cover all work
  * enqueued on it.
@@ -212,8 +220,10 @@ pa_status pa_decode(void* out, const void* q, pa_dtype q_dt,
  * race on it: the caller must order them.  Nothing in the array needs to
  * start at zero; a call reads only partials it wrote itself.
  * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress, with that device current) and caches it; make that
- * first call before any stream capture.
+ * (cudaGetSymbolAddress, with that device current) and caches it with the
+ * device's context; make that first call before any stream capture.  After a
+ * cudaDeviceReset the device has a new context, and the next call looks the
+ * address up again (again: outside any capture).
  */
 #define PA_DECODE_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20) /* 32 MiB */
 pa_status pa_decode_noalloc(void* out, const void* q, pa_dtype q_dt,
@@ -231,9 +241,12 @@ pa_status pa_decode_noalloc(void* out, const void* q, pa_dtype q_dt,
  * device's SM count (148 without a device).  It is the planned value: the
  * launch falls back to 1 where the group's merge area would cost a resident
  * CTA per SM (fp8 tiles, 16-head groups).  *group >= 1 on success.
+ * The shape and dtype rules are pa_decode's (same return codes for a shape
+ * pa_decode would refuse); partition must be >= 0.
  */
-pa_status pa_decode_partition_group(int S, int Hq, int Hkv, int D, pa_dtype cache_dt, int max_ctx,
-                                    int partition, int num_sms, int* group);
+pa_status pa_decode_partition_group(int S, int Hq, int Hkv, int D, int bs, pa_dtype q_dt,
+                                    pa_dtype cache_dt, int max_ctx, int partition, int num_sms,
+                                    int* group);
 
 /*
  * Kernel selection and tuning for pa_decode (process-wide; for tests and
@@ -252,6 +265,10 @@ pa_status pa_decode_partition_group(int S, int Hq, int Hkv, int D, pa_dtype cach
  *      Each partition still gets its own record, so the result is the same.
  *      Tensor-core consumer only, and only where the CTA's extra merge area
  *      costs no resident CTA per SM.
+ *  16: pa_decode_shared_prefix with suffixes of at most 4096 tokens: one CTA
+ *      per (sequence, kv head) suffix, instead of the default persistent grid
+ *      in which each CTA streams a contiguous run of whole (sequence, kv head)
+ *      suffixes of about equal total length without draining its pipeline.
  * Default 4.  Every setting computes the same function.
  */
 pa_status pa_decode_select(int mode);
@@ -334,8 +351,9 @@ pa_status pa_prefill(void* out, const void* q, pa_dtype q_dt, const void* key_ca
  * empty) with the FIFO free queue of "01. PagedAttention 详解" self-check 3
  * (get_new_blocks takes from the head, free_blocks returns a block to the
  * tail when its count reaches 0), per-sequence block tables ("PagedAttention
- * 机制" §5.3.2), sharing by reference counts (same page §6: prefix sharing,
- * beam search and parallel sampling) and copy-on-write (intelliparadigm
+ * 机制" §5.3.2), sharing by reference counts ("01. PagedAttention 详解" §6
+ * and its summary: prefix sharing, beam search and parallel sampling) and
+ * copy-on-write (intelliparadigm
  * PagedAttention article §3.3).
  *
  * Not thread-safe: one scheduler thread owns a pool.  No device access.

@@ -19,7 +19,7 @@ from typing import Optional, Sequence
 import torch
 
 __all__ = [
-    "PaError", "lib", "pa_version", "pa_last_error", "pa_device_status",
+    "PaError", "lib", "pa_version", "pa_launch_count", "pa_last_error", "pa_device_status",
     "pa_reshape_and_cache", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_size",
     "pa_decode_suggest_partition", "pa_decode_partition_group", "pa_decode_select", "pa_decode_noalloc", "pa_prefill",
     "pa_decode_shared_prefix", "pa_decode_shared_prefix_workspace_size",
@@ -71,12 +71,13 @@ def lib() -> ctypes.CDLL:
     sig = {
         "pa_last_error": ([], ctypes.c_char_p),
         "pa_version": ([], I),
+        "pa_launch_count": ([], ctypes.c_uint64),
         "pa_device_status": ([ctypes.POINTER(ctypes.c_uint), I, P], I),
         "pa_reshape_and_cache": ([P, P, I, P, P, I, P, I, I, I, I, I64, F, F, P], I),
         "pa_copy_blocks": ([P, P, SZ, I64, P, I, P], I),
         "pa_decode_workspace_size": ([I, I, I, I, I, ctypes.POINTER(SZ)], I),
         "pa_decode_suggest_partition": ([I, I, I, P, ctypes.POINTER(I)], I),
-        "pa_decode_partition_group": ([I, I, I, I, I, I, I, I, ctypes.POINTER(I)], I),
+        "pa_decode_partition_group": ([I, I, I, I, I, I, I, I, I, I, ctypes.POINTER(I)], I),
         "pa_decode_select": ([I], I),
         "pa_decode": ([P, P, I, P, P, I, P, I, P, I, I, I, I, I, I64, I, F, F, F, I, P, SZ, P], I),
         "pa_decode_noalloc": ([P, P, I, P, P, I, P, I, P, I, I, I, I, I, I64, I, F, F, F, I, P], I),
@@ -125,6 +126,11 @@ def _check(st: int) -> None:
 
 def pa_version() -> int:
     return lib().pa_version()
+
+
+def pa_launch_count() -> int:
+    """Kernels the library has enqueued in this process (all devices, streams)."""
+    return int(lib().pa_launch_count())
 
 
 def _stream(stream) -> ctypes.c_void_p:
@@ -201,26 +207,32 @@ def pa_decode_suggest_partition(Hkv: int, block_size: int, context_lens_host) ->
     return out.value
 
 
-def pa_decode_partition_group(S: int, Hq: int, Hkv: int, D: int, cache_dtype, max_ctx: int,
-                              partition: int, num_sms: int = 0) -> int:
+def pa_decode_partition_group(S: int, Hq: int, Hkv: int, D: int, block_size: int, q_dtype,
+                              cache_dtype, max_ctx: int, partition: int, num_sms: int = 0) -> int:
     """Consecutive split-K partitions one pa_decode CTA streams for this shape
     (planned; each partition keeps its own record)."""
-    dt = _TORCH_DT[cache_dtype] if isinstance(cache_dtype, torch.dtype) else int(cache_dtype)
+    def code(t):
+        return _TORCH_DT[t] if isinstance(t, torch.dtype) else int(t)
     out = ctypes.c_int(0)
-    _check(lib().pa_decode_partition_group(S, Hq, Hkv, D, dt, max_ctx, partition, num_sms,
+    _check(lib().pa_decode_partition_group(S, Hq, Hkv, D, block_size, code(q_dtype),
+                                           code(cache_dtype), max_ctx, partition, num_sms,
                                            ctypes.byref(out)))
     return out.value
 
 
 DECODE_SIMT_ONLY, DECODE_EVICT_FIRST, DECODE_PARTITION_MAJOR = 1, 2, 4
 DECODE_GROUP_PARTITIONS = 8
+DECODE_SUFFIX_PER_CTA = 16
 DECODE_DEFAULT = DECODE_PARTITION_MAJOR
+PA_PARTITION_BALANCED = -1                        # include/pa.h: the persistent balanced grid
+PA_DECODE_NOALLOC_SCRATCH_BYTES = 32 << 20        # include/pa.h: pa_decode_noalloc's array
 
 
 def pa_decode_select(mode: int) -> None:
     """Bit mask: 1 CUDA-core consumer everywhere, 2 L2 evict-first K/V loads,
     4 partition-major grid, 8 split-K partitions grouped three to a CTA whenever
-    there are several (default 4)."""
+    there are several, 16 shared-prefix decode with one CTA per (sequence, kv
+    head) suffix instead of the persistent whole-item grid (default 4)."""
     _check(lib().pa_decode_select(int(mode)))
 
 

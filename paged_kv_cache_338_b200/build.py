@@ -4,6 +4,11 @@ Each translation unit under csrc/ is compiled in parallel into _build/, then
 linked into paged_kv_cache_338_b200/libpa_b200.so with the CUDA runtime linked
 statically and its symbols kept private (so the library's runtime never
 resolves against another copy loaded in the same process).
+
+``--nvtx`` compiles in an NVTX range around every C-ABI call that enqueues
+work (for an Nsight Systems timeline; off by default).  The defines of the
+last build are kept in _build/defines.txt; a build with other defines
+recompiles everything.
 """
 from __future__ import annotations
 
@@ -42,13 +47,13 @@ def _headers_mtime() -> float:
     return max(os.path.getmtime(h) for h in hs)
 
 
-def _compile(src: str, verbose_ptxas: bool) -> str:
+def _compile(src: str, verbose_ptxas: bool, defines: list) -> str:
     obj = os.path.join(BUILD, src + ".o")
     path = os.path.join(CSRC, src)
     if (os.path.exists(obj) and os.path.getmtime(obj) >= os.path.getmtime(path)
             and os.path.getmtime(obj) >= _headers_mtime() and not verbose_ptxas):
         return obj
-    cmd = [nvcc()] + NVCC_FLAGS + ["-c", path, "-o", obj + ".tmp"]
+    cmd = [nvcc()] + NVCC_FLAGS + [f"-D{d}" for d in defines] + ["-c", path, "-o", obj + ".tmp"]
     if verbose_ptxas:
         cmd += ["-Xptxas", "-v"]
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -60,9 +65,15 @@ def _compile(src: str, verbose_ptxas: bool) -> str:
     return obj
 
 
-def build(force: bool = False, verbose_ptxas: bool = False, jobs: int | None = None) -> str:
+def build(force: bool = False, verbose_ptxas: bool = False, jobs: int | None = None,
+          nvtx: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
     srcs = sources()
+    defines = ["PA_WITH_NVTX"] if nvtx else []
+    stamp = os.path.join(BUILD, "defines.txt")
+    old = open(stamp).read() if os.path.exists(stamp) else ""
+    if old != " ".join(defines):
+        force = True
     if force:
         for s in srcs:
             o = os.path.join(BUILD, s + ".o")
@@ -70,7 +81,9 @@ def build(force: bool = False, verbose_ptxas: bool = False, jobs: int | None = N
                 os.remove(o)
     jobs = jobs or min(len(srcs), os.cpu_count() or 4)
     with cf.ThreadPoolExecutor(jobs) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose_ptxas), srcs))
+        objs = list(ex.map(lambda s: _compile(s, verbose_ptxas, defines), srcs))
+    with open(stamp, "w") as f:
+        f.write(" ".join(defines))
     if os.path.exists(LIB) and all(os.path.getmtime(LIB) >= os.path.getmtime(o) for o in objs):
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"
@@ -84,4 +97,5 @@ def build(force: bool = False, verbose_ptxas: bool = False, jobs: int | None = N
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose_ptxas="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose_ptxas="-v" in sys.argv,
+                nvtx="--nvtx" in sys.argv))

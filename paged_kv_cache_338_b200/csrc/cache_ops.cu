@@ -3,6 +3,7 @@
 // copy-on-write block copy.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -31,25 +32,54 @@ pa_status fail(pa_status st, const char* fmt, ...) {
 
 void clear_error() { t_error.clear(); }
 
+static std::atomic<unsigned long long> g_launches{0};
+
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
 pa_status cuda_fail(int err, const char* what) {
     return fail(PA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(static_cast<cudaError_t>(err)));
 }
 
-unsigned int* device_error_word() {
-    static std::mutex mu;
-    static unsigned int* addr[256] = {};
+// The calling thread's current CUDA context (nullptr before the runtime has
+// made one current), through the driver entry point the runtime exposes.
+static const void* current_context() {
+    using Fn = CUresult (*)(CUcontext*);
+    static Fn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 4000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<Fn>(p);
+    });
+    CUcontext c = nullptr;
+    if (fn && fn(&c) != CUDA_SUCCESS) c = nullptr;
+    return c;
+}
+
+void* symbol_address(const void* symbol, SymbolCache* cache, const char* what) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) { cuda_fail(e, "cudaGetDevice"); return nullptr; }
     if (dev < 0 || dev >= 256) { fail(PA_ERR_CUDA, "device ordinal %d", dev); return nullptr; }
-    std::lock_guard<std::mutex> lk(mu);
-    if (!addr[dev]) {
+    std::lock_guard<std::mutex> lk(cache->mu);
+    const void* ctx = current_context();
+    if (!cache->addr[dev] || !ctx || cache->ctx[dev] != ctx) {
         void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_pa_device_error);
-        if (e != cudaSuccess) { cuda_fail(e, "cudaGetSymbolAddress"); return nullptr; }
-        addr[dev] = static_cast<unsigned int*>(p);
+        e = cudaGetSymbolAddress(&p, symbol);    // makes the device's context current
+        if (e != cudaSuccess) { cuda_fail(e, what); return nullptr; }
+        cache->addr[dev] = p;
+        cache->ctx[dev] = current_context();
     }
-    return addr[dev];
+    return cache->addr[dev];
+}
+
+unsigned int* device_error_word() {
+    static SymbolCache cache;
+    return static_cast<unsigned int*>(
+        symbol_address(&g_pa_device_error, &cache, "cudaGetSymbolAddress(error word)"));
 }
 
 namespace {
@@ -166,7 +196,10 @@ extern "C" const char* pa_last_error(void) { return t_error.c_str(); }
 
 extern "C" int pa_version(void) { return 10000; }
 
+extern "C" uint64_t pa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
 extern "C" pa_status pa_device_status(unsigned int* bits, int clear, pa_stream_t stream) {
+    PA_NVTX_RANGE("pa_device_status");
     clear_error();
     if (!bits) return fail(PA_ERR_INVALID_ARG, "bits is NULL");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -192,6 +225,7 @@ extern "C" pa_status pa_reshape_and_cache(const void* key, const void* value, pa
                                           const int64_t* slot_mapping, int T, int Hkv, int D,
                                           int bs, int64_t NB, float k_scale, float v_scale,
                                           pa_stream_t stream) {
+    PA_NVTX_RANGE("pa_reshape_and_cache");
     clear_error();
     if (!valid_dtype(in_dt) || !valid_dtype(cache_dt)) return fail(PA_ERR_INVALID_ARG, "bad dtype");
     if (T < 0 || Hkv <= 0 || D <= 0 || bs <= 0 || NB <= 0)
@@ -246,6 +280,7 @@ extern "C" pa_status pa_reshape_and_cache(const void* key, const void* value, pa
 
 extern "C" pa_status pa_copy_blocks(void* key_cache, void* value_cache, size_t block_bytes,
                                     int64_t NB, const int32_t* pairs, int n, pa_stream_t stream) {
+    PA_NVTX_RANGE("pa_copy_blocks");
     clear_error();
     if (n < 0 || NB <= 0 || block_bytes == 0 || block_bytes % 16)
         return fail(PA_ERR_INVALID_ARG, "bad sizes (block_bytes must be a positive multiple of 16)");

@@ -27,22 +27,12 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 // Device address of the scratch array for the current device.  In host code
 // the array's name is only a host-side stand-in, so the address is looked up
-// once per device (with that device current) and cached.
+// with that device current, and cached per device and context (a
+// cudaDeviceReset gives the device a new context, and the next call looks the
+// address up again).
 void* scratch_address() {
-    static std::mutex mu;
-    static void* addr[256] = {};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) { pa::cuda_fail(e, "cudaGetDevice"); return nullptr; }
-    if (dev < 0 || dev >= 256) { pa::fail(PA_ERR_CUDA, "device ordinal %d", dev); return nullptr; }
-    std::lock_guard<std::mutex> lk(mu);
-    if (!addr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) { pa::cuda_fail(e, "cudaGetSymbolAddress(scratch)"); return nullptr; }
-        addr[dev] = p;
-    }
-    return addr[dev];
+    static pa::SymbolCache cache;
+    return pa::symbol_address(g_noalloc_scratch, &cache, "cudaGetSymbolAddress(scratch)");
 }
 
 }  // namespace
@@ -54,6 +44,7 @@ extern "C" pa_status pa_decode_noalloc(void* out, const void* q, pa_dtype q_dt,
                                        int bs, int64_t NB, int max_ctx, float scale,
                                        float k_scale, float v_scale, int partition,
                                        pa_stream_t stream) {
+    PA_NVTX_RANGE("pa_decode_noalloc");
     pa::clear_error();
     size_t need = 0;
     pa_status st = pa_decode_workspace_size(S, Hq, D, max_ctx, partition, &need);

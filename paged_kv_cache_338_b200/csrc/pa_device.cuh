@@ -14,6 +14,10 @@
 #include "pa.h"
 
 namespace pa {
+
+// Count one kernel enqueued by this library (pa_launch_count()).
+void note_launch();
+
 namespace dev {
 
 // ------------------------------------------------------------ storage types
@@ -200,7 +204,9 @@ inline cudaError_t launch_pdl(void (*kern)(Params...), dim3 grid, dim3 block, si
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+    if (e == cudaSuccess) note_launch();
+    return e;
 }
 
 // 5-D tiled tensor-map load into shared memory, completing on `bar`.

@@ -4,11 +4,31 @@
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
+#include <mutex>
 #include <string>
 
 #include <vector_types.h>
 
 #include "pa.h"
+
+// Profiler ranges around the C-ABI entry points (a named NVTX range per call,
+// seen on an Nsight Systems timeline).  Compiled in only when the library is
+// built with PA_WITH_NVTX (python -m paged_kv_cache_338_b200.build --nvtx);
+// otherwise the macro is empty and costs nothing.
+#ifdef PA_WITH_NVTX
+#include <nvtx3/nvToolsExt.h>
+namespace pa {
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
+}  // namespace pa
+#define PA_NVTX_RANGE(name) ::pa::NvtxRange pa_nvtx_range_(name)
+#else
+#define PA_NVTX_RANGE(name) ((void)0)
+#endif
 
 namespace pa {
 
@@ -32,6 +52,19 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // Device address of the sticky error word of the current device (nullptr and
 // a recorded error if the runtime call fails).
 unsigned int* device_error_word();
+
+// Per-device cache of a __device__ symbol's address.  An entry is keyed on
+// the device's current context as well, so it is looked up again after a
+// cudaDeviceReset (the next context may load the module elsewhere).
+struct SymbolCache {
+    std::mutex mu;
+    const void* ctx[256] = {};
+    void* addr[256] = {};
+};
+
+// Address of `symbol` on the current device (nullptr and a recorded error if
+// a runtime call fails).
+void* symbol_address(const void* symbol, SymbolCache* cache, const char* what);
 
 // Translate a CUDA runtime error into PA_ERR_CUDA with context.
 pa_status cuda_fail(int err, const char* what);

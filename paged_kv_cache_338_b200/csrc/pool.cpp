@@ -408,6 +408,7 @@ extern "C" pa_status pa_pool_seq_match_prefix(pa_pool* pool, int64_t seq, const 
 extern "C" pa_status pa_pool_step(pa_pool* pool, const int64_t* seqs, int n, int MB, int64_t* slots,
                                   int32_t* cow_pairs, int* n_cow, int32_t* tables_host,
                                   int32_t* ctx_lens_host) {
+    PA_NVTX_RANGE("pa_pool_step");
     pa::clear_error();
     if (!pool || n < 0 || MB < 0 || !n_cow ||
         (n > 0 && (!seqs || !slots || !cow_pairs || !ctx_lens_host || (MB > 0 && !tables_host))))

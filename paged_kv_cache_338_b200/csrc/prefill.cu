@@ -725,7 +725,9 @@ cudaError_t launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorM
         prefill_kernel<DT, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Smem<D>::BYTES);
     if (attr != cudaSuccess) return attr;
     prefill_kernel<DT, D><<<grid, kThreads, Smem<D>::BYTES, st>>>(mq, mk, mv, p);
-    return cudaGetLastError();
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) pa::note_launch();
+    return e;
 }
 
 }  // namespace pf
@@ -798,6 +800,7 @@ extern "C" pa_status pa_prefill(void* out, const void* q, pa_dtype q_dt, const v
                                 const int32_t* query_start, int S, int T, int Hq, int Hkv, int D,
                                 int bs, int64_t NB, int max_query_len, float scale,
                                 pa_stream_t stream) {
+    PA_NVTX_RANGE("pa_prefill");
     pa::clear_error();
     if (!pa::valid_dtype(q_dt) || !pa::valid_dtype(cache_dt))
         return fail(PA_ERR_INVALID_ARG, "unknown dtype");

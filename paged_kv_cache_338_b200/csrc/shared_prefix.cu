@@ -126,6 +126,7 @@ extern "C" pa_status pa_decode_shared_prefix(void* out, const void* q, pa_dtype 
                                              float scale, float k_scale, float v_scale,
                                              int prefix_tokens, void* workspace,
                                              size_t workspace_bytes, pa_stream_t stream) {
+    PA_NVTX_RANGE("pa_decode_shared_prefix");
     pa::clear_error();
     if (!pa::valid_dtype(q_dt) || !pa::valid_dtype(cache_dt))
         return fail(PA_ERR_INVALID_ARG, "bad dtype");
@@ -194,6 +195,7 @@ extern "C" pa_status pa_decode_shared_prefix(void* out, const void* q, pa_dtype 
                 block_tables, NB, blk_elems, sk, sv, err);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return pa::cuda_fail(e, "prefix conversion launch");
+        pa::note_launch();
         k_src = sk;
         v_src = sv;
         src_blocks = nblk;

@@ -34,6 +34,15 @@ def test_library_exports_every_declared_symbol():
     assert pa.pa_version() == 10000
 
 
+def test_binding_constants_match_the_header():
+    """The few #defines the binding mirrors have the header's values."""
+    src = open(os.path.join(ROOT, "include", "pa.h")).read()
+    assert re.search(r"#define PA_PARTITION_BALANCED \(-1\)", src)
+    assert pa.PA_PARTITION_BALANCED == -1
+    m = re.search(r"#define PA_DECODE_NOALLOC_SCRATCH_BYTES \(\(size_t\)(\d+) << (\d+)\)", src)
+    assert m and pa.PA_DECODE_NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))
+
+
 def test_no_symbol_leaks_beyond_the_abi():
     # the static CUDA runtime stays private to the library
     out = os.popen(f"nm -D --defined-only {pa.LIB_PATH}").read().split("\n")
@@ -82,12 +91,12 @@ def test_host_argument_checks():
 
 
 def test_decode_select_modes():
-    """Every documented bit combination is accepted (0..15, bit 8 included)
-    and anything else refused; the default is restored afterwards."""
+    """Every documented bit combination is accepted (0..31, bits 8 and 16
+    included) and anything else refused; the default is restored afterwards."""
     try:
-        for mode in range(16):
+        for mode in range(32):
             pa.pa_decode_select(mode)
-        for bad in (-1, 16, 64):
+        for bad in (-1, 32, 64):
             _bad(pa.pa_decode_select, bad)
     finally:
         pa.pa_decode_select(pa.DECODE_DEFAULT)
@@ -97,33 +106,55 @@ def test_partition_group_plan():
     """The grouped split-K plan (host logic, 148 SMs): the 4 x 100k bf16
     workload with 512-token partitions streams 16 partitions per CTA (416 CTAs,
     one wave of 3 per SM); long partitions, a single pass, the CUDA-core
-    consumer and fp32 caches stay at one; the test bit forces three."""
-    grp = pa.pa_decode_partition_group
+    consumer and fp32 caches stay at one; the test bit forces three.  Shapes
+    pa_decode refuses are refused here with the same codes."""
+    bf, f8, f16, f32 = torch.bfloat16, torch.float8_e4m3fn, torch.float16, torch.float32
+
+    def grp(S, Hq, Hkv, D, ct, ctx, part, sms, bs=16, qt=None):
+        qt = qt if qt is not None else (bf if ct == f8 else ct)
+        return pa.pa_decode_partition_group(S, Hq, Hkv, D, bs, qt, ct, ctx, part, sms)
     try:
         pa.pa_decode_select(pa.DECODE_DEFAULT)
-        assert grp(4, 32, 8, 128, torch.bfloat16, 100000, 512, 148) == 16
-        assert grp(4, 32, 8, 128, torch.float8_e4m3fn, 100000, 512, 148) == 16
-        assert grp(128, 32, 8, 128, torch.bfloat16, 8192, 2048, 148) == 1   # 1 MB partitions
-        assert grp(4, 32, 8, 128, torch.bfloat16, 100000, 0, 148) == 1      # single pass
-        assert grp(4, 32, 32, 128, torch.float16, 100000, 512, 148) == 1    # MHA: CUDA-core
-        assert grp(4, 32, 8, 128, torch.float32, 100000, 512, 148) == 1
-        assert grp(4, 32, 8, 128, torch.bfloat16, 400, 512, 148) == 1       # one partition
+        assert grp(4, 32, 8, 128, bf, 100000, 512, 148) == 16
+        assert grp(4, 32, 8, 128, f8, 100000, 512, 148) == 16
+        assert grp(128, 32, 8, 128, bf, 8192, 2048, 148) == 1   # 1 MB partitions
+        assert grp(4, 32, 8, 128, bf, 100000, 0, 148) == 1      # single pass
+        assert grp(4, 32, 32, 128, f16, 100000, 512, 148) == 1  # MHA: CUDA-core
+        assert grp(4, 32, 8, 128, f32, 100000, 512, 148) == 1
+        assert grp(4, 32, 8, 128, bf, 400, 512, 148) == 1       # one partition
         # never more partitions per CTA than a sequence has; no part-filled
         # second wave when the groups would fit one
         for S, ctx in ((1, 20000), (2, 50000), (16, 30000), (64, 9000)):
-            g = grp(S, 32, 8, 128, torch.bfloat16, ctx, 256, 148)
+            g = grp(S, 32, 8, 128, bf, ctx, 256, 148)
             parts = -(-ctx // 256)
             ctas = S * 8 * (-(-parts // g))
             assert 1 <= g <= parts
             assert not (444 < ctas < 2 * 444 and S * 8 * (-(-parts // (g + 1))) <= 444)
         pa.pa_decode_select(pa.DECODE_DEFAULT | pa.DECODE_GROUP_PARTITIONS)
-        assert grp(4, 32, 8, 128, torch.bfloat16, 100000, 512, 148) == 3
+        assert grp(4, 32, 8, 128, bf, 100000, 512, 148) == 3
         pa.pa_decode_select(pa.DECODE_DEFAULT | pa.DECODE_SIMT_ONLY)
-        assert grp(4, 32, 8, 128, torch.bfloat16, 100000, 512, 148) == 1
+        assert grp(4, 32, 8, 128, bf, 100000, 512, 148) == 1
     finally:
         pa.pa_decode_select(pa.DECODE_DEFAULT)
-    _bad(grp, 4, 32, 6, 128, torch.bfloat16, 1000, 512, 148)           # 32 % 6
-    _bad(grp, 4, 32, 8, 96, torch.bfloat16, 1000, 512, 148)            # head dim
+    G = pa.pa_decode_partition_group
+    # 32 % 6
+    _bad(G, 4, 32, 6, 128, 16, bf, bf, 1000, 512, 148)
+    # head dim
+    _bad(G, 4, 32, 8, 96, 16, bf, bf, 1000, 512, 148, status="PA_ERR_UNSUPPORTED")
+    # group of 3
+    _bad(G, 4, 24, 8, 128, 16, bf, bf, 1000, 512, 148, status="PA_ERR_UNSUPPORTED")
+    # partition % bs
+    _bad(G, 4, 32, 8, 128, 16, bf, bf, 1000, 500, 148)
+    # block size
+    _bad(G, 4, 32, 8, 128, 12, bf, bf, 1000, 480, 148, status="PA_ERR_UNSUPPORTED")
+    # q f16, cache bf16
+    _bad(G, 4, 32, 8, 128, 16, f16, bf, 1000, 512, 148, status="PA_ERR_UNSUPPORTED")
+    # fp8 queries
+    _bad(G, 4, 32, 8, 128, 16, f8, f8, 1000, 512, 148, status="PA_ERR_UNSUPPORTED")
+    # fp32 q, fp8 cache
+    _bad(G, 4, 32, 8, 128, 16, f32, f8, 1000, 512, 148, status="PA_ERR_UNSUPPORTED")
+    # balanced: no plan
+    _bad(G, 4, 32, 8, 128, 16, bf, bf, 1000, -1, 148)
 
 
 def test_copy_blocks_host_rejections():
