@@ -69,6 +69,9 @@ LOG_DIR = os.environ.get("PA_BENCH_LOG_DIR", os.path.join(ROOT, "bench_logs"))
 import workloads as wl  # noqa: E402
 
 METRIC = "paged decode KV-read GB/s (% of B200 HBM peak) and decode seqs/s"
+# the other multi-sequence decode workloads the default run also times (device only)
+EXTRA_WORKLOADS = ("llama2_7b_mha_fp16_b64", "long_context_splitk_bf16_4x100k",
+                   "prefix_shared_fp8_b256")
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -118,7 +121,8 @@ def algorithmic_bytes(cfg: wl.DecodeConfig, lens: torch.Tensor) -> dict:
     append = S * Hkv * D * 2 * (e_q + e_kv) + S * 8
     # with a shared prefix every sequence reads the same prefix blocks: count them once
     unique_kv = kv - max(S - 1, 0) * cfg.prefix_tokens * Hkv * D * 2 * e_kv
-    return {"decode": decode, "append": append, "kv": kv, "unique_kv": unique_kv}
+    return {"decode": decode, "append": append, "kv": kv, "unique_kv": unique_kv,
+            "decode_unique": unique_kv + qo + tables}
 
 
 def _pci_id(dev: int) -> str | None:
@@ -306,14 +310,47 @@ def _config_dict(cfg, args, partition=None, l2_note=None):
 
 # --------------------------------------------------------------------- GPU arm
 
-def run_gpu(args, cfg, rank, world, local_rank):
-    import paged_kv_cache_338_b200 as pa
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
+def _traffic(cfg, part, shared):
+    """DRAM read + write bytes of one attention call from the committed ncu
+    capture of the same workload and path (profiles/traffic_<workload>[_shared_prefix].json),
+    or None when there is none, it was taken for another partition, or the
+    kernel sources changed since (the file records their hash)."""
+    name = f"traffic_{cfg.name}{'_shared_prefix' if shared else ''}.json"
+    prof = os.path.join(ROOT, "profiles", name)
+    if not os.path.exists(prof):
+        return None
+    try:
+        with open(prof) as f:
+            pj = json.load(f)
+    except Exception:
+        return None
+    if not shared and pj.get("partition") != part:
+        return None
+    sha = pj.get("csrc_sha256")
+    if sha is not None and sha != csrc_sha256():
+        return None
+    return pj.get("dram_bytes_per_launch")
+
+
+def csrc_sha256() -> str:
+    """Hash of the library's kernel sources (every file under csrc/)."""
+    import hashlib
+    d = os.path.join(ROOT, "paged_kv_cache_338_b200", "csrc")
+    h = hashlib.sha256()
+    for fn in sorted(os.listdir(d)):
+        with open(os.path.join(d, fn), "rb") as f:
+            h.update(fn.encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
+def device_leg(args, cfg, pa, dev, seed, steps, warmup, partition=-1):
+    """Append [+ copy-on-write] + decode on device-resident inputs: W untimed
+    steps, then K steps timed with CUDA events on the launching stream, clocks
+    sampled inside the timed region."""
     stream = torch.cuda.current_stream()
-    inp = wl.make_decode_inputs(cfg, seed=args.seed + rank, device=dev)
+    inp = wl.make_decode_inputs(cfg, seed=seed, device=dev)
     S, Hq, D = inp.q.shape
-    part = args.partition if args.partition >= 0 else (
+    part = partition if partition >= 0 else (
         cfg.partition or pa.pa_decode_suggest_partition(cfg.num_kv_heads, cfg.block_size,
                                                         inp.context_lens.cpu()))
     max_ctx = inp.max_ctx
@@ -330,7 +367,6 @@ def run_gpu(args, cfg, rank, world, local_rank):
     kc, vc = inp.key_cache, inp.value_cache
     pairs = inp.copy_pairs
     nbytes = algorithmic_bytes(cfg, inp.context_lens.cpu())
-    step_bytes = nbytes["decode"] + nbytes["append"]
 
     def decode(out_t, q_t, tables, lens):
         if shared:
@@ -354,44 +390,74 @@ def run_gpu(args, cfg, rank, world, local_rank):
         if ev is not None:
             ev[1].record(stream)
 
-    # copy-on-write, append, then the decode's kernels: partitions [+ merge];
-    # shared prefix: [fp8 conversion +] prefix records + partitions [+ merge
-    # when a suffix can exceed 4096 tokens]
-    if shared:
-        dec_launches = (1 if cfg.kv_dtype == "fp8_e4m3" else 0) + 1 + 1 + (
-            1 if max_ctx - cfg.prefix_tokens > 4096 else 0)
-    else:
-        dec_launches = 1 + (1 if ws_bytes else 0)
-    launches_per_step = (1 if pairs.numel() else 0) + 1 + dec_launches
-    for _ in range(args.warmup):
+    # copy-on-write, append, then the decode's kernels (counted by the library)
+    for _ in range(warmup):
         step()
     torch.cuda.synchronize()
     assert pa.pa_device_status() == 0
+    n0 = pa.pa_launch_count()
+    step()
+    torch.cuda.synchronize()
+    launches_per_step = pa.pa_launch_count() - n0
 
-    dist = world > 1
+    dist = torch.distributed.is_available() and torch.distributed.is_initialized()
     if dist:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    clocks = ClockSampler(local_rank)
-    evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3))
-           for _ in range(args.steps)]
+    clocks = ClockSampler(dev.index or 0)
+    evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks.mark_start()
     t0.record(stream)
-    for i in range(args.steps):
+    for i in range(steps):
         step(evs[i])
     t1.record(stream)
     torch.cuda.synchronize()
     clocks.mark_end()
     clk = clocks.stop()
+    assert pa.pa_device_status() == 0
     if dist:
         torch.distributed.barrier()
-    ms = t0.elapsed_time(t1)
     dec_ms = [a.elapsed_time(b) for a, b, _ in evs]
-    dec_avg = sum(dec_ms) / len(dec_ms)
-    app_avg = sum(c.elapsed_time(a) for a, _, c in evs) / len(evs)
-    value = whole_job_rate(step_bytes * args.steps, ms, dev) / 1e9
-    ms = max_over_ranks(ms, dev)
+    res = {"ms": t0.elapsed_time(t1), "dec_avg": sum(dec_ms) / len(dec_ms),
+           "app_avg": sum(c.elapsed_time(a) for a, _, c in evs) / len(evs),
+           "nbytes": nbytes, "part": part, "shared": shared, "S": S,
+           "launches_per_step": launches_per_step, "clocks": clk,
+           "kv_gb": nbytes["kv"] / 1e9}
+    del inp, ws, out, kc, vc
+    torch.cuda.empty_cache()
+    return res
+
+
+def roofline_of(cfg, r, peak, peak_kind):
+    """The attention call against the HBM roofline.  With a shared prefix the
+    algorithmic bytes count the prefix once (it is the same physical blocks for
+    every sequence); logical bytes, which count it per sequence, are reported
+    beside it and are no HBM fraction."""
+    nb, t = r["nbytes"], r["dec_avg"] * 1e-3
+    alg = nb["decode_unique"] if r["shared"] else nb["decode"]
+    achieved = alg / t / 1e9
+    d = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+         "frac": round(achieved / peak, 4), "traffic": _traffic(cfg, r["part"], r["shared"]),
+         "peak_kind": peak_kind, "algorithmic_bytes": alg,
+         "kernel": "pa_decode_shared_prefix (prefix records + suffix decode)"
+         if r["shared"] else "pa_decode (partition + merge)"}
+    if r["shared"]:
+        d["logical_gbs_not_hbm"] = round(nb["decode"] / t / 1e9, 1)
+    return d
+
+
+def run_gpu(args, cfg, rank, world, local_rank):
+    import paged_kv_cache_338_b200 as pa
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    if args.decode_select is not None:
+        pa.pa_decode_select(args.decode_select)
+    r = device_leg(args, cfg, pa, dev, args.seed + rank, args.steps, args.warmup, args.partition)
+    S, part, nbytes = r["S"], r["part"], r["nbytes"]
+    step_bytes = nbytes["decode"] + nbytes["append"]
+    value = whole_job_rate(step_bytes * args.steps, r["ms"], dev) / 1e9
+    ms = max_over_ranks(r["ms"], dev)
     ms_step = ms / args.steps
     seqs_all = sum_over_ranks(S, dev)
 
@@ -400,52 +466,64 @@ def run_gpu(args, cfg, rank, world, local_rank):
     if e2e is not None:
         e2e["value"] = whole_job_rate(e2e["bytes"], e2e["ms"], dev) / 1e9
 
+    # ---- the other multi-sequence decode workloads, device-timed only ------
+    extras = {}
+    if args.workloads_also:
+        for name in args.workloads_also.split(","):
+            wcfg = wl.DECODE_WORKLOADS[name]
+            x = device_leg(args, wcfg, pa, dev, args.seed + rank, args.steps, args.warmup)
+            xv = whole_job_rate((x["nbytes"]["decode"] + x["nbytes"]["append"]) * args.steps,
+                                x["ms"], dev) / 1e9
+            extras[name] = (wcfg, x, xv, max_over_ranks(x["ms"], dev) / args.steps)
+
     if rank != 0:
         return
     peak, peak_kind = _peaks()
-    achieved = nbytes["decode"] / (dec_avg * 1e-3) / 1e9
-    traffic = None
-    prof = os.path.join(ROOT, "profiles", f"traffic_{cfg.name}.json")
-    if os.path.exists(prof) and not shared:       # the capture is of the plain decode
-        try:
-            with open(prof) as f:
-                pj = json.load(f)
-            if pj.get("partition") == part:
-                traffic = pj.get("dram_bytes_per_launch")
-        except Exception:
-            traffic = None
+    roof = roofline_of(cfg, r, peak, peak_kind)
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        r = cpu_oracle_rate(cfg, args.seed, budget_s=args.cpu_budget)
-        cpu = {"value": round(r["gbs"], 4), "unit": "GB/s", "cores": r["cores"],
-               "kind": "oracle", "sample": r["sample"], "seqs_per_s": round(r["seqs_per_s"], 3)}
-    kv_gb = nbytes["kv"] / 1e9
+        c = cpu_oracle_rate(cfg, args.seed, budget_s=args.cpu_budget)
+        cpu = {"value": round(c["gbs"], 4), "unit": "GB/s", "cores": c["cores"],
+               "kind": "oracle", "sample": c["sample"], "seqs_per_s": round(c["seqs_per_s"], 3)}
+    workloads = {}
+    for name, (wcfg, x, xv, xms) in extras.items():
+        workloads[name] = {
+            "value": round(xv, 2), "unit": "GB/s", "ms_per_step": round(xms, 4),
+            "decode_ms": round(x["dec_avg"], 4), "append_cow_ms": round(x["app_avg"], 4),
+            "seqs_per_s": round(x["S"] * world / (xms * 1e-3), 1), "partition": x["part"],
+            "path": "pa_decode_shared_prefix" if x["shared"] else "pa_decode",
+            "unique_kv_gbs": round(x["nbytes"]["unique_kv"] / (x["dec_avg"] * 1e-3) / 1e9, 1),
+            "roofline": roofline_of(wcfg, x, peak, peak_kind),
+            "gpu_launches": x["launches_per_step"] * args.steps,
+            "clocks": x["clocks"],
+            "config": _config_dict(wcfg, args, x["part"]),
+        }
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.kv_dtype,
         "data": "synthetic",
         "config": _config_dict(cfg, args, part,
-                               f"inputs larger than L2 ({kv_gb:.2f} GB of K/V per step), no flush"),
+                               f"inputs larger than L2 ({r['kv_gb']:.2f} GB of K/V per step), "
+                               "no flush" if r["kv_gb"] > 0.126 else
+                               f"K/V ({r['kv_gb']:.3f} GB per step) may stay in L2"),
         "seqs_per_s": round(seqs_all / (ms_step * 1e-3), 1),
         "pct_of_hbm_peak": {"measured_copy": round(100 * value / world / peak, 2),
                             "spec_8000": round(100 * value / world / 8000.0, 2)},
-        "decode_ms": round(dec_avg, 4),
-        "append_cow_ms": round(app_avg, 4),
-        "unique_kv_gbs": round(nbytes["unique_kv"] / (dec_avg * 1e-3) / 1e9, 1),
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
-                     "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "peak_kind": peak_kind,
-                     "kernel": "pa_decode_shared_prefix (prefix records + partitions + merge)"
-                     if shared else "pa_decode (partition + merge)"},
+        "decode_ms": round(r["dec_avg"], 4),
+        "append_cow_ms": round(r["app_avg"], 4),
+        "unique_kv_gbs": round(nbytes["unique_kv"] / (r["dec_avg"] * 1e-3) / 1e9, 1),
+        "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": None if e2e is None else {
             "value": round(e2e["value"], 2), "unit": "GB/s",
             "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
             "ms_per_step": round(e2e["ms"], 4)},
-        "gpu_launches": launches_per_step * args.steps,
-        "clocks": clk,
+        "gpu_launches": r["launches_per_step"] * args.steps,
+        "clocks": r["clocks"],
     }
+    if workloads:
+        line["workloads"] = workloads
     print(json.dumps(line), flush=True)
 
 
@@ -854,6 +932,14 @@ def main():
                     help="profiling only: a sub-batch of this many sequences of the workload")
     ap.add_argument("--no-shared-prefix", action="store_true",
                     help="shared-prefix workload: time pa_decode instead of pa_decode_shared_prefix")
+    ap.add_argument("--decode-select", type=int, default=None,
+                    help="pa_decode_select bit mask for the run (tuning; default: the library's)")
+    ap.add_argument("--block-size", type=int, default=0, choices=[0, 8, 16, 32],
+                    help="the workload's shape with another block size (0: its own)")
+    ap.add_argument("--workloads-also", default=None,
+                    help="comma-separated decode workloads also timed on the device and reported "
+                         "under 'workloads' (default with the default workload: " +
+                         ",".join(EXTRA_WORKLOADS) + "; '' for none)")
     ap.add_argument("--op", choices=["decode", "prefill"], default="decode",
                     help="decode: the paged decode step (default); prefill: the chunked-prefill "
                          "attention step")
@@ -873,8 +959,15 @@ def main():
                                       name=cfg.name + f"_small{args.seqs}")
     else:
         cfg = wl.DECODE_WORKLOADS[args.workload] if args.workload else wl.CONFIGS[args.config]
+        default_shape = not (args.seqs or args.block_size or args.workload or args.config != 3)
         if args.seqs:
             cfg = _sample_cfg(cfg, args.seqs)
+        if args.block_size and args.block_size != cfg.block_size:
+            import dataclasses
+            cfg = dataclasses.replace(cfg, block_size=args.block_size,
+                                      name=cfg.name + f"_bs{args.block_size}")
+        if args.workloads_also is None:
+            args.workloads_also = ",".join(EXTRA_WORKLOADS) if default_shape else ""
     if args.impl == "reference":
         (run_reference_prefill if args.op == "prefill" else run_reference)(args, cfg, rank, world)
         return

@@ -18,7 +18,9 @@ namespace {
 // pa_decode_select bits: 1 = CUDA-core consumer only, 2 = L2 evict-first
 // hint on K/V loads, 4 = partition-major grid (kv heads of a partition side
 // by side), 8 = group split-K partitions three to a CTA whenever there are
-// several (a test hook for the grouped path at small sizes); the default is 4.
+// several (a test hook for the grouped path at small sizes), 16 = shared-prefix
+// decode with one CTA per (sequence, kv head) suffix instead of the persistent
+// whole-item grid; the default is 4.
 std::atomic<int> g_select{4};
 
 // Plain split-K with short partitions: one CTA streams g consecutive
@@ -50,12 +52,16 @@ int plan_part_group(int64_t units, int64_t max_parts, int64_t part_bytes, int nu
 
 // SMs of the current device (cached per device; 148 if the query fails).
 int sm_count() {
-    static int sms[256] = {};
+    static std::atomic<int> sms[256] = {};      // threads may race to fill an entry: same value
     int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 256 && !sms[dev])
-        cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
-    return (dev >= 0 && dev < 256 && sms[dev] > 0) ? sms[dev] : 148;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return 148;
+    int n = sms[dev].load(std::memory_order_relaxed);
+    if (n <= 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            return 148;
+        sms[dev].store(n, std::memory_order_relaxed);
+    }
+    return n;
 }
 
 // Launched as a programmatic dependent of the partition kernel so its launch
@@ -71,7 +77,9 @@ cudaError_t launch_merge_t(const dec::Params& p, int wph, dim3 grid, cudaStream_
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, dec::decode_merge<QT, D, NW>, p, wph);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, dec::decode_merge<QT, D, NW>, p, wph);
+    if (e == cudaSuccess) note_launch();
+    return e;
 }
 
 template <int QT, int D>
@@ -115,6 +123,29 @@ int64_t parts_for(int max_ctx, int partition) {
 }
 
 bool is_pow2_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8 || g == 16; }
+
+// The shape and dtype rules every decode launch obeys (pa_decode and the
+// plan query pa_decode_partition_group share them, so the query never
+// describes a launch that pa_decode would refuse).
+pa_status check_decode_shape(pa_dtype q_dt, pa_dtype cache_dt, int S, int Hq, int Hkv, int D,
+                             int bs, int max_ctx, int partition) {
+    if (!valid_dtype(q_dt) || !valid_dtype(cache_dt)) return fail(PA_ERR_INVALID_ARG, "bad dtype");
+    if (S < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || max_ctx < 0 || partition < PA_PARTITION_BALANCED)
+        return fail(PA_ERR_INVALID_ARG, "negative or zero size");
+    if (Hq % Hkv) return fail(PA_ERR_INVALID_ARG, "Hq (%d) is not a multiple of Hkv (%d)", Hq, Hkv);
+    if (!(bs == 8 || bs == 16 || bs == 32))
+        return fail(PA_ERR_UNSUPPORTED, "block size %d (supported: 8, 16, 32)", bs);
+    if (partition != PA_PARTITION_BALANCED && partition % bs)
+        return fail(PA_ERR_INVALID_ARG, "partition %d is not a multiple of bs", partition);
+    const bool pair_ok = (cache_dt == q_dt && cache_dt != PA_FP8_E4M3) ||
+                         (cache_dt == PA_FP8_E4M3 && (q_dt == PA_F16 || q_dt == PA_BF16));
+    if (!pair_ok) return fail(PA_ERR_UNSUPPORTED, "cache dtype %d with q dtype %d", cache_dt, q_dt);
+    const int row = D * elem_size(cache_dt);
+    if (!((D == 64 || D == 128 || D == 256) && (row == 128 || row == 256 || row == 512)))
+        return fail(PA_ERR_UNSUPPORTED, "head dim %d with this cache dtype", D);
+    if (!is_pow2_group(Hq / Hkv)) return fail(PA_ERR_UNSUPPORTED, "group size %d", Hq / Hkv);
+    return PA_OK;
+}
 
 }  // namespace
 }  // namespace pa
@@ -177,13 +208,14 @@ extern "C" pa_status pa_decode_suggest_partition(int S, int Hkv, int bs,
     return PA_OK;
 }
 
-extern "C" pa_status pa_decode_partition_group(int S, int Hq, int Hkv, int D, pa_dtype cache_dt,
-                                               int max_ctx, int partition, int num_sms,
-                                               int* group) {
+extern "C" pa_status pa_decode_partition_group(int S, int Hq, int Hkv, int D, int bs,
+                                               pa_dtype q_dt, pa_dtype cache_dt, int max_ctx,
+                                               int partition, int num_sms, int* group) {
     clear_error();
-    if (!group || S < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || max_ctx < 0 || partition < 0 ||
-        !valid_dtype(cache_dt) || !(D == 64 || D == 128 || D == 256))
-        return fail(PA_ERR_INVALID_ARG, "bad arguments");
+    if (!group) return fail(PA_ERR_INVALID_ARG, "group is NULL");
+    if (partition < 0) return fail(PA_ERR_INVALID_ARG, "partition must be >= 0 (no balanced grid)");
+    pa_status chk = check_decode_shape(q_dt, cache_dt, S, Hq, Hkv, D, bs, max_ctx, partition);
+    if (chk) return chk;
     const int G = Hq / Hkv;
     const int sel = g_select.load();
     const bool use_mma = !(sel & 1) && G >= 2 && D <= 128 && cache_dt != PA_F32;
@@ -199,7 +231,7 @@ extern "C" pa_status pa_decode_partition_group(int S, int Hq, int Hkv, int D, pa
 
 extern "C" pa_status pa_decode_select(int mode) {
     clear_error();
-    if (mode < 0 || mode > 15) return fail(PA_ERR_INVALID_ARG, "mode must be in [0, 15]");
+    if (mode < 0 || mode > 31) return fail(PA_ERR_INVALID_ARG, "mode must be in [0, 31]");
     g_select.store(mode);
     return PA_OK;
 }
@@ -215,30 +247,17 @@ pa_status pa::decode_impl(void* out, const void* q, pa_dtype q_dt, const void* k
                           float v_scale, int partition, void* workspace, size_t workspace_bytes,
                           pa_stream_t stream, int prefix_parts, int force_ws,
                           int fuse_prefix_blocks) {
-    if (!valid_dtype(q_dt) || !valid_dtype(cache_dt)) return fail(PA_ERR_INVALID_ARG, "bad dtype");
-    if (S < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || MB < 0 || NB <= 0 || max_ctx < 0 ||
-        partition < PA_PARTITION_BALANCED)
-        return fail(PA_ERR_INVALID_ARG, "negative or zero size");
-    if (Hq % Hkv) return fail(PA_ERR_INVALID_ARG, "Hq (%d) is not a multiple of Hkv (%d)", Hq, Hkv);
-    if (!(bs == 8 || bs == 16 || bs == 32))
-        return fail(PA_ERR_UNSUPPORTED, "block size %d (supported: 8, 16, 32)", bs);
+    pa_status chk = check_decode_shape(q_dt, cache_dt, S, Hq, Hkv, D, bs, max_ctx, partition);
+    if (chk) return chk;
+    if (MB < 0 || NB <= 0) return fail(PA_ERR_INVALID_ARG, "negative or zero size");
     const bool balanced = partition == PA_PARTITION_BALANCED;
-    if (!balanced && partition % bs)
-        return fail(PA_ERR_INVALID_ARG, "partition %d is not a multiple of bs", partition);
     if (NB > 0x7fffffffLL) return fail(PA_ERR_INVALID_ARG, "NB exceeds int32 block ids");
     if (!(std::isfinite(scale)) || !(std::isfinite(k_scale) && k_scale > 0) ||
         !(std::isfinite(v_scale) && v_scale > 0))
         return fail(PA_ERR_INVALID_ARG, "scales must be finite (k_scale, v_scale > 0)");
     if (cache_dt != PA_FP8_E4M3 && (k_scale != 1.f || v_scale != 1.f))
         return fail(PA_ERR_INVALID_ARG, "k_scale / v_scale apply to fp8 caches only");
-    const bool pair_ok = (cache_dt == q_dt && cache_dt != PA_FP8_E4M3) ||
-                         (cache_dt == PA_FP8_E4M3 && (q_dt == PA_F16 || q_dt == PA_BF16));
-    if (!pair_ok) return fail(PA_ERR_UNSUPPORTED, "cache dtype %d with q dtype %d", cache_dt, q_dt);
-    const int row = D * elem_size(cache_dt);
-    if (!((D == 64 || D == 128 || D == 256) && (row == 128 || row == 256 || row == 512)))
-        return fail(PA_ERR_UNSUPPORTED, "head dim %d with this cache dtype", D);
     const int G = Hq / Hkv;
-    if (!is_pow2_group(G)) return fail(PA_ERR_UNSUPPORTED, "group size %d", G);
     if (S == 0) return PA_OK;
     if (S > 65535 || (int64_t)Hkv * G > 65535) return fail(PA_ERR_UNSUPPORTED, "grid too large");
     if (!out || !q || !key_cache || !value_cache || !block_tables || !context_lens)
@@ -263,6 +282,10 @@ pa_status pa::decode_impl(void* out, const void* q, pa_dtype q_dt, const void* k
     const int gc = use_mma ? G : gc_simt;
     const int chunks = use_mma ? 1 : G / gc_simt;
     const int num_sms = sm_count();
+    // shared-prefix decode with whole suffixes: a persistent grid streams the
+    // (sequence, kv head) items back to back, each CTA a contiguous run of
+    // whole items of about equal work (one CTA per item with bit 16)
+    const bool items = fuse && !(sel & 16);
     int part_group = 1;
     if (use_mma && !balanced && !fuse && prefix_parts == 0 && !force_ws && max_parts > 1)
         part_group = (sel & 8) ? 3
@@ -314,7 +337,8 @@ pa_status pa::decode_impl(void* out, const void* q, pa_dtype q_dt, const void* k
     p.v_scale = v_scale;
     p.bs = bs;
     p.gc = gc;
-    p.balanced = balanced ? 1 : 0;
+    p.balanced = balanced || items ? 1 : 0;
+    p.whole_items = items ? 1 : 0;
     if (balanced) {
         const size_t items = (size_t)S * (Hq / gc);
         const size_t rows = (items + dec::kMaxBalancedCtas) * gc;
@@ -335,7 +359,7 @@ pa_status pa::decode_impl(void* out, const void* q, pa_dtype q_dt, const void* k
     L.mma = use_mma;
     L.mrows = G <= 8 ? 8 : 16;
     L.gc = gc_simt;
-    L.balanced = balanced;
+    L.balanced = balanced || items;
     L.G = G;
     L.num_sms = num_sms;
     L.grid = p.heads_fastest ? dim3((unsigned)(Hkv * chunks), (unsigned)grid_parts, (unsigned)S)
@@ -364,6 +388,7 @@ extern "C" pa_status pa_decode(void* out, const void* q, pa_dtype q_dt, const vo
                                int S, int Hq, int Hkv, int D, int bs, int64_t NB, int max_ctx,
                                float scale, float k_scale, float v_scale, int partition,
                                void* workspace, size_t workspace_bytes, pa_stream_t stream) {
+    PA_NVTX_RANGE("pa_decode");
     clear_error();
     return decode_impl(out, q, q_dt, key_cache, value_cache, cache_dt, block_tables, MB,
                        context_lens, S, Hq, Hkv, D, bs, NB, max_ctx, scale, k_scale, v_scale,

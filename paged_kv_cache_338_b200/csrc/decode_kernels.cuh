@@ -80,6 +80,10 @@ struct Params {
                                  // merges the prefix_parts prefix records and writes the output
     int part_group;              // plain split-K: consecutive partitions one CTA streams (>= 1),
                                  // still one record per partition
+    int whole_items;             // balanced grid only: 1 = every item stays on one CTA (CTA
+                                 // ranges end at item boundaries), whose output it writes;
+                                 // with fuse_prefix_blocks the regular items read their suffix
+                                 // and fold the prefix_parts prefix records in
 };
 
 // Record a wait that gave up, with the site that gave up (bits 16-23).
@@ -1098,7 +1102,7 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
 constexpr int kItemQ = 4;
 
 struct PieceDesc {
-    int s, hc, off, take, nblk, n, k0, end;
+    int s, hc, off, take, nblk, n, k0, end, fold;
 };
 
 template <class C>
@@ -1115,9 +1119,52 @@ struct BalancedSmem {
     static size_t bytes(int gc) { return FIXED + size_t(C::NW) * gc * (C::D + 2) * 4; }
 };
 
+// Work of each of sequence s's items in the balanced grid's block space.
+// Split pieces: its blocks.  Whole items: its blocks past a shared prefix it
+// is expected to skip (long enough to hold it; the producer checks the table
+// itself, so a wrong guess costs balance, never correctness), plus one for
+// the item's own start-up and epilogue (an item with no block still needs its
+// output written).
 template <class C>
 __device__ __forceinline__ int blocks_of(const Params& p, int s) {
-    return (checked_len(p, s, C::BS) + C::BS - 1) / C::BS;
+    const int n = checked_len(p, s, C::BS);
+    const int nb = (n + C::BS - 1) / C::BS;
+    if (!p.whole_items) return nb;
+    const int pb = p.fuse_prefix_blocks;
+    return (pb > 0 && n >= pb * C::BS ? nb - pb : nb) + 1;
+}
+
+// Fold the prefix_parts prefix records of (sequence s, head h) into a state
+// (M in log2 units, L, O already times v_scale) and return the output value.
+// The records are loaded first, so their latencies overlap.
+__device__ __forceinline__ float fold_prefix_records(const Params& p, int s, int h, int d,
+                                                     float M, float L, float O, int D) {
+    constexpr int kMaxUnrolled = 8;
+    const size_t row0 = ((size_t)s * p.Hq + h) * p.max_parts;
+    for (int pp = 0; pp < p.prefix_parts; pp += kMaxUnrolled) {
+        float2 ml[kMaxUnrolled];
+        float o[kMaxUnrolled];
+        #pragma unroll
+        for (int i = 0; i < kMaxUnrolled; ++i) {
+            if (pp + i < p.prefix_parts) {
+                ml[i] = p.ws_ml[row0 + pp + i];
+                o[i] = p.ws_o[(row0 + pp + i) * D + d];
+            } else {
+                ml[i] = make_float2(-INFINITY, 0.f);
+                o[i] = 0.f;
+            }
+        }
+        #pragma unroll
+        for (int i = 0; i < kMaxUnrolled; ++i) {
+            const float Mn = fmaxf(M, ml[i].x);
+            if (Mn == -INFINITY) continue;
+            const float a = exp2f(M - Mn), b = exp2f(ml[i].x - Mn);
+            L = L * a + ml[i].y * b;
+            O = O * a + o[i] * b;
+            M = Mn;
+        }
+    }
+    return L > 0.f ? O / L : 0.f;
 }
 
 // The configuration of the balanced kernel: the same tile shapes, a deeper ring.
@@ -1250,24 +1297,57 @@ decode_balanced(const __grid_constant__ CUtensorMap tmk, const __grid_constant__
             }
             return __shfl_sync(0xffffffffu, bad, 0) != 0;
         };
-        while (!stop && b < b1 && s < p.S) {
-            const int n = checked_len(p, s, C::BS);
-            const int nb = (n + C::BS - 1) / C::BS;
-            if (nb > off) {
-                const int take = (int)min((long long)(nb - off), b1 - b);
-                PieceDesc d{s, hc, off, take, nb, n, k, 0};
+        if (p.whole_items) {
+            // Whole items: this CTA takes the items that start inside
+            // [b0, b1); the item holding b0 is its own only if it starts there.
+            b -= off;
+            if (!stop && off > 0) {
+                b += blocks_of<C>(p, s);
+                if (++hc == HC) { hc = 0; ++s; }
+            }
+            const int pb = p.fuse_prefix_blocks;
+            int reg_s = -1, reg = 0;                   // regularity of sequence reg_s
+            while (!stop && b < b1 && s < p.S) {
+                const int n = checked_len(p, s, C::BS);
+                const int nb = (n + C::BS - 1) / C::BS;
+                if (pb > 0 && s != reg_s) {
+                    // regular: long enough, and its table starts with row 0's prefix blocks
+                    int diff = n < pb * C::BS;
+                    for (int i = lane; i < pb && !diff; i += 32)
+                        diff = __ldg(p.block_tables + (size_t)s * p.MB + i) != __ldg(p.block_tables + i);
+                    reg = !__any_sync(0xffffffffu, diff);
+                    reg_s = s;
+                }
+                const int blk0 = pb > 0 && reg ? pb : 0;
+                PieceDesc d{s, hc, blk0, nb - blk0, nb, n, k, 0, blk0 > 0};
                 if (publish(d)) break;
-                produce<C>(&tmk, &tmv, p, p.block_tables + (size_t)s * p.MB, off, take,
+                produce<C>(&tmk, &tmv, p, p.block_tables + (size_t)s * p.MB, blk0, nb - blk0,
                             hc / chunks, stages, full0, empty0, &s_abort, &k);
                 if (*(volatile int*)&s_abort) break;
-                b += take;
+                b += blocks_of<C>(p, s);
                 ++ci;
+                if (++hc == HC) { hc = 0; ++s; }
             }
-            off = 0;
-            if (++hc == HC) { hc = 0; ++s; }
+        } else {
+            while (!stop && b < b1 && s < p.S) {
+                const int n = checked_len(p, s, C::BS);
+                const int nb = (n + C::BS - 1) / C::BS;
+                if (nb > off) {
+                    const int take = (int)min((long long)(nb - off), b1 - b);
+                    PieceDesc d{s, hc, off, take, nb, n, k, 0, 0};
+                    if (publish(d)) break;
+                    produce<C>(&tmk, &tmv, p, p.block_tables + (size_t)s * p.MB, off, take,
+                                hc / chunks, stages, full0, empty0, &s_abort, &k);
+                    if (*(volatile int*)&s_abort) break;
+                    b += take;
+                    ++ci;
+                }
+                off = 0;
+                if (++hc == HC) { hc = 0; ++s; }
+            }
         }
         if (!*(volatile int*)&s_abort) {
-            PieceDesc d{0, 0, 0, 0, 0, 0, k, 1};
+            PieceDesc d{0, 0, 0, 0, 0, 0, k, 1, 0};
             publish(d);
         }
         if (lane == 0) s_issued = k;
@@ -1316,7 +1396,8 @@ decode_balanced(const __grid_constant__ CUtensorMap tmk, const __grid_constant__
             }
             // ---- combine the four warps' states for this piece -----------
             const int item = d.s * HC + d.hc;
-            const bool first = d.off == 0, last = d.off + d.take == d.nblk;
+            const bool whole = p.whole_items != 0;
+            const bool first = whole || d.off == 0, last = whole || d.off + d.take == d.nblk;
             const int piece = item + blockIdx.x;
             for (int idx = threadIdx.x; idx < gc * C::D; idx += C::NW * 32) {
                 const int g = idx / C::D, dd = idx % C::D;
@@ -1332,7 +1413,11 @@ decode_balanced(const __grid_constant__ CUtensorMap tmk, const __grid_constant__
                         O = fmaf(f, co[(w * gc + g) * C::D + dd], O);
                     }
                 }
-                if (first && last) {
+                if (d.fold) {
+                    dev::store_out<C::QT>(p.out, ((size_t)d.s * p.Hq + h0 + g) * C::D + dd,
+                                          fold_prefix_records(p, d.s, h0 + g, dd, M, L,
+                                                              O * p.v_scale, C::D));
+                } else if (first && last) {
                     dev::store_out<C::QT>(p.out, ((size_t)d.s * p.Hq + h0 + g) * C::D + dd,
                                           L > 0.f ? (O / L) * p.v_scale : 0.f);
                 } else {
@@ -1345,7 +1430,7 @@ decode_balanced(const __grid_constant__ CUtensorMap tmk, const __grid_constant__
                     }
                 }
             }
-            if (threadIdx.x == 0) {
+            if (threadIdx.x == 0 && !whole) {
                 if (first) p.ws_item[item].x = blockIdx.x;
                 if (last) p.ws_item[item].y = blockIdx.x;
             }

@@ -7,6 +7,12 @@ caches, prefixes of one chunk, several chunks and an uneven length; a sequence
 whose table does not start with row 0's prefix blocks (its own prefix has other
 values: a wrong fall-back shows up as an error), a sequence shorter than the
 prefix and one that holds exactly the prefix.  Tolerances are the decode bars.
+
+Short suffixes are decoded two ways, both checked: the default persistent grid
+(each CTA streams a contiguous run of whole (sequence, kv head) suffixes and
+folds the prefix records into each) and one CTA per suffix
+(DECODE_SUFFIX_PER_CTA).  A batch of many short suffixes puts several items
+on every CTA of the persistent grid.
 """
 import dataclasses
 
@@ -29,6 +35,17 @@ def _cuda():
         pytest.skip("needs a GPU")
     pa.pa_device_status(clear=True)
     yield
+
+
+MODES = {"persistent": pa.DECODE_DEFAULT,
+         "per_cta": pa.DECODE_DEFAULT | pa.DECODE_SUFFIX_PER_CTA}
+
+
+@pytest.fixture(params=sorted(MODES))
+def mode(request):
+    pa.pa_decode_select(MODES[request.param])
+    yield request.param
+    pa.pa_decode_select(pa.DECODE_DEFAULT)
 
 
 def _appended(inp: wl.DecodeInputs):
@@ -87,11 +104,13 @@ CASES = [
     ("bf16_d64_g2", dataclasses.replace(wl.DECODE_WORKLOADS["prefix_shared_fp8_b256"], kv_dtype="bf16", head_dim=64,
                                         num_q_heads=8, num_kv_heads=4, block_size=16,
                                         fp8_scaled=False), 6, 1, 150, 256),
+    # 1600 items of 1..4 blocks: several whole items per CTA of the persistent grid
+    ("fp8_bs32_many", wl.DECODE_WORKLOADS["prefix_shared_fp8_b256"], 200, 1, 120, 128),
 ]
 
 
 @pytest.mark.parametrize("name,base,nseq,lo,hi,prefix", CASES, ids=[c[0] for c in CASES])
-def test_shared_prefix_matches_decode(name, base, nseq, lo, hi, prefix):
+def test_shared_prefix_matches_decode(name, base, nseq, lo, hi, prefix, mode):
     cfg = wl.small_variant(base, nseq, lo, hi, prefix_tokens=prefix)
     inp = wl.make_decode_inputs(cfg, seed=len(name))
     kc, vc = _appended(inp)
@@ -101,7 +120,7 @@ def test_shared_prefix_matches_decode(name, base, nseq, lo, hi, prefix):
     _check(out, inp, kc, vc, inp.block_tables, inp.context_lens, name)
 
 
-def test_sequences_outside_the_shared_prefix_fall_back():
+def test_sequences_outside_the_shared_prefix_fall_back(mode):
     cfg = wl.small_variant(wl.DECODE_WORKLOADS["prefix_shared_fp8_b256"], 8, 20, 200, prefix_tokens=512)
     inp = wl.make_decode_inputs(cfg, seed=3)
     kc, vc = _appended(inp)
@@ -144,3 +163,27 @@ def test_long_suffixes_take_the_split_path():
     out = _run(inp, kc, vc, tables, lens, 256, inp.max_ctx)
     assert pa.pa_device_status() == 0
     _check(out, inp, kc, vc, tables, lens, "split")
+
+
+def test_irregular_sequences_inside_a_long_batch(mode):
+    """Regular and irregular sequences side by side in the runs of whole items a
+    persistent CTA streams: a foreign first block, one shorter than the prefix,
+    one holding exactly the prefix (an item with no suffix block), next to
+    regular ones."""
+    cfg = wl.small_variant(wl.DECODE_WORKLOADS["prefix_shared_fp8_b256"], 160, 1, 100,
+                           prefix_tokens=128)
+    inp = wl.make_decode_inputs(cfg, seed=21)
+    kc, vc = _appended(inp)
+    tables, lens = inp.block_tables.clone(), inp.context_lens.clone()
+    g = torch.Generator().manual_seed(5)
+    for s, fb in ((5, 0), (50, 1), (51, 2)):
+        own = int(inp.free_blocks[fb])
+        kc[own] = (torch.randn(kc[own].shape, generator=g) / inp.k_scale).clamp(-448, 448).to(kc.dtype)
+        vc[own] = (torch.randn(vc[own].shape, generator=g) / inp.v_scale).clamp(-448, 448).to(vc.dtype)
+        tables[s, fb] = own                         # its prefix differs in block fb
+    lens[7] = 70                                    # shorter than the prefix
+    lens[8] = 128                                   # exactly the prefix
+    lens[9] = 129                                   # one suffix token
+    out = _run(inp, kc, vc, tables, lens, 128, inp.max_ctx)
+    assert pa.pa_device_status() == 0
+    _check(out, inp, kc, vc, tables, lens, "irregular in a long batch")
