@@ -527,11 +527,13 @@ def run_gpu(args, cfg, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
-def run_e2e(args, cfg, pa, dev, part):
+def run_e2e(args, cfg, pa, dev, part, keep_state=False):
     """Host pool + pinned host buffers + H2D / step / D2H every step, pipelined
     the way a serving loop runs: the host builds step i + 1's slots and tables
     while the GPU runs step i; every step's inputs still cross H2D and its
-    output D2H inside the timed region."""
+    output D2H inside the timed region.  keep_state: also return the last
+    step's host-side inputs and output and the caches after it (for a check
+    of the loop's result)."""
     g = torch.Generator().manual_seed(args.seed + 77)
     inp = wl.make_decode_inputs(cfg, seed=args.seed + 5, device=dev)
     max_ctx = inp.max_ctx + args.warmup + args.steps + 2     # sequences grow one token a step
@@ -663,9 +665,16 @@ def run_e2e(args, cfg, pa, dev, part):
     h2d = total
     d2h = out_h[0].numel() * out_h[0].element_size()
     pool.close()
-    return {"ms": ms / args.steps, "bytes": total_bytes / args.steps,
-            "value": (total_bytes / args.steps) / (ms / args.steps * 1e-3) / 1e9,
-            "h2d": h2d, "d2h": d2h}
+    res = {"ms": ms / args.steps, "bytes": total_bytes / args.steps,
+           "value": (total_bytes / args.steps) / (ms / args.steps * 1e-3) / 1e9,
+           "h2d": h2d, "d2h": d2h}
+    if keep_state:
+        k = (args.warmup + args.steps - 1) % NSLOT
+        res["state"] = {"q": hv[k]["q"].clone(), "tables": hv[k]["tables"].clone(),
+                        "lens": hv[k]["lens"].clone(), "out": out_h[k].clone(),
+                        "key_cache": kc.cpu(), "value_cache": vc.cpu(),
+                        "scale": inp.scale, "k_scale": inp.k_scale, "v_scale": inp.v_scale}
+    return res
 
 
 # ------------------------------------------------------------- prefill (next row)

@@ -173,10 +173,14 @@ struct CopyList {
     int2 pair[kMaxPairsPerLaunch];
 };
 
-// blockIdx.x = pair, blockIdx.y = 0 (K) / 1 (V); 16-byte vectors.
+// blockIdx.x = pair, blockIdx.y = 0 (K) / 1 (V); 16-byte vectors.  The host
+// has checked that no destination is also a source, so each thread loads a
+// batch of vectors before it stores any (a plain load-store loop would keep
+// one load in flight per thread).
 __global__ void __launch_bounds__(256) copy_blocks_kernel(uint8_t* __restrict__ kc,
                                                           uint8_t* __restrict__ vc, size_t block_bytes,
                                                           const __grid_constant__ CopyList list) {
+    constexpr int kBatch = 8;
     dev::grid_dependency_wait();       // launched as a dependent of the kernel before it
     dev::launch_dependents();
     const int2 pr = list.pair[blockIdx.x];
@@ -184,7 +188,19 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(uint8_t* __restrict__ 
     const uint4* src = reinterpret_cast<const uint4*>(base + (size_t)pr.x * block_bytes);
     uint4* dst = reinterpret_cast<uint4*>(base + (size_t)pr.y * block_bytes);
     const size_t n16 = block_bytes / 16;
-    for (size_t i = threadIdx.x; i < n16; i += blockDim.x) dst[i] = src[i];
+    for (size_t i0 = threadIdx.x; i0 < n16; i0 += (size_t)kBatch * blockDim.x) {
+        uint4 r[kBatch];
+        #pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const size_t i = i0 + (size_t)u * blockDim.x;
+            if (i < n16) r[u] = src[i];
+        }
+        #pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const size_t i = i0 + (size_t)u * blockDim.x;
+            if (i < n16) dst[i] = r[u];
+        }
+    }
 }
 
 }  // namespace

@@ -119,12 +119,9 @@ struct Cfg {
     static constexpr int STAGE = 2 * TILE;
     static constexpr int NW = 4;             // consumer warps
     static constexpr int THREADS = (NW + 1) * 32;
-    // fp8 + tensor cores: each consumer warp dequantises V into an f16 tile
-    static constexpr bool FP8MMA = MMA && DT == PA_FP8_E4M3;
-    static constexpr int VSTG = FP8MMA ? BS * D * 2 : 0;     // per-warp staging bytes
-    static constexpr int BUDGET = (FP8MMA ? 72 : 64) * 1024;  // 3 CTAs per SM fit
+    static constexpr int BUDGET = 64 * 1024;                  // 3 CTAs per SM fit
     static constexpr int COMBINE_FLOATS = NW * GC * (D + 2);   // warp merge reuses the stages
-    static constexpr int STAGES_RAW = (BUDGET - NW * VSTG) / STAGE;
+    static constexpr int STAGES_RAW = BUDGET / STAGE;
     static constexpr int STAGES_MIN_C = (COMBINE_FLOATS * 4 + STAGE - 1) / STAGE;
     static constexpr int STAGES_MIN = STAGES_MIN_C > NW ? STAGES_MIN_C : NW;
     static constexpr int STAGES_MAX = STAGES_MIN > 16 ? STAGES_MIN : 16;
@@ -139,8 +136,7 @@ struct Cfg {
     static constexpr int STAGES_DOWN = STAGES_CLAMPED / NW * NW;
     static constexpr int STAGES = STAGES_DOWN >= STAGES_MIN ? STAGES_DOWN
                                   : (STAGES_MIN + NW - 1) / NW * NW;
-    static constexpr size_t SMEM = 1024 /*align slack*/ + size_t(STAGES) * STAGE +
-                                   size_t(NW) * VSTG + 2 * 8 * STAGES;
+    static constexpr size_t SMEM = 1024 /*align slack*/ + size_t(STAGES) * STAGE + 2 * 8 * STAGES;
     static_assert(R == 128 || R == 256 || R == 512, "row bytes must be 128, 256 or 512");
     static_assert(BS == 8 || BS == 16 || BS == 32, "block size");
     static_assert(STAGES % NW == 0, "each stage must have a single consumer warp");
@@ -434,8 +430,13 @@ __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
 // (a b16 lane holds 2 codes, so a thread receives 4 consecutive dims) and are
 // widened with cvt.f16x2.e4m3x2; the contraction index is permuted the same
 // way on Q, so logical k (2t, 2t+1 | 2t+8, 2t+9) of a 16-dim step is physical
-// dim (4t, 4t+1 | 4t+2, 4t+3).  V is widened into a per-warp f16 tile first
-// (ldmatrix.trans has no byte form), with rows past the valid tokens zeroed.
+// dim (4t, 4t+1 | 4t+2, 4t+3).  V^T fragments also come straight from the
+// codes: ldmatrix.trans on 16-bit units hands a thread tokens (2t, 2t+1) of
+// dims (2g, 2g+1), a byte permute pairs the two tokens of one dim and the
+// pair is widened; so logical row g of an O^T m-tile is physical dim 2g and
+// row g + 8 is dim 2g + 1 (undone when the accumulators are published).
+// Codes of tokens past the valid ones are cleared before widening (a zero
+// weight times a NaN code would still be NaN).
 template <class C>
 struct MmaState {
     static constexpr bool FP8 = C::DT == PA_FP8_E4M3;
@@ -508,39 +509,9 @@ __device__ __forceinline__ uint32_t chunk_addr(uint32_t tile, int t, int c) {
     return tile + tile_off<C>(t, c >> 3, c & 7);
 }
 
-// fp8 V tile -> f16 tile (same segment-major swizzled layout, 64 dims per
-// segment); rows at or past nvalid become zeros.
-template <class C>
-__device__ __forceinline__ void stage_v_f16(const uint8_t* vt, uint8_t* dst, int nvalid) {
-    const int lane = threadIdx.x & 31;
-    __syncwarp();                                  // previous block's reads of dst are done
-    #pragma unroll
-    for (int i = 0; i < C::BS / 4; ++i) {
-        const int idx = lane + 32 * i;
-        const int t = idx >> 3, j = idx & 7;       // token, 16-dim chunk of the fp8 row
-        uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
-        if (t < nvalid) {
-            const uint4 r = *reinterpret_cast<const uint4*>(vt + tile_off<C>(t, 0, j));
-            lo = make_uint4(e4m3x2_to_f16x2(r.x), e4m3x2_to_f16x2(r.x >> 16),
-                            e4m3x2_to_f16x2(r.y), e4m3x2_to_f16x2(r.y >> 16));
-            hi = make_uint4(e4m3x2_to_f16x2(r.z), e4m3x2_to_f16x2(r.z >> 16),
-                            e4m3x2_to_f16x2(r.w), e4m3x2_to_f16x2(r.w >> 16));
-        }
-        // f16 dims 16j..16j+7 -> segment j/4, chunk 2(j%4); +8.. -> chunk 2(j%4)+1.
-        // Lanes j >= 4 store their second chunk first, so each store instruction
-        // covers 8 distinct bank groups.
-        const int seg = j >> 2, c0 = 2 * (j & 3);
-        const bool swap = j >= 4;
-        uint8_t* base = dst + seg * (C::BS * 128);
-        *reinterpret_cast<uint4*>(base + dev::swz128(t, c0 + (swap ? 1 : 0))) = swap ? hi : lo;
-        *reinterpret_cast<uint4*>(base + dev::swz128(t, c0 + (swap ? 0 : 1))) = swap ? lo : hi;
-    }
-    __syncwarp();
-}
-
 template <class C>
 __device__ __forceinline__ void mma_block(MmaState<C>& st, uint8_t* ktile_p, uint8_t* vtile_p,
-                                          uint8_t* vstage_p, int nvalid, float qk_scale) {
+                                          int nvalid, float qk_scale) {
     using S = MmaState<C>;
     constexpr int BS = C::BS;
     constexpr int CT = S::CT;
@@ -690,12 +661,64 @@ __device__ __forceinline__ void mma_block(MmaState<C>& st, uint8_t* ktile_p, uin
             }
         }
     }
-    // ---- V operand: the 16-bit tile itself (tail rows zeroed), or fp8 widened
-    uint32_t vtile;
+    // ---- O^T += V^T P^T ---------------------------------------------------------
     if constexpr (S::FP8) {
-        stage_v_f16<C>(vtile_p, vstage_p, nvalid);
-        vtile = dev::smem_addr(vstage_p);
+        const uint32_t vt = dev::smem_addr(vtile_p);
+        const int tig = lane & 3;
+        const bool tail = nvalid < BS;
+        if constexpr (BS >= 16) {
+            #pragma unroll
+            for (int kt = 0; kt < MT; ++kt) {
+                // bytes 0-1 of a fragment word: token 2tig; bytes 2-3: token 2tig + 1
+                uint32_t keep0 = 0xffffffffu, keep1 = 0xffffffffu;
+                if (tail) {
+                    const int t0 = kt * 16 + 2 * tig;
+                    keep0 = (t0 < nvalid ? 0x0000ffffu : 0u) | (t0 + 1 < nvalid ? 0xffff0000u : 0u);
+                    keep1 = (t0 + 8 < nvalid ? 0x0000ffffu : 0u) | (t0 + 9 < nvalid ? 0xffff0000u : 0u);
+                }
+                #pragma unroll
+                for (int md = 0; md < S::MD; md += 2) {
+                    // matrices: (tok 0-7, chunk md) (tok 8-15, md) (tok 0-7, md+1) (tok 8-15, md+1)
+                    uint32_t r0, r1, r2, r3;
+                    ldsm_x4_t(chunk_addr<C>(vt, kt * 16 + ((lane >> 3) & 1) * 8 + (lane & 7),
+                                            md + (lane >> 4)),
+                              r0, r1, r2, r3);
+                    const uint32_t s0 = __byte_perm(r0 & keep0, 0, 0x3120);
+                    const uint32_t s1 = __byte_perm(r1 & keep1, 0, 0x3120);
+                    const uint32_t s2 = __byte_perm(r2 & keep0, 0, 0x3120);
+                    const uint32_t s3 = __byte_perm(r3 & keep1, 0, 0x3120);
+                    const uint32_t a0 = e4m3x2_to_f16x2(s0), a1 = e4m3x2_to_f16x2(s0 >> 16);
+                    const uint32_t a2 = e4m3x2_to_f16x2(s1), a3 = e4m3x2_to_f16x2(s1 >> 16);
+                    const uint32_t b0 = e4m3x2_to_f16x2(s2), b1 = e4m3x2_to_f16x2(s2 >> 16);
+                    const uint32_t b2 = e4m3x2_to_f16x2(s3), b3 = e4m3x2_to_f16x2(s3 >> 16);
+                    #pragma unroll
+                    for (int nh = 0; nh < S::NH; ++nh) {
+                        mma16816<CT>(st.o[nh][md], a0, a1, a2, a3, pb[kt][nh][0], pb[kt][nh][1]);
+                        mma16816<CT>(st.o[nh][md + 1], b0, b1, b2, b3, pb[kt][nh][0],
+                                     pb[kt][nh][1]);
+                    }
+                }
+            }
+        } else {
+            uint32_t keep = 0xffffffffu;
+            if (tail)
+                keep = (2 * tig < nvalid ? 0x0000ffffu : 0u) | (2 * tig + 1 < nvalid ? 0xffff0000u : 0u);
+            #pragma unroll
+            for (int md = 0; md < S::MD; md += 4) {
+                // matrices: tokens 0-7 of chunks md, md+1, md+2, md+3
+                uint32_t r[4];
+                ldsm_x4_t(chunk_addr<C>(vt, lane & 7, md + (lane >> 3)), r[0], r[1], r[2], r[3]);
+                #pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t sw = __byte_perm(r[i] & keep, 0, 0x3120);
+                    const uint32_t a0 = e4m3x2_to_f16x2(sw), a1 = e4m3x2_to_f16x2(sw >> 16);
+                    #pragma unroll
+                    for (int nh = 0; nh < S::NH; ++nh) mma1688<CT>(st.o[nh][md + i], a0, a1, pb[0][nh][0]);
+                }
+            }
+        }
     } else {
+        // the 16-bit tile itself, tail rows zeroed
         if (nvalid < BS) {
             #pragma unroll
             for (int k = 0; k < C::CH; ++k) {
@@ -704,34 +727,33 @@ __device__ __forceinline__ void mma_block(MmaState<C>& st, uint8_t* ktile_p, uin
             }
             __syncwarp();
         }
-        vtile = dev::smem_addr(vtile_p);
-    }
-    // ---- O^T += V^T P^T -------------------------------------------------------
-    if constexpr (BS >= 16) {
-        #pragma unroll
-        for (int kt = 0; kt < MT; ++kt) {
+        const uint32_t vtile = dev::smem_addr(vtile_p);
+        if constexpr (BS >= 16) {
             #pragma unroll
-            for (int md = 0; md < S::MD; ++md) {
-                // matrices: (tok 0-7, chunk 2md) (tok 0-7, 2md+1) (tok 8-15, 2md) (tok 8-15, 2md+1)
-                uint32_t a0, a1, a2, a3;
-                ldsm_x4_t(chunk_addr<C>(vtile, kt * 16 + (lane >> 4) * 8 + (lane & 7),
-                                        2 * md + ((lane >> 3) & 1)),
-                          a0, a1, a2, a3);
+            for (int kt = 0; kt < MT; ++kt) {
                 #pragma unroll
-                for (int nh = 0; nh < S::NH; ++nh)
-                    mma16816<CT>(st.o[nh][md], a0, a1, a2, a3, pb[kt][nh][0], pb[kt][nh][1]);
+                for (int md = 0; md < S::MD; ++md) {
+                    // matrices: (tok 0-7, chunk 2md) (tok 0-7, 2md+1) (tok 8-15, 2md) (tok 8-15, 2md+1)
+                    uint32_t a0, a1, a2, a3;
+                    ldsm_x4_t(chunk_addr<C>(vtile, kt * 16 + (lane >> 4) * 8 + (lane & 7),
+                                            2 * md + ((lane >> 3) & 1)),
+                              a0, a1, a2, a3);
+                    #pragma unroll
+                    for (int nh = 0; nh < S::NH; ++nh)
+                        mma16816<CT>(st.o[nh][md], a0, a1, a2, a3, pb[kt][nh][0], pb[kt][nh][1]);
+                }
             }
-        }
-    } else {
-        #pragma unroll
-        for (int md = 0; md < S::MD; md += 2) {
-            // matrices: tokens 0-7 of chunks 2md, 2md+1, 2md+2, 2md+3
-            uint32_t a0, a1, b0, b1;
-            ldsm_x4_t(chunk_addr<C>(vtile, lane & 7, 2 * md + (lane >> 3)), a0, a1, b0, b1);
+        } else {
             #pragma unroll
-            for (int nh = 0; nh < S::NH; ++nh) {
-                mma1688<CT>(st.o[nh][md], a0, a1, pb[0][nh][0]);
-                mma1688<CT>(st.o[nh][md + 1], b0, b1, pb[0][nh][0]);
+            for (int md = 0; md < S::MD; md += 2) {
+                // matrices: tokens 0-7 of chunks 2md, 2md+1, 2md+2, 2md+3
+                uint32_t a0, a1, b0, b1;
+                ldsm_x4_t(chunk_addr<C>(vtile, lane & 7, 2 * md + (lane >> 3)), a0, a1, b0, b1);
+                #pragma unroll
+                for (int nh = 0; nh < S::NH; ++nh) {
+                    mma1688<CT>(st.o[nh][md], a0, a1, pb[0][nh][0]);
+                    mma1688<CT>(st.o[nh][md + 1], b0, b1, pb[0][nh][0]);
+                }
             }
         }
     }
@@ -762,8 +784,11 @@ __device__ __forceinline__ void mma_publish(MmaState<C>& st, float* cm, float* c
                 }
                 #pragma unroll
                 for (int md = 0; md < S::MD; ++md) {
-                    co[(w * gs + head) * C::D + md * 16 + gid] = st.o[nh][md][j];
-                    co[(w * gs + head) * C::D + md * 16 + gid + 8] = st.o[nh][md][2 + j];
+                    // fp8: logical rows gid, gid + 8 are dims 2 gid, 2 gid + 1
+                    const int d0 = S::FP8 ? md * 16 + 2 * gid : md * 16 + gid;
+                    const int d1 = S::FP8 ? d0 + 1 : d0 + 8;
+                    co[(w * gs + head) * C::D + d0] = st.o[nh][md][j];
+                    co[(w * gs + head) * C::D + d1] = st.o[nh][md][2 + j];
                 }
             }
         }
@@ -819,8 +844,8 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     __shared__ int s_issued;
     uint8_t* stages = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* vstage = stages + (size_t)C::STAGES * C::STAGE;         // C::NW * C::VSTG bytes
-    const uint32_t full0 = dev::smem_addr(vstage + (size_t)C::NW * C::VSTG);
+    uint8_t* after = stages + (size_t)C::STAGES * C::STAGE;          // barriers, merge area
+    const uint32_t full0 = dev::smem_addr(after);
     const uint32_t empty0 = full0 + 8 * C::STAGES;
 
     const int G = p.Hq / p.Hkv;
@@ -924,7 +949,7 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
         // a warp merge through a dedicated area (the stages keep streaming)
         // and write its record, exactly as nq one-partition CTAs would.
         const int gh = gc;
-        float* gm = reinterpret_cast<float*>(vstage + (size_t)C::NW * C::VSTG + 16 * C::STAGES);
+        float* gm = reinterpret_cast<float*>(after + 16 * C::STAGES);
         float* gl = gm + C::NW * gh;
         float* go = gl + C::NW * gh;
         if (warp == C::NW) {
@@ -950,8 +975,7 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                     uint8_t* kt = stages + (size_t)stg * C::STAGE;
                     const int nvalid = min(C::BS, n - (blk0 + j) * C::BS);
                     if constexpr (C::MMA)
-                        mma_block<C>(st, kt, kt + C::TILE, vstage + warp * C::VSTG, nvalid,
-                                     p.qk_scale);
+                        mma_block<C>(st, kt, kt + C::TILE, nvalid, p.qk_scale);
                     else simt_block<C>(st, kt, kt + C::TILE, nvalid);
                     __syncwarp();
                     if (lane == 0) dev::mbar_arrive(empty0 + 8 * stg);
@@ -1019,7 +1043,7 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
             uint8_t* kt = stages + (size_t)stg * C::STAGE;
             const int nvalid = min(C::BS, n - (blk0 + j) * C::BS);
             if constexpr (C::MMA)
-                mma_block<C>(st, kt, kt + C::TILE, vstage + warp * C::VSTG, nvalid, p.qk_scale);
+                mma_block<C>(st, kt, kt + C::TILE, nvalid, p.qk_scale);
             else simt_block<C>(st, kt, kt + C::TILE, nvalid);
             __syncwarp();
             if (lane == 0) dev::mbar_arrive(empty0 + 8 * stg);
@@ -1107,14 +1131,14 @@ struct PieceDesc {
 
 template <class C>
 struct BalancedSmem {
-    static constexpr int STAGES_RAW = (64 * 1024 - C::NW * C::VSTG) / C::STAGE;  // 3 CTAs per SM fit
+    static constexpr int STAGES_RAW = 64 * 1024 / C::STAGE;  // 3 CTAs per SM fit
     // a multiple of NW: each stage has a single consumer warp (see Cfg)
     static constexpr int STAGES_CLAMPED = STAGES_RAW < C::NW ? C::NW : (STAGES_RAW > 32 ? 32 : STAGES_RAW);
     static constexpr int STAGES = STAGES_CLAMPED / C::NW * C::NW;
     static_assert(STAGES % C::NW == 0, "each stage must have a single consumer warp");
     // the warp-merge area holds NW * gc * (D + 2) floats, gc = query heads per
     // item (known at launch); it follows the barriers
-    static constexpr size_t FIXED = 1024 + size_t(STAGES) * C::STAGE + size_t(C::NW) * C::VSTG +
+    static constexpr size_t FIXED = 1024 + size_t(STAGES) * C::STAGE +
                                     8 * (2 * STAGES + 2 * kItemQ + 2);
     static size_t bytes(int gc) { return FIXED + size_t(C::NW) * gc * (C::D + 2) * 4; }
 };
@@ -1187,14 +1211,14 @@ decode_balanced(const __grid_constant__ CUtensorMap tmk, const __grid_constant__
     __shared__ PieceDesc s_ring[kItemQ];
     uint8_t* stages = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* vstage = stages + (size_t)STAGES * C::STAGE;
-    const uint32_t full0 = dev::smem_addr(vstage + (size_t)C::NW * C::VSTG);
+    uint8_t* after = stages + (size_t)STAGES * C::STAGE;                  // barriers, merge area
+    const uint32_t full0 = dev::smem_addr(after);
     const uint32_t empty0 = full0 + 8 * STAGES;
     const uint32_t ifull0 = empty0 + 8 * STAGES;
     const uint32_t iempty0 = ifull0 + 8 * kItemQ;
     const uint32_t rdv_pub = iempty0 + 8 * kItemQ;     // consumers published their states
     const uint32_t rdv_done = rdv_pub + 8;              // consumers finished the combine
-    float* comb = reinterpret_cast<float*>(vstage + (size_t)C::NW * C::VSTG +
+    float* comb = reinterpret_cast<float*>(after +
                                            8 * (2 * STAGES + 2 * kItemQ + 2));
 
     const int G = p.Hq / p.Hkv;
@@ -1378,7 +1402,7 @@ decode_balanced(const __grid_constant__ CUtensorMap tmk, const __grid_constant__
                 uint8_t* kt = stages + (size_t)stg * C::STAGE;
                 const int nvalid = min(C::BS, d.n - (d.off + jj) * C::BS);
                 if constexpr (C::MMA)
-                    mma_block<C>(st, kt, kt + C::TILE, vstage + warp * C::VSTG, nvalid, p.qk_scale);
+                    mma_block<C>(st, kt, kt + C::TILE, nvalid, p.qk_scale);
                 else simt_block<C>(st, kt, kt + C::TILE, nvalid);
                 __syncwarp();
                 if (lane == 0) dev::mbar_arrive(empty0 + 8 * stg);

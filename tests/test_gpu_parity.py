@@ -119,7 +119,9 @@ SHAPES = [(bs, G, D, dt) for bs in (8, 16, 32) for G in (1, 2, 4, 8) for D in (6
           for dt in ("bf16", "f16")] + [(16, 4, 256, "bf16"), (32, 2, 256, "f16"),
                                           (16, 2, 64, "f32"), (8, 4, 128, "fp8_e4m3"),
                                           (32, 8, 256, "fp8_e4m3"), (16, 16, 128, "bf16"),
-                                          (8, 16, 64, "f16")]
+                                          (8, 16, 64, "f16"), (16, 8, 128, "fp8_e4m3"),
+                                          (32, 2, 128, "fp8_e4m3"), (16, 16, 128, "fp8_e4m3"),
+                                          (8, 16, 128, "fp8_e4m3")]
 
 
 @pytest.mark.parametrize("bs,G,D,dt", SHAPES)
