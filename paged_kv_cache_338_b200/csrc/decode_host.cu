@@ -286,6 +286,11 @@ pa_status pa::decode_impl(void* out, const void* q, pa_dtype q_dt, const void* k
     // (sequence, kv head) items back to back, each CTA a contiguous run of
     // whole items of about equal work (one CTA per item with bit 16)
     const bool items = fuse && !(sel & 16);
+    // 8-token blocks go two to a stage (16 tokens) in the partition kernel,
+    // where partitions are whole stages
+    const bool pair = bs == 8 && !balanced && !fuse && prefix_parts == 0 && !force_ws &&
+                      partition % 16 == 0;
+    const int stage_tokens = pair ? 16 : bs;
     int part_group = 1;
     if (use_mma && !balanced && !fuse && prefix_parts == 0 && !force_ws && max_parts > 1)
         part_group = (sel & 8) ? 3
@@ -323,7 +328,7 @@ pa_status pa::decode_impl(void* out, const void* q, pa_dtype q_dt, const void* k
     p.Hkv = Hkv;
     p.MB = MB;
     p.max_parts = (int)max_parts;
-    p.part_blocks = !fuse && (max_parts > 1 || force_ws) ? partition / bs : 0;
+    p.part_blocks = !fuse && (max_parts > 1 || force_ws) ? partition / stage_tokens : 0;
     p.part_tokens = !fuse && (max_parts > 1 || force_ws) ? partition : 0;
     p.prefix_parts = prefix_parts;
     p.force_ws = force_ws ? 1 : 0;
@@ -355,6 +360,7 @@ pa_status pa::decode_impl(void* out, const void* q, pa_dtype q_dt, const void* k
     }
 
     L.bs = bs;
+    L.pair = pair;
     L.D = D;
     L.mma = use_mma;
     L.mrows = G <= 8 ? 8 : 16;

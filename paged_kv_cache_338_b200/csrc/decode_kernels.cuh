@@ -105,9 +105,15 @@ __device__ __forceinline__ int checked_len(const Params& p, int s, int bs) {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-template <int DT_, int QT_, int BS_, int D_, int GC_, bool MMA_, int MROWS_ = 8>
+// BS is the tokens of one stage; PB the tokens of one physical cache block.
+// A stage holds PER = BS / PB consecutive blocks of a sequence (two blocks of
+// 8 tokens make a 16-token stage, so an 8-token cache pays the per-stage
+// costs -- barrier round trips, softmax updates, half-empty MMA tiles -- once
+// per 16 tokens).
+template <int DT_, int QT_, int BS_, int D_, int GC_, bool MMA_, int MROWS_ = 8, int PB_ = BS_>
 struct Cfg {
     static constexpr int DT = DT_, QT = QT_, BS = BS_, D = D_, GC = GC_, MROWS = MROWS_;
+    static constexpr int PB = PB_, PER = BS_ / PB_;
     static constexpr bool MMA = MMA_;
     static constexpr int E = dev::Storage<DT>::bytes;
     static constexpr int R = D * E;          // bytes of one token row of one kv head
@@ -139,6 +145,7 @@ struct Cfg {
     static constexpr size_t SMEM = 1024 /*align slack*/ + size_t(STAGES) * STAGE + 2 * 8 * STAGES;
     static_assert(R == 128 || R == 256 || R == 512, "row bytes must be 128, 256 or 512");
     static_assert(BS == 8 || BS == 16 || BS == 32, "block size");
+    static_assert(PER == 1 || (PER == 2 && PB == 8), "a stage holds one block, or two of 8 tokens");
     static_assert(STAGES % NW == 0, "each stage must have a single consumer warp");
     static_assert(COMBINE_FLOATS * 4 <= STAGES * STAGE, "combine area must fit in the stages");
     static_assert(SMEM <= 227 * 1024, "shared memory");
@@ -157,21 +164,40 @@ __device__ __forceinline__ uint32_t tile_off(int t, int seg, int chunk) {
 // One warp; lane 0 issues.  Block ids are fetched 32 at a time (one per lane)
 // and handed to lane 0 with a shuffle, so the issue loop never waits on a
 // dependent global load.
+//
+// A lane's id of the first 32 blocks can be loaded ahead of time (while the
+// CTA still reads its context length and sets up its barriers):
+// table_entry_ahead() loads it for a guessed first physical block, and
+// produce() uses it when the guess was right (pre_pblk0 == blk0 * PER).
+__device__ __forceinline__ int table_entry_ahead(const Params& p, int s, int pblk0_guess) {
+    const int i = pblk0_guess + (threadIdx.x & 31);
+    return (pblk0_guess >= 0 && i < p.MB) ? __ldg(p.block_tables + (size_t)s * p.MB + i) : 0;
+}
+
 template <class C>
 __device__ __forceinline__ void produce(const CUtensorMap* tmk, const CUtensorMap* tmv,
                                         const Params& p, const int32_t* bt_row, int blk0, int nblk,
-                                        int kvh, uint8_t* stages, uint32_t full0, uint32_t empty0,
-                                        volatile int* s_abort, int* k_io) {
-    // Streams blocks [blk0, blk0 + nblk) of one (sequence, kv head) through the
-    // stage ring; *k_io is the CTA's running block counter (stage = k % STAGES).
+                                        int nphys, int kvh, uint8_t* stages, uint32_t full0,
+                                        uint32_t empty0, volatile int* s_abort, int* k_io,
+                                        int pre_pblk0 = -1, int pre = 0) {
+    // Streams stages [blk0, blk0 + nblk) of one (sequence, kv head) through the
+    // stage ring; *k_io is the CTA's running stage counter (slot = k % STAGES).
+    // Stage j holds physical blocks (blk0 + j) * PER + r, r < PER, of which the
+    // first nphys (counted from blk0 * PER) exist; a stage past them is left
+    // part-filled (its tokens are past the sequence's length).
     const int lane = threadIdx.x & 31;
     const uint64_t pol = p.evict_first ? dev::policy_evict_first() : dev::policy_evict_normal();
+    const int pblk0 = blk0 * C::PER;
     int k = *k_io;
-    for (int jb = 0; jb < nblk; jb += 32) {
-        const int mine = (jb + lane < nblk) ? __ldg(bt_row + blk0 + jb + lane) : 0;
-        const int cnt = min(32, nblk - jb);
+    for (int jb = 0; jb < nblk * C::PER; jb += 32) {          // 32 physical ids per round
+        const int mine = jb + lane >= nphys ? 0
+                         : (jb == 0 && pre_pblk0 == pblk0) ? pre
+                                                           : __ldg(bt_row + pblk0 + jb + lane);
+        const int cnt = min(32, nblk * C::PER - jb) / C::PER;   // stages of this round
         for (int jj = 0; jj < cnt; ++jj) {
-            const int id = __shfl_sync(0xffffffffu, mine, jj);
+            int id[C::PER];
+            #pragma unroll
+            for (int r = 0; r < C::PER; ++r) id[r] = __shfl_sync(0xffffffffu, mine, jj * C::PER + r);
             int stop = 0;
             if (lane == 0) {
                 const int st = k % C::STAGES;
@@ -184,15 +210,22 @@ __device__ __forceinline__ void produce(const CUtensorMap* tmk, const CUtensorMa
                     }
                 }
                 if (!stop) {
-                    if (id < 0 || (int64_t)id >= p.NB) dev::raise_error(p.err, PA_DEV_BAD_BLOCK);
+                    const int have = min(C::PER, nphys - (jb + jj * C::PER));   // >= 1
                     const uint32_t bar = full0 + 8 * st;
                     const uint32_t dk = dev::smem_addr(stages + (size_t)st * C::STAGE);
-                    dev::mbar_arrive_expect_tx(bar, C::STAGE);
+                    dev::mbar_arrive_expect_tx(bar, (uint32_t)have * 2 * C::PB * C::R);
                     #pragma unroll
-                    for (int c = 0; c < C::CH; ++c) {
-                        dev::tma_load_4d(dk + c * C::BS * 128, tmk, bar, c * C::EPS, kvh, 0, id, pol);
-                        dev::tma_load_4d(dk + C::TILE + c * C::BS * 128, tmv, bar, c * C::EPS, kvh,
-                                         0, id, pol);
+                    for (int r = 0; r < C::PER; ++r) {
+                        if (r >= have) break;
+                        if (id[r] < 0 || (int64_t)id[r] >= p.NB)
+                            dev::raise_error(p.err, PA_DEV_BAD_BLOCK);
+                        #pragma unroll
+                        for (int c = 0; c < C::CH; ++c) {
+                            const uint32_t off = c * C::BS * 128 + r * C::PB * 128;
+                            dev::tma_load_4d(dk + off, tmk, bar, c * C::EPS, kvh, 0, id[r], pol);
+                            dev::tma_load_4d(dk + C::TILE + off, tmv, bar, c * C::EPS, kvh, 0,
+                                             id[r], pol);
+                        }
                     }
                 }
             }
@@ -824,6 +857,39 @@ __device__ __forceinline__ bool consumers_sync_or(bool pred) {
     return r != 0;
 }
 
+// Fold the prefix_parts prefix records of (sequence s, head h) into a state
+// (M in log2 units, L, O already times v_scale) and return the output value.
+// The records are loaded first, so their latencies overlap.
+__device__ __forceinline__ float fold_prefix_records(const Params& p, int s, int h, int d,
+                                                     float M, float L, float O, int D) {
+    constexpr int kMaxUnrolled = 8;
+    const size_t row0 = ((size_t)s * p.Hq + h) * p.max_parts;
+    for (int pp = 0; pp < p.prefix_parts; pp += kMaxUnrolled) {
+        float2 ml[kMaxUnrolled];
+        float o[kMaxUnrolled];
+        #pragma unroll
+        for (int i = 0; i < kMaxUnrolled; ++i) {
+            if (pp + i < p.prefix_parts) {
+                ml[i] = p.ws_ml[row0 + pp + i];
+                o[i] = p.ws_o[(row0 + pp + i) * D + d];
+            } else {
+                ml[i] = make_float2(-INFINITY, 0.f);
+                o[i] = 0.f;
+            }
+        }
+        #pragma unroll
+        for (int i = 0; i < kMaxUnrolled; ++i) {
+            const float Mn = fmaxf(M, ml[i].x);
+            if (Mn == -INFINITY) continue;
+            const float a = exp2f(M - Mn), b = exp2f(ml[i].x - Mn);
+            L = L * a + ml[i].y * b;
+            O = O * a + o[i] * b;
+            M = Mn;
+        }
+    }
+    return L > 0.f ? O / L : 0.f;
+}
+
 // Smem bytes of the per-partition warp merge area of the grouped-partition
 // mode (it cannot reuse the stages, which keep streaming).
 template <class C>
@@ -838,7 +904,12 @@ template <class C, bool GROUPED>
 __global__ void __launch_bounds__(C::THREADS, C::MMA ? 3 : 2)
 decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                  const Params p) {
-    dev::grid_dependency_wait();       // launched as a dependent of the kernel before it
+    // Launched as a dependent of the kernel before it.  The shared-prefix
+    // suffix pass reads nothing that kernel (the prefix kernel) writes until it
+    // folds the prefix records in, so it waits there and streams its suffix
+    // meanwhile; everything the kernels before that one wrote was complete
+    // when the prefix kernel started (an ordinary launch).
+    if (p.fuse_prefix_blocks == 0) dev::grid_dependency_wait();
     extern __shared__ uint8_t smem_raw[];
     __shared__ int s_abort;
     __shared__ int s_issued;
@@ -856,7 +927,14 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     const int kvh = hc / chunks;
     const int h0 = kvh * G + (hc % chunks) * gc;
     const int s = blockIdx.z;
-    const int n = checked_len(p, s, C::BS);
+    // the producer's first 32 block ids, for the first block this CTA most
+    // likely reads, fetched beside the context length
+    const int pblk0_guess = p.fuse_prefix_blocks > 0 ? p.fuse_prefix_blocks
+                            : p.prefix_parts > 0     ? -1
+                                                     : part * p.part_group * p.part_blocks * C::PER;
+    const int pre = (threadIdx.x >> 5) == C::NW ? table_entry_ahead(p, s, pblk0_guess) : 0;
+    const int n = checked_len(p, s, C::PB);
+    const int nphys_all = (n + C::PB - 1) / C::PB;
     const int nblk_all = (n + C::BS - 1) / C::BS;
     int blk0 = 0, nblk = nblk_all, nparts = 1;
     int q0 = part, nq = 1;                      // partitions (records) this CTA writes
@@ -954,8 +1032,9 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
         float* go = gl + C::NW * gh;
         if (warp == C::NW) {
             int k = 0;
-            produce<C>(&tmk, &tmv, p, p.block_tables + (size_t)s * p.MB, blk0, nblk, kvh, stages,
-                       full0, empty0, &s_abort, &k);
+            produce<C>(&tmk, &tmv, p, p.block_tables + (size_t)s * p.MB, blk0, nblk,
+                       min(nblk * C::PER, nphys_all - blk0 * C::PER), kvh, stages, full0, empty0,
+                       &s_abort, &k, pblk0_guess, pre);
             if (lane == 0) s_issued = k;
         } else {
             if constexpr (C::MMA) mma_load_q<C>(st, p, s, h0, G);
@@ -1028,8 +1107,9 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     }
     if (warp == C::NW) {
         int k = 0;
-        produce<C>(&tmk, &tmv, p, p.block_tables + (size_t)s * p.MB, blk0, nblk, kvh, stages,
-                   full0, empty0, &s_abort, &k);
+        produce<C>(&tmk, &tmv, p, p.block_tables + (size_t)s * p.MB, blk0, nblk,
+                   min(nblk * C::PER, nphys_all - blk0 * C::PER), kvh, stages, full0, empty0,
+                   &s_abort, &k, pblk0_guess, pre);
         if (lane == 0) s_issued = k;
     } else {
         if constexpr (C::MMA) mma_load_q<C>(st, p, s, h0, G);
@@ -1066,6 +1146,7 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
         if constexpr (C::MMA) mma_publish<C>(st, cm, cl, co, warp, G);
         else simt_publish<C>(st, cm, cl, co, warp);
     }
+    if (p.fuse_prefix_blocks > 0) dev::grid_dependency_wait();   // the prefix records are written
     __syncthreads();
 
     // ---- merge the warps' states and write -----------------------------
@@ -1086,19 +1167,8 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
         const int h = h0 + g;
         if (fuse_records) {
             // combine with the prefix records (o already times v_scale there)
-            O *= p.v_scale;
-            for (int pp = 0; pp < p.prefix_parts; ++pp) {
-                const size_t row = ((size_t)s * p.Hq + h) * p.max_parts + pp;
-                const float2 ml = p.ws_ml[row];
-                const float Mn = fmaxf(M, ml.x);
-                if (Mn == -INFINITY) continue;
-                const float a = exp2f(M - Mn), b = exp2f(ml.x - Mn);
-                L = L * a + ml.y * b;
-                O = O * a + p.ws_o[row * C::D + d] * b;
-                M = Mn;
-            }
             dev::store_out<C::QT>(p.out, ((size_t)s * p.Hq + h) * C::D + d,
-                                  L > 0.f ? O / L : 0.f);
+                                  fold_prefix_records(p, s, h, d, M, L, O * p.v_scale, C::D));
         } else if (nparts == 1 && !p.force_ws) {
             dev::store_out<C::QT>(p.out, ((size_t)s * p.Hq + h) * C::D + d,
                                   L > 0.f ? (O / L) * p.v_scale : 0.f);
@@ -1158,38 +1228,6 @@ __device__ __forceinline__ int blocks_of(const Params& p, int s) {
     return (pb > 0 && n >= pb * C::BS ? nb - pb : nb) + 1;
 }
 
-// Fold the prefix_parts prefix records of (sequence s, head h) into a state
-// (M in log2 units, L, O already times v_scale) and return the output value.
-// The records are loaded first, so their latencies overlap.
-__device__ __forceinline__ float fold_prefix_records(const Params& p, int s, int h, int d,
-                                                     float M, float L, float O, int D) {
-    constexpr int kMaxUnrolled = 8;
-    const size_t row0 = ((size_t)s * p.Hq + h) * p.max_parts;
-    for (int pp = 0; pp < p.prefix_parts; pp += kMaxUnrolled) {
-        float2 ml[kMaxUnrolled];
-        float o[kMaxUnrolled];
-        #pragma unroll
-        for (int i = 0; i < kMaxUnrolled; ++i) {
-            if (pp + i < p.prefix_parts) {
-                ml[i] = p.ws_ml[row0 + pp + i];
-                o[i] = p.ws_o[(row0 + pp + i) * D + d];
-            } else {
-                ml[i] = make_float2(-INFINITY, 0.f);
-                o[i] = 0.f;
-            }
-        }
-        #pragma unroll
-        for (int i = 0; i < kMaxUnrolled; ++i) {
-            const float Mn = fmaxf(M, ml[i].x);
-            if (Mn == -INFINITY) continue;
-            const float a = exp2f(M - Mn), b = exp2f(ml[i].x - Mn);
-            L = L * a + ml[i].y * b;
-            O = O * a + o[i] * b;
-            M = Mn;
-        }
-    }
-    return L > 0.f ? O / L : 0.f;
-}
 
 // The configuration of the balanced kernel: the same tile shapes, a deeper ring.
 template <class C>
@@ -1226,10 +1264,21 @@ decode_balanced(const __grid_constant__ CUtensorMap tmk, const __grid_constant__
     const int chunks = G / gc;
     const int HC = p.Hkv * chunks;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // Whole items are striped by head: the grid is HC CTAs per group, group g
+    // takes a contiguous run of sequences of about equal total work and CTA
+    // (g, hc) serves head hc of each.  The heads of a sequence have the same
+    // length, so a group's CTAs keep pace and read each block's head rows
+    // (neighbours in memory) at about the same time.  The split mode spreads
+    // (sequence, head) items over single CTAs.
+    const bool whole = p.whole_items != 0;
+    const int span = whole ? 1 : HC;                    // items per sequence in the space
+    const long long units = whole ? (long long)(gridDim.x / HC) : (long long)gridDim.x;
+    const long long unit = whole ? (long long)(blockIdx.x / HC) : (long long)blockIdx.x;
+    const int my_hc = whole ? (int)(blockIdx.x % HC) : 0;
 
     // ---- W and this CTA's block range --------------------------------------
     long long acc = 0;
-    for (int s = threadIdx.x; s < p.S; s += C::THREADS) acc += (long long)blocks_of<C>(p, s) * HC;
+    for (int s = threadIdx.x; s < p.S; s += C::THREADS) acc += (long long)blocks_of<C>(p, s) * span;
     #pragma unroll
     for (int x = 16; x > 0; x >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, x);
     if (lane == 0) s_red[warp] = acc;
@@ -1238,18 +1287,18 @@ decode_balanced(const __grid_constant__ CUtensorMap tmk, const __grid_constant__
     long long W = 0;
     #pragma unroll
     for (int w = 0; w <= C::NW; ++w) W += s_red[w];
-    // With fewer blocks than CTAs only the first W CTAs work, so every working
-    // CTA's share is non-empty and an item's pieces sit on consecutive CTAs.
-    const long long nctas = W < (long long)gridDim.x ? W : (long long)gridDim.x;
-    if ((long long)blockIdx.x >= nctas) return;         // CTA-uniform: no work
-    const long long b0 = (long long)blockIdx.x * W / nctas;
-    const long long b1 = ((long long)blockIdx.x + 1) * W / nctas;
+    // With fewer blocks than CTAs (groups) only the first W work, so every
+    // working share is non-empty and an item's pieces sit on consecutive CTAs.
+    const long long nctas = W < units ? W : units;
+    if (unit >= nctas) return;                          // CTA-uniform: no work
+    const long long b0 = unit * W / nctas;
+    const long long b1 = (unit + 1) * W / nctas;
     __syncthreads();                                    // s_red is reused below
     long long R = 0;
     for (int base = 0; base < p.S; base += C::THREADS) {
         const int s = base + threadIdx.x;
         const int nb = s < p.S ? blocks_of<C>(p, s) : 0;
-        const long long v = (long long)nb * HC;
+        const long long v = (long long)nb * span;
         long long inc = v;
         #pragma unroll
         for (int x = 1; x < 32; x <<= 1) {
@@ -1321,13 +1370,15 @@ decode_balanced(const __grid_constant__ CUtensorMap tmk, const __grid_constant__
             }
             return __shfl_sync(0xffffffffu, bad, 0) != 0;
         };
-        if (p.whole_items) {
-            // Whole items: this CTA takes the items that start inside
-            // [b0, b1); the item holding b0 is its own only if it starts there.
+        if (whole) {
+            // Whole items: this CTA takes head my_hc of the sequences that
+            // start inside [b0, b1); the sequence holding b0 is its group's
+            // only if it starts there.
+            hc = my_hc;
             b -= off;
             if (!stop && off > 0) {
                 b += blocks_of<C>(p, s);
-                if (++hc == HC) { hc = 0; ++s; }
+                ++s;
             }
             const int pb = p.fuse_prefix_blocks;
             int reg_s = -1, reg = 0;                   // regularity of sequence reg_s
@@ -1346,11 +1397,11 @@ decode_balanced(const __grid_constant__ CUtensorMap tmk, const __grid_constant__
                 PieceDesc d{s, hc, blk0, nb - blk0, nb, n, k, 0, blk0 > 0};
                 if (publish(d)) break;
                 produce<C>(&tmk, &tmv, p, p.block_tables + (size_t)s * p.MB, blk0, nb - blk0,
-                            hc / chunks, stages, full0, empty0, &s_abort, &k);
+                            nb - blk0, hc / chunks, stages, full0, empty0, &s_abort, &k);
                 if (*(volatile int*)&s_abort) break;
                 b += blocks_of<C>(p, s);
                 ++ci;
-                if (++hc == HC) { hc = 0; ++s; }
+                ++s;
             }
         } else {
             while (!stop && b < b1 && s < p.S) {
@@ -1361,7 +1412,7 @@ decode_balanced(const __grid_constant__ CUtensorMap tmk, const __grid_constant__
                     PieceDesc d{s, hc, off, take, nb, n, k, 0, 0};
                     if (publish(d)) break;
                     produce<C>(&tmk, &tmv, p, p.block_tables + (size_t)s * p.MB, off, take,
-                                hc / chunks, stages, full0, empty0, &s_abort, &k);
+                                take, hc / chunks, stages, full0, empty0, &s_abort, &k);
                     if (*(volatile int*)&s_abort) break;
                     b += take;
                     ++ci;

@@ -14,6 +14,7 @@ struct Launch {
     CUtensorMap tmk, tmv;
     Params p;
     int bs, D;
+    bool pair;     // two 8-token blocks per 16-token stage
     int gc;        // SIMT: query heads per CTA
     bool mma;      // tensor-core consumer
     int mrows;     // MMA: 8 or 16 query rows
@@ -35,7 +36,9 @@ cudaError_t launch_fp8_q_bf16(const Launch& L);
 
 template <class C>
 cudaError_t launch_one(const Launch& L) {
-    if (L.balanced) {
+    if constexpr (C::PER != 1) {
+        if (L.balanced) return cudaErrorNotSupported;   // the host pairs blocks for partitions only
+    } else if (L.balanced) {
         auto kern = decode_balanced<C>;
         const int smem = static_cast<int>(BalancedSmem<C>::bytes(L.mma ? L.G : L.gc));
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -46,6 +49,11 @@ cudaError_t launch_one(const Launch& L) {
         if (per_sm < 1) per_sm = 1;
         int ctas = per_sm * L.num_sms;
         if (ctas > kMaxBalancedCtas) ctas = kMaxBalancedCtas;
+        if (L.p.whole_items) {
+            // whole items: groups of one CTA per (kv head, head chunk)
+            const int hc = L.p.Hkv * (C::MMA ? 1 : L.G / C::GC);
+            ctas = ctas >= hc ? ctas / hc * hc : hc;
+        }
         return dev::launch_pdl(kern, dim3((unsigned)ctas), dim3(C::THREADS), (size_t)smem,
                                L.stream, L.tmk, L.tmv, L.p);
     }
@@ -89,7 +97,8 @@ constexpr bool row_ok() {
            D * dev::Storage<DT>::bytes == 512;
 }
 
-template <int DT, int QT, int BS, int D>
+// BS: tokens per stage; PB: tokens per physical block (BS / PB blocks a stage)
+template <int DT, int QT, int BS, int D, int PB>
 cudaError_t launch_by_heads(const Launch& L) {
     if constexpr (!row_ok<DT, D>()) {
         return cudaErrorNotSupported;
@@ -97,29 +106,29 @@ cudaError_t launch_by_heads(const Launch& L) {
         if (L.mma) {
             if constexpr (((DT == QT && (DT == PA_F16 || DT == PA_BF16)) || DT == PA_FP8_E4M3) &&
                           D <= 128) {
-                if (L.mrows == 8) return launch_one<Cfg<DT, QT, BS, D, 8, true, 8>>(L);
-                return launch_one<Cfg<DT, QT, BS, D, 16, true, 16>>(L);
+                if (L.mrows == 8) return launch_one<Cfg<DT, QT, BS, D, 8, true, 8, PB>>(L);
+                return launch_one<Cfg<DT, QT, BS, D, 16, true, 16, PB>>(L);
             } else {
                 return cudaErrorNotSupported;
             }
         }
         switch (L.gc) {
-        case 1: return launch_one<Cfg<DT, QT, BS, D, 1, false>>(L);
-        case 2: return launch_one<Cfg<DT, QT, BS, D, 2, false>>(L);
+        case 1: return launch_one<Cfg<DT, QT, BS, D, 1, false, 8, PB>>(L);
+        case 2: return launch_one<Cfg<DT, QT, BS, D, 2, false, 8, PB>>(L);
         case 4:
-            if constexpr (D <= 128) return launch_one<Cfg<DT, QT, BS, D, 4, false>>(L);
+            if constexpr (D <= 128) return launch_one<Cfg<DT, QT, BS, D, 4, false, 8, PB>>(L);
             else return cudaErrorNotSupported;
         }
         return cudaErrorNotSupported;
     }
 }
 
-template <int DT, int QT, int BS>
+template <int DT, int QT, int BS, int PB>
 cudaError_t launch_by_dim(const Launch& L) {
     switch (L.D) {
-    case 64: return launch_by_heads<DT, QT, BS, 64>(L);
-    case 128: return launch_by_heads<DT, QT, BS, 128>(L);
-    case 256: return launch_by_heads<DT, QT, BS, 256>(L);
+    case 64: return launch_by_heads<DT, QT, BS, 64, PB>(L);
+    case 128: return launch_by_heads<DT, QT, BS, 128, PB>(L);
+    case 256: return launch_by_heads<DT, QT, BS, 256, PB>(L);
     }
     return cudaErrorNotSupported;
 }
@@ -127,9 +136,9 @@ cudaError_t launch_by_dim(const Launch& L) {
 template <int DT, int QT>
 cudaError_t launch_dtype(const Launch& L) {
     switch (L.bs) {
-    case 8: return launch_by_dim<DT, QT, 8>(L);
-    case 16: return launch_by_dim<DT, QT, 16>(L);
-    case 32: return launch_by_dim<DT, QT, 32>(L);
+    case 8: return L.pair ? launch_by_dim<DT, QT, 16, 8>(L) : launch_by_dim<DT, QT, 8, 8>(L);
+    case 16: return launch_by_dim<DT, QT, 16, 16>(L);
+    case 32: return launch_by_dim<DT, QT, 32, 32>(L);
     }
     return cudaErrorNotSupported;
 }

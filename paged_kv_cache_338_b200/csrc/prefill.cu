@@ -330,6 +330,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                const __grid_constant__ CUtensorMap tmv, const Params p) {
     using L = Smem<D>;
     constexpr int NSEG = L::NSEG, ST = L::ST;
+    // Prefix mode: the suffix decode launched next reads the records only at
+    // its very end (after its own griddepcontrol.wait), so let its CTAs start
+    // on the SMs this grid leaves free.
+    if (p.prefix) launch_dependents();
     // grid (kPairGroup tile pairs x kv heads, sequences | prefix chunks, pair
     // groups): a group of adjacent tile pairs of one (sequence, kv head) runs
     // side by side and shares its K/V through L2, while groups run longest

@@ -10,6 +10,8 @@ pa_decode_shared_prefix for the shared-prefix workload -- and compares sampled
 sequences (the first, the last, the longest and two drawn at random) with the
 fp64 oracle's own copy, append and attention.  Bars as in test_gpu_parity.
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -21,8 +23,10 @@ import workloads as wl
 pytestmark = pytest.mark.gpu
 
 TOL = {"f32": 1e-5, "f16": 2e-3, "bf16": 1e-2, "fp8_e4m3": 3e-2}
-FULL = ["llama2_7b_mha_fp16_b64", "llama3_8b_gqa_bf16_b128",
-        "long_context_splitk_bf16_4x100k", "prefix_shared_fp8_b256"]
+FULL = [("llama2_7b_mha_fp16_b64", 0), ("llama3_8b_gqa_bf16_b128", 0),
+        ("long_context_splitk_bf16_4x100k", 0), ("prefix_shared_fp8_b256", 0),
+        # the Llama-3-8B shape at the other block sizes (bench.py --block-size)
+        ("llama3_8b_gqa_bf16_b128", 8), ("llama3_8b_gqa_bf16_b128", 32)]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -50,9 +54,11 @@ def _oracle(inp: wl.DecodeInputs, seqs):
                                inp.context_lens, inp.scale, inp.k_scale, inp.v_scale, seqs=seqs)
 
 
-@pytest.mark.parametrize("name", FULL)
-def test_full_size_sampled(name):
+@pytest.mark.parametrize("name,bs", FULL, ids=[f"{n}_bs{b}" if b else n for n, b in FULL])
+def test_full_size_sampled(name, bs):
     cfg = wl.DECODE_WORKLOADS[name]
+    if bs:
+        cfg = dataclasses.replace(cfg, block_size=bs, name=f"{name}_bs{bs}")
     inp = wl.make_decode_inputs(cfg, seed=2)
     S, Hq, D = inp.q.shape
     lens = inp.context_lens

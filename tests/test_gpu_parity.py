@@ -131,18 +131,21 @@ def test_decode_shapes(bs, G, D, dt):
                           3 * bs + 1, fp8_scaled=dt == "fp8_e4m3")
     inp = wl.make_decode_inputs(cfg, seed=bs * 1000 + G * 10 + D)
     want, _, _ = oracle_step(inp)
-    for part in (0, bs, -1):
-        for mode in BOTH:
+    # at block 8, partitions of whole 16-token stages read two blocks a stage
+    modes = BOTH + ([pa.DECODE_DEFAULT | pa.DECODE_GROUP_PARTITIONS] if bs == 8 else [])
+    for part in (0, bs, 2 * bs, -1):
+        for mode in modes:
             out, _, _ = gpu_step(inp, part, mode)
             _check_out(out, want, dt, f"P={part} mode={mode}")
     assert pa.pa_device_status() == 0
 
 
+@pytest.mark.parametrize("bs", [16, 8])
 @pytest.mark.parametrize("dt", ["bf16", "fp8_e4m3"])
-def test_lengths_at_partition_edges(dt):
+def test_lengths_at_partition_edges(dt, bs):
     P = 64
     lens = (1, P - 1, P, P + 1, 2 * P - 1, 2 * P, 2 * P + 1, 5 * P + 3)
-    cfg = wl.DecodeConfig("edges", len(lens), 8, 2, 128, 16, dt, "bf16", 0, 0,
+    cfg = wl.DecodeConfig("edges", len(lens), 8, 2, 128, bs, dt, "bf16", 0, 0,
                           fixed_lens=lens, fp8_scaled=dt == "fp8_e4m3")
     inp = wl.make_decode_inputs(cfg, seed=7)
     want, _, _ = oracle_step(inp)
