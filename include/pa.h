@@ -265,10 +265,11 @@ pa_status pa_decode_partition_group(int S, int Hq, int Hkv, int D, int bs, pa_dt
  *      Each partition still gets its own record, so the result is the same.
  *      Tensor-core consumer only, and only where the CTA's extra merge area
  *      costs no resident CTA per SM.
- *  16: pa_decode_shared_prefix with suffixes of at most 4096 tokens: one CTA
- *      per (sequence, kv head) suffix, instead of the default persistent grid
- *      in which each CTA streams a contiguous run of whole (sequence, kv head)
- *      suffixes of about equal total length without draining its pipeline.
+ *  16: pa_decode_shared_prefix with suffixes of at most 4096 tokens: a
+ *      persistent grid in groups of one CTA per kv head, each group streaming
+ *      a run of whole sequences' suffixes of about equal total length without
+ *      draining its pipeline, instead of the default one CTA per (sequence,
+ *      kv head) suffix.
  * Default 4.  Every setting computes the same function.
  */
 pa_status pa_decode_select(int mode);

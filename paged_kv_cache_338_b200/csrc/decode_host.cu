@@ -19,8 +19,8 @@ namespace {
 // hint on K/V loads, 4 = partition-major grid (kv heads of a partition side
 // by side), 8 = group split-K partitions three to a CTA whenever there are
 // several (a test hook for the grouped path at small sizes), 16 = shared-prefix
-// decode with one CTA per (sequence, kv head) suffix instead of the persistent
-// whole-item grid; the default is 4.
+// decode with the persistent whole-item grid for the suffixes instead of one
+// CTA per (sequence, kv head) suffix; the default is 4.
 std::atomic<int> g_select{4};
 
 // Plain split-K with short partitions: one CTA streams g consecutive
@@ -282,10 +282,10 @@ pa_status pa::decode_impl(void* out, const void* q, pa_dtype q_dt, const void* k
     const int gc = use_mma ? G : gc_simt;
     const int chunks = use_mma ? 1 : G / gc_simt;
     const int num_sms = sm_count();
-    // shared-prefix decode with whole suffixes: a persistent grid streams the
-    // (sequence, kv head) items back to back, each CTA a contiguous run of
-    // whole items of about equal work (one CTA per item with bit 16)
-    const bool items = fuse && !(sel & 16);
+    // shared-prefix decode with whole suffixes: one CTA per (sequence, kv
+    // head) item, or with bit 16 a persistent grid that streams the items back
+    // to back, each CTA a run of whole items of about equal work
+    const bool items = fuse && (sel & 16);
     // 8-token blocks go two to a stage (16 tokens) in the partition kernel,
     // where partitions are whole stages
     const bool pair = bs == 8 && !balanced && !fuse && prefix_parts == 0 && !force_ws &&

@@ -944,10 +944,10 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
         // holds the whole prefix) reads only its suffix here and merges the
         // prefix kernel's records in the epilogue; any other reads everything.
         const int pb = p.fuse_prefix_blocks;
-        int irregular = n < pb * C::BS;
-        for (int i = threadIdx.x; i < pb && !irregular; i += blockDim.x)
-            irregular = p.block_tables[(size_t)s * p.MB + i] != p.block_tables[i];
-        irregular = __syncthreads_or(irregular);
+        int irregular = 0;                      // the table loads do not wait for n
+        for (int i = threadIdx.x; i < pb; i += blockDim.x)
+            irregular |= p.block_tables[(size_t)s * p.MB + i] != p.block_tables[i];
+        irregular = __syncthreads_or(irregular || n < pb * C::BS);
         if (!irregular) {
             blk0 = pb;
             nblk = nblk_all - pb;               // may be 0: the prefix alone

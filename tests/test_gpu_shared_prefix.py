@@ -8,11 +8,11 @@ whose table does not start with row 0's prefix blocks (its own prefix has other
 values: a wrong fall-back shows up as an error), a sequence shorter than the
 prefix and one that holds exactly the prefix.  Tolerances are the decode bars.
 
-Short suffixes are decoded two ways, both checked: the default persistent grid
-(each CTA streams a contiguous run of whole (sequence, kv head) suffixes and
-folds the prefix records into each) and one CTA per suffix
-(DECODE_SUFFIX_PER_CTA).  A batch of many short suffixes puts several items
-on every CTA of the persistent grid.
+Short suffixes are decoded two ways, both checked: one CTA per (sequence, kv
+head) suffix (the default) and the persistent grid (DECODE_SUFFIX_PERSISTENT:
+groups of one CTA per kv head, each group streaming a run of whole sequences'
+suffixes and folding the prefix records into each).  A batch of many short
+suffixes puts several items on every CTA of the persistent grid.
 """
 import dataclasses
 
@@ -37,8 +37,8 @@ def _cuda():
     yield
 
 
-MODES = {"persistent": pa.DECODE_DEFAULT,
-         "per_cta": pa.DECODE_DEFAULT | pa.DECODE_SUFFIX_PER_CTA}
+MODES = {"per_cta": pa.DECODE_DEFAULT,
+         "persistent": pa.DECODE_DEFAULT | pa.DECODE_SUFFIX_PERSISTENT}
 
 
 @pytest.fixture(params=sorted(MODES))
