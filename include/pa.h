@@ -270,6 +270,12 @@ pa_status pa_decode_partition_group(int S, int Hq, int Hkv, int D, int bs, pa_dt
  *      a run of whole sequences' suffixes of about equal total length without
  *      draining its pipeline, instead of the default one CTA per (sequence,
  *      kv head) suffix.
+ *  32: one kv head per CTA everywhere.  Otherwise, with the tensor-core
+ *      consumer and Hkv a multiple of 4, a CTA of the partition kernel serves
+ *      four neighbouring kv heads (one per consumer warp) and reads each
+ *      block's rows of all four with one tensor-map copy per 128-byte
+ *      segment (not with grouped partitions, the balanced grid or the
+ *      shared-prefix decode's suffix passes).
  * Default 4.  Every setting computes the same function.
  */
 pa_status pa_decode_select(int mode);

@@ -223,6 +223,7 @@ def pa_decode_partition_group(S: int, Hq: int, Hkv: int, D: int, block_size: int
 DECODE_SIMT_ONLY, DECODE_EVICT_FIRST, DECODE_PARTITION_MAJOR = 1, 2, 4
 DECODE_GROUP_PARTITIONS = 8
 DECODE_SUFFIX_PERSISTENT = 16
+DECODE_ONE_HEAD_PER_CTA = 32
 DECODE_DEFAULT = DECODE_PARTITION_MAJOR
 PA_PARTITION_BALANCED = -1                        # include/pa.h: the persistent balanced grid
 PA_DECODE_NOALLOC_SCRATCH_BYTES = 32 << 20        # include/pa.h: pa_decode_noalloc's array
@@ -232,8 +233,8 @@ def pa_decode_select(mode: int) -> None:
     """Bit mask: 1 CUDA-core consumer everywhere, 2 L2 evict-first K/V loads,
     4 partition-major grid, 8 split-K partitions grouped three to a CTA whenever
     there are several, 16 shared-prefix decode with the persistent whole-item
-    grid for the suffixes instead of one CTA per (sequence, kv head) suffix
-    (default 4)."""
+    grid for the suffixes instead of one CTA per (sequence, kv head) suffix,
+    32 one kv head per CTA everywhere instead of groups of four (default 4)."""
     _check(lib().pa_decode_select(int(mode)))
 
 

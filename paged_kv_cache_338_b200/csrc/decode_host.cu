@@ -20,7 +20,8 @@ namespace {
 // by side), 8 = group split-K partitions three to a CTA whenever there are
 // several (a test hook for the grouped path at small sizes), 16 = shared-prefix
 // decode with the persistent whole-item grid for the suffixes instead of one
-// CTA per (sequence, kv head) suffix; the default is 4.
+// CTA per (sequence, kv head) suffix, 32 = one kv head per CTA everywhere (no
+// head groups); the default is 4.
 std::atomic<int> g_select{4};
 
 // Plain split-K with short partitions: one CTA streams g consecutive
@@ -231,7 +232,7 @@ extern "C" pa_status pa_decode_partition_group(int S, int Hq, int Hkv, int D, in
 
 extern "C" pa_status pa_decode_select(int mode) {
     clear_error();
-    if (mode < 0 || mode > 31) return fail(PA_ERR_INVALID_ARG, "mode must be in [0, 31]");
+    if (mode < 0 || mode > 63) return fail(PA_ERR_INVALID_ARG, "mode must be in [0, 63]");
     g_select.store(mode);
     return PA_OK;
 }
@@ -297,6 +298,17 @@ pa_status pa::decode_impl(void* out, const void* q, pa_dtype q_dt, const void* k
                                : plan_part_group((int64_t)S * Hkv * chunks, max_parts,
                                                  (int64_t)partition * D * elem_size(cache_dt) * 2,
                                                  num_sms);
+    // four neighbouring kv heads per CTA (one per consumer warp), read by one
+    // tensor-map copy per block and segment, where a stage of the four heads'
+    // K and V is at most 32 KB (two stages in flight at three CTAs per SM);
+    // one head per CTA with bit 32, the CUDA-core consumer, grouped or
+    // balanced partitions and the shared-prefix suffix passes (short suffixes
+    // measured slower in groups: four times fewer CTAs to hide their latency)
+    const bool hg_fits = 2 * 4 * stage_tokens * D * elem_size(cache_dt) <= 32 * 1024;
+    const int hg = use_mma && hg_fits && Hkv % 4 == 0 && !(sel & 32) && !balanced && !items &&
+                           !force_ws && prefix_parts == 0 && part_group == 1
+                       ? 4
+                       : 1;
     const int64_t grid_parts = fuse ? 1
                                : prefix_parts > 0 ? max_parts - prefix_parts
                                                   : (max_parts + part_group - 1) / part_group;
@@ -310,9 +322,11 @@ pa_status pa::decode_impl(void* out, const void* q, pa_dtype q_dt, const void* k
                     need, workspace_bytes);
 
     dec::Launch L{};
-    pa_status st = make_cache_map(&L.tmk, key_cache, cache_dt, NB, bs, Hkv, D);
+    pa_status st = hg > 1 ? make_cache_map_heads(&L.tmk, key_cache, cache_dt, NB, bs, Hkv, D, hg)
+                          : make_cache_map(&L.tmk, key_cache, cache_dt, NB, bs, Hkv, D);
     if (st) return st;
-    st = make_cache_map(&L.tmv, value_cache, cache_dt, NB, bs, Hkv, D);
+    st = hg > 1 ? make_cache_map_heads(&L.tmv, value_cache, cache_dt, NB, bs, Hkv, D, hg)
+                : make_cache_map(&L.tmv, value_cache, cache_dt, NB, bs, Hkv, D);
     if (st) return st;
     unsigned int* err = device_error_word();
     if (!err) return PA_ERR_CUDA;
@@ -361,6 +375,7 @@ pa_status pa::decode_impl(void* out, const void* q, pa_dtype q_dt, const void* k
 
     L.bs = bs;
     L.pair = pair;
+    L.hg = hg;
     L.D = D;
     L.mma = use_mma;
     L.mrows = G <= 8 ? 8 : 16;
@@ -368,8 +383,9 @@ pa_status pa::decode_impl(void* out, const void* q, pa_dtype q_dt, const void* k
     L.balanced = balanced || items;
     L.G = G;
     L.num_sms = num_sms;
-    L.grid = p.heads_fastest ? dim3((unsigned)(Hkv * chunks), (unsigned)grid_parts, (unsigned)S)
-                             : dim3((unsigned)grid_parts, (unsigned)(Hkv * chunks), (unsigned)S);
+    const unsigned head_ctas = (unsigned)(Hkv * chunks / hg);
+    L.grid = p.heads_fastest ? dim3(head_ctas, (unsigned)grid_parts, (unsigned)S)
+                             : dim3((unsigned)grid_parts, head_ctas, (unsigned)S);
     L.stream = reinterpret_cast<cudaStream_t>(stream);
 
     cudaError_t e;

@@ -110,10 +110,18 @@ constexpr float kLog2e = 1.4426950408889634f;
 // 8 tokens make a 16-token stage, so an 8-token cache pays the per-stage
 // costs -- barrier round trips, softmax updates, half-empty MMA tiles -- once
 // per 16 tokens).
-template <int DT_, int QT_, int BS_, int D_, int GC_, bool MMA_, int MROWS_ = 8, int PB_ = BS_>
+//
+// HG is the kv heads one CTA serves.  With HG > 1 (= NW) every stage holds
+// the rows of HG neighbouring kv heads, fetched by one tensor-map copy per
+// block and 128-byte segment (the heads' rows of a token are adjacent in
+// memory, so a copy reads HG x 128 contiguous bytes per token instead of 128),
+// and consumer warp w serves kv head w of the group over every stage: no warp
+// merge, no split of a head's blocks between warps.
+template <int DT_, int QT_, int BS_, int D_, int GC_, bool MMA_, int MROWS_ = 8, int PB_ = BS_,
+          int HG_ = 1>
 struct Cfg {
     static constexpr int DT = DT_, QT = QT_, BS = BS_, D = D_, GC = GC_, MROWS = MROWS_;
-    static constexpr int PB = PB_, PER = BS_ / PB_;
+    static constexpr int PB = PB_, PER = BS_ / PB_, HG = HG_;
     static constexpr bool MMA = MMA_;
     static constexpr int E = dev::Storage<DT>::bytes;
     static constexpr int R = D * E;          // bytes of one token row of one kv head
@@ -121,32 +129,38 @@ struct Cfg {
     static constexpr int EPS = 128 / E;      // elements per segment
     static constexpr int EPC = 16 / E;       // elements per 16-byte chunk
     static constexpr int DPL = D / 8;        // dims per lane (SIMT consumer)
-    static constexpr int TILE = BS * R;      // bytes of a K (or V) tile
+    static constexpr int TILE = HG * BS * R; // bytes of the K (or V) tiles of a stage
     static constexpr int STAGE = 2 * TILE;
+    static constexpr int SEGSTRIDE = HG * BS * 128;   // bytes between 128-byte segments
     static constexpr int NW = 4;             // consumer warps
     static constexpr int THREADS = (NW + 1) * 32;
     static constexpr int BUDGET = 64 * 1024;                  // 3 CTAs per SM fit
     static constexpr int COMBINE_FLOATS = NW * GC * (D + 2);   // warp merge reuses the stages
     static constexpr int STAGES_RAW = BUDGET / STAGE;
     static constexpr int STAGES_MIN_C = (COMBINE_FLOATS * 4 + STAGE - 1) / STAGE;
-    static constexpr int STAGES_MIN = STAGES_MIN_C > NW ? STAGES_MIN_C : NW;
+    static constexpr int OWN = HG > 1 ? 1 : NW;  // stage count granule (see below)
+    static constexpr int STAGES_MIN = STAGES_MIN_C > (HG > 1 ? 2 : NW) ? STAGES_MIN_C
+                                                                       : (HG > 1 ? 2 : NW);
     static constexpr int STAGES_MAX = STAGES_MIN > 16 ? STAGES_MIN : 16;
     static constexpr int STAGES_CLAMPED = STAGES_RAW < STAGES_MIN ? STAGES_MIN
                                           : (STAGES_RAW > STAGES_MAX ? STAGES_MAX : STAGES_RAW);
-    // Block j goes to consumer warp j % NW and to stage j % STAGES.  With
-    // STAGES a multiple of NW every stage has exactly one consumer warp, so a
-    // warp waiting on a stage's "full" barrier is never more than one phase
-    // behind it and the parity wait cannot mistake an older, still pending
-    // phase for the one it wants.  Round down, or up when the warp merge needs
-    // the room.
-    static constexpr int STAGES_DOWN = STAGES_CLAMPED / NW * NW;
+    // One head per CTA: block j goes to consumer warp j % NW and to stage
+    // j % STAGES.  With STAGES a multiple of NW every stage has exactly one
+    // consumer warp, so a warp waiting on a stage's "full" barrier is never
+    // more than one phase behind it and the parity wait cannot mistake an
+    // older, still pending phase for the one it wants.  Round down, or up when
+    // the warp merge needs the room.  Head groups: every warp consumes every
+    // stage and the stage's "empty" barrier waits for all of them, so no warp
+    // can fall a phase behind either.
+    static constexpr int STAGES_DOWN = STAGES_CLAMPED / OWN * OWN;
     static constexpr int STAGES = STAGES_DOWN >= STAGES_MIN ? STAGES_DOWN
-                                  : (STAGES_MIN + NW - 1) / NW * NW;
+                                  : (STAGES_MIN + OWN - 1) / OWN * OWN;
     static constexpr size_t SMEM = 1024 /*align slack*/ + size_t(STAGES) * STAGE + 2 * 8 * STAGES;
     static_assert(R == 128 || R == 256 || R == 512, "row bytes must be 128, 256 or 512");
     static_assert(BS == 8 || BS == 16 || BS == 32, "block size");
     static_assert(PER == 1 || (PER == 2 && PB == 8), "a stage holds one block, or two of 8 tokens");
-    static_assert(STAGES % NW == 0, "each stage must have a single consumer warp");
+    static_assert(HG > 1 || STAGES % NW == 0, "each stage must have a single consumer warp");
+    static_assert(HG == 1 || (HG == NW && MMA), "a head group is one kv head per consumer warp");
     static_assert(COMBINE_FLOATS * 4 <= STAGES * STAGE, "combine area must fit in the stages");
     static_assert(SMEM <= 227 * 1024, "shared memory");
 };
@@ -155,9 +169,17 @@ struct Cfg {
 // 128-byte row swizzled by its token index (TMA SWIZZLE_128B, one box per
 // segment).  Eight consecutive tokens of one 16-byte chunk column therefore
 // sit in eight different bank groups, which keeps ldmatrix conflict-free.
+// With head groups a segment is [block of the stage][head][token][128 bytes]
+// and a head's tile starts at its own offset (head * PB * 128); with one head,
+// [token][128 bytes].  A head's block slices are 1024-byte aligned, so a
+// row's swizzle phase is its token index either way.
+template <class C>
+__device__ __forceinline__ int tile_row(int t) {
+    return C::HG == 1 ? t : (t / C::PB) * C::HG * C::PB + (t % C::PB);
+}
 template <class C>
 __device__ __forceinline__ uint32_t tile_off(int t, int seg, int chunk) {
-    return (uint32_t)seg * (C::BS * 128) + dev::swz128(t, chunk);
+    return (uint32_t)seg * C::SEGSTRIDE + dev::swz128(tile_row<C>(t), chunk);
 }
 
 // ------------------------------------------------------------------ producer
@@ -213,7 +235,7 @@ __device__ __forceinline__ void produce(const CUtensorMap* tmk, const CUtensorMa
                     const int have = min(C::PER, nphys - (jb + jj * C::PER));   // >= 1
                     const uint32_t bar = full0 + 8 * st;
                     const uint32_t dk = dev::smem_addr(stages + (size_t)st * C::STAGE);
-                    dev::mbar_arrive_expect_tx(bar, (uint32_t)have * 2 * C::PB * C::R);
+                    dev::mbar_arrive_expect_tx(bar, (uint32_t)have * 2 * C::HG * C::PB * C::R);
                     #pragma unroll
                     for (int r = 0; r < C::PER; ++r) {
                         if (r >= have) break;
@@ -221,10 +243,16 @@ __device__ __forceinline__ void produce(const CUtensorMap* tmk, const CUtensorMa
                             dev::raise_error(p.err, PA_DEV_BAD_BLOCK);
                         #pragma unroll
                         for (int c = 0; c < C::CH; ++c) {
-                            const uint32_t off = c * C::BS * 128 + r * C::PB * 128;
-                            dev::tma_load_4d(dk + off, tmk, bar, c * C::EPS, kvh, 0, id[r], pol);
-                            dev::tma_load_4d(dk + C::TILE + off, tmv, bar, c * C::EPS, kvh, 0,
-                                             id[r], pol);
+                            const uint32_t off = c * C::SEGSTRIDE + r * C::HG * C::PB * 128;
+                            if constexpr (C::HG == 1) {   // map {D, Hkv, bs, NB}
+                                dev::tma_load_4d(dk + off, tmk, bar, c * C::EPS, kvh, 0, id[r], pol);
+                                dev::tma_load_4d(dk + C::TILE + off, tmv, bar, c * C::EPS, kvh, 0,
+                                                 id[r], pol);
+                            } else {                      // map {D, bs, Hkv, NB}, kvh the first head
+                                dev::tma_load_4d(dk + off, tmk, bar, c * C::EPS, 0, kvh, id[r], pol);
+                                dev::tma_load_4d(dk + C::TILE + off, tmv, bar, c * C::EPS, 0, kvh,
+                                                 id[r], pol);
+                            }
                         }
                     }
                 }
@@ -753,10 +781,11 @@ __device__ __forceinline__ void mma_block(MmaState<C>& st, uint8_t* ktile_p, uin
     } else {
         // the 16-bit tile itself, tail rows zeroed
         if (nvalid < BS) {
-            #pragma unroll
-            for (int k = 0; k < C::CH; ++k) {
-                uint4* v4 = reinterpret_cast<uint4*>(vtile_p + k * BS * 128 + nvalid * 128);
-                for (int i = lane; i < (BS - nvalid) * 8; i += 32) v4[i] = make_uint4(0, 0, 0, 0);
+            // whole 128-byte rows of this warp's head, so the swizzle does not matter
+            for (int i = lane; i < (BS - nvalid) * C::CH * 8; i += 32) {
+                const int t = nvalid + i / (C::CH * 8), k = (i / 8) % C::CH;
+                *reinterpret_cast<uint4*>(vtile_p + k * C::SEGSTRIDE + tile_row<C>(t) * 128 +
+                                          (i % 8) * 16) = make_uint4(0, 0, 0, 0);
             }
             __syncwarp();
         }
@@ -924,8 +953,10 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     const int chunks = G / gc;                  // head chunks per kv head
     int part = p.heads_fastest ? blockIdx.y : blockIdx.x;
     const int hc = p.heads_fastest ? blockIdx.x : blockIdx.y;
-    const int kvh = hc / chunks;
-    const int h0 = kvh * G + (hc % chunks) * gc;
+    // one kv head (or head chunk) per CTA, or HG neighbouring kv heads: kvh
+    // is the first, h0 its first query head
+    const int kvh = C::HG > 1 ? hc * C::HG : hc / chunks;
+    const int h0 = C::HG > 1 ? kvh * G : kvh * G + (hc % chunks) * gc;
     const int s = blockIdx.z;
     // the producer's first 32 block ids, for the first block this CTA most
     // likely reads, fetched beside the context length
@@ -1002,7 +1033,7 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::STAGES; ++i) {
             dev::mbar_init(full0 + 8 * i, 1);
-            dev::mbar_init(empty0 + 8 * i, 1);
+            dev::mbar_init(empty0 + 8 * i, C::HG > 1 ? C::NW : 1);   // head groups: every warp
         }
         dev::fence_mbar_init();
         s_abort = 0;
@@ -1021,6 +1052,7 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
 
     using State = typename std::conditional<C::MMA, MmaState<C>, SimtState<C>>::type;
     State st;
+    static_assert(!(GROUPED && C::HG > 1), "grouped partitions take one head per CTA");
     if constexpr (GROUPED) {
         // Grouped partitions: the producer streams the blocks of all nq
         // partitions without a break; the consumers close each partition with
@@ -1112,15 +1144,18 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                    &s_abort, &k, pblk0_guess, pre);
         if (lane == 0) s_issued = k;
     } else {
-        if constexpr (C::MMA) mma_load_q<C>(st, p, s, h0, G);
+        // one head per CTA: warp w takes stages w, w + NW, ...; head groups:
+        // warp w takes every stage, and the tiles of kv head kvh + w in it
+        const int hw = C::HG > 1 ? warp : 0;
+        if constexpr (C::MMA) mma_load_q<C>(st, p, s, h0 + hw * G, G);
         else simt_load_q<C>(st, p, s, h0);
-        for (int j = warp; j < nblk; j += C::NW) {
+        for (int j = C::HG > 1 ? 0 : warp; j < nblk; j += C::HG > 1 ? 1 : C::NW) {
             const int stg = j % C::STAGES;
             if (!dev::mbar_wait_bounded(full0 + 8 * stg, (j / C::STAGES) & 1)) {
                 if (lane == 0) { wait_timeout(p, 2); s_abort = 1; }
                 break;
             }
-            uint8_t* kt = stages + (size_t)stg * C::STAGE;
+            uint8_t* kt = stages + (size_t)stg * C::STAGE + hw * C::PB * 128;
             const int nvalid = min(C::BS, n - (blk0 + j) * C::BS);
             if constexpr (C::MMA)
                 mma_block<C>(st, kt, kt + C::TILE, nvalid, p.qk_scale);
@@ -1150,21 +1185,29 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     __syncthreads();
 
     // ---- merge the warps' states and write -----------------------------
-    for (int idx = threadIdx.x; idx < gc * C::D; idx += C::THREADS) {
-        const int g = idx / C::D, d = idx % C::D;
-        float M = -INFINITY;
-        #pragma unroll
-        for (int w = 0; w < C::NW; ++w) M = fmaxf(M, cm[w * C::GC + g]);
-        float L = 0.f, O = 0.f;
-        if (M != -INFINITY) {
+    // (head groups: warp w's state is the whole of its kv head's; nothing to merge)
+    for (int idx = threadIdx.x; idx < C::HG * gc * C::D; idx += C::THREADS) {
+        const int g = (idx / C::D) % gc, d = idx % C::D;
+        float M = -INFINITY, L = 0.f, O = 0.f;
+        int h = h0 + g;
+        if constexpr (C::HG > 1) {
+            const int w = idx / (gc * C::D), r = w * C::GC + g;
+            M = cm[r];
+            L = cl[r];
+            O = co[r * C::D + d];
+            h = h0 + w * G + g;
+        } else {
             #pragma unroll
-            for (int w = 0; w < C::NW; ++w) {
-                const float f = exp2f(cm[w * C::GC + g] - M);
-                L = fmaf(f, cl[w * C::GC + g], L);
-                O = fmaf(f, co[(w * C::GC + g) * C::D + d], O);
+            for (int w = 0; w < C::NW; ++w) M = fmaxf(M, cm[w * C::GC + g]);
+            if (M != -INFINITY) {
+                #pragma unroll
+                for (int w = 0; w < C::NW; ++w) {
+                    const float f = exp2f(cm[w * C::GC + g] - M);
+                    L = fmaf(f, cl[w * C::GC + g], L);
+                    O = fmaf(f, co[(w * C::GC + g) * C::D + d], O);
+                }
             }
         }
-        const int h = h0 + g;
         if (fuse_records) {
             // combine with the prefix records (o already times v_scale there)
             dev::store_out<C::QT>(p.out, ((size_t)s * p.Hq + h) * C::D + d,

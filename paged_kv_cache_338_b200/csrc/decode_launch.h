@@ -15,6 +15,7 @@ struct Launch {
     Params p;
     int bs, D;
     bool pair;     // two 8-token blocks per 16-token stage
+    int hg;        // kv heads per CTA (1, or 4 with the tensor-core consumer)
     int gc;        // SIMT: query heads per CTA
     bool mma;      // tensor-core consumer
     int mrows;     // MMA: 8 or 16 query rows
@@ -36,8 +37,9 @@ cudaError_t launch_fp8_q_bf16(const Launch& L);
 
 template <class C>
 cudaError_t launch_one(const Launch& L) {
-    if constexpr (C::PER != 1) {
-        if (L.balanced) return cudaErrorNotSupported;   // the host pairs blocks for partitions only
+    if constexpr (C::PER != 1 || C::HG != 1) {
+        // the host pairs blocks and groups heads for the partition kernel only
+        if (L.balanced) return cudaErrorNotSupported;
     } else if (L.balanced) {
         auto kern = decode_balanced<C>;
         const int smem = static_cast<int>(BalancedSmem<C>::bytes(L.mma ? L.G : L.gc));
@@ -58,7 +60,7 @@ cudaError_t launch_one(const Launch& L) {
                                L.stream, L.tmk, L.tmv, L.p);
     }
     Params p = L.p;
-    if constexpr (C::MMA) if (p.part_group > 1) {
+    if constexpr (C::MMA && C::HG == 1) if (p.part_group > 1) {
         // Grouped partitions need a warp-merge area of their own; use them
         // only if it costs no resident CTA per SM.
         auto kern = decode_partition<C, true>;
@@ -106,6 +108,10 @@ cudaError_t launch_by_heads(const Launch& L) {
         if (L.mma) {
             if constexpr (((DT == QT && (DT == PA_F16 || DT == PA_BF16)) || DT == PA_FP8_E4M3) &&
                           D <= 128) {
+                if (L.hg == 4) {
+                    if (L.mrows == 8) return launch_one<Cfg<DT, QT, BS, D, 8, true, 8, PB, 4>>(L);
+                    return launch_one<Cfg<DT, QT, BS, D, 16, true, 16, PB, 4>>(L);
+                }
                 if (L.mrows == 8) return launch_one<Cfg<DT, QT, BS, D, 8, true, 8, PB>>(L);
                 return launch_one<Cfg<DT, QT, BS, D, 16, true, 16, PB>>(L);
             } else {

@@ -56,6 +56,23 @@ pa_status make_cache_map(CUtensorMap* m, const void* base, pa_dtype dt, int64_t 
     return PA_OK;
 }
 
+pa_status make_cache_map_heads(CUtensorMap* m, const void* base, pa_dtype dt, int64_t NB, int bs,
+                               int Hkv, int D, int hg) {
+    auto fn = encode_fn();
+    if (!fn) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    const int e = elem_size(dt);
+    const cuuint64_t row = (cuuint64_t)D * e;            // bytes of one (token, head) row
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)bs, (cuuint64_t)Hkv, (cuuint64_t)NB};
+    cuuint64_t strides[3] = {row * Hkv, row, row * Hkv * bs};   // token, head, block
+    cuuint32_t box[4] = {(cuuint32_t)(128 / e), (cuuint32_t)bs, (cuuint32_t)hg, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, tma_type(dt), 4, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled (head groups) failed (%d)", (int)r);
+    return PA_OK;
+}
+
 pa_status make_rows_map(CUtensorMap* m, const void* base, pa_dtype dt, int64_t T, int H, int D,
                         int box_h, int box_t) {
     auto fn = encode_fn();

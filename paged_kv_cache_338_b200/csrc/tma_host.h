@@ -13,6 +13,14 @@ namespace pa {
 pa_status make_cache_map(CUtensorMap* m, const void* base, pa_dtype dt, int64_t NB, int bs, int Hkv,
                          int D);
 
+// The same cache as a 4-D tensor {D, bs, Hkv, NB} (tokens before heads; the
+// strides keep the memory order) with box {128 bytes of D, bs, hg, 1}: one
+// 128-byte segment of the K (or V) rows of one block for hg neighbouring kv
+// heads, laid out head-major in shared memory ([head][token][128 B]), so each
+// head's rows form the same swizzled tile as a one-head box.
+pa_status make_cache_map_heads(CUtensorMap* m, const void* base, pa_dtype dt, int64_t NB, int bs,
+                               int Hkv, int D, int hg);
+
 // Token-major rows [T, H, D] as a 3-D tensor {D, H, T} with box
 // {128 bytes of D, box_h, box_t}: box_t tokens x box_h heads of one 128-byte
 // segment, 128-byte swizzled, rows past T read as zeros.

@@ -222,3 +222,25 @@ def test_balanced_many_pieces_per_cta():
         bits = pa.pa_device_status()
         assert bits == 0, f"device status {bits:#x} (mode {mode})"
         _check_out(out, want, "bf16", f"mode={mode}")
+
+
+HEAD_GROUPS = [(bs, G, D, dt, hkv) for bs in (8, 16, 32) for G in (2, 4, 16) for D in (64, 128)
+               for dt in ("bf16", "f16", "fp8_e4m3") for hkv in (4, 8)
+               if not (dt == "fp8_e4m3" and D == 64) and not (G == 16 and hkv == 8)]
+
+
+@pytest.mark.parametrize("bs,G,D,dt,hkv", HEAD_GROUPS)
+def test_head_groups(bs, G, D, dt, hkv):
+    """Four kv heads per CTA (one per consumer warp, one tensor-map copy per
+    block for all four) against the oracle, single pass and split-K, paired
+    8-token blocks included; and against one head per CTA."""
+    qdt = dt if dt != "fp8_e4m3" else "bf16"
+    cfg = wl.DecodeConfig(f"hg_{bs}_{G}_{D}_{dt}_{hkv}", 5, hkv * G, hkv, D, bs, dt, qdt, 1,
+                          9 * bs + 3, fp8_scaled=dt == "fp8_e4m3")
+    inp = wl.make_decode_inputs(cfg, seed=bs * 7 + G * 3 + D + hkv)
+    want, _, _ = oracle_step(inp)
+    for part in (0, 2 * bs, 64):
+        for mode in (pa.DECODE_DEFAULT, pa.DECODE_DEFAULT | pa.DECODE_ONE_HEAD_PER_CTA):
+            out, _, _ = gpu_step(inp, part, mode)
+            _check_out(out, want, dt, f"P={part} mode={mode}")
+    assert pa.pa_device_status() == 0
