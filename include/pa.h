@@ -74,7 +74,8 @@ enum {
 };
 /* Bits 16-23 of the device word, when PA_DEV_WAIT_TIMEOUT is set: which wait
  * gave up last (diagnostics; decode: 1 stage-free, 2 stage-full,
- * 3 descriptor-free, 4 descriptor-ready, 5 states-published, 6 merge-done;
+ * 3 descriptor-free, 4 descriptor-ready, 5 states-published, 6 merge-done,
+ * 19 prefix-records;
  * prefill: 7 q-tile, 8 k-tile-full, 9 v-tile-full, 10 k-tile-free,
  * 11 v-tile-free, 12 scores-ready, 13 probabilities-ready, 14 p.v-done,
  * 15 output-ready, 16 tensor-core drain, 17 load drain, 18 exponential turn). */

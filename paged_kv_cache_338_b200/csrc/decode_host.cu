@@ -277,6 +277,10 @@ pa_status pa::decode_impl(void* out, const void* q, pa_dtype q_dt, const void* k
                                   : parts_for(max_ctx, partition);
     if (max_parts > 65535 || (int64_t)Hkv * G > 65535)
         return fail(PA_ERR_UNSUPPORTED, "too many partitions or heads for the grid");
+    // the suffix pass merges its warps' states and the prefix records with
+    // weights kept behind the warp-merge area in its stage memory
+    if (fuse && 4 * (4 * 16 * (D + 2) + (int64_t)G * (4 + prefix_parts + 2)) > 48 * 1024)
+        return fail(PA_ERR_UNSUPPORTED, "shared prefix of %d partitions is too long", prefix_parts);
     const int sel = g_select.load();
     const bool use_mma = !(sel & 1) && G >= 2 && D <= 128 && cache_dt != PA_F32;
     const int gc_simt = G < (D == 256 ? 2 : 4) ? G : (D == 256 ? 2 : 4);
@@ -348,6 +352,14 @@ pa_status pa::decode_impl(void* out, const void* q, pa_dtype q_dt, const void* k
     p.force_ws = force_ws ? 1 : 0;
     p.fuse_prefix_blocks = fuse_prefix_blocks;
     p.part_group = part_group;
+    // one CTA per suffix: room for the prefix records behind the stage
+    // barriers, fetched while the suffix streams (records and their offsets
+    // 16-byte aligned: an even record count per head)
+    p.rec_smem = 0;
+    if (fuse && !items && max_parts % 2 == 0) {
+        const size_t rb = 16 + (size_t)gc * hg * max_parts * ((size_t)D * 4 + 8);
+        if (rb <= 12 * 1024) p.rec_smem = (int)rb;
+    }
     p.max_ctx = max_ctx;
     p.evict_first = (sel & 2) ? 1 : 0;
     p.heads_fastest = (sel & 4) ? 1 : 0;

@@ -84,6 +84,9 @@ struct Params {
                                  // ranges end at item boundaries), whose output it writes;
                                  // with fuse_prefix_blocks the regular items read their suffix
                                  // and fold the prefix_parts prefix records in
+    int rec_smem;                // one CTA per suffix: bytes of dynamic shared memory past the
+                                 // barriers for its prefix records, fetched by a bulk copy while
+                                 // the suffix streams (0: copied into the stages afterwards)
 };
 
 // Record a wait that gave up, with the site that gave up (bits 16-23).
@@ -942,11 +945,16 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     extern __shared__ uint8_t smem_raw[];
     __shared__ int s_abort;
     __shared__ int s_issued;
+    __shared__ int s_rec_issued;
     uint8_t* stages = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* after = stages + (size_t)C::STAGES * C::STAGE;          // barriers, merge area
     const uint32_t full0 = dev::smem_addr(after);
     const uint32_t empty0 = full0 + 8 * C::STAGES;
+    // one CTA per suffix: the prefix records' barrier and buffer follow the
+    // stage barriers (rec_smem bytes of dynamic shared memory)
+    const uint32_t rec_bar = empty0 + 8 * C::STAGES;
+    float* rec_buf = reinterpret_cast<float*>(after + 16 * C::STAGES + 16);
 
     const int G = p.Hq / p.Hkv;
     const int gc = C::MMA ? G : C::GC;          // query heads this CTA serves
@@ -1030,14 +1038,19 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    // the prefix records of a regular suffix arrive by a bulk copy the
+    // producer issues after its last K/V copy (and after the prefix kernel)
+    const bool rec_async = fuse_records && p.rec_smem > 0;
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::STAGES; ++i) {
             dev::mbar_init(full0 + 8 * i, 1);
             dev::mbar_init(empty0 + 8 * i, C::HG > 1 ? C::NW : 1);   // head groups: every warp
         }
+        if (rec_async) dev::mbar_init(rec_bar, 1);
         dev::fence_mbar_init();
         s_abort = 0;
         s_issued = 0;
+        s_rec_issued = 0;
     }
     if (warp == C::NW && lane == 0) {
         dev::prefetch_tensormap(&tmk);
@@ -1139,9 +1152,29 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     }
     if (warp == C::NW) {
         int k = 0;
-        produce<C>(&tmk, &tmv, p, p.block_tables + (size_t)s * p.MB, blk0, nblk,
-                   min(nblk * C::PER, nphys_all - blk0 * C::PER), kvh, stages, full0, empty0,
-                   &s_abort, &k, pblk0_guess, pre);
+        const int32_t* bt_row = p.block_tables + (size_t)s * p.MB;
+        const int nphys = min(nblk * C::PER, nphys_all - blk0 * C::PER);
+        // a regular suffix's prefix records are fetched once the ring is first
+        // full (the producer would wait for a free stage next anyway)
+        const int first = rec_async ? min(nblk, C::STAGES) : nblk;
+        produce<C>(&tmk, &tmv, p, bt_row, blk0, first, min(nphys, first * C::PER), kvh, stages,
+                   full0, empty0, &s_abort, &k, pblk0_guess, pre);
+        if (rec_async && lane == 0 && !*(volatile int*)&s_abort) {
+            // [heads][max_parts][D] then [heads][max_parts], contiguous in the workspace
+            dev::grid_dependency_wait();            // the prefix kernel has written them
+            const int nh = C::HG * gc;
+            const size_t row0 = ((size_t)s * p.Hq + h0) * p.max_parts;
+            const uint32_t bo = (uint32_t)(nh * p.max_parts * C::D * 4);
+            const uint32_t bm = (uint32_t)(nh * p.max_parts * 8);
+            dev::mbar_arrive_expect_tx(rec_bar, bo + bm);
+            dev::bulk_load(dev::smem_addr(rec_buf), p.ws_o + row0 * C::D, bo, rec_bar);
+            dev::bulk_load(dev::smem_addr(rec_buf) + bo, p.ws_ml + row0, bm, rec_bar);
+            s_rec_issued = 1;
+        }
+        __syncwarp();
+        if (first < nblk && !*(volatile int*)&s_abort)
+            produce<C>(&tmk, &tmv, p, bt_row, blk0 + first, nblk - first,
+                       nphys - first * C::PER, kvh, stages, full0, empty0, &s_abort, &k);
         if (lane == 0) s_issued = k;
     } else {
         // one head per CTA: warp w takes stages w, w + NW, ...; head groups:
@@ -1174,6 +1207,7 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
             const int issued = s_issued;
             for (int j = max(0, issued - C::STAGES); j < issued; ++j)
                 dev::mbar_wait_bounded(full0 + 8 * (j % C::STAGES), (j / C::STAGES) & 1);
+            if (s_rec_issued) dev::mbar_wait_bounded(rec_bar, 0);
         }
         return;
     }
@@ -1184,41 +1218,107 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     if (p.fuse_prefix_blocks > 0) dev::grid_dependency_wait();   // the prefix records are written
     __syncthreads();
 
-    // ---- merge the warps' states and write -----------------------------
-    // (head groups: warp w's state is the whole of its kv head's; nothing to merge)
-    for (int idx = threadIdx.x; idx < C::HG * gc * C::D; idx += C::THREADS) {
-        const int g = (idx / C::D) % gc, d = idx % C::D;
-        float M = -INFINITY, L = 0.f, O = 0.f;
-        int h = h0 + g;
-        if constexpr (C::HG > 1) {
-            const int w = idx / (gc * C::D), r = w * C::GC + g;
-            M = cm[r];
-            L = cl[r];
-            O = co[r * C::D + d];
-            h = h0 + w * G + g;
-        } else {
-            #pragma unroll
-            for (int w = 0; w < C::NW; ++w) M = fmaxf(M, cm[w * C::GC + g]);
-            if (M != -INFINITY) {
-                #pragma unroll
-                for (int w = 0; w < C::NW; ++w) {
-                    const float f = exp2f(cm[w * C::GC + g] - M);
-                    L = fmaf(f, cl[w * C::GC + g], L);
-                    O = fmaf(f, co[(w * C::GC + g) * C::D + d], O);
-                }
-            }
+    // Shared-prefix records of this CTA's query heads, copied to shared memory
+    // behind the warp-merge area with every load in flight at once (one round
+    // trip instead of one per output element a thread writes).  They are
+    // contiguous in the workspace: [heads][max_parts][D] and [heads][max_parts].
+    const int nh = C::HG * gc;                  // query heads this CTA writes
+    float* rec_o = rec_async ? rec_buf : comb + C::COMBINE_FLOATS;
+    float2* rec_ml = reinterpret_cast<float2*>(rec_o + (size_t)nh * p.max_parts * C::D);
+    // (staged: also room for the merge weights, nh * (NW + max_parts + 2) floats)
+    const bool staged = fuse_records &&
+                        (rec_async || (size_t)(C::COMBINE_FLOATS + nh * p.max_parts * (C::D + 2) +
+                                               nh * (C::NW + p.max_parts + 2)) *
+                                              4 <= (size_t)C::STAGES * C::STAGE);
+    if (rec_async) {
+        // issued by the producer after its last K/V copy; normally landed by now
+        if (!dev::mbar_wait_bounded(rec_bar, 0)) {
+            if (threadIdx.x == 0) wait_timeout(p, 19);
+            return;
         }
+    } else if (staged) {
+        const size_t row0 = ((size_t)s * p.Hq + h0) * p.max_parts;
+        const float4* src = reinterpret_cast<const float4*>(p.ws_o + row0 * C::D);
+        float4* dst = reinterpret_cast<float4*>(rec_o);
+        const int n4 = nh * p.max_parts * C::D / 4;
+        constexpr int U = 4;
+        for (int i0 = threadIdx.x; i0 < n4; i0 += U * C::THREADS) {
+            float4 r[U];
+            #pragma unroll
+            for (int u = 0; u < U; ++u)
+                if (i0 + u * C::THREADS < n4) r[u] = src[i0 + u * C::THREADS];
+            #pragma unroll
+            for (int u = 0; u < U; ++u)
+                if (i0 + u * C::THREADS < n4) dst[i0 + u * C::THREADS] = r[u];
+        }
+        for (int i = threadIdx.x; i < nh * p.max_parts; i += C::THREADS) rec_ml[i] = p.ws_ml[row0 + i];
+        __syncthreads();
+    }
+
+    // ---- merge the warps' states (and the prefix records) and write -----
+    // Phase 1, one thread per query head: the common maximum M of its partial
+    // states (the consumer warps', or with head groups its warp's; then its
+    // prefix records), the weight 2^(m_i - M) of each and the sum L.  Phase 2,
+    // one thread per output element: the weighted sum of the partial outputs,
+    // with no exponential per element.  (The split-K identity: up to rounding
+    // order the same as merging the states one after another.)
+    const int nsrc = C::HG > 1 ? 1 : C::NW;     // partial states per head
+    const int npre = fuse_records ? p.prefix_parts : 0;
+    const int ncoef = nsrc + npre + 2;          // weights, then M and L
+    float* coef = comb + C::COMBINE_FLOATS +
+                  (staged && !rec_async ? (size_t)nh * p.max_parts * (C::D + 2) : 0);
+    // partial state i of head row r (r = local query head: w * G + g with head groups)
+    auto src_row = [&](int r, int i) { return C::HG > 1 ? (r / gc) * C::GC + r % gc : i * C::GC + r; };
+    const size_t grow0 = ((size_t)s * p.Hq + h0) * p.max_parts;   // records of row 0 (global)
+    for (int r = threadIdx.x; r < nh; r += C::THREADS) {
+        float M = -INFINITY;
+        for (int i = 0; i < nsrc; ++i) M = fmaxf(M, cm[src_row(r, i)]);
+        for (int pp = 0; pp < npre; ++pp)
+            M = fmaxf(M, staged ? rec_ml[r * p.max_parts + pp].x
+                                : p.ws_ml[grow0 + (size_t)r * p.max_parts + pp].x);
+        float L = 0.f;
+        float* c = coef + r * ncoef;
+        for (int i = 0; i < nsrc; ++i) {
+            const int q = src_row(r, i);
+            const float e = M == -INFINITY ? 0.f : exp2f(cm[q] - M);
+            c[i] = e;
+            L = fmaf(e, cl[q], L);
+        }
+        for (int pp = 0; pp < npre; ++pp) {
+            const float2 ml = staged ? rec_ml[r * p.max_parts + pp]
+                                     : p.ws_ml[grow0 + (size_t)r * p.max_parts + pp];
+            const float e = M == -INFINITY ? 0.f : exp2f(ml.x - M);
+            c[nsrc + pp] = e;
+            L = fmaf(e, ml.y, L);
+        }
+        c[ncoef - 2] = M;
+        c[ncoef - 1] = L;
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < nh * C::D; idx += C::THREADS) {
+        const int r = idx / C::D, d = idx % C::D;
+        const int h = C::HG > 1 ? h0 + (r / gc) * G + r % gc : h0 + r;
+        const float* c = coef + r * ncoef;
+        const float L = c[ncoef - 1];
+        float O = 0.f;
+        for (int i = 0; i < nsrc; ++i) O = fmaf(c[i], co[src_row(r, i) * C::D + d], O);
         if (fuse_records) {
-            // combine with the prefix records (o already times v_scale there)
+            // the prefix records' o is already times v_scale
+            float Op = 0.f;
+            for (int pp = 0; pp < npre; ++pp)
+                Op = fmaf(c[nsrc + pp],
+                          staged ? rec_o[((size_t)r * p.max_parts + pp) * C::D + d]
+                                 : p.ws_o[(grow0 + (size_t)r * p.max_parts + pp) * C::D + d],
+                          Op);
             dev::store_out<C::QT>(p.out, ((size_t)s * p.Hq + h) * C::D + d,
-                                  fold_prefix_records(p, s, h, d, M, L, O * p.v_scale, C::D));
+                                  L > 0.f ? fmaf(O, p.v_scale, Op) / L : 0.f);
         } else if (nparts == 1 && !p.force_ws) {
             dev::store_out<C::QT>(p.out, ((size_t)s * p.Hq + h) * C::D + d,
                                   L > 0.f ? (O / L) * p.v_scale : 0.f);
         } else {
             const size_t row = ((size_t)s * p.Hq + h) * p.max_parts + part;
             p.ws_o[row * C::D + d] = O * p.v_scale;
-            if (d == 0) p.ws_ml[row] = make_float2(M, L);
+            if (d == 0) p.ws_ml[row] = make_float2(c[ncoef - 2], L);
         }
     }
 }

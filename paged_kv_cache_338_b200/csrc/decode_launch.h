@@ -86,11 +86,12 @@ cudaError_t launch_one(const Launch& L) {
         (p.heads_fastest ? grid.y : grid.x) = (unsigned)p.max_parts;
     }
     auto kern = decode_partition<C, false>;
+    const size_t smem = C::SMEM + (size_t)p.rec_smem;   // + the shared-prefix records
     // opt in to > 48 KB of dynamic shared memory (idempotent, cheap)
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(C::SMEM));
+                                         static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    return dev::launch_pdl(kern, grid, dim3(C::THREADS), C::SMEM, L.stream, L.tmk, L.tmv, p);
+    return dev::launch_pdl(kern, grid, dim3(C::THREADS), smem, L.stream, L.tmk, L.tmv, p);
 }
 
 template <int DT, int D>
