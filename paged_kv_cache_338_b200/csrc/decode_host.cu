@@ -354,9 +354,10 @@ pa_status pa::decode_impl(void* out, const void* q, pa_dtype q_dt, const void* k
     p.part_group = part_group;
     // one CTA per suffix: room for the prefix records behind the stage
     // barriers, fetched while the suffix streams (records and their offsets
-    // 16-byte aligned: an even record count per head)
+    // 16-byte aligned: an even record count per head, or an even number of
+    // heads per CTA starting at an even head)
     p.rec_smem = 0;
-    if (fuse && !items && max_parts % 2 == 0) {
+    if (fuse && !items && (max_parts % 2 == 0 || (gc % 2 == 0 && G % 2 == 0))) {
         const size_t rb = 16 + (size_t)gc * hg * max_parts * ((size_t)D * 4 + 8);
         if (rb <= 12 * 1024) p.rec_smem = (int)rb;
     }

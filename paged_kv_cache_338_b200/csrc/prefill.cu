@@ -88,6 +88,7 @@ struct Params {
     // identity_blocks), no causal mask, and the result is the split-K record
     // (m, l, o * v_scale) of partition `chunk` of every (sequence, head)
     int prefix, chunk_tokens, identity_blocks, max_parts;
+    int pair_group;               // adjacent tile pairs per grid group (kPairGroup, or fewer)
     float2* ws_ml;
     float* ws_o;
     float v_scale;
@@ -330,17 +331,22 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                const __grid_constant__ CUtensorMap tmv, const Params p) {
     using L = Smem<D>;
     constexpr int NSEG = L::NSEG, ST = L::ST;
+    // Launched as a programmatic dependent of the kernel before it: wait for
+    // its memory (the cache append, or the prefix conversion) before reading.
+    grid_dependency_wait();
     // Prefix mode: the suffix decode launched next reads the records only at
     // its very end (after its own griddepcontrol.wait), so let its CTAs start
-    // on the SMs this grid leaves free.
+    // on the SMs this grid leaves free.  Everything the kernels before this one
+    // wrote is complete once the wait above returns (each of them waited for
+    // its own predecessor), which the suffix decode relies on.
     if (p.prefix) launch_dependents();
     // grid (kPairGroup tile pairs x kv heads, sequences | prefix chunks, pair
     // groups): a group of adjacent tile pairs of one (sequence, kv head) runs
     // side by side and shares its K/V through L2, while groups run longest
     // first across all sequences (the causal tail stays short)
-    const int g = (int)blockIdx.x / kPairGroup;
-    const int pair = ((int)gridDim.z - 1 - (int)blockIdx.z) * kPairGroup +
-                     (kPairGroup - 1 - (int)blockIdx.x % kPairGroup);
+    const int PG = p.pair_group;
+    const int g = (int)blockIdx.x / PG;
+    const int pair = ((int)gridDim.z - 1 - (int)blockIdx.z) * PG + (PG - 1 - (int)blockIdx.x % PG);
     if (pair >= p.n_pairs) return;                        // past the last pair
     const bool pfx = p.prefix != 0;
     const int s = pfx ? 0 : (int)blockIdx.y;              // the sequence (table row)
@@ -728,10 +734,8 @@ cudaError_t launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorM
     static const cudaError_t attr = cudaFuncSetAttribute(
         prefill_kernel<DT, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Smem<D>::BYTES);
     if (attr != cudaSuccess) return attr;
-    prefill_kernel<DT, D><<<grid, kThreads, Smem<D>::BYTES, st>>>(mq, mk, mv, p);
-    const cudaError_t e = cudaGetLastError();
-    if (e == cudaSuccess) pa::note_launch();
-    return e;
+    return launch_pdl(prefill_kernel<DT, D>, grid, dim3(kThreads), (size_t)Smem<D>::BYTES, st, mq,
+                      mk, mv, p);
 }
 
 }  // namespace pf
@@ -784,8 +788,11 @@ pa_status pa::prefix_records(const void* q, pa_dtype dt, const void* k_src, cons
     p.ws_ml = ws_ml;
     p.ws_o = ws_o;
     p.v_scale = v_scale;
-    const dim3 grid((unsigned)(Hkv * pf::kPairGroup), (unsigned)chunks,
-                    (unsigned)((n_pairs + pf::kPairGroup - 1) / pf::kPairGroup));
+    // as many pair slots per group as there are pairs (no CTA that only exits:
+    // each would hold a whole SM's shared memory for a moment)
+    p.pair_group = (int)(n_pairs < pf::kPairGroup ? n_pairs : pf::kPairGroup);
+    const dim3 grid((unsigned)(Hkv * p.pair_group), (unsigned)chunks,
+                    (unsigned)((n_pairs + p.pair_group - 1) / p.pair_group));
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     cudaError_t e;
     if (dt == PA_BF16)
@@ -862,6 +869,7 @@ extern "C" pa_status pa_prefill(void* out, const void* q, pa_dtype q_dt, const v
     p.max_qlen = max_query_len;
     p.n_pairs = (int)n_pairs;
     p.sl = scale * 1.4426950408889634f;
+    p.pair_group = pf::kPairGroup;
 
     const dim3 grid((unsigned)(Hkv * pf::kPairGroup), (unsigned)S,
                     (unsigned)((n_pairs + pf::kPairGroup - 1) / pf::kPairGroup));

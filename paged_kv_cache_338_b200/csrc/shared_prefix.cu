@@ -39,6 +39,10 @@ template <int QT>
 __global__ void prefix_to_16bit(const uint8_t* kc, const uint8_t* vc, const int32_t* table_row0,
                                 int64_t NB, int blk_elems, uint16_t* sk, uint16_t* sv,
                                 unsigned int* err) {
+    // a programmatic dependent of the cache append: wait for its memory, and
+    // let the prefix kernel's CTAs get resident meanwhile
+    pa::dev::grid_dependency_wait();
+    pa::dev::launch_dependents();
     const int lb = blockIdx.y;
     const int e = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
     if (e >= blk_elems) return;
@@ -185,17 +189,14 @@ extern "C" pa_status pa_decode_shared_prefix(void* out, const void* q, pa_dtype 
         unsigned int* err = pa::device_error_word();
         if (!err) return PA_ERR_CUDA;
         const dim3 grid((unsigned)((blk_elems / 8 + 255) / 256), (unsigned)nblk, 2);
-        if (q_dt == PA_BF16)
-            prefix_to_16bit<PA_BF16><<<grid, 256, 0, cs>>>(
-                static_cast<const uint8_t*>(key_cache), static_cast<const uint8_t*>(value_cache),
-                block_tables, NB, blk_elems, sk, sv, err);
-        else
-            prefix_to_16bit<PA_F16><<<grid, 256, 0, cs>>>(
-                static_cast<const uint8_t*>(key_cache), static_cast<const uint8_t*>(value_cache),
-                block_tables, NB, blk_elems, sk, sv, err);
-        cudaError_t e = cudaGetLastError();
+        const uint8_t* kc8 = static_cast<const uint8_t*>(key_cache);
+        const uint8_t* vc8 = static_cast<const uint8_t*>(value_cache);
+        cudaError_t e = q_dt == PA_BF16
+                            ? pa::dev::launch_pdl(prefix_to_16bit<PA_BF16>, grid, dim3(256), 0, cs,
+                                                  kc8, vc8, block_tables, NB, blk_elems, sk, sv, err)
+                            : pa::dev::launch_pdl(prefix_to_16bit<PA_F16>, grid, dim3(256), 0, cs,
+                                                  kc8, vc8, block_tables, NB, blk_elems, sk, sv, err);
         if (e != cudaSuccess) return pa::cuda_fail(e, "prefix conversion launch");
-        pa::note_launch();
         k_src = sk;
         v_src = sv;
         src_blocks = nblk;
