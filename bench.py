@@ -25,8 +25,11 @@ Printed (rank 0, one JSON line):
 
 --impl reference runs the oracle (the only reference this method has here) on
 a bounded sample of the same workload on the host cores.
-With torchrun, N ranks each run an independent replica (no data-path
-collective); value = the units all ranks processed / max time over ranks.
+With torchrun (decode), the N ranks split one global batch of N x the
+workload's sequences by sequence (pa_plan_shards: longest first, to the rank
+with the fewest tokens; decode needs no data exchange between ranks), each
+rank running its share on its own GPU; prefill runs N independent replicas.
+value = the units all ranks processed / max time over ranks.
 """
 from __future__ import annotations
 
@@ -298,7 +301,7 @@ def _config_dict(cfg, args, partition=None, l2_note=None):
          "kv_heads": cfg.num_kv_heads, "head_dim": cfg.head_dim, "block_size": cfg.block_size,
          "kv_dtype": cfg.kv_dtype, "q_dtype": cfg.q_dtype,
          "context_lens": list(cfg.fixed_lens[:1]) * 1 if cfg.fixed_lens else [cfg.ctx_lo, cfg.ctx_hi],
-         "parallelism": f"replicas{args.gpus}"}
+         "parallelism": f"seq-shards{args.gpus}" if args.gpus > 1 else "single"}
     if cfg.prefix_tokens:
         d.update(prefix_tokens=cfg.prefix_tokens, suffix=[cfg.suffix_lo, cfg.suffix_hi])
     if partition is not None:
@@ -333,11 +336,15 @@ def _traffic(cfg, part, shared):
 
 
 def csrc_sha256() -> str:
-    """Hash of the library's kernel sources (every file under csrc/)."""
+    """Hash of the library's CUDA sources and headers under csrc/ (the .cu,
+    .cuh and .h files: kernels and their launches; the host-only .cpp files
+    do not change what a kernel reads)."""
     import hashlib
     d = os.path.join(ROOT, "paged_kv_cache_338_b200", "csrc")
     h = hashlib.sha256()
     for fn in sorted(os.listdir(d)):
+        if not fn.endswith((".cu", ".cuh", ".h")):
+            continue
         with open(os.path.join(d, fn), "rb") as f:
             h.update(fn.encode() + b"\0" + f.read())
     return h.hexdigest()
@@ -447,13 +454,31 @@ def roofline_of(cfg, r, peak, peak_kind):
     return d
 
 
+def sharded_cfg(cfg, seed, rank, world, pa):
+    """This rank's share of one global batch: world x num_seqs sequences drawn
+    like the workload's (the same draw on every rank), split by sequence with
+    pa_plan_shards (longest first, to the least loaded rank), so every rank
+    streams about the same K/V and no rank waits on another's data."""
+    if world == 1:
+        return cfg
+    import dataclasses
+    g = dataclasses.replace(cfg, num_seqs=cfg.num_seqs * world, fixed_num_blocks=None,
+                            fixed_lens=tuple(cfg.fixed_lens) * world if cfg.fixed_lens else None)
+    lens = wl.draw_context_lens(g, seed)
+    dev_of, _ = pa.pa_plan_shards(lens, world)
+    mine = lens[dev_of.to(torch.int64) == rank]
+    return dataclasses.replace(cfg, num_seqs=int(mine.numel()), fixed_lens=tuple(mine.tolist()),
+                               fixed_num_blocks=None, name=f"{cfg.name}_shard{rank}of{world}")
+
+
 def run_gpu(args, cfg, rank, world, local_rank):
     import paged_kv_cache_338_b200 as pa
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     if args.decode_select is not None:
         pa.pa_decode_select(args.decode_select)
-    r = device_leg(args, cfg, pa, dev, args.seed + rank, args.steps, args.warmup, args.partition)
+    shard = sharded_cfg(cfg, args.seed, rank, world, pa)     # the workload itself at N = 1
+    r = device_leg(args, shard, pa, dev, args.seed + rank, args.steps, args.warmup, args.partition)
     S, part, nbytes = r["S"], r["part"], r["nbytes"]
     step_bytes = nbytes["decode"] + nbytes["append"]
     value = whole_job_rate(step_bytes * args.steps, r["ms"], dev) / 1e9
@@ -462,7 +487,7 @@ def run_gpu(args, cfg, rank, world, local_rank):
     seqs_all = sum_over_ranks(S, dev)
 
     # ---- end to end through the public API with host buffers -------------
-    e2e = run_e2e(args, cfg, pa, dev, part) if not args.no_e2e else None
+    e2e = run_e2e(args, shard, pa, dev, part) if not args.no_e2e else None
     if e2e is not None:
         e2e["value"] = whole_job_rate(e2e["bytes"], e2e["ms"], dev) / 1e9
 
@@ -471,7 +496,8 @@ def run_gpu(args, cfg, rank, world, local_rank):
     if args.workloads_also:
         for name in args.workloads_also.split(","):
             wcfg = wl.DECODE_WORKLOADS[name]
-            x = device_leg(args, wcfg, pa, dev, args.seed + rank, args.steps, args.warmup)
+            x = device_leg(args, sharded_cfg(wcfg, args.seed, rank, world, pa), pa, dev,
+                           args.seed + rank, args.steps, args.warmup)
             xv = whole_job_rate((x["nbytes"]["decode"] + x["nbytes"]["append"]) * args.steps,
                                 x["ms"], dev) / 1e9
             extras[name] = (wcfg, x, xv, max_over_ranks(x["ms"], dev) / args.steps)

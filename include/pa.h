@@ -484,6 +484,22 @@ pa_status pa_pool_cache_lookup(pa_pool* pool, uint64_t hash, int32_t* block);
 pa_status pa_pool_seq_match_prefix(pa_pool* pool, int64_t seq, const uint64_t* hashes, int n,
                                    int* matched);
 
+/*
+ * Sequence sharding over several GPUs (host only; the pages have no
+ * counterpart: they describe one GPU).  Decode reads no other sequence's
+ * blocks, so a batch splits by sequence with no exchange between devices;
+ * each device then runs its own step over its own cache.  The plan balances
+ * the K/V bytes each device streams, which are proportional to the context
+ * lengths: sequences are taken longest first (ties: lower index first) and
+ * each goes to the device with the fewest tokens so far (ties: lower device).
+ *
+ * context_lens_host: [S] lengths (>= 0).  device_of_seq_host: [S] out, the
+ * device of each sequence.  tokens_per_device_host: [ndev] out (may be NULL).
+ * S >= 0, ndev >= 1, else PA_ERR_INVALID_ARG.
+ */
+pa_status pa_plan_shards(const int32_t* context_lens_host, int S, int ndev,
+                         int32_t* device_of_seq_host, int64_t* tokens_per_device_host);
+
 #ifdef __cplusplus
 }
 #endif

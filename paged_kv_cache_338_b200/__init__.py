@@ -23,7 +23,7 @@ __all__ = [
     "pa_reshape_and_cache", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_size",
     "pa_decode_suggest_partition", "pa_decode_partition_group", "pa_decode_select", "pa_decode_noalloc", "pa_prefill",
     "pa_decode_shared_prefix", "pa_decode_shared_prefix_workspace_size",
-    "BlockPool",
+    "BlockPool", "pa_plan_shards",
     "PA_DEV_BAD_SLOT", "PA_DEV_BAD_BLOCK", "PA_DEV_WAIT_TIMEOUT", "PA_DEV_BAD_CONTEXT",
 ]
 
@@ -106,6 +106,7 @@ def lib() -> ctypes.CDLL:
         "pa_pool_cache_block": ([P, I32, ctypes.c_uint64, ctypes.POINTER(I)], I),
         "pa_pool_cache_lookup": ([P, ctypes.c_uint64, ctypes.POINTER(I32)], I),
         "pa_pool_seq_match_prefix": ([P, I64, P, I, ctypes.POINTER(I)], I),
+        "pa_plan_shards": ([P, I, I, P, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -329,6 +330,19 @@ def pa_prefill(out: torch.Tensor, q: torch.Tensor, key_cache: torch.Tensor,
                             _dt(key_cache), _ptr(block_tables), MB, _ptr(context_lens),
                             _ptr(query_start), S, T, Hq, Hkv, D, bs, NB, int(max_query_len),
                             float(scale), _stream(stream)))
+
+
+def pa_plan_shards(context_lens, ndev: int):
+    """Split a batch over ndev GPUs by sequence (host): -> (device of each
+    sequence int32 [S], tokens per device int64 [ndev]).  Longest first, each to
+    the device with the fewest tokens so far."""
+    lens = torch.as_tensor(context_lens, dtype=torch.int32).cpu().contiguous()
+    S = lens.numel()
+    dev = torch.empty(S, dtype=torch.int32)
+    tok = torch.empty(max(int(ndev), 1), dtype=torch.int64)
+    _check(lib().pa_plan_shards(lens.data_ptr() if S else None, S, int(ndev),
+                                dev.data_ptr() if S else None, tok.data_ptr()))
+    return dev, tok
 
 
 class BlockPool:

@@ -513,3 +513,39 @@ def test_pool_step_equals_append_then_pack(seed):
             assert torch.equal(slots_a, slots_b) and torch.equal(pairs_a, pairs_b)
             assert torch.equal(tab_a, tab_b) and torch.equal(len_a, len_b)
         assert [a.ref(i) for i in range(nb)] == [b.ref(i) for i in range(nb)]
+
+
+def _lpt(lens, ndev):
+    """Longest first (stable), each to the least loaded device (lowest on ties)."""
+    order = sorted(range(len(lens)), key=lambda s: -lens[s])
+    load, dev = [0] * ndev, [0] * len(lens)
+    for s in order:
+        d = min(range(ndev), key=lambda i: (load[i], i))
+        dev[s] = d
+        load[d] += lens[s]
+    return dev, load
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_plan_shards_is_lpt_and_balanced(seed):
+    """pa_plan_shards: the longest-first greedy plan exactly; every sequence on
+    one device; per-device tokens add up; within Graham's 4/3 bound of the
+    best split (brute force on small batches)."""
+    import itertools
+    g = torch.Generator().manual_seed(seed)
+    for trial in range(30):
+        S = int(torch.randint(0, 9, (1,), generator=g))
+        nd = int(torch.randint(1, 4, (1,), generator=g))
+        lens = torch.randint(0, 50, (S,), generator=g).tolist()
+        dev, tok = pa.pa_plan_shards(lens, nd)
+        want_dev, want_load = _lpt(lens, nd)
+        assert dev.tolist() == want_dev and tok.tolist() == want_load
+        if S:
+            best = min(max(sum(l for l, a in zip(lens, asg) if a == d) for d in range(nd))
+                       for asg in itertools.product(range(nd), repeat=S))
+            assert max(want_load) <= (4 / 3 - 1 / (3 * nd)) * best + 1e-9
+    big = torch.randint(1, 8193, (1024,), generator=g)
+    dev, tok = pa.pa_plan_shards(big, 8)
+    assert int(tok.sum()) == int(big.sum()) and int(tok.max() - tok.min()) <= 8192
+    _bad(pa.pa_plan_shards, [3, 4], 0)
+    _bad(pa.pa_plan_shards, [3, -1], 2)

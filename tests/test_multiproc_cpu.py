@@ -88,3 +88,46 @@ def test_reference_arm_runs_on_rank_zero_only(tmp_path):
     mp.start_processes(_reference_rank, args=(2, port, str(tmp_path)), nprocs=2, join=True,
                        start_method="spawn")
     assert (tmp_path / "ref1.txt").read_text() == ""      # rank 1 did no work, printed nothing
+
+
+def _shard_rank(rank: int, world: int, port: int, out_dir: str):
+    sys.path.insert(0, ROOT)
+    import bench
+    import paged_kv_cache_338_b200 as pa
+    import workloads as wl
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    try:
+        cfg = wl.DECODE_WORKLOADS["llama3_8b_gqa_bf16_b128"]
+        mine = bench.sharded_cfg(cfg, 2, rank, world, pa)
+        # every rank's share, gathered over the process group
+        lens = torch.tensor(mine.fixed_lens, dtype=torch.int64)
+        sizes = [torch.zeros(1, dtype=torch.int64) for _ in range(world)]
+        dist.all_gather(sizes, torch.tensor([lens.numel()]))
+        padded = torch.zeros(int(max(s.item() for s in sizes)), dtype=torch.int64)
+        padded[:lens.numel()] = lens
+        parts = [torch.zeros_like(padded) for _ in range(world)]
+        dist.all_gather(parts, padded)
+        got = sorted(sum((p[:int(n.item())].tolist() for p, n in zip(parts, sizes)), []))
+        import dataclasses
+        glob = dataclasses.replace(cfg, num_seqs=cfg.num_seqs * world)
+        want = sorted(wl.draw_context_lens(glob, 2).tolist())
+        with open(os.path.join(out_dir, f"shard{rank}.json"), "w") as f:
+            json.dump({"n": lens.numel(), "tokens": int(lens.sum()), "union_ok": got == want,
+                       "name": mine.name}, f)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_bench_splits_one_global_batch_by_sequence(tmp_path):
+    """Under torchrun the decode bench splits one global batch (2 x 128
+    sequences) over the ranks: the shares are disjoint, cover the batch, and
+    carry about the same tokens."""
+    port = _free_port()
+    mp.start_processes(_shard_rank, args=(2, port, str(tmp_path)), nprocs=2, join=True,
+                       start_method="spawn")
+    res = [json.loads((tmp_path / f"shard{r}.json").read_text()) for r in range(2)]
+    assert all(r["union_ok"] for r in res)
+    assert res[0]["n"] + res[1]["n"] == 256
+    assert abs(res[0]["tokens"] - res[1]["tokens"]) <= 8192
+    assert res[0]["name"].endswith("shard0of2") and res[1]["name"].endswith("shard1of2")

@@ -158,6 +158,11 @@ def _draw_lens(cfg: DecodeConfig, g: torch.Generator) -> torch.Tensor:
     return torch.randint(cfg.ctx_lo, cfg.ctx_hi + 1, (cfg.num_seqs,), generator=g)
 
 
+def draw_context_lens(cfg: DecodeConfig, seed: int) -> torch.Tensor:
+    """The context lengths make_decode_inputs(cfg, seed) draws (int64 [S])."""
+    return _draw_lens(cfg, torch.Generator(device="cpu").manual_seed(seed))
+
+
 def _fill_normal(t: torch.Tensor, dtype_name: str, g: torch.Generator,
                  scale_div: float = 1.0, chunk: int = 1 << 26) -> None:
     """Fill t (any shape) with N(0,1) draws cast to its dtype, chunked to bound memory.
