@@ -316,9 +316,19 @@ def _config_dict(cfg, args, partition=None, l2_note=None):
 def _traffic(cfg, part, shared):
     """DRAM read + write bytes of one attention call from the committed ncu
     capture of the same workload and path (profiles/traffic_<workload>[_shared_prefix].json),
-    or None when there is none, it was taken for another partition, or the
-    kernel sources changed since (the file records their hash)."""
+    or None when there is none, it was taken for another partition, or it does
+    not carry the hash of the kernel sources it was taken on (a capture of
+    kernels that have changed since says nothing about the ones timed)."""
     name = f"traffic_{cfg.name}{'_shared_prefix' if shared else ''}.json"
+    pj = _committed_capture(name)
+    if pj is None or (not shared and pj.get("partition") != part):
+        return None
+    return pj.get("dram_bytes_per_launch")
+
+
+def _committed_capture(name):
+    """The profiles/<name> traffic record if it was taken on the current kernel
+    sources (its csrc_sha256 equals csrc_sha256()), else None."""
     prof = os.path.join(ROOT, "profiles", name)
     if not os.path.exists(prof):
         return None
@@ -327,12 +337,9 @@ def _traffic(cfg, part, shared):
             pj = json.load(f)
     except Exception:
         return None
-    if not shared and pj.get("partition") != part:
+    if pj.get("csrc_sha256") != csrc_sha256():
         return None
-    sha = pj.get("csrc_sha256")
-    if sha is not None and sha != csrc_sha256():
-        return None
-    return pj.get("dram_bytes_per_launch")
+    return pj
 
 
 def csrc_sha256() -> str:
@@ -829,13 +836,9 @@ def run_gpu_prefill(args, cfg: wl.PrefillConfig, rank, world, local_rank):
     peak, peak_kind = _prefill_peak(ms)
     achieved = flops / (k_ms * 1e-3) / 1e12
     traffic = None                  # DRAM bytes of one pa_prefill, from the committed capture
-    prof = os.path.join(ROOT, "profiles", f"traffic_{cfg.name}.json")
-    if os.path.exists(prof) and not args.seqs:
-        try:
-            with open(prof) as f:
-                traffic = json.load(f).get("dram_bytes_per_launch")
-        except Exception:
-            traffic = None
+    pj = None if args.seqs else _committed_capture(f"traffic_{cfg.name}.json")
+    if pj is not None:
+        traffic = pj.get("dram_bytes_per_launch")
     cpu = None
     if not args.no_cpu_baseline and world == 1:
         r = prefill_oracle_rate(cfg, args.seed, args.cpu_budget)

@@ -131,3 +131,23 @@ def test_bench_splits_one_global_batch_by_sequence(tmp_path):
     assert res[0]["n"] + res[1]["n"] == 256
     assert abs(res[0]["tokens"] - res[1]["tokens"]) <= 8192
     assert res[0]["name"].endswith("shard0of2") and res[1]["name"].endswith("shard1of2")
+
+
+def test_committed_traffic_needs_the_hash_of_the_current_kernels(tmp_path, monkeypatch):
+    """A traffic record counts only when it was taken on the kernel sources
+    that are built now: one without a hash, or with another one, gives None."""
+    import bench
+    import workloads as wl
+    cfg = wl.DECODE_WORKLOADS["llama3_8b_gqa_bf16_b128"]
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "csrc_sha256", lambda: "abc")
+    f = tmp_path / "profiles" / f"traffic_{cfg.name}.json"
+    rec = {"dram_bytes_per_launch": 123, "partition": 2048}
+    f.write_text(json.dumps(rec))
+    assert bench._traffic(cfg, 2048, False) is None
+    f.write_text(json.dumps(dict(rec, csrc_sha256="def")))
+    assert bench._traffic(cfg, 2048, False) is None
+    f.write_text(json.dumps(dict(rec, csrc_sha256="abc")))
+    assert bench._traffic(cfg, 2048, False) == 123
+    assert bench._traffic(cfg, 512, False) is None          # taken for another partition
