@@ -186,9 +186,11 @@ __device__ __forceinline__ uint32_t tile_off(int t, int seg, int chunk) {
 }
 
 // ------------------------------------------------------------------ producer
-// One warp; lane 0 issues.  Block ids are fetched 32 at a time (one per lane)
-// and handed to lane 0 with a shuffle, so the issue loop never waits on a
-// dependent global load.
+// One warp.  Block ids are fetched 32 at a time (one per lane) and handed out
+// with shuffles, so the issue loop never waits on a dependent global load.
+// Stages whose slot has not been used yet (the CTA's first ring) need no wait
+// on an "empty" barrier: one lane each issues them, side by side; every later
+// stage is issued by lane 0 once its slot is free.
 //
 // A lane's id of the first 32 blocks can be loaded ahead of time (while the
 // CTA still reads its context length and sets up its barriers):
@@ -197,6 +199,35 @@ __device__ __forceinline__ uint32_t tile_off(int t, int seg, int chunk) {
 __device__ __forceinline__ int table_entry_ahead(const Params& p, int s, int pblk0_guess) {
     const int i = pblk0_guess + (threadIdx.x & 31);
     return (pblk0_guess >= 0 && i < p.MB) ? __ldg(p.block_tables + (size_t)s * p.MB + i) : 0;
+}
+
+// Issue stage slot `st`: `have` (>= 1) physical blocks id[0 .. have-1] of
+// kv head kvh (the first head of the group), every 128-byte segment of K and
+// V, completing on the slot's "full" barrier.
+template <class C>
+__device__ __forceinline__ void issue_stage(const CUtensorMap* tmk, const CUtensorMap* tmv,
+                                            const Params& p, const int (&id)[C::PER], int have,
+                                            int kvh, int st, uint8_t* stages, uint32_t full0,
+                                            uint64_t pol) {
+    const uint32_t bar = full0 + 8 * st;
+    const uint32_t dk = dev::smem_addr(stages + (size_t)st * C::STAGE);
+    dev::mbar_arrive_expect_tx(bar, (uint32_t)have * 2 * C::HG * C::PB * C::R);
+    #pragma unroll
+    for (int r = 0; r < C::PER; ++r) {
+        if (r >= have) break;
+        if (id[r] < 0 || (int64_t)id[r] >= p.NB) dev::raise_error(p.err, PA_DEV_BAD_BLOCK);
+        #pragma unroll
+        for (int c = 0; c < C::CH; ++c) {
+            const uint32_t off = c * C::SEGSTRIDE + r * C::HG * C::PB * 128;
+            if constexpr (C::HG == 1) {   // map {D, Hkv, bs, NB}
+                dev::tma_load_4d(dk + off, tmk, bar, c * C::EPS, kvh, 0, id[r], pol);
+                dev::tma_load_4d(dk + C::TILE + off, tmv, bar, c * C::EPS, kvh, 0, id[r], pol);
+            } else {                      // map {D, bs, Hkv, NB}, kvh the first head
+                dev::tma_load_4d(dk + off, tmk, bar, c * C::EPS, 0, kvh, id[r], pol);
+                dev::tma_load_4d(dk + C::TILE + off, tmv, bar, c * C::EPS, 0, kvh, id[r], pol);
+            }
+        }
+    }
 }
 
 template <class C>
@@ -219,45 +250,33 @@ __device__ __forceinline__ void produce(const CUtensorMap* tmk, const CUtensorMa
                          : (jb == 0 && pre_pblk0 == pblk0) ? pre
                                                            : __ldg(bt_row + pblk0 + jb + lane);
         const int cnt = min(32, nblk * C::PER - jb) / C::PER;   // stages of this round
-        for (int jj = 0; jj < cnt; ++jj) {
+        // the round's stages in never-used slots: lane jj issues stage jj
+        const int nfree = max(0, min(cnt, C::STAGES - k));
+        {
+            int id[C::PER];
+            #pragma unroll
+            for (int r = 0; r < C::PER; ++r)
+                id[r] = __shfl_sync(0xffffffffu, mine, (lane * C::PER + r) & 31);
+            if (lane < nfree)
+                issue_stage<C>(tmk, tmv, p, id, min(C::PER, nphys - (jb + lane * C::PER)), kvh,
+                               (k + lane) % C::STAGES, stages, full0, pol);
+        }
+        k += nfree;
+        for (int jj = nfree; jj < cnt; ++jj) {
             int id[C::PER];
             #pragma unroll
             for (int r = 0; r < C::PER; ++r) id[r] = __shfl_sync(0xffffffffu, mine, jj * C::PER + r);
             int stop = 0;
             if (lane == 0) {
                 const int st = k % C::STAGES;
-                if (k >= C::STAGES) {
-                    const uint32_t par = ((k / C::STAGES) & 1) ^ 1;
-                    if (!dev::mbar_wait_bounded(empty0 + 8 * st, par)) {
-                        wait_timeout(p, 1);
-                        *s_abort = 1;
-                        stop = 1;
-                    }
-                }
-                if (!stop) {
-                    const int have = min(C::PER, nphys - (jb + jj * C::PER));   // >= 1
-                    const uint32_t bar = full0 + 8 * st;
-                    const uint32_t dk = dev::smem_addr(stages + (size_t)st * C::STAGE);
-                    dev::mbar_arrive_expect_tx(bar, (uint32_t)have * 2 * C::HG * C::PB * C::R);
-                    #pragma unroll
-                    for (int r = 0; r < C::PER; ++r) {
-                        if (r >= have) break;
-                        if (id[r] < 0 || (int64_t)id[r] >= p.NB)
-                            dev::raise_error(p.err, PA_DEV_BAD_BLOCK);
-                        #pragma unroll
-                        for (int c = 0; c < C::CH; ++c) {
-                            const uint32_t off = c * C::SEGSTRIDE + r * C::HG * C::PB * 128;
-                            if constexpr (C::HG == 1) {   // map {D, Hkv, bs, NB}
-                                dev::tma_load_4d(dk + off, tmk, bar, c * C::EPS, kvh, 0, id[r], pol);
-                                dev::tma_load_4d(dk + C::TILE + off, tmv, bar, c * C::EPS, kvh, 0,
-                                                 id[r], pol);
-                            } else {                      // map {D, bs, Hkv, NB}, kvh the first head
-                                dev::tma_load_4d(dk + off, tmk, bar, c * C::EPS, 0, kvh, id[r], pol);
-                                dev::tma_load_4d(dk + C::TILE + off, tmv, bar, c * C::EPS, 0, kvh,
-                                                 id[r], pol);
-                            }
-                        }
-                    }
+                const uint32_t par = ((k / C::STAGES) & 1) ^ 1;
+                if (!dev::mbar_wait_bounded(empty0 + 8 * st, par)) {
+                    wait_timeout(p, 1);
+                    *s_abort = 1;
+                    stop = 1;
+                } else {
+                    issue_stage<C>(tmk, tmv, p, id, min(C::PER, nphys - (jb + jj * C::PER)), kvh,
+                                   st, stages, full0, pol);
                 }
             }
             stop = __shfl_sync(0xffffffffu, stop, 0);
@@ -524,10 +543,17 @@ __device__ __forceinline__ uint32_t to_f16x2(uint32_t w) {
     }
 }
 
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
-    __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_codes & 0xffffu),
-                                               __NV_E4M3);
-    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+// Four E4M3 codes (bytes 0..3 of w) to two f16x2 words: lo = (code 0, code 1),
+// hi = (code 2, code 3).  Every E4M3 value is an f16 value, so the conversion
+// is exact; the word is split into its 16-bit halves inside the asm so that
+// each half feeds its conversion directly.
+__device__ __forceinline__ void e4m3x4_to_f16x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    asm("{\n\t.reg .b16 l, h;\n\t"
+        "mov.b32 {l, h}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, l;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
 }
 
 template <class C>
@@ -613,12 +639,13 @@ __device__ __forceinline__ void mma_block(MmaState<C>& st, uint8_t* ktile_p, uin
                     ldsm_x4(chunk_addr<C>(ktile, lane & 7, ks + ((lane >> 3) & 1)), r0, r2, u0, u1);
                     r1 = r3 = 0u;
                 }
-                const uint32_t a00 = e4m3x2_to_f16x2(r0), a02 = e4m3x2_to_f16x2(r0 >> 16);
-                const uint32_t a01 = BS >= 16 ? e4m3x2_to_f16x2(r1) : 0u;
-                const uint32_t a03 = BS >= 16 ? e4m3x2_to_f16x2(r1 >> 16) : 0u;
-                const uint32_t a10 = e4m3x2_to_f16x2(r2), a12 = e4m3x2_to_f16x2(r2 >> 16);
-                const uint32_t a11 = BS >= 16 ? e4m3x2_to_f16x2(r3) : 0u;
-                const uint32_t a13 = BS >= 16 ? e4m3x2_to_f16x2(r3 >> 16) : 0u;
+                uint32_t a00, a02, a10, a12, a01 = 0u, a03 = 0u, a11 = 0u, a13 = 0u;
+                e4m3x4_to_f16x2(r0, a00, a02);
+                e4m3x4_to_f16x2(r2, a10, a12);
+                if constexpr (BS >= 16) {
+                    e4m3x4_to_f16x2(r1, a01, a03);
+                    e4m3x4_to_f16x2(r3, a11, a13);
+                }
                 #pragma unroll
                 for (int nh = 0; nh < S::NH; ++nh) {
                     mma16816<CT>(sc[mt][nh], a00, a01, a02, a03, st.qb[nh][ks][0], st.qb[nh][ks][1]);
@@ -731,38 +758,48 @@ __device__ __forceinline__ void mma_block(MmaState<C>& st, uint8_t* ktile_p, uin
         const int tig = lane & 3;
         const bool tail = nvalid < BS;
         if constexpr (BS >= 16) {
-            #pragma unroll
-            for (int kt = 0; kt < MT; ++kt) {
-                // bytes 0-1 of a fragment word: token 2tig; bytes 2-3: token 2tig + 1
-                uint32_t keep0 = 0xffffffffu, keep1 = 0xffffffffu;
-                if (tail) {
-                    const int t0 = kt * 16 + 2 * tig;
-                    keep0 = (t0 < nvalid ? 0x0000ffffu : 0u) | (t0 + 1 < nvalid ? 0xffff0000u : 0u);
-                    keep1 = (t0 + 8 < nvalid ? 0x0000ffffu : 0u) | (t0 + 9 < nvalid ? 0xffff0000u : 0u);
-                }
+            // one pass over the tile; TAIL: codes of tokens at or past nvalid are
+            // zeroed first (a zero weight times a NaN code would still be NaN)
+            auto pass = [&](auto tail_tag) {
+                constexpr bool TAIL = decltype(tail_tag)::value;
                 #pragma unroll
-                for (int md = 0; md < S::MD; md += 2) {
-                    // matrices: (tok 0-7, chunk md) (tok 8-15, md) (tok 0-7, md+1) (tok 8-15, md+1)
-                    uint32_t r0, r1, r2, r3;
-                    ldsm_x4_t(chunk_addr<C>(vt, kt * 16 + ((lane >> 3) & 1) * 8 + (lane & 7),
-                                            md + (lane >> 4)),
-                              r0, r1, r2, r3);
-                    const uint32_t s0 = __byte_perm(r0 & keep0, 0, 0x3120);
-                    const uint32_t s1 = __byte_perm(r1 & keep1, 0, 0x3120);
-                    const uint32_t s2 = __byte_perm(r2 & keep0, 0, 0x3120);
-                    const uint32_t s3 = __byte_perm(r3 & keep1, 0, 0x3120);
-                    const uint32_t a0 = e4m3x2_to_f16x2(s0), a1 = e4m3x2_to_f16x2(s0 >> 16);
-                    const uint32_t a2 = e4m3x2_to_f16x2(s1), a3 = e4m3x2_to_f16x2(s1 >> 16);
-                    const uint32_t b0 = e4m3x2_to_f16x2(s2), b1 = e4m3x2_to_f16x2(s2 >> 16);
-                    const uint32_t b2 = e4m3x2_to_f16x2(s3), b3 = e4m3x2_to_f16x2(s3 >> 16);
+                for (int kt = 0; kt < MT; ++kt) {
+                    // bytes 0-1 of a fragment word: token 2tig; bytes 2-3: token 2tig + 1
+                    uint32_t keep0 = 0xffffffffu, keep1 = 0xffffffffu;
+                    if constexpr (TAIL) {
+                        const int t0 = kt * 16 + 2 * tig;
+                        keep0 = (t0 < nvalid ? 0x0000ffffu : 0u) | (t0 + 1 < nvalid ? 0xffff0000u : 0u);
+                        keep1 = (t0 + 8 < nvalid ? 0x0000ffffu : 0u) | (t0 + 9 < nvalid ? 0xffff0000u : 0u);
+                    }
                     #pragma unroll
-                    for (int nh = 0; nh < S::NH; ++nh) {
-                        mma16816<CT>(st.o[nh][md], a0, a1, a2, a3, pb[kt][nh][0], pb[kt][nh][1]);
-                        mma16816<CT>(st.o[nh][md + 1], b0, b1, b2, b3, pb[kt][nh][0],
-                                     pb[kt][nh][1]);
+                    for (int md = 0; md < S::MD; md += 2) {
+                        // matrices: (tok 0-7, chunk md) (tok 8-15, md) (tok 0-7, md+1) (tok 8-15, md+1)
+                        uint32_t r0, r1, r2, r3;
+                        ldsm_x4_t(chunk_addr<C>(vt, kt * 16 + ((lane >> 3) & 1) * 8 + (lane & 7),
+                                                md + (lane >> 4)),
+                                  r0, r1, r2, r3);
+                        if constexpr (TAIL) {
+                            r0 &= keep0;
+                            r1 &= keep1;
+                            r2 &= keep0;
+                            r3 &= keep1;
+                        }
+                        uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
+                        e4m3x4_to_f16x2(__byte_perm(r0, 0, 0x3120), a0, a1);
+                        e4m3x4_to_f16x2(__byte_perm(r1, 0, 0x3120), a2, a3);
+                        e4m3x4_to_f16x2(__byte_perm(r2, 0, 0x3120), b0, b1);
+                        e4m3x4_to_f16x2(__byte_perm(r3, 0, 0x3120), b2, b3);
+                        #pragma unroll
+                        for (int nh = 0; nh < S::NH; ++nh) {
+                            mma16816<CT>(st.o[nh][md], a0, a1, a2, a3, pb[kt][nh][0], pb[kt][nh][1]);
+                            mma16816<CT>(st.o[nh][md + 1], b0, b1, b2, b3, pb[kt][nh][0],
+                                         pb[kt][nh][1]);
+                        }
                     }
                 }
-            }
+            };
+            if (tail) pass(std::true_type{});
+            else pass(std::false_type{});
         } else {
             uint32_t keep = 0xffffffffu;
             if (tail)
@@ -774,8 +811,8 @@ __device__ __forceinline__ void mma_block(MmaState<C>& st, uint8_t* ktile_p, uin
                 ldsm_x4_t(chunk_addr<C>(vt, lane & 7, md + (lane >> 3)), r[0], r[1], r[2], r[3]);
                 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const uint32_t sw = __byte_perm(r[i] & keep, 0, 0x3120);
-                    const uint32_t a0 = e4m3x2_to_f16x2(sw), a1 = e4m3x2_to_f16x2(sw >> 16);
+                    uint32_t a0, a1;
+                    e4m3x4_to_f16x2(__byte_perm(r[i] & keep, 0, 0x3120), a0, a1);
                     #pragma unroll
                     for (int nh = 0; nh < S::NH; ++nh) mma1688<CT>(st.o[nh][md + i], a0, a1, pb[0][nh][0]);
                 }
@@ -941,6 +978,10 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     // folds the prefix records in, so it waits there and streams its suffix
     // meanwhile; everything the kernels before that one wrote was complete
     // when the prefix kernel started (an ordinary launch).
+    if (threadIdx.x == C::NW * 32) {            // the producer's copies need both maps first
+        dev::prefetch_tensormap(&tmk);
+        dev::prefetch_tensormap(&tmv);
+    }
     if (p.fuse_prefix_blocks == 0) dev::grid_dependency_wait();
     extern __shared__ uint8_t smem_raw[];
     __shared__ int s_abort;
@@ -1051,10 +1092,6 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
         s_abort = 0;
         s_issued = 0;
         s_rec_issued = 0;
-    }
-    if (warp == C::NW && lane == 0) {
-        dev::prefetch_tensormap(&tmk);
-        dev::prefetch_tensormap(&tmv);
     }
     __syncthreads();
 
@@ -1256,69 +1293,103 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     }
 
     // ---- merge the warps' states (and the prefix records) and write -----
-    // Phase 1, one thread per query head: the common maximum M of its partial
-    // states (the consumer warps', or with head groups its warp's; then its
-    // prefix records), the weight 2^(m_i - M) of each and the sum L.  Phase 2,
-    // one thread per output element: the weighted sum of the partial outputs,
-    // with no exponential per element.  (The split-K identity: up to rounding
-    // order the same as merging the states one after another.)
+    // Phase 1, one warp per query head row: lane i takes partial state i (the
+    // consumer warps', or with head groups its warp's; then the prefix
+    // records), and the warp reduces the common maximum M, the weights
+    // 2^(m_i - M) and the sum L = sum of weight_i * l_i.  Phase 2, four
+    // neighbouring output elements per thread: the weighted sum of the partial
+    // outputs, with no exponential per element.  (The split-K identity: up to
+    // rounding order the same as merging the states one after another.)
     const int nsrc = C::HG > 1 ? 1 : C::NW;     // partial states per head
     const int npre = fuse_records ? p.prefix_parts : 0;
-    const int ncoef = nsrc + npre + 2;          // weights, then M and L
+    const int ncoef = nsrc + npre + 2;          // weights, then M and 1/L (0 for L = 0)
     float* coef = comb + C::COMBINE_FLOATS +
                   (staged && !rec_async ? (size_t)nh * p.max_parts * (C::D + 2) : 0);
     // partial state i of head row r (r = local query head: w * G + g with head groups)
     auto src_row = [&](int r, int i) { return C::HG > 1 ? (r / gc) * C::GC + r % gc : i * C::GC + r; };
     const size_t grow0 = ((size_t)s * p.Hq + h0) * p.max_parts;   // records of row 0 (global)
-    for (int r = threadIdx.x; r < nh; r += C::THREADS) {
+    auto src_ml = [&](int r, int i) -> float2 {
+        if (i < nsrc) {
+            const int q = src_row(r, i);
+            return make_float2(cm[q], cl[q]);
+        }
+        const int pp = i - nsrc;
+        return staged ? rec_ml[r * p.max_parts + pp] : p.ws_ml[grow0 + (size_t)r * p.max_parts + pp];
+    };
+    for (int r = warp; r < nh; r += C::THREADS / 32) {
         float M = -INFINITY;
-        for (int i = 0; i < nsrc; ++i) M = fmaxf(M, cm[src_row(r, i)]);
-        for (int pp = 0; pp < npre; ++pp)
-            M = fmaxf(M, staged ? rec_ml[r * p.max_parts + pp].x
-                                : p.ws_ml[grow0 + (size_t)r * p.max_parts + pp].x);
+        for (int i = lane; i < nsrc + npre; i += 32) M = fmaxf(M, src_ml(r, i).x);
+        #pragma unroll
+        for (int x = 16; x >= 1; x >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, x));
         float L = 0.f;
         float* c = coef + r * ncoef;
-        for (int i = 0; i < nsrc; ++i) {
-            const int q = src_row(r, i);
-            const float e = M == -INFINITY ? 0.f : exp2f(cm[q] - M);
-            c[i] = e;
-            L = fmaf(e, cl[q], L);
-        }
-        for (int pp = 0; pp < npre; ++pp) {
-            const float2 ml = staged ? rec_ml[r * p.max_parts + pp]
-                                     : p.ws_ml[grow0 + (size_t)r * p.max_parts + pp];
+        for (int i = lane; i < nsrc + npre; i += 32) {
+            const float2 ml = src_ml(r, i);
             const float e = M == -INFINITY ? 0.f : exp2f(ml.x - M);
-            c[nsrc + pp] = e;
+            c[i] = e;
             L = fmaf(e, ml.y, L);
         }
-        c[ncoef - 2] = M;
-        c[ncoef - 1] = L;
+        #pragma unroll
+        for (int x = 16; x >= 1; x >>= 1) L += __shfl_xor_sync(0xffffffffu, L, x);
+        if (lane == 0) {
+            c[ncoef - 2] = M;
+            c[ncoef - 1] = L > 0.f ? 1.f / L : 0.f;
+            if (!fuse_records && !(nparts == 1 && !p.force_ws)) {
+                const int h = C::HG > 1 ? h0 + (r / gc) * G + r % gc : h0 + r;
+                p.ws_ml[((size_t)s * p.Hq + h) * p.max_parts + part] = make_float2(M, L);
+            }
+        }
     }
     __syncthreads();
-    for (int idx = threadIdx.x; idx < nh * C::D; idx += C::THREADS) {
-        const int r = idx / C::D, d = idx % C::D;
+    constexpr int D4 = C::D / 4;
+    for (int idx = threadIdx.x; idx < nh * D4; idx += C::THREADS) {
+        const int r = idx / D4, d = (idx % D4) * 4;
         const int h = C::HG > 1 ? h0 + (r / gc) * G + r % gc : h0 + r;
         const float* c = coef + r * ncoef;
-        const float L = c[ncoef - 1];
-        float O = 0.f;
-        for (int i = 0; i < nsrc; ++i) O = fmaf(c[i], co[src_row(r, i) * C::D + d], O);
+        const float inv_l = c[ncoef - 1];
+        float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i = 0; i < nsrc; ++i) {
+            const float4 v = *reinterpret_cast<const float4*>(co + src_row(r, i) * C::D + d);
+            O.x = fmaf(c[i], v.x, O.x);
+            O.y = fmaf(c[i], v.y, O.y);
+            O.z = fmaf(c[i], v.z, O.z);
+            O.w = fmaf(c[i], v.w, O.w);
+        }
+        const size_t o0 = ((size_t)s * p.Hq + h) * C::D + d;
         if (fuse_records) {
             // the prefix records' o is already times v_scale
-            float Op = 0.f;
-            for (int pp = 0; pp < npre; ++pp)
-                Op = fmaf(c[nsrc + pp],
-                          staged ? rec_o[((size_t)r * p.max_parts + pp) * C::D + d]
-                                 : p.ws_o[(grow0 + (size_t)r * p.max_parts + pp) * C::D + d],
-                          Op);
-            dev::store_out<C::QT>(p.out, ((size_t)s * p.Hq + h) * C::D + d,
-                                  L > 0.f ? fmaf(O, p.v_scale, Op) / L : 0.f);
+            float4 Op = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int pp = 0; pp < npre; ++pp) {
+                const float w = c[nsrc + pp];
+                float4 v;
+                if (staged) {
+                    v = *reinterpret_cast<const float4*>(rec_o + ((size_t)r * p.max_parts + pp) * C::D + d);
+                } else {
+                    const float* g = p.ws_o + (grow0 + (size_t)r * p.max_parts + pp) * C::D + d;
+                    v = make_float4(g[0], g[1], g[2], g[3]);
+                }
+                Op.x = fmaf(w, v.x, Op.x);
+                Op.y = fmaf(w, v.y, Op.y);
+                Op.z = fmaf(w, v.z, Op.z);
+                Op.w = fmaf(w, v.w, Op.w);
+            }
+            dev::store_out<C::QT>(p.out, o0 + 0, fmaf(O.x, p.v_scale, Op.x) * inv_l);
+            dev::store_out<C::QT>(p.out, o0 + 1, fmaf(O.y, p.v_scale, Op.y) * inv_l);
+            dev::store_out<C::QT>(p.out, o0 + 2, fmaf(O.z, p.v_scale, Op.z) * inv_l);
+            dev::store_out<C::QT>(p.out, o0 + 3, fmaf(O.w, p.v_scale, Op.w) * inv_l);
         } else if (nparts == 1 && !p.force_ws) {
-            dev::store_out<C::QT>(p.out, ((size_t)s * p.Hq + h) * C::D + d,
-                                  L > 0.f ? (O / L) * p.v_scale : 0.f);
+            const float f = inv_l * p.v_scale;
+            dev::store_out<C::QT>(p.out, o0 + 0, O.x * f);
+            dev::store_out<C::QT>(p.out, o0 + 1, O.y * f);
+            dev::store_out<C::QT>(p.out, o0 + 2, O.z * f);
+            dev::store_out<C::QT>(p.out, o0 + 3, O.w * f);
         } else {
             const size_t row = ((size_t)s * p.Hq + h) * p.max_parts + part;
-            p.ws_o[row * C::D + d] = O * p.v_scale;
-            if (d == 0) p.ws_ml[row] = make_float2(c[ncoef - 2], L);
+            float* w = p.ws_o + row * C::D + d;
+            w[0] = O.x * p.v_scale;
+            w[1] = O.y * p.v_scale;
+            w[2] = O.z * p.v_scale;
+            w[3] = O.w * p.v_scale;
         }
     }
 }
