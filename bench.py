@@ -360,7 +360,9 @@ def csrc_sha256() -> str:
 def device_leg(args, cfg, pa, dev, seed, steps, warmup, partition=-1):
     """Append [+ copy-on-write] + decode on device-resident inputs: W untimed
     steps, then K steps timed with CUDA events on the launching stream, clocks
-    sampled inside the timed region."""
+    sampled inside the timed region.  The timed steps replay the step's kernels
+    from CUDA graphs (unless --no-graph); 20 eagerly launched steps are timed
+    before them for comparison."""
     stream = torch.cuda.current_stream()
     inp = wl.make_decode_inputs(cfg, seed=seed, device=dev)
     S, Hq, D = inp.q.shape
@@ -391,16 +393,27 @@ def device_leg(args, cfg, pa, dev, seed, steps, warmup, partition=-1):
             pa.pa_decode(out_t, q_t, kc, vc, tables, lens, max_ctx, inp.scale, inp.k_scale,
                          inp.v_scale, part, ws if ws_bytes else None)
 
-    def step(ev=None):
-        if ev is not None:
-            ev[2].record(stream)
+    def append():
         if pairs.numel():
             pa.pa_copy_blocks(kc, vc, pairs)
         pa.pa_reshape_and_cache(inp.key_new, inp.value_new, kc, vc, inp.slot_mapping,
                                 inp.k_scale, inp.v_scale)
+
+    graphs = None
+
+    def step(ev=None):
+        if ev is not None:
+            ev[2].record(stream)
+        if graphs:
+            graphs[0].replay()
+        else:
+            append()
         if ev is not None:
             ev[0].record(stream)
-        decode(out, inp.q, inp.block_tables, inp.context_lens)
+        if graphs:
+            graphs[1].replay()
+        else:
+            decode(out, inp.q, inp.block_tables, inp.context_lens)
         if ev is not None:
             ev[1].record(stream)
 
@@ -413,6 +426,36 @@ def device_leg(args, cfg, pa, dev, seed, steps, warmup, partition=-1):
     step()
     torch.cuda.synchronize()
     launches_per_step = pa.pa_launch_count() - n0
+
+    def timed(nsteps):
+        evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(nsteps)]
+        for i in range(nsteps):
+            step(evs[i])
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b, _ in evs) / nsteps
+
+    # The decode step as a serving loop runs it: the same kernels launched from
+    # two CUDA graphs (append + copy-on-write, decode) captured once, so the
+    # timed region measures the GPU's work rather than the host's launch rate.
+    # The eagerly launched step is timed beside it (decode_ms_eager).
+    eager_dec = timed(min(steps, 20))
+    graph_note = None
+    if not args.no_graph:
+        try:
+            cap = [torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()]
+            with torch.cuda.graph(cap[0]):
+                append()
+            with torch.cuda.graph(cap[1]):
+                decode(out, inp.q, inp.block_tables, inp.context_lens)
+            graphs = cap
+            for _ in range(warmup):
+                step()
+            torch.cuda.synchronize()
+            assert pa.pa_device_status() == 0
+        except RuntimeError as e:      # capture refused: time the eager loop
+            graphs = None
+            graph_note = f"eager (graph capture failed: {str(e).splitlines()[0][:120]})"
+            torch.cuda.synchronize()
 
     dist = torch.distributed.is_available() and torch.distributed.is_initialized()
     if dist:
@@ -434,11 +477,13 @@ def device_leg(args, cfg, pa, dev, seed, steps, warmup, partition=-1):
         torch.distributed.barrier()
     dec_ms = [a.elapsed_time(b) for a, b, _ in evs]
     res = {"ms": t0.elapsed_time(t1), "dec_avg": sum(dec_ms) / len(dec_ms),
+           "dec_eager": eager_dec,
+           "launch": "cuda graph" if graphs else (graph_note or "eager"),
            "app_avg": sum(c.elapsed_time(a) for a, _, c in evs) / len(evs),
            "nbytes": nbytes, "part": part, "shared": shared, "S": S,
            "launches_per_step": launches_per_step, "clocks": clk,
            "kv_gb": nbytes["kv"] / 1e9}
-    del inp, ws, out, kc, vc
+    del graphs, inp, ws, out, kc, vc
     torch.cuda.empty_cache()
     return res
 
@@ -522,7 +567,8 @@ def run_gpu(args, cfg, rank, world, local_rank):
     for name, (wcfg, x, xv, xms) in extras.items():
         workloads[name] = {
             "value": round(xv, 2), "unit": "GB/s", "ms_per_step": round(xms, 4),
-            "decode_ms": round(x["dec_avg"], 4), "append_cow_ms": round(x["app_avg"], 4),
+            "decode_ms": round(x["dec_avg"], 4), "decode_ms_eager": round(x["dec_eager"], 4),
+            "launch": x["launch"], "append_cow_ms": round(x["app_avg"], 4),
             "seqs_per_s": round(x["S"] * world / (xms * 1e-3), 1), "partition": x["part"],
             "path": "pa_decode_shared_prefix" if x["shared"] else "pa_decode",
             "unique_kv_gbs": round(x["nbytes"]["unique_kv"] / (x["dec_avg"] * 1e-3) / 1e9, 1),
@@ -544,6 +590,8 @@ def run_gpu(args, cfg, rank, world, local_rank):
         "pct_of_hbm_peak": {"measured_copy": round(100 * value / world / peak, 2),
                             "spec_8000": round(100 * value / world / 8000.0, 2)},
         "decode_ms": round(r["dec_avg"], 4),
+        "decode_ms_eager": round(r["dec_eager"], 4),
+        "launch": r["launch"],
         "append_cow_ms": round(r["app_avg"], 4),
         "unique_kv_gbs": round(nbytes["unique_kv"] / (r["dec_avg"] * 1e-3) / 1e9, 1),
         "roofline": roof,
@@ -966,6 +1014,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time the eagerly launched step instead of its CUDA-graph replay")
     ap.add_argument("--seqs", type=int, default=0,
                     help="profiling only: a sub-batch of this many sequences of the workload")
     ap.add_argument("--no-shared-prefix", action="store_true",

@@ -134,11 +134,17 @@ def pa_launch_count() -> int:
     return int(lib().pa_launch_count())
 
 
+_CUDA_AVAILABLE = None
+
+
 def _stream(stream) -> ctypes.c_void_p:
+    global _CUDA_AVAILABLE
     if stream is None:
-        if not torch.cuda.is_available():       # host-only calls (argument checks)
+        if _CUDA_AVAILABLE is None:
+            _CUDA_AVAILABLE = torch.cuda.is_available()
+        if not _CUDA_AVAILABLE:                 # host-only calls (argument checks)
             return ctypes.c_void_p(0)
-        stream = torch.cuda.current_stream()
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     if isinstance(stream, torch.cuda.Stream):
         stream = stream.cuda_stream
     return ctypes.c_void_p(int(stream))

@@ -43,10 +43,10 @@ cudaError_t launch_one(const Launch& L) {
     } else if (L.balanced) {
         auto kern = decode_balanced<C>;
         const int smem = static_cast<int>(BalancedSmem<C>::bytes(L.mma ? L.G : L.gc));
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        cudaError_t e = dev::ensure_dynamic_smem<decode_balanced<C>>((size_t)smem);
         if (e != cudaSuccess) return e;
         int per_sm = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, C::THREADS, smem);
+        e = dev::occupancy<decode_balanced<C>>(&per_sm, C::THREADS, (size_t)smem);
         if (e != cudaSuccess) return e;
         if (per_sm < 1) per_sm = 1;
         int ctas = per_sm * L.num_sms;
@@ -65,14 +65,12 @@ cudaError_t launch_one(const Launch& L) {
         // only if it costs no resident CTA per SM.
         auto kern = decode_partition<C, true>;
         const size_t big = C::SMEM + group_merge_bytes<C>(L.G);
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(big));
+        cudaError_t e = dev::ensure_dynamic_smem<decode_partition<C, true>>(big);
         if (e != cudaSuccess) return e;
         int occ1 = 0, occ2 = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ1, decode_partition<C, false>,
-                                                          C::THREADS, C::SMEM);
+        e = dev::occupancy<decode_partition<C, false>>(&occ1, C::THREADS, C::SMEM);
         if (e != cudaSuccess) return e;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ2, kern, C::THREADS, big);
+        e = dev::occupancy<decode_partition<C, true>>(&occ2, C::THREADS, big);
         if (e != cudaSuccess) return e;
         if (occ2 >= occ1 && occ2 > 0) {
             return dev::launch_pdl(kern, L.grid, dim3(C::THREADS), big, L.stream, L.tmk, L.tmv,
@@ -87,9 +85,8 @@ cudaError_t launch_one(const Launch& L) {
     }
     auto kern = decode_partition<C, false>;
     const size_t smem = C::SMEM + (size_t)p.rec_smem;   // + the shared-prefix records
-    // opt in to > 48 KB of dynamic shared memory (idempotent, cheap)
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    // opt in to > 48 KB of dynamic shared memory
+    cudaError_t e = dev::ensure_dynamic_smem<decode_partition<C, false>>(smem);
     if (e != cudaSuccess) return e;
     return dev::launch_pdl(kern, grid, dim3(C::THREADS), smem, L.stream, L.tmk, L.tmv, p);
 }

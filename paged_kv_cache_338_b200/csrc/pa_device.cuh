@@ -8,6 +8,7 @@
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <utility>
 
@@ -216,6 +217,52 @@ inline cudaError_t launch_pdl(void (*kern)(Params...), dim3 grid, dim3 block, si
     cfg.numAttrs = 1;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
     if (e == cudaSuccess) note_launch();
+    return e;
+}
+
+// Opt kernel Kern in to `bytes` of dynamic shared memory on the current device.
+// The attribute belongs to the kernel in each device's context; a driver call
+// per launch costs microseconds of host time, so the largest size already set
+// is remembered per device and a launch that needs no more skips the call.
+template <auto Kern>
+inline cudaError_t ensure_dynamic_smem(size_t bytes) {
+    constexpr int kDevices = 64;
+    static std::atomic<int> set_bytes[kDevices] = {};
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevices)
+        return cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (set_bytes[dev].load(std::memory_order_acquire) >= (int)bytes) return cudaSuccess;
+    const cudaError_t e =
+        cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) {
+        int cur = set_bytes[dev].load(std::memory_order_relaxed);
+        while (cur < (int)bytes &&
+               !set_bytes[dev].compare_exchange_weak(cur, (int)bytes, std::memory_order_release))
+        {
+        }
+    }
+    return e;
+}
+
+// cudaOccupancyMaxActiveBlocksPerMultiprocessor for kernel Kern, remembered
+// per device for the last shared-memory size asked (the launchers ask the same
+// sizes call after call).
+template <auto Kern>
+inline cudaError_t occupancy(int* per_sm, int threads, size_t smem) {
+    constexpr int kDevices = 64;
+    static std::atomic<unsigned long long> memo[kDevices] = {};   // (smem + 1) << 32 | blocks
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevices)
+        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(per_sm, Kern, threads, smem);
+    const unsigned long long m = memo[dev].load(std::memory_order_acquire);
+    if ((m >> 32) == (unsigned long long)smem + 1) {
+        *per_sm = (int)(m & 0xffffffffu);
+        return cudaSuccess;
+    }
+    const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(per_sm, Kern, threads, smem);
+    if (e == cudaSuccess)
+        memo[dev].store((((unsigned long long)smem + 1) << 32) | (unsigned)*per_sm,
+                        std::memory_order_release);
     return e;
 }
 

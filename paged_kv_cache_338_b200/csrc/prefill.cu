@@ -730,9 +730,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
 template <int DT, int D>
 cudaError_t launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                    const Params& p, dim3 grid, cudaStream_t st) {
-    // once per instantiation (a function-local static initialises thread-safely)
-    static const cudaError_t attr = cudaFuncSetAttribute(
-        prefill_kernel<DT, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Smem<D>::BYTES);
+    const cudaError_t attr = pa::dev::ensure_dynamic_smem<prefill_kernel<DT, D>>(Smem<D>::BYTES);
     if (attr != cudaSuccess) return attr;
     return launch_pdl(prefill_kernel<DT, D>, grid, dim3(kThreads), (size_t)Smem<D>::BYTES, st, mq,
                       mk, mv, p);
