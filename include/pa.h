@@ -252,8 +252,9 @@ pa_status pa_decode_partition_group(int S, int Hq, int Hkv, int D, int bs, pa_dt
 /*
  * Kernel selection and tuning for pa_decode (process-wide; for tests and
  * tuning), a bit mask:
- *   1: CUDA-core consumer everywhere (otherwise grouped-query heads with
- *      f16 / bf16 / fp8 caches and D <= 128 use the tensor-core consumer);
+ *   1: CUDA-core consumer everywhere (otherwise f16 / bf16 / fp8 caches with
+ *      D <= 128 use the tensor-core consumer, multi-head attention included:
+ *      its one query row per kv head fills one of the tile's eight);
  *   2: stream K/V with an L2 evict-first hint;
  *   4: partition-major grid (the kv heads of one partition are neighbouring
  *      CTAs, so the interleaved heads of a block are read at about the same

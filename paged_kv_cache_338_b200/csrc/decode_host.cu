@@ -219,7 +219,7 @@ extern "C" pa_status pa_decode_partition_group(int S, int Hq, int Hkv, int D, in
     if (chk) return chk;
     const int G = Hq / Hkv;
     const int sel = g_select.load();
-    const bool use_mma = !(sel & 1) && G >= 2 && D <= 128 && cache_dt != PA_F32;
+    const bool use_mma = !(sel & 1) && D <= 128 && cache_dt != PA_F32;
     const int64_t max_parts = partition > 0 ? parts_for(max_ctx, partition) : 1;
     *group = 1;
     if (use_mma && max_parts > 1)
@@ -282,7 +282,7 @@ pa_status pa::decode_impl(void* out, const void* q, pa_dtype q_dt, const void* k
     if (fuse && 4 * (4 * 16 * (D + 2) + (int64_t)G * (4 + prefix_parts + 2)) > 48 * 1024)
         return fail(PA_ERR_UNSUPPORTED, "shared prefix of %d partitions is too long", prefix_parts);
     const int sel = g_select.load();
-    const bool use_mma = !(sel & 1) && G >= 2 && D <= 128 && cache_dt != PA_F32;
+    const bool use_mma = !(sel & 1) && D <= 128 && cache_dt != PA_F32;
     const int gc_simt = G < (D == 256 ? 2 : 4) ? G : (D == 256 ? 2 : 4);
     const int gc = use_mma ? G : gc_simt;
     const int chunks = use_mma ? 1 : G / gc_simt;

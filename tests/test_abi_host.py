@@ -105,9 +105,10 @@ def test_decode_select_modes():
 def test_partition_group_plan():
     """The grouped split-K plan (host logic, 148 SMs): the 4 x 100k bf16
     workload with 512-token partitions streams 16 partitions per CTA (416 CTAs,
-    one wave of 3 per SM); long partitions, a single pass, the CUDA-core
-    consumer and fp32 caches stay at one; the test bit forces three.  Shapes
-    pa_decode refuses are refused here with the same codes."""
+    one wave of 3 per SM); multi-head attention (the tensor-core consumer too)
+    groups as well; long partitions, a single pass, the CUDA-core consumer and
+    fp32 caches stay at one; the test bit forces three.  Shapes pa_decode
+    refuses are refused here with the same codes."""
     bf, f8, f16, f32 = torch.bfloat16, torch.float8_e4m3fn, torch.float16, torch.float32
 
     def grp(S, Hq, Hkv, D, ct, ctx, part, sms, bs=16, qt=None):
@@ -119,7 +120,7 @@ def test_partition_group_plan():
         assert grp(4, 32, 8, 128, f8, 100000, 512, 148) == 16
         assert grp(128, 32, 8, 128, bf, 8192, 2048, 148) == 1   # 1 MB partitions
         assert grp(4, 32, 8, 128, bf, 100000, 0, 148) == 1      # single pass
-        assert grp(4, 32, 32, 128, f16, 100000, 512, 148) == 1  # MHA: CUDA-core
+        assert grp(4, 32, 32, 128, f16, 100000, 512, 148) > 1   # MHA: tensor-core consumer
         assert grp(4, 32, 8, 128, f32, 100000, 512, 148) == 1
         assert grp(4, 32, 8, 128, bf, 400, 512, 148) == 1       # one partition
         # never more partitions per CTA than a sequence has; no part-filled

@@ -96,7 +96,8 @@ class DecodeConfig:
 CONFIGS = {
     1: DecodeConfig("tiny_paged_decode_fp32", 4, 4, 4, 64, 16, "f32", "f32", 0, 0,
                     fixed_lens=(17, 33, 64, 100), fixed_num_blocks=24, slack=0.0),
-    2: DecodeConfig("llama2_7b_mha_fp16_b64", 64, 32, 32, 128, 16, "f16", "f16", 512, 2048),
+    2: DecodeConfig("llama2_7b_mha_fp16_b64", 64, 32, 32, 128, 16, "f16", "f16", 512, 2048,
+                    partition=1024),
     3: DecodeConfig("llama3_8b_gqa_bf16_b128", 128, 32, 8, 128, 16, "bf16", "bf16", 1024, 8192),
     4: DecodeConfig("long_context_splitk_bf16_4x100k", 4, 32, 8, 128, 16, "bf16", "bf16", 0, 0,
                     fixed_lens=(100000,) * 4, partition=512, slack=0.02),
