@@ -276,7 +276,8 @@ pa_status pa_decode_partition_group(int S, int Hq, int Hkv, int D, int bs, pa_dt
  *      consumer and Hkv a multiple of 4, a CTA of the partition kernel serves
  *      four neighbouring kv heads (one per consumer warp) and reads each
  *      block's rows of all four with one tensor-map copy per 128-byte
- *      segment (not with grouped partitions, the balanced grid or the
+ *      segment (grouped partitions included: each warp then closes its
+ *      head's partition records alone; not with the balanced grid or the
  *      shared-prefix decode's suffix passes).
  * Default 4.  Every setting computes the same function.
  */

@@ -35,8 +35,9 @@ std::atomic<int> g_select{4};
 // units: CTAs one partition per CTA would need per partition index (sequences
 // x kv heads x head chunks); part_bytes: K/V bytes of one partition of one kv
 // head.  Partitions of 512 KB or more are long enough on their own: g = 1.
-int plan_part_group(int64_t units, int64_t max_parts, int64_t part_bytes, int num_sms) {
-    if (max_parts <= 1 || part_bytes >= (512 << 10)) return 1;
+int plan_part_group(int64_t units, int64_t max_parts, int64_t part_bytes, int num_sms,
+                    int heads_per_cta = 1) {
+    if (max_parts <= 1 || part_bytes / heads_per_cta >= (512 << 10)) return 1;
     const int64_t slots = 3LL * (num_sms > 0 ? num_sms : 148);
     double best = 0.0;
     int group = 1;
@@ -49,6 +50,16 @@ int plan_part_group(int64_t units, int64_t max_parts, int64_t part_bytes, int nu
         }
     }
     return group;
+}
+
+// Four kv heads per CTA (head groups) for the partition kernel: the
+// tensor-core consumer, Hkv a multiple of 4, a stage of the four heads' K and
+// V at most 32 KB, and select bit 32 off.  (The callers add the paths that
+// keep one head: the balanced grid and the shared-prefix passes.)
+bool decode_heads_per_cta(bool use_mma, int stage_tokens, int D, pa_dtype cache_dt, int Hkv,
+                          int sel) {
+    return use_mma && 2 * 4 * stage_tokens * D * elem_size(cache_dt) <= 32 * 1024 &&
+           Hkv % 4 == 0 && !(sel & 32);
 }
 
 // SMs of the current device (cached per device; 148 if the query fails).
@@ -221,12 +232,14 @@ extern "C" pa_status pa_decode_partition_group(int S, int Hq, int Hkv, int D, in
     const int sel = g_select.load();
     const bool use_mma = !(sel & 1) && D <= 128 && cache_dt != PA_F32;
     const int64_t max_parts = partition > 0 ? parts_for(max_ctx, partition) : 1;
+    const bool pair = bs == 8 && partition % 16 == 0;
+    const int hg = decode_heads_per_cta(use_mma, pair ? 16 : bs, D, cache_dt, Hkv, sel) ? 4 : 1;
     *group = 1;
     if (use_mma && max_parts > 1)
         *group = (sel & 8) ? 3
-                           : plan_part_group((int64_t)S * Hkv, max_parts,
-                                             (int64_t)partition * D * elem_size(cache_dt) * 2,
-                                             num_sms > 0 ? num_sms : sm_count());
+                           : plan_part_group((int64_t)S * Hkv / hg, max_parts,
+                                             (int64_t)partition * D * elem_size(cache_dt) * 2 * hg,
+                                             num_sms > 0 ? num_sms : sm_count(), hg);
     return PA_OK;
 }
 
@@ -296,23 +309,22 @@ pa_status pa::decode_impl(void* out, const void* q, pa_dtype q_dt, const void* k
     const bool pair = bs == 8 && !balanced && !fuse && prefix_parts == 0 && !force_ws &&
                       partition % 16 == 0;
     const int stage_tokens = pair ? 16 : bs;
-    int part_group = 1;
-    if (use_mma && !balanced && !fuse && prefix_parts == 0 && !force_ws && max_parts > 1)
-        part_group = (sel & 8) ? 3
-                               : plan_part_group((int64_t)S * Hkv * chunks, max_parts,
-                                                 (int64_t)partition * D * elem_size(cache_dt) * 2,
-                                                 num_sms);
     // four neighbouring kv heads per CTA (one per consumer warp), read by one
     // tensor-map copy per block and segment, where a stage of the four heads'
     // K and V is at most 32 KB (two stages in flight at three CTAs per SM);
-    // one head per CTA with bit 32, the CUDA-core consumer, grouped or
-    // balanced partitions and the shared-prefix suffix passes (short suffixes
-    // measured slower in groups: four times fewer CTAs to hide their latency)
-    const bool hg_fits = 2 * 4 * stage_tokens * D * elem_size(cache_dt) <= 32 * 1024;
-    const int hg = use_mma && hg_fits && Hkv % 4 == 0 && !(sel & 32) && !balanced && !items &&
-                           !force_ws && prefix_parts == 0 && part_group == 1
+    // one head per CTA with bit 32, the CUDA-core consumer, the balanced grid
+    // and the shared-prefix suffix passes (short suffixes measured slower in
+    // groups: four times fewer CTAs to hide their latency)
+    const int hg = decode_heads_per_cta(use_mma, stage_tokens, D, cache_dt, Hkv, sel) &&
+                           !balanced && !items && !force_ws && prefix_parts == 0
                        ? 4
                        : 1;
+    int part_group = 1;
+    if (use_mma && !balanced && !fuse && prefix_parts == 0 && !force_ws && max_parts > 1)
+        part_group = (sel & 8) ? 3
+                               : plan_part_group((int64_t)S * Hkv * chunks / hg, max_parts,
+                                                 (int64_t)partition * D * elem_size(cache_dt) * 2 * hg,
+                                                 num_sms, hg);
     const int64_t grid_parts = fuse ? 1
                                : prefix_parts > 0 ? max_parts - prefix_parts
                                                   : (max_parts + part_group - 1) / part_group;

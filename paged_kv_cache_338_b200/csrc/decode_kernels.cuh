@@ -1102,12 +1102,13 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
 
     using State = typename std::conditional<C::MMA, MmaState<C>, SimtState<C>>::type;
     State st;
-    static_assert(!(GROUPED && C::HG > 1), "grouped partitions take one head per CTA");
     if constexpr (GROUPED) {
         // Grouped partitions: the producer streams the blocks of all nq
         // partitions without a break; the consumers close each partition with
         // a warp merge through a dedicated area (the stages keep streaming)
-        // and write its record, exactly as nq one-partition CTAs would.
+        // and write its record, exactly as nq one-partition CTAs would.  With
+        // head groups each warp holds a whole head's state and closes the
+        // partition alone, through its own slice of that area.
         const int gh = gc;
         float* gm = reinterpret_cast<float*>(after + 16 * C::STAGES);
         float* gl = gm + C::NW * gh;
@@ -1118,6 +1119,48 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                        min(nblk * C::PER, nphys_all - blk0 * C::PER), kvh, stages, full0, empty0,
                        &s_abort, &k, pblk0_guess, pre);
             if (lane == 0) s_issued = k;
+        } else if constexpr (C::HG > 1) {
+            // warp w: kv head kvh + w, its tiles in every stage
+            const int hw = warp;
+            mma_load_q<C>(st, p, s, h0 + hw * G, G);
+            bool stop = false;
+            for (int qq = 0; qq < nq && !stop; ++qq) {
+                const int jb = qq * p.part_blocks, je = min(jb + p.part_blocks, nblk);
+                for (int j = jb; j < je; ++j) {
+                    const int stg = j % C::STAGES;
+                    if (!dev::mbar_wait_bounded(full0 + 8 * stg, (j / C::STAGES) & 1)) {
+                        if (lane == 0) { wait_timeout(p, 2); s_abort = 1; }
+                        stop = true;
+                        break;
+                    }
+                    uint8_t* kt = stages + (size_t)stg * C::STAGE + hw * C::PB * 128;
+                    const int nvalid = min(C::BS, n - (blk0 + j) * C::BS);
+                    mma_block<C>(st, kt, kt + C::TILE, nvalid, p.qk_scale);
+                    __syncwarp();
+                    if (lane == 0) dev::mbar_arrive(empty0 + 8 * stg);
+                    if (*(volatile int*)&s_abort) { stop = true; break; }
+                }
+                if (stop) break;
+                // this partition's record of the warp's query heads (the output
+                // itself for a sequence of one partition: the merge skips it)
+                mma_publish<C>(st, gm + hw * gh, gl + hw * gh, go + (size_t)hw * gh * C::D, 0, G, gh);
+                __syncwarp();
+                for (int idx = lane; idx < G * C::D; idx += 32) {
+                    const int g = idx / C::D, d = idx % C::D;
+                    const int h = h0 + hw * G + g;
+                    const float O = go[((size_t)hw * gh + g) * C::D + d], L = gl[hw * gh + g];
+                    if (nparts == 1) {
+                        dev::store_out<C::QT>(p.out, ((size_t)s * p.Hq + h) * C::D + d,
+                                              L > 0.f ? (O / L) * p.v_scale : 0.f);
+                    } else {
+                        const size_t row = ((size_t)s * p.Hq + h) * p.max_parts + q0 + qq;
+                        p.ws_o[row * C::D + d] = O * p.v_scale;
+                        if (d == 0) p.ws_ml[row] = make_float2(gm[hw * gh + g], L);
+                    }
+                }
+                __syncwarp();
+                mma_reset<C>(st);
+            }
         } else {
             if constexpr (C::MMA) mma_load_q<C>(st, p, s, h0, G);
             else simt_load_q<C>(st, p, s, h0);

@@ -60,7 +60,7 @@ cudaError_t launch_one(const Launch& L) {
                                L.stream, L.tmk, L.tmv, L.p);
     }
     Params p = L.p;
-    if constexpr (C::MMA && C::HG == 1) if (p.part_group > 1) {
+    if constexpr (C::MMA) if (p.part_group > 1) {
         // Grouped partitions need a warp-merge area of their own; use them
         // only if it costs no resident CTA per SM.
         auto kern = decode_partition<C, true>;

@@ -104,11 +104,12 @@ def test_decode_select_modes():
 
 def test_partition_group_plan():
     """The grouped split-K plan (host logic, 148 SMs): the 4 x 100k bf16
-    workload with 512-token partitions streams 16 partitions per CTA (416 CTAs,
-    one wave of 3 per SM); multi-head attention (the tensor-core consumer too)
-    groups as well; long partitions, a single pass, the CUDA-core consumer and
-    fp32 caches stay at one; the test bit forces three.  Shapes pa_decode
-    refuses are refused here with the same codes."""
+    workload with 512-token partitions streams 4 partitions per CTA of four kv
+    heads (392 CTAs, one wave of 3 per SM), and 16 with one kv head per CTA
+    (416 CTAs); multi-head attention (the tensor-core consumer too) groups as
+    well; long partitions, a single pass, the CUDA-core consumer and fp32
+    caches stay at one; the test bit forces three.  Shapes pa_decode refuses
+    are refused here with the same codes."""
     bf, f8, f16, f32 = torch.bfloat16, torch.float8_e4m3fn, torch.float16, torch.float32
 
     def grp(S, Hq, Hkv, D, ct, ctx, part, sms, bs=16, qt=None):
@@ -116,8 +117,8 @@ def test_partition_group_plan():
         return pa.pa_decode_partition_group(S, Hq, Hkv, D, bs, qt, ct, ctx, part, sms)
     try:
         pa.pa_decode_select(pa.DECODE_DEFAULT)
-        assert grp(4, 32, 8, 128, bf, 100000, 512, 148) == 16
-        assert grp(4, 32, 8, 128, f8, 100000, 512, 148) == 16
+        assert grp(4, 32, 8, 128, bf, 100000, 512, 148) == 4
+        assert grp(4, 32, 8, 128, f8, 100000, 512, 148) == 4
         assert grp(128, 32, 8, 128, bf, 8192, 2048, 148) == 1   # 1 MB partitions
         assert grp(4, 32, 8, 128, bf, 100000, 0, 148) == 1      # single pass
         assert grp(4, 32, 32, 128, f16, 100000, 512, 148) > 1   # MHA: tensor-core consumer
@@ -128,9 +129,11 @@ def test_partition_group_plan():
         for S, ctx in ((1, 20000), (2, 50000), (16, 30000), (64, 9000)):
             g = grp(S, 32, 8, 128, bf, ctx, 256, 148)
             parts = -(-ctx // 256)
-            ctas = S * 8 * (-(-parts // g))
+            ctas = S * 2 * (-(-parts // g))                      # two CTAs of four kv heads
             assert 1 <= g <= parts
-            assert not (444 < ctas < 2 * 444 and S * 8 * (-(-parts // (g + 1))) <= 444)
+            assert not (444 < ctas < 2 * 444 and S * 2 * (-(-parts // (g + 1))) <= 444)
+        pa.pa_decode_select(pa.DECODE_DEFAULT | pa.DECODE_ONE_HEAD_PER_CTA)
+        assert grp(4, 32, 8, 128, bf, 100000, 512, 148) == 16
         pa.pa_decode_select(pa.DECODE_DEFAULT | pa.DECODE_GROUP_PARTITIONS)
         assert grp(4, 32, 8, 128, bf, 100000, 512, 148) == 3
         pa.pa_decode_select(pa.DECODE_DEFAULT | pa.DECODE_SIMT_ONLY)
