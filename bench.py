@@ -830,6 +830,8 @@ def prefill_oracle_rate(cfg: wl.PrefillConfig, seed: int, budget_s: float) -> di
 
 def run_gpu_prefill(args, cfg: wl.PrefillConfig, rank, world, local_rank):
     import paged_kv_cache_338_b200 as pa
+    if args.decode_select is not None:
+        pa.pa_decode_select(args.decode_select)
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()

@@ -250,7 +250,7 @@ pa_status pa_decode_partition_group(int S, int Hq, int Hkv, int D, int bs, pa_dt
                                     int* group);
 
 /*
- * Kernel selection and tuning for pa_decode (process-wide; for tests and
+ * Kernel selection and tuning for pa_decode and pa_prefill (process-wide; for tests and
  * tuning), a bit mask:
  *   1: CUDA-core consumer everywhere (otherwise f16 / bf16 / fp8 caches with
  *      D <= 128 use the tensor-core consumer, multi-head attention included:
@@ -279,7 +279,14 @@ pa_status pa_decode_partition_group(int S, int Hq, int Hkv, int D, int bs, pa_dt
  *      segment (grouped partitions included: each warp then closes its
  *      head's partition records alone; not with the balanced grid or the
  *      shared-prefix decode's suffix passes).
- * Default 4.  Every setting computes the same function.
+ *  64: pa_prefill with D = 128 (outside the shared-prefix decode) runs the
+ *      two query tiles of a pair on a cluster of two CTAs whose tensor-core
+ *      instructions span both SMs (cta_group::2: each SM loads half of every
+ *      K and V tile and keeps two score buffers, so the scores of the next key
+ *      tile are computed while the softmax works on this one) instead of one
+ *      CTA per pair.  Same results; measured about 6 % slower.
+ * Default 4; a mode outside [0, 127] is refused (PA_ERR_INVALID_ARG).
+ * Every setting computes the same function.
  */
 pa_status pa_decode_select(int mode);
 

@@ -231,6 +231,7 @@ DECODE_SIMT_ONLY, DECODE_EVICT_FIRST, DECODE_PARTITION_MAJOR = 1, 2, 4
 DECODE_GROUP_PARTITIONS = 8
 DECODE_SUFFIX_PERSISTENT = 16
 DECODE_ONE_HEAD_PER_CTA = 32
+PREFILL_CTA_PAIRS = 64
 DECODE_DEFAULT = DECODE_PARTITION_MAJOR
 PA_PARTITION_BALANCED = -1                        # include/pa.h: the persistent balanced grid
 PA_DECODE_NOALLOC_SCRATCH_BYTES = 32 << 20        # include/pa.h: pa_decode_noalloc's array

@@ -21,7 +21,8 @@ namespace {
 // several (a test hook for the grouped path at small sizes), 16 = shared-prefix
 // decode with the persistent whole-item grid for the suffixes instead of one
 // CTA per (sequence, kv head) suffix, 32 = one kv head per CTA everywhere (no
-// head groups); the default is 4.
+// head groups), 64 = pa_prefill on clusters of two CTAs, one per query tile of
+// a pair (cta_group::2); the default is 4.
 std::atomic<int> g_select{4};
 
 // Plain split-K with short partitions: one CTA streams g consecutive
@@ -245,10 +246,12 @@ extern "C" pa_status pa_decode_partition_group(int S, int Hq, int Hkv, int D, in
 
 extern "C" pa_status pa_decode_select(int mode) {
     clear_error();
-    if (mode < 0 || mode > 63) return fail(PA_ERR_INVALID_ARG, "mode must be in [0, 63]");
+    if (mode < 0 || mode > 127) return fail(PA_ERR_INVALID_ARG, "mode must be in [0, 127]");
     g_select.store(mode);
     return PA_OK;
 }
+
+int pa::decode_select_mode() { return g_select.load(); }
 
 // pa_decode, plus the shared-prefix decode's two switches: the first
 // `prefix_parts` partitions of sequences whose table starts with row 0's

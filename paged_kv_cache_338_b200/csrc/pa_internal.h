@@ -53,6 +53,9 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // a recorded error if the runtime call fails).
 unsigned int* device_error_word();
 
+// The process-wide pa_decode_select mode (its prefill bits included).
+int decode_select_mode();
+
 // Per-device cache of a __device__ symbol's address.  An entry is keyed on
 // the device's current context as well, so it is looked up again after a
 // cudaDeviceReset (the next context may load the module elsewhere).

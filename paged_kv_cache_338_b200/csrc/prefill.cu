@@ -736,6 +736,475 @@ cudaError_t launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorM
                       mk, mv, p);
 }
 
+// ------------------------------------------------- CTA-pair kernel (D = 128)
+// The same attention with the two query tiles of a pair on two SMs, one per
+// CTA of a cluster of two, and the tensor-core instructions of the pair
+// (cta_group::2): one MMA of M = 256 rows computes both tiles' scores (each CTA
+// holds its tile's 128 query rows and half the key tile, 64 keys; each SM's
+// tensor memory receives its tile's 128 rows of all 128 keys), and one of
+// M = 256 adds P.V (each CTA holds half the value tile, 64 dims of 128 keys,
+// and its tile's P in its own tensor memory).  Each SM thus loads half of every
+// K and V tile, and its tensor memory holds two score buffers and O
+// (S_0 0..127, S_1 128..255, O 256..383): the scores of key tile j + 1 are
+// computed while the softmax works on tile j, so the softmax warpgroup of each
+// SM runs its tiles back to back instead of waiting for P.V and the next S
+// after every tile.  The leader CTA (cluster rank 0, tile A) issues every MMA
+// from one thread and commits each to both CTAs' barriers; each CTA's copies
+// land in its own shared memory and complete on the leader's barriers, except
+// the last V tile, whose rows past the tile's keys each CTA zeroes itself
+// before it signals the leader.  192 threads: warps 0-3 the softmax (one query
+// row per thread), warp 4 the copies, warp 5 tensor memory and (leader) the
+// MMAs.  Chunked prefill and prefill only (no prefix mode).
+constexpr int kThreads2 = 192;
+
+struct Smem2 {
+    static constexpr int ST = 3;                        // K and V ring depth
+    static constexpr int KSEG = kSeg / 2;               // 64 key rows x 128 bytes
+    static constexpr int KH = 2 * KSEG;                 // this CTA's 64 keys x 128 dims
+    static constexpr int VH = kSeg;                     // 128 keys x this CTA's 64 dims
+    static constexpr int Q = 0;                         // this CTA's 128 query rows, 2 segments
+    static constexpr int K = Q + 2 * kSeg;
+    static constexpr int V = K + ST * KH;
+    static constexpr int BAR = V + ST * VH;
+    // q_full, k_full[ST], v_full[ST] (leader: both CTAs' copies), k_free[ST],
+    // v_free[ST] (each CTA: the pair's MMAs are done with the slot), s_full[2],
+    // p_full[2] (leader: the 8 softmax warps), pv_done, o_full, drain (leader),
+    // v_last (leader: both CTAs' last V tile zeroed past the keys), v_mine
+    static constexpr int NBAR = 1 + 4 * ST + 2 + 2 + 1 + 1 + 1 + 1 + 1;
+    static constexpr int TMEM_SLOT = BAR + NBAR * 8;
+    static constexpr int ABORT = TMEM_SLOT + 4;
+    static constexpr int BYTES = ABORT + 4 + 1024;
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// The shared::cluster address of `local` in the CTA of cluster rank `rank`.
+__device__ __forceinline__ uint32_t cluster_addr(uint32_t local, uint32_t rank) {
+    uint32_t a;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(local), "r"(rank));
+    return a;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+                 ::: "memory");
+}
+// Arrive on an mbarrier of a CTA of the cluster.  What it orders is tensor
+// memory (tcgen05.wait::st and fence::before_thread_sync before it) and this
+// CTA's shared memory ahead of the peer's bulk copies, not generic memory
+// the other CTA reads, so it takes the default semantics rather than a
+// cluster-scope release (whose fence stalled the softmax warps).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+__device__ __forceinline__ void tmem_alloc2(uint32_t slot, uint32_t cols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(slot), "r"(cols) : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish2() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t cols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols)
+                 : "memory");
+}
+// The completion of this thread's earlier tcgen05 operations, on the mbarrier
+// at `bar`'s offset in both CTAs of the pair.
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;" ::"r"(bar), "h"((uint16_t)3) : "memory");
+}
+// ... on this CTA's mbarrier only.
+__device__ __forceinline__ void tc_commit_local2(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_mma2(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                        uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void tc_mma_ts2(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Tensor-map copies into this CTA's shared memory that complete on an
+// mbarrier of the pair's leader (`bar` a shared::cluster address).
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                                 int c0, int c1, int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_4d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                                 int c0, int c1, int c2, int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2),
+          "r"(c3)
+        : "memory");
+}
+// Instruction descriptor of kind::f16 for the pair: M 256 (128 rows per CTA).
+__device__ __forceinline__ uint32_t idesc2_f16(int ab_bf16, int b_mn_major, int N) {
+    return (1u << 4) | ((uint32_t)ab_bf16 << 7) | ((uint32_t)ab_bf16 << 10) |
+           ((uint32_t)b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
+}
+
+template <int DT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
+prefill2_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                const __grid_constant__ CUtensorMap tmv, const Params p) {
+    using L = Smem2;
+    constexpr int D = 128, ST = L::ST;
+    grid_dependency_wait();
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
+    // grid (2 x kPairGroup pairs x kv heads, sequences, pair groups); the two
+    // CTAs of a cluster are the tiles A and B of one pair, and take every early
+    // exit together (their conditions depend on the pair and sequence only)
+    const int PG = p.pair_group;
+    const int unit = (int)blockIdx.x >> 1;
+    const int g = unit / PG;
+    const int pair = ((int)gridDim.z - 1 - (int)blockIdx.z) * PG + (PG - 1 - unit % PG);
+    if (pair >= p.n_pairs) return;
+    const int s = (int)blockIdx.y;
+    const int q0 = p.query_start[s];
+    const int Ls = p.query_start[s + 1] - q0;
+    const int n = p.context_lens[s];
+    if (Ls < 0 || Ls > n || Ls > p.max_qlen || (long long)n > (long long)p.MB * p.bs) {
+        if (leader && pair == 0 && g == 0 && threadIdx.x == 0) atomicOr(p.err, PA_DEV_BAD_CONTEXT);
+        return;
+    }
+    const int c = n - Ls;
+    const int TQ = p.TQ;
+    const int iA = 2 * pair * TQ, iB = iA + TQ;
+    if (iA >= Ls) return;
+    const bool hasB = iB < Ls;
+    const int kvA = c + min(Ls, iB);
+    const int kv_len = hasB ? c + min(Ls, iB + TQ) : kvA;     // keys the pair reads
+    const int nt = (kv_len + kBN - 1) / kBN;
+    const int iX = leader ? iA : iB;                          // this CTA's first new token
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+    const uint32_t sb = smem_addr(sm);
+    const uint32_t sQ = sb + L::Q, sK = sb + L::K, sV = sb + L::V;
+    const uint32_t bar0 = sb + L::BAR;
+    const uint32_t q_full = bar0;
+    auto k_full = [&](int i) { return bar0 + 8u * (1 + i); };
+    auto v_full = [&](int i) { return bar0 + 8u * (1 + ST + i); };
+    auto k_free = [&](int i) { return bar0 + 8u * (1 + 2 * ST + i); };
+    auto v_free = [&](int i) { return bar0 + 8u * (1 + 3 * ST + i); };
+    auto s_full = [&](int b) { return bar0 + 8u * (1 + 4 * ST + b); };
+    auto p_full = [&](int b) { return bar0 + 8u * (3 + 4 * ST + b); };
+    const uint32_t pv_done = bar0 + 8u * (5 + 4 * ST);
+    const uint32_t o_full = bar0 + 8u * (6 + 4 * ST);
+    const uint32_t drain = bar0 + 8u * (7 + 4 * ST);
+    const uint32_t v_last = bar0 + 8u * (8 + 4 * ST);
+    const uint32_t v_mine = bar0 + 8u * (9 + 4 * ST);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::ABORT);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int i = 0; i < ST; ++i) {
+            mbar_init(k_full(i), 1);
+            mbar_init(v_full(i), 1);
+            mbar_init(k_free(i), 1);
+            mbar_init(v_free(i), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(s_full(b), 1);
+            mbar_init(p_full(b), 8);
+        }
+        mbar_init(pv_done, 1);
+        mbar_init(o_full, 1);
+        mbar_init(drain, 1);
+        mbar_init(v_last, 2);
+        mbar_init(v_mine, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 5) {
+        tmem_alloc2(sb + L::TMEM_SLOT, kTmemCols);
+        tmem_relinquish2();
+    }
+    // both CTAs' barriers and tensor memory exist before either touches the other's
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + L::TMEM_SLOT);
+    auto tS = [&](int b) { return tmem + 128u * b; };        // scores, then P over them
+    const uint32_t tO = tmem + 256u;                           // output accumulator
+
+    if (warp == 4) {
+        // ------------------------------------------------------------ loads
+        const int bpt = kBN >> p.log2bs;                       // blocks per key tile
+        const int half = bpt >> 1;                             // blocks of this CTA's K half
+        const int need = (kv_len + p.bs - 1) >> p.log2bs;
+        const uint32_t box = (uint32_t)p.bs * 128u;
+        const uint32_t lq = cluster_addr(q_full, 0);
+        if (lane == 0) {
+            if (leader) mbar_arrive_expect_tx(q_full, 2 * 2 * kSeg);
+            for (int sg = 0; sg < 2; ++sg)
+                tma_load_3d_pair(sQ + sg * kSeg, &tmq, lq, sg * 64, g * p.G, q0 + iX);
+        }
+        int nk = 0;
+        for (int j = 0; j < nt; ++j) {
+            const int st = j % ST;
+            const uint32_t par = ((j / ST) & 1) ^ 1;
+            const int lb = j * bpt + lane;
+            const bool want = lane < bpt && lb < need;
+            int id = -1;
+            if (want) id = p.block_tables[(size_t)s * p.MB + lb];
+            const bool valid = want && id >= 0 && (long long)id < p.NB;
+            if (leader && want && !valid) atomicOr(p.err, PA_DEV_BAD_BLOCK);
+            const uint32_t nvalid = (uint32_t)__popc(__ballot_sync(~0u, valid));
+            // K: this CTA's half of the tile's blocks, two 64-dim segments each
+            if (!warp_wait(k_free(st), par, abort_flag, p.err, 10)) break;
+            if (leader && lane == 0) mbar_arrive_expect_tx(k_full(st), nvalid * 2 * box);
+            __syncwarp();
+            if (valid && lane / half == (int)rank)
+                for (int sg = 0; sg < 2; ++sg)
+                    tma_load_4d_pair(sK + st * L::KH + sg * L::KSEG + (lane - (int)rank * half) * box,
+                                     &tmk, cluster_addr(k_full(st), 0), sg * 64, g, 0, id);
+            nk = j + 1;
+            // V: this CTA's 64 dims of every block of the tile
+            if (!warp_wait(v_free(st), par, abort_flag, p.err, 11)) break;
+            if (j + 1 < nt) {
+                if (leader && lane == 0) mbar_arrive_expect_tx(v_full(st), nvalid * 2 * box);
+                __syncwarp();
+                if (valid)
+                    tma_load_4d_pair(sV + st * L::VH + lane * box, &tmv, cluster_addr(v_full(st), 0),
+                                     (int)rank * 64, g, 0, id);
+            } else {
+                // The last tile lands on this CTA's own barrier: its rows at or
+                // past the pair's keys hold another token's values, the cache's
+                // unused tail slots or stale tiles, and are zeroed here (a zero
+                // probability times a NaN would still poison the product).
+                if (lane == 0) mbar_arrive_expect_tx(v_mine, nvalid * box);
+                __syncwarp();
+                if (valid)
+                    tma_load_4d_plain(sV + st * L::VH + lane * box, &tmv, v_mine, (int)rank * 64, g,
+                                      0, id);
+                if (!warp_wait(v_mine, 0, abort_flag, p.err, 9, false)) break;
+                const int z0 = kv_len - j * kBN;
+                for (int xx = lane; xx < (kBN - z0) * 8; xx += 32)
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};"
+                                 ::"r"(sV + st * L::VH + z0 * 128 + xx * 16), "r"(0) : "memory");
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    if (leader) mbar_arrive(v_last);
+                    else mbar_arrive_cluster(cluster_addr(v_last, 0));
+                }
+            }
+        }
+        // (leader) every copy of the pair has landed before the CTAs may exit:
+        // immediate on the normal path, where the MMAs consumed them all
+        if (leader)
+            for (int i = 0; i < ST && i < nk; ++i) {
+                const int jl = i + (nk - 1 - i) / ST * ST;
+                warp_wait(k_full(i), (jl / ST) & 1, abort_flag, p.err, 17, false);
+                if (jl + 1 < nt) warp_wait(v_full(i), (jl / ST) & 1, abort_flag, p.err, 17, false);
+            }
+        if (leader) warp_wait(q_full, 0, abort_flag, p.err, 17, false);
+    } else if (warp == 5) {
+        // ------------------------------------------------ MMAs (leader only)
+        if (leader) {
+            constexpr int ABF = DT == PA_BF16 ? 1 : 0;
+            const uint32_t id_s = idesc2_f16(ABF, 0, kBN);
+            const uint32_t id_o = idesc2_f16(ABF, 1, D);
+            // S_b = Q K_j^T, both tiles: K_j's halves in both CTAs' ring slot st
+            auto issue_s = [&](int b, int st) {
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t kb = sK + st * L::KH;
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        tc_mma2(tS(b), sdesc(sQ + (kk >> 2) * kSeg + (kk & 3) * 32, 16),
+                                sdesc(kb + (kk >> 2) * L::KSEG + (kk & 3) * 32, 16), id_s, kk > 0);
+                    }
+                    tc_commit_pair(s_full(b));
+                    tc_commit_pair(k_free(st));
+                }
+                __syncwarp();
+            };
+            bool ok = warp_wait(q_full, 0, abort_flag, p.err, 7) &&
+                      warp_wait(k_full(0), 0, abort_flag, p.err, 8);
+            if (ok) issue_s(0, 0);
+            if (ok && nt > 1 && (ok = warp_wait(k_full(1 % ST), (1 / ST) & 1, abort_flag, p.err, 8)))
+                issue_s(1, 1 % ST);
+            for (int j = 0; j < nt && ok; ++j) {
+                const int st = j % ST, b = j & 1;
+                if (!(ok = warp_wait(p_full(b), (j >> 1) & 1, abort_flag, p.err, 13))) break;
+                if (!(ok = j + 1 < nt ? warp_wait(v_full(st), (j / ST) & 1, abort_flag, p.err, 9)
+                                      : warp_wait(v_last, 0, abort_flag, p.err, 9)))
+                    break;
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t vb = sV + st * L::VH;
+#pragma unroll
+                    for (int kk = 0; kk < kBN / 16; ++kk)
+                        tc_mma_ts2(tO, tS(b) + kk * 8, sdesc(vb + kk * 16 * 128, kSeg), id_o,
+                                   (j > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit_pair(pv_done);
+                    tc_commit_pair(v_free(st));
+                    if (j == nt - 1) tc_commit_pair(o_full);
+                }
+                __syncwarp();
+                if (j + 2 < nt) {
+                    // S_b(j + 2) overwrites P_b(j): issued behind P_b(j).V, and one
+                    // thread's MMAs execute in issue order
+                    const int st2 = (j + 2) % ST;
+                    if (!(ok = warp_wait(k_full(st2), ((j + 2) / ST) & 1, abort_flag, p.err, 8)))
+                        break;
+                    issue_s(b, st2);
+                }
+            }
+            if (lane == 0) tc_commit_local2(drain);
+            __syncwarp();
+            warp_wait(drain, 0, abort_flag, p.err, 16, false);
+        }
+    } else {
+        // ------------------------------------------------ softmax (4 warps)
+        const int r = threadIdx.x;                           // row = tensor-memory lane
+        const int it = iX + (r >> p.log2G);                  // new-token index of the row
+        const bool row_ok = it < Ls;
+        const int limit = row_ok ? c + it + 1 : kv_len;      // keys 0..limit-1 are visible
+        const uint32_t lrow = (uint32_t)(warp * 32) << 16;
+        const float sl = p.sl;
+        const uint32_t my_p_full0 = leader ? p_full(0) : cluster_addr(p_full(0), 0);
+        const uint32_t my_p_full1 = leader ? p_full(1) : cluster_addr(p_full(1), 0);
+        float m_use = -INFINITY, lsum = 0.f;
+        bool ok = true;
+        for (int j = 0; j < nt; ++j) {
+            const int b = j & 1;
+            if (!(ok = warp_wait(s_full(b), (j >> 1) & 1, abort_flag, p.err, 12))) break;
+            tc_fence_after();
+            float sv[kBN];
+#pragma unroll
+            for (int c4 = 0; c4 < kBN / 32; ++c4) tmem_ld32(tS(b) + lrow + c4 * 32, sv + c4 * 32);
+            tmem_wait_ld();
+            if ((j + 1) * kBN > c + iX + 1) {
+                const int nv = limit - j * kBN;
+#pragma unroll
+                for (int k = 0; k < kBN; ++k)
+                    if (k >= nv) sv[k] = -INFINITY;
+            }
+            float pm[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) pm[i] = sv[i];
+#pragma unroll
+            for (int k = 8; k < kBN; k += 2) pm[(k >> 1) & 7] = max3(pm[(k >> 1) & 7], sv[k], sv[k + 1]);
+            const float tmax = fmaxf(max3(pm[0], pm[1], pm[2]),
+                                     fmaxf(max3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+            const float m_new = fmaxf(m_use, tmax * sl);
+            const bool raise = m_new > m_use + kRescaleLog2;
+            const float alpha = raise ? ex2(m_use - m_new) : 1.f;
+            if (raise) m_use = m_new;
+            lsum *= alpha;
+            if (j > 0 && __any_sync(~0u, raise)) {
+                // O holds P.V of tiles 0..j-1 once the last of them completes
+                if (!(ok = warp_wait(pv_done, (j - 1) & 1, abort_flag, p.err, 14))) break;
+                tc_fence_after();
+#pragma unroll 1
+                for (int c4 = 0; c4 < D / 32; ++c4) {
+                    float o[32];
+                    tmem_ld32(tO + lrow + c4 * 32, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] *= alpha;
+                    tmem_st32(tO + lrow + c4 * 32, o);
+                }
+                tmem_wait_st();
+            }
+            const float2 sl2 = make_float2(sl, sl), nm2 = make_float2(-m_use, -m_use);
+#pragma unroll
+            for (int c16 = 0; c16 < kBN / 32; ++c16) {
+                uint32_t w[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const int k = c16 * 32 + 2 * e;
+                    const float2 xy = fma2(make_float2(sv[k], sv[k + 1]), sl2, nm2);
+                    sv[k] = ex2(xy.x);
+                    sv[k + 1] = ex2(xy.y);
+                    w[e] = pack2<DT>(sv[k], sv[k + 1]);
+                }
+                tmem_st16(tS(b) + lrow + c16 * 16, w);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if (leader) mbar_arrive(p_full(b));
+                else mbar_arrive_cluster(b ? my_p_full1 : my_p_full0);
+            }
+            float2 ps[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+            for (int k = 0; k < kBN; k += 2)
+                ps[(k >> 1) & 3] = add2(ps[(k >> 1) & 3], make_float2(sv[k], sv[k + 1]));
+            lsum += ((ps[0].x + ps[0].y) + (ps[1].x + ps[1].y)) +
+                    ((ps[2].x + ps[2].y) + (ps[3].x + ps[3].y));
+        }
+        if (ok) ok = warp_wait(o_full, 0, abort_flag, p.err, 15);
+        if (ok) {
+            tc_fence_after();
+            const float inv = 1.f / lsum;
+            const int h = g * p.G + (r & (p.G - 1));
+            uint8_t* orow = static_cast<uint8_t*>(p.out) + ((size_t)(q0 + it) * p.Hq + h) * (size_t)D * 2;
+#pragma unroll 1
+            for (int c4 = 0; c4 < D / 32; ++c4) {
+                float o[32];
+                tmem_ld32(tO + lrow + c4 * 32, o);
+                tmem_wait_ld();
+                if (row_ok) {
+                    uint32_t w[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) w[e] = pack2<DT>(o[2 * e] * inv, o[2 * e + 1] * inv);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v)
+                        reinterpret_cast<uint4*>(orow + c4 * 64)[v] =
+                            make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+                }
+            }
+        }
+    }
+    // Every MMA of the pair has completed (the leader drained them) and no lane
+    // of either CTA reads tensor memory any more: free it, in both CTAs.
+    tc_fence_before();
+    cluster_sync();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc2(tmem, kTmemCols);
+    }
+}
+
+template <int DT>
+cudaError_t launch2(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                    const Params& p, dim3 grid, cudaStream_t st) {
+    const cudaError_t attr = pa::dev::ensure_dynamic_smem<prefill2_kernel<DT>>(Smem2::BYTES);
+    if (attr != cudaSuccess) return attr;
+    return launch_pdl(prefill2_kernel<DT>, grid, dim3(kThreads2), (size_t)Smem2::BYTES, st, mq, mk,
+                      mv, p);
+}
+
 }  // namespace pf
 
 using pa::fail;
@@ -873,6 +1342,14 @@ extern "C" pa_status pa_prefill(void* out, const void* q, pa_dtype q_dt, const v
                     (unsigned)((n_pairs + pf::kPairGroup - 1) / pf::kPairGroup));
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     cudaError_t e;
+    if (D == 128 && (pa::decode_select_mode() & 64)) {
+        // the two query tiles of a pair on a pair of SMs (cta_group::2)
+        const dim3 grid2(2 * grid.x, grid.y, grid.z);
+        e = q_dt == PA_BF16 ? pf::launch2<PA_BF16>(mq, mk, mv, p, grid2, cs)
+                            : pf::launch2<PA_F16>(mq, mk, mv, p, grid2, cs);
+        if (e != cudaSuccess) return pa::cuda_fail(e, "prefill launch");
+        return PA_OK;
+    }
     if (q_dt == PA_BF16)
         e = D == 64 ? pf::launch<PA_BF16, 64>(mq, mk, mv, p, grid, cs)
                     : pf::launch<PA_BF16, 128>(mq, mk, mv, p, grid, cs);

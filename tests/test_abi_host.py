@@ -91,12 +91,12 @@ def test_host_argument_checks():
 
 
 def test_decode_select_modes():
-    """Every documented bit combination is accepted (0..63, bits 8, 16 and 32
-    included) and anything else refused; the default is restored afterwards."""
+    """Every documented bit combination is accepted (0..127, bits 8, 16, 32 and
+    64 included) and anything else refused; the default is restored afterwards."""
     try:
-        for mode in range(64):
+        for mode in range(128):
             pa.pa_decode_select(mode)
-        for bad in (-1, 64, 128):
+        for bad in (-1, 128, 256):
             _bad(pa.pa_decode_select, bad)
     finally:
         pa.pa_decode_select(pa.DECODE_DEFAULT)

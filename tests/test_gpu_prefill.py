@@ -6,6 +6,8 @@ the new tokens' K, V through slot_mapping (bit-exact against the oracle), then
 pa_prefill (max abs error against the oracle's double result: bf16 1e-2,
 f16 2e-3, the decode bars: P is rounded to the operand type and accumulated in
 fp32 as there).  Unused blocks, tail slots and table padding are poisoned.
+Head size 128 runs two kernels, both checked: one CTA per pair of query tiles
+(the default) and a cluster of two CTAs per pair (PREFILL_CTA_PAIRS).
 """
 import numpy as np
 import pytest
@@ -26,6 +28,16 @@ def _cuda():
         pytest.skip("needs a GPU")
     pa.pa_device_status(clear=True)
     yield
+
+
+KERNELS = {"single": pa.DECODE_DEFAULT, "pair": pa.DECODE_DEFAULT | pa.PREFILL_CTA_PAIRS}
+
+
+@pytest.fixture(params=sorted(KERNELS))
+def kernel(request):
+    pa.pa_decode_select(KERNELS[request.param])
+    yield request.param
+    pa.pa_decode_select(pa.DECODE_DEFAULT)
 
 
 def gpu_prefill(inp: wl.PrefillInputs, max_query_len=None, tables=None, lens=None):
@@ -66,7 +78,7 @@ def _bits_equal(a, b, dt):
     return torch.equal(wl.raw_view(a.contiguous(), dt), wl.raw_view(b.contiguous(), dt))
 
 
-def test_first_case_small():
+def test_first_case_small(kernel):
     cfg = wl.PrefillConfig("first", 2, 8, 2, 128, 16, "bf16", 5, 150, 0, 200)
     inp = wl.make_prefill_inputs(cfg, seed=1)
     want, kc_o, vc_o = oracle_prefill(inp)
@@ -82,7 +94,7 @@ SHAPES = [(G, D, bs, dt) for G in (1, 2, 4, 8, 16) for D in (64, 128) for bs in 
 
 
 @pytest.mark.parametrize("G,D,bs,dt", SHAPES)
-def test_prefill_shapes(G, D, bs, dt):
+def test_prefill_shapes(G, D, bs, dt, kernel):
     Hkv = 2
     cfg = wl.PrefillConfig(f"s{G}_{D}_{bs}_{dt}", 3, G * Hkv, Hkv, D, bs, dt, 1, 300, 0, 400)
     inp = wl.make_prefill_inputs(cfg, seed=G * 100 + D + bs)
@@ -94,7 +106,7 @@ def test_prefill_shapes(G, D, bs, dt):
 
 
 @pytest.mark.parametrize("G", [1, 4, 16])
-def test_tile_edges(G):
+def test_tile_edges(G, kernel):
     """Chunk lengths at the query-tile size +-1, cached lengths that put the last
     key at a key-tile edge +-1, a one-token chunk and a chunk from an empty cache."""
     TQ = 128 // G
@@ -138,7 +150,7 @@ def test_long_context_rows_sampled():
     _check(out[rows], want, "bf16", "sampled rows")
 
 
-def test_device_errors_are_reported():
+def test_device_errors_are_reported(kernel):
     cfg = wl.PrefillConfig("errs", 2, 8, 2, 128, 16, "bf16", 20, 20, 30, 30)
     inp = wl.make_prefill_inputs(cfg, seed=6)
     pa.pa_device_status(clear=True)
