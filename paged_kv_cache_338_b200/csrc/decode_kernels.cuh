@@ -956,7 +956,7 @@ __device__ __forceinline__ float fold_prefix_records(const Params& p, int s, int
             M = Mn;
         }
     }
-    return L > 0.f ? O / L : 0.f;
+    return L == 0.f ? 0.f : O / L;
 }
 
 // Smem bytes of the per-partition warp merge area of the grouped-partition
@@ -1151,7 +1151,7 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                     const float O = go[((size_t)hw * gh + g) * C::D + d], L = gl[hw * gh + g];
                     if (nparts == 1) {
                         dev::store_out<C::QT>(p.out, ((size_t)s * p.Hq + h) * C::D + d,
-                                              L > 0.f ? (O / L) * p.v_scale : 0.f);
+                                              L == 0.f ? 0.f : (O / L) * p.v_scale);
                     } else {
                         const size_t row = ((size_t)s * p.Hq + h) * p.max_parts + q0 + qq;
                         p.ws_o[row * C::D + d] = O * p.v_scale;
@@ -1206,7 +1206,7 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
                         const int h = h0 + g;
                         if (nparts == 1) {
                             dev::store_out<C::QT>(p.out, ((size_t)s * p.Hq + h) * C::D + d,
-                                                  L > 0.f ? (O / L) * p.v_scale : 0.f);
+                                                  L == 0.f ? 0.f : (O / L) * p.v_scale);
                         } else {
                             const size_t row = ((size_t)s * p.Hq + h) * p.max_parts + q0 + qq;
                             p.ws_o[row * C::D + d] = O * p.v_scale;
@@ -1376,7 +1376,7 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
         for (int x = 16; x >= 1; x >>= 1) L += __shfl_xor_sync(0xffffffffu, L, x);
         if (lane == 0) {
             c[ncoef - 2] = M;
-            c[ncoef - 1] = L > 0.f ? 1.f / L : 0.f;
+            c[ncoef - 1] = L == 0.f ? 0.f : 1.f / L;
             if (!fuse_records && !(nparts == 1 && !p.force_ws)) {
                 const int h = C::HG > 1 ? h0 + (r / gc) * G + r % gc : h0 + r;
                 p.ws_ml[((size_t)s * p.Hq + h) * p.max_parts + part] = make_float2(M, L);
@@ -1751,7 +1751,7 @@ decode_balanced(const __grid_constant__ CUtensorMap tmk, const __grid_constant__
                                                               O * p.v_scale, C::D));
                 } else if (first && last) {
                     dev::store_out<C::QT>(p.out, ((size_t)d.s * p.Hq + h0 + g) * C::D + dd,
-                                          L > 0.f ? (O / L) * p.v_scale : 0.f);
+                                          L == 0.f ? 0.f : (O / L) * p.v_scale);
                 } else {
                     const size_t row = (size_t)piece * gc + g;
                     if ((int64_t)row < p.ws_rows) {
@@ -1893,7 +1893,7 @@ __global__ void __launch_bounds__(NWARPS * 32) decode_merge(const Params p, int 
             Lt += s_l[w];
             Ot += s_o[w][d];
         }
-        dev::store_out<QT>(p.out, ((size_t)s * p.Hq + head) * D + d, Lt > 0.f ? Ot / Lt : 0.f);
+        dev::store_out<QT>(p.out, ((size_t)s * p.Hq + head) * D + d, Lt == 0.f ? 0.f : Ot / Lt);
     }
 }
 
