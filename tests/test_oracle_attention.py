@@ -13,7 +13,8 @@ The attention oracle is checked against things other than itself:
   logit far above the rest picks that value, GQA equals MHA with each kv head
   replicated over its group;
 * poisoned storage (unused blocks, tail slots, table entries past the end) is
-  never read.
+  never read; a NaN in an attended key or value reaches exactly the outputs
+  that textbook attention (and SDPA) sends it to.
 """
 import numpy as np
 import pytest
@@ -207,6 +208,38 @@ def test_poison_is_never_read():
     assert (inp.block_tables == -1).any()
     kc, vc = _step_caches(inp)
     assert np.isfinite(_oracle(inp, kc, vc)).all()
+
+
+def test_nan_reaches_exactly_the_attending_outputs():
+    """A NaN in an attended key makes the whole output row of each query head of
+    that kv head NaN; a NaN in one dimension of an attended value makes only
+    that output dimension NaN; the same NaN past the length reaches nothing.
+    torch SDPA (float64) on the unpaged gather agrees element for element, and
+    every untouched output equals the clean run's exactly."""
+    cfg = wl.DecodeConfig("nan", 3, 8, 2, 64, 16, "f32", "f32", 20, 60)
+    inp = wl.make_decode_inputs(cfg, seed=4)
+    kc, vc = _step_caches(inp)
+    clean = _oracle(inp, kc, vc)
+    G, bs = cfg.group, cfg.block_size
+    kp, vp = kc.clone(), vc.clone()
+    n0, n2 = int(inp.context_lens[0]), int(inp.context_lens[2])
+    b, o = int(inp.block_tables[0, 7 // bs]), 7 % bs
+    kp[b, o, 1, 3] = float("nan")                      # key of token 7, sequence 0, kv head 1
+    b, o = int(inp.block_tables[2, (n2 - 1) // bs]), (n2 - 1) % bs
+    vp[b, o, 0, 5] = float("nan")                      # value dim 5 of the last token of seq 2
+    if n0 % bs:                                         # the slot after sequence 0's last token
+        b, o = int(inp.block_tables[0, n0 // bs]), n0 % bs
+        kp[b, o, 0, :] = float("nan")
+        vp[b, o, 0, :] = float("nan")
+    got = _oracle(inp, kp, vp)
+    want = np.zeros_like(got, dtype=bool)
+    want[0, G:2 * G, :] = True
+    want[2, :G, 5] = True
+    assert np.array_equal(np.isnan(got), want)
+    assert np.array_equal(got[~want], clean[~want])
+    ref = _gather_sdpa(inp, kp, vp)
+    assert np.array_equal(np.isnan(ref), want)
+    assert np.abs(ref[~want] - got[~want]).max() < 1e-12
 
 
 def test_zero_length_sequence_gives_zero_row():
