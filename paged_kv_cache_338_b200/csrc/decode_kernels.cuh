@@ -926,37 +926,84 @@ __device__ __forceinline__ bool consumers_sync_or(bool pred) {
     return r != 0;
 }
 
-// Fold the prefix_parts prefix records of (sequence s, head h) into a state
-// (M in log2 units, L, O already times v_scale) and return the output value.
-// The records are loaded first, so their latencies overlap.
-__device__ __forceinline__ float fold_prefix_records(const Params& p, int s, int h, int d,
-                                                     float M, float L, float O, int D) {
-    constexpr int kMaxUnrolled = 8;
-    const size_t row0 = ((size_t)s * p.Hq + h) * p.max_parts;
-    for (int pp = 0; pp < p.prefix_parts; pp += kMaxUnrolled) {
-        float2 ml[kMaxUnrolled];
-        float o[kMaxUnrolled];
+// A whole item's outputs: the consumer warps' states (cm, cl, co in shared
+// memory, stride gc) merged, then the prefix kernel's records of the item's
+// heads folded in one after another (the split-K identity), four outputs per
+// thread at a time with the loads of all their records in flight together
+// (one round trip to L2 per four records instead of one per output).
+template <class C>
+__device__ __forceinline__ void fold_item(const Params& p, int s, int h0, int gc, const float* cm,
+                                          const float* cl, const float* co) {
+    constexpr int T = C::NW * 32, U = 4;
+    const int total = gc * C::D;
+    for (int base = threadIdx.x; base < total; base += U * T) {
+        float M[U], L[U], O[U];
         #pragma unroll
-        for (int i = 0; i < kMaxUnrolled; ++i) {
-            if (pp + i < p.prefix_parts) {
-                ml[i] = p.ws_ml[row0 + pp + i];
-                o[i] = p.ws_o[(row0 + pp + i) * D + d];
-            } else {
-                ml[i] = make_float2(-INFINITY, 0.f);
-                o[i] = 0.f;
+        for (int u = 0; u < U; ++u) {
+            const int idx = base + u * T;
+            M[u] = -INFINITY;
+            L[u] = 0.f;
+            O[u] = 0.f;
+            if (idx < total) {
+                const int g = idx / C::D, dd = idx % C::D;
+                float m = -INFINITY;
+                #pragma unroll
+                for (int w = 0; w < C::NW; ++w) m = fmaxf(m, cm[w * gc + g]);
+                float l = 0.f, o = 0.f;
+                if (m != -INFINITY) {
+                    #pragma unroll
+                    for (int w = 0; w < C::NW; ++w) {
+                        const float f = exp2f(cm[w * gc + g] - m);
+                        l = fmaf(f, cl[w * gc + g], l);
+                        o = fmaf(f, co[(w * gc + g) * C::D + dd], o);
+                    }
+                }
+                M[u] = m;
+                L[u] = l;
+                O[u] = o * p.v_scale;
+            }
+        }
+        for (int pp0 = 0; pp0 < p.prefix_parts; pp0 += U) {
+            float2 ml[U][U];
+            float ro[U][U];
+            #pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int idx = base + u * T;
+                const int g = idx / C::D, dd = idx % C::D;
+                #pragma unroll
+                for (int i = 0; i < U; ++i) {
+                    if (idx < total && pp0 + i < p.prefix_parts) {
+                        const size_t row = ((size_t)s * p.Hq + h0 + g) * p.max_parts + pp0 + i;
+                        ml[u][i] = p.ws_ml[row];
+                        ro[u][i] = p.ws_o[row * C::D + dd];
+                    } else {
+                        ml[u][i] = make_float2(-INFINITY, 0.f);
+                        ro[u][i] = 0.f;
+                    }
+                }
+            }
+            #pragma unroll
+            for (int u = 0; u < U; ++u) {
+                #pragma unroll
+                for (int i = 0; i < U; ++i) {
+                    const float Mn = fmaxf(M[u], ml[u][i].x);
+                    if (Mn == -INFINITY) continue;
+                    const float a = exp2f(M[u] - Mn), b = exp2f(ml[u][i].x - Mn);
+                    L[u] = L[u] * a + ml[u][i].y * b;
+                    O[u] = O[u] * a + ro[u][i] * b;
+                    M[u] = Mn;
+                }
             }
         }
         #pragma unroll
-        for (int i = 0; i < kMaxUnrolled; ++i) {
-            const float Mn = fmaxf(M, ml[i].x);
-            if (Mn == -INFINITY) continue;
-            const float a = exp2f(M - Mn), b = exp2f(ml[i].x - Mn);
-            L = L * a + ml[i].y * b;
-            O = O * a + o[i] * b;
-            M = Mn;
+        for (int u = 0; u < U; ++u) {
+            const int idx = base + u * T;
+            if (idx < total)
+                dev::store_out<C::QT>(p.out,
+                                      ((size_t)s * p.Hq + h0 + idx / C::D) * C::D + idx % C::D,
+                                      L[u] == 0.f ? 0.f : O[u] / L[u]);
         }
     }
-    return L == 0.f ? 0.f : O / L;
 }
 
 // Smem bytes of the per-partition warp merge area of the grouped-partition
@@ -1496,7 +1543,12 @@ template <class C0>
 __global__ void __launch_bounds__(C0::THREADS, 3)
 decode_balanced(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                 const Params p) {
-    dev::grid_dependency_wait();       // launched as a dependent of the kernel before it
+    // Launched as a dependent of the kernel before it.  Whole items of the
+    // shared-prefix decode read nothing that kernel (the prefix kernel) writes
+    // until they fold its records in, so they wait there and stream their
+    // suffixes meanwhile; everything the kernels before that one wrote was
+    // complete when its CTAs let this grid start.
+    if (!p.whole_items) dev::grid_dependency_wait();
     using B = BalancedSmem<C0>;
     using C = Balanced<C0>;
     constexpr int STAGES = B::STAGES;
@@ -1653,6 +1705,16 @@ decode_balanced(const __grid_constant__ CUtensorMap tmk, const __grid_constant__
                 const int blk0 = pb > 0 && reg ? pb : 0;
                 PieceDesc d{s, hc, blk0, nb - blk0, nb, n, k, 0, blk0 > 0};
                 if (publish(d)) break;
+                {
+                    // the consumers load this item's query rows when they reach
+                    // it: have them in L2 by then
+                    constexpr int QB = C::QT == PA_F32 ? 4 : 2;
+                    const int hq0 = (hc / chunks) * G + (hc % chunks) * gc;
+                    const char* qrow = static_cast<const char*>(p.q) +
+                                       ((size_t)s * p.Hq + hq0) * C::D * QB;
+                    for (int i = lane; i < (gc * C::D * QB + 127) / 128; i += 32)
+                        dev::prefetch_l2(qrow + (size_t)i * 128);
+                }
                 produce<C>(&tmk, &tmv, p, p.block_tables + (size_t)s * p.MB, blk0, nb - blk0,
                             nb - blk0, hc / chunks, stages, full0, empty0, &s_abort, &k);
                 if (*(volatile int*)&s_abort) break;
@@ -1688,6 +1750,7 @@ decode_balanced(const __grid_constant__ CUtensorMap tmk, const __grid_constant__
         float* cm = comb;                              // stride gc (heads per item)
         float* cl = cm + C::NW * gc;
         float* co = cl + C::NW * gc;
+        bool records_ready = false;
         for (int ci = 0;; ++ci) {
             const int slot = ci % kItemQ;
             if (!dev::mbar_wait_bounded(ifull0 + 8 * slot, (ci / kItemQ) & 1)) {
@@ -1731,6 +1794,13 @@ decode_balanced(const __grid_constant__ CUtensorMap tmk, const __grid_constant__
             const bool whole = p.whole_items != 0;
             const bool first = whole || d.off == 0, last = whole || d.off + d.take == d.nblk;
             const int piece = item + blockIdx.x;
+            if (d.fold) {
+                if (!records_ready) {
+                    dev::grid_dependency_wait();        // the prefix kernel wrote them
+                    records_ready = true;
+                }
+                fold_item<C>(p, d.s, h0, gc, cm, cl, co);
+            } else
             for (int idx = threadIdx.x; idx < gc * C::D; idx += C::NW * 32) {
                 const int g = idx / C::D, dd = idx % C::D;
                 float M = -INFINITY;
@@ -1745,11 +1815,7 @@ decode_balanced(const __grid_constant__ CUtensorMap tmk, const __grid_constant__
                         O = fmaf(f, co[(w * gc + g) * C::D + dd], O);
                     }
                 }
-                if (d.fold) {
-                    dev::store_out<C::QT>(p.out, ((size_t)d.s * p.Hq + h0 + g) * C::D + dd,
-                                          fold_prefix_records(p, d.s, h0 + g, dd, M, L,
-                                                              O * p.v_scale, C::D));
-                } else if (first && last) {
+                if (first && last) {
                     dev::store_out<C::QT>(p.out, ((size_t)d.s * p.Hq + h0 + g) * C::D + dd,
                                           L == 0.f ? 0.f : (O / L) * p.v_scale);
                 } else {
