@@ -6,7 +6,10 @@ Every entry point of the step enqueues only kernels on the caller's stream
 (no allocation, no synchronisation, no host read of device memory), so the
 step can be captured.  Here the append + copy-on-write and the decode are
 captured, the inputs are changed in place, and the replayed outputs must be
-bit-identical to the eagerly launched calls on the same inputs.
+bit-identical to the eagerly launched calls on the same inputs.  The
+shared-prefix step is replayed with both suffix passes (one CTA per suffix,
+and the persistent grid, whose whole items wait for the prefix kernel only
+before they fold its records); the prefill step (append + pa_prefill) too.
 """
 import pytest
 import torch
@@ -26,14 +29,25 @@ def _cuda():
 
 
 CASES = [
-    ("llama3_8b_gqa_bf16_b128", 16, 300, 3000, None, 512),
-    ("long_context_splitk_bf16_4x100k", 2, 20000, 30000, None, 512),
-    ("prefix_shared_fp8_b256", 48, 10, 400, 512, 0),
+    ("llama3_8b_gqa_bf16_b128", 16, 300, 3000, None, 512, pa.DECODE_DEFAULT),
+    ("long_context_splitk_bf16_4x100k", 2, 20000, 30000, None, 512, pa.DECODE_DEFAULT),
+    ("prefix_shared_fp8_b256", 48, 10, 400, 512, 0, pa.DECODE_DEFAULT),
+    ("prefix_shared_fp8_b256", 300, 10, 400, 512, 0,
+     pa.DECODE_DEFAULT | pa.DECODE_SUFFIX_PERSISTENT),
 ]
 
 
-@pytest.mark.parametrize("name,nseq,lo,hi,prefix,part", CASES, ids=[c[0] for c in CASES])
-def test_graph_replay_matches_eager_calls(name, nseq, lo, hi, prefix, part):
+@pytest.fixture
+def select():
+    yield pa.pa_decode_select
+    pa.pa_decode_select(pa.DECODE_DEFAULT)
+
+
+@pytest.mark.parametrize("name,nseq,lo,hi,prefix,part,mode", CASES,
+                         ids=[c[0] + ("_persistent" if c[6] & pa.DECODE_SUFFIX_PERSISTENT else "")
+                              for c in CASES])
+def test_graph_replay_matches_eager_calls(name, nseq, lo, hi, prefix, part, mode, select):
+    select(mode)
     cfg = wl.small_variant(wl.DECODE_WORKLOADS[name], nseq, lo, hi, prefix_tokens=prefix)
     inp = wl.make_decode_inputs(cfg, seed=21, device="cuda")
     S, Hq, D = inp.q.shape
@@ -85,5 +99,39 @@ def test_graph_replay_matches_eager_calls(name, nseq, lo, hi, prefix, part):
         assert pa.pa_device_status() == 0
         assert torch.equal(wl.raw_view(kc_g, cfg.kv_dtype), wl.raw_view(kc, cfg.kv_dtype))
         assert torch.equal(wl.raw_view(vc_g, cfg.kv_dtype), wl.raw_view(vc, cfg.kv_dtype))
+        assert torch.isfinite(got).all()
+        assert torch.equal(got, out), "graph replay differs from the eager calls"
+
+
+def test_prefill_graph_replay_matches_eager_calls():
+    cfg = wl.PrefillConfig("graph", 3, 32, 8, 128, 16, "bf16", 100, 700, 0, 900)
+    inp = wl.make_prefill_inputs(cfg, seed=22)
+    d = {k: getattr(inp, k).cuda() for k in ("q", "key_cache", "value_cache", "key_new",
+                                              "value_new", "slot_mapping", "block_tables",
+                                              "context_lens", "query_start")}
+    kc, vc = d["key_cache"].clone(), d["value_cache"].clone()
+    out = torch.empty_like(d["q"])
+
+    def step():
+        pa.pa_reshape_and_cache(d["key_new"], d["value_new"], kc, vc, d["slot_mapping"])
+        pa.pa_prefill(out, d["q"], kc, vc, d["block_tables"], d["context_lens"], d["query_start"],
+                      inp.max_query_len, inp.scale)
+
+    step()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    gen = torch.Generator(device="cuda").manual_seed(6)
+    for _ in range(3):
+        for k in ("q", "key_new", "value_new"):
+            d[k].copy_(torch.randn(d[k].shape, generator=gen, device="cuda").to(d[k].dtype))
+        g.replay()
+        torch.cuda.synchronize()
+        got, kc_g = out.clone(), kc.clone()
+        step()
+        torch.cuda.synchronize()
+        assert pa.pa_device_status() == 0
+        assert torch.equal(wl.raw_view(kc_g, cfg.dtype), wl.raw_view(kc, cfg.dtype))   # NaN-poisoned slots
         assert torch.isfinite(got).all()
         assert torch.equal(got, out), "graph replay differs from the eager calls"
