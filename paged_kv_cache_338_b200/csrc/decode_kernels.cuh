@@ -1023,8 +1023,10 @@ decode_partition(const __grid_constant__ CUtensorMap tmk, const __grid_constant_
     // Launched as a dependent of the kernel before it.  The shared-prefix
     // suffix pass reads nothing that kernel (the prefix kernel) writes until it
     // folds the prefix records in, so it waits there and streams its suffix
-    // meanwhile; everything the kernels before that one wrote was complete
-    // when the prefix kernel started (an ordinary launch).
+    // meanwhile; everything the kernels before that one wrote is complete when
+    // this grid starts (the prefix kernel lets its dependents launch only after
+    // its wait for the kernel before it returns, and every kernel of the step
+    // waits for its predecessor before it finishes).
     if (threadIdx.x == C::NW * 32) {            // the producer's copies need both maps first
         dev::prefetch_tensormap(&tmk);
         dev::prefetch_tensormap(&tmv);
