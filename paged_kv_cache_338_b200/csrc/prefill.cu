@@ -28,15 +28,17 @@
 // Warp roles (384 threads): warps 0-3 and 4-7 are the softmax and epilogue
 // warpgroups of tiles A and B (warp w reads TMEM lanes 32(w%4)..32(w%4)+31,
 // i.e. its 32 query rows); warp 8 loads (tensor-map copies of the two Q tiles
-// once, then K and V tiles into rings); warp 9 allocates tensor memory and one
-// of its lanes issues every MMA; warps 10-11 only complete the third
-// warpgroup, whose registers go to the softmax warps.  The two softmax warps
-// that share a scheduler (w and w + 4) take turns with their exponentials, so
-// each has the special-function unit to itself, and a row's sum is taken
-// after its P is handed to the MMA warp.  Tensor memory: S_A
-// 0..127, O_A 128..255, S_B 256..383, O_B 384..511.  The MMA lane issues the
-// next S_X into the same columns right behind P_X.V (one thread's MMAs run in
-// issue order), so the tensor core never idles waiting for P_X.V to finish.
+// once, then K and V tiles into rings); warp 9 allocates tensor memory, and
+// one lane of warp 9 issues tile A's MMAs and one lane of warp 10 tile B's,
+// each from its own scheduler (a tile's MMAs never queue behind the other
+// tile's issue); warp 11 only completes the third warpgroup, whose registers
+// go to the softmax warps.  The two softmax warps that share a scheduler (w
+// and w + 4) take turns with their exponentials, so each has the special-
+// function unit to itself, and a row's sum is taken after its P is handed to
+// the MMA warp.  Tensor memory: S_A 0..127, O_A 128..255, S_B 256..383, O_B
+// 384..511.  A tile's MMA lane issues its next S_X into the same columns right
+// behind P_X.V (one thread's MMAs run in issue order), so the tensor core
+// never idles waiting for P_X.V to finish.
 // Every wait is bounded (2 s): on timeout the CTA records PA_DEV_WAIT_TIMEOUT
 // with the wait's site, drains its own copies and MMAs, frees its tensor
 // memory and exits.
@@ -106,7 +108,7 @@ struct Smem {
     // barriers: q, k_full[ST], k_free[ST], v_full[ST], v_free[ST], then per
     // query tile s_full, p_full, pv_done, o_full; drain; then per query tile
     // and softmax warp the turn of its exponentials
-    static constexpr int NBAR = 1 + 4 * ST + 8 + 1 + 8;
+    static constexpr int NBAR = 1 + 4 * ST + 8 + 1 + 8 + 1;
     static constexpr int TMEM_SLOT = BAR + NBAR * 8;
     static constexpr int ABORT = TMEM_SLOT + 4;
     static constexpr int BYTES = ABORT + 4 + 1024;  // + slack to align the base to 1024
@@ -401,16 +403,18 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
     auto o_full = [&](int x) { return bar0 + 8u * (7 + 4 * ST + x); };
     const uint32_t drain = bar0 + 8u * (9 + 4 * ST);
     auto turn = [&](int x, int w) { return bar0 + 8u * (10 + 4 * ST + 4 * x + w); };
+    const uint32_t v_zeroed = bar0 + 8u * (18 + 4 * ST);     // the last V tile's tail is zero
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::ABORT);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
+        // with tile B, both MMA warps release every K and V stage
         for (int i = 0; i < ST; ++i) {
             mbar_init(k_full(i), 1);
-            mbar_init(k_free(i), 1);
+            mbar_init(k_free(i), hasB ? 2 : 1);
             mbar_init(v_full(i), 1);
-            mbar_init(v_free(i), 1);
+            mbar_init(v_free(i), hasB ? 2 : 1);
         }
         for (int x = 0; x < 2; ++x) {
             mbar_init(s_full(x), 1);
@@ -418,8 +422,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             mbar_init(pv_done(x), 1);
             mbar_init(o_full(x), 1);
         }
-        mbar_init(drain, 1);
+        mbar_init(drain, hasB ? 2 : 1);
         for (int i = 0; i < 8; ++i) mbar_init(turn(i >> 2, i & 3), 1);
+        mbar_init(v_zeroed, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -491,14 +496,26 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             }
         }
         warp_wait(q_full, 0, abort_flag, p.err, 17, false);
-    } else if (warp == 9) {
+    } else if (warp == 9 || (warp == 10 && hasB)) {
         // ------------------------------------------------------------- MMAs
+        // Warp 9 issues tile A's MMAs and warp 10 tile B's, each from its own
+        // scheduler, so a tile's P.V and next S go out as soon as its P is
+        // handed over rather than behind the other tile's.  With tile B both
+        // warps release every K and V stage (the free barriers count two); a
+        // warp whose tile needs fewer key tiles arrives on the stages it does
+        // not read once they are filled, so both warps' arrivals on a barrier
+        // are always for the same use of the stage.
         regs_dec<kRegsOther>();
+        const int x = warp - 9;
+        const int ntx = x ? ntB : ntA;
+        // the pair's last key tile (read by B, and by A when ntA == nt): the
+        // warp of the tile that reads it last zeroes its V tail
+        const bool zeroes = hasB ? x == 1 : true;
         constexpr int ABF = DT == PA_BF16 ? 1 : 0;
         const uint32_t id_s = idesc_f16(ABF, 0, kBN);
         const uint32_t id_o = idesc_f16(ABF, 1, D);
         // S_X = Q_X K^T for key tile j (K in ring slot st)
-        auto issue_s = [&](int x, int st) {
+        auto issue_s = [&](int st) {
             tc_fence_after();
             if (lane == 0) {
                 const uint32_t kb = sK + st * L::TILE, qb = sQ + x * L::TILE;
@@ -513,22 +530,18 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                     tc_mma_lh(d, alo + off, hi, blo + off, hi, id_s, kk > 0);
                 }
                 tc_commit(s_full(x));
+                tc_commit(k_free(st));
             }
             __syncwarp();
         };
         bool ok = warp_wait(q_full, 0, abort_flag, p.err, 7) &&
                   warp_wait(k_full(0), 0, abort_flag, p.err, 8);
-        if (ok) {
-            issue_s(0, 0);
-            if (ntB > 0) issue_s(1, 0);
-            if (lane == 0) tc_commit(k_free(0));
-            __syncwarp();
-        }
+        if (ok) issue_s(0);
         for (int j = 0; j < nt && ok; ++j) {
             const int st = j % ST, st1 = (j + 1) % ST;
             if (!(ok = warp_wait(v_full(st), (j / ST) & 1, abort_flag, p.err, 9))) break;
             const uint32_t vb = sV + st * L::TILE;
-            if (j == nt - 1) {
+            if (j == nt - 1 && zeroes) {
                 // Rows at or past kv_len hold another token's values, the cache's
                 // unused tail slots or stale tiles: zero them, since a zero
                 // probability times a NaN would still poison the product.
@@ -540,11 +553,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                                      ::"r"(vb + sg * kSeg + z0 * 128 + xx * 16), "r"(0) : "memory");
                 fence_proxy_async_smem();
                 __syncwarp();
+                if (hasB && ntA == nt && lane == 0) mbar_arrive(v_zeroed);
+                __syncwarp();
+            } else if (j == nt - 1 && j < ntx) {
+                if (!(ok = warp_wait(v_zeroed, 0, abort_flag, p.err, 9))) break;
             }
-            bool k_next = false;
-            for (int x = 0; x < 2 && ok; ++x) {
-                const int ntx = x ? ntB : ntA;
-                if (j >= ntx) continue;
+            if (j < ntx) {
                 if (!(ok = warp_wait(p_full(x), j & 1, abort_flag, p.err, 13))) break;
                 tc_fence_after();
                 if (lane == 0) {
@@ -557,26 +571,24 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                                      (j > 0 || kk > 0) ? 1u : 0u);
                     tc_commit(pv_done(x));
                     if (j == ntx - 1) tc_commit(o_full(x));
+                    tc_commit(v_free(st));
                 }
-                __syncwarp();
-                if (j + 1 < ntx) {
-                    // The next scores overwrite P_X in the same columns.  They are
-                    // issued right behind P_X.V: the MMAs one thread issues run in
-                    // issue order, so P_X.V has read P_X before S_X(j+1) is written.
-                    if (!k_next) {
-                        if (!(ok = warp_wait(k_full(st1), ((j + 1) / ST) & 1, abort_flag, p.err,
-                                             8)))
-                            break;
-                        k_next = true;
-                    }
-                    issue_s(x, st1);
-                }
-            }
-            if (lane == 0) {
-                tc_commit(v_free(st));
-                if (k_next) tc_commit(k_free(st1));
+            } else if (lane == 0) {
+                mbar_arrive(v_free(st));                       // this tile does not read tile j
             }
             __syncwarp();
+            if (j + 1 < nt) {
+                // The next scores overwrite P_X in the same columns.  They are
+                // issued right behind P_X.V: the MMAs one thread issues run in
+                // issue order, so P_X.V has read P_X before S_X(j+1) is written.
+                if (!(ok = warp_wait(k_full(st1), ((j + 1) / ST) & 1, abort_flag, p.err, 8))) break;
+                if (j + 1 < ntx) {
+                    issue_s(st1);
+                } else {
+                    if (lane == 0) mbar_arrive(k_free(st1));
+                    __syncwarp();
+                }
+            }
         }
         // every MMA this warp issued completes before tensor memory is freed
         if (lane == 0) tc_commit(drain);
